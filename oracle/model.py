@@ -1,0 +1,197 @@
+"""fp64 forward and backward of the GPT decoder step (plain numpy).
+
+TEST INFRASTRUCTURE ONLY: see the package header.
+
+Model ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "1. Modelo GPT";
+"Como Treinar Seu Próprio ChatGPT por 50 Dólares?", section "1. O Modelo
+GPT"): untied token embedding and lm_head, rotary embeddings, QK
+normalisation, causal attention, an MLP with ReLU^2, and (implied by the
+pre-norm design and the lack of any norm gains in the optimizer table of
+section "2. Optimizador Muon") gain-free RMSNorm before attention, before the
+MLP and before the lm_head.  Loss: mean next-token cross-entropy over all
+B*T positions.
+
+Readings where the pages are silent (shared with the CUDA path):
+  * RMSNorm eps = 1e-6, no gain.
+  * RoPE: base 10000, rotate-half pairs (i, i + hd/2), angle t * base^(-2i/hd),
+    out_lo = x_lo cos - x_hi sin, out_hi = x_lo sin + x_hi cos, t = position
+    within the row.
+  * QK norm: per-head gain-free RMSNorm applied after RoPE (the order does
+    not matter mathematically: a rotation keeps the RMS).
+  * attention scale 1/sqrt(hd); n_kv_head = n_head; full causal window.
+  * weights are [in, out]; the fused projection's columns are q | k | v and
+    head h owns columns h*hd .. h*hd+hd-1 of each.
+
+Every intermediate is fp64; weights enter as their bf16 values.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+EPS = 1e-6
+ROPE_BASE = 10000.0
+
+
+# --- building blocks -------------------------------------------------------
+
+def rms_norm(x):
+    """y = x / sqrt(mean(x^2) + eps) along the last axis; returns (y, rstd)."""
+    rstd = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + EPS)
+    return x * rstd, rstd
+
+
+def rms_norm_bwd(dy, y, rstd):
+    """Gradient of the gain-free RMSNorm given its output y = x * rstd."""
+    return rstd * (dy - y * np.mean(dy * y, axis=-1, keepdims=True))
+
+
+def rope_angles(seq_len, head_dim):
+    i = np.arange(head_dim // 2, dtype=np.float64)
+    inv_freq = ROPE_BASE ** (-2.0 * i / head_dim)
+    t = np.arange(seq_len, dtype=np.float64)
+    ang = np.outer(t, inv_freq)                     # [T, hd/2]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x, cos, sin):
+    """Rotate pairs (i, i + hd/2) of x [..., T, hd] by the position angle."""
+    h = x.shape[-1] // 2
+    lo, hi = x[..., :h], x[..., h:]
+    return np.concatenate([lo * cos - hi * sin, lo * sin + hi * cos], axis=-1)
+
+
+def rope_bwd(dy, cos, sin):
+    """Transpose of the rotation (rotate by the negative angle)."""
+    h = dy.shape[-1] // 2
+    lo, hi = dy[..., :h], dy[..., h:]
+    return np.concatenate([lo * cos + hi * sin, -lo * sin + hi * cos], axis=-1)
+
+
+def causal_attention(q, k, v):
+    """softmax(q k^T / sqrt(hd) + causal mask) v for [B, H, T, hd]; returns (y, P)."""
+    hd = q.shape[-1]
+    T = q.shape[-2]
+    s = np.matmul(q, np.swapaxes(k, -1, -2)) / np.sqrt(hd)
+    mask = np.triu(np.ones((T, T), dtype=bool), k=1)
+    s = np.where(mask, -np.inf, s)
+    s = s - np.max(s, axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / np.sum(p, axis=-1, keepdims=True)
+    return np.matmul(p, v), p
+
+
+def causal_attention_bwd(dy, q, k, v, p):
+    hd = q.shape[-1]
+    dv = np.matmul(np.swapaxes(p, -1, -2), dy)
+    dp = np.matmul(dy, np.swapaxes(v, -1, -2))
+    ds = p * (dp - np.sum(dp * p, axis=-1, keepdims=True)) / np.sqrt(hd)
+    dq = np.matmul(ds, k)
+    dk = np.matmul(np.swapaxes(ds, -1, -2), q)
+    return dq, dk, dv
+
+
+def logsumexp(z):
+    m = np.max(z, axis=-1, keepdims=True)
+    return (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))[..., 0]
+
+
+# --- the step --------------------------------------------------------------
+
+def _split_heads(a, B, T, H, hd):
+    return a.reshape(B, T, H, hd).transpose(0, 2, 1, 3)
+
+
+def _merge_heads(a):
+    B, H, T, hd = a.shape
+    return a.transpose(0, 2, 1, 3).reshape(B * T, H * hd)
+
+
+def forward(params, tok, tgt, n_layer, head_dim=128, keep=True):
+    """Loss (and the saved activations) of one batch.
+
+    params: dict of fp64-castable [in, out] matrices (wte is [V, d]).
+    tok, tgt: int arrays [B, T].
+    """
+    B, T = tok.shape
+    wte = np.asarray(params["wte"], dtype=np.float64)
+    d = wte.shape[1]
+    H = d // head_dim
+    cos, sin = rope_angles(T, head_dim)
+    x = wte[tok.reshape(-1)]                         # [M, d] exact row copy
+    acts = []
+    for l in range(n_layer):
+        W = {n: np.asarray(params[f"h{l}.{n}"], dtype=np.float64)
+             for n in ("c_qkv", "c_proj", "c_fc", "mlp_proj")}
+        a = {}
+        xn1, r1 = rms_norm(x)
+        qkv = xn1 @ W["c_qkv"]
+        q = _split_heads(qkv[:, :d], B, T, H, head_dim)
+        k = _split_heads(qkv[:, d:2 * d], B, T, H, head_dim)
+        v = _split_heads(qkv[:, 2 * d:], B, T, H, head_dim)
+        qn, rq = rms_norm(rope(q, cos, sin))
+        kn, rk = rms_norm(rope(k, cos, sin))
+        y, P = causal_attention(qn, kn, v)
+        ym = _merge_heads(y)
+        x = x + ym @ W["c_proj"]
+        xn2, r2 = rms_norm(x)
+        u = xn2 @ W["c_fc"]
+        h = np.maximum(u, 0.0) ** 2
+        x = x + h @ W["mlp_proj"]
+        if keep:
+            a.update(xn1=xn1, r1=r1, qn=qn, rq=rq, kn=kn, rk=rk, v=v, P=P, ym=ym,
+                     xn2=xn2, r2=r2, u=u, h=h)
+        acts.append(a)
+    xf, rf = rms_norm(x)
+    z = xf @ np.asarray(params["lm_head"], dtype=np.float64)
+    lse = logsumexp(z)
+    t = tgt.reshape(-1)
+    row_loss = lse - z[np.arange(z.shape[0]), t]
+    loss = float(np.mean(row_loss))
+    cache = dict(acts=acts, xf=xf, rf=rf, z=z, lse=lse, row_loss=row_loss,
+                 B=B, T=T, H=H, d=d, cos=cos, sin=sin) if keep else None
+    return loss, cache
+
+
+def backward(params, tok, tgt, cache, n_layer, head_dim=128):
+    """Exact gradients of the mean loss w.r.t. every parameter ([in, out] layout)."""
+    B, T, H, d = cache["B"], cache["T"], cache["H"], cache["d"]
+    cos, sin = cache["cos"], cache["sin"]
+    M = B * T
+    z, lse = cache["z"], cache["lse"]
+    t = tgt.reshape(-1)
+    dz = np.exp(z - lse[:, None])
+    dz[np.arange(M), t] -= 1.0
+    dz /= M
+    grads = {}
+    Wlm = np.asarray(params["lm_head"], dtype=np.float64)
+    grads["lm_head"] = cache["xf"].T @ dz
+    dx = rms_norm_bwd(dz @ Wlm.T, cache["xf"], cache["rf"])
+    for l in reversed(range(n_layer)):
+        a = cache["acts"][l]
+        W = {n: np.asarray(params[f"h{l}.{n}"], dtype=np.float64)
+             for n in ("c_qkv", "c_proj", "c_fc", "mlp_proj")}
+        # MLP: x_out = x_mid + relu(rms(x_mid) Wfc)^2 Wd
+        grads[f"h{l}.mlp_proj"] = a["h"].T @ dx
+        dh = dx @ W["mlp_proj"].T
+        du = dh * 2.0 * np.maximum(a["u"], 0.0)
+        grads[f"h{l}.c_fc"] = a["xn2"].T @ du
+        dx = dx + rms_norm_bwd(du @ W["c_fc"].T, a["xn2"], a["r2"])
+        # attention: x_mid = x_in + attn(rms(x_in)) Wo
+        grads[f"h{l}.c_proj"] = a["ym"].T @ dx
+        dy = _split_heads(dx @ W["c_proj"].T, B, T, H, head_dim)
+        dqn, dkn, dv = causal_attention_bwd(dy, a["qn"], a["kn"], a["v"], a["P"])
+        dq = rope_bwd(rms_norm_bwd(dqn, a["qn"], a["rq"]), cos, sin)
+        dk = rope_bwd(rms_norm_bwd(dkn, a["kn"], a["rk"]), cos, sin)
+        dqkv = np.concatenate([_merge_heads(dq), _merge_heads(dk), _merge_heads(dv)], axis=1)
+        grads[f"h{l}.c_qkv"] = a["xn1"].T @ dqkv
+        dx = dx + rms_norm_bwd(dqkv @ W["c_qkv"].T, a["xn1"], a["r1"])
+    V = params["wte"].shape[0]
+    dwte = np.zeros((V, d))
+    np.add.at(dwte, tok.reshape(-1), dx)
+    grads["wte"] = dwte
+    return grads
+
+
+def fwd_bwd(params, tok, tgt, n_layer, head_dim=128):
+    loss, cache = forward(params, tok, tgt, n_layer, head_dim)
+    return loss, backward(params, tok, tgt, cache, n_layer, head_dim), cache

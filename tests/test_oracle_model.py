@@ -1,0 +1,232 @@
+"""Pins of the fp64 model oracle against what the pages and mathematics fix (CPU only)."""
+import numpy as np
+import pytest
+
+import synthetic as syn
+from oracle import model as om
+
+
+def small_case(depth=2, d=128, vocab=64, batch=2, seq=16, seed=0, std=0.02):
+    s = syn.make_shape(depth=depth, batch=batch, seq_len=seq, vocab=vocab, d_model=d)
+    p = syn.init_params(s, seed=seed, std=std)
+    tok = syn.tokens(s, seed=seed + 1)
+    tgt = syn.targets(s, seed=seed + 2)
+    return s, p, tok, tgt
+
+
+# --- loss closed forms ------------------------------------------------------
+
+def test_zero_lm_head_loss_is_log_vocab():
+    s, p, tok, tgt = small_case()
+    p["lm_head"] = np.zeros_like(p["lm_head"])
+    loss, _ = om.forward(p, tok, tgt, s.depth)
+    assert loss == pytest.approx(np.log(s.vocab), abs=1e-12)
+
+
+def test_zero_lm_head_grad_closed_form():
+    # with z = 0, dz = (1/V - onehot(target)) / M, so every row of dW_lm sums to 0
+    # and the target-column total is -(sum of xf rows with that target)/M*(1-1/V)
+    s, p, tok, tgt = small_case()
+    p["lm_head"] = np.zeros_like(p["lm_head"])
+    loss, g, cache = om.fwd_bwd(p, tok, tgt, s.depth)
+    assert np.abs(g["lm_head"].sum(axis=1)).max() < 1e-14
+    xf = cache["xf"]
+    M = s.tokens
+    t = tgt.reshape(-1)
+    expect = xf.sum(0)[:, None] / (M * s.vocab) * np.ones((1, s.vocab))
+    for m in range(M):
+        expect[:, t[m]] -= xf[m] / M
+    assert np.allclose(g["lm_head"], expect, atol=1e-15)
+
+
+def test_initial_loss_matches_gaussian_logit_closed_form():
+    # xf has RMS 1 so, given xf, the logits are iid N(0, sigma^2) with
+    # sigma^2 = std^2 * d; E[loss] = ln V + sigma^2/2 - (e^{sigma^2}-1)/(2V)
+    s = syn.make_shape(depth=1, batch=4, seq_len=256, vocab=4096, d_model=256)
+    p = syn.init_params(s, seed=5)
+    tok, tgt = syn.tokens(s, seed=6), syn.targets(s, seed=7)
+    loss, cache = om.forward(p, tok, tgt, s.depth)
+    sig2 = 0.02 ** 2 * s.d_model
+    expect = np.log(s.vocab) + sig2 / 2 - (np.exp(sig2) - 1) / (2 * s.vocab)
+    # the target logit term dominates the sampling error: std ~ sigma / sqrt(M)
+    assert abs(loss - expect) < 4 * np.sqrt(sig2 / s.tokens)
+    # and the oracle's own logits have the variance the closed form assumes
+    assert np.var(cache["z"]) == pytest.approx(sig2, rel=0.05)
+
+
+def test_zero_blocks_are_identity():
+    # with every block matrix zero the residual stream passes through unchanged,
+    # so the loss equals that of the embedding -> norm -> lm_head model
+    s, p, tok, tgt = small_case(depth=3)
+    for name, *_ in syn.param_specs(s):
+        if name.startswith("h"):
+            p[name] = np.zeros_like(p[name])
+    loss, _ = om.forward(p, tok, tgt, s.depth)
+    loss0, _ = om.forward(p, tok, tgt, 0)
+    assert loss == pytest.approx(loss0, abs=1e-13)
+
+
+def test_single_position_attention_is_value():
+    # T = 1: softmax over one key is 1, so attention returns v exactly
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.standard_normal((2, 3, 1, 128)) for _ in range(3))
+    y, P = om.causal_attention(q, k, v)
+    assert np.array_equal(P, np.ones_like(P))
+    assert np.allclose(y, v, atol=0)
+
+
+def test_attention_scale_and_mask():
+    # two positions; q1.k0/sqrt(128) = 0 and q1.k1/sqrt(128) = ln 3 give
+    # weights (1/4, 3/4) on row 1; row 0 sees only key 0
+    hd = 128
+    q = np.zeros((1, 1, 2, hd)); k = np.zeros((1, 1, 2, hd)); v = np.zeros((1, 1, 2, hd))
+    q[..., 1, 0] = 1.0
+    k[..., 1, 0] = np.log(3.0) * np.sqrt(hd)
+    k[..., 0, 1] = 5.0           # orthogonal to q1
+    q[..., 0, 1] = 7.0
+    v[..., 0, 2] = 1.0
+    v[..., 1, 3] = 1.0
+    y, P = om.causal_attention(q, k, v)
+    assert P[0, 0, 0].tolist() == [1.0, 0.0]
+    assert np.allclose(P[0, 0, 1], [0.25, 0.75], atol=1e-15)
+    assert np.allclose(y[0, 0, 1, 2:4], [0.25, 0.75], atol=1e-15)
+
+
+def test_equal_keys_give_prefix_mean():
+    rng = np.random.default_rng(4)
+    T, hd = 9, 128
+    q = rng.standard_normal((1, 1, T, hd))
+    k = np.tile(rng.standard_normal((1, 1, 1, hd)), (1, 1, T, 1))
+    v = rng.standard_normal((1, 1, T, hd))
+    y, _ = om.causal_attention(q, k, v)
+    prefix_mean = np.cumsum(v, axis=2) / np.arange(1, T + 1)[None, None, :, None]
+    assert np.allclose(y, prefix_mean, atol=1e-13)
+
+
+def test_causality():
+    # changing tokens at positions > t leaves the per-position loss at <= t unchanged
+    s, p, tok, tgt = small_case(seq=16)
+    _, c1 = om.forward(p, tok, tgt, s.depth)
+    tok2 = tok.copy()
+    tok2[:, 10:] = (tok2[:, 10:] + 7) % s.vocab
+    _, c2 = om.forward(p, tok2, tgt, s.depth)
+    r1 = c1["row_loss"].reshape(s.batch, s.seq_len)
+    r2 = c2["row_loss"].reshape(s.batch, s.seq_len)
+    assert np.allclose(r1[:, :10], r2[:, :10], atol=1e-12, rtol=0)
+    assert np.abs(r1[:, 10:] - r2[:, 10:]).max() > 1e-3
+
+
+def test_target_index_moves_loss():
+    s, p, tok, tgt = small_case()
+    _, c1 = om.forward(p, tok, tgt, s.depth)
+    tgt2 = tgt.copy()
+    tgt2[0, 3] = (tgt2[0, 3] + 1) % s.vocab
+    _, c2 = om.forward(p, tok, tgt2, s.depth)
+    z = c1["z"]
+    m = 3
+    assert c2["row_loss"][m] - c1["row_loss"][m] == pytest.approx(
+        z[m, tgt[0, 3]] - z[m, tgt2[0, 3]], abs=1e-12)
+
+
+# --- RoPE / RMSNorm invariants -------------------------------------------------
+
+def test_rope_is_rotation_and_relative():
+    T, hd = 40, 128
+    cos, sin = om.rope_angles(T, hd)
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal(hd)
+    k = rng.standard_normal(hd)
+    Q = om.rope(np.tile(q, (T, 1)), cos, sin)
+    K = om.rope(np.tile(k, (T, 1)), cos, sin)
+    assert np.allclose(np.linalg.norm(Q, axis=1), np.linalg.norm(q), rtol=1e-14)
+    dots = Q @ K.T
+    for off in (0, 3, 17):
+        diag = np.diagonal(dots, offset=off)
+        assert np.allclose(diag, diag[0], atol=1e-11)
+    # position 0 is the identity, and the backward is the inverse rotation
+    assert np.allclose(Q[0], q, atol=0)
+    assert np.allclose(om.rope_bwd(Q, cos, sin), np.tile(q, (T, 1)), atol=1e-13)
+
+
+def test_rope_first_pair_angle():
+    # pair 0 rotates by t radians (base^0 = 1); the last pair by t * base^(-126/128)
+    cos, sin = om.rope_angles(8, 128)
+    assert np.allclose(cos[:, 0], np.cos(np.arange(8)))
+    assert np.allclose(sin[:, 63], np.sin(np.arange(8) * 10000.0 ** (-126 / 128)))
+
+
+def test_rmsnorm_invariants():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 256)) * 3.0
+    y, r = om.rms_norm(x)
+    ms = np.mean(x * x, axis=1)
+    assert np.allclose(np.mean(y * y, axis=1), ms / (ms + om.EPS), rtol=1e-14)
+    y2, _ = om.rms_norm(10.0 * x)
+    assert np.allclose(y, y2, atol=1e-7)   # scale invariant up to eps
+    # gradient is orthogonal to y (scale invariance) up to the eps term
+    dy = rng.standard_normal(x.shape)
+    dx = om.rms_norm_bwd(dy, y, r)
+    assert np.abs(np.sum(dx * x, axis=1)).max() < 1e-5
+
+
+# --- finite differences --------------------------------------------------------
+
+def _fd_check(p, tok, tgt, depth, names, n_coords=6, h=1e-5, seed=0):
+    loss, g, _ = om.fwd_bwd(p, tok, tgt, depth)
+    rng = np.random.default_rng(seed)
+    worst = 0.0
+    for name in names:
+        W = p[name].astype(np.float64)
+        G = g[name]
+        scale = np.abs(G).max()
+        assert scale > 0, name
+        if name == "wte":
+            rows = np.unique(tok)
+            coords = [(rng.choice(rows), rng.integers(W.shape[1])) for _ in range(n_coords)]
+        else:
+            # half at random, half at the largest gradient entries
+            flat = np.argsort(np.abs(G).ravel())[-n_coords // 2:]
+            coords = [np.unravel_index(i, W.shape) for i in flat]
+            coords += [(rng.integers(W.shape[0]), rng.integers(W.shape[1]))
+                       for _ in range(n_coords - len(coords))]
+        for (i, j) in coords:
+            pp = dict(p); Wp = W.copy(); Wp[i, j] += h; pp[name] = Wp
+            lp, _ = om.forward(pp, tok, tgt, depth, keep=False)
+            Wm = W.copy(); Wm[i, j] -= h; pp[name] = Wm
+            lm, _ = om.forward(pp, tok, tgt, depth, keep=False)
+            fd = (lp - lm) / (2 * h)
+            err = abs(fd - G[i, j]) / scale
+            worst = max(worst, err)
+            assert err < 1e-6, (name, i, j, fd, G[i, j], scale)
+    return worst
+
+
+def test_finite_difference_every_tensor():
+    s, p, tok, tgt = small_case(depth=2, d=128, vocab=64, batch=2, seq=16, std=0.05)
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    names = [n for n, *_ in syn.param_specs(s)]
+    _fd_check(p, tok, tgt, s.depth, names)
+
+
+def test_finite_difference_two_heads():
+    # two heads: checks the head split/merge and per-head QK norm
+    s, p, tok, tgt = small_case(depth=1, d=256, vocab=48, batch=1, seq=12, std=0.05, seed=9)
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    _fd_check(p, tok, tgt, s.depth, ["h0.c_qkv", "h0.c_proj", "wte"], n_coords=8)
+
+
+def test_embedding_grad_rows():
+    s, p, tok, tgt = small_case(vocab=64)
+    _, g, _ = om.fwd_bwd(p, tok, tgt, s.depth)
+    absent = np.setdiff1d(np.arange(s.vocab), np.unique(tok))
+    assert len(absent) > 0
+    assert np.all(g["wte"][absent] == 0.0)
+
+
+def test_embedding_forward_is_row_copy():
+    s, p, tok, tgt = small_case()
+    # depth 0 and zero lm_head: xf = rms(wte[tok]); check via the cache
+    _, c = om.forward(p, tok, tgt, 0)
+    x0 = p["wte"][tok.reshape(-1)].astype(np.float64)
+    xf, _ = om.rms_norm(x0)
+    assert np.array_equal(c["xf"], xf)
