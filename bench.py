@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Training-step benchmark: tokens/s and MFU of one GPT pretraining step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config d20] [--impl ours|reference]
+
+A step is the whole hot path on one batch of synthetic input: forward and
+backward of the decoder, the Muon update of every block matrix and the AdamW
+update of the embedding and lm_head, all through libgpt's C ABI.  Inputs are
+resident in HBM when the timed region starts; the activations (tens of GB)
+exceed the 126 MB L2 many times over, so no L2 flush is needed between steps.
+For N > 1 (launched by torch.distributed.run) every rank trains on its own
+batch and the gradients are averaged with one NCCL all-reduce per step before
+the (replicated) optimizer step; the reported time is the max over ranks.
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
+on a bounded sample of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "training tokens/sec and MFU (fwd+bwd+Muon step) on 1 B200, d20 seq 2048 bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="d20", choices=["d12", "d20", "d24", "d26"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ns-tf32-steps", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--breakdown", action="store_true", help="per-category device times in the JSON line")
+    a = ap.parse_args()
+    a.warmup = max(a.warmup, 3)
+    return a
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ FLOPs
+
+def model_flops_per_token(s):
+    """PaLM-style model FLOPs per token: 6 N_matmul + 12 L d T (embeddings excluded)."""
+    n_matmul = s.depth * 12 * s.d_model ** 2 + s.d_model * s.vocab
+    return 6 * n_matmul + 12 * s.depth * s.d_model * s.seq_len
+
+
+def category_work(s):
+    """Algorithmic FLOPs (tensor categories) or bytes (HBM categories) per step."""
+    M, d, F, V, L, B, H, T = s.tokens, s.d_model, s.mlp_hidden, s.vocab, s.depth, s.batch, s.n_head, s.seq_len
+    causal = B * H * 128 * T * (T + 1) / 2          # q.k products that the causal mask keeps
+    r = d
+    ns = 0.0
+    for nmat, c in ((L, 3 * d), (L, d), (2 * L, F)):
+        ns += nmat * 5 * (r * r * c + r ** 3 + 2 * r * r * c)   # symmetric Gram and square, dense update
+    return {
+        "qkv_gemm": ("tensor", 2 * M * d * 3 * d * L),
+        "proj_gemm": ("tensor", 2 * M * d * d * L),
+        "fc_gemm": ("tensor", 2 * M * d * F * L),
+        "down_gemm": ("tensor", 2 * M * F * d * L),
+        "attn_fwd": ("tensor", 4 * causal * L),
+        "attn_bwd": ("tensor", 10 * causal * L),
+        "logits_gemm": ("tensor", 2 * M * d * V),
+        "lm_dx_gemm": ("tensor", 2 * M * d * V),
+        "lm_dw_gemm": ("tensor", 2 * M * d * V),
+        "dx_gemm": ("tensor", 24 * M * d * d * L),
+        "dw_gemm": ("tensor", 24 * M * d * d * L),
+        "ns_gemm": ("tensor", ns),
+        # bytes: read fp32 x, write bf16 y (+ rstd) forward; read fp32 dy, bf16 y,
+        # fp32 dx, write fp32 dx and bf16 dx backward
+        "norm": ("hbm", (2 * L + 1) * M * d * 6 + (2 * L + 1) * M * d * 14),
+        "ce_finish": ("hbm", M * V * 2 * 2),
+        "qk_bwd": ("hbm", L * M * d * (4 + 2 * 4 + 3 * 2)),
+        "embed": ("hbm", M * d * (2 + 4) + M * d * 4 + V * d * 4),
+        "muon_elem": ("hbm", L * 12 * d * d * (12 + 4 + 4 + 10)),
+        "adamw": ("hbm", 2 * V * d * 30),
+    }
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.file.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------- CPU oracle
+
+def oracle_sample(s, tokens_per_sample=128, seed=0, ns_kinds=(0, 1, 2, 3), adam_frac=1 / 32):
+    """Times the fp64 oracle on a bounded slice of one step and scales it to the step.
+
+    Returns (scaled step seconds, description, threads): forward+backward of the
+    whole model on one sequence prefix of ``tokens_per_sample`` tokens (scaled by
+    tokens), Newton-Schulz on one matrix per block kind (scaled by the number of
+    matrices of that kind) and AdamW on a fraction of the embedding and lm_head.
+    """
+    import numpy as np
+    from oracle import model as om
+    from oracle import optim as oo
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    params = syn.init_params(s, seed=seed)
+    tok = syn.tokens(s)[:1, :tokens_per_sample]
+    tgt = syn.targets(s)[:1, :tokens_per_sample]
+    t0 = time.perf_counter()
+    _, grads, _ = om.fwd_bwd(params, tok, tgt, s.depth)
+    t_fb = time.perf_counter() - t0
+    kinds = ["c_qkv", "c_proj", "c_fc", "mlp_proj"]
+    t_ns = {}
+    for k in ns_kinds:
+        G = grads[f"h0.{kinds[k]}"]
+        W = params[f"h0.{kinds[k]}"]
+        t0 = time.perf_counter()
+        oo.muon_step(W, G, np.zeros_like(G), 0.02)
+        t_ns[k] = time.perf_counter() - t0
+    n = int(s.vocab * s.d_model * adam_frac)
+    p = params["wte"].ravel()[:n].astype(np.float64)
+    g = grads["wte"].ravel()[:n]
+    t0 = time.perf_counter()
+    oo.adamw_step(p, g, np.zeros(n), np.zeros(n), 1, 3e-3)
+    t_ad = time.perf_counter() - t0
+    mean_ns = sum(t_ns.values()) / len(t_ns)
+    step = t_fb * s.tokens / tokens_per_sample + sum(s.depth * t_ns.get(k, mean_ns) for k in range(4)) \
+        + t_ad * 2 / adam_frac
+    desc = (f"fp64 oracle: fwd+bwd of all {s.depth} layers on 1x{tokens_per_sample} tokens scaled x"
+            f"{s.tokens // tokens_per_sample}; Newton-Schulz on {len(t_ns)} matrices scaled to {4 * s.depth}; "
+            f"AdamW on {adam_frac:.3f} of the embedding scaled to wte+lm_head")
+    return step, desc, threads, t_fb + sum(t_ns.values()) + t_ad
+
+
+def run_reference(a):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = syn.config_shape(a.config)
+    times, wall, threads, desc = [], 0.0, 1, ""
+    for i in range(a.warmup + a.steps):
+        step, desc, threads, spent = oracle_sample(s, tokens_per_sample=64, ns_kinds=(i % 4,), adam_frac=1 / 64)
+        if i >= a.warmup:
+            times.append(step)
+            wall += spent
+    st = statistics.mean(times)
+    value = s.tokens / st
+    sample = desc + f"; {a.steps} timed steps, {wall:.1f} s of CPU work"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": a.gpus,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": st * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{a.config} GPT step", "global_batch": s.batch, "seq_len": s.seq_len,
+                   "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# --------------------------------------------------------------- GPU arm
+
+def run_ours(a):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import gpt_pretraining_step_b200 as g
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    g.lib()
+    s = syn.config_shape(a.config)
+    stream = torch.cuda.Stream()
+    torch.cuda.set_stream(stream)
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream)
+    tok = torch.tensor(syn.tokens(s, seed=1 + 100 * rank)).cuda()
+    tgt = torch.tensor(syn.targets(s, seed=2 + 100 * rank)).cuda()
+    grads = st.grad_view() if world > 1 else None
+    hp = dict(muon=(0.02, 0.95, 0.0), adam=(3e-3, 0.8, 0.95, 1e-10, 0.0))
+
+    def step():
+        st.fwd_bwd(tok, tgt)
+        if grads is not None:
+            dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+        st.muon_step(*hp["muon"])
+        st.adamw_step(*hp["adam"])
+
+    # warm-up; the last warm-up step records every launch category
+    for i in range(a.warmup):
+        if i == a.warmup - 1:
+            st.profile_enable(g.PROF_CATEGORIES)
+        step()
+    torch.cuda.synchronize()
+    st.check()
+    prof = st.profile_read()
+    work = category_work(s)
+    tensor_cats = [c for c in prof if work.get(c, ("", 0))[0] == "tensor"]
+    dominant = max(prof, key=lambda c: prof[c][0]) if prof else None
+    st.profile_enable([dominant] if dominant else [])
+
+    pk, pk_src = peaks()
+    sampler = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    n0 = st.launch_count()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(a.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    launches = st.launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1) / a.steps
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    st.check()
+    live = st.profile_read()
+    st.profile_enable([])
+    loss = float(st.loss[0].item())
+
+    tokens_per_step = s.tokens * world
+    value = tokens_per_step / (ms / 1e3)
+    fpt = model_flops_per_token(s)
+    mfu_sust = fpt * s.tokens / (ms / 1e3) / (pk["bf16_tflops_sustained"] * 1e12)
+    mfu_nominal = fpt * s.tokens / (ms / 1e3) / 2.25e15
+
+    roof = None
+    if dominant and dominant in live and live[dominant][1]:
+        kind, amount = work[dominant]
+        per_launch_ms = live[dominant][0] / live[dominant][1]
+        per_launch_work = amount / (live[dominant][1] / a.steps)
+        if kind == "tensor":
+            achieved = per_launch_work / (per_launch_ms / 1e3) / 1e12
+            peak = pk["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                    "peak_source": f"{pk_src} bf16_tflops_sustained"}
+        else:
+            achieved = per_launch_work / (per_launch_ms / 1e3) / 1e9
+            peak = pk["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": None, "kernel": dominant, "peak_source": f"{pk_src} hbm_gbs"}
+
+    breakdown = {}
+    if True:
+        for c, (tms, n) in sorted(prof.items(), key=lambda kv: -kv[1][0]):
+            kind, amount = work.get(c, ("", 0))
+            e = {"ms": round(tms, 3), "launches": n}
+            if tms > 0 and amount:
+                if kind == "tensor":
+                    e["tflops"] = round(amount / (tms / 1e3) / 1e12, 1)
+                else:
+                    e["gbs"] = round(amount / (tms / 1e3) / 1e9, 1)
+            breakdown[c] = e
+
+    e2e = None
+    if not a.no_e2e:
+        e2e = run_e2e(a, st, s, rank, world, grads, stream)
+        if world > 1:
+            t = torch.tensor([e2e["ms_per_step"]], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+            e2e["value"] = tokens_per_step / (e2e["ms_per_step"] / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        step_s, desc, threads, spent = oracle_sample(s)
+        cpu = {"value": s.tokens / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": desc + f" ({spent:.1f} s of CPU work)"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
+            "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{a.config} GPT step (fwd+bwd+Muon+AdamW)", "global_batch": s.batch * world,
+                       "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
+                       "parallelism": f"dp{world}", "ns_tf32_steps": a.ns_tf32_steps,
+                       "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2"},
+            "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
+            "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",
+            "model_tflop_per_step": fpt * s.tokens / 1e12,
+            "loss": loss, "clocks": clocks, "gpu_launches": launches, "roofline": roof, "cpu_baseline": cpu,
+            "e2e": None if e2e is None else {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step",
+                                                                 "d2h_bytes_per_step")},
+            "breakdown_ms_per_step_category": breakdown,
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(a, st, s, rank, world, grads, stream):
+    """Whole steps through the public API from host buffers: H2D of tokens and
+    targets from pinned memory, the step, D2H of the loss, all timed.  One GPU
+    uses the single host-buffer entry point; data-parallel ranks compose the
+    public calls with the gradient all-reduce in between."""
+    import torch
+    import torch.distributed as dist
+
+    import gpt_pretraining_step_b200 as g
+    tok = torch.tensor(syn.tokens(s, seed=11 + 100 * rank)).pin_memory()
+    tgt = torch.tensor(syn.targets(s, seed=12 + 100 * rank)).pin_memory()
+    hp = g.HParams(muon_lr=0.02, muon_momentum=0.95, muon_wd=0.0, adam_lr=3e-3, adam_beta1=0.8, adam_beta2=0.95,
+                   adam_eps=1e-10, adam_wd=0.0)
+    dtok = torch.empty_like(tok, device="cuda")
+    dtgt = torch.empty_like(tgt, device="cuda")
+    loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
+
+    def one():
+        if world == 1:
+            return st.train_step_host(tok, tgt, hp)
+        dtok.copy_(tok, non_blocking=True)
+        dtgt.copy_(tgt, non_blocking=True)
+        loss = st.fwd_bwd(dtok, dtgt)
+        dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+        st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)
+        st.adamw_step(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd)
+        loss_host.copy_(loss.reshape(1), non_blocking=True)
+        stream.synchronize()
+        return float(loss_host[0])
+
+    one()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        one()
+    dt = (time.perf_counter() - t0) / a.steps
+    return {"value": s.tokens / dt, "unit": "tokens/s", "ms_per_step": dt * 1e3,
+            "h2d_bytes_per_step": int(tok.numel() * 4 + tgt.numel() * 4), "d2h_bytes_per_step": 4}
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

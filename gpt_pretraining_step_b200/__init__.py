@@ -1,0 +1,289 @@
+"""Python binding of libgpt.so, the B200 GPT pretraining-step library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/gpt.h.  PyTorch provides device
+memory and the stream.  If the compiled library is missing the import of
+``lib()`` raises; there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgpt.so")
+
+GPT_OK, GPT_EINVAL, GPT_ERANGE, GPT_ETIMEOUT, GPT_ECUDA = 0, -1, -2, -3, -4
+KIND_PARAM, KIND_GRAD, KIND_MOM, KIND_ADAM_M, KIND_ADAM_V = 0, 1, 2, 3, 4
+GROUP_ADAMW, GROUP_MUON = 0, 1
+PROF_CATEGORIES = ["qkv_gemm", "proj_gemm", "fc_gemm", "down_gemm", "attn_fwd", "attn_bwd", "logits_gemm",
+                   "ce_finish", "lm_dx_gemm", "lm_dw_gemm", "dx_gemm", "dw_gemm", "norm", "qk_bwd", "embed",
+                   "ns_gemm", "muon_elem", "adamw"]
+
+ABI_FUNCTIONS = [
+    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "adamw_step", "gpt_train_step_host",
+    "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
+    "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_attention_fwd",
+    "gpt_op_attention_bwd", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
+]
+
+
+class GptError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"libgpt error {code}: {msg}")
+        self.code = code
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("depth", ctypes.c_int32), ("d_model", ctypes.c_int32), ("vocab", ctypes.c_int32),
+                ("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("mlp_mult", ctypes.c_int32), ("precision", ctypes.c_int32), ("ns_tf32_steps", ctypes.c_int32),
+                ("lm_chunk_rows", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class HParams(ctypes.Structure):
+    _fields_ = [("muon_lr", ctypes.c_float), ("muon_momentum", ctypes.c_float), ("muon_wd", ctypes.c_float),
+                ("adam_lr", ctypes.c_float), ("adam_beta1", ctypes.c_float), ("adam_beta2", ctypes.c_float),
+                ("adam_eps", ctypes.c_float), ("adam_wd", ctypes.c_float)]
+
+
+_LIB = None
+
+
+def lib():
+    """The loaded library (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m gpt_pretraining_step_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        sig = {
+            "gpt_workspace_size": (i32, [ctypes.POINTER(Config), ctypes.POINTER(sz), ctypes.POINTER(sz),
+                                         ctypes.POINTER(sz)]),
+            "gpt_init": (i32, [ctypes.POINTER(Config), vp, vp, vp, vp, ctypes.POINTER(vp)]),
+            "gpt_fwd_bwd": (i32, [vp, vp, vp, vp, i32]),
+            "muon_step": (i32, [vp, f32, f32, f32]),
+            "adamw_step": (i32, [vp, f32, f32, f32, f32, f32]),
+            "gpt_train_step_host": (i32, [vp, vp, vp, ctypes.POINTER(HParams), vp]),
+            "gpt_num_tensors": (i32, [vp]),
+            "gpt_tensor_info": (i32, [vp, i32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
+                                      ctypes.POINTER(ctypes.c_int32)]),
+            "gpt_get_tensor": (i32, [vp, i32, i32, vp]),
+            "gpt_set_tensor": (i32, [vp, i32, i32, vp]),
+            "gpt_get_row_loss": (i32, [vp, vp]),
+            "gpt_grad_region": (i32, [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+            "gpt_check": (i32, [vp]),
+            "gpt_launch_count": (ctypes.c_int64, [vp]),
+            "gpt_profile_enable": (i32, [vp, ctypes.c_uint32]),
+            "gpt_profile_read": (i32, [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
+            "gpt_destroy": (None, [vp]),
+            "gpt_last_error": (ctypes.c_char_p, []),
+            "gpt_op_matmul_bf16": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
+            "gpt_op_matmul_tf32": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
+            "gpt_op_attention_fwd": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp]),
+            "gpt_op_attention_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp]),
+            "gpt_op_rmsnorm_fwd": (i32, [vp, vp, vp, i32, i32, vp]),
+            "gpt_op_newton_schulz_scratch": (sz, [i32, i32, i32]),
+            "gpt_op_newton_schulz": (i32, [vp, vp, i32, i32, i32, i32, vp, vp]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def _check(rc):
+    if rc != GPT_OK:
+        raise GptError(rc, lib().gpt_last_error().decode())
+    return rc
+
+
+def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=2, lm_chunk_rows=0, seed=0):
+    return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
+                  mlp_mult=4, precision=0, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows, seed=seed)
+
+
+def workspace_size(cfg: Config):
+    p, s, a = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().gpt_workspace_size(ctypes.byref(cfg), ctypes.byref(p), ctypes.byref(s), ctypes.byref(a)))
+    return p.value, s.value, a.value
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+class GPTStep:
+    """One GPT training-step context on the current CUDA device.
+
+    The three workspace buffers are allocated with torch and owned by this
+    object; every computation runs in libgpt's kernels on ``stream``.
+    """
+
+    def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=2, lm_chunk_rows=0,
+                 seed=0, stream=None):
+        import torch
+        self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed)
+        self.sizes = workspace_size(self.cfg)
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        self.bufs = [torch.empty(max(n, 256), dtype=torch.uint8, device=dev) for n in self.sizes]
+        self.loss = torch.zeros(4, dtype=torch.float32, device=dev)
+        h = ctypes.c_void_p()
+        _check(lib().gpt_init(ctypes.byref(self.cfg), *[_ptr(b) for b in self.bufs], _stream(self.stream),
+                              ctypes.byref(h)))
+        self.h = h
+        self.d_model = self.cfg.d_model or 64 * depth
+
+    def __del__(self):
+        h = getattr(self, "h", None)
+        if h is not None and _LIB is not None:
+            _LIB.gpt_destroy(h)
+            self.h = None
+
+    # -- the step
+    def fwd_bwd(self, tokens, targets, accumulate=False, loss_out=None):
+        out = self.loss if loss_out is None else loss_out
+        _check(lib().gpt_fwd_bwd(self.h, _ptr(tokens), _ptr(targets), _ptr(out), int(bool(accumulate))))
+        return out[0] if loss_out is None else out
+
+    def muon_step(self, lr=0.02, momentum=0.95, weight_decay=0.0):
+        _check(lib().muon_step(self.h, lr, momentum, weight_decay))
+
+    def adamw_step(self, lr=3e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.0):
+        _check(lib().adamw_step(self.h, lr, beta1, beta2, eps, weight_decay))
+
+    def train_step_host(self, tokens_host, targets_host, hp: HParams):
+        """Whole step from host int32 arrays (numpy or pinned torch); returns the loss."""
+        loss = ctypes.c_float()
+        tp = tokens_host.ctypes.data if hasattr(tokens_host, "ctypes") else tokens_host.data_ptr()
+        gp = targets_host.ctypes.data if hasattr(targets_host, "ctypes") else targets_host.data_ptr()
+        _check(lib().gpt_train_step_host(self.h, ctypes.c_void_p(tp), ctypes.c_void_p(gp), ctypes.byref(hp),
+                                         ctypes.byref(loss)))
+        return loss.value
+
+    # -- tensors
+    def num_tensors(self):
+        return lib().gpt_num_tensors(self.h)
+
+    def tensor_info(self, tid):
+        r, c, g = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+        _check(lib().gpt_tensor_info(self.h, tid, ctypes.byref(r), ctypes.byref(c), ctypes.byref(g)))
+        return r.value, c.value, g.value
+
+    def get(self, tid, kind=KIND_PARAM):
+        import torch
+        r, c, _ = self.tensor_info(tid)
+        out = torch.empty((r, c), dtype=torch.float32, device=self.bufs[0].device)
+        _check(lib().gpt_get_tensor(self.h, tid, kind, _ptr(out)))
+        return out
+
+    def set(self, tid, value, kind=KIND_PARAM):
+        import torch
+        r, c, _ = self.tensor_info(tid)
+        v = torch.as_tensor(value, dtype=torch.float32).to(self.bufs[0].device).contiguous()
+        if tuple(v.shape) != (r, c):
+            raise ValueError(f"tensor {tid} has shape {(r, c)}, got {tuple(v.shape)}")
+        _check(lib().gpt_set_tensor(self.h, tid, kind, _ptr(v)))
+        self.stream.synchronize()
+
+    def grad_view(self):
+        """fp32 view of every gradient (one span of the state buffer), e.g. for an all-reduce."""
+        import torch
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_grad_region(self.h, ctypes.byref(off), ctypes.byref(n)))
+        return self.bufs[1][off.value:off.value + n.value].view(torch.float32)
+
+    def row_loss(self):
+        import torch
+        out = torch.empty((self.cfg.batch, self.cfg.seq_len), dtype=torch.float32, device=self.bufs[0].device)
+        _check(lib().gpt_get_row_loss(self.h, _ptr(out)))
+        return out
+
+    def check(self):
+        return _check(lib().gpt_check(self.h))
+
+    def launch_count(self):
+        return lib().gpt_launch_count(self.h)
+
+    def profile_enable(self, categories):
+        """Record events around the launches of the named categories (empty = off)."""
+        mask = 0
+        for c in categories:
+            mask |= 1 << PROF_CATEGORIES.index(c)
+        _check(lib().gpt_profile_enable(self.h, mask))
+
+    def profile_read(self):
+        """{category: (ms, launches)} since the last read (synchronises)."""
+        n = len(PROF_CATEGORIES)
+        ms = (ctypes.c_double * n)()
+        cnt = (ctypes.c_int64 * n)()
+        _check(lib().gpt_profile_read(self.h, ms, cnt))
+        return {PROF_CATEGORIES[i]: (ms[i], cnt[i]) for i in range(n) if cnt[i]}
+
+
+# ---------------------------------------------------------------- op level
+
+def matmul_bf16(A, B, M, N, K, batch=1, a_trans=False, b_trans=False, out=None, stream=None):
+    import torch
+    C = out if out is not None else torch.empty((batch, M, N), dtype=torch.float32, device=A.device)
+    _check(lib().gpt_op_matmul_bf16(_ptr(A), _ptr(B), _ptr(C), M, N, K, batch, int(a_trans), int(b_trans),
+                                    _stream(stream)))
+    return C
+
+
+def matmul_tf32(A, B, M, N, K, b_trans=False, stream=None):
+    import torch
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _check(lib().gpt_op_matmul_tf32(_ptr(A), _ptr(B), _ptr(C), M, N, K, int(b_trans), _stream(stream)))
+    return C
+
+
+def attention_fwd(q, k, v, stream=None):
+    import torch
+    B, H, T, hd = q.shape
+    o = torch.empty((B, T, H, hd), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check(lib().gpt_op_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, _stream(stream)))
+    return o, lse
+
+
+def attention_bwd(q, k, v, o, lse, dout, stream=None):
+    import torch
+    B, H, T, hd = q.shape
+    dq = torch.empty((B, H, T, hd), dtype=torch.float32, device=q.device)
+    dk = torch.empty_like(k)
+    dv = torch.empty_like(v)
+    D = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
+    _check(lib().gpt_op_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(D),
+                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, T, _stream(stream)))
+    return dq, dk, dv
+
+
+def rmsnorm_fwd(x, stream=None):
+    import torch
+    M, d = x.shape
+    y = torch.empty((M, d), dtype=torch.bfloat16, device=x.device)
+    r = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check(lib().gpt_op_rmsnorm_fwd(_ptr(x), _ptr(y), _ptr(r), M, d, _stream(stream)))
+    return y, r
+
+
+def newton_schulz(G, tf32_steps=2, stream=None):
+    import torch
+    batch, rows, cols = G.shape
+    X = torch.empty_like(G)
+    n = lib().gpt_op_newton_schulz_scratch(batch, rows, cols)
+    scratch = torch.empty(n, dtype=torch.uint8, device=G.device)
+    _check(lib().gpt_op_newton_schulz(_ptr(G), _ptr(X), batch, rows, cols, tf32_steps, _ptr(scratch),
+                                      _stream(stream)))
+    return X

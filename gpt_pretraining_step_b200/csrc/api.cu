@@ -1,0 +1,1097 @@
+// C ABI of the step library: configuration, the caller-owned memory plan,
+// the forward/backward schedule, Muon and AdamW, tensor access and the
+// op-level entry points.  See include/gpt.h for the contract.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <string>
+#include <vector>
+
+#include "../../include/gpt.h"
+#include "attention.cuh"
+#include "common.cuh"
+#include "gemm.h"
+#include "kernels.cuh"
+#include "polar_express_table.h"
+
+using namespace gpt;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+#define GPT_CK(expr)                                                                            \
+  do {                                                                                          \
+    cudaError_t e_ = (expr);                                                                    \
+    if (e_ != cudaSuccess)                                                                      \
+      return fail(GPT_ECUDA, std::string(#expr) + ": " + cudaGetErrorString(e_));               \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+
+struct Dims {
+  int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32;
+};
+
+// Offsets (bytes) into the three caller buffers.
+struct Plan {
+  // params: fp32 masters then bf16 copies
+  size_t w[6], wb[6];   // 0 wte, 1 lm_head, 2 qkv, 3 proj, 4 fc, 5 mproj (per-group contiguous over layers)
+  size_t param_bytes;
+  // state
+  size_t g[6], mom[6], am[2], av[2];
+  size_t state_bytes;
+  // activations
+  size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
+  size_t xf, rf, z, stats, zt, row_loss, loss;
+  size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv;
+  size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, rope, err, tok, tgt;
+  size_t act_bytes;
+  size_t splitk_elems;
+  int splits_w[4];    // dW split-K factors: qkv, proj, fc, mproj
+  int splits_lm;      // lm_head dx split-K factor
+};
+
+size_t al(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Bump {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    size_t o = off;
+    off = al(off + bytes);
+    return o;
+  }
+};
+
+int choose_splits(long long tiles, long long kblocks) {
+  const int sms = 148;
+  int best = 1;
+  double best_cost = 1e30;
+  for (int s = 1; s <= 16; ++s) {
+    if (kblocks / s < 8 && s > 1) break;
+    const double waves = std::ceil(static_cast<double>(tiles * s) / sms);
+    const double cost = waves * std::ceil(static_cast<double>(kblocks) / s) * (s > 1 ? 1.03 : 1.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
+}
+
+int dims_from(const gpt_config* c, Dims& D) {
+  if (!c) return fail(GPT_EINVAL, "null config");
+  if (c->depth < 1 || c->depth > 256) return fail(GPT_EINVAL, "depth out of range");
+  if (c->head_dim != 128) return fail(GPT_EINVAL, "head_dim must be 128");
+  if (c->mlp_mult != 4) return fail(GPT_EINVAL, "mlp_mult must be 4");
+  if (c->precision != 0) return fail(GPT_EINVAL, "only precision 0 (bf16) is supported");
+  if (c->ns_tf32_steps < 0 || c->ns_tf32_steps > 5) return fail(GPT_EINVAL, "ns_tf32_steps must be in 0..5");
+  D.L = c->depth;
+  D.d = c->d_model ? c->d_model : 64 * c->depth;
+  if (D.d % 128 || D.d > 2048) return fail(GPT_EINVAL, "d_model must be a multiple of 128, at most 2048");
+  D.H = D.d / 128;
+  D.F = 4 * D.d;
+  D.V = c->vocab;
+  if (D.V < 8 || D.V % 8 || D.V > 131072) return fail(GPT_EINVAL, "vocab must be a multiple of 8 in [8, 131072]");
+  D.B = c->batch;
+  D.T = c->seq_len;
+  if (D.B < 1 || D.T < 1) return fail(GPT_EINVAL, "batch and seq_len must be positive");
+  const long long M = 1ll * D.B * D.T;
+  if (M > (1ll << 30)) return fail(GPT_EINVAL, "batch * seq_len too large");
+  D.M = static_cast<int>(M);
+  D.Mc = c->lm_chunk_rows > 0 ? c->lm_chunk_rows : 8192;
+  D.Mc = std::min(D.Mc, D.M);
+  D.tiles_lm = (D.V + 255) / 256;
+  D.n_tf32 = c->ns_tf32_steps;
+  return GPT_OK;
+}
+
+void make_plan(const Dims& D, Plan& P) {
+  const size_t L = D.L, d = D.d, F = D.F, V = D.V, M = D.M, H = D.H;
+  const size_t numel[6] = {V * d, d * V, L * d * 3 * d, L * d * d, L * d * F, L * F * d};
+  Bump pb;
+  for (int i = 0; i < 6; ++i) P.w[i] = pb.take(numel[i] * 4);
+  for (int i = 0; i < 6; ++i) P.wb[i] = pb.take(numel[i] * 2);
+  P.param_bytes = pb.off;
+  Bump sb;
+  for (int i = 0; i < 6; ++i) P.g[i] = sb.take(numel[i] * 4);
+  P.mom[0] = P.mom[1] = 0;
+  for (int i = 2; i < 6; ++i) P.mom[i] = sb.take(numel[i] * 4);
+  for (int i = 0; i < 2; ++i) {
+    P.am[i] = sb.take(numel[i] * 4);
+    P.av[i] = sb.take(numel[i] * 4);
+  }
+  P.state_bytes = sb.off;
+
+  // split-K plans for the weight gradients (contraction over the M tokens)
+  const long long kb = (M + 63) / 64;
+  const long long shp[4][2] = {{(long long)d, 3 * (long long)d}, {(long long)d, (long long)d},
+                               {(long long)d, (long long)F}, {(long long)F, (long long)d}};
+  size_t sk = 0;
+  for (int i = 0; i < 4; ++i) {
+    const long long tiles = ((shp[i][0] + 127) / 128) * ((shp[i][1] + 255) / 256);
+    P.splits_w[i] = choose_splits(tiles, kb);
+    if (P.splits_w[i] > 1) sk = std::max<size_t>(sk, static_cast<size_t>(P.splits_w[i]) * shp[i][0] * shp[i][1]);
+  }
+  {
+    const long long tiles = ((D.Mc + 127) / 128) * ((d + 255) / 256);
+    P.splits_lm = choose_splits(tiles, (V + 63) / 64);
+    if (P.splits_lm > 1) sk = std::max<size_t>(sk, static_cast<size_t>(P.splits_lm) * D.Mc * d);
+  }
+  P.splitk_elems = sk;
+
+  Bump ab;
+  P.x = ab.take(M * d * 4);
+  P.xn1 = ab.take(L * M * d * 2);
+  P.r1 = ab.take(L * M * 4);
+  P.q = ab.take(L * M * d * 2);
+  P.k = ab.take(L * M * d * 2);
+  P.v = ab.take(L * M * d * 2);
+  P.rq = ab.take(L * M * H * 4);
+  P.rk = ab.take(L * M * H * 4);
+  P.o = ab.take(L * M * d * 2);
+  P.lse = ab.take(L * M * H * 4);
+  P.xn2 = ab.take(L * M * d * 2);
+  P.r2 = ab.take(L * M * 4);
+  P.h = ab.take(L * M * F * 2);
+  P.xf = ab.take(M * d * 2);
+  P.rf = ab.take(M * 4);
+  P.z = ab.take(static_cast<size_t>(D.Mc) * V * 2);
+  P.stats = ab.take(static_cast<size_t>(D.Mc) * D.tiles_lm * 8);
+  P.zt = ab.take(static_cast<size_t>(D.Mc) * 4);
+  P.row_loss = ab.take(M * 4);
+  P.loss = ab.take(16);
+  P.dx = ab.take(M * d * 4);
+  P.dxb = ab.take(M * d * 2);
+  P.dxn = ab.take(M * d * 4);
+  P.du = ab.take(M * F * 2);
+  P.dy = ab.take(M * d * 2);
+  P.dqf = ab.take(M * d * 4);
+  P.dk = ab.take(M * d * 2);
+  P.dv = ab.take(M * d * 2);
+  P.Dv = ab.take(M * H * 4);
+  P.dqkv = ab.take(M * 3 * d * 2);
+  P.splitk = ab.take(std::max<size_t>(sk, 4) * 4);
+  P.embws = ab.take(embed_bwd_workspace(D.M));
+  const size_t xelems = std::max({L * d * 3 * d, L * d * d, 2 * L * d * F});
+  P.X0 = ab.take(xelems * 4);
+  P.X1 = ab.take(xelems * 4);
+  // transposed copies, read K-major by the tf32 steps of Newton-Schulz
+  P.XT0 = ab.take(D.n_tf32 > 0 ? xelems * 4 : 16);
+  P.XT1 = ab.take(D.n_tf32 > 1 ? xelems * 4 : 16);
+  P.Abuf = ab.take(2 * L * d * d * 4);
+  P.Bbuf = ab.take(2 * L * d * d * 4);
+  P.inv_norm = ab.take(4 * L * 4);
+  P.normws = ab.take(muon_norm_workspace(4 * D.L));
+  P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8);
+  P.err = ab.take(16);
+  P.tok = ab.take(M * 4);
+  P.tgt = ab.take(M * 4);
+  P.act_bytes = ab.off;
+}
+
+// ------------------------------------------------------- device-side init
+
+__device__ __forceinline__ uint64_t splitmix64(uint64_t x) {
+  x += 0x9E3779B97F4A7C15ull;
+  x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+  x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+  return x ^ (x >> 31);
+}
+
+__global__ void init_normal_kernel(float* w, bf16* wb, long long n, uint64_t seed, uint64_t stream_id, float std) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const uint64_t h1 = splitmix64(seed ^ splitmix64(stream_id * 0x100000001B3ull + 2 * i));
+    const uint64_t h2 = splitmix64(seed ^ splitmix64(stream_id * 0x100000001B3ull + 2 * i + 1));
+    const double u1 = (static_cast<double>(h1 >> 11) + 1.0) * (1.0 / 9007199254740992.0);
+    const double u2 = static_cast<double>(h2 >> 11) * (1.0 / 9007199254740992.0);
+    const float g = static_cast<float>(sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2)) * std;
+    const bf16 b = __float2bfloat16_rn(g);
+    wb[i] = b;
+    w[i] = __bfloat162float(b);
+  }
+}
+
+__global__ void check_range_kernel(const int* v, int n, int V, int* err) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    if (v[i] < 0 || v[i] >= V) atomicOr(err, ERRF_TOKEN_RANGE);
+}
+
+// targets out of range are clamped to 0 (the error word already records them)
+__global__ void clamp_targets_kernel(const int* src, int* dst, int n, int V) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int t = src[i];
+    dst[i] = (t < 0 || t >= V) ? 0 : t;
+  }
+}
+
+}  // namespace
+
+struct gpt_ctx {
+  gpt_config cfg;
+  Dims D;
+  Plan P;
+  uint8_t* pbuf;
+  uint8_t* sbuf;
+  uint8_t* abuf;
+  cudaStream_t stream;
+  long long adam_step = 0;
+  int64_t launches = 0;
+  // event profiler
+  uint32_t prof_mask = 0;
+  struct Rec { cudaEvent_t a, b; int cat; };
+  std::vector<Rec> recs;
+  size_t recs_used = 0;
+  double prof_ms[GPT_PROF_COUNT] = {};
+  int64_t prof_n[GPT_PROF_COUNT] = {};
+  ~gpt_ctx() {
+    for (Rec& r : recs) {
+      cudaEventDestroy(r.a);
+      cudaEventDestroy(r.b);
+    }
+  }
+  Rec* next_rec() {
+    if (recs_used == recs.size()) {
+      Rec r{};
+      if (cudaEventCreate(&r.a) != cudaSuccess || cudaEventCreate(&r.b) != cudaSuccess) return nullptr;
+      recs.push_back(r);
+    }
+    return &recs[recs_used++];
+  }
+
+  template <typename T = float>
+  T* W(int i) const { return reinterpret_cast<T*>(pbuf + P.w[i]); }
+  bf16* Wb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wb[i]); }
+  float* G(int i) const { return reinterpret_cast<float*>(sbuf + P.g[i]); }
+  float* Mom(int i) const { return reinterpret_cast<float*>(sbuf + P.mom[i]); }
+  template <typename T>
+  T* A(size_t off) const { return reinterpret_cast<T*>(abuf + off); }
+  int* err() const { return A<int>(P.err); }
+};
+
+namespace {
+
+// Records a pair of events around the launches in its scope when the
+// category is enabled.
+struct ProfScope {
+  gpt_ctx* c;
+  gpt_ctx::Rec* r = nullptr;
+  ProfScope(gpt_ctx* ctx, int cat) : c(ctx) {
+    if (c && ((c->prof_mask >> cat) & 1u)) {
+      r = c->next_rec();
+      if (r) {
+        r->cat = cat;
+        cudaEventRecord(r->a, c->stream);
+      }
+    }
+  }
+  ~ProfScope() {
+    if (r) cudaEventRecord(r->b, c->stream);
+  }
+};
+
+// group index (0..5) and element offset of tensor id
+bool locate(const gpt_ctx* c, int id, int& grp, size_t& off, int& rows, int& cols) {
+  const Dims& D = c->D;
+  if (id == 0) { grp = 0; off = 0; rows = D.V; cols = D.d; return true; }
+  if (id == 1) { grp = 1; off = 0; rows = D.d; cols = D.V; return true; }
+  const int k = id - 2;
+  if (k < 0 || k >= 4 * D.L) return false;
+  const int l = k / 4, j = k % 4;
+  const int shp[4][2] = {{D.d, 3 * D.d}, {D.d, D.d}, {D.d, D.F}, {D.F, D.d}};
+  grp = 2 + j;
+  rows = shp[j][0];
+  cols = shp[j][1];
+  off = static_cast<size_t>(l) * rows * cols;
+  return true;
+}
+
+GemmCall base_call(int M, int N, int K) {
+  GemmCall c;
+  c.M = M; c.N = N; c.K = K;
+  return c;
+}
+
+// fp32 output [M][N] (contiguous), optionally split over K with a deterministic reduce.
+int run_f32(gpt_ctx* c, GemmCall g, float* out, bool accumulate, int splits, int cat) {
+  ProfScope ps(c, cat);
+  g.out_es = 4;
+  g.aux_es = 4;
+  g.p.err = c->err();
+  if (splits <= 1) {
+    g.epi = accumulate ? EPI_ACC : EPI_STORE;
+    g.splits = 1;
+    g.p.out = out;
+    g.p.ldo = g.N;
+    GPT_CK(gemm_run(g, c->stream));
+    c->launches += 1;
+    return GPT_OK;
+  }
+  float* part = c->A<float>(c->P.splitk);
+  const long long n = 1ll * g.M * g.N;
+  if (static_cast<size_t>(n) * splits > c->P.splitk_elems) return fail(GPT_EINVAL, "split-K scratch too small");
+  g.epi = EPI_STORE;
+  g.splits = splits;
+  g.p.out = part;
+  g.p.ldo = g.N;
+  g.p.split_stride = n;
+  GPT_CK(gemm_run(g, c->stream));
+  launch_splitk_reduce(part, g.p.splits, n, n, out, accumulate, c->stream);
+  c->launches += 2;
+  return GPT_OK;
+}
+
+int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_out, bool acc) {
+  const Dims& D = c->D;
+  const Plan& P = c->P;
+  cudaStream_t s = c->stream;
+  const int M = D.M, d = D.d, F = D.F, V = D.V, H = D.H, L = D.L;
+  const size_t Md = static_cast<size_t>(M) * d;
+  float* x = c->A<float>(P.x);
+  bf16* xn1 = c->A<bf16>(P.xn1);
+  bf16* xn2 = c->A<bf16>(P.xn2);
+  float* r1 = c->A<float>(P.r1);
+  float* r2 = c->A<float>(P.r2);
+  bf16* q = c->A<bf16>(P.q);
+  bf16* k = c->A<bf16>(P.k);
+  bf16* v = c->A<bf16>(P.v);
+  float* rq = c->A<float>(P.rq);
+  float* rk = c->A<float>(P.rk);
+  bf16* o = c->A<bf16>(P.o);
+  float* lse = c->A<float>(P.lse);
+  bf16* h = c->A<bf16>(P.h);
+  bf16* xf = c->A<bf16>(P.xf);
+  float* rf = c->A<float>(P.rf);
+  const float2* rope = c->A<float2>(P.rope);
+  int* tgt = c->A<int>(P.tgt);
+  int* err = c->err();
+
+  // ids: range check (latched), targets clamped into the private copy
+  {
+    ProfScope ps(c, GPT_PROF_EMBED);
+    check_range_kernel<<<64, 256, 0, s>>>(tgt_in, M, V, err);
+    if (tgt_in != tgt) clamp_targets_kernel<<<64, 256, 0, s>>>(tgt_in, tgt, M, V);
+    else clamp_targets_kernel<<<64, 256, 0, s>>>(tgt, tgt, M, V);
+    launch_embed_fwd(tok, c->Wb(0), x, M, d, V, err, s);
+  }
+  c->launches += 3;
+
+  // ---------------------------------------------------------------- forward
+  for (int l = 0; l < L; ++l) {
+    bf16* xn1l = xn1 + l * Md;
+    bf16* xn2l = xn2 + l * Md;
+    bf16* ql = q + l * Md;
+    bf16* kl = k + l * Md;
+    bf16* vl = v + l * Md;
+    bf16* ol = o + l * Md;
+    bf16* hl = h + static_cast<size_t>(l) * M * F;
+    float* lsel = lse + static_cast<size_t>(l) * M * H;
+    {
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
+    }
+    {
+      ProfScope ps(c, GPT_PROF_QKV_GEMM);
+      GemmCall g = base_call(M, 3 * d, d);
+      g.A = xn1l; g.lda = d;
+      g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.b_mn = true; g.ldb = 3 * d;
+      g.bn = 128; g.epi = EPI_QKV; g.out_es = 2; g.aux_es = 2;
+      g.p.qkv_out[0] = ql; g.p.qkv_out[1] = kl; g.p.qkv_out[2] = vl;
+      g.p.f32a = rq + static_cast<size_t>(l) * M * H;
+      g.p.f32b = rk + static_cast<size_t>(l) * M * H;
+      g.p.rope = rope; g.p.T = D.T; g.p.H = H; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      ProfScope ps(c, GPT_PROF_ATTN_FWD);
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s);
+    }
+    {
+      ProfScope ps(c, GPT_PROF_PROJ_GEMM);
+      GemmCall g = base_call(M, d, d);
+      g.A = ol; g.lda = d;
+      g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.b_mn = true; g.ldb = d;
+      g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
+      g.p.out = x; g.p.ldo = d; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_rmsnorm_fwd(x, xn2l, r2 + static_cast<size_t>(l) * M, M, d, s);
+    }
+    {
+      ProfScope ps(c, GPT_PROF_FC_GEMM);
+      GemmCall g = base_call(M, F, d);
+      g.A = xn2l; g.lda = d;
+      g.B = c->Wb(4) + static_cast<size_t>(l) * d * F; g.b_mn = true; g.ldb = F;
+      g.epi = EPI_RELU2; g.out_es = 2; g.aux_es = 2;
+      g.p.out = hl; g.p.ldo = F; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      ProfScope ps(c, GPT_PROF_DOWN_GEMM);
+      GemmCall g = base_call(M, d, F);
+      g.A = hl; g.lda = F;
+      g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.b_mn = true; g.ldb = d;
+      g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
+      g.p.out = x; g.p.ldo = d; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    c->launches += 7;
+  }
+  {
+    ProfScope ps(c, GPT_PROF_NORM);
+    launch_rmsnorm_fwd(x, xf, rf, M, d, s);
+  }
+  c->launches += 1;
+
+  // ------------------------------------- fused lm_head + cross-entropy, chunked
+  float* dxn = c->A<float>(P.dxn);
+  bf16* z = c->A<bf16>(P.z);
+  float* row_loss = c->A<float>(P.row_loss);
+  for (int r0 = 0; r0 < M; r0 += D.Mc) {
+    const int rows = std::min(D.Mc, M - r0);
+    {
+      ProfScope ps(c, GPT_PROF_LOGITS_GEMM);
+      GemmCall g = base_call(rows, V, d);
+      g.A = xf + static_cast<size_t>(r0) * d; g.lda = d;
+      g.B = c->Wb(1); g.b_mn = true; g.ldb = V;
+      g.epi = EPI_LOGITS; g.out_es = 2; g.aux_es = 2;
+      g.p.out = z; g.p.ldo = V;
+      g.p.f32a = c->A<float>(P.stats); g.p.f32b = c->A<float>(P.zt); g.p.tgt = tgt + r0; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      ProfScope ps(c, GPT_PROF_CE_FINISH);
+      launch_ce_finish(z, c->A<float2>(P.stats), c->A<float>(P.zt), tgt + r0, row_loss + r0, rows, V, D.tiles_lm,
+                       1.f / static_cast<float>(M), s);
+    }
+    c->launches += 2;
+    {
+      // dxf rows = dz W_lm^T  (contraction over the vocabulary)
+      GemmCall g = base_call(rows, d, V);
+      g.A = z; g.lda = V;
+      g.B = c->Wb(1); g.ldb = V;   // B(n = model dim, k = vocab) = W_lm[n][k]
+      int rc = run_f32(c, g, dxn + static_cast<size_t>(r0) * d, false, P.splits_lm, GPT_PROF_LM_DX_GEMM);
+      if (rc) return rc;
+    }
+    {
+      // dW_lm += xf^T dz  (contraction over the rows of the chunk)
+      GemmCall g = base_call(d, V, rows);
+      g.A = xf + static_cast<size_t>(r0) * d; g.a_mn = true; g.lda = d;
+      g.B = z; g.b_mn = true; g.ldb = V;
+      int rc = run_f32(c, g, c->G(1), acc || r0 > 0, 1, GPT_PROF_LM_DW_GEMM);
+      if (rc) return rc;
+    }
+  }
+  launch_sum_scale(row_loss, M, 1.f / static_cast<float>(M), loss_out, s);
+  c->launches += 1;
+
+  // --------------------------------------------------------------- backward
+  float* dx = c->A<float>(P.dx);
+  bf16* dxb = c->A<bf16>(P.dxb);
+  bf16* du = c->A<bf16>(P.du);
+  bf16* dy = c->A<bf16>(P.dy);
+  float* dqf = c->A<float>(P.dqf);
+  bf16* dk = c->A<bf16>(P.dk);
+  bf16* dv = c->A<bf16>(P.dv);
+  bf16* dqkv = c->A<bf16>(P.dqkv);
+  {
+    ProfScope ps(c, GPT_PROF_NORM);
+    launch_rmsnorm_bwd(dxn, xf, rf, dx, dxb, M, d, false, s);
+  }
+  c->launches += 1;
+  for (int l = L - 1; l >= 0; --l) {
+    bf16* xn1l = xn1 + l * Md;
+    bf16* xn2l = xn2 + l * Md;
+    bf16* hl = h + static_cast<size_t>(l) * M * F;
+    bf16* ol = o + l * Md;
+    // MLP down: dh = dx W_d^T, du = dh * 2 relu(u) with relu(u) = sqrt(h)
+    {
+      ProfScope ps(c, GPT_PROF_DX_GEMM);
+      GemmCall g = base_call(M, F, d);
+      g.A = dxb; g.lda = d;
+      g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.ldb = d;   // B(n = F index, k = d index)
+      g.epi = EPI_DRELU2; g.out_es = 2; g.aux_es = 2;
+      g.p.out = du; g.p.ldo = F; g.p.aux = hl; g.p.ld_aux = F; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+      c->launches += 1;
+    }
+    {
+      GemmCall g = base_call(F, d, M);   // dW_d = h^T dx
+      g.A = hl; g.a_mn = true; g.lda = F;
+      g.B = dxb; g.b_mn = true; g.ldb = d;
+      int rc = run_f32(c, g, c->G(5) + static_cast<size_t>(l) * F * d, acc, P.splits_w[3], GPT_PROF_DW_GEMM);
+      if (rc) return rc;
+    }
+    {
+      GemmCall g = base_call(M, d, F);   // dxn2 = du W_fc^T
+      g.A = du; g.lda = F;
+      g.B = c->Wb(4) + static_cast<size_t>(l) * d * F; g.ldb = F;
+      int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
+      if (rc) return rc;
+    }
+    {
+      GemmCall g = base_call(d, F, M);   // dW_fc = xn2^T du
+      g.A = xn2l; g.a_mn = true; g.lda = d;
+      g.B = du; g.b_mn = true; g.ldb = F;
+      int rc = run_f32(c, g, c->G(4) + static_cast<size_t>(l) * d * F, acc, P.splits_w[2], GPT_PROF_DW_GEMM);
+      if (rc) return rc;
+    }
+    {
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_rmsnorm_bwd(dxn, xn2l, r2 + static_cast<size_t>(l) * M, dx, dxb, M, d, true, s);
+    }
+    c->launches += 1;
+    // attention output projection
+    {
+      ProfScope ps(c, GPT_PROF_DX_GEMM);
+      GemmCall g = base_call(M, d, d);   // dy = dx W_o^T
+      g.A = dxb; g.lda = d;
+      g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.ldb = d;
+      g.epi = EPI_STORE; g.out_es = 2; g.aux_es = 2;
+      g.p.out = dy; g.p.ldo = d; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+      c->launches += 1;
+    }
+    {
+      GemmCall g = base_call(d, d, M);   // dW_o = o^T dx
+      g.A = ol; g.a_mn = true; g.lda = d;
+      g.B = dxb; g.b_mn = true; g.ldb = d;
+      int rc = run_f32(c, g, c->G(3) + static_cast<size_t>(l) * d * d, acc, P.splits_w[1], GPT_PROF_DW_GEMM);
+      if (rc) return rc;
+    }
+    {
+      ProfScope ps(c, GPT_PROF_ATTN_BWD);
+      launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s);
+    }
+    {
+      ProfScope ps(c, GPT_PROF_QK_BWD);
+      launch_qk_bwd(dqf, dk, dv, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
+                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s);
+    }
+    c->launches += 3;
+    {
+      GemmCall g = base_call(M, d, 3 * d);   // dxn1 = dqkv W_qkv^T
+      g.A = dqkv; g.lda = 3 * d;
+      g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.ldb = 3 * d;
+      int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
+      if (rc) return rc;
+    }
+    {
+      GemmCall g = base_call(d, 3 * d, M);   // dW_qkv = xn1^T dqkv
+      g.A = xn1l; g.a_mn = true; g.lda = d;
+      g.B = dqkv; g.b_mn = true; g.ldb = 3 * d;
+      int rc = run_f32(c, g, c->G(2) + static_cast<size_t>(l) * d * 3 * d, acc, P.splits_w[0], GPT_PROF_DW_GEMM);
+      if (rc) return rc;
+    }
+    {
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_rmsnorm_bwd(dxn, xn1l, r1 + static_cast<size_t>(l) * M, dx, dxb, M, d, true, s);
+    }
+    c->launches += 1;
+  }
+  {
+    ProfScope ps(c, GPT_PROF_EMBED);
+    launch_embed_bwd(tok, dx, c->G(0), M, d, V, c->A<void>(P.embws), acc, s);
+  }
+  c->launches += 2 * ((M + 32767) / 32768);
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+// Five Polar Express steps on X0 ([z][r][c], es0-typed); returns the buffer
+// and element size holding the result.  Steps run on tf32 (fp32 storage) while
+// t < n_tf32, then on bf16.  A tf32 step reads X^T (XT0, [z][c][r]) as its
+// K-major B operand and, when the next step is tf32 too, writes X'^T beside X'.
+int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* XT0, void* XT1, void* Ab,
+                  void* Bb, int n_tf32, cudaStream_t s, int* err, void** out, int* out_es, int64_t* launches) {
+  ProfScope ps(pc, GPT_PROF_NS_GEMM);
+  void* cur = X0;
+  void* nxt = X1;
+  void* curT = XT0;
+  void* nxtT = XT1;
+  const double (*kPolarCoef)[3] = polar_coefficients();
+  for (int t = 0; t < kPolarSteps; ++t) {
+    const int es = t < n_tf32 ? 4 : 2;
+    const bool last = t + 1 == kPolarSteps;
+    const int es_next = last ? es : ((t + 1) < n_tf32 ? 4 : 2);
+    const bool next_T = !last && (t + 1) < n_tf32;
+    const double a = kPolarCoef[t][0], b = kPolarCoef[t][1], cf = kPolarCoef[t][2];
+    {
+      GemmCall g = base_call(r, r, cc);   // A = X X^T
+      g.batch = nz; g.es = es;
+      g.A = cur; g.lda = cc; g.a_bs = 1ll * r * cc;
+      g.B = cur; g.ldb = cc; g.b_bs = 1ll * r * cc;
+      g.bn = 128; g.sym = true; g.epi = EPI_STORE; g.out_es = es; g.aux_es = es;
+      g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      GemmCall g = base_call(r, r, r);    // B = b A + c A A
+      g.batch = nz; g.es = es;
+      g.A = Ab; g.lda = r; g.a_bs = 1ll * r * r;
+      g.B = Ab; g.ldb = r; g.b_bs = 1ll * r * r;
+      g.bn = 128; g.sym = true; g.epi = EPI_AXPBY; g.out_es = es; g.aux_es = es;
+      g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
+      g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
+      g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    {
+      GemmCall g = base_call(r, cc, r);   // X' = a X + B X
+      g.batch = nz; g.es = es;
+      g.A = Bb; g.lda = r; g.a_bs = 1ll * r * r;
+      if (es == 4) {
+        g.B = curT; g.b_mn = false; g.ldb = r; g.b_bs = 1ll * r * cc;   // B(n, k) = X[k][n] = X^T[n][k]
+      } else {
+        g.B = cur; g.b_mn = true; g.ldb = cc; g.b_bs = 1ll * r * cc;
+      }
+      g.bn = 256; g.epi = EPI_AXPBY; g.out_es = es_next; g.aux_es = es;
+      g.p.out = nxt; g.p.ldo = cc; g.p.out_bs = 1ll * r * cc;
+      if (next_T) {
+        g.p.out_t = nxtT;
+        g.p.ldo_t = r;
+      }
+      g.p.aux = cur; g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
+      g.p.alpha = static_cast<float>(a); g.p.beta = 1.f; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    *launches += 3;
+    std::swap(cur, nxt);
+    std::swap(curT, nxtT);
+    *out_es = es_next;
+  }
+  *out = cur;
+  return GPT_OK;
+}
+
+int check_ctx(const gpt_ctx* c) { return c ? GPT_OK : fail(GPT_EINVAL, "null context"); }
+
+}  // namespace
+
+// ======================================================================== ABI
+
+extern "C" {
+
+const char* gpt_last_error(void) { return g_last_error.c_str(); }
+
+int gpt_workspace_size(const gpt_config* cfg, size_t* param_bytes, size_t* state_bytes, size_t* act_bytes) {
+  Dims D;
+  int rc = dims_from(cfg, D);
+  if (rc) return rc;
+  Plan P;
+  make_plan(D, P);
+  if (param_bytes) *param_bytes = P.param_bytes;
+  if (state_bytes) *state_bytes = P.state_bytes;
+  if (act_bytes) *act_bytes = P.act_bytes;
+  return GPT_OK;
+}
+
+int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_buf, void* stream, gpt_ctx** out) {
+  if (!out) return fail(GPT_EINVAL, "null output pointer");
+  *out = nullptr;
+  Dims D;
+  int rc = dims_from(cfg, D);
+  if (rc) return rc;
+  if (!param_buf || !state_buf || !act_buf) return fail(GPT_EINVAL, "null buffer");
+  if ((reinterpret_cast<uintptr_t>(param_buf) | reinterpret_cast<uintptr_t>(state_buf) |
+       reinterpret_cast<uintptr_t>(act_buf)) & (kAlign - 1))
+    return fail(GPT_EINVAL, "buffers must be 256-byte aligned");
+  gpt_ctx* c = new gpt_ctx();
+  c->cfg = *cfg;
+  c->D = D;
+  make_plan(D, c->P);
+  c->pbuf = static_cast<uint8_t*>(param_buf);
+  c->sbuf = static_cast<uint8_t*>(state_buf);
+  c->abuf = static_cast<uint8_t*>(act_buf);
+  c->stream = static_cast<cudaStream_t>(stream);
+  cudaStream_t s = c->stream;
+  auto bad = [&](cudaError_t e, const char* what) {
+    delete c;
+    return fail(GPT_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+  };
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(c->sbuf, 0, c->P.state_bytes, s)) != cudaSuccess) return bad(e, "zero state");
+  if ((e = cudaMemsetAsync(c->A<int>(c->P.err), 0, 16, s)) != cudaSuccess) return bad(e, "zero error word");
+  const size_t numel[6] = {static_cast<size_t>(D.V) * D.d, static_cast<size_t>(D.d) * D.V,
+                           static_cast<size_t>(D.L) * D.d * 3 * D.d, static_cast<size_t>(D.L) * D.d * D.d,
+                           static_cast<size_t>(D.L) * D.d * D.F, static_cast<size_t>(D.L) * D.F * D.d};
+  for (int i = 0; i < 6; ++i) {
+    init_normal_kernel<<<1024, 256, 0, s>>>(c->W(i), c->Wb(i), static_cast<long long>(numel[i]), cfg->seed, i, 0.02f);
+  }
+  launch_rope_table(c->A<float2>(c->P.rope), D.T, s);
+  if ((e = cudaGetLastError()) != cudaSuccess) return bad(e, "init kernels");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return bad(e, "init sync");
+  c->launches = 7;
+  *out = c;
+  return GPT_OK;
+}
+
+int gpt_fwd_bwd(gpt_ctx* c, const int32_t* tokens, const int32_t* targets, float* loss_out, int accumulate) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!tokens || !targets || !loss_out) return fail(GPT_EINVAL, "null pointer");
+  if ((reinterpret_cast<uintptr_t>(tokens) | reinterpret_cast<uintptr_t>(targets)) & 3)
+    return fail(GPT_EINVAL, "token/target pointers must be 4-byte aligned");
+  return forward_backward(c, tokens, targets, loss_out, accumulate != 0);
+}
+
+int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  const Dims& D = c->D;
+  const Plan& P = c->P;
+  cudaStream_t s = c->stream;
+  const int L = D.L, d = D.d, F = D.F;
+  float* inv = c->A<float>(P.inv_norm);
+  // momentum and Frobenius norms of every block matrix
+  const long long ne[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+  {
+    ProfScope ps(c, GPT_PROF_MUON_ELEM);
+    for (int j = 0; j < 4; ++j)
+      launch_muon_momentum(c->Mom(2 + j), c->G(2 + j), ne[j], L, momentum, 1e-7f, inv + j * L, c->A<void>(P.normws),
+                           s);
+  }
+  c->launches += 8;
+  const int es0 = D.n_tf32 > 0 ? 4 : 2;
+  void* X0 = c->A<void>(P.X0);
+  void* X1 = c->A<void>(P.X1);
+  void* XT0 = c->A<void>(P.XT0);
+  void* XT1 = c->A<void>(P.XT1);
+  void* Ab = c->A<void>(P.Abuf);
+  void* Bb = c->A<void>(P.Bbuf);
+  // three Newton-Schulz batches, all with r = d rows: q|k|v (c = 3d), attention
+  // output (c = d), and MLP up plus transposed MLP down (c = 4d)
+  struct Member { int grp; bool transpose; };
+  struct Batch { int nz; int cc; Member m[2]; int nm; };
+  const Batch batches[3] = {{L, 3 * d, {{2, false}}, 1}, {L, d, {{3, false}}, 1},
+                            {2 * L, F, {{4, false}, {5, true}}, 2}};
+  for (const Batch& bt : batches) {
+    const size_t per = static_cast<size_t>(d) * bt.cc;
+    for (int i = 0; i < bt.nm; ++i) {
+      ProfScope ps(c, GPT_PROF_MUON_ELEM);
+      const Member& mm = bt.m[i];
+      void* dst = static_cast<uint8_t*>(X0) + static_cast<size_t>(i) * L * per * es0;
+      launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, es0, L, d, bt.cc, mm.transpose, s);
+      c->launches += 1;
+      if (D.n_tf32 > 0) {
+        void* dstT = static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * L * per * es0;
+        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, es0, L, bt.cc, d, !mm.transpose, s);
+        c->launches += 1;
+      }
+    }
+    void* res = nullptr;
+    int res_es = es0;
+    rc = newton_schulz(c, bt.nz, d, bt.cc, X0, X1, XT0, XT1, Ab, Bb, D.n_tf32, s, c->err(), &res, &res_es,
+                       &c->launches);
+    if (rc) return rc;
+    for (int i = 0; i < bt.nm; ++i) {
+      ProfScope ps(c, GPT_PROF_MUON_ELEM);
+      const Member& mm = bt.m[i];
+      const int rows = mm.grp == 5 ? F : d;
+      const int cols = mm.grp == 2 ? 3 * d : (mm.grp == 3 ? d : (mm.grp == 4 ? F : d));
+      const float scale = sqrtf(std::max(1.f, static_cast<float>(rows) / static_cast<float>(cols)));
+      const void* src = static_cast<const uint8_t*>(res) + static_cast<size_t>(i) * L * per * res_es;
+      launch_muon_apply(c->W(mm.grp), c->Wb(mm.grp), src, res_es, L, d, bt.cc, mm.transpose, lr, weight_decay,
+                        scale, s);
+      c->launches += 1;
+    }
+  }
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  c->adam_step += 1;
+  const double t = static_cast<double>(c->adam_step);
+  const float bc1 = static_cast<float>(1.0 - pow(static_cast<double>(beta1), t));
+  const float bc2 = static_cast<float>(1.0 - pow(static_cast<double>(beta2), t));
+  const long long n = 1ll * c->D.V * c->D.d;
+  ProfScope ps(c, GPT_PROF_ADAMW);
+  for (int i = 0; i < 2; ++i) {
+    launch_adamw(c->W(i), c->G(i), reinterpret_cast<float*>(c->sbuf + c->P.am[i]),
+                 reinterpret_cast<float*>(c->sbuf + c->P.av[i]), c->Wb(i), n, lr, beta1, beta2, eps, weight_decay,
+                 bc1, bc2, c->stream);
+  }
+  c->launches += 2;
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_train_step_host(gpt_ctx* c, const int32_t* tokens_host, const int32_t* targets_host, const gpt_hparams* hp,
+                        float* loss_host) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!tokens_host || !targets_host || !hp || !loss_host) return fail(GPT_EINVAL, "null pointer");
+  const size_t bytes = static_cast<size_t>(c->D.M) * 4;
+  int* tok = c->A<int>(c->P.tok);
+  int* tgt = c->A<int>(c->P.tgt);
+  GPT_CK(cudaMemcpyAsync(tok, tokens_host, bytes, cudaMemcpyHostToDevice, c->stream));
+  GPT_CK(cudaMemcpyAsync(tgt, targets_host, bytes, cudaMemcpyHostToDevice, c->stream));
+  float* loss = c->A<float>(c->P.loss);
+  rc = forward_backward(c, tok, tgt, loss, false);
+  if (rc) return rc;
+  rc = muon_step(c, hp->muon_lr, hp->muon_momentum, hp->muon_wd);
+  if (rc) return rc;
+  rc = adamw_step(c, hp->adam_lr, hp->adam_beta1, hp->adam_beta2, hp->adam_eps, hp->adam_wd);
+  if (rc) return rc;
+  GPT_CK(cudaMemcpyAsync(loss_host, loss, sizeof(float), cudaMemcpyDeviceToHost, c->stream));
+  GPT_CK(cudaStreamSynchronize(c->stream));
+  return gpt_check(c);
+}
+
+int gpt_num_tensors(const gpt_ctx* c) { return c ? 2 + 4 * c->D.L : 0; }
+
+int gpt_tensor_info(const gpt_ctx* c, int id, int32_t* rows, int32_t* cols, int32_t* group) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  int grp, r, cc;
+  size_t off;
+  if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
+  if (rows) *rows = r;
+  if (cols) *cols = cc;
+  if (group) *group = grp < 2 ? GPT_GROUP_ADAMW : GPT_GROUP_MUON;
+  return GPT_OK;
+}
+
+static int tensor_ptr(gpt_ctx* c, int id, int kind, float** p, size_t* n, int* grp_out, size_t* off_out) {
+  int grp, r, cc;
+  size_t off;
+  if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
+  float* base = nullptr;
+  switch (kind) {
+    case GPT_KIND_PARAM: base = c->W(grp); break;
+    case GPT_KIND_GRAD: base = c->G(grp); break;
+    case GPT_KIND_MOM:
+      if (grp < 2) return fail(GPT_EINVAL, "momentum exists only for block matrices");
+      base = c->Mom(grp);
+      break;
+    case GPT_KIND_ADAM_M:
+    case GPT_KIND_ADAM_V:
+      if (grp >= 2) return fail(GPT_EINVAL, "AdamW moments exist only for the embedding and lm_head");
+      base = reinterpret_cast<float*>(c->sbuf + (kind == GPT_KIND_ADAM_M ? c->P.am[grp] : c->P.av[grp]));
+      break;
+    default:
+      return fail(GPT_EINVAL, "unknown tensor kind");
+  }
+  *p = base + off;
+  *n = static_cast<size_t>(r) * cc;
+  *grp_out = grp;
+  *off_out = off;
+  return GPT_OK;
+}
+
+int gpt_get_tensor(gpt_ctx* c, int id, int kind, float* dst) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!dst) return fail(GPT_EINVAL, "null destination");
+  float* p;
+  size_t n, off;
+  int grp;
+  rc = tensor_ptr(c, id, kind, &p, &n, &grp, &off);
+  if (rc) return rc;
+  GPT_CK(cudaMemcpyAsync(dst, p, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  return GPT_OK;
+}
+
+int gpt_set_tensor(gpt_ctx* c, int id, int kind, const float* src) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!src) return fail(GPT_EINVAL, "null source");
+  float* p;
+  size_t n, off;
+  int grp;
+  rc = tensor_ptr(c, id, kind, &p, &n, &grp, &off);
+  if (rc) return rc;
+  GPT_CK(cudaMemcpyAsync(p, src, n * 4, cudaMemcpyDeviceToDevice, c->stream));
+  if (kind == GPT_KIND_PARAM) {
+    launch_cast_bf16(p, c->Wb(grp) + off, static_cast<long long>(n), c->stream);
+    c->launches += 1;
+  }
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_grad_region(const gpt_ctx* c, size_t* offset_bytes, size_t* size_bytes) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  const size_t last = c->P.g[5] + static_cast<size_t>(c->D.L) * c->D.F * c->D.d * 4;
+  if (offset_bytes) *offset_bytes = c->P.g[0];
+  if (size_bytes) *size_bytes = al(last) - c->P.g[0];
+  return GPT_OK;
+}
+
+int gpt_get_row_loss(gpt_ctx* c, float* dst) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!dst) return fail(GPT_EINVAL, "null destination");
+  GPT_CK(cudaMemcpyAsync(dst, c->A<float>(c->P.row_loss), static_cast<size_t>(c->D.M) * 4,
+                         cudaMemcpyDeviceToDevice, c->stream));
+  return GPT_OK;
+}
+
+int gpt_check(gpt_ctx* c) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  GPT_CK(cudaStreamSynchronize(c->stream));
+  int flag = 0;
+  GPT_CK(cudaMemcpy(&flag, c->err(), sizeof(int), cudaMemcpyDeviceToHost));
+  if (flag) GPT_CK(cudaMemset(c->err(), 0, sizeof(int)));
+  if (flag & ERRF_TIMEOUT) return fail(GPT_ETIMEOUT, "a bounded device wait expired");
+  if (flag & ERRF_TOKEN_RANGE) return fail(GPT_ERANGE, "token or target id outside [0, vocab)");
+  if (flag) return fail(GPT_ECUDA, "device error flag set");
+  return GPT_OK;
+}
+
+int64_t gpt_launch_count(const gpt_ctx* c) { return c ? c->launches : 0; }
+
+int gpt_profile_enable(gpt_ctx* c, uint32_t mask) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  c->prof_mask = mask & ((1u << GPT_PROF_COUNT) - 1u);
+  return GPT_OK;
+}
+
+int gpt_profile_read(gpt_ctx* c, double* ms, int64_t* launches) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  GPT_CK(cudaStreamSynchronize(c->stream));
+  for (size_t i = 0; i < c->recs_used; ++i) {
+    float t = 0.f;
+    GPT_CK(cudaEventElapsedTime(&t, c->recs[i].a, c->recs[i].b));
+    c->prof_ms[c->recs[i].cat] += t;
+    c->prof_n[c->recs[i].cat] += 1;
+  }
+  c->recs_used = 0;
+  for (int k = 0; k < GPT_PROF_COUNT; ++k) {
+    if (ms) ms[k] = c->prof_ms[k];
+    if (launches) launches[k] = c->prof_n[k];
+    c->prof_ms[k] = 0.0;
+    c->prof_n[k] = 0;
+  }
+  return GPT_OK;
+}
+
+void gpt_destroy(gpt_ctx* c) { delete c; }
+
+// ------------------------------------------------------------ op-level calls
+
+int gpt_op_matmul_bf16(const void* A, const void* B, float* C, int M, int N, int K, int batch, int a_trans,
+                       int b_trans, void* stream) {
+  if (!A || !B || !C) return fail(GPT_EINVAL, "null pointer");
+  if (M < 0 || N < 0 || K <= 0 || batch < 1 || N % 8 || K % 8) return fail(GPT_EINVAL, "bad matmul shape");
+  if (a_trans && M % 8) return fail(GPT_EINVAL, "M must be a multiple of 8 when A is transposed");
+  GemmCall g = base_call(M, N, K);
+  g.batch = batch;
+  g.A = A; g.a_mn = a_trans != 0; g.lda = a_trans ? M : K; g.a_bs = 1ll * M * K;
+  g.B = B; g.b_mn = b_trans == 0; g.ldb = b_trans ? K : N; g.b_bs = 1ll * K * N;
+  g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
+  g.p.out = C; g.p.ldo = N; g.p.out_bs = 1ll * M * N;
+  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  return GPT_OK;
+}
+
+int gpt_op_matmul_tf32(const float* A, const float* B, float* C, int M, int N, int K, int b_trans, void* stream) {
+  if (!A || !B || !C) return fail(GPT_EINVAL, "null pointer");
+  if (M < 0 || N < 0 || K <= 0 || N % 8 || K % 4) return fail(GPT_EINVAL, "bad matmul shape");
+  if (!b_trans) return fail(GPT_EINVAL, "tf32 operands must be K-major: pass B as [N, K] with b_trans = 1");
+  GemmCall g = base_call(M, N, K);
+  g.es = 4;
+  g.A = A; g.lda = K;
+  g.B = B; g.ldb = K;
+  g.bn = 128; g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
+  g.p.out = C; g.p.ldo = N;
+  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  return GPT_OK;
+}
+
+int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+                         void* stream) {
+  if (!q || !k || !v || !o || !lse) return fail(GPT_EINVAL, "null pointer");
+  if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
+  launch_attn_fwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
+                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream));
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_op_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int T,
+                         void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !Dscratch || !dq || !dk || !dv) return fail(GPT_EINVAL, "null pointer");
+  if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
+  launch_attn_bwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
+                  static_cast<const bf16*>(o), static_cast<const bf16*>(dout), lse, Dscratch, dq,
+                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream));
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream) {
+  if (!x || !y || !rstd) return fail(GPT_EINVAL, "null pointer");
+  if (M < 0 || d < 4 || d % 4 || d > 2048) return fail(GPT_EINVAL, "bad rmsnorm shape");
+  launch_rmsnorm_fwd(x, static_cast<bf16*>(y), rstd, M, d, static_cast<cudaStream_t>(stream));
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+size_t gpt_op_newton_schulz_scratch(int batch, int rows, int cols) {
+  const size_t r = std::min(rows, cols), cc = std::max(rows, cols), n = static_cast<size_t>(batch) * r * cc;
+  return 4 * al(n * 4) + 2 * al(static_cast<size_t>(batch) * r * r * 4) + al(batch * 4) +
+         al(muon_norm_workspace(batch)) + al(n * 2) + al(16);
+}
+
+int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols, int tf32_steps, void* scratch,
+                         void* stream) {
+  if (!G || !X || !scratch) return fail(GPT_EINVAL, "null pointer");
+  if (batch < 1 || rows < 8 || cols < 8 || rows % 8 || cols % 8) return fail(GPT_EINVAL, "bad matrix shape");
+  if (tf32_steps < 0 || tf32_steps > 5) return fail(GPT_EINVAL, "tf32_steps must be in 0..5");
+  if (reinterpret_cast<uintptr_t>(scratch) & (kAlign - 1)) return fail(GPT_EINVAL, "scratch must be 256-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tr = rows > cols;
+  const int r = tr ? cols : rows, cc = tr ? rows : cols;
+  const size_t n = static_cast<size_t>(batch) * r * cc;
+  Bump b;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  void* X0 = base + b.take(n * 4);
+  void* X1 = base + b.take(n * 4);
+  void* XT0 = base + b.take(n * 4);
+  void* XT1 = base + b.take(n * 4);
+  void* Ab = base + b.take(static_cast<size_t>(batch) * r * r * 4);
+  void* Bb = base + b.take(static_cast<size_t>(batch) * r * r * 4);
+  float* inv = reinterpret_cast<float*>(base + b.take(batch * 4));
+  void* normws = base + b.take(muon_norm_workspace(batch));
+  bf16* Xb = reinterpret_cast<bf16*>(base + b.take(n * 2));
+  int* err = reinterpret_cast<int*>(base + b.take(16));
+  GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
+  GPT_CK(cudaMemsetAsync(err, 0, 16, s));
+  launch_muon_momentum(X, G, static_cast<long long>(rows) * cols, batch, 0.f, 1e-7f, inv, normws, s);
+  const int es0 = tf32_steps > 0 ? 4 : 2;
+  launch_muon_make_x(X, inv, X0, es0, batch, r, cc, tr, s);
+  if (tf32_steps > 0) launch_muon_make_x(X, inv, XT0, es0, batch, cc, r, !tr, s);
+  GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
+  void* res = nullptr;
+  int res_es = es0;
+  int64_t launches = 0;
+  int rc = newton_schulz(nullptr, batch, r, cc, X0, X1, XT0, XT1, Ab, Bb, tf32_steps, s, err, &res, &res_es,
+                         &launches);
+  if (rc) return rc;
+  // X = 0 * (1 - 0) + 1 * NS(G): the apply kernel with lr = -1 writes the (un-transposed) result
+  launch_muon_apply(X, Xb, res, res_es, batch, r, cc, tr, -1.f, 0.f, 1.f, s);
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// Host side of the tcgen05 GEMM: TMA tensor maps, tile/split bookkeeping and
+// the table of compiled variants.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+#include "gemm.h"
+
+namespace gpt {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 3-D map over [batch][outer][inner] with 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
+              long long ld, long long bs, int box_inner, int box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  if (bs == 0 || batch == 1) bs = ld * outer;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer),
+                        static_cast<cuuint64_t>(batch)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld * es), static_cast<cuuint64_t>(bs * es)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (strides[0] & 15) || (strides[1] & 15)) return false;
+  CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, cudaStream_t s) {
+  using C = GemmCfg<sizeof(T), BN>;
+  auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
+  kern<<<grid, 192, C::SMEM, s>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+using bf16 = __nv_bfloat16;
+
+}  // namespace
+
+int device_sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+int gemm_tiles(const GemmCall& c) {
+  const int tm = (c.M + 127) / 128;
+  const int tn = (c.N + c.bn - 1) / c.bn;
+  return (c.sym ? tm * (tm + 1) / 2 : tm * tn) * c.batch;
+}
+
+cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
+  if (c.M <= 0 || c.N <= 0 || c.batch <= 0) return cudaSuccess;
+  if (c.K <= 0 || (c.bn != 128 && c.bn != 256) || (c.es != 2 && c.es != 4)) return cudaErrorInvalidValue;
+  if (c.sym && (c.M != c.N || c.bn != 128)) return cudaErrorInvalidValue;
+  if (c.N % 8) return cudaErrorInvalidValue;
+  // 32-bit operands are staged K-major only (the 128-byte swizzle atom used here
+  // describes MN-major layouts of 16-bit types)
+  if (c.es == 4 && (c.a_mn || c.b_mn)) return cudaErrorInvalidValue;
+  const int bk = 128 / c.es;
+  GemmParams& p = c.p;
+  p.M = c.M; p.N = c.N; p.K = c.K; p.batch = c.batch;
+  p.tiles_m = (c.M + 127) / 128;
+  p.tiles_n = (c.N + c.bn - 1) / c.bn;
+  p.kblocks = (c.K + bk - 1) / bk;
+  int splits = c.splits < 1 ? 1 : c.splits;
+  if (splits > p.kblocks) splits = p.kblocks;
+  p.kb_per_split = (p.kblocks + splits - 1) / splits;
+  p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
+  p.sym = c.sym ? 1 : 0;
+  const long long ntiles = c.sym ? 1ll * p.tiles_m * (p.tiles_m + 1) / 2 : 1ll * p.tiles_m * p.tiles_n;
+  const long long units = ntiles * p.splits * c.batch;
+  if (units > 0x7fffffffll) return cudaErrorInvalidValue;
+  p.units = static_cast<int>(units);
+
+  CUtensorMap ma, mb;
+  const int mn_box = bk;   // 128 bytes of the MN dimension
+  bool ok;
+  if (!c.a_mn)
+    ok = make_map(&ma, c.A, c.es, c.K, c.M, c.batch, c.lda, c.a_bs, bk, 128);
+  else
+    ok = make_map(&ma, c.A, c.es, c.M, c.K, c.batch, c.lda, c.a_bs, mn_box, bk);
+  if (!ok) return cudaErrorInvalidValue;
+  if (!c.b_mn)
+    ok = make_map(&mb, c.B, c.es, c.K, c.N, c.batch, c.ldb, c.b_bs, bk, c.bn);
+  else
+    ok = make_map(&mb, c.B, c.es, c.N, c.K, c.batch, c.ldb, c.b_bs, mn_box, bk);
+  if (!ok) return cudaErrorInvalidValue;
+
+#define GPT_GEMM_CASE(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                       \
+  if (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ && \
+      c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_))                               \
+    return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, p, stream);
+
+  // forward
+  GPT_GEMM_CASE(bf16, 128, false, true, EPI_QKV, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_ACC, float, float)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_RELU2, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_LOGITS, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_STORE, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_STORE, float, float)
+  GPT_GEMM_CASE(bf16, 128, false, true, EPI_STORE, float, float)
+  // backward: activation gradients (B is a weight read K-major)
+  GPT_GEMM_CASE(bf16, 256, false, false, EPI_DRELU2, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, false, EPI_STORE, float, float)
+  GPT_GEMM_CASE(bf16, 256, false, false, EPI_STORE, bf16, bf16)
+  // backward: weight gradients (both operands token-major)
+  GPT_GEMM_CASE(bf16, 256, true, true, EPI_STORE, float, float)
+  GPT_GEMM_CASE(bf16, 256, true, true, EPI_ACC, float, float)
+  GPT_GEMM_CASE(bf16, 256, true, false, EPI_STORE, float, float)
+  // Newton-Schulz, bf16 steps
+  GPT_GEMM_CASE(bf16, 128, false, false, EPI_STORE, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 128, false, false, EPI_AXPBY, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_AXPBY, bf16, bf16)
+  // Newton-Schulz, tf32 steps
+  GPT_GEMM_CASE(float, 128, false, false, EPI_STORE, float, float)
+  GPT_GEMM_CASE(float, 128, false, false, EPI_AXPBY, float, float)
+  GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, float, float)
+  GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, bf16, float)
+#undef GPT_GEMM_CASE
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace gpt

@@ -1,0 +1,407 @@
+// tcgen05 GEMM for sm_100a: D[z][m][n] = sum_k A[z](m, k) * B[z](n, k), fp32
+// accumulators in TMEM, operands staged by TMA into a 128-byte-swizzled
+// shared-memory ring, and a fused epilogue.
+//
+// Roles (192 threads, one CTA per SM, persistent over work units):
+//   warp 0      TMA producer (one elected lane)
+//   warp 1      TMEM allocator and MMA issuer (one elected lane)
+//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane)
+// Two accumulator buffers in TMEM let the epilogue of tile i overlap the
+// MMAs of tile i+1.  Every mbarrier wait is bounded; on expiry the CTA
+// raises an abort flag, drains its in-flight copies and MMAs, frees TMEM
+// and returns with ERRF_TIMEOUT set in the error word.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_params.h"
+
+namespace gpt {
+
+template <int ES, int BN>
+struct GemmCfg {
+  static constexpr int BK = 128 / ES;                 // elements of K per stage (one 128 B row)
+  static constexpr int MMA_K = 32 / ES;               // K per tcgen05.mma
+  static constexpr int A_BYTES = 128 * 128;
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int CHUNK_BYTES = BK * 128;        // one MN-major box: BK rows of 128 B
+  static constexpr int TMEM_COLS = 2 * BN;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+};
+
+__device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
+                                            int& kb0, int& kb1, int& split) {
+  const int ntiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  const int per_z = ntiles * p.splits;
+  z = u / per_z;
+  int r = u - z * per_z;
+  split = r / ntiles;
+  int t = r - split * ntiles;
+  if (p.sym) {
+    int m = 0;
+    while (t >= p.tiles_m - m) {
+      t -= p.tiles_m - m;
+      ++m;
+    }
+    mb = m;
+    nb = m + t;
+  } else {
+    constexpr int G = 16;
+    const int gsz = G * p.tiles_n;
+    const int g = t / gsz;
+    const int first = g * G;
+    const int gm = min(G, p.tiles_m - first);
+    const int tt = t - g * gsz;
+    mb = first + tt % gm;
+    nb = tt / gm;
+  }
+  kb0 = split * p.kb_per_split;
+  kb1 = min(p.kblocks, kb0 + p.kb_per_split);
+}
+
+// ------------------------------------------------------------ epilogue stores
+
+template <typename OutT>
+__device__ __forceinline__ void store_row32(OutT* dst, const float (&v)[32], int nvalid) {
+  if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (8 * g < nvalid) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+        w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+        w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+        w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + 8 * g) = w;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (4 * g < nvalid)
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(dst) + 4 * g) =
+            make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+    }
+  }
+}
+
+template <typename AuxT>
+__device__ __forceinline__ void load_row32(const AuxT* src, float (&v)[32], int nvalid) {
+  if constexpr (sizeof(AuxT) == 2) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (8 * g < nvalid)
+        w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + 8 * g);
+      v[8 * g + 0] = bf16_lo(w.x); v[8 * g + 1] = bf16_hi(w.x);
+      v[8 * g + 2] = bf16_lo(w.y); v[8 * g + 3] = bf16_hi(w.y);
+      v[8 * g + 4] = bf16_lo(w.z); v[8 * g + 5] = bf16_hi(w.z);
+      v[8 * g + 6] = bf16_lo(w.w); v[8 * g + 7] = bf16_hi(w.w);
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (4 * g < nvalid) w = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + 4 * g);
+      v[4 * g] = w.x; v[4 * g + 1] = w.y; v[4 * g + 2] = w.z; v[4 * g + 3] = w.w;
+    }
+  }
+}
+
+template <typename OutT>
+__device__ __forceinline__ void store_scalar(OutT* dst, float x) {
+  if constexpr (sizeof(OutT) == 2)
+    *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(x);
+  else
+    *reinterpret_cast<float*>(dst) = x;
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ GemmParams p) {
+  constexpr int ES = sizeof(T);
+  using C = GemmCfg<ES, BN>;
+  constexpr uint32_t IDESC = make_idesc(ES == 2 ? 1 : 2, BN, A_MN, B_MN);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int stage = 0;
+      uint32_t phase = 0;
+      long long issued = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int z, mb, nb, kb0, kb1, split;
+        decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          const int k0 = kb * C::BK;
+          if constexpr (!A_MN) {
+            tma_load_3d(sA, &tmA, &full[stage], k0, mb * 128, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 128 / C::BK; ++j)
+              tma_load_3d(sA + j * C::CHUNK_BYTES, &tmA, &full[stage], mb * 128 + j * C::BK, k0, z);
+          }
+          if constexpr (!B_MN) {
+            tma_load_3d(sB, &tmB, &full[stage], k0, nb * BN, z);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / C::BK; ++j)
+              tma_load_3d(sB + j * C::CHUNK_BYTES, &tmB, &full[stage], nb * BN + j * C::BK, k0, z);
+          }
+          ++issued;
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // let every copy this thread started land before the CTA exits
+        for (int s = 0; s < C::STAGES; ++s) {
+          const bool used = s < stage || issued >= C::STAGES;
+          const uint32_t par = s < stage ? phase : (phase ^ 1u);
+          if (used) {
+            for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&full[s], par); ++i) {}
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ----------------------------------------------------------------- MMA
+      int stage = 0;
+      uint32_t phase = 0;
+      int local = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++local) {
+        int z, mb, nb, kb0, kb1, split;
+        decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+        const int acc = local & 1;
+        const uint32_t acc_par = (local >> 1) & 1;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(a0 + kk * C::MMA_K * 128, C::CHUNK_BYTES, 1024)
+                                     : smem_desc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(b0 + kk * C::MMA_K * 128, C::CHUNK_BYTES, 1024)
+                                     : smem_desc_sw128(b0 + kk * 32, 16, 1024);
+            const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
+            if constexpr (ES == 2)
+              umma_f16(d_tmem, ad, bd, IDESC, accum);
+            else
+              umma_tf32(d_tmem, ad, bd, IDESC, accum);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+      }
+      // all MMAs of this thread complete before TMEM is released
+      umma_commit(drain);
+      for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
+    }
+  } else {
+    // ------------------------------------------------------------- epilogue
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int r = quarter * 32 + lane;            // accumulator row within the tile
+    int local = 0;
+    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
+      int z, mb, nb, kb0, kb1, split;
+      decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+      const int acc = local & 1;
+      const uint32_t acc_par = (local >> 1) & 1;
+      const bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
+      __syncwarp();   // tcgen05.ld is warp-collective: reconverge after the spin
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
+      const int row = mb * 128 + r;
+      const bool row_ok = row < p.M;
+
+      if constexpr (EPI == EPI_QKV) {
+        // BN = 128: the tile is one head of q, k or v for 128 tokens
+        const int which = nb / p.H;
+        const int head = nb - which * p.H;
+        const int b = row / p.T;
+        const int t = row - b * p.T;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.qkv_out[which]) +
+                             ((static_cast<long long>(b) * p.H + head) * p.T + t) * 128;
+        float v[32];
+        if (which == 2) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            tmem_load32(tbase + c * 32, v);
+            if (row_ok) store_row32(dst + c * 32, v, 32);
+          }
+        } else {
+          float ss = 0.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            tmem_load32(tbase + c * 32, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+          }
+          // a rotation keeps the sum of squares, so the norm is taken before RoPE
+          const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
+          if (row_ok) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
+          float w[32];
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            tmem_load32(tbase + c * 32, v);        // pair index i = 32c + j   (low half)
+            tmem_load32(tbase + 64 + c * 32, w);   // pair index i + 64       (high half)
+            const float2* cs = p.rope + static_cast<long long>(t) * 64 + c * 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float2 e = row_ok ? cs[j] : make_float2(1.f, 0.f);
+              const float lo = v[j], hi = w[j];
+              v[j] = (lo * e.x - hi * e.y) * rstd;
+              w[j] = (lo * e.y + hi * e.x) * rstd;
+            }
+            if (row_ok) {
+              store_row32(dst + c * 32, v, 32);
+              store_row32(dst + 64 + c * 32, w, 32);
+            }
+          }
+        }
+      } else if constexpr (EPI == EPI_LOGITS) {
+        float mx = -INFINITY, sm = 0.f, zt = 0.f;
+        bool have_t = false;
+        const int tg = row_ok ? p.tgt[row] : -1;
+        OutT* orow = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(row) * p.ldo;
+        float v[32];
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_load32(tbase + c * 32, v);
+          const int col0 = nb * BN + c * 32;
+          const int nvalid = min(32, p.N - col0);
+          if (nvalid > 0) {
+            float cm = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) if (j < nvalid) cm = fmaxf(cm, v[j]);
+            if (cm > mx) { sm *= __expf(mx - cm); mx = cm; }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) if (j < nvalid) sm += __expf(v[j] - mx);
+            if (tg >= col0 && tg < col0 + 32) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) if (j == tg - col0) zt = v[j];
+              have_t = true;
+            }
+            if (row_ok) store_row32(orow + col0, v, nvalid);
+          }
+        }
+        if (row_ok) {
+          reinterpret_cast<float2*>(p.f32a)[static_cast<long long>(row) * p.tiles_n + nb] = make_float2(mx, sm);
+          if (have_t) p.f32b[row] = zt;
+        }
+      } else {
+        OutT* obase = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(z) * p.out_bs +
+                      static_cast<long long>(split) * p.split_stride;
+        const bool mirror = p.sym && nb != mb;
+        float v[32];
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          tmem_load32(tbase + c * 32, v);
+          const int col0 = nb * BN + c * 32;
+          const int nvalid = min(32, p.N - col0);
+          if (!row_ok || nvalid <= 0) continue;
+          OutT* dst = obase + static_cast<long long>(row) * p.ldo + col0;
+          if constexpr (EPI == EPI_ACC) {
+            float o[32];
+            load_row32(dst, o, nvalid);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] += o[j];
+          } else if constexpr (EPI == EPI_RELU2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) { const float a = fmaxf(v[j], 0.f); v[j] = a * a; }
+          } else if constexpr (EPI == EPI_DRELU2) {
+            float h[32];
+            load_row32(reinterpret_cast<const AuxT*>(p.aux) + static_cast<long long>(row) * p.ld_aux + col0, h, nvalid);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= 2.f * sqrtf(h[j]);
+          } else if constexpr (EPI == EPI_AXPBY) {
+            float a[32];
+            load_row32(reinterpret_cast<const AuxT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
+                           static_cast<long long>(row) * p.ld_aux + col0, a, nvalid);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = p.alpha * a[j] + p.beta * v[j];
+          }
+          store_row32(dst, v, nvalid);
+          if (p.out_t) {
+            OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[j]);
+          }
+          if (mirror) {
+            // the transposed tile of a symmetric product: lanes write consecutive columns
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[j]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace gpt

@@ -1,0 +1,41 @@
+// Host interface of the tcgen05 GEMM (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "gemm_params.h"
+
+namespace gpt {
+
+// D[z](m, n) = sum_k A[z](m, k) B[z](n, k), z < batch.
+//   A storage: a_mn ? [K][lda] (m contiguous) : [M][lda] (k contiguous); z stride a_bs
+//   B storage: b_mn ? [K][ldb] (n contiguous) : [N][ldb] (k contiguous); z stride b_bs
+//   es: operand element size, 2 = bf16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32)
+//   out_es / aux_es: element sizes of the epilogue output and auxiliary input
+//   bn: 128 or 256 output columns per tile; splits: K split count (> 1 writes
+//   partials at out + s * split_stride); sym: only tiles on or above the
+//   diagonal are computed and mirrored (M == N, bn == 128).
+struct GemmCall {
+  int M = 0, N = 0, K = 0, batch = 1;
+  int es = 2;
+  bool a_mn = false, b_mn = false;
+  const void* A = nullptr;
+  long long lda = 0, a_bs = 0;
+  const void* B = nullptr;
+  long long ldb = 0, b_bs = 0;
+  int bn = 256, splits = 1;
+  bool sym = false;
+  int epi = 0, out_es = 4, aux_es = 4;
+  GemmParams p{};   // epilogue fields (out, ldo, aux, ...) filled by the caller
+};
+
+// Returns cudaSuccess or the launch error; cudaErrorInvalidValue for a
+// shape/alignment/variant the kernels do not cover.
+cudaError_t gemm_run(GemmCall& c, cudaStream_t stream);
+
+// Number of work units a call would launch without a K split.
+int gemm_tiles(const GemmCall& c);
+
+int device_sm_count();
+
+}  // namespace gpt

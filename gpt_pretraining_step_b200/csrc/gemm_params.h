@@ -1,0 +1,37 @@
+// Epilogue kinds and kernel parameters of the tcgen05 GEMM (host and device).
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace gpt {
+
+enum EpiKind : int {
+  EPI_STORE = 0,    // out = acc                       (OutT)
+  EPI_ACC = 1,      // out += acc                      (fp32)
+  EPI_RELU2 = 2,    // out = relu(acc)^2               (bf16)
+  EPI_DRELU2 = 3,   // out = acc * 2 sqrt(aux)         (bf16, aux = relu(u)^2 in bf16)
+  EPI_AXPBY = 4,    // out = alpha * aux + beta * acc  (OutT, aux AuxT)
+  EPI_QKV = 5,      // RoPE + per-head RMSNorm, scatter to q/k/v [B, H, T, 128]
+  EPI_LOGITS = 6,   // out = acc (bf16) + per-(row, tile) softmax partials
+};
+
+struct GemmParams {
+  int M, N, K, batch;
+  int tiles_m, tiles_n, kblocks, splits, kb_per_split, sym, units;
+  void* out;
+  long long ldo, out_bs, split_stride;
+  const void* aux;
+  long long ld_aux, aux_bs;
+  float alpha, beta;
+  float* f32a;          // QKV: rstd of q [M, H];   LOGITS: (max, sumexp) pairs [M, tiles_n]
+  float* f32b;          // QKV: rstd of k [M, H];   LOGITS: target logit [M]
+  const int* tgt;       // LOGITS: targets of the rows
+  const float2* rope;   // QKV: (cos, sin) [T, 64]
+  void* qkv_out[3];     // QKV: q, k, v [B, H, T, 128] bf16
+  void* out_t;          // STORE/AXPBY: optional transposed copy of out, [N][M] with row stride ldo_t
+  long long ldo_t;
+  int T, H;
+  int* err;
+};
+
+}  // namespace gpt

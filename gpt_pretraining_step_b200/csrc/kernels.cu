@@ -1,0 +1,575 @@
+// Bandwidth-bound kernels of the step: embedding, RMSNorm, QK-norm/RoPE
+// backward, cross-entropy finish, deterministic reductions, AdamW and the
+// elementwise parts of Muon.  Rows are processed one warp per row with
+// 16-byte vector accesses; grids are sized from the row count.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace gpt {
+
+namespace {
+
+constexpr int kMaxVec = 16;   // float4 per lane per row: d <= 2048
+
+inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+__device__ __forceinline__ void store_bf16x4(bf16* dst, float4 v) {
+  uint2 w;
+  w.x = pack_bf16x2(v.x, v.y);
+  w.y = pack_bf16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(dst) = w;
+}
+
+__device__ __forceinline__ float4 load_bf16x4(const bf16* src) {
+  const uint2 w = *reinterpret_cast<const uint2*>(src);
+  return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+}
+
+// ------------------------------------------------------------------ RoPE
+
+__global__ void rope_table_kernel(float2* tab, int T) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= T * 64) return;
+  const int t = idx / 64, i = idx % 64;
+  const double inv_freq = pow(10000.0, -2.0 * i / 128.0);
+  double sn, cs;
+  sincos(static_cast<double>(t) * inv_freq, &sn, &cs);
+  tab[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+}
+
+// ------------------------------------------------------------- embedding
+
+__global__ void embed_fwd_kernel(const int* __restrict__ tok, const bf16* __restrict__ wte,
+                                 float* __restrict__ x, int M, int d, int V, int* err) {
+  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+  if (row >= M) return;
+  int t = tok[row];
+  const bool bad = t < 0 || t >= V;
+  if (bad) {
+    if (lane_id() == 0) atomicOr(err, ERRF_TOKEN_RANGE);
+  }
+  const bf16* src = wte + static_cast<long long>(bad ? 0 : t) * d;
+  float* dst = x + static_cast<long long>(row) * d;
+  for (int c = lane_id() * 4; c < d; c += 128) {
+    float4 v = bad ? make_float4(0.f, 0.f, 0.f, 0.f) : load_bf16x4(src + c);
+    *reinterpret_cast<float4*>(dst + c) = v;
+  }
+}
+
+// Single-CTA bitonic sort of (token, position) keys of one chunk of <= 32768 positions.
+constexpr int kEmbChunk = 32768;
+
+__global__ void __launch_bounds__(1024) embed_sort_kernel(const int* __restrict__ tok, int n, int npow2,
+                                                          uint32_t* __restrict__ keys_out, int V) {
+  extern __shared__ uint32_t keys[];
+  for (int i = threadIdx.x; i < npow2; i += blockDim.x) {
+    uint32_t k = 0xFFFFFFFFu;
+    if (i < n) {
+      int t = tok[i];
+      t = (t < 0 || t >= V) ? 0 : t;
+      k = static_cast<uint32_t>(t) * kEmbChunk + static_cast<uint32_t>(i);
+    }
+    keys[i] = k;
+  }
+  __syncthreads();
+  for (int size = 2; size <= npow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = threadIdx.x; i < npow2 / 2; i += blockDim.x) {
+        const int lo = 2 * i - (i & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const uint32_t a = keys[lo], b = keys[hi];
+        if ((a > b) == up) {
+          keys[lo] = b;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < n; i += blockDim.x) keys_out[i] = keys[i];
+}
+
+// One warp per run of equal tokens in the sorted keys: sums dx rows in position order.
+__global__ void embed_segsum_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ dx,
+                                    int base, float* __restrict__ dwte, int d) {
+  const int w = blockIdx.x * (blockDim.x / 32) + warp_id();
+  if (w >= n) return;
+  const uint32_t tokw = keys[w] / kEmbChunk;
+  if (w > 0 && keys[w - 1] / kEmbChunk == tokw) return;
+  int end = w + 1;
+  while (end < n && keys[end] / kEmbChunk == tokw) ++end;
+  float* dst = dwte + static_cast<long long>(tokw) * d;
+  for (int c = lane_id() * 4; c < d; c += 128) {
+    float4 acc = *reinterpret_cast<const float4*>(dst + c);
+    for (int j = w; j < end; ++j) {
+      const int m = base + static_cast<int>(keys[j] % kEmbChunk);
+      const float4 v = *reinterpret_cast<const float4*>(dx + static_cast<long long>(m) * d + c);
+      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    *reinterpret_cast<float4*>(dst + c) = acc;
+  }
+}
+
+// --------------------------------------------------------------- RMSNorm
+
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, bf16* __restrict__ y, float* __restrict__ rstd,
+                                   int M, int d) {
+  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+  if (row >= M) return;
+  const float* xr = x + static_cast<long long>(row) * d;
+  float4 buf[kMaxVec];
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = (i * 32 + lane_id()) * 4;
+    if (c < d) {
+      buf[i] = *reinterpret_cast<const float4*>(xr + c);
+      ss += buf[i].x * buf[i].x + buf[i].y * buf[i].y + buf[i].z * buf[i].z + buf[i].w * buf[i].w;
+    }
+  }
+  ss = warp_sum(ss);
+  const float r = rsqrtf(ss / d + 1e-6f);
+  bf16* yr = y + static_cast<long long>(row) * d;
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = (i * 32 + lane_id()) * 4;
+    if (c < d) store_bf16x4(yr + c, make_float4(buf[i].x * r, buf[i].y * r, buf[i].z * r, buf[i].w * r));
+  }
+  if (lane_id() == 0) rstd[row] = r;
+}
+
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const bf16* __restrict__ y,
+                                   const float* __restrict__ rstd, float* __restrict__ dx,
+                                   bf16* __restrict__ dxb, int M, int d, int accumulate) {
+  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+  if (row >= M) return;
+  const long long off = static_cast<long long>(row) * d;
+  float4 g[kMaxVec], yy[kMaxVec];
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = (i * 32 + lane_id()) * 4;
+    if (c < d) {
+      g[i] = *reinterpret_cast<const float4*>(dy + off + c);
+      yy[i] = load_bf16x4(y + off + c);
+      dot += g[i].x * yy[i].x + g[i].y * yy[i].y + g[i].z * yy[i].z + g[i].w * yy[i].w;
+    }
+  }
+  dot = warp_sum(dot) / d;
+  const float r = rstd[row];
+#pragma unroll
+  for (int i = 0; i < kMaxVec; ++i) {
+    const int c = (i * 32 + lane_id()) * 4;
+    if (c < d) {
+      float4 o = make_float4(r * (g[i].x - yy[i].x * dot), r * (g[i].y - yy[i].y * dot),
+                             r * (g[i].z - yy[i].z * dot), r * (g[i].w - yy[i].w * dot));
+      if (accumulate) {
+        const float4 p = *reinterpret_cast<const float4*>(dx + off + c);
+        o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
+      }
+      *reinterpret_cast<float4*>(dx + off + c) = o;
+      store_bf16x4(dxb + off + c, o);
+    }
+  }
+}
+
+// -------------------------------------------------- QK-norm / RoPE backward
+
+__global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restrict__ dk,
+                              const bf16* __restrict__ dv, const bf16* __restrict__ qn,
+                              const bf16* __restrict__ kn, const float* __restrict__ rq,
+                              const float* __restrict__ rk, const float2* __restrict__ rope,
+                              bf16* __restrict__ dqkv, int B, int T, int H) {
+  const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + warp_id();
+  const long long total = static_cast<long long>(B) * H * T;
+  if (w >= total) return;
+  // w enumerates (b, h, t) in the head-major layout of q/k/v
+  const int t = static_cast<int>(w % T);
+  const int h = static_cast<int>((w / T) % H);
+  const int b = static_cast<int>(w / (static_cast<long long>(T) * H));
+  const long long m = static_cast<long long>(b) * T + t;
+  const int d = H * 128;
+  const long long src = w * 128;
+  const int i0 = 2 * lane_id();
+  const float2 e0 = rope[t * 64 + i0], e1 = rope[t * 64 + i0 + 1];
+  bf16* out = dqkv + m * 3 * d + h * 128;
+#pragma unroll
+  for (int which = 0; which < 2; ++which) {
+    const bf16* yv = which == 0 ? qn : kn;
+    const float r = (which == 0 ? rq : rk)[m * H + h];
+    float gl0, gl1, gh0, gh1;
+    if (which == 0) {
+      const float2 a = *reinterpret_cast<const float2*>(dq + src + i0);
+      const float2 c = *reinterpret_cast<const float2*>(dq + src + 64 + i0);
+      gl0 = a.x; gl1 = a.y; gh0 = c.x; gh1 = c.y;
+    } else {
+      const uint32_t glo = *reinterpret_cast<const uint32_t*>(dk + src + i0);
+      const uint32_t ghi = *reinterpret_cast<const uint32_t*>(dk + src + 64 + i0);
+      gl0 = bf16_lo(glo); gl1 = bf16_hi(glo); gh0 = bf16_lo(ghi); gh1 = bf16_hi(ghi);
+    }
+    const uint32_t ylo = *reinterpret_cast<const uint32_t*>(yv + src + i0);
+    const uint32_t yhi = *reinterpret_cast<const uint32_t*>(yv + src + 64 + i0);
+    float yl0 = bf16_lo(ylo), yl1 = bf16_hi(ylo), yh0 = bf16_lo(yhi), yh1 = bf16_hi(yhi);
+    float dot = gl0 * yl0 + gl1 * yl1 + gh0 * yh0 + gh1 * yh1;
+    dot = warp_sum(dot) * (1.f / 128.f);
+    // gradient w.r.t. the rotated vector, then the transposed rotation
+    const float rl0 = r * (gl0 - yl0 * dot), rl1 = r * (gl1 - yl1 * dot);
+    const float rh0 = r * (gh0 - yh0 * dot), rh1 = r * (gh1 - yh1 * dot);
+    const float ol0 = rl0 * e0.x + rh0 * e0.y, oh0 = -rl0 * e0.y + rh0 * e0.x;
+    const float ol1 = rl1 * e1.x + rh1 * e1.y, oh1 = -rl1 * e1.y + rh1 * e1.x;
+    *reinterpret_cast<uint32_t*>(out + which * d + i0) = pack_bf16x2(ol0, ol1);
+    *reinterpret_cast<uint32_t*>(out + which * d + 64 + i0) = pack_bf16x2(oh0, oh1);
+  }
+  const uint2 vv = *reinterpret_cast<const uint2*>(dv + src + 4 * lane_id());
+  *reinterpret_cast<uint2*>(out + 2 * d + 4 * lane_id()) = vv;
+}
+
+// ------------------------------------------------------- cross-entropy finish
+
+__global__ void __launch_bounds__(256) ce_finish_kernel(bf16* __restrict__ z, const float2* __restrict__ stats,
+                                                        const float* __restrict__ zt, const int* __restrict__ tgt,
+                                                        float* __restrict__ row_loss, int V, int tiles_n,
+                                                        float inv_count) {
+  __shared__ float red[8];
+  __shared__ float bc;
+  const int row = blockIdx.x;
+  const float2* st = stats + static_cast<long long>(row) * tiles_n;
+  float mx = -INFINITY;
+  for (int i = threadIdx.x; i < tiles_n; i += blockDim.x) mx = fmaxf(mx, st[i].x);
+  mx = warp_max(mx);
+  if (lane_id() == 0) red[warp_id()] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = red[0];
+    for (int i = 1; i < 8; ++i) m = fmaxf(m, red[i]);
+    bc = m;
+  }
+  __syncthreads();
+  mx = bc;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < tiles_n; i += blockDim.x) s += st[i].y * __expf(st[i].x - mx);
+  s = warp_sum(s);
+  __syncthreads();
+  if (lane_id() == 0) red[warp_id()] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < 8; ++i) t += red[i];
+    const float lse = mx + logf(t);
+    bc = lse;
+    row_loss[row] = lse - zt[row];
+  }
+  __syncthreads();
+  const float lse = bc;
+  const int tg = tgt[row];
+  bf16* zr = z + static_cast<long long>(row) * V;
+  for (int c = threadIdx.x * 8; c < V; c += blockDim.x * 8) {
+    uint4 w = *reinterpret_cast<const uint4*>(zr + c);
+    uint32_t* u = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float a = __expf(bf16_lo(u[j]) - lse), b = __expf(bf16_hi(u[j]) - lse);
+      if (c + 2 * j == tg) a -= 1.f;
+      if (c + 2 * j + 1 == tg) b -= 1.f;
+      u[j] = pack_bf16x2(a * inv_count, b * inv_count);
+    }
+    *reinterpret_cast<uint4*>(zr + c) = w;
+  }
+}
+
+__global__ void __launch_bounds__(1024) sum_scale_kernel(const float* __restrict__ v, int n, float scale,
+                                                         float* __restrict__ out) {
+  __shared__ float red[32];
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += v[i];
+  s = warp_sum(s);
+  if (lane_id() == 0) red[warp_id()] = s;
+  __syncthreads();
+  if (warp_id() == 0) {
+    float t = lane_id() < static_cast<int>(blockDim.x / 32) ? red[lane_id()] : 0.f;
+    t = warp_sum(t);
+    if (lane_id() == 0) *out = t * scale;
+  }
+}
+
+// ---------------------------------------------------------------- split-K
+
+__global__ void splitk_reduce_kernel(const float* __restrict__ part, int splits, long long stride, long long n4,
+                                     float* __restrict__ out, int accumulate) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 a = accumulate ? reinterpret_cast<const float4*>(out)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < splits; ++s) {
+      const float4 b = reinterpret_cast<const float4*>(part + s * stride)[i];
+      a.x += b.x; a.y += b.y; a.z += b.z; a.w += b.w;
+    }
+    reinterpret_cast<float4*>(out)[i] = a;
+  }
+}
+
+// ------------------------------------------------------------------ AdamW
+
+__global__ void adamw_kernel(float* __restrict__ p, const float* __restrict__ g, float* __restrict__ m,
+                             float* __restrict__ v, bf16* __restrict__ pb, long long n4, float lr, float b1,
+                             float b2, float eps, float wd, float bc1, float bc2) {
+  const float decay = 1.f - lr * wd;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 pp = reinterpret_cast<float4*>(p)[i];
+    const float4 gg = reinterpret_cast<const float4*>(g)[i];
+    float4 mm = reinterpret_cast<float4*>(m)[i];
+    float4 vv = reinterpret_cast<float4*>(v)[i];
+    float* pa = &pp.x; const float* ga = &gg.x; float* ma = &mm.x; float* va = &vv.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ma[j] = b1 * ma[j] + (1.f - b1) * ga[j];
+      va[j] = b2 * va[j] + (1.f - b2) * ga[j] * ga[j];
+      const float mh = ma[j] / bc1;
+      const float vh = va[j] / bc2;
+      pa[j] = pa[j] * decay - lr * mh / (sqrtf(vh) + eps);
+    }
+    reinterpret_cast<float4*>(p)[i] = pp;
+    reinterpret_cast<float4*>(m)[i] = mm;
+    reinterpret_cast<float4*>(v)[i] = vv;
+    store_bf16x4(pb + 4 * i, pp);
+  }
+}
+
+// ------------------------------------------------------------------- Muon
+
+constexpr int kNormBlocks = 64;
+
+__global__ void __launch_bounds__(256) muon_momentum_kernel(float* __restrict__ mom, const float* __restrict__ g,
+                                                            long long n4, float beta, float* __restrict__ part) {
+  const int z = blockIdx.y;
+  float4* mz = reinterpret_cast<float4*>(mom) + z * n4;
+  const float4* gz = reinterpret_cast<const float4*>(g) + z * n4;
+  float ss = 0.f;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n4; i += kNormBlocks * 256ll) {
+    float4 a = mz[i];
+    const float4 b = gz[i];
+    a.x = beta * a.x + b.x; a.y = beta * a.y + b.y; a.z = beta * a.z + b.z; a.w = beta * a.w + b.w;
+    mz[i] = a;
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  __shared__ float red[8];
+  ss = warp_sum(ss);
+  if (lane_id() == 0) red[warp_id()] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int i = 0; i < 8; ++i) t += red[i];
+    part[z * kNormBlocks + blockIdx.x] = t;
+  }
+}
+
+__global__ void muon_norm_kernel(const float* __restrict__ part, int nmat, float eps, float* __restrict__ inv_norm) {
+  const int z = blockIdx.x;
+  if (z >= nmat) return;
+  float s = 0.f;
+  for (int i = lane_id(); i < kNormBlocks; i += 32) s += part[z * kNormBlocks + i];
+  s = warp_sum(s);
+  if (lane_id() == 0) inv_norm[z] = 1.f / (sqrtf(s) + eps);
+}
+
+// X[z] (r x c) from mom[z]; when transposing, mom[z] is (c x r).
+template <typename OutT>
+__global__ void muon_make_x_kernel(const float* __restrict__ mom, const float* __restrict__ inv_norm,
+                                   OutT* __restrict__ X, int r, int c, int transpose) {
+  __shared__ float tile[32][33];
+  const int z = blockIdx.z;
+  const float s = inv_norm[z];
+  const long long n = static_cast<long long>(r) * c;
+  const float* mz = mom + z * n;
+  OutT* xz = X + z * n;
+  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
+  if (!transpose) {
+    const int row0 = blockIdx.y * 32, col0 = blockIdx.x * 32;
+    for (int i = ty; i < 32; i += 8) {
+      const int rr = row0 + i, cc = col0 + tx;
+      if (rr < r && cc < c) {
+        const float v = mz[static_cast<long long>(rr) * c + cc] * s;
+        if constexpr (sizeof(OutT) == 2) xz[static_cast<long long>(rr) * c + cc] = __float2bfloat16_rn(v);
+        else xz[static_cast<long long>(rr) * c + cc] = v;
+      }
+    }
+  } else {
+    // source rows are X columns: read a 32x32 block of mom (c x r), write it transposed
+    const int srow0 = blockIdx.x * 32, scol0 = blockIdx.y * 32;   // mom row (< c), mom col (< r)
+    for (int i = ty; i < 32; i += 8) {
+      const int sr = srow0 + i, sc = scol0 + tx;
+      tile[i][tx] = (sr < c && sc < r) ? mz[static_cast<long long>(sr) * r + sc] * s : 0.f;
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+      const int xr = scol0 + i, xc = srow0 + tx;
+      if (xr < r && xc < c) {
+        const float v = tile[tx][i];
+        if constexpr (sizeof(OutT) == 2) xz[static_cast<long long>(xr) * c + xc] = __float2bfloat16_rn(v);
+        else xz[static_cast<long long>(xr) * c + xc] = v;
+      }
+    }
+  }
+}
+
+template <typename XT>
+__global__ void muon_apply_kernel(float* __restrict__ W, bf16* __restrict__ Wb, const XT* __restrict__ X, int r,
+                                  int c, int transpose, float decay, float step) {
+  __shared__ float tile[32][33];
+  const int z = blockIdx.z;
+  const long long n = static_cast<long long>(r) * c;
+  float* wz = W + z * n;
+  bf16* wbz = Wb + z * n;
+  const XT* xz = X + z * n;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  auto ld = [](const XT* p) -> float {
+    if constexpr (sizeof(XT) == 2) return __bfloat162float(*p);
+    else return *p;
+  };
+  if (!transpose) {
+    const int row0 = blockIdx.y * 32, col0 = blockIdx.x * 32;
+    for (int i = ty; i < 32; i += 8) {
+      const int rr = row0 + i, cc = col0 + tx;
+      if (rr < r && cc < c) {
+        const long long o = static_cast<long long>(rr) * c + cc;
+        const float w = wz[o] * decay - step * ld(xz + o);
+        wz[o] = w;
+        wbz[o] = __float2bfloat16_rn(w);
+      }
+    }
+  } else {
+    // W is (c x r): W[i][j] takes X[j][i]
+    const int xrow0 = blockIdx.y * 32, xcol0 = blockIdx.x * 32;
+    for (int i = ty; i < 32; i += 8) {
+      const int xr = xrow0 + i, xc = xcol0 + tx;
+      tile[i][tx] = (xr < r && xc < c) ? ld(xz + static_cast<long long>(xr) * c + xc) : 0.f;
+    }
+    __syncthreads();
+    for (int i = ty; i < 32; i += 8) {
+      const int wr = xcol0 + i, wc = xrow0 + tx;   // W row < c, W col < r
+      if (wr < c && wc < r) {
+        const long long o = static_cast<long long>(wr) * r + wc;
+        const float w = wz[o] * decay - step * tile[tx][i];
+        wz[o] = w;
+        wbz[o] = __float2bfloat16_rn(w);
+      }
+    }
+  }
+}
+
+__global__ void cast_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+int stream_grid(long long work, int threads) {
+  // a few resident blocks per SM, never more than the work needs
+  long long g = (work + threads - 1) / threads;
+  const long long cap = 148ll * 8;
+  return static_cast<int>(g < cap ? (g > 0 ? g : 1) : cap);
+}
+
+}  // namespace
+
+void launch_rope_table(float2* tab, int T, cudaStream_t s) {
+  rope_table_kernel<<<cdiv(T * 64, 256), 256, 0, s>>>(tab, T);
+}
+
+void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, int V, int* err, cudaStream_t s) {
+  embed_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(tok, wte, x, M, d, V, err);
+}
+
+void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s) {
+  rmsnorm_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(x, y, rstd, M, d);
+}
+
+void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dxb, int M, int d,
+                        bool accumulate, cudaStream_t s) {
+  rmsnorm_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dy, y, rstd, dx, dxb, M, d, accumulate ? 1 : 0);
+}
+
+void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn, const float* rq,
+                   const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s) {
+  const long long rows = 1ll * B * H * T;
+  qk_bwd_kernel<<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H);
+}
+
+void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* tgt, float* row_loss, int rows,
+                      int V, int tiles_n, float inv_count, cudaStream_t s) {
+  if (rows <= 0) return;
+  ce_finish_kernel<<<rows, 256, 0, s>>>(z, stats, zt, tgt, row_loss, V, tiles_n, inv_count);
+}
+
+void launch_sum_scale(const float* v, int n, float scale, float* out, cudaStream_t s) {
+  sum_scale_kernel<<<1, 1024, 0, s>>>(v, n, scale, out);
+}
+
+size_t embed_bwd_workspace(int M) { return static_cast<size_t>(kEmbChunk) * sizeof(uint32_t) + 256; }
+
+void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws, bool accumulate,
+                      cudaStream_t s) {
+  static bool configured = false;
+  if (!configured) {
+    cudaFuncSetAttribute(embed_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmbChunk * 4);
+    configured = true;
+  }
+  if (!accumulate) cudaMemsetAsync(dwte, 0, static_cast<size_t>(V) * d * sizeof(float), s);
+  uint32_t* keys = static_cast<uint32_t*>(ws);
+  for (int base = 0; base < M; base += kEmbChunk) {
+    const int n = M - base < kEmbChunk ? M - base : kEmbChunk;
+    int npow2 = 1;
+    while (npow2 < n) npow2 <<= 1;
+    embed_sort_kernel<<<1, 1024, npow2 * 4, s>>>(tok + base, n, npow2, keys, V);
+    embed_segsum_kernel<<<cdiv(n, 8), 256, 0, s>>>(keys, n, dx, base, dwte, d);
+  }
+}
+
+void launch_splitk_reduce(const float* part, int splits, long long stride, long long n, float* out, bool accumulate,
+                          cudaStream_t s) {
+  const long long n4 = n / 4;
+  splitk_reduce_kernel<<<stream_grid(n4, 256), 256, 0, s>>>(part, splits, stride, n4, out, accumulate ? 1 : 0);
+}
+
+void launch_adamw(float* p, const float* g, float* m, float* v, bf16* pb, long long n, float lr, float b1, float b2,
+                  float eps, float wd, float bc1, float bc2, cudaStream_t s) {
+  const long long n4 = n / 4;
+  adamw_kernel<<<stream_grid(n4, 256), 256, 0, s>>>(p, g, m, v, pb, n4, lr, b1, b2, eps, wd, bc1, bc2);
+}
+
+size_t muon_norm_workspace(int nmat) { return static_cast<size_t>(nmat) * kNormBlocks * sizeof(float); }
+
+void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, float beta, float eps, float* inv_norm,
+                          void* ws, cudaStream_t s) {
+  float* part = static_cast<float*>(ws);
+  muon_momentum_kernel<<<dim3(kNormBlocks, nmat), 256, 0, s>>>(mom, g, n / 4, beta, part);
+  muon_norm_kernel<<<nmat, 32, 0, s>>>(part, nmat, eps, inv_norm);
+}
+
+void launch_muon_make_x(const float* mom, const float* inv_norm, void* X, int out_es, int nmat, int r, int c,
+                        bool transpose, cudaStream_t s) {
+  dim3 grid = transpose ? dim3(cdiv(c, 32), cdiv(r, 32), nmat) : dim3(cdiv(c, 32), cdiv(r, 32), nmat);
+  if (out_es == 2)
+    muon_make_x_kernel<bf16><<<grid, dim3(32, 8), 0, s>>>(mom, inv_norm, static_cast<bf16*>(X), r, c, transpose);
+  else
+    muon_make_x_kernel<float><<<grid, dim3(32, 8), 0, s>>>(mom, inv_norm, static_cast<float*>(X), r, c, transpose);
+}
+
+void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
+                       float lr, float wd, float scale, cudaStream_t s) {
+  dim3 grid(cdiv(c, 32), cdiv(r, 32), nmat);
+  const float decay = 1.f - lr * wd, step = lr * scale;
+  if (x_es == 2)
+    muon_apply_kernel<bf16><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const bf16*>(X), r, c, transpose, decay, step);
+  else
+    muon_apply_kernel<float><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const float*>(X), r, c, transpose, decay, step);
+}
+
+void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s) {
+  cast_bf16_kernel<<<stream_grid(n, 256), 256, 0, s>>>(src, dst, n);
+}
+
+}  // namespace gpt

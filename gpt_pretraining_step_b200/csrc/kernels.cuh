@@ -1,0 +1,70 @@
+// Launchers of the bandwidth-bound kernels (internal to the library).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gpt {
+
+using bf16 = __nv_bfloat16;
+
+// (cos, sin) of t * 10000^(-2i/128) for t < T, i < 64, evaluated in fp64.
+void launch_rope_table(float2* tab, int T, cudaStream_t s);
+
+// x[m, :] = wte[tok[m], :] (bf16 weights into the fp32 residual stream).
+void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, int V, int* err,
+                      cudaStream_t s);
+
+// y = x / sqrt(mean(x^2) + 1e-6) per row (bf16 out), rstd saved.
+void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s);
+
+// dx (+)= rstd * (dy - y * mean(dy * y)); also writes dx in bf16.
+void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dx_bf16,
+                        int M, int d, bool accumulate, cudaStream_t s);
+
+// Per-head QK-norm and RoPE backward plus the v copy, into dqkv [M, 3d]
+// (dq is the fp32 attention-backward accumulator, dk and dv bf16).
+void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn,
+                   const float* rq, const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H,
+                   cudaStream_t s);
+
+// Per row: lse from the (max, sumexp) tile partials, row loss = lse - z[target],
+// and z <- (softmax(z) - onehot(target)) * inv_count in place.
+void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* tgt, float* row_loss,
+                      int rows, int V, int tiles_n, float inv_count, cudaStream_t s);
+
+// loss = sum(row_loss) * scale, deterministic single-block reduction.
+void launch_sum_scale(const float* v, int n, float scale, float* out, cudaStream_t s);
+
+// Deterministic embedding gradient: dwte (+)= scatter of dx rows by token.
+size_t embed_bwd_workspace(int M);
+void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws,
+                      bool accumulate, cudaStream_t s);
+
+// out (+)= sum over splits of part[s*stride + i], i < n.
+void launch_splitk_reduce(const float* part, int splits, long long stride, long long n, float* out,
+                          bool accumulate, cudaStream_t s);
+
+// AdamW over n elements; writes the bf16 working copy.
+void launch_adamw(float* p, const float* g, float* m, float* v, bf16* pb, long long n, float lr, float b1,
+                  float b2, float eps, float wd, float bc1, float bc2, cudaStream_t s);
+
+// Muon: mom = beta * mom + g over a batch of nmat matrices of n elements each,
+// then inv_norm[z] = 1 / (||mom[z]||_F + eps) (deterministic two-level sum).
+size_t muon_norm_workspace(int nmat);
+void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, float beta, float eps,
+                          float* inv_norm, void* ws, cudaStream_t s);
+
+// X[z] = mom[z] * inv_norm[z], stored [r][c] (transpose: mom is [c][r]); bf16 or fp32 out.
+void launch_muon_make_x(const float* mom, const float* inv_norm, void* X, int out_es, int nmat, int r,
+                        int c, bool transpose, cudaStream_t s);
+
+// W[z] = W[z] (1 - lr wd) - lr * scale * X[z] (X is [r][c]; W is [c][r] when transpose).
+void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
+                       float lr, float wd, float scale, cudaStream_t s);
+
+// dst = bf16(src), n elements.
+void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s);
+
+}  // namespace gpt

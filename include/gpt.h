@@ -1,0 +1,244 @@
+/*
+ * gpt.h — C ABI of the B200 GPT pretraining-step library (libgpt.so).
+ *
+ * One training step of the depth-parameterised GPT decoder described in
+ * "¿Cómo Entrenar Tu Propio ChatGPT por $50?" (dev.to): the forward and
+ * backward pass of the decoder stack (section "1. Modelo GPT": rotary
+ * embeddings, QK normalisation, untied token/output weights, ReLU^2 MLP,
+ * causal attention), followed by the optimizer of section "2. Optimizador
+ * Muon" (Newton-Schulz "Polar Express" orthogonalised momentum for the 2-D
+ * block matrices, AdamW for the embedding and lm_head) with fp32 master
+ * weights and bf16 compute (section "3. Gestión de Precisión"; the Portuguese
+ * page "Como Treinar Seu Próprio ChatGPT por 50 Dólares?" states the fp32
+ * masters explicitly).  Width and heads derive from the depth knob (section
+ * "La Filosofía: Un Solo Selector para Controlar Todo"); the vocabulary is
+ * 32,768 (section "Lo que nanochat cubre").
+ *
+ * Conventions for every call:
+ *   - Memory is owned by the caller.  The library allocates no device
+ *     memory: gpt_workspace_size() reports three byte counts, the caller
+ *     allocates them (256-byte aligned device memory) and passes them to
+ *     gpt_init().  The context itself is a small host object.
+ *   - Calls are asynchronous on the stream given to gpt_init() unless
+ *     stated otherwise.  Device-side failures (token ids out of range, an
+ *     expired bounded wait) are latched in a device error word and
+ *     reported by gpt_check(), which synchronises the stream.
+ *   - Status codes: GPT_OK (0) or a negative GPT_E* value; the message of
+ *     the last failure on the calling thread is gpt_last_error().  No C++
+ *     exception crosses this boundary.
+ *   - Matrices are row-major [in, out] (y = x W); the token embedding is
+ *     [vocab, d_model].  Tensors exchanged through gpt_get_tensor /
+ *     gpt_set_tensor are fp32 device buffers of rows * cols elements.
+ */
+#ifndef GPT_B200_H
+#define GPT_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  GPT_OK = 0,
+  GPT_EINVAL = -1,    /* bad configuration, pointer, alignment or id */
+  GPT_ERANGE = -2,    /* a token or target id outside [0, vocab) reached the device */
+  GPT_ETIMEOUT = -3,  /* a bounded device-side wait expired; the step's results are invalid */
+  GPT_ECUDA = -4      /* a CUDA runtime call failed */
+};
+
+/* Tensor kinds for gpt_get_tensor / gpt_set_tensor. */
+enum {
+  GPT_KIND_PARAM = 0,  /* fp32 master weight (setting it also refreshes the bf16 copy) */
+  GPT_KIND_GRAD = 1,   /* fp32 gradient of the mean loss */
+  GPT_KIND_MOM = 2,    /* Muon momentum (block matrices only) */
+  GPT_KIND_ADAM_M = 3, /* AdamW first moment (embedding, lm_head only) */
+  GPT_KIND_ADAM_V = 4  /* AdamW second moment (embedding, lm_head only) */
+};
+
+/* Optimizer group reported by gpt_tensor_info. */
+enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
+
+/*
+ * Model and batch configuration.
+ *   depth     number of decoder blocks (the single shape knob)
+ *   d_model   0 derives 64 * depth; any multiple of head_dim is accepted
+ *   vocab     vocabulary size, a multiple of 8 (32768 in the pages' runs)
+ *   batch     sequences per step; seq_len tokens each
+ *   head_dim  must be 128; mlp_mult must be 4
+ *   precision 0 = bf16 GEMMs (the only value accepted by this version)
+ *   ns_tf32_steps  how many of the five Newton-Schulz steps run with fp32
+ *             operands on the tensor cores (kind::tf32) before switching
+ *             to bf16; 0..5
+ *   seed      seed of the N(0, 0.02) initial weights drawn by gpt_init
+ */
+typedef struct gpt_config {
+  int32_t depth;
+  int32_t d_model;
+  int32_t vocab;
+  int32_t batch;
+  int32_t seq_len;
+  int32_t head_dim;
+  int32_t mlp_mult;
+  int32_t precision;
+  int32_t ns_tf32_steps;
+  int32_t lm_chunk_rows; /* rows of logits held at once by the fused lm_head/CE; 0 = 8192 */
+  uint64_t seed;
+} gpt_config;
+
+typedef struct gpt_ctx gpt_ctx;
+
+/* Byte counts of the three caller-owned device buffers for cfg:
+ *   param_bytes  fp32 masters and their bf16 working copies
+ *   state_bytes  fp32 gradients, Muon momenta, AdamW moments
+ *   act_bytes    saved activations, scratch and the small device scalars
+ * Returns GPT_EINVAL for an unsupported configuration. */
+int gpt_workspace_size(const gpt_config* cfg, size_t* param_bytes, size_t* state_bytes, size_t* act_bytes);
+
+/* Binds the buffers and the CUDA stream (a cudaStream_t; NULL = legacy
+ * default stream) to a new context.  Draws the initial weights on the
+ * device (N(0, 0.02) rounded to bf16, masters equal to their bf16 copies),
+ * zeroes gradients and optimizer state.  Synchronous. */
+int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_buf, void* stream,
+             gpt_ctx** out);
+
+/* Forward and backward pass over one batch.
+ *   tokens, targets  device int32 [batch, seq_len]; position t of a row
+ *                    predicts targets[row, t] from tokens[row, 0..t]
+ *   loss_out         device fp32 scalar, receives the mean cross-entropy
+ *   accumulate       0: gradients are overwritten; 1: added to the stored ones
+ * Ids outside [0, vocab) are treated as 0 and latched as GPT_ERANGE. */
+int gpt_fwd_bwd(gpt_ctx* ctx, const int32_t* tokens, const int32_t* targets, float* loss_out, int accumulate);
+
+/* Muon update of every 2-D block matrix (fused q|k|v, attention output, MLP
+ * up, MLP down): mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
+ * with the Polar Express coefficients; W = W (1 - lr * weight_decay)
+ * - lr * sqrt(max(1, rows / cols)) * X.  Refreshes the bf16 copies. */
+int muon_step(gpt_ctx* ctx, float lr, float momentum, float weight_decay);
+
+/* AdamW update of the token embedding and lm_head with bias correction
+ * (the step count is kept in the context) and decoupled weight decay. */
+int adamw_step(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay);
+
+/* Whole step from HOST buffers: copies tokens and targets (int32
+ * [batch, seq_len], pinned memory recommended) to the device, runs
+ * gpt_fwd_bwd, muon_step and adamw_step with the given hyper-parameters,
+ * copies the loss back to *loss_host and synchronises the stream. */
+typedef struct gpt_hparams {
+  float muon_lr, muon_momentum, muon_wd;
+  float adam_lr, adam_beta1, adam_beta2, adam_eps, adam_wd;
+} gpt_hparams;
+int gpt_train_step_host(gpt_ctx* ctx, const int32_t* tokens_host, const int32_t* targets_host,
+                        const gpt_hparams* hp, float* loss_host);
+
+/* Parameter tensors: id 0 = token embedding [vocab, d], 1 = lm_head [d, vocab],
+ * 2 + 4 l + j for block l with j = 0 fused q|k|v [d, 3d], 1 attention output
+ * [d, d], 2 MLP up [d, 4d], 3 MLP down [4d, d]. */
+int gpt_num_tensors(const gpt_ctx* ctx);
+int gpt_tensor_info(const gpt_ctx* ctx, int id, int32_t* rows, int32_t* cols, int32_t* group);
+
+/* Device-to-device copies of rows*cols fp32 values (asynchronous). */
+int gpt_get_tensor(gpt_ctx* ctx, int id, int kind, float* dst);
+int gpt_set_tensor(gpt_ctx* ctx, int id, int kind, const float* src);
+
+/* Byte range of the fp32 gradients of every parameter inside state_buf
+ * (one contiguous span; alignment padding inside it stays zero).  Data
+ * parallel training averages this span across ranks between gpt_fwd_bwd and
+ * the optimizer calls. */
+int gpt_grad_region(const gpt_ctx* ctx, size_t* offset_bytes, size_t* size_bytes);
+
+/* Per-position cross-entropy of the last gpt_fwd_bwd: batch * seq_len fp32
+ * values (row-major [batch, seq_len]) copied device-to-device into dst. */
+int gpt_get_row_loss(gpt_ctx* ctx, float* dst);
+
+/* Launch-site categories for the event profiler. */
+enum {
+  GPT_PROF_QKV_GEMM = 0,  /* q|k|v projection + RoPE + QK-norm epilogue */
+  GPT_PROF_PROJ_GEMM,     /* attention output projection + residual add */
+  GPT_PROF_FC_GEMM,       /* MLP up projection + ReLU^2 */
+  GPT_PROF_DOWN_GEMM,     /* MLP down projection + residual add */
+  GPT_PROF_ATTN_FWD,      /* causal flash attention forward */
+  GPT_PROF_ATTN_BWD,      /* causal flash attention backward (with its D pre-pass) */
+  GPT_PROF_LOGITS_GEMM,   /* lm_head logits + per-tile softmax partials */
+  GPT_PROF_CE_FINISH,     /* log-sum-exp, row loss, dlogits in place */
+  GPT_PROF_LM_DX_GEMM,    /* dlogits W_lm^T (+ split-K reduce) */
+  GPT_PROF_LM_DW_GEMM,    /* xf^T dlogits */
+  GPT_PROF_DX_GEMM,       /* block activation-gradient GEMMs */
+  GPT_PROF_DW_GEMM,       /* block weight-gradient GEMMs (+ split-K reduce) */
+  GPT_PROF_NORM,          /* RMSNorm forward and backward */
+  GPT_PROF_QK_BWD,        /* QK-norm and RoPE backward */
+  GPT_PROF_EMBED,         /* embedding forward and backward, id checks */
+  GPT_PROF_NS_GEMM,       /* Newton-Schulz GEMMs */
+  GPT_PROF_MUON_ELEM,     /* Muon momentum, norms, normalise, apply */
+  GPT_PROF_ADAMW,         /* AdamW */
+  GPT_PROF_COUNT
+};
+
+/* Record CUDA events around every launch of the categories set in mask
+ * (bit i = category i); 0 turns recording off. */
+int gpt_profile_enable(gpt_ctx* ctx, uint32_t mask);
+
+/* Synchronises the stream, then writes per category the summed device time
+ * (ms) and the number of recorded launches since the last read (arrays of
+ * GPT_PROF_COUNT entries; either may be NULL), and clears the record. */
+int gpt_profile_read(gpt_ctx* ctx, double* ms, int64_t* launches);
+
+/* Synchronises the stream and reports (then clears) latched device errors. */
+int gpt_check(gpt_ctx* ctx);
+
+/* Number of kernels the library has launched through this context. */
+int64_t gpt_launch_count(const gpt_ctx* ctx);
+
+void gpt_destroy(gpt_ctx* ctx);
+const char* gpt_last_error(void);
+
+/* --------------------------------------------------------------------
+ * Op-level entry points: single kernels of the step on caller buffers,
+ * for testing and for composing other models.  All pointers are device
+ * pointers; the stream is a cudaStream_t; asynchronous.
+ * ------------------------------------------------------------------ */
+
+/* C[z] = A[z] * B[z] with fp32 accumulation on the tensor cores.
+ *   A [M, K] row-major bf16 (z stride M*K), B [K, N] row-major bf16 (z stride K*N),
+ *   C [M, N] row-major fp32 (z stride M*N).  N and K multiples of 8.
+ *   a_trans / b_trans = 1 read A as [K, M] and B as [N, K] instead. */
+int gpt_op_matmul_bf16(const void* A, const void* B, float* C, int M, int N, int K, int batch, int a_trans,
+                       int b_trans, void* stream);
+
+/* C = A * B^T with fp32 operands read as tf32 by the tensor cores
+ * (kind::tf32), fp32 accumulation.  A [M, K] row-major fp32, B given as
+ * [N, K] row-major fp32 (b_trans must be 1: both operands are staged
+ * K-major), C [M, N] fp32.  K a multiple of 4, N of 8.  b_trans = 0 is
+ * GPT_EINVAL. */
+int gpt_op_matmul_tf32(const float* A, const float* B, float* C, int M, int N, int K, int b_trans, void* stream);
+
+/* Causal attention forward: q, k, v bf16 [B, H, T, 128] -> o bf16 [B, T, H, 128]
+ * and lse fp32 [B, H, T] (natural log of the softmax denominator of
+ * q.k / sqrt(128)). */
+int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+                         void* stream);
+
+/* Causal attention backward: given o, lse from the forward and dout bf16
+ * [B, T, H, 128], writes dq fp32, dk and dv bf16 [B, H, T, 128]; Dscratch is
+ * fp32 [B, H, T]. */
+int gpt_op_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                         const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int T,
+                         void* stream);
+
+/* Gain-free RMSNorm of fp32 rows [M, d] -> bf16 y and fp32 rstd [M]. */
+int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream);
+
+/* Newton-Schulz (Polar Express, five steps) of a batch of fp32 matrices
+ * G [batch, rows, cols] -> fp32 X of the same shape, via the same kernels
+ * as muon_step; scratch is a device buffer of gpt_op_newton_schulz_scratch()
+ * bytes. */
+size_t gpt_op_newton_schulz_scratch(int batch, int rows, int cols);
+int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols, int tf32_steps, void* scratch,
+                         void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPT_B200_H */

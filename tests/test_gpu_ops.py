@@ -1,0 +1,157 @@
+"""Op-level parity of the CUDA kernels against the fp64 oracle (B200 only).
+
+Each case uses seeded inputs with ragged sizes that span several tiles.
+Tolerances follow from the arithmetic: bf16 operands are exact in fp64,
+products accumulate in fp32 (relative error ~1e-6 per add), so GEMMs must
+agree to ~1e-5 relative; attention rounds P to bf16 before P.V (relative
+2^-9 per weight), so outputs agree to ~1e-2 relative; Newton-Schulz must
+meet the 2e-2 relative Frobenius bound of the Muon update.
+"""
+import numpy as np
+import pytest
+
+import synthetic as syn
+from oracle import model as om
+from oracle import optim as oo
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as t
+    import gpt_pretraining_step_b200 as g
+    g.lib()
+    return t
+
+
+def bf16_t(torch, a):
+    return torch.tensor(syn.round_to_bf16(np.asarray(a, dtype=np.float32))).to(torch.bfloat16).cuda()
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def relfro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def cosine(a, b):
+    a, b = a.ravel(), b.ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
+
+
+@pytest.mark.parametrize("a_trans", [0, 1])
+@pytest.mark.parametrize("b_trans", [0, 1])
+@pytest.mark.parametrize("M,N,K,batch", [(264, 392, 200, 2), (128, 256, 64, 1), (8, 8, 8, 1), (520, 1032, 1000, 1)])
+def test_matmul_bf16(torch, a_trans, b_trans, M, N, K, batch):
+    import gpt_pretraining_step_b200 as g
+    A = syn.round_to_bf16(syn.gaussian((batch, M, K), seed=M + K))
+    B = syn.round_to_bf16(syn.gaussian((batch, K, N), seed=N + K + 1))
+    At = A.transpose(0, 2, 1).copy() if a_trans else A
+    Bt = B.transpose(0, 2, 1).copy() if b_trans else B
+    C = g.matmul_bf16(bf16_t(torch, At), bf16_t(torch, Bt), M, N, K, batch=batch, a_trans=a_trans, b_trans=b_trans)
+    torch.cuda.synchronize()
+    ref = np.matmul(A.astype(np.float64), B.astype(np.float64))
+    got = f64(C)
+    assert relfro(got, ref) < 1e-5
+    assert np.abs(got - ref).max() < 1e-4 * np.sqrt(K) * 4
+
+
+def _tf32(a):
+    # keep the 10 explicit mantissa bits the tensor cores read (truncation)
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32) & np.uint32(0xFFFFE000)
+    return u.view(np.float32).astype(np.float64)
+
+
+@pytest.mark.parametrize("b_trans", [1])
+@pytest.mark.parametrize("M,N,K", [(128, 128, 32), (256, 384, 200), (136, 264, 136)])
+def test_matmul_tf32(torch, b_trans, M, N, K):
+    import gpt_pretraining_step_b200 as g
+    A = syn.gaussian((M, K), seed=M + 3 * K)
+    B = syn.gaussian((K, N), seed=N + 5 * K)
+    Bs = B.T.copy() if b_trans else B
+    C = g.matmul_tf32(torch.tensor(A).cuda(), torch.tensor(Bs).cuda(), M, N, K, b_trans=b_trans)
+    torch.cuda.synchronize()
+    got = f64(C)
+    ref = _tf32(A) @ _tf32(B)
+    err = relfro(got, ref)
+    if err > 1e-4:
+        exact = A.astype(np.float64) @ B.astype(np.float64)
+        print("tf32 mismatch", b_trans, M, N, K, err, "vs exact", relfro(got, exact),
+              "got[:2,:4]", got[:2, :4], "ref[:2,:4]", ref[:2, :4])
+    assert err < 1e-4
+
+
+def test_rmsnorm_fwd(torch):
+    import gpt_pretraining_step_b200 as g
+    x = syn.gaussian((300, 1280), seed=3, std=2.0)
+    y, r = g.rmsnorm_fwd(torch.tensor(x).cuda())
+    torch.cuda.synchronize()
+    yr, rr = om.rms_norm(x.astype(np.float64))
+    assert np.abs(f64(y) - yr).max() <= np.abs(yr).max() * 2 ** -8
+    assert np.allclose(f64(r), rr[:, 0], rtol=1e-5)
+
+
+def _attn_inputs(B, H, T, seed):
+    # q, k as the QK-norm produces them (RMS 1 per head), v unit Gaussian
+    q = syn.gaussian((B, H, T, 128), seed=seed)
+    k = syn.gaussian((B, H, T, 128), seed=seed + 1)
+    v = syn.gaussian((B, H, T, 128), seed=seed + 2)
+    q = syn.round_to_bf16(om.rms_norm(q.astype(np.float64))[0].astype(np.float32))
+    k = syn.round_to_bf16(om.rms_norm(k.astype(np.float64))[0].astype(np.float32))
+    v = syn.round_to_bf16(v)
+    return q, k, v
+
+
+@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 64), (1, 1, 384), (2, 1, 129)])
+def test_attention_fwd(torch, B, H, T):
+    import gpt_pretraining_step_b200 as g
+    q, k, v = _attn_inputs(B, H, T, seed=T)
+    o, lse = g.attention_fwd(bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v))
+    torch.cuda.synchronize()
+    ref, P = om.causal_attention(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64))
+    got = f64(o).transpose(0, 2, 1, 3)           # [B, T, H, hd] -> [B, H, T, hd]
+    assert relfro(got, ref) < 1e-2
+    assert np.abs(got - ref).max() < 3e-2
+    s = np.matmul(q.astype(np.float64), np.swapaxes(k.astype(np.float64), -1, -2)) / np.sqrt(128)
+    s = np.where(np.triu(np.ones((T, T), bool), 1), -np.inf, s)
+    lse_ref = om.logsumexp(s)
+    assert np.abs(f64(lse) - lse_ref).max() < 2e-3
+
+
+@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 256), (1, 1, 333)])
+def test_attention_bwd(torch, B, H, T):
+    import gpt_pretraining_step_b200 as g
+    q, k, v = _attn_inputs(B, H, T, seed=7 * T)
+    dout = syn.round_to_bf16(syn.gaussian((B, T, H, 128), seed=T + 99))
+    qt, kt, vt = bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v)
+    o, lse = g.attention_fwd(qt, kt, vt)
+    dq, dk, dv = g.attention_bwd(qt, kt, vt, o, lse, bf16_t(torch, dout))
+    torch.cuda.synchronize()
+    _, P = om.causal_attention(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64))
+    dq_r, dk_r, dv_r = om.causal_attention_bwd(dout.astype(np.float64).transpose(0, 2, 1, 3),
+                                               q.astype(np.float64), k.astype(np.float64),
+                                               v.astype(np.float64), P)
+    for got, ref in ((f64(dq), dq_r), (f64(dk), dk_r), (f64(dv), dv_r)):
+        if np.linalg.norm(ref) < 1e-9:
+            # T = 1: the softmax is constant, so dq = dk = 0 exactly
+            assert np.abs(got).max() < 1e-6
+            continue
+        assert cosine(got, ref) > 0.9999
+        assert relfro(got, ref) < 2e-2
+
+
+@pytest.mark.parametrize("batch,rows,cols", [(2, 256, 768), (1, 640, 128), (3, 128, 128), (1, 136, 264)])
+@pytest.mark.parametrize("tf32_steps", [0, 2, 5])
+def test_newton_schulz(torch, batch, rows, cols, tf32_steps):
+    import gpt_pretraining_step_b200 as g
+    G = syn.gaussian((batch, rows, cols), seed=rows + cols)
+    X = g.newton_schulz(torch.tensor(G).cuda(), tf32_steps=tf32_steps)
+    torch.cuda.synchronize()
+    got = f64(X)
+    for z in range(batch):
+        ref = oo.newton_schulz(G[z].astype(np.float64))
+        err = relfro(got[z], ref)
+        assert err < (2e-2 if tf32_steps < 5 else 1e-2), (z, err)
