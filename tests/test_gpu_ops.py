@@ -144,7 +144,7 @@ def test_attention_bwd(torch, B, H, T):
 
 
 @pytest.mark.parametrize("batch,rows,cols", [(2, 256, 768), (1, 640, 128), (3, 128, 128), (1, 136, 264)])
-@pytest.mark.parametrize("tf32_steps", [0, 2, 5])
+@pytest.mark.parametrize("tf32_steps", [0, 3, 5])
 def test_newton_schulz(torch, batch, rows, cols, tf32_steps):
     import gpt_pretraining_step_b200 as g
     G = syn.gaussian((batch, rows, cols), seed=rows + cols)
