@@ -25,6 +25,7 @@ ABI_FUNCTIONS = [
     "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
     "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_attention_fwd",
     "gpt_op_attention_bwd", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
+    "gpt_op_newton_schulz_noalloc",
 ]
 
 
@@ -86,6 +87,7 @@ def lib():
             "gpt_op_rmsnorm_fwd": (i32, [vp, vp, vp, i32, i32, vp]),
             "gpt_op_newton_schulz_scratch": (sz, [i32, i32, i32]),
             "gpt_op_newton_schulz": (i32, [vp, vp, i32, i32, i32, i32, vp, vp]),
+            "gpt_op_newton_schulz_noalloc": (i32, [vp, vp, i32, i32, i32, i32, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -286,4 +288,19 @@ def newton_schulz(G, tf32_steps=3, stream=None):
     scratch = torch.empty(n, dtype=torch.uint8, device=G.device)
     _check(lib().gpt_op_newton_schulz(_ptr(G), _ptr(X), batch, rows, cols, tf32_steps, _ptr(scratch),
                                       _stream(stream)))
+    return X
+
+
+def newton_schulz_noalloc(G, tf32_steps=3, X=None, stream=None):
+    """Newton-Schulz through the entry point that allocates no device memory.
+
+    The library keeps the scratch in its own fixed device array (at most
+    batch * rows * cols = 262144 elements); only the output is caller memory.
+    Calls that overlap on the GPU share that array and must not run
+    concurrently.
+    """
+    import torch
+    batch, rows, cols = G.shape
+    X = torch.empty_like(G) if X is None else X
+    _check(lib().gpt_op_newton_schulz_noalloc(_ptr(G), _ptr(X), batch, rows, cols, tf32_steps, _stream(stream)))
     return X

@@ -6,6 +6,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -1092,6 +1093,70 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
   launch_muon_apply(X, Xb, res, res_es, batch, r, cc, tr, -1.f, 0.f, 1.f, s);
   GPT_CK(cudaGetLastError());
   return GPT_OK;
+}
+
+// ----------------------------------------------- Newton-Schulz without allocation
+//
+// Some callers cannot hand this library device scratch: code whose device
+// memory is entirely owned by another allocator (a framework's caching pool
+// that has already reserved the GPU), runtimes that forbid cudaMalloc after
+// start-up, and C callers whose interface has no place for a scratch buffer.
+// This variant keeps its scratch in a fixed array in device global memory
+// that is part of the loaded library instead.
+
+namespace {
+
+constexpr long long kNsStaticMaxElems = 1ll << 18;   // batch * rows * cols
+constexpr int kNsStaticMaxBatch = 64;
+constexpr size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+// layout of gpt_op_newton_schulz's scratch at the largest accepted size
+// (its r x r products never exceed the r x c inputs)
+constexpr size_t kNsStaticBytes = 6 * align256(kNsStaticMaxElems * 4) + align256(kNsStaticMaxBatch * 4) +
+                                  align256(kNsStaticMaxBatch * 64 * 4) + align256(kNsStaticMaxElems * 2) +
+                                  align256(16);
+
+// Every GPU that loads the library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_ns_static_scratch[kNsStaticBytes];
+
+std::mutex g_ns_static_mu;
+void* g_ns_static_ptr[256] = {};
+
+// Device address of the array on the current device, looked up once per device.
+int ns_static_scratch(void** out) {
+  int dev = 0;
+  GPT_CK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 256) return fail(GPT_EINVAL, "device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_ns_static_mu);
+  if (!g_ns_static_ptr[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(GPT_ECUDA, std::string("cudaGetSymbolAddress of the static scratch: ") + cudaGetErrorString(e));
+    g_ns_static_ptr[dev] = p;
+  }
+  *out = g_ns_static_ptr[dev];
+  return GPT_OK;
+}
+
+}  // namespace
+
+int gpt_op_newton_schulz_noalloc(const float* G, float* X, int batch, int rows, int cols, int tf32_steps,
+                                 void* stream) {
+  if (batch < 1 || rows < 8 || cols < 8) return fail(GPT_EINVAL, "bad matrix shape");
+  const long long n = 1ll * batch * rows * cols;
+  if (n > kNsStaticMaxElems || batch > kNsStaticMaxBatch)
+    return fail(GPT_EINVAL, "gpt_op_newton_schulz_noalloc accepts at most 262144 elements (batch * rows * cols) "
+                            "and batch <= 64; use gpt_op_newton_schulz with caller scratch for larger inputs");
+  if (gpt_op_newton_schulz_scratch(batch, rows, cols) > kNsStaticBytes)
+    return fail(GPT_EINVAL, "input needs more scratch than the static array holds");
+  void* scratch = nullptr;
+  int rc = ns_static_scratch(&scratch);
+  if (rc) return rc;
+  // The same computation as gpt_op_newton_schulz on the static array.  It
+  // clears the error word and the output before use; every other scratch
+  // region is written before it is read, so leftovers of an earlier call
+  // cannot leak into this one.
+  return gpt_op_newton_schulz(G, X, batch, rows, cols, tf32_steps, scratch, stream);
 }
 
 }  // extern "C"

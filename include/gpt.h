@@ -239,6 +239,26 @@ size_t gpt_op_newton_schulz_scratch(int batch, int rows, int cols);
 int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols, int tf32_steps, void* scratch,
                          void* stream);
 
+/* Newton-Schulz without any device allocation (the pages have no
+ * counterpart of this call).  Same computation and arguments as
+ * gpt_op_newton_schulz, but its scratch is a fixed array in device memory
+ * that belongs to the loaded library, for callers that cannot hand device
+ * scratch to the library: code whose device memory is owned entirely by
+ * another allocator, runtimes that forbid cudaMalloc after start-up, and
+ * interfaces with no place for a scratch pointer.
+ *   Limits: batch * rows * cols <= 262144 fp32 elements and batch <= 64;
+ *   larger inputs return GPT_EINVAL.  The array (6,832,640 bytes) stays
+ *   resident on every GPU that loads the library until the process exits.
+ *   The first call on a device looks up the array's device address (once
+ *   per device, with that device current); make that first call before
+ *   any stream capture.
+ *   All calls share the one array: calls that overlap on the GPU (other
+ *   streams, other threads) race on it and must be serialised by the caller.
+ * This call performs no cudaMalloc/cudaFree and calls no allocating
+ * library routine. */
+int gpt_op_newton_schulz_noalloc(const float* G, float* X, int batch, int rows, int cols, int tf32_steps,
+                                 void* stream);
+
 #ifdef __cplusplus
 }
 #endif
