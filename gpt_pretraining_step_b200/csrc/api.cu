@@ -413,7 +413,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
-      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s);
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err);
     }
     {
       ProfScope ps(c, GPT_PROF_PROJ_GEMM);
@@ -1023,7 +1023,7 @@ int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, f
   if (!q || !k || !v || !o || !lse) return fail(GPT_EINVAL, "null pointer");
   if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
   launch_attn_fwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
-                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream));
+                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream), nullptr);
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }

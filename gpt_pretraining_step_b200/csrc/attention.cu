@@ -7,10 +7,12 @@
 // projection GEMMs); dq is accumulated in fp32 [B, H, T, 128]; lse and
 // D = rowsum(dO * O) are [B, H, T].
 //
-// This version issues warp-level mma.sync m16n8k16 tiles from a swizzled
-// shared-memory ring filled by cp.async.
+// The forward runs on tcgen05 with TMEM accumulators; the backward issues
+// warp-level mma.sync m16n8k16 tiles from a swizzled shared-memory ring
+// filled by cp.async.
 #include "attention.cuh"
 #include "common.cuh"
+#include "gemm.h"
 
 namespace gpt {
 
@@ -61,160 +63,316 @@ __device__ __forceinline__ void load_tile(uint8_t* sm, const bf16* g, long long 
   }
 }
 
-// ------------------------------------------------------------------ forward
+// ------------------------------------------------- forward on tcgen05 / TMEM
+//
+// One CTA per (128-query tile, batch*head), 192 threads:
+//   warp 0      TMA: Q once, K_j and V_j through two-slot rings
+//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
+//               S buffers and O += P_j V_j into the TMEM output accumulator;
+//               S_{j+1} is issued before P_j is ready so the tensor cores
+//               keep working while the softmax runs
+//   warps 2..5  softmax, one query row (TMEM lane) per thread: the block max
+//               from a first pass over the S row, exp2 into bf16 P written to
+//               shared memory (128-byte swizzle, the A operand of P V).
+// The reference max of a row only moves when the block max exceeds it by
+// more than 8 (log2 units), so P stays below 2^8; when it moves, the warp
+// rescales its rows of O in TMEM after the previous P V has completed.
+// TMEM: S0 @ col 0, S1 @ 128, O @ 256 (fp32, lane = query row).
 
-constexpr int FWD_BM = 128, FWD_BN = 64, FWD_THREADS = 256;
+constexpr int TF_TILE = 16384;                // one [128 rows][128 B] swizzled tile
+constexpr int TF_BUF = 2 * TF_TILE;           // 128 x 128 bf16 as two 64-column tiles
+constexpr int TF_SMEM = 7 * TF_BUF + 1024 + 512;
+constexpr float TF_RESCALE = 8.f;
 
-__global__ void __launch_bounds__(FWD_THREADS, 1)
-    attn_fwd_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-                    bf16* __restrict__ o, float* __restrict__ lse, int B, int H, int T, float scale_log2) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sQ = smem;                              // 128 x 128
-  uint8_t* sK = sQ + FWD_BM * 256;                 // 2 x 64 x 128
-  uint8_t* sV = sK + 2 * FWD_BN * 256;             // 2 x 64 x 128
-  const int qb = (gridDim.x - 1) - blockIdx.x;     // longest rows first
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
+                       int H, int T, float scale_log2, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = sm;
+  uint8_t* sK = sm + TF_BUF;         // two slots
+  uint8_t* sV = sm + 3 * TF_BUF;     // two slots
+  uint8_t* sP = sm + 5 * TF_BUF;     // two slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * TF_BUF);
+  uint64_t* q_full = bars + 0;
+  uint64_t* k_full = bars + 1;    // [2]
+  uint64_t* k_empty = bars + 3;   // [2]
+  uint64_t* v_full = bars + 5;    // [2]
+  uint64_t* v_empty = bars + 7;   // [2]
+  uint64_t* s_full = bars + 9;    // [2]
+  uint64_t* s_free = bars + 11;   // [2]
+  uint64_t* p_full = bars + 13;   // [2]
+  uint64_t* pv_done = bars + 15;  // [2]: P slot may be rewritten; O may be rescaled or read
+  uint64_t* drain = bars + 17;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int qt = (gridDim.x - 1) - blockIdx.x;    // longest rows first
   const int bh = blockIdx.y;
-  const int b = bh / H, h = bh % H;
-  const int q0 = qb * FWD_BM;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long head_off = static_cast<long long>(bh) * T * HD;
-  const bf16* qg = q + head_off;
-  const bf16* kg = k + head_off;
-  const bf16* vg = v + head_off;
+  const int q0 = qt * 128;
+  const int nkv = qt + 1;                          // causal: key blocks 0..qt
 
-  load_tile(sQ, qg, HD, q0, FWD_BM, T, tid, FWD_THREADS);
-  const int q_end = min(T, q0 + FWD_BM);
-  const int nkb = (q_end + FWD_BN - 1) / FWD_BN;
-  load_tile(sK, kg, HD, 0, FWD_BN, T, tid, FWD_THREADS);
-  load_tile(sV, vg, HD, 0, FWD_BN, T, tid, FWD_THREADS);
-  cp_async_commit();
-
-  const int g = lane >> 2, t4 = lane & 3;
-  const int row_a = q0 + warp * 16 + g;   // this thread's two query rows
-  const int row_b = row_a + 8;
-  float acc[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-  uint32_t qf[8][4];
-
-  for (int kb = 0; kb < nkb; ++kb) {
-    if (kb + 1 < nkb) {
-      const int nb = (kb + 1) & 1;
-      load_tile(sK + nb * FWD_BN * 256, kg, HD, (kb + 1) * FWD_BN, FWD_BN, T, tid, FWD_THREADS);
-      load_tile(sV + nb * FWD_BN * 256, vg, HD, (kb + 1) * FWD_BN, FWD_BN, T, tid, FWD_THREADS);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128);
+      mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1);
     }
-    __syncthreads();
-    if (kb == 0) {
-      const uint32_t qbase = smem_u32(sQ);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int r = warp * 16 + (lane & 15);
-        const int c = kk * 2 + (lane >> 4);
-        ldsm_x4(qbase + swz(r, c), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-      }
-    }
-    const uint32_t kbase = smem_u32(sK + (kb & 1) * FWD_BN * 256);
-    const uint32_t vbase = smem_u32(sV + (kb & 1) * FWD_BN * 256);
-    const int k0 = kb * FWD_BN;
-    // S = Q K^T for this warp's 16 rows x 64 keys
-    float s[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int r = j * 8 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = kk * 2 + ((lane >> 3) & 1);
-        ldsm_x4(kbase + swz(r, c), b0, b1, b2, b3);
-        mma16816(s[j], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-        mma16816(s[j + 1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
-      }
-    }
-    // mask (causal and ragged tail), online softmax in the log2 domain
-    float mx_a = m_a, mx_b = m_b;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c0 = k0 + j * 8 + 2 * t4;
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int col = c0 + e;
-        float va = s[j][e] * scale_log2, vb = s[j][2 + e] * scale_log2;
-        if (col > row_a || col >= T) va = -INFINITY;
-        if (col > row_b || col >= T) vb = -INFINITY;
-        s[j][e] = va;
-        s[j][2 + e] = vb;
-        mx_a = fmaxf(mx_a, va);
-        mx_b = fmaxf(mx_b, vb);
-      }
-    }
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float base_a = mx_a == -INFINITY ? 0.f : mx_a;
-    const float base_b = mx_b == -INFINITY ? 0.f : mx_b;
-    const float alpha_a = exp2f(m_a - base_a), alpha_b = exp2f(m_b - base_b);
-    m_a = mx_a;
-    m_b = mx_b;
-    l_a *= alpha_a;
-    l_b *= alpha_b;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      acc[j][0] *= alpha_a; acc[j][1] *= alpha_a;
-      acc[j][2] *= alpha_b; acc[j][3] *= alpha_b;
-    }
-    uint32_t pf[8][2];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float p0 = exp2f(s[j][0] - base_a), p1 = exp2f(s[j][1] - base_a);
-      const float p2 = exp2f(s[j][2] - base_b), p3 = exp2f(s[j][3] - base_b);
-      l_a += p0 + p1;
-      l_b += p2 + p3;
-      pf[j][0] = pack_bf16x2(p0, p1);
-      pf[j][1] = pack_bf16x2(p2, p3);
-    }
-    // O += P V
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t a0 = pf[2 * ks][0], a1 = pf[2 * ks][1], a2 = pf[2 * ks + 1][0], a3 = pf[2 * ks + 1][1];
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int c = j + (lane >> 4);
-        ldsm_x4_t(vbase + swz(r, c), b0, b1, b2, b3);
-        mma16816(acc[j], a0, a1, a2, a3, b0, b1);
-        mma16816(acc[j + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    __syncthreads();
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
   }
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-  const float inv_a = l_a > 0.f ? 1.f / l_a : 0.f, inv_b = l_b > 0.f ? 1.f / l_b : 0.f;
-  const long long d = static_cast<long long>(H) * HD;
-  if (row_a < T) {
-    bf16* orow = o + (static_cast<long long>(b) * T + row_a) * d + h * HD;
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      *reinterpret_cast<uint32_t*>(orow + j * 8 + 2 * t4) = pack_bf16x2(acc[j][0] * inv_a, acc[j][1] * inv_a);
-    if (t4 == 0) lse[static_cast<long long>(bh) * T + row_a] = (m_a + log2f(l_a)) * 0.69314718055994531f;
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
   }
-  if (row_b < T) {
-    bf16* orow = o + (static_cast<long long>(b) * T + row_b) * d + h * HD;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- TMA
+      bool ok = true;
+      int issued_k = 0, issued_v = 0;
+      mbar_arrive_expect_tx(q_full, TF_BUF);
+      tma_load_3d(sQ, &tq, q_full, 0, q0, bh);
+      tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, q0, bh);
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (!mbar_wait(&k_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&k_full[s], TF_BUF);
+        tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, j * 128, bh);
+        tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, j * 128, bh);
+        ++issued_k;
+        if (!mbar_wait(&v_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&v_full[s], TF_BUF);
+        tma_load_3d(sV + s * TF_BUF, &tv, &v_full[s], 0, j * 128, bh);
+        tma_load_3d(sV + s * TF_BUF + TF_TILE, &tv, &v_full[s], 64, j * 128, bh);
+        ++issued_v;
+      }
+      if (!ok) {
+        // let the copies already started land before the CTA exits
+        for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(q_full, 0); ++i) {}
+        for (int j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&k_full[j & 1], (j >> 1) & 1); ++i) {}
+        for (int j = (issued_v > 2 ? issued_v - 2 : 0); j < issued_v; ++j)
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&v_full[j & 1], (j >> 1) & 1); ++i) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- MMA
+      constexpr uint32_t IDESC_S = make_idesc(1, 128, false, false);
+      constexpr uint32_t IDESC_O = make_idesc(1, 128, false, true);
+      const uint32_t q_addr = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0, abort_flag, err);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (!mbar_wait(&k_full[s], par, abort_flag, err)) return false;
+        if (!mbar_wait(&s_free[s], par ^ 1u, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sK + s * TF_BUF);
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      *reinterpret_cast<uint32_t*>(orow + j * 8 + 2 * t4) = pack_bf16x2(acc[j][2] * inv_b, acc[j][3] * inv_b);
-    if (t4 == 0) lse[static_cast<long long>(bh) * T + row_b] = (m_b + log2f(l_b)) * 0.69314718055994531f;
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          umma_f16(tmem + s * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                   smem_desc_sw128(k_addr + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[s]);
+        umma_commit(&k_empty[s]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int s = j & 1;
+        const uint32_t par = (j >> 1) & 1;
+        if (!mbar_wait(&p_full[s], par, abort_flag, err)) return false;
+        if (!mbar_wait(&v_full[s], par, abort_flag, err)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(sV + s * TF_BUF);
+        const uint32_t p_addr = smem_u32(sP + s * TF_BUF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          umma_f16(tmem + 256, smem_desc_sw128(p_addr + aoff, 16, 1024),
+                   smem_desc_sw128(v_addr + kk * 2048, TF_TILE, 1024), IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&v_empty[s]);
+        umma_commit(&pv_done[s]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j + 1 < nkv) ok = issue_s(j + 1);
+        if (ok) ok = issue_pv(j);
+      }
+      umma_commit(drain);
+      for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
+    }
+  } else {
+    // ---------------------------------------------------------- softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int q = q0 + r;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_o = tmem + lane_base + 256;
+    float m_ref = -INFINITY, l = 0.f;   // reference max (log2 units) and row sum relative to it
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool got = mbar_wait(bar, par, abort_flag, err);
+      __syncwarp();
+      return __all_sync(0xffffffffu, got);
+    };
+    for (int j = 0; j < nkv && ok; ++j) {
+      const int s = j & 1;
+      if (!wait_all(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      // the whole S row at once; the S buffer is free again as soon as it is read
+      uint32_t sr[128];
+      {
+        const uint32_t ts = tmem + lane_base + s * 128;
+        uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        uint32_t (&r2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+        uint32_t (&r3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+        tmem_load32_async(ts, r0);
+        tmem_load32_async(ts + 32, r1);
+        tmem_load32_async(ts + 64, r2);
+        tmem_load32_async(ts + 96, r3);
+        tmem_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[s]);
+      const int kbase = j * 128;
+      if ((j == qt) || (kbase + 128 > T)) {
+        // causal diagonal / ragged tail: masked scores become -inf
+#pragma unroll
+        for (int k = 0; k < 128; ++k) {
+          const int key = kbase + k;
+          if (key > q || key >= T) sr[k] = __float_as_uint(-INFINITY);
+        }
+      }
+      // block max of the raw scores (the scale is positive), eight independent chains
+      float mx8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
+#pragma unroll
+      for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(sr[k]));
+      const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mblk = mraw * scale_log2;
+      const bool move = mblk > m_ref + TF_RESCALE;   // always true on the first block
+      const float m_new = move ? mblk : m_ref;
+      const float factor = ex2_approx(m_ref - m_new);  // 1 when the reference stays, 0 on the first block
+      // O may only be rescaled once the previous P V has accumulated into it
+      if (j >= 1 && __any_sync(0xffffffffu, move)) {
+        if (!wait_all(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t ra[32];
+          tmem_load32_async(t_o + c * 32, ra);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ra[k] = __float_as_uint(__uint_as_float(ra[k]) * factor);
+          tmem_store32(t_o + c * 32, ra);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+      }
+      // the P slot is free once the P V two blocks back has read it
+      if (j >= 2 && !wait_all(&pv_done[s], ((j >> 1) & 1) ^ 1u)) { ok = false; break; }
+      // probabilities relative to the reference, row sum, bf16 P tile (masked scores give 0)
+      const float bias = -m_new;
+      float rs8[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) rs8[t] = 0.f;
+      uint8_t* pslot = sP + s * TF_BUF;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 2) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + k]), scale_log2, bias));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + k + 1]), scale_log2, bias));
+          rs8[(k >> 1) & 7] += p0 + p1;
+          pk[k >> 1] = pack_bf16x2(p0, p1);
+        }
+        uint8_t* prow = pslot + (c >> 1) * TF_TILE + r * 128;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int unit = ((c & 1) * 4 + t) ^ (r & 7);
+          *reinterpret_cast<uint4*>(prow + unit * 16) =
+              make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(&p_full[s]);
+      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
+      l = l * factor + rs;
+      m_ref = m_new;
+    }
+    // epilogue: O / l once the last P V has landed
+    if (ok) ok = wait_all(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1);
+    if (ok) {
+      tc_fence_after();
+      const int b = bh / H, h = bh - (bh / H) * H;
+      const float inv = 1.f / l;
+      bf16* orow = o + (static_cast<long long>(b) * T + q) * (static_cast<long long>(H) * 128) + h * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ra[32];
+        tmem_load32_async(t_o + c * 32, ra);
+        tmem_wait_ld();
+        if (q < T) {
+#pragma unroll
+          for (int k = 0; k < 32; k += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(ra[k]) * inv, __uint_as_float(ra[k + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(ra[k + 2]) * inv, __uint_as_float(ra[k + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(ra[k + 4]) * inv, __uint_as_float(ra[k + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(ra[k + 6]) * inv, __uint_as_float(ra[k + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + k) = w;
+          }
+        }
+      }
+      if (q < T) lse[static_cast<long long>(bh) * T + q] = (m_ref + log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -451,16 +609,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 }  // namespace
 
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s) {
+                     cudaStream_t s, int* err) {
   static bool configured = false;
-  constexpr int smem = FWD_BM * 256 + 4 * FWD_BN * 256;
   if (!configured) {
-    cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
     configured = true;
   }
-  dim3 grid((T + FWD_BM - 1) / FWD_BM, B * H);
+  CUtensorMap mq, mk, mv;
+  const long long bh = 1ll * B * H;
+  if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128)) {
+    if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
+    return;
+  }
+  dim3 grid((T + 127) / 128, B * H);
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_kernel<<<grid, FWD_THREADS, smem, s>>>(q, k, v, o, lse, B, H, T, scale_log2);
+  attn_fwd_tc_kernel<<<grid, 192, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,

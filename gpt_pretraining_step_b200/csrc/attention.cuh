@@ -9,8 +9,9 @@ namespace gpt {
 using bf16 = __nv_bfloat16;
 
 // q, k, v [B, H, T, 128] -> o [B, T, H, 128], lse [B, H, T] (natural log).
+// err: device error word for expired waits (may be null).
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s);
+                     cudaStream_t s, int* err);
 
 // Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32, zeroed
 // here, then accumulated), dk, dv [B, H, T, 128]; Dv [B, H, T] is scratch.

@@ -17,17 +17,13 @@ enum : int {
   ERRF_SHAPE = 4,         // a launch saw a shape it cannot handle
 };
 
-// A wait gives up after this long (nanoseconds of %globaltimer).
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// A wait gives up after this many SM clock cycles (about 2 s at 2 GHz, longer
+// at lower clocks).  The SM-local cycle counter is cheap to read, unlike the
+// global nanosecond timer.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -71,17 +67,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Returns false if
-// another thread raised *abort or the wait ran past kWaitLimitNs; in the
+// another thread raised *abort or the wait ran past kWaitLimitCycles; in the
 // latter case this thread raises *abort itself and sets the error flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err) {
   if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
+  const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
+      if (clock64() - t0 > kWaitLimitCycles) {
         *abort = 1;
         if (err) atomicOr(err, ERRF_TIMEOUT);
         return false;
@@ -189,6 +185,10 @@ __host__ __device__ constexpr uint32_t make_idesc(int fmt, int n, bool a_mn, boo
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),            \
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])             \
       : "r"(taddr))
+
+// Issue a load of 32 accumulator columns; the values are valid after tmem_wait_ld().
+__device__ __forceinline__ void tmem_load32_async(uint32_t taddr, uint32_t (&r)[32]) { GPT_TMEM_LD32(taddr, r); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Load 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_load32(uint32_t taddr, float (&v)[32]) {

@@ -24,6 +24,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 3-D map over [batch][outer][inner] with 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
               long long ld, long long bs, int box_inner, int box_outer) {
@@ -42,6 +44,8 @@ bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long lon
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
 cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, cudaStream_t s) {

@@ -12,6 +12,8 @@
 // and returns with ERRF_TIMEOUT set in the error word.
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "gemm_params.h"
 
@@ -261,6 +263,23 @@ __global__ void __launch_bounds__(192, 1)
       decode_unit(p, u, z, mb, nb, kb0, kb1, split);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
+      if constexpr (EPI == EPI_ACC || EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
+        // pull this row's slice of the epilogue input into L2 while the MMAs run
+        const int prow = mb * 128 + r;
+        const int pcol = nb * BN;
+        if (prow < p.M && pcol < p.N) {
+          using PT = typename std::conditional<EPI == EPI_ACC, OutT, AuxT>::type;
+          const PT* src = EPI == EPI_ACC
+                              ? reinterpret_cast<const PT*>(reinterpret_cast<const OutT*>(p.out) +
+                                                            static_cast<long long>(z) * p.out_bs +
+                                                            static_cast<long long>(split) * p.split_stride +
+                                                            static_cast<long long>(prow) * p.ldo + pcol)
+                              : reinterpret_cast<const PT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
+                                    static_cast<long long>(prow) * p.ld_aux + pcol;
+          const uint32_t bytes = static_cast<uint32_t>(min(BN, p.N - pcol) * sizeof(PT));
+          asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+        }
+      }
       const bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
       __syncwarp();   // tcgen05.ld is warp-collective: reconverge after the spin
       if (!__all_sync(0xffffffffu, got)) break;
@@ -348,46 +367,89 @@ __global__ void __launch_bounds__(192, 1)
         OutT* obase = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(z) * p.out_bs +
                       static_cast<long long>(split) * p.split_stride;
         const bool mirror = p.sym && nb != mb;
-        float v[32];
+        // Auxiliary input of the epilogue (the fp32 output itself for EPI_ACC),
+        // prefetched one 32-column chunk ahead to hide its global-load latency.
+        constexpr bool HAS_AUX = EPI == EPI_ACC || EPI == EPI_DRELU2 || EPI == EPI_AXPBY;
+        using AT = typename std::conditional<EPI == EPI_ACC, OutT, AuxT>::type;
+        const AT* abase = nullptr;
+        if constexpr (EPI == EPI_ACC)
+          abase = reinterpret_cast<const AT*>(obase) + static_cast<long long>(row) * p.ldo;
+        else if constexpr (HAS_AUX)
+          abase = reinterpret_cast<const AT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
+                  static_cast<long long>(row) * p.ld_aux;
+        constexpr int AUX_VEC = HAS_AUX ? (32 * static_cast<int>(sizeof(AT))) / 16 : 1;   // uint4 per chunk
+        uint4 pf[AUX_VEC];
+        auto prefetch = [&](int c) {
+          if constexpr (HAS_AUX) {
+            const int col0 = nb * BN + c * 32;
+            const int nvalid = min(32, p.N - col0);
+            constexpr int EPV = 16 / static_cast<int>(sizeof(AT));   // elements per uint4
+#pragma unroll
+            for (int g = 0; g < AUX_VEC; ++g) {
+              pf[g] = make_uint4(0, 0, 0, 0);
+              if (row_ok && g * EPV < nvalid) pf[g] = reinterpret_cast<const uint4*>(abase + col0)[g];
+            }
+          }
+        };
+        prefetch(0);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_load32(tbase + c * 32, v);
-          const int col0 = nb * BN + c * 32;
-          const int nvalid = min(32, p.N - col0);
-          if (!row_ok || nvalid <= 0) continue;
-          OutT* dst = obase + static_cast<long long>(row) * p.ldo + col0;
-          if constexpr (EPI == EPI_ACC) {
-            float o[32];
-            load_row32(dst, o, nvalid);
+        for (int c = 0; c < BN / 32; c += 2) {
+          uint32_t ra[32], rb[32];
+          tmem_load32_async(tbase + c * 32, ra);
+          tmem_load32_async(tbase + (c + 1) * 32, rb);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] += o[j];
-          } else if constexpr (EPI == EPI_RELU2) {
+          for (int half = 0; half < 2; ++half) {
+            const int cc = c + half;
+            float v[32], a[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) { const float a = fmaxf(v[j], 0.f); v[j] = a * a; }
-          } else if constexpr (EPI == EPI_DRELU2) {
-            float h[32];
-            load_row32(reinterpret_cast<const AuxT*>(p.aux) + static_cast<long long>(row) * p.ld_aux + col0, h, nvalid);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(half ? rb[j] : ra[j]);
+            if constexpr (HAS_AUX) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] *= 2.f * sqrtf(h[j]);
-          } else if constexpr (EPI == EPI_AXPBY) {
-            float a[32];
-            load_row32(reinterpret_cast<const AuxT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
-                           static_cast<long long>(row) * p.ld_aux + col0, a, nvalid);
+              for (int g = 0; g < AUX_VEC; ++g) {
+                const uint32_t w[4] = {pf[g].x, pf[g].y, pf[g].z, pf[g].w};
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = p.alpha * a[j] + p.beta * v[j];
-          }
-          store_row32(dst, v, nvalid);
-          if (p.out_t) {
-            OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
+                for (int e = 0; e < 4; ++e) {
+                  if constexpr (sizeof(AT) == 2) {
+                    a[8 * g + 2 * e] = bf16_lo(w[e]);
+                    a[8 * g + 2 * e + 1] = bf16_hi(w[e]);
+                  } else {
+                    a[4 * g + e] = __uint_as_float(w[e]);
+                  }
+                }
+              }
+              if (cc + 1 < BN / 32) prefetch(cc + 1);
+            }
+            const int col0 = nb * BN + cc * 32;
+            const int nvalid = min(32, p.N - col0);
+            if (!row_ok || nvalid <= 0) continue;
+            OutT* dst = obase + static_cast<long long>(row) * p.ldo + col0;
+            if constexpr (EPI == EPI_ACC) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[j]);
-          }
-          if (mirror) {
-            // the transposed tile of a symmetric product: lanes write consecutive columns
+              for (int j = 0; j < 32; ++j) v[j] += a[j];
+            } else if constexpr (EPI == EPI_RELU2) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[j]);
+              for (int j = 0; j < 32; ++j) { const float t = fmaxf(v[j], 0.f); v[j] = t * t; }
+            } else if constexpr (EPI == EPI_DRELU2) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= 2.f * sqrtf(a[j]);
+            } else if constexpr (EPI == EPI_AXPBY) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = p.alpha * a[j] + p.beta * v[j];
+            }
+            store_row32(dst, v, nvalid);
+            if (p.out_t) {
+              OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[j]);
+            }
+            if (mirror) {
+              // the transposed tile of a symmetric product: lanes write consecutive columns
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[j]);
+            }
           }
         }
       }

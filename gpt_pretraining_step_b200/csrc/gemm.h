@@ -1,6 +1,7 @@
 // Host interface of the tcgen05 GEMM (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "gemm_params.h"
@@ -37,5 +38,12 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream);
 int gemm_tiles(const GemmCall& c);
 
 int device_sm_count();
+
+// TMA descriptor of a bf16 (es = 2) or fp32 (es = 4) tensor [batch][outer][inner]
+// with row stride ld and batch stride bs (elements), 128-byte swizzle, box
+// box_inner x box_outer.  False if the driver entry point is missing or the
+// base/strides are not 16-byte aligned.
+bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
+              long long ld, long long bs, int box_inner, int box_outer);
 
 }  // namespace gpt
