@@ -573,7 +573,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s);
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err);
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
@@ -1035,14 +1035,14 @@ int gpt_op_attention_bwd(const void* q, const void* k, const void* v, const void
   if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
   launch_attn_bwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
                   static_cast<const bf16*>(o), static_cast<const bf16*>(dout), lse, Dscratch, dq,
-                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream));
+                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream), nullptr);
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
 
 int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream) {
   if (!x || !y || !rstd) return fail(GPT_EINVAL, "null pointer");
-  if (M < 0 || d < 4 || d % 4 || d > 2048) return fail(GPT_EINVAL, "bad rmsnorm shape");
+  if (M < 0 || d < 128 || d % 128 || d > 2048) return fail(GPT_EINVAL, "bad rmsnorm shape (d: a multiple of 128 up to 2048)");
   launch_rmsnorm_fwd(x, static_cast<bf16*>(y), rstd, M, d, static_cast<cudaStream_t>(stream));
   GPT_CK(cudaGetLastError());
   return GPT_OK;

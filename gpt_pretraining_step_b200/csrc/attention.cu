@@ -7,9 +7,9 @@
 // projection GEMMs); dq is accumulated in fp32 [B, H, T, 128]; lse and
 // D = rowsum(dO * O) are [B, H, T].
 //
-// The forward runs on tcgen05 with TMEM accumulators; the backward issues
-// warp-level mma.sync m16n8k16 tiles from a swizzled shared-memory ring
-// filled by cp.async.
+// Both directions run on the 5th-generation tensor cores (tcgen05.mma with
+// TMEM accumulators), fed by TMA; softmax work runs in dedicated warps that
+// exchange tiles with the MMA issuer through mbarriers.
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemm.h"
@@ -19,49 +19,6 @@ namespace gpt {
 namespace {
 
 constexpr int HD = 128;
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
-  const uint32_t d = smem_u32(dst);
-  const int n = pred ? 16 : 0;
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Row r, 16-byte chunk c of a [rows][128] bf16 tile, chunks XOR-swizzled by r % 8.
-__device__ __forceinline__ uint32_t swz(int r, int c) { return r * 256 + ((c ^ (r & 7)) << 4); }
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Copy rows [r0, r0 + nrows) of a 128-wide bf16 tile; rows >= limit are zero-filled.
-__device__ __forceinline__ void load_tile(uint8_t* sm, const bf16* g, long long row_stride, int r0, int nrows,
-                                          int limit, int tid, int nthreads) {
-  for (int i = tid; i < nrows * 16; i += nthreads) {
-    const int r = i >> 4, c = i & 15;
-    const bool ok = r0 + r < limit;
-    const bf16* src = g + static_cast<long long>(ok ? r0 + r : 0) * row_stride + c * 8;
-    cp_async16(sm + swz(r, c), src, ok);
-  }
-}
 
 // ------------------------------------------------- forward on tcgen05 / TMEM
 //
@@ -376,6 +333,301 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+// ------------------------------------------------ backward on tcgen05 / TMEM
+//
+// One CTA per (128-key block j, batch*head), looping over the query blocks
+// i >= j that see those keys.  192 threads:
+//   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i
+//   warp 1      TMEM owner and MMA issuer, per query block:
+//                 S^T = K Q^T and dP^T = V dO^T          (TMEM cols 0 and 128)
+//                 dV += P^T dO, dK += dS^T Q              (TMEM cols 256, 384)
+//                 dQ_i = dS K into cols 0 (S^T is consumed by then)
+//   warps 2..5  one key row (TMEM lane) per thread: P^T = exp(S^T/sqrt(d) - lse),
+//               dS^T = P^T (dP^T - D) / sqrt(d) as bf16 tiles in shared memory
+//               (the dS^T tile is also the MN-major A operand of dS K); then one
+//               query row per thread to add dQ_i into the fp32 dq buffer with
+//               vector reductions; finally dK and dV of the block to global.
+
+constexpr int TB_SMEM = 7 * TF_BUF + 1024 + 1024 + 512;
+
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                       const float* __restrict__ lse, const float* __restrict__ Dv, float* __restrict__ dq,
+                       bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int T, float scale, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = sm;
+  uint8_t* sV = sm + TF_BUF;
+  uint8_t* sQ = sm + 2 * TF_BUF;     // two slots
+  uint8_t* sdO = sm + 4 * TF_BUF;
+  uint8_t* sPt = sm + 5 * TF_BUF;
+  uint8_t* sdSt = sm + 6 * TF_BUF;
+  float* lse_s = reinterpret_cast<float*>(sm + 7 * TF_BUF);     // 128: lse * log2(e) of the query block
+  float* dd_s = lse_s + 128;                                     // 128: D of the query block
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * TF_BUF + 1024);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;    // [2]
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;
+  uint64_t* sd_full = bars + 7;
+  uint64_t* p_full = bars + 8;
+  uint64_t* mm_done = bars + 9;
+  uint64_t* s_free = bars + 10;
+  uint64_t* drain = bars + 11;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = warp_id(), lane = lane_id();
+  const int j = blockIdx.x;
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh - (bh / H) * H;
+  const int k0 = j * 128;
+  const int nq = (T + 127) / 128;
+  const int n_it = nq - j;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
+    mbar_init(sd_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(mm_done, 1);
+    mbar_init(s_free, 128);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&tdo);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- TMA
+      bool ok = true;
+      int issued_q = 0, issued_do = 0;
+      mbar_arrive_expect_tx(kv_full, 2 * TF_BUF);
+      tma_load_3d(sK, &tk, kv_full, 0, k0, bh);
+      tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, k0, bh);
+      tma_load_3d(sV, &tv, kv_full, 0, k0, bh);
+      tma_load_3d(sV + TF_TILE, &tv, kv_full, 64, k0, bh);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int i = j + it;
+        const int s = it & 1;
+        const uint32_t par = (it >> 1) & 1;
+        if (!mbar_wait(&q_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[s], TF_BUF);
+        tma_load_3d(sQ + s * TF_BUF, &tq, &q_full[s], 0, i * 128, bh);
+        tma_load_3d(sQ + s * TF_BUF + TF_TILE, &tq, &q_full[s], 64, i * 128, bh);
+        ++issued_q;
+        if (!mbar_wait(do_empty, (it & 1) ^ 1u, abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(do_full, TF_BUF);
+        tma_load_4d(sdO, &tdo, do_full, 0, h, i * 128, b);
+        tma_load_4d(sdO + TF_TILE, &tdo, do_full, 64, h, i * 128, b);
+        ++issued_do;
+      }
+      if (!ok) {
+        for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(kv_full, 0); ++x) {}
+        for (int it = (issued_q > 2 ? issued_q - 2 : 0); it < issued_q; ++it)
+          for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(&q_full[it & 1], (it >> 1) & 1); ++x) {}
+        if (issued_do > 0)
+          for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(do_full, (issued_do - 1) & 1); ++x) {}
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // -------------------------------------------------------------- MMA
+      constexpr uint32_t IDESC_KK = make_idesc(1, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t IDESC_KM = make_idesc(1, 128, false, true);    // dV, dK
+      constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), do_addr = smem_u32(sdO);
+      const uint32_t pt_addr = smem_u32(sPt), dst_addr = smem_u32(sdSt);
+      bool ok = mbar_wait(kv_full, 0, abort_flag, err);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int s = it & 1;
+        const uint32_t par = (it >> 1) & 1;
+        if (!mbar_wait(&q_full[s], par, abort_flag, err) || !mbar_wait(do_full, it & 1, abort_flag, err) ||
+            !mbar_wait(s_free, (it & 1) ^ 1u, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ + s * TF_BUF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          umma_f16(tmem, smem_desc_sw128(k_addr + off, 16, 1024), smem_desc_sw128(q_addr + off, 16, 1024),
+                   IDESC_KK, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          umma_f16(tmem + 128, smem_desc_sw128(v_addr + off, 16, 1024), smem_desc_sw128(do_addr + off, 16, 1024),
+                   IDESC_KK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(sd_full);
+        if (!mbar_wait(p_full, it & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;   // K-major A: 16 queries per step
+          const uint32_t boff = kk * 2048;                              // MN-major B: 16 query rows per step
+          const uint32_t accum = (it > 0 || kk > 0) ? 1u : 0u;
+          umma_f16(tmem + 256, smem_desc_sw128(pt_addr + aoff, 16, 1024),
+                   smem_desc_sw128(do_addr + boff, TF_TILE, 1024), IDESC_KM, accum);
+          umma_f16(tmem + 384, smem_desc_sw128(dst_addr + aoff, 16, 1024),
+                   smem_desc_sw128(q_addr + boff, TF_TILE, 1024), IDESC_KM, accum);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = kk * 2048;   // 16 keys per step, both operands MN-major
+          umma_f16(tmem, smem_desc_sw128(dst_addr + off, TF_TILE, 1024), smem_desc_sw128(k_addr + off, TF_TILE, 1024),
+                   IDESC_MM, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(mm_done);
+        umma_commit(&q_empty[s]);
+        umma_commit(do_empty);
+      }
+      umma_commit(drain);
+      for (uint32_t x = 0; x < (1u << 22) && !mbar_try_wait(drain, 0); ++x) {}
+    }
+  } else {
+    // --------------------------------------------- P^T, dS^T, dQ, dK, dV
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;       // key row for P/dS, query row for dQ
+    const int t128 = threadIdx.x - 64;       // 0..127
+    const int key = k0 + r;
+    const bool key_ok = key < T;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const float scale_log2 = scale * 1.4426950408889634f;
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      const bool got = mbar_wait(bar, par, abort_flag, err);
+      __syncwarp();
+      return __all_sync(0xffffffffu, got);
+    };
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int i = j + it;
+      const int q0 = i * 128;
+      // the query block's lse (log2 units; +inf past T so P = 0) and D
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      {
+        const int qq = q0 + t128;
+        lse_s[t128] = qq < T ? lse[static_cast<long long>(bh) * T + qq] * 1.4426950408889634f : INFINITY;
+        dd_s[t128] = qq < T ? Dv[static_cast<long long>(bh) * T + qq] : 0.f;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!wait_all(sd_full, it & 1)) { ok = false; break; }
+      tc_fence_after();
+      const bool diag = i == j;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sr[32], dr[32];
+        tmem_load32_async(tmem + lane_base + c * 32, sr);
+        tmem_load32_async(tmem + lane_base + 128 + c * 32, dr);
+        tmem_wait_ld();
+        uint32_t pk[16], dk2[16];
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
+          const float4 d4 = *reinterpret_cast<const float4*>(dd_s + c * 32 + k);
+          const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float da[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float p = ex2_approx(fmaf(__uint_as_float(sr[k + e]), scale_log2, -la[e]));
+            if (!key_ok || (diag && key > q0 + c * 32 + k + e)) p = 0.f;
+            pv[e] = p;
+            dsv[e] = p * (__uint_as_float(dr[k + e]) - da[e]) * scale;
+          }
+          pk[k >> 1] = pack_bf16x2(pv[0], pv[1]);
+          pk[(k >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk2[k >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+          dk2[(k >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
+        }
+        const int rowoff = (c >> 1) * TF_TILE + r * 128;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int unit = ((c & 1) * 4 + t) ^ (r & 7);
+          *reinterpret_cast<uint4*>(sPt + rowoff + unit * 16) = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          *reinterpret_cast<uint4*>(sdSt + rowoff + unit * 16) =
+              make_uint4(dk2[4 * t], dk2[4 * t + 1], dk2[4 * t + 2], dk2[4 * t + 3]);
+        }
+      }
+      tc_fence_before();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(p_full);
+      // dQ_i: one query row per thread, added to the fp32 accumulator
+      if (!wait_all(mm_done, it & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int qrow = q0 + r;
+      float* dqrow = dq + (static_cast<long long>(bh) * T + qrow) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t qr[32];
+        tmem_load32_async(tmem + lane_base + c * 32, qr);
+        tmem_wait_ld();
+        if (qrow < T) {
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dqrow + c * 32 + 4 * g),
+                         "f"(__uint_as_float(qr[4 * g])), "f"(__uint_as_float(qr[4 * g + 1])),
+                         "f"(__uint_as_float(qr[4 * g + 2])), "f"(__uint_as_float(qr[4 * g + 3]))
+                         : "memory");
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(s_free);
+    }
+    // dK and dV of this key block (complete after the last mm_done)
+    if (ok) {
+      tc_fence_after();
+      bf16* dkrow = dk + (static_cast<long long>(bh) * T + key) * 128;
+      bf16* dvrow = dv + (static_cast<long long>(bh) * T + key) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t vr[32], kr[32];
+        tmem_load32_async(tmem + lane_base + 256 + c * 32, vr);
+        tmem_load32_async(tmem + lane_base + 384 + c * 32, kr);
+        tmem_wait_ld();
+        if (key_ok) {
+#pragma unroll
+          for (int g = 0; g < 32; g += 8) {
+            uint4 wv, wk;
+            wv.x = pack_bf16x2(__uint_as_float(vr[g]), __uint_as_float(vr[g + 1]));
+            wv.y = pack_bf16x2(__uint_as_float(vr[g + 2]), __uint_as_float(vr[g + 3]));
+            wv.z = pack_bf16x2(__uint_as_float(vr[g + 4]), __uint_as_float(vr[g + 5]));
+            wv.w = pack_bf16x2(__uint_as_float(vr[g + 6]), __uint_as_float(vr[g + 7]));
+            wk.x = pack_bf16x2(__uint_as_float(kr[g]), __uint_as_float(kr[g + 1]));
+            wk.y = pack_bf16x2(__uint_as_float(kr[g + 2]), __uint_as_float(kr[g + 3]));
+            wk.z = pack_bf16x2(__uint_as_float(kr[g + 4]), __uint_as_float(kr[g + 5]));
+            wk.w = pack_bf16x2(__uint_as_float(kr[g + 6]), __uint_as_float(kr[g + 7]));
+            *reinterpret_cast<uint4*>(dvrow + c * 32 + g) = wv;
+            *reinterpret_cast<uint4*>(dkrow + c * 32 + g) = wk;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------- backward prepass
 
 // D[b, h, t] = sum_i dO[b, t, h, i] * O[b, t, h, i]
@@ -393,217 +645,6 @@ __global__ void attn_bwd_dot_kernel(const bf16* __restrict__ o, const bf16* __re
             bf16_hi(x.y) * bf16_hi(y.y);
   s = warp_sum(s);
   if (lane_id() == 0) Dv[w] = s;
-}
-
-// --------------------------------------------------------------- backward
-
-// One CTA per (128-key block, b, h); loops over 64-query blocks at or below
-// the diagonal.  Warp w owns keys 16w..16w+15 for S^T, dP^T, dV and dK; for
-// dQ it owns query rows 16(w%4).. and head columns 64(w/4)...
-constexpr int BWD_BN = 128, BWD_BM = 64, BWD_THREADS = 256;
-
-__global__ void __launch_bounds__(BWD_THREADS, 1)
-    attn_bwd_kernel(const bf16* __restrict__ q, const bf16* __restrict__ k, const bf16* __restrict__ v,
-                    const bf16* __restrict__ dout, const float* __restrict__ lse, const float* __restrict__ Dv,
-                    float* __restrict__ dq, bf16* __restrict__ dk, bf16* __restrict__ dv, int B, int H, int T,
-                    float scale) {
-  extern __shared__ __align__(1024) uint8_t smem[];
-  uint8_t* sK = smem;                          // 128 x 128
-  uint8_t* sV = sK + BWD_BN * 256;             // 128 x 128
-  uint8_t* sQ = sV + BWD_BN * 256;             // 2 x 64 x 128
-  uint8_t* sO = sQ + 2 * BWD_BM * 256;         // 2 x 64 x 128 (dO)
-  uint8_t* sS = sO + 2 * BWD_BM * 256;         // dS^T: 128 keys x 64 queries bf16, 128 B rows
-  float* sL = reinterpret_cast<float*>(sS + BWD_BN * 128);   // 2 x 64 lse
-  float* sD = sL + 2 * BWD_BM;                               // 2 x 64 D
-
-  const int kblk = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh % H;
-  const int k0 = kblk * BWD_BN;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t4 = lane & 3;
-  const long long head_off = static_cast<long long>(bh) * T * HD;
-  const long long dstride = static_cast<long long>(H) * HD;
-  const bf16* qg = q + head_off;
-  const bf16* dog = dout + static_cast<long long>(b) * T * dstride + h * HD;
-  const float* lg = lse + static_cast<long long>(bh) * T;
-  const float* Dg = Dv + static_cast<long long>(bh) * T;
-
-  load_tile(sK, k + head_off, HD, k0, BWD_BN, T, tid, BWD_THREADS);
-  load_tile(sV, v + head_off, HD, k0, BWD_BN, T, tid, BWD_THREADS);
-  const int qb_first = k0 / BWD_BM;
-  const int nqb = (T + BWD_BM - 1) / BWD_BM;
-  auto load_q = [&](int qb, int buf) {
-    load_tile(sQ + buf * BWD_BM * 256, qg, HD, qb * BWD_BM, BWD_BM, T, tid, BWD_THREADS);
-    load_tile(sO + buf * BWD_BM * 256, dog, dstride, qb * BWD_BM, BWD_BM, T, tid, BWD_THREADS);
-    if (tid < BWD_BM) {
-      const int r = qb * BWD_BM + tid;
-      sL[buf * BWD_BM + tid] = r < T ? lg[r] : 0.f;
-      sD[buf * BWD_BM + tid] = r < T ? Dg[r] : 0.f;
-    }
-  };
-  if (qb_first < nqb) load_q(qb_first, 0);
-  cp_async_commit();
-
-  float dK[16][4], dV[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dK[j][e] = dV[j][e] = 0.f;
-
-  const uint32_t kbase = smem_u32(sK), vbase = smem_u32(sV), sbase = smem_u32(sS);
-  const int key_a = k0 + warp * 16 + g, key_b = key_a + 8;   // this thread's two key rows
-  const float scale_log2 = scale * 1.4426950408889634f;
-
-  for (int qb = qb_first; qb < nqb; ++qb) {
-    const int buf = (qb - qb_first) & 1;
-    if (qb + 1 < nqb) {
-      load_q(qb + 1, buf ^ 1);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t qbase = smem_u32(sQ + buf * BWD_BM * 256);
-    const uint32_t obase = smem_u32(sO + buf * BWD_BM * 256);
-    const float* L = sL + buf * BWD_BM;
-    const float* Dd = sD + buf * BWD_BM;
-    const int q0 = qb * BWD_BM;
-
-    // S^T = K Q^T and dP^T = V dO^T for 16 keys x 64 queries
-    float st[8][4], dpt[8][4];
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) st[j][e] = dpt[j][e] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      uint32_t a0, a1, a2, a3, c0, c1, c2, c3;
-      const int ar = warp * 16 + (lane & 15);
-      const int ac = kk * 2 + (lane >> 4);
-      ldsm_x4(kbase + swz(ar, ac), a0, a1, a2, a3);
-      ldsm_x4(vbase + swz(ar, ac), c0, c1, c2, c3);
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int r = j * 8 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = kk * 2 + ((lane >> 3) & 1);
-        ldsm_x4(qbase + swz(r, c), b0, b1, b2, b3);
-        mma16816(st[j], a0, a1, a2, a3, b0, b1);
-        mma16816(st[j + 1], a0, a1, a2, a3, b2, b3);
-        ldsm_x4(obase + swz(r, c), b0, b1, b2, b3);
-        mma16816(dpt[j], c0, c1, c2, c3, b0, b1);
-        mma16816(dpt[j + 1], c0, c1, c2, c3, b2, b3);
-      }
-    }
-    // P^T = exp(S^T * scale - lse[q]) masked; dS^T = P^T (dP^T - D[q]) * scale
-    uint32_t pf[8][2], sf[8][2];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      float pv[4], dsv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qi = j * 8 + 2 * t4 + (e & 1);
-        const int key = (e < 2) ? key_a : key_b;
-        const int qrow = q0 + qi;
-        float p = exp2f(st[j][e] * scale_log2 - L[qi] * 1.4426950408889634f);
-        if (key > qrow || qrow >= T || key >= T) p = 0.f;
-        pv[e] = p;
-        dsv[e] = p * (dpt[j][e] - Dd[qi]) * scale;
-      }
-      pf[j][0] = pack_bf16x2(pv[0], pv[1]);
-      pf[j][1] = pack_bf16x2(pv[2], pv[3]);
-      sf[j][0] = pack_bf16x2(dsv[0], dsv[1]);
-      sf[j][1] = pack_bf16x2(dsv[2], dsv[3]);
-      // dS^T rows (keys) to shared memory for the dQ product: 64 queries x 2 B = 128 B per key row
-      const int kr_a = warp * 16 + g, kr_b = kr_a + 8;
-      const int chunk = j;   // 8 queries = 16 B
-      *reinterpret_cast<uint32_t*>(sS + kr_a * 128 + (((chunk ^ (kr_a & 7)) << 4)) + t4 * 4) = sf[j][0];
-      *reinterpret_cast<uint32_t*>(sS + kr_b * 128 + (((chunk ^ (kr_b & 7)) << 4)) + t4 * 4) = sf[j][1];
-    }
-    // dV += P^T dO, dK += dS^T Q (k = 64 queries in 4 steps)
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const uint32_t pa0 = pf[2 * ks][0], pa1 = pf[2 * ks][1], pa2 = pf[2 * ks + 1][0], pa3 = pf[2 * ks + 1][1];
-      const uint32_t sa0 = sf[2 * ks][0], sa1 = sf[2 * ks][1], sa2 = sf[2 * ks + 1][0], sa3 = sf[2 * ks + 1][1];
-#pragma unroll
-      for (int j = 0; j < 16; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-        const int c = j + (lane >> 4);
-        ldsm_x4_t(obase + swz(r, c), b0, b1, b2, b3);
-        mma16816(dV[j], pa0, pa1, pa2, pa3, b0, b1);
-        mma16816(dV[j + 1], pa0, pa1, pa2, pa3, b2, b3);
-        ldsm_x4_t(qbase + swz(r, c), b0, b1, b2, b3);
-        mma16816(dK[j], sa0, sa1, sa2, sa3, b0, b1);
-        mma16816(dK[j + 1], sa0, sa1, sa2, sa3, b2, b3);
-      }
-    }
-    __syncthreads();   // dS^T complete
-    // dQ[q0 + 16(w%4) .., 64(w/4) ..] += dS K: A = dS (rows = queries) read transposed from dS^T
-    {
-      float dqa[8][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) dqa[j][0] = dqa[j][1] = dqa[j][2] = dqa[j][3] = 0.f;
-      const int qr0 = (warp & 3) * 16;
-      const int hc0 = (warp >> 2) * 64;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {   // 128 keys in steps of 16
-        // A fragment rows = queries qr0.., cols = keys 16ks..; stored as dS^T[key][query]
-        uint32_t a0, a1, a2, a3;
-        {
-          const int key = ks * 16 + (lane & 7) + ((lane >> 4) << 3);
-          const int qc = qr0 + (((lane >> 3) & 1) << 3);   // query chunk start (8 queries)
-          const int chunk = qc >> 3;
-          ldsm_x4_t(sbase + key * 128 + ((chunk ^ (key & 7)) << 4), a0, a1, a2, a3);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          uint32_t b0, b1, b2, b3;
-          const int r = ks * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
-          const int c = (hc0 >> 3) + j + (lane >> 4);
-          ldsm_x4_t(kbase + swz(r, c), b0, b1, b2, b3);
-          mma16816(dqa[j], a0, a1, a2, a3, b0, b1);
-          mma16816(dqa[j + 1], a0, a1, a2, a3, b2, b3);
-        }
-      }
-      const int qa = q0 + qr0 + g, qb2 = qa + 8;
-      float* dqh = dq + head_off;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int col = hc0 + j * 8 + 2 * t4;
-        if (qa < T) {
-          atomicAdd(dqh + static_cast<long long>(qa) * HD + col, dqa[j][0]);
-          atomicAdd(dqh + static_cast<long long>(qa) * HD + col + 1, dqa[j][1]);
-        }
-        if (qb2 < T) {
-          atomicAdd(dqh + static_cast<long long>(qb2) * HD + col, dqa[j][2]);
-          atomicAdd(dqh + static_cast<long long>(qb2) * HD + col + 1, dqa[j][3]);
-        }
-      }
-    }
-    __syncthreads();   // buffers of this query block may be refilled
-  }
-  // write dK, dV for this warp's 16 keys
-  if (key_a < T) {
-    bf16* kr = dk + head_off + static_cast<long long>(key_a) * HD;
-    bf16* vr = dv + head_off + static_cast<long long>(key_a) * HD;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      *reinterpret_cast<uint32_t*>(kr + j * 8 + 2 * t4) = pack_bf16x2(dK[j][0], dK[j][1]);
-      *reinterpret_cast<uint32_t*>(vr + j * 8 + 2 * t4) = pack_bf16x2(dV[j][0], dV[j][1]);
-    }
-  }
-  if (key_b < T) {
-    bf16* kr = dk + head_off + static_cast<long long>(key_b) * HD;
-    bf16* vr = dv + head_off + static_cast<long long>(key_b) * HD;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      *reinterpret_cast<uint32_t*>(kr + j * 8 + 2 * t4) = pack_bf16x2(dK[j][2], dK[j][3]);
-      *reinterpret_cast<uint32_t*>(vr + j * 8 + 2 * t4) = pack_bf16x2(dV[j][2], dV[j][3]);
-    }
-  }
 }
 
 }  // namespace
@@ -630,19 +671,29 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s) {
+                     cudaStream_t s, int* err) {
   static bool configured = false;
-  constexpr int smem = 2 * BWD_BN * 256 + 4 * BWD_BM * 256 + BWD_BN * 128 + 4 * BWD_BM * 4;
   if (!configured) {
-    cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
     configured = true;
   }
   const long long rows = 1ll * B * H * T;
   attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
-  dim3 grid((T + BWD_BN - 1) / BWD_BN, B * H);
-  attn_bwd_kernel<<<grid, BWD_THREADS, smem, s>>>(q, k, v, dout, lse, Dv, dq, dk, dv, B, H, T,
-                                                  1.f / sqrtf(static_cast<float>(HD)));
+  CUtensorMap mq, mk, mv, mdo;
+  const long long bh = 1ll * B * H;
+  const long long dims[4] = {HD, H, T, B};
+  const long long strides[3] = {HD * 2ll, 1ll * H * HD * 2, 1ll * T * H * HD * 2};
+  const int box[4] = {64, 1, 128, 1};
+  if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box)) {
+    if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
+    return;
+  }
+  dim3 grid((T + 127) / 128, B * H);
+  attn_bwd_tc_kernel<<<grid, 192, TB_SMEM, s>>>(mq, mk, mv, mdo, lse, Dv, dq, dk, dv, H, T,
+                                                1.f / sqrtf(static_cast<float>(HD)), err);
 }
 
 }  // namespace gpt

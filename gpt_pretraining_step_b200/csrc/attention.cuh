@@ -17,6 +17,6 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 // here, then accumulated), dk, dv [B, H, T, 128]; Dv [B, H, T] is scratch.
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s);
+                     cudaStream_t s, int* err);
 
 }  // namespace gpt

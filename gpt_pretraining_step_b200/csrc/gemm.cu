@@ -45,6 +45,29 @@ bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long lon
   return r == CUDA_SUCCESS;
 }
 
+// 4-D bf16 map over dims {d0, d1, d2, d3} (d0 innermost) with byte strides
+// s1, s2, s3 of dims 1..3, box {b0, b1, b2, b3}, 128-byte swizzle.
+bool make_map_4d(CUtensorMap* m, const void* ptr, const long long (&dims)[4], const long long (&strides)[3],
+                 const int (&box)[4]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[4], gs[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < 4; ++i) {
+    gd[i] = static_cast<cuuint64_t>(dims[i]);
+    bx[i] = static_cast<cuuint32_t>(box[i]);
+  }
+  for (int i = 0; i < 3; ++i) {
+    gs[i] = static_cast<cuuint64_t>(strides[i]);
+    if (gs[i] & 15) return false;
+  }
+  if (reinterpret_cast<uintptr_t>(ptr) & 15) return false;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>

@@ -432,7 +432,13 @@ __global__ void __launch_bounds__(192, 1)
               for (int j = 0; j < 32; ++j) { const float t = fmaxf(v[j], 0.f); v[j] = t * t; }
             } else if constexpr (EPI == EPI_DRELU2) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= 2.f * sqrtf(a[j]);
+              for (int j = 0; j < 32; ++j) {
+                // relu(u) = sqrt(h); h = relu(u)^2 is exact zero on half the entries, where
+                // the IEEE sqrt takes its slow path, so use the single-instruction form
+                float rt;
+                asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(a[j]));
+                v[j] *= 2.f * rt;
+              }
             } else if constexpr (EPI == EPI_AXPBY) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] = p.alpha * a[j] + p.beta * v[j];

@@ -46,4 +46,9 @@ int device_sm_count();
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
               long long ld, long long bs, int box_inner, int box_outer);
 
+// 4-D bf16 map, dims {d0 (innermost), d1, d2, d3}, byte strides of dims 1..3,
+// box {b0, b1, b2, b3}, 128-byte swizzle.
+bool make_map_4d(CUtensorMap* m, const void* ptr, const long long (&dims)[4], const long long (&strides)[3],
+                 const int (&box)[4]);
+
 }  // namespace gpt

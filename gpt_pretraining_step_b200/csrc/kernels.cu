@@ -114,65 +114,65 @@ __global__ void embed_segsum_kernel(const uint32_t* __restrict__ keys, int n, co
 }
 
 // --------------------------------------------------------------- RMSNorm
+//
+// One warp per row of d = 128 * NV fp32 values; every load of the row is
+// issued before the warp reduction so one memory latency covers the row.
 
-__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, bf16* __restrict__ y, float* __restrict__ rstd,
-                                   int M, int d) {
-  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+template <int NV>
+__global__ void __launch_bounds__(128) rmsnorm_fwd_kernel(const float* __restrict__ x, bf16* __restrict__ y,
+                                                          float* __restrict__ rstd, int M) {
+  constexpr int d = 128 * NV;
+  const int row = blockIdx.x * 4 + warp_id();
   if (row >= M) return;
   const float* xr = x + static_cast<long long>(row) * d;
-  float4 buf[kMaxVec];
+  float4 buf[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) buf[i] = *reinterpret_cast<const float4*>(xr + (i * 32 + lane_id()) * 4);
   float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    const int c = (i * 32 + lane_id()) * 4;
-    if (c < d) {
-      buf[i] = *reinterpret_cast<const float4*>(xr + c);
-      ss += buf[i].x * buf[i].x + buf[i].y * buf[i].y + buf[i].z * buf[i].z + buf[i].w * buf[i].w;
-    }
-  }
+  for (int i = 0; i < NV; ++i) ss += buf[i].x * buf[i].x + buf[i].y * buf[i].y + buf[i].z * buf[i].z + buf[i].w * buf[i].w;
   ss = warp_sum(ss);
-  const float r = rsqrtf(ss / d + 1e-6f);
+  const float r = rsqrtf(ss * (1.f / d) + 1e-6f);
   bf16* yr = y + static_cast<long long>(row) * d;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    const int c = (i * 32 + lane_id()) * 4;
-    if (c < d) store_bf16x4(yr + c, make_float4(buf[i].x * r, buf[i].y * r, buf[i].z * r, buf[i].w * r));
-  }
+  for (int i = 0; i < NV; ++i)
+    store_bf16x4(yr + (i * 32 + lane_id()) * 4, make_float4(buf[i].x * r, buf[i].y * r, buf[i].z * r, buf[i].w * r));
   if (lane_id() == 0) rstd[row] = r;
 }
 
-__global__ void rmsnorm_bwd_kernel(const float* __restrict__ dy, const bf16* __restrict__ y,
-                                   const float* __restrict__ rstd, float* __restrict__ dx,
-                                   bf16* __restrict__ dxb, int M, int d, int accumulate) {
-  const int row = blockIdx.x * (blockDim.x / 32) + warp_id();
+template <int NV>
+__global__ void __launch_bounds__(128) rmsnorm_bwd_kernel(const float* __restrict__ dy, const bf16* __restrict__ y,
+                                                          const float* __restrict__ rstd, float* __restrict__ dx,
+                                                          bf16* __restrict__ dxb, int M, int accumulate) {
+  constexpr int d = 128 * NV;
+  const int row = blockIdx.x * 4 + warp_id();
   if (row >= M) return;
   const long long off = static_cast<long long>(row) * d;
-  float4 g[kMaxVec], yy[kMaxVec];
+  float4 g[NV], p[NV];
+  uint2 yy[NV];
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    const int c = (i * 32 + lane_id()) * 4;
+    g[i] = *reinterpret_cast<const float4*>(dy + off + c);
+    yy[i] = *reinterpret_cast<const uint2*>(y + off + c);
+    p[i] = accumulate ? *reinterpret_cast<const float4*>(dx + off + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float r = rstd[row];
   float dot = 0.f;
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
-    const int c = (i * 32 + lane_id()) * 4;
-    if (c < d) {
-      g[i] = *reinterpret_cast<const float4*>(dy + off + c);
-      yy[i] = load_bf16x4(y + off + c);
-      dot += g[i].x * yy[i].x + g[i].y * yy[i].y + g[i].z * yy[i].z + g[i].w * yy[i].w;
-    }
-  }
-  dot = warp_sum(dot) / d;
-  const float r = rstd[row];
+  for (int i = 0; i < NV; ++i)
+    dot += g[i].x * bf16_lo(yy[i].x) + g[i].y * bf16_hi(yy[i].x) + g[i].z * bf16_lo(yy[i].y) + g[i].w * bf16_hi(yy[i].y);
+  dot = warp_sum(dot) * (1.f / d);
 #pragma unroll
-  for (int i = 0; i < kMaxVec; ++i) {
+  for (int i = 0; i < NV; ++i) {
     const int c = (i * 32 + lane_id()) * 4;
-    if (c < d) {
-      float4 o = make_float4(r * (g[i].x - yy[i].x * dot), r * (g[i].y - yy[i].y * dot),
-                             r * (g[i].z - yy[i].z * dot), r * (g[i].w - yy[i].w * dot));
-      if (accumulate) {
-        const float4 p = *reinterpret_cast<const float4*>(dx + off + c);
-        o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
-      }
-      *reinterpret_cast<float4*>(dx + off + c) = o;
-      store_bf16x4(dxb + off + c, o);
-    }
+    float4 o;
+    o.x = p[i].x + r * (g[i].x - bf16_lo(yy[i].x) * dot);
+    o.y = p[i].y + r * (g[i].y - bf16_hi(yy[i].x) * dot);
+    o.z = p[i].z + r * (g[i].z - bf16_lo(yy[i].y) * dot);
+    o.w = p[i].w + r * (g[i].w - bf16_hi(yy[i].y) * dot);
+    *reinterpret_cast<float4*>(dx + off + c) = o;
+    store_bf16x4(dxb + off + c, o);
   }
 }
 
@@ -483,13 +483,28 @@ void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, i
   embed_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(tok, wte, x, M, d, V, err);
 }
 
+#define GPT_NV_CASES(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
+
 void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s) {
-  rmsnorm_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(x, y, rstd, M, d);
+  if (M <= 0) return;
+  switch (d / 128) {
+#define GPT_FWD_CASE(n) case n: rmsnorm_fwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(x, y, rstd, M); break;
+    GPT_NV_CASES(GPT_FWD_CASE)
+#undef GPT_FWD_CASE
+    default: break;
+  }
 }
 
 void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dxb, int M, int d,
                         bool accumulate, cudaStream_t s) {
-  rmsnorm_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dy, y, rstd, dx, dxb, M, d, accumulate ? 1 : 0);
+  if (M <= 0) return;
+  switch (d / 128) {
+#define GPT_BWD_CASE(n) \
+  case n: rmsnorm_bwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(dy, y, rstd, dx, dxb, M, accumulate ? 1 : 0); break;
+    GPT_NV_CASES(GPT_BWD_CASE)
+#undef GPT_BWD_CASE
+    default: break;
+  }
 }
 
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn, const float* rq,

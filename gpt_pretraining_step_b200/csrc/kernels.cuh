@@ -16,7 +16,7 @@ void launch_rope_table(float2* tab, int T, cudaStream_t s);
 void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, int V, int* err,
                       cudaStream_t s);
 
-// y = x / sqrt(mean(x^2) + 1e-6) per row (bf16 out), rstd saved.
+// y = x / sqrt(mean(x^2) + 1e-6) per row (bf16 out), rstd saved; d a multiple of 128, <= 2048.
 void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s);
 
 // dx (+)= rstd * (dy - y * mean(dy * y)); also writes dx in bf16.
