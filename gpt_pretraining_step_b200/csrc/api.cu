@@ -52,11 +52,10 @@ struct Plan {
   // activations
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
   size_t xf, rf, z, stats, zt, row_loss, loss;
-  size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv;
+  size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, rope, err, tok, tgt;
   size_t act_bytes;
   size_t splitk_elems;
-  int splits_w[4];    // dW split-K factors: qkv, proj, fc, mproj
   int splits_lm;      // lm_head dx split-K factor
 };
 
@@ -131,16 +130,8 @@ void make_plan(const Dims& D, Plan& P) {
   }
   P.state_bytes = sb.off;
 
-  // split-K plans for the weight gradients (contraction over the M tokens)
-  const long long kb = (M + 63) / 64;
-  const long long shp[4][2] = {{(long long)d, 3 * (long long)d}, {(long long)d, (long long)d},
-                               {(long long)d, (long long)F}, {(long long)F, (long long)d}};
+  // split-K plan of the lm_head input gradient (contraction over the vocabulary)
   size_t sk = 0;
-  for (int i = 0; i < 4; ++i) {
-    const long long tiles = ((shp[i][0] + 127) / 128) * ((shp[i][1] + 255) / 256);
-    P.splits_w[i] = choose_splits(tiles, kb);
-    if (P.splits_w[i] > 1) sk = std::max<size_t>(sk, static_cast<size_t>(P.splits_w[i]) * shp[i][0] * shp[i][1]);
-  }
   {
     const long long tiles = ((D.Mc + 127) / 128) * ((d + 255) / 256);
     P.splits_lm = choose_splits(tiles, (V + 63) / 64);
@@ -171,14 +162,18 @@ void make_plan(const Dims& D, Plan& P) {
   P.loss = ab.take(16);
   P.dx = ab.take(M * d * 4);
   P.dxb = ab.take(M * d * 2);
+  // per-layer gradient inputs of the weight-gradient GEMMs, which run batched
+  // over the layers after the backward sweep: the bf16 residual gradient at the
+  // attention output (slot 2l) and at the block output (slot 2l+1), du, dqkv
+  P.gx = ab.take(2 * L * M * d * 2);
   P.dxn = ab.take(M * d * 4);
-  P.du = ab.take(M * F * 2);
+  P.du = ab.take(L * M * F * 2);
   P.dy = ab.take(M * d * 2);
   P.dqf = ab.take(M * d * 4);
   P.dk = ab.take(M * d * 2);
   P.dv = ab.take(M * d * 2);
   P.Dv = ab.take(M * H * 4);
-  P.dqkv = ab.take(M * 3 * d * 2);
+  P.dqkv = ab.take(L * M * 3 * d * 2);
   P.splitk = ab.take(std::max<size_t>(sk, 4) * 4);
   P.embws = ab.take(embed_bwd_workspace(D.M));
   const size_t xelems = std::max({L * d * 3 * d, L * d * d, 2 * L * d * F});
@@ -498,40 +493,36 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
 
   // --------------------------------------------------------------- backward
   float* dx = c->A<float>(P.dx);
-  bf16* dxb = c->A<bf16>(P.dxb);
-  bf16* du = c->A<bf16>(P.du);
   bf16* dy = c->A<bf16>(P.dy);
   float* dqf = c->A<float>(P.dqf);
   bf16* dk = c->A<bf16>(P.dk);
   bf16* dv = c->A<bf16>(P.dv);
-  bf16* dqkv = c->A<bf16>(P.dqkv);
+  bf16* gx = c->A<bf16>(P.gx);
+  bf16* du_all = c->A<bf16>(P.du);
+  bf16* dqkv_all = c->A<bf16>(P.dqkv);
+  auto gatt = [&](int l) { return gx + (2 * static_cast<size_t>(l)) * Md; };       // grad at attention output
+  auto gmlp = [&](int l) { return gx + (2 * static_cast<size_t>(l) + 1) * Md; };   // grad at block output
   {
     ProfScope ps(c, GPT_PROF_NORM);
-    launch_rmsnorm_bwd(dxn, xf, rf, dx, dxb, M, d, false, s);
+    launch_rmsnorm_bwd(dxn, xf, rf, dx, gmlp(L - 1), M, d, false, s);
   }
   c->launches += 1;
   for (int l = L - 1; l >= 0; --l) {
-    bf16* xn1l = xn1 + l * Md;
     bf16* xn2l = xn2 + l * Md;
     bf16* hl = h + static_cast<size_t>(l) * M * F;
     bf16* ol = o + l * Md;
+    bf16* du = du_all + static_cast<size_t>(l) * M * F;
+    bf16* dqkv = dqkv_all + static_cast<size_t>(l) * M * 3 * d;
     // MLP down: dh = dx W_d^T, du = dh * 2 relu(u) with relu(u) = sqrt(h)
     {
       ProfScope ps(c, GPT_PROF_DX_GEMM);
       GemmCall g = base_call(M, F, d);
-      g.A = dxb; g.lda = d;
+      g.A = gmlp(l); g.lda = d;
       g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.ldb = d;   // B(n = F index, k = d index)
       g.epi = EPI_DRELU2; g.out_es = 2; g.aux_es = 2;
       g.p.out = du; g.p.ldo = F; g.p.aux = hl; g.p.ld_aux = F; g.p.err = err;
       GPT_CK(gemm_run(g, s));
       c->launches += 1;
-    }
-    {
-      GemmCall g = base_call(F, d, M);   // dW_d = h^T dx
-      g.A = hl; g.a_mn = true; g.lda = F;
-      g.B = dxb; g.b_mn = true; g.ldb = d;
-      int rc = run_f32(c, g, c->G(5) + static_cast<size_t>(l) * F * d, acc, P.splits_w[3], GPT_PROF_DW_GEMM);
-      if (rc) return rc;
     }
     {
       GemmCall g = base_call(M, d, F);   // dxn2 = du W_fc^T
@@ -541,34 +532,20 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       if (rc) return rc;
     }
     {
-      GemmCall g = base_call(d, F, M);   // dW_fc = xn2^T du
-      g.A = xn2l; g.a_mn = true; g.lda = d;
-      g.B = du; g.b_mn = true; g.ldb = F;
-      int rc = run_f32(c, g, c->G(4) + static_cast<size_t>(l) * d * F, acc, P.splits_w[2], GPT_PROF_DW_GEMM);
-      if (rc) return rc;
-    }
-    {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_bwd(dxn, xn2l, r2 + static_cast<size_t>(l) * M, dx, dxb, M, d, true, s);
+      launch_rmsnorm_bwd(dxn, xn2l, r2 + static_cast<size_t>(l) * M, dx, gatt(l), M, d, true, s);
     }
     c->launches += 1;
     // attention output projection
     {
       ProfScope ps(c, GPT_PROF_DX_GEMM);
       GemmCall g = base_call(M, d, d);   // dy = dx W_o^T
-      g.A = dxb; g.lda = d;
+      g.A = gatt(l); g.lda = d;
       g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.ldb = d;
       g.epi = EPI_STORE; g.out_es = 2; g.aux_es = 2;
       g.p.out = dy; g.p.ldo = d; g.p.err = err;
       GPT_CK(gemm_run(g, s));
       c->launches += 1;
-    }
-    {
-      GemmCall g = base_call(d, d, M);   // dW_o = o^T dx
-      g.A = ol; g.a_mn = true; g.lda = d;
-      g.B = dxb; g.b_mn = true; g.ldb = d;
-      int rc = run_f32(c, g, c->G(3) + static_cast<size_t>(l) * d * d, acc, P.splits_w[1], GPT_PROF_DW_GEMM);
-      if (rc) return rc;
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
@@ -589,17 +566,34 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       if (rc) return rc;
     }
     {
-      GemmCall g = base_call(d, 3 * d, M);   // dW_qkv = xn1^T dqkv
-      g.A = xn1l; g.a_mn = true; g.lda = d;
-      g.B = dqkv; g.b_mn = true; g.ldb = 3 * d;
-      int rc = run_f32(c, g, c->G(2) + static_cast<size_t>(l) * d * 3 * d, acc, P.splits_w[0], GPT_PROF_DW_GEMM);
-      if (rc) return rc;
-    }
-    {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_bwd(dxn, xn1l, r1 + static_cast<size_t>(l) * M, dx, dxb, M, d, true, s);
+      // the bf16 copy feeds the next (lower) block; below block 0 only the fp32 gradient is used
+      launch_rmsnorm_bwd(dxn, xn1 + l * Md, r1 + static_cast<size_t>(l) * M, dx,
+                         l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), M, d, true, s);
     }
     c->launches += 1;
+  }
+  // weight gradients of every block matrix, each kind as one GEMM batched over the layers:
+  // dW[l] = act[l]^T grad[l], contraction over the M tokens
+  {
+    ProfScope ps(c, GPT_PROF_DW_GEMM);
+    struct DW { const bf16* a; long long lda, a_bs; const bf16* b; long long ldb, b_bs; int rows, cols; float* out; };
+    const DW dws[4] = {
+        {xn1, d, static_cast<long long>(Md), dqkv_all, 3ll * d, 3ll * Md, d, 3 * d, c->G(2)},
+        {o, d, static_cast<long long>(Md), gx, d, 2ll * Md, d, d, c->G(3)},
+        {xn2, d, static_cast<long long>(Md), du_all, F, 1ll * M * F, d, F, c->G(4)},
+        {h, F, 1ll * M * F, gx + Md, d, 2ll * Md, F, d, c->G(5)},
+    };
+    for (const DW& w : dws) {
+      GemmCall g = base_call(w.rows, w.cols, M);
+      g.batch = L;
+      g.A = w.a; g.a_mn = true; g.lda = w.lda; g.a_bs = w.a_bs;
+      g.B = w.b; g.b_mn = true; g.ldb = w.ldb; g.b_bs = w.b_bs;
+      g.epi = acc ? EPI_ACC : EPI_STORE; g.out_es = 4; g.aux_es = 4;
+      g.p.out = w.out; g.p.ldo = w.cols; g.p.out_bs = 1ll * w.rows * w.cols; g.p.err = err;
+      GPT_CK(gemm_run(g, s));
+    }
+    c->launches += 4;
   }
   {
     ProfScope ps(c, GPT_PROF_EMBED);
