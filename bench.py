@@ -231,6 +231,7 @@ def run_ours(a):
     import torch.distributed as dist
 
     import gpt_pretraining_step_b200 as g
+    from gpt_pretraining_step_b200 import dp
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -245,15 +246,15 @@ def run_ours(a):
     torch.cuda.set_stream(stream)
     st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
                    ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream)
-    tok = torch.tensor(syn.tokens(s, seed=1 + 100 * rank)).cuda()
-    tgt = torch.tensor(syn.targets(s, seed=2 + 100 * rank)).cuda()
+    tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(1, rank))).cuda()
+    tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(2, rank))).cuda()
     grads = st.grad_view() if world > 1 else None
     hp = dict(muon=(0.02, 0.95, 0.0), adam=(3e-3, 0.8, 0.95, 1e-10, 0.0))
 
     def step():
         st.fwd_bwd(tok, tgt)
         if grads is not None:
-            dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+            dp.average_gradients(grads)
         st.muon_step(*hp["muon"])
         st.adamw_step(*hp["adam"])
 
@@ -288,11 +289,7 @@ def run_ours(a):
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
-    ms = ev0.elapsed_time(ev1) / a.steps
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = dp.max_over_ranks(ev0.elapsed_time(ev1) / a.steps, device="cuda")
     st.check()
     live = st.profile_read()
     st.profile_enable([])
@@ -337,9 +334,7 @@ def run_ours(a):
     if not a.no_e2e:
         e2e = run_e2e(a, st, s, rank, world, grads, stream)
         if world > 1:
-            t = torch.tensor([e2e["ms_per_step"]], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(t.item())
+            e2e["ms_per_step"] = dp.max_over_ranks(e2e["ms_per_step"], device="cuda")
             e2e["value"] = tokens_per_step / (e2e["ms_per_step"] / 1e3)
 
     cpu = None
@@ -380,8 +375,9 @@ def run_e2e(a, st, s, rank, world, grads, stream):
     import torch.distributed as dist
 
     import gpt_pretraining_step_b200 as g
-    tok = torch.tensor(syn.tokens(s, seed=11 + 100 * rank)).pin_memory()
-    tgt = torch.tensor(syn.targets(s, seed=12 + 100 * rank)).pin_memory()
+    from gpt_pretraining_step_b200 import dp
+    tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(11, rank))).pin_memory()
+    tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(12, rank))).pin_memory()
     hp = g.HParams(muon_lr=0.02, muon_momentum=0.95, muon_wd=0.0, adam_lr=3e-3, adam_beta1=0.8, adam_beta2=0.95,
                    adam_eps=1e-10, adam_wd=0.0)
     dtok = torch.empty_like(tok, device="cuda")
@@ -394,7 +390,7 @@ def run_e2e(a, st, s, rank, world, grads, stream):
         dtok.copy_(tok, non_blocking=True)
         dtgt.copy_(tgt, non_blocking=True)
         loss = st.fwd_bwd(dtok, dtgt)
-        dist.all_reduce(grads, op=dist.ReduceOp.AVG)
+        dp.average_gradients(grads)
         st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)
         st.adamw_step(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd)
         loss_host.copy_(loss.reshape(1), non_blocking=True)
