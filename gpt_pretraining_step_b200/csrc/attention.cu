@@ -342,18 +342,21 @@ __global__ void __launch_bounds__(192, 1)
 //                 S^T = K Q^T and dP^T = V dO^T          (TMEM cols 0 and 128)
 //                 dV += P^T dO, dK += dS^T Q              (TMEM cols 256, 384)
 //                 dQ_i = dS K into cols 0 (S^T is consumed by then)
-//   warps 2..5  one key row (TMEM lane) per thread: P^T = exp(S^T/sqrt(d) - lse),
-//               dS^T = P^T (dP^T - D) / sqrt(d) as bf16 tiles in shared memory
-//               (the dS^T tile is also the MN-major A operand of dS K); then one
-//               query row per thread to add dQ_i into the fp32 dq buffer with
-//               vector reductions; finally dK and dV of the block to global.
+//   warps 2..9  two warps per TMEM lane quarter, each on half of the 128
+//               columns: P^T = exp(S^T/sqrt(d) - lse), dS^T = P^T (dP^T - D)
+//               / sqrt(d) as bf16 tiles in shared memory (the dS^T tile is also
+//               the MN-major A operand of dS K); then dQ_i is staged through
+//               the two (by then idle) tiles as fp32 in TMA's 128-byte-swizzled
+//               layout and added into the fp32 dq buffer by TMA bulk reduce-add;
+//               finally dK and dV of the block to global memory.
 
 constexpr int TB_SMEM = 7 * TF_BUF + 1024 + 1024 + 512;
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                       const float* __restrict__ lse, const float* __restrict__ Dv, float* __restrict__ dq,
+                       const __grid_constant__ CUtensorMap tdq,
+                       const float* __restrict__ lse, const float* __restrict__ Dv,
                        bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int T, float scale, int* err) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -393,9 +396,9 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(do_full, 1);
     mbar_init(do_empty, 1);
     mbar_init(sd_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 256);
     mbar_init(mm_done, 1);
-    mbar_init(s_free, 128);
+    mbar_init(s_free, 256);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -503,8 +506,9 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // --------------------------------------------- P^T, dS^T, dQ, dK, dV
     const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;        // which 64 columns of the row
     const int r = quarter * 32 + lane;       // key row for P/dS, query row for dQ
-    const int t128 = threadIdx.x - 64;       // 0..127
+    const int t256 = threadIdx.x - 64;       // 0..255
     const int key = k0 + r;
     const bool key_ok = key < T;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
@@ -515,22 +519,31 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       return __all_sync(0xffffffffu, got);
     };
+    // this thread's share of the query block's lse (log2 units; +inf past T so P = 0)
+    // or D, fetched one block ahead so the load latency hides behind a whole block
+    auto fetch = [&](int it2) -> float {
+      const int q0f = (j + it2) * 128;
+      if (t256 < 128) {
+        const int qq = q0f + t256;
+        return qq < T ? __ldg(lse + static_cast<long long>(bh) * T + qq) * 1.4426950408889634f : INFINITY;
+      }
+      const int qq = q0f + t256 - 128;
+      return qq < T ? __ldg(Dv + static_cast<long long>(bh) * T + qq) : 0.f;
+    };
+    float staged = n_it > 0 ? fetch(0) : 0.f;
     for (int it = 0; it < n_it && ok; ++it) {
       const int i = j + it;
       const int q0 = i * 128;
-      // the query block's lse (log2 units; +inf past T so P = 0) and D
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      {
-        const int qq = q0 + t128;
-        lse_s[t128] = qq < T ? lse[static_cast<long long>(bh) * T + qq] * 1.4426950408889634f : INFINITY;
-        dd_s[t128] = qq < T ? Dv[static_cast<long long>(bh) * T + qq] : 0.f;
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (t256 < 128) lse_s[t256] = staged;
+      else dd_s[t256 - 128] = staged;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (it + 1 < n_it) staged = fetch(it + 1);
       if (!wait_all(sd_full, it & 1)) { ok = false; break; }
       tc_fence_after();
       const bool diag = i == j;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t sr[32], dr[32];
         tmem_load32_async(tmem + lane_base + c * 32, sr);
         tmem_load32_async(tmem + lane_base + 128 + c * 32, dr);
@@ -567,35 +580,56 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       mbar_arrive(p_full);
-      // dQ_i: one query row per thread, added to the fp32 accumulator
+      // dQ_i (TMEM lane = query row): stage it in the P^T/dS^T tiles, which the
+      // finished MMAs no longer read, then add it to dq with TMA reduce-add
       if (!wait_all(mm_done, it & 1)) { ok = false; break; }
       tc_fence_after();
-      const int qrow = q0 + r;
-      float* dqrow = dq + (static_cast<long long>(bh) * T + qrow) * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t qr[32];
-        tmem_load32_async(tmem + lane_base + c * 32, qr);
+      {
+        uint32_t qa[32], qb[32];
+        tmem_load32_async(tmem + lane_base + (2 * half) * 32, qa);
+        tmem_load32_async(tmem + lane_base + (2 * half + 1) * 32, qb);
         tmem_wait_ld();
-        if (qrow < T) {
+        tc_fence_before();
+        mbar_arrive(s_free);   // the S/dQ columns may take the next S^T now
+        // rows 0..63 go to the P^T tile, 64..127 to the dS^T tile; each holds four
+        // [64 rows][32 fp32] boxes of 8 KB in 128-byte-swizzled order
+        uint8_t* stage = (r < 64 ? sPt : sdSt);
+        const int rr = r & 63;
 #pragma unroll
-          for (int g = 0; g < 8; ++g)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dqrow + c * 32 + 4 * g),
-                         "f"(__uint_as_float(qr[4 * g])), "f"(__uint_as_float(qr[4 * g + 1])),
-                         "f"(__uint_as_float(qr[4 * g + 2])), "f"(__uint_as_float(qr[4 * g + 3]))
-                         : "memory");
+        for (int cc = 0; cc < 2; ++cc) {
+          const uint32_t* src = cc == 0 ? qa : qb;
+          uint8_t* box = stage + (2 * half + cc) * 8192 + rr * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4*>(box + ((u ^ (rr & 7)) << 4)) =
+                make_uint4(src[4 * u], src[4 * u + 1], src[4 * u + 2], src[4 * u + 3]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(s_free);
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (t256 == 0) {
+#pragma unroll
+        for (int rh = 0; rh < 2; ++rh)
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            asm volatile(
+                "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                    reinterpret_cast<uint64_t>(&tdq)),
+                "r"(smem_u32((rh ? sdSt : sPt) + c * 8192)), "r"(c * 32), "r"(q0 + rh * 64), "r"(bh)
+                : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        // the tiles are rewritten by the next block's softmax: wait until TMA has read them
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+      }
     }
+    if (t256 == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     // dK and dV of this key block (complete after the last mm_done)
     if (ok) {
       tc_fence_after();
       bf16* dkrow = dk + (static_cast<long long>(bh) * T + key) * 128;
       bf16* dvrow = dv + (static_cast<long long>(bh) * T + key) * 128;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t vr[32], kr[32];
         tmem_load32_async(tmem + lane_base + 256 + c * 32, vr);
         tmem_load32_async(tmem + lane_base + 384 + c * 32, kr);
@@ -680,19 +714,20 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const long long rows = 1ll * B * H * T;
   attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const long long bh = 1ll * B * H;
   const long long dims[4] = {HD, H, T, B};
   const long long strides[3] = {HD * 2ll, 1ll * H * HD * 2, 1ll * T * H * HD * 2};
   const int box[4] = {64, 1, 128, 1};
   if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box)) {
+      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
+      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }
   dim3 grid((T + 127) / 128, B * H);
-  attn_bwd_tc_kernel<<<grid, 192, TB_SMEM, s>>>(mq, mk, mv, mdo, lse, Dv, dq, dk, dv, H, T,
+  attn_bwd_tc_kernel<<<grid, 320, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, T,
                                                 1.f / sqrtf(static_cast<float>(HD)), err);
 }
 
