@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--config", default="d20", choices=["d12", "d20", "d24", "d26"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ns-tf32-steps", type=int, default=3)
+    ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
+                    help="fp8: forward block projections on e4m3 operands")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="per-category device times in the JSON line")
@@ -245,7 +247,8 @@ def run_ours(a):
     stream = torch.cuda.Stream()
     torch.cuda.set_stream(stream)
     st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
-                   ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream)
+                   ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream,
+                   precision=1 if a.precision == "fp8" else 0)
     tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(1, rank))).cuda()
     tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(2, rank))).cuda()
     grads = st.grad_view() if world > 1 else None
@@ -347,7 +350,7 @@ def run_ours(a):
         out = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
             "config": {"workload": f"{a.config} GPT step (fwd+bwd+Muon+AdamW)", "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
                        "parallelism": f"dp{world}", "ns_tf32_steps": a.ns_tf32_steps,

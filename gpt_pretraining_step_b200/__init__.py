@@ -18,12 +18,13 @@ KIND_PARAM, KIND_GRAD, KIND_MOM, KIND_ADAM_M, KIND_ADAM_V = 0, 1, 2, 3, 4
 GROUP_ADAMW, GROUP_MUON = 0, 1
 PROF_CATEGORIES = ["qkv_gemm", "proj_gemm", "fc_gemm", "down_gemm", "attn_fwd", "attn_bwd", "logits_gemm",
                    "ce_finish", "lm_dx_gemm", "lm_dw_gemm", "dx_gemm", "dw_gemm", "norm", "qk_bwd", "embed",
-                   "ns_gemm", "muon_elem", "adamw"]
+                   "ns_gemm", "muon_elem", "adamw", "fp8_quant"]
 
 ABI_FUNCTIONS = [
     "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "adamw_step", "gpt_train_step_host",
     "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
-    "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_attention_fwd",
+    "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3",
+    "gpt_op_matmul_fp8", "gpt_op_attention_fwd",
     "gpt_op_attention_bwd", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
     "gpt_op_newton_schulz_noalloc",
 ]
@@ -82,6 +83,8 @@ def lib():
             "gpt_last_error": (ctypes.c_char_p, []),
             "gpt_op_matmul_bf16": (i32, [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]),
             "gpt_op_matmul_tf32": (i32, [vp, vp, vp, i32, i32, i32, i32, vp]),
+            "gpt_op_quantize_e4m3": (i32, [vp, ctypes.c_longlong, vp, vp, vp, vp]),
+            "gpt_op_matmul_fp8": (i32, [vp, vp, vp, i32, i32, i32, vp, vp, i32, vp]),
             "gpt_op_attention_fwd": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp]),
             "gpt_op_attention_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp]),
             "gpt_op_rmsnorm_fwd": (i32, [vp, vp, vp, i32, i32, vp]),
@@ -103,9 +106,11 @@ def _check(rc):
     return rc
 
 
-def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=3, lm_chunk_rows=0, seed=0):
+def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=3, lm_chunk_rows=0, seed=0,
+                precision=0):
     return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
-                  mlp_mult=4, precision=0, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows, seed=seed)
+                  mlp_mult=4, precision=precision, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows,
+                  seed=seed)
 
 
 def workspace_size(cfg: Config):
@@ -132,9 +137,9 @@ class GPTStep:
     """
 
     def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=3, lm_chunk_rows=0,
-                 seed=0, stream=None):
+                 seed=0, stream=None, precision=0):
         import torch
-        self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed)
+        self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision)
         self.sizes = workspace_size(self.cfg)
         dev = torch.device("cuda", torch.cuda.current_device())
         self.stream = stream if stream is not None else torch.cuda.current_stream()
@@ -247,6 +252,24 @@ def matmul_tf32(A, B, M, N, K, b_trans=False, stream=None):
     import torch
     C = torch.empty((M, N), dtype=torch.float32, device=A.device)
     _check(lib().gpt_op_matmul_tf32(_ptr(A), _ptr(B), _ptr(C), M, N, K, int(b_trans), _stream(stream)))
+    return C
+
+
+def quantize_e4m3(x, stream=None):
+    """(q uint8 tensor of e4m3 codes, inv scale tensor) for a bf16 tensor x."""
+    import torch
+    q = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    inv = torch.empty(1, dtype=torch.float32, device=x.device)
+    amax = torch.empty(1, dtype=torch.int32, device=x.device)
+    _check(lib().gpt_op_quantize_e4m3(_ptr(x), x.numel(), _ptr(q), _ptr(inv), _ptr(amax), _stream(stream)))
+    return q.view(x.shape), inv
+
+
+def matmul_fp8(A, B, M, N, K, inv_a, inv_b, b_trans=False, stream=None):
+    import torch
+    C = torch.empty((M, N), dtype=torch.float32, device=A.device)
+    _check(lib().gpt_op_matmul_fp8(_ptr(A), _ptr(B), _ptr(C), M, N, K, _ptr(inv_a), _ptr(inv_b), int(b_trans),
+                                   _stream(stream)))
     return C
 
 

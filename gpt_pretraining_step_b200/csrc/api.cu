@@ -38,7 +38,7 @@ int fail(int code, const std::string& msg) {
 constexpr size_t kAlign = 256;
 
 struct Dims {
-  int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32;
+  int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32, fp8;
 };
 
 // Offsets (bytes) into the three caller buffers.
@@ -54,6 +54,7 @@ struct Plan {
   size_t xf, rf, z, stats, zt, row_loss, loss;
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, rope, err, tok, tgt;
+  size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
   int splits_lm;      // lm_head dx split-K factor
@@ -91,7 +92,7 @@ int dims_from(const gpt_config* c, Dims& D) {
   if (c->depth < 1 || c->depth > 256) return fail(GPT_EINVAL, "depth out of range");
   if (c->head_dim != 128) return fail(GPT_EINVAL, "head_dim must be 128");
   if (c->mlp_mult != 4) return fail(GPT_EINVAL, "mlp_mult must be 4");
-  if (c->precision != 0) return fail(GPT_EINVAL, "only precision 0 (bf16) is supported");
+  if (c->precision != 0 && c->precision != 1) return fail(GPT_EINVAL, "precision must be 0 (bf16) or 1 (fp8)");
   if (c->ns_tf32_steps < 0 || c->ns_tf32_steps > 5) return fail(GPT_EINVAL, "ns_tf32_steps must be in 0..5");
   D.L = c->depth;
   D.d = c->d_model ? c->d_model : 64 * c->depth;
@@ -110,6 +111,7 @@ int dims_from(const gpt_config* c, Dims& D) {
   D.Mc = std::min(D.Mc, D.M);
   D.tiles_lm = (D.V + 255) / 256;
   D.n_tf32 = c->ns_tf32_steps;
+  D.fp8 = c->precision == 1;
   return GPT_OK;
 }
 
@@ -156,7 +158,7 @@ void make_plan(const Dims& D, Plan& P) {
   P.xf = ab.take(M * d * 2);
   P.rf = ab.take(M * 4);
   P.z = ab.take(static_cast<size_t>(D.Mc) * V * 2);
-  P.stats = ab.take(static_cast<size_t>(D.Mc) * D.tiles_lm * 8);
+  P.stats = ab.take(static_cast<size_t>(D.Mc) * D.tiles_lm * 2 * 8);   // one partial per half tile
   P.zt = ab.take(static_cast<size_t>(D.Mc) * 4);
   P.row_loss = ab.take(M * 4);
   P.loss = ab.take(16);
@@ -190,6 +192,17 @@ void make_plan(const Dims& D, Plan& P) {
   P.err = ab.take(16);
   P.tok = ab.take(M * 4);
   P.tgt = ab.take(M * 4);
+  {
+    // fp8 e4m3 copies of the block weights and one activation operand, with their scales
+    const bool f8 = D.fp8 != 0;
+    const size_t wn[4] = {L * d * 3 * d, L * d * d, L * d * F, L * F * d};
+    for (int i = 0; i < 4; ++i) P.wq8[i] = ab.take(f8 ? wn[i] : 16);
+    P.winv = ab.take(4 * L * 4);
+    P.wamax = ab.take(4 * L * 4);
+    P.act8 = ab.take(f8 ? M * F : 16);
+    P.act_inv = ab.take(16);
+    P.act_amax = ab.take(16);
+  }
   P.act_bytes = ab.off;
 }
 
@@ -378,6 +391,37 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     else clamp_targets_kernel<<<64, 256, 0, s>>>(tgt, tgt, M, V);
     launch_embed_fwd(tok, c->Wb(0), x, M, d, V, err, s);
   }
+  // fp8: e4m3 copies of every block matrix, one scale per matrix
+  uint8_t* act8 = c->A<uint8_t>(P.act8);
+  float* act_inv = c->A<float>(P.act_inv);
+  unsigned int* act_amax = c->A<unsigned int>(P.act_amax);
+  float* winv = c->A<float>(P.winv);
+  if (D.fp8) {
+    ProfScope ps(c, GPT_PROF_FP8_QUANT);
+    const long long wn[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+    for (int gi = 0; gi < 4; ++gi)
+      launch_quantize_e4m3(c->Wb(2 + gi), wn[gi], L, c->A<unsigned int>(P.wamax) + gi * L,
+                           c->A<uint8_t>(P.wq8[gi]), winv + gi * L, s);
+    c->launches += 8;
+  }
+  // operand A of a forward projection: bf16 as it is, or quantised to e4m3 into act8
+  auto fwd_a = [&](GemmCall& g, const bf16* a, long long rows, long long cols, int grp, int l) {
+    if (!D.fp8) {
+      g.A = a;
+      return;
+    }
+    {
+      ProfScope ps(c, GPT_PROF_FP8_QUANT);
+      launch_quantize_e4m3(a, rows * cols, 1, act_amax, act8, act_inv, s);
+      c->launches += 2;
+    }
+    g.es = 1;
+    g.A = act8;
+    const long long wn[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+    g.B = c->A<uint8_t>(P.wq8[grp - 2]) + static_cast<size_t>(l) * wn[grp - 2];
+    g.p.dq_a = act_inv;
+    g.p.dq_b = winv + (grp - 2) * L + l;
+  };
   c->launches += 3;
 
   // ---------------------------------------------------------------- forward
@@ -395,10 +439,10 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
     }
     {
-      ProfScope ps(c, GPT_PROF_QKV_GEMM);
       GemmCall g = base_call(M, 3 * d, d);
-      g.A = xn1l; g.lda = d;
       g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.b_mn = true; g.ldb = 3 * d;
+      fwd_a(g, xn1l, M, d, 2, l); g.lda = d;
+      ProfScope ps(c, GPT_PROF_QKV_GEMM);
       g.bn = 128; g.epi = EPI_QKV; g.out_es = 2; g.aux_es = 2;
       g.p.qkv_out[0] = ql; g.p.qkv_out[1] = kl; g.p.qkv_out[2] = vl;
       g.p.f32a = rq + static_cast<size_t>(l) * M * H;
@@ -411,10 +455,10 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err);
     }
     {
-      ProfScope ps(c, GPT_PROF_PROJ_GEMM);
       GemmCall g = base_call(M, d, d);
-      g.A = ol; g.lda = d;
       g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.b_mn = true; g.ldb = d;
+      fwd_a(g, ol, M, d, 3, l); g.lda = d;
+      ProfScope ps(c, GPT_PROF_PROJ_GEMM);
       g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
       g.p.out = x; g.p.ldo = d; g.p.err = err;
       GPT_CK(gemm_run(g, s));
@@ -424,19 +468,19 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       launch_rmsnorm_fwd(x, xn2l, r2 + static_cast<size_t>(l) * M, M, d, s);
     }
     {
-      ProfScope ps(c, GPT_PROF_FC_GEMM);
       GemmCall g = base_call(M, F, d);
-      g.A = xn2l; g.lda = d;
       g.B = c->Wb(4) + static_cast<size_t>(l) * d * F; g.b_mn = true; g.ldb = F;
+      fwd_a(g, xn2l, M, d, 4, l); g.lda = d;
+      ProfScope ps(c, GPT_PROF_FC_GEMM);
       g.epi = EPI_RELU2; g.out_es = 2; g.aux_es = 2;
       g.p.out = hl; g.p.ldo = F; g.p.err = err;
       GPT_CK(gemm_run(g, s));
     }
     {
-      ProfScope ps(c, GPT_PROF_DOWN_GEMM);
       GemmCall g = base_call(M, d, F);
-      g.A = hl; g.lda = F;
       g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.b_mn = true; g.ldb = d;
+      fwd_a(g, hl, M, F, 5, l); g.lda = F;
+      ProfScope ps(c, GPT_PROF_DOWN_GEMM);
       g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
       g.p.out = x; g.p.ldo = d; g.p.err = err;
       GPT_CK(gemm_run(g, s));
@@ -467,8 +511,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_CE_FINISH);
-      launch_ce_finish(z, c->A<float2>(P.stats), c->A<float>(P.zt), tgt + r0, row_loss + r0, rows, V, D.tiles_lm,
-                       1.f / static_cast<float>(M), s);
+      launch_ce_finish(z, c->A<float2>(P.stats), c->A<float>(P.zt), tgt + r0, row_loss + r0, rows, V,
+                       2 * D.tiles_lm, 1.f / static_cast<float>(M), s);
     }
     c->launches += 2;
     {
@@ -1008,6 +1052,31 @@ int gpt_op_matmul_tf32(const float* A, const float* B, float* C, int M, int N, i
   g.B = B; g.ldb = K;
   g.bn = 128; g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
   g.p.out = C; g.p.ldo = N;
+  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  return GPT_OK;
+}
+
+int gpt_op_quantize_e4m3(const void* x, long long n, void* q, float* inv, unsigned int* amax_scratch, void* stream) {
+  if (!x || !q || !inv || !amax_scratch) return fail(GPT_EINVAL, "null pointer");
+  if (n < 0) return fail(GPT_EINVAL, "negative size");
+  if (reinterpret_cast<uintptr_t>(x) & 15 || reinterpret_cast<uintptr_t>(q) & 7)
+    return fail(GPT_EINVAL, "x must be 16-byte and q 8-byte aligned");
+  launch_quantize_e4m3(static_cast<const bf16*>(x), n, 1, amax_scratch, static_cast<uint8_t*>(q), inv,
+                       static_cast<cudaStream_t>(stream));
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_op_matmul_fp8(const void* A, const void* B, float* C, int M, int N, int K, const float* inv_a,
+                      const float* inv_b, int b_trans, void* stream) {
+  if (!A || !B || !C || !inv_a || !inv_b) return fail(GPT_EINVAL, "null pointer");
+  if (M < 0 || N < 0 || K <= 0 || N % 16 || K % 16) return fail(GPT_EINVAL, "bad matmul shape (N, K multiples of 16)");
+  GemmCall g = base_call(M, N, K);
+  g.es = 1;
+  g.A = A; g.lda = K;
+  g.B = B; g.b_mn = b_trans == 0; g.ldb = b_trans ? K : N;
+  g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
+  g.p.out = C; g.p.ldo = N; g.p.dq_a = inv_a; g.p.dq_b = inv_b;
   GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
   return GPT_OK;
 }

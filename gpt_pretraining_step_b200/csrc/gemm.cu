@@ -38,7 +38,9 @@ bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long lon
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (strides[0] & 15) || (strides[1] & 15)) return false;
-  CUresult r = fn(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+  const CUtensorMapDataType dt = es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                : (es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  CUresult r = fn(m, dt, 3,
                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -81,7 +83,7 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParam
     configured = true;
   }
   const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
-  kern<<<grid, 192, C::SMEM, s>>>(ma, mb, p);
+  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, p);
   return cudaGetLastError();
 }
 
@@ -108,7 +110,7 @@ int gemm_tiles(const GemmCall& c) {
 
 cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   if (c.M <= 0 || c.N <= 0 || c.batch <= 0) return cudaSuccess;
-  if (c.K <= 0 || (c.bn != 128 && c.bn != 256) || (c.es != 2 && c.es != 4)) return cudaErrorInvalidValue;
+  if (c.K <= 0 || (c.bn != 128 && c.bn != 256) || (c.es != 1 && c.es != 2 && c.es != 4)) return cudaErrorInvalidValue;
   if (c.sym && (c.M != c.N || c.bn != 128)) return cudaErrorInvalidValue;
   if (c.N % 8) return cudaErrorInvalidValue;
   // 32-bit operands are staged K-major only (the 128-byte swizzle atom used here
@@ -174,6 +176,12 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(float, 128, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, bf16, float)
+  // fp8 e4m3 forward projections (operands as raw bytes)
+  GPT_GEMM_CASE(uint8_t, 128, false, true, EPI_QKV, bf16, bf16)
+  GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_ACC, float, float)
+  GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_RELU2, bf16, bf16)
+  GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_STORE, float, float)
+  GPT_GEMM_CASE(uint8_t, 256, false, false, EPI_STORE, float, float)
 #undef GPT_GEMM_CASE
   return cudaErrorInvalidValue;
 }

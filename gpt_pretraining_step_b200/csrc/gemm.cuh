@@ -2,10 +2,11 @@
 // accumulators in TMEM, operands staged by TMA into a 128-byte-swizzled
 // shared-memory ring, and a fused epilogue.
 //
-// Roles (192 threads, one CTA per SM, persistent over work units):
+// Roles (320 threads, one CTA per SM, persistent over work units):
 //   warp 0      TMA producer (one elected lane)
 //   warp 1      TMEM allocator and MMA issuer (one elected lane)
-//   warps 2..5  epilogue: each thread owns one accumulator row (TMEM lane)
+//   warps 2..9  epilogue: two warps per TMEM lane quarter, each thread owning
+//               one accumulator row (TMEM lane) and half of the tile's columns
 // Two accumulator buffers in TMEM let the epilogue of tile i overlap the
 // MMAs of tile i+1.  Every mbarrier wait is bounded; on expiry the CTA
 // raises an abort flag, drains its in-flight copies and MMAs, frees TMEM
@@ -22,14 +23,14 @@ namespace gpt {
 template <int ES, int BN>
 struct GemmCfg {
   static constexpr int BK = 128 / ES;                 // elements of K per stage (one 128 B row)
-  static constexpr int MMA_K = 32 / ES;               // K per tcgen05.mma
+  static constexpr int MMA_K = 32 / ES;               // K per tcgen05.mma (16 bf16, 8 tf32, 32 fp8)
   static constexpr int A_BYTES = 128 * 128;
   static constexpr int B_BYTES = BN * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int CHUNK_BYTES = BK * 128;        // one MN-major box: BK rows of 128 B
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + 1024;   // + epilogue exchange
 };
 
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
@@ -122,12 +123,12 @@ __device__ __forceinline__ void store_scalar(OutT* dst, float x) {
 // ------------------------------------------------------------------ kernel
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ GemmParams p) {
   constexpr int ES = sizeof(T);
   using C = GemmCfg<ES, BN>;
-  constexpr uint32_t IDESC = make_idesc(ES == 2 ? 1 : 2, BN, A_MN, B_MN);
+  constexpr uint32_t IDESC = make_idesc(ES == 2 ? 1 : (ES == 4 ? 2 : 0), BN, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,6 +139,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  float* xchg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + 256);   // [2][128] row partials
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -149,7 +151,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 256);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -240,8 +242,10 @@ __global__ void __launch_bounds__(192, 1)
             const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
             if constexpr (ES == 2)
               umma_f16(d_tmem, ad, bd, IDESC, accum);
-            else
+            else if constexpr (ES == 4)
               umma_tf32(d_tmem, ad, bd, IDESC, accum);
+            else
+              umma_f8(d_tmem, ad, bd, IDESC, accum);
           }
           umma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
@@ -256,7 +260,10 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     // ------------------------------------------------------------- epilogue
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int half = (warp - 2) >> 2;             // which half of the tile's columns
     const int r = quarter * 32 + lane;            // accumulator row within the tile
+    constexpr int NCH = BN / 64;                  // 32-column chunks per half
+    const int c_begin = half * NCH, c_end = c_begin + NCH;
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
       int z, mb, nb, kb0, kb1, split;
@@ -266,7 +273,7 @@ __global__ void __launch_bounds__(192, 1)
       if constexpr (EPI == EPI_ACC || EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
         // pull this row's slice of the epilogue input into L2 while the MMAs run
         const int prow = mb * 128 + r;
-        const int pcol = nb * BN;
+        const int pcol = nb * BN + half * (BN / 2);
         if (prow < p.M && pcol < p.N) {
           using PT = typename std::conditional<EPI == EPI_ACC, OutT, AuxT>::type;
           const PT* src = EPI == EPI_ACC
@@ -276,17 +283,30 @@ __global__ void __launch_bounds__(192, 1)
                                                             static_cast<long long>(prow) * p.ldo + pcol)
                               : reinterpret_cast<const PT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
                                     static_cast<long long>(prow) * p.ld_aux + pcol;
-          const uint32_t bytes = static_cast<uint32_t>(min(BN, p.N - pcol) * sizeof(PT));
+          const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, p.N - pcol) * sizeof(PT));
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
         }
       }
-      const bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
+      bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
       __syncwarp();   // tcgen05.ld is warp-collective: reconverge after the spin
+      if constexpr (EPI == EPI_QKV) {
+        // the QKV epilogue synchronises its 8 warps: make the exit decision uniform
+        uint32_t any_fail;
+        asm volatile(
+            "{\n\t.reg .pred pi, po;\n\tsetp.eq.u32 pi, %1, 0;\n\t"
+            "bar.red.or.pred po, 1, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+            : "=r"(any_fail)
+            : "r"(got ? 1u : 0u)
+            : "memory");
+        got = any_fail == 0;
+      }
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       const int row = mb * 128 + r;
       const bool row_ok = row < p.M;
+      float dqs = 1.f;   // dequantisation of fp8 operands
+      if constexpr (ES == 1) dqs = (p.dq_a ? p.dq_a[0] : 1.f) * (p.dq_b ? p.dq_b[0] : 1.f);
 
       if constexpr (EPI == EPI_QKV) {
         // BN = 128: the tile is one head of q, k or v for 128 tokens
@@ -299,38 +319,43 @@ __global__ void __launch_bounds__(192, 1)
         float v[32];
         if (which == 2) {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
+          for (int c = c_begin; c < c_end; ++c) {
             tmem_load32(tbase + c * 32, v);
+            if constexpr (ES == 1) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] *= dqs;
+            }
             if (row_ok) store_row32(dst + c * 32, v, 32);
           }
         } else {
-          float ss = 0.f;
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            tmem_load32(tbase + c * 32, v);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
-          }
-          // a rotation keeps the sum of squares, so the norm is taken before RoPE
-          const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
-          if (row_ok) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
+          // this warp owns RoPE pairs 32*half .. 32*half+31: columns 32*half + j and 64 + 32*half + j
           float w[32];
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            tmem_load32(tbase + c * 32, v);        // pair index i = 32c + j   (low half)
-            tmem_load32(tbase + 64 + c * 32, w);   // pair index i + 64       (high half)
-            const float2* cs = p.rope + static_cast<long long>(t) * 64 + c * 32;
+          tmem_load32(tbase + half * 32, v);
+          tmem_load32(tbase + 64 + half * 32, w);
+          float ss = 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float2 e = row_ok ? cs[j] : make_float2(1.f, 0.f);
-              const float lo = v[j], hi = w[j];
-              v[j] = (lo * e.x - hi * e.y) * rstd;
-              w[j] = (lo * e.y + hi * e.x) * rstd;
-            }
-            if (row_ok) {
-              store_row32(dst + c * 32, v, 32);
-              store_row32(dst + 64 + c * 32, w, 32);
-            }
+          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], fmaf(w[j], w[j], ss));
+          // a rotation keeps the sum of squares, so the norm is taken before RoPE;
+          // the two warps of a row exchange their partial sums
+          xchg[half * 128 + r] = ss;
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          ss += xchg[(half ^ 1) * 128 + r];
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          ss *= dqs * dqs;
+          const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
+          if (row_ok && half == 0) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
+          const float sc = rstd * dqs;
+          const float2* cs = p.rope + static_cast<long long>(t) * 64 + half * 32;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float2 e = row_ok ? cs[j] : make_float2(1.f, 0.f);
+            const float lo = v[j], hi = w[j];
+            v[j] = (lo * e.x - hi * e.y) * sc;
+            w[j] = (lo * e.y + hi * e.x) * sc;
+          }
+          if (row_ok) {
+            store_row32(dst + half * 32, v, 32);
+            store_row32(dst + 64 + half * 32, w, 32);
           }
         }
       } else if constexpr (EPI == EPI_LOGITS) {
@@ -340,7 +365,7 @@ __global__ void __launch_bounds__(192, 1)
         OutT* orow = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(row) * p.ldo;
         float v[32];
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = c_begin; c < c_end; ++c) {
           tmem_load32(tbase + c * 32, v);
           const int col0 = nb * BN + c * 32;
           const int nvalid = min(32, p.N - col0);
@@ -360,7 +385,9 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
         if (row_ok) {
-          reinterpret_cast<float2*>(p.f32a)[static_cast<long long>(row) * p.tiles_n + nb] = make_float2(mx, sm);
+          // one (max, sumexp) partial per half tile
+          reinterpret_cast<float2*>(p.f32a)[static_cast<long long>(row) * (2 * p.tiles_n) + 2 * nb + half] =
+              make_float2(mx, sm);
           if (have_t) p.f32b[row] = zt;
         }
       } else {
@@ -391,9 +418,9 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         };
-        prefetch(0);
+        prefetch(c_begin);
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; c += 2) {
+        for (int c = c_begin; c < c_end; c += 2) {
           uint32_t ra[32], rb[32];
           tmem_load32_async(tbase + c * 32, ra);
           tmem_load32_async(tbase + (c + 1) * 32, rb);
@@ -403,7 +430,7 @@ __global__ void __launch_bounds__(192, 1)
             const int cc = c + half;
             float v[32], a[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(half ? rb[j] : ra[j]);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(half ? rb[j] : ra[j]) * dqs;
             if constexpr (HAS_AUX) {
 #pragma unroll
               for (int g = 0; g < AUX_VEC; ++g) {
@@ -418,7 +445,7 @@ __global__ void __launch_bounds__(192, 1)
                   }
                 }
               }
-              if (cc + 1 < BN / 32) prefetch(cc + 1);
+              if (cc + 1 < c_end) prefetch(cc + 1);
             }
             const int col0 = nb * BN + cc * 32;
             const int nvalid = min(32, p.N - col0);

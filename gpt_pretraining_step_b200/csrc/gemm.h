@@ -11,7 +11,8 @@ namespace gpt {
 // D[z](m, n) = sum_k A[z](m, k) B[z](n, k), z < batch.
 //   A storage: a_mn ? [K][lda] (m contiguous) : [M][lda] (k contiguous); z stride a_bs
 //   B storage: b_mn ? [K][ldb] (n contiguous) : [N][ldb] (k contiguous); z stride b_bs
-//   es: operand element size, 2 = bf16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32)
+//   es: operand element size, 2 = bf16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32),
+//       1 = fp8 e4m3 (kind::f8f6f4; p.dq_a / p.dq_b dequantise the accumulator)
 //   out_es / aux_es: element sizes of the epilogue output and auxiliary input
 //   bn: 128 or 256 output columns per tile; splits: K split count (> 1 writes
 //   partials at out + s * split_stride); sym: only tiles on or above the

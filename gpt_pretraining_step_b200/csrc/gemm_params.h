@@ -30,6 +30,8 @@ struct GemmParams {
   void* qkv_out[3];     // QKV: q, k, v [B, H, T, 128] bf16
   void* out_t;          // STORE/AXPBY: optional transposed copy of out, [N][M] with row stride ldo_t
   long long ldo_t;
+  const float* dq_a;    // fp8 operands: device inverse scales of A and B; the accumulator is
+  const float* dq_b;    //   multiplied by dq_a[0] * dq_b[0] before the epilogue (null: 1)
   int T, H;
   int* err;
 };

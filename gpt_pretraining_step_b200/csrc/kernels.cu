@@ -2,7 +2,10 @@
 // backward, cross-entropy finish, deterministic reductions, AdamW and the
 // elementwise parts of Muon.  Rows are processed one warp per row with
 // 16-byte vector accesses; grids are sized from the row count.
+#include <cuda_fp8.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.cuh"
@@ -460,6 +463,65 @@ __global__ void muon_apply_kernel(float* __restrict__ W, bf16* __restrict__ Wb, 
   }
 }
 
+// ------------------------------------------------------- fp8 e4m3 quantisation
+//
+// Per-tensor dynamic scaling: scale = 448 / amax(|x|) of the tensor being
+// quantised, q = e4m3(x * scale) rounded to nearest even and saturated at
+// +-448, and the inverse scale amax / 448 kept for the GEMM epilogue.
+
+// amax of nmat matrices of n bf16 values each (z = blockIdx.y); the maxima of
+// non-negative floats order like their bit patterns, so an integer atomicMax
+// gives the same result in any order.  amax_bits must start at zero.
+__global__ void __launch_bounds__(256) amax_bf16_kernel(const bf16* __restrict__ x, long long n,
+                                                        unsigned int* __restrict__ amax_bits) {
+  const bf16* xz = x + blockIdx.y * n;
+  float m = 0.f;
+  const long long n8 = n / 8;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n8; i += gridDim.x * 256ll) {
+    const uint4 w = reinterpret_cast<const uint4*>(xz)[i];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) m = fmaxf(m, fmaxf(fabsf(bf16_lo(u[e])), fabsf(bf16_hi(u[e]))));
+  }
+  for (long long i = n8 * 8 + blockIdx.x * 256ll + threadIdx.x; i < n; i += gridDim.x * 256ll)
+    m = fmaxf(m, fabsf(__bfloat162float(xz[i])));
+  m = warp_max(m);
+  __shared__ float red[8];
+  if (lane_id() == 0) red[warp_id()] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = red[0];
+    for (int i = 1; i < 8; ++i) t = fmaxf(t, red[i]);
+    atomicMax(amax_bits + blockIdx.y, __float_as_uint(t));
+  }
+}
+
+__global__ void __launch_bounds__(256) quantize_e4m3_kernel(const bf16* __restrict__ x, long long n,
+                                                            const unsigned int* __restrict__ amax_bits,
+                                                            uint8_t* __restrict__ q, float* __restrict__ inv) {
+  const int z = blockIdx.y;
+  const float amax = __uint_as_float(amax_bits[z]);
+  const float sc = amax > 0.f ? 448.f / amax : 1.f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) inv[z] = amax > 0.f ? amax / 448.f : 1.f;
+  const bf16* xz = x + z * n;
+  uint8_t* qz = q + z * n;
+  const long long n8 = n / 8;
+  for (long long i = blockIdx.x * 256ll + threadIdx.x; i < n8; i += gridDim.x * 256ll) {
+    const uint4 w = reinterpret_cast<const uint4*>(xz)[i];
+    const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+    uint32_t o[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_fp8x2_storage_t pr =
+          __nv_cvt_float2_to_fp8x2(make_float2(bf16_lo(u[e]) * sc, bf16_hi(u[e]) * sc), __NV_SATFINITE, __NV_E4M3);
+      o[e >> 1] |= static_cast<uint32_t>(pr) << (16 * (e & 1));
+    }
+    reinterpret_cast<uint2*>(qz)[i] = make_uint2(o[0], o[1]);
+  }
+  for (long long i = n8 * 8 + blockIdx.x * 256ll + threadIdx.x; i < n; i += gridDim.x * 256ll)
+    qz[i] = __nv_cvt_float_to_fp8(__bfloat162float(xz[i]) * sc, __NV_SATFINITE, __NV_E4M3);
+}
+
 __global__ void cast_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long long n) {
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<long long>(gridDim.x) * blockDim.x)
@@ -581,6 +643,15 @@ void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, in
     muon_apply_kernel<bf16><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const bf16*>(X), r, c, transpose, decay, step);
   else
     muon_apply_kernel<float><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const float*>(X), r, c, transpose, decay, step);
+}
+
+void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* amax_bits, uint8_t* q, float* inv,
+                          cudaStream_t s) {
+  if (n <= 0 || nmat <= 0) return;
+  cudaMemsetAsync(amax_bits, 0, static_cast<size_t>(nmat) * sizeof(unsigned int), s);
+  const int blocks = static_cast<int>(std::min<long long>((n / 8 + 255) / 256 + 1, 4 * 148));
+  amax_bf16_kernel<<<dim3(blocks, nmat), 256, 0, s>>>(x, n, amax_bits);
+  quantize_e4m3_kernel<<<dim3(blocks, nmat), 256, 0, s>>>(x, n, amax_bits, q, inv);
 }
 
 void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s) {

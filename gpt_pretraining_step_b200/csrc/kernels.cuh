@@ -64,6 +64,12 @@ void launch_muon_make_x(const float* mom, const float* inv_norm, void* X, int ou
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
                        float lr, float wd, float scale, cudaStream_t s);
 
+// Per-tensor e4m3 quantisation of nmat matrices of n bf16 values each (z-th at
+// x + z n): q = e4m3(x * 448 / amax) with round-to-nearest-even and saturation,
+// inv[z] = amax / 448 (1 for an all-zero matrix).  amax_bits: nmat words of scratch.
+void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* amax_bits, uint8_t* q, float* inv,
+                          cudaStream_t s);
+
 // dst = bf16(src), n elements.
 void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s);
 

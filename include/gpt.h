@@ -67,7 +67,10 @@ enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
  *   vocab     vocabulary size, a multiple of 8 (32768 in the pages' runs)
  *   batch     sequences per step; seq_len tokens each
  *   head_dim  must be 128; mlp_mult must be 4
- *   precision 0 = bf16 GEMMs (the only value accepted by this version)
+ *   precision 0 = bf16 GEMMs; 1 = the four block projections of the forward
+ *             pass (q|k|v, attention output, MLP up, MLP down) on fp8 e4m3
+ *             operands with dynamic per-tensor scales (448 / amax of the
+ *             tensor); attention, lm_head and the backward stay bf16
  *   ns_tf32_steps  how many of the five Newton-Schulz steps run with fp32
  *             operands on the tensor cores (kind::tf32) before switching
  *             to bf16; 0..5.  Three keep the update within 1% of fp64 on
@@ -174,6 +177,7 @@ enum {
   GPT_PROF_NS_GEMM,       /* Newton-Schulz GEMMs */
   GPT_PROF_MUON_ELEM,     /* Muon momentum, norms, normalise, apply */
   GPT_PROF_ADAMW,         /* AdamW */
+  GPT_PROF_FP8_QUANT,     /* fp8 amax and e4m3 quantisation (precision 1) */
   GPT_PROF_COUNT
 };
 
@@ -214,6 +218,20 @@ int gpt_op_matmul_bf16(const void* A, const void* B, float* C, int M, int N, int
  * K-major), C [M, N] fp32.  K a multiple of 4, N of 8.  b_trans = 0 is
  * GPT_EINVAL. */
 int gpt_op_matmul_tf32(const float* A, const float* B, float* C, int M, int N, int K, int b_trans, void* stream);
+
+/* Per-tensor e4m3 quantisation ("3. Gestión de Precisión": FP8 training with
+ * per-tensor scaling): q = e4m3(x * 448 / amax|x|), round to nearest even,
+ * saturating at +-448; *inv = amax / 448 (1 if x is all zero).
+ *   x: n bf16 values (16-byte aligned); q: n bytes (8-byte aligned);
+ *   amax_scratch: one device word. */
+int gpt_op_quantize_e4m3(const void* x, long long n, void* q, float* inv, unsigned int* amax_scratch, void* stream);
+
+/* C = (A * B) * inv_a * inv_b on e4m3 operands (tcgen05 kind::f8f6f4), fp32
+ * accumulation.  A [M, K] row-major bytes; B [K, N] row-major, or [N, K] with
+ * b_trans = 1; inv_a, inv_b: device inverse scales; C [M, N] fp32.
+ * N and K multiples of 16. */
+int gpt_op_matmul_fp8(const void* A, const void* B, float* C, int M, int N, int K, const float* inv_a,
+                      const float* inv_b, int b_trans, void* stream);
 
 /* Causal attention forward: q, k, v bf16 [B, H, T, 128] -> o bf16 [B, T, H, 128]
  * and lse fp32 [B, H, T] (natural log of the softmax denominator of

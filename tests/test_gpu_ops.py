@@ -155,3 +155,39 @@ def test_newton_schulz(torch, batch, rows, cols, tf32_steps):
         ref = oo.newton_schulz(G[z].astype(np.float64))
         err = relfro(got[z], ref)
         assert err < (2e-2 if tf32_steps < 5 else 1e-2), (z, err)
+
+
+def test_quantize_e4m3_bit_exact(torch):
+    # the scale 448 / amax and the product x * scale are formed in fp32 on both
+    # sides (the decision precision of the kernel); the rounding to the e4m3 grid
+    # is the oracle's
+    import gpt_pretraining_step_b200 as g
+    from oracle import fp8 as of
+    x = syn.round_to_bf16(np.concatenate([syn.gaussian(40000, seed=21) * 3.0,
+                                          syn.gaussian(1000, seed=22) * 1e-3, [0.0, -7.5]]).astype(np.float32))
+    q, inv = g.quantize_e4m3(bf16_t(torch, x))
+    torch.cuda.synchronize()
+    amax = np.float32(np.abs(x).max())
+    sc = np.float32(448.0) / amax
+    want = of.round_e4m3((x * sc).astype(np.float32).astype(np.float64))
+    got = q.view(torch.float8_e4m3fn).float().cpu().numpy().astype(np.float64)
+    assert np.array_equal(got, want)
+    assert float(inv.item()) == float(amax / np.float32(448.0))
+
+
+@pytest.mark.parametrize("b_trans", [0, 1])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (200, 272, 160)])
+def test_matmul_fp8(torch, b_trans, M, N, K):
+    import gpt_pretraining_step_b200 as g
+    from oracle import fp8 as of
+    qa = of.round_e4m3(syn.gaussian((M, K), seed=M + K) * 100)
+    qb = of.round_e4m3(syn.gaussian((K, N), seed=N + K) * 100)
+    ta = torch.tensor(qa, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).cuda()
+    bs = qb.T.copy() if b_trans else qb
+    tb = torch.tensor(bs, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).cuda()
+    inv_a = torch.tensor([0.5], dtype=torch.float32).cuda()
+    inv_b = torch.tensor([0.125], dtype=torch.float32).cuda()
+    C = g.matmul_fp8(ta, tb, M, N, K, inv_a, inv_b, b_trans=bool(b_trans))
+    torch.cuda.synchronize()
+    ref = (qa @ qb) * 0.5 * 0.125
+    assert relfro(f64(C), ref) < 1e-6

@@ -340,3 +340,48 @@ def test_d20_muon_sampled_matrices(d20, torch):
         W_ref, _ = oo.muon_step(W0[tid], Gs[tid], np.zeros_like(W0[tid]), 0.02, 0.95, 0.0)
         W_got = f64(st.get(tid, g.KIND_PARAM))
         assert relfro(W_got - W0[tid], W_ref - W0[tid]) <= MUON_RELFRO, specs[tid][0]
+
+
+# ----------------------------------------------------------------- fp8 e4m3
+
+FP8_LOSS_RTOL = 3e-2
+FP8_GRAD_COS = 0.99
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_fp8_step_matches_oracle(torch, name):
+    # the four block projections of the forward on e4m3 operands with dynamic
+    # per-tensor scales, against the fp64 oracle at the fp8 tolerances
+    import gpt_pretraining_step_b200 as g
+    s = SMALL[name]
+    params = syn.init_params(s, seed=0)
+    tok, tgt = syn.tokens(s), syn.targets(s)
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model, precision=1)
+    for tid, (pname, *_r) in enumerate(syn.param_specs(s)):
+        st.set(tid, params[pname])
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    loss_ref, grads, _ = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= FP8_LOSS_RTOL
+    for tid, (pname, *_r) in enumerate(syn.param_specs(s)):
+        c = cosine(f64(st.get(tid, g.KIND_GRAD)), grads[pname])
+        assert c >= FP8_GRAD_COS, (pname, c)
+    st.muon_step(0.02, 0.95, 0.0)
+    st.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.0)
+    st.check()
+
+
+def test_d26_fp8_initial_loss(torch):
+    # the d26 configuration with fp8 projections: the initial loss keeps the
+    # Gaussian closed form within the fp8 tolerance
+    import gpt_pretraining_step_b200 as g
+    s = syn.config_shape("d26")
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, precision=1)
+    tok, tgt = syn.tokens(s), syn.targets(s)
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.muon_step(0.02, 0.95, 0.0)
+    st.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.0)
+    st.check()
+    sig2 = 0.02 ** 2 * s.d_model
+    expect = math.log(s.vocab) + sig2 / 2 - (math.exp(sig2) - 1) / (2 * s.vocab)
+    assert abs(loss - expect) / expect <= FP8_LOSS_RTOL
