@@ -73,7 +73,8 @@ bool make_map_4d(CUtensorMap* m, const void* ptr, const long long (&dims)[4], co
 namespace {
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParams& p, cudaStream_t s) {
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmParams& p,
+                   cudaStream_t s) {
   using C = GemmCfg<sizeof(T), BN>;
   auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT>;
   static bool configured = false;
@@ -83,7 +84,7 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const GemmParam
     configured = true;
   }
   const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
-  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, p);
+  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, p);
   return cudaGetLastError();
 }
 
@@ -146,10 +147,25 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
     ok = make_map(&mb, c.B, c.es, c.N, c.K, c.batch, c.ldb, c.b_bs, mn_box, bk);
   if (!ok) return cudaErrorInvalidValue;
 
+  // Output written by TMA stores of 32-row x 128-byte boxes when the output's
+  // base and strides are 16-byte aligned; otherwise by per-thread stores.
+  // The map's third dimension is the batch index, or the K split of a
+  // split-K partial (never both).
+  CUtensorMap mc;
+  p.tma_out = 0;
+  if (c.epi != EPI_QKV && !(c.batch > 1 && p.splits > 1) && (c.out_es == 2 || c.out_es == 4)) {
+    const long long n3 = p.splits > 1 ? p.splits : c.batch;
+    const long long s3 = p.splits > 1 ? p.split_stride : p.out_bs;
+    if (make_map(&mc, p.out, c.out_es, c.N, c.M, n3, p.ldo, s3, 128 / c.out_es, 32)) p.tma_out = 1;
+  }
+  // fp32 accumulation (out += acc) is done by TMA add-reduction only
+  if (c.epi == EPI_ACC && !p.tma_out) return cudaErrorInvalidValue;
+  if (!p.tma_out) mc = ma;   // unused by the kernel
+
 #define GPT_GEMM_CASE(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                       \
   if (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ && \
       c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_))                               \
-    return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, p, stream);
+    return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, mc, p, stream);
 
   // forward
   GPT_GEMM_CASE(bf16, 128, false, true, EPI_QKV, bf16, bf16)

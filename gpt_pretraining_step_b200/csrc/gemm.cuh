@@ -30,7 +30,9 @@ struct GemmCfg {
   static constexpr int STAGES = BN == 256 ? 4 : 6;
   static constexpr int CHUNK_BYTES = BK * 128;        // one MN-major box: BK rows of 128 B
   static constexpr int TMEM_COLS = 2 * BN;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + 256 + 1024;   // + epilogue exchange
+  // output staging: one 32-row x 128-byte box per epilogue warp
+  static constexpr int STG_BYTES = 8 * 4096;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + 1024 + 256 + 1024;   // + epilogue exchange
 };
 
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
@@ -120,26 +122,52 @@ __device__ __forceinline__ void store_scalar(OutT* dst, float x) {
     *reinterpret_cast<float*>(dst) = x;
 }
 
+// Online (max, sum of exp) of one row's 32-column logits chunk starting at
+// column col0 (columns >= n are ignored), and the target's logit if it falls
+// in the chunk.
+__device__ __forceinline__ void logits_chunk(const float (&v)[32], int col0, int n, int tg, float& mx, float& sm,
+                                             float& zt, bool& have_t) {
+  const int nvalid = min(32, n - col0);
+  if (nvalid <= 0) return;
+  float cm = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) if (j < nvalid) cm = fmaxf(cm, v[j]);
+  if (cm > mx) { sm *= __expf(mx - cm); mx = cm; }
+#pragma unroll
+  for (int j = 0; j < 32; ++j) if (j < nvalid) sm += __expf(v[j] - mx);
+  if (tg >= col0 && tg < col0 + 32) {
+    // select without an indexed access, which would move v to local memory
+    const int idx = tg - col0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+      asm("{\n\t.reg .pred q;\n\tsetp.eq.s32 q, %2, %3;\n\tselp.f32 %0, %1, %0, q;\n\t}"
+          : "+f"(zt)
+          : "f"(v[j]), "r"(j), "r"(idx));
+    have_t = true;
+  }
+}
+
 // ------------------------------------------------------------------ kernel
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ GemmParams p) {
   constexpr int ES = sizeof(T);
   using C = GemmCfg<ES, BN>;
   constexpr uint32_t IDESC = make_idesc(ES == 2 ? 1 : (ES == 4 ? 2 : 0), BN, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t* stg_base = smem + C::STAGES * C::STAGE_BYTES;   // 1024-aligned output staging
+  uint64_t* full = reinterpret_cast<uint64_t*>(stg_base + C::STG_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* xchg = reinterpret_cast<float*>(smem + C::STAGES * C::STAGE_BYTES + 256);   // [2][128] row partials
+  float* xchg = reinterpret_cast<float*>(stg_base + C::STG_BYTES + 256);   // [2][128] row partials
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -158,6 +186,7 @@ __global__ void __launch_bounds__(320, 1)
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (p.tma_out) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -264,26 +293,71 @@ __global__ void __launch_bounds__(320, 1)
     const int r = quarter * 32 + lane;            // accumulator row within the tile
     constexpr int NCH = BN / 64;                  // 32-column chunks per half
     const int c_begin = half * NCH, c_end = c_begin + NCH;
+    // This warp's output box: 32 rows x 128 bytes (32 fp32 or 64 bf16 columns),
+    // laid out with the 128-byte swizzle of the output tensor map: 16-byte unit
+    // u of box row i sits at unit u ^ (i & 7).  Lane i owns box row i.
+    uint8_t* stg = stg_base + (warp - 2) * 4096;
+    uint8_t* stg_row = stg + lane * 128;
+    const int stg_sw = lane & 7;
+    auto box_open = [&]() {
+      if (lane == 0) bulk_wait_read_all();   // the previous box has been read by TMA
+      __syncwarp();
+    };
+    auto box_put = [&](int u, uint4 w) { *reinterpret_cast<uint4*>(stg_row + ((u ^ stg_sw) << 4)) = w; };
+    auto box_close = [&](int col0, int row0, int z3) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0 && row0 < p.M && col0 < p.N) {
+        if constexpr (EPI == EPI_ACC)
+          tma_reduce_add_3d(&tmC, stg, col0, row0, z3);
+        else
+          tma_store_3d(&tmC, stg, col0, row0, z3);
+        bulk_commit();
+      }
+    };
+    // 64 accumulator columns (two 32-column halves) to boxes: one bf16 box or two fp32 boxes
+    auto emit64 = [&](const float (&v0)[32], const float (&v1)[32], int col0, int row0, int z3) {
+      if constexpr (sizeof(OutT) == 2) {
+        box_open();
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          box_put(u, make_uint4(pack_bf16x2(v0[8 * u], v0[8 * u + 1]), pack_bf16x2(v0[8 * u + 2], v0[8 * u + 3]),
+                                pack_bf16x2(v0[8 * u + 4], v0[8 * u + 5]), pack_bf16x2(v0[8 * u + 6], v0[8 * u + 7])));
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          box_put(4 + u, make_uint4(pack_bf16x2(v1[8 * u], v1[8 * u + 1]), pack_bf16x2(v1[8 * u + 2], v1[8 * u + 3]),
+                                    pack_bf16x2(v1[8 * u + 4], v1[8 * u + 5]),
+                                    pack_bf16x2(v1[8 * u + 6], v1[8 * u + 7])));
+        box_close(col0, row0, z3);
+      } else {
+        box_open();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          box_put(u, make_uint4(__float_as_uint(v0[4 * u]), __float_as_uint(v0[4 * u + 1]),
+                                __float_as_uint(v0[4 * u + 2]), __float_as_uint(v0[4 * u + 3])));
+        box_close(col0, row0, z3);
+        box_open();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          box_put(u, make_uint4(__float_as_uint(v1[4 * u]), __float_as_uint(v1[4 * u + 1]),
+                                __float_as_uint(v1[4 * u + 2]), __float_as_uint(v1[4 * u + 3])));
+        box_close(col0 + 32, row0, z3);
+      }
+    };
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
       int z, mb, nb, kb0, kb1, split;
       decode_unit(p, u, z, mb, nb, kb0, kb1, split);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
-      if constexpr (EPI == EPI_ACC || EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
+      if constexpr (EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
         // pull this row's slice of the epilogue input into L2 while the MMAs run
         const int prow = mb * 128 + r;
         const int pcol = nb * BN + half * (BN / 2);
         if (prow < p.M && pcol < p.N) {
-          using PT = typename std::conditional<EPI == EPI_ACC, OutT, AuxT>::type;
-          const PT* src = EPI == EPI_ACC
-                              ? reinterpret_cast<const PT*>(reinterpret_cast<const OutT*>(p.out) +
-                                                            static_cast<long long>(z) * p.out_bs +
-                                                            static_cast<long long>(split) * p.split_stride +
-                                                            static_cast<long long>(prow) * p.ldo + pcol)
-                              : reinterpret_cast<const PT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
-                                    static_cast<long long>(prow) * p.ld_aux + pcol;
-          const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, p.N - pcol) * sizeof(PT));
+          const AuxT* src = reinterpret_cast<const AuxT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
+                            static_cast<long long>(prow) * p.ld_aux + pcol;
+          const uint32_t bytes = static_cast<uint32_t>(min(BN / 2, p.N - pcol) * sizeof(AuxT));
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
         }
       }
@@ -305,9 +379,10 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
       const int row = mb * 128 + r;
       const bool row_ok = row < p.M;
+      const int box_row0 = mb * 128 + quarter * 32;
+      const int z3 = p.splits > 1 ? split : z;   // third coordinate of the output map
       float dqs = 1.f;   // dequantisation of fp8 operands
       if constexpr (ES == 1) dqs = (p.dq_a ? p.dq_a[0] : 1.f) * (p.dq_b ? p.dq_b[0] : 1.f);
-
       if constexpr (EPI == EPI_QKV) {
         // BN = 128: the tile is one head of q, k or v for 128 tokens
         const int which = nb / p.H;
@@ -363,26 +438,25 @@ __global__ void __launch_bounds__(320, 1)
         bool have_t = false;
         const int tg = row_ok ? p.tgt[row] : -1;
         OutT* orow = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(row) * p.ldo;
-        float v[32];
 #pragma unroll 1
-        for (int c = c_begin; c < c_end; ++c) {
-          tmem_load32(tbase + c * 32, v);
-          const int col0 = nb * BN + c * 32;
-          const int nvalid = min(32, p.N - col0);
-          if (nvalid > 0) {
-            float cm = -INFINITY;
+        for (int c = c_begin; c < c_end; c += 2) {
+          uint32_t ra[32], rb[32];
+          tmem_load32_async(tbase + c * 32, ra);
+          tmem_load32_async(tbase + (c + 1) * 32, rb);
+          tmem_wait_ld();
+          float v0[32], v1[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) if (j < nvalid) cm = fmaxf(cm, v[j]);
-            if (cm > mx) { sm *= __expf(mx - cm); mx = cm; }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) if (j < nvalid) sm += __expf(v[j] - mx);
-            if (tg >= col0 && tg < col0 + 32) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) if (j == tg - col0) zt = v[j];
-              have_t = true;
-            }
-            if (row_ok) store_row32(orow + col0, v, nvalid);
+          for (int j = 0; j < 32; ++j) {
+            v0[j] = __uint_as_float(ra[j]);
+            v1[j] = __uint_as_float(rb[j]);
           }
+          auto stats = [&](const float (&v)[32], int col0) {
+            logits_chunk(v, col0, p.N, tg, mx, sm, zt, have_t);
+            if (!p.tma_out && row_ok && col0 < p.N) store_row32(orow + col0, v, min(32, p.N - col0));
+          };
+          stats(v0, nb * BN + c * 32);
+          stats(v1, nb * BN + c * 32 + 32);
+          if (p.tma_out) emit64(v0, v1, nb * BN + c * 32, box_row0, 0);
         }
         if (row_ok) {
           // one (max, sumexp) partial per half tile
@@ -394,14 +468,13 @@ __global__ void __launch_bounds__(320, 1)
         OutT* obase = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(z) * p.out_bs +
                       static_cast<long long>(split) * p.split_stride;
         const bool mirror = p.sym && nb != mb;
-        // Auxiliary input of the epilogue (the fp32 output itself for EPI_ACC),
-        // prefetched one 32-column chunk ahead to hide its global-load latency.
-        constexpr bool HAS_AUX = EPI == EPI_ACC || EPI == EPI_DRELU2 || EPI == EPI_AXPBY;
-        using AT = typename std::conditional<EPI == EPI_ACC, OutT, AuxT>::type;
+        // Auxiliary input of the epilogue, prefetched one 32-column chunk ahead to
+        // hide its load latency.  (EPI_ACC adds into the output by TMA
+        // add-reduction and reads nothing.)
+        constexpr bool HAS_AUX = EPI == EPI_DRELU2 || EPI == EPI_AXPBY;
+        using AT = AuxT;
         const AT* abase = nullptr;
-        if constexpr (EPI == EPI_ACC)
-          abase = reinterpret_cast<const AT*>(obase) + static_cast<long long>(row) * p.ldo;
-        else if constexpr (HAS_AUX)
+        if constexpr (HAS_AUX)
           abase = reinterpret_cast<const AT*>(p.aux) + static_cast<long long>(z) * p.aux_bs +
                   static_cast<long long>(row) * p.ld_aux;
         constexpr int AUX_VEC = HAS_AUX ? (32 * static_cast<int>(sizeof(AT))) / 16 : 1;   // uint4 per chunk
@@ -425,12 +498,13 @@ __global__ void __launch_bounds__(320, 1)
           tmem_load32_async(tbase + c * 32, ra);
           tmem_load32_async(tbase + (c + 1) * 32, rb);
           tmem_wait_ld();
+          float v[2][32];
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int cc = c + half;
-            float v[32], a[32];
+          for (int hh = 0; hh < 2; ++hh) {
+            const int cc = c + hh;
+            float a[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(half ? rb[j] : ra[j]) * dqs;
+            for (int j = 0; j < 32; ++j) v[hh][j] = __uint_as_float(hh ? rb[j] : ra[j]) * dqs;
             if constexpr (HAS_AUX) {
 #pragma unroll
               for (int g = 0; g < AUX_VEC; ++g) {
@@ -447,16 +521,9 @@ __global__ void __launch_bounds__(320, 1)
               }
               if (cc + 1 < c_end) prefetch(cc + 1);
             }
-            const int col0 = nb * BN + cc * 32;
-            const int nvalid = min(32, p.N - col0);
-            if (!row_ok || nvalid <= 0) continue;
-            OutT* dst = obase + static_cast<long long>(row) * p.ldo + col0;
-            if constexpr (EPI == EPI_ACC) {
+            if constexpr (EPI == EPI_RELU2) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] += a[j];
-            } else if constexpr (EPI == EPI_RELU2) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) { const float t = fmaxf(v[j], 0.f); v[j] = t * t; }
+              for (int j = 0; j < 32; ++j) { const float t = fmaxf(v[hh][j], 0.f); v[hh][j] = t * t; }
             } else if constexpr (EPI == EPI_DRELU2) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -464,24 +531,31 @@ __global__ void __launch_bounds__(320, 1)
                 // the IEEE sqrt takes its slow path, so use the single-instruction form
                 float rt;
                 asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(a[j]));
-                v[j] *= 2.f * rt;
+                v[hh][j] *= 2.f * rt;
               }
             } else if constexpr (EPI == EPI_AXPBY) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = p.alpha * a[j] + p.beta * v[j];
+              for (int j = 0; j < 32; ++j) v[hh][j] = p.alpha * a[j] + p.beta * v[hh][j];
             }
-            store_row32(dst, v, nvalid);
+          }
+          if (p.tma_out) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int col0 = nb * BN + (c + hh) * 32;
+            const int nvalid = min(32, p.N - col0);
+            if (!row_ok || nvalid <= 0) continue;
+            if (!p.tma_out) store_row32(obase + static_cast<long long>(row) * p.ldo + col0, v[hh], nvalid);
             if (p.out_t) {
               OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[j]);
+                if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[hh][j]);
             }
             if (mirror) {
               // the transposed tile of a symmetric product: lanes write consecutive columns
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[j]);
+                if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
             }
           }
         }
@@ -491,6 +565,7 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
 
+  if (warp >= 2 && lane == 0) bulk_wait_all();   // output boxes written before the CTA exits
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -33,6 +33,7 @@ struct GemmParams {
   const float* dq_a;    // fp8 operands: device inverse scales of A and B; the accumulator is
   const float* dq_b;    //   multiplied by dq_a[0] * dq_b[0] before the epilogue (null: 1)
   int T, H;
+  int tma_out;          // 1: the main output is written by TMA stores through the output tensor map
   int* err;
 };
 
