@@ -66,10 +66,12 @@ def peaks():
 
 # ------------------------------------------------------------------ FLOPs
 
-def model_flops_per_token(s):
-    """PaLM-style model FLOPs per token: 6 N_matmul + 12 L d T (embeddings excluded)."""
+def model_flops_per_token(s, causal=False):
+    """PaLM-style model FLOPs per token: 6 N_matmul + 12 L d T (embeddings
+    excluded); with causal=True the attention term counts only the half of the
+    score matrix that the causal mask keeps (6 L d T)."""
     n_matmul = s.depth * 12 * s.d_model ** 2 + s.d_model * s.vocab
-    return 6 * n_matmul + 12 * s.depth * s.d_model * s.seq_len
+    return 6 * n_matmul + (6 if causal else 12) * s.depth * s.d_model * s.seq_len
 
 
 def category_work(s):
@@ -303,6 +305,7 @@ def run_ours(a):
     fpt = model_flops_per_token(s)
     mfu_sust = fpt * s.tokens / (ms / 1e3) / (pk["bf16_tflops_sustained"] * 1e12)
     mfu_nominal = fpt * s.tokens / (ms / 1e3) / 2.25e15
+    mfu_causal = model_flops_per_token(s, causal=True) * s.tokens / (ms / 1e3) / (pk["bf16_tflops_sustained"] * 1e12)
 
     roof = None
     if dominant and dominant in live and live[dominant][1]:
@@ -333,6 +336,14 @@ def run_ours(a):
                     e["gbs"] = round(amount / (tms / 1e3) / 1e9, 1)
             breakdown[c] = e
 
+    # device time of the optimizer calls (Newton-Schulz, Muon elementwise, AdamW)
+    # against the rest of the step
+    opt_ms = sum(prof.get(c, (0.0, 0))[0] for c in ("ns_gemm", "muon_elem", "adamw"))
+    split = {"optimizer_ms": round(opt_ms, 3), "fwd_bwd_ms": round(ms - opt_ms, 3)} if prof else None
+    if split and a.precision == "fp8":
+        # against the fp8 dense peak (twice the measured bf16 figure, the nominal ratio)
+        split["mfu_vs_fp8_peak"] = mfu_sust / 2
+
     e2e = None
     if not a.no_e2e:
         e2e = run_e2e(a, st, s, rank, world, grads, stream)
@@ -358,10 +369,12 @@ def run_ours(a):
             "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
             "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",
             "model_tflop_per_step": fpt * s.tokens / 1e12,
+            "mfu_attention_causal_half": mfu_causal,
             "loss": loss, "clocks": clocks, "gpu_launches": launches, "roofline": roof, "cpu_baseline": cpu,
             "e2e": None if e2e is None else {k: e2e[k] for k in ("value", "unit", "h2d_bytes_per_step",
                                                                  "d2h_bytes_per_step")},
             "breakdown_ms_per_step_category": breakdown,
+            "step_split": split,
         }
         print(json.dumps(out), flush=True)
     if world > 1:

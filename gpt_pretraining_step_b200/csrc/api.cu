@@ -188,7 +188,7 @@ void make_plan(const Dims& D, Plan& P) {
   P.Bbuf = ab.take(2 * L * d * d * 4);
   P.inv_norm = ab.take(4 * L * 4);
   P.normws = ab.take(muon_norm_workspace(4 * D.L));
-  P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8);
+  P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
   P.tok = ab.take(M * 4);
   P.tgt = ab.take(M * 4);
@@ -443,11 +443,11 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.b_mn = true; g.ldb = 3 * d;
       fwd_a(g, xn1l, M, d, 2, l); g.lda = d;
       ProfScope ps(c, GPT_PROF_QKV_GEMM);
-      g.bn = 128; g.epi = EPI_QKV; g.out_es = 2; g.aux_es = 2;
+      g.bn = 256; g.epi = EPI_QKV; g.out_es = 2; g.aux_es = 2;
       g.p.qkv_out[0] = ql; g.p.qkv_out[1] = kl; g.p.qkv_out[2] = vl;
       g.p.f32a = rq + static_cast<size_t>(l) * M * H;
       g.p.f32b = rk + static_cast<size_t>(l) * M * H;
-      g.p.rope = rope; g.p.T = D.T; g.p.H = H; g.p.err = err;
+      g.p.rope = rope + static_cast<size_t>(D.T) * 64; g.p.T = D.T; g.p.H = H; g.p.err = err;
       GPT_CK(gemm_run(g, s));
     }
     {

@@ -336,18 +336,22 @@ __global__ void __launch_bounds__(192, 1)
 // ------------------------------------------------ backward on tcgen05 / TMEM
 //
 // One CTA per (128-key block j, batch*head), looping over the query blocks
-// i >= j that see those keys.  192 threads:
+// i >= j that see those keys.  320 threads:
 //   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i
 //   warp 1      TMEM owner and MMA issuer, per query block:
 //                 S^T = K Q^T and dP^T = V dO^T          (TMEM cols 0 and 128)
-//                 dV += P^T dO, dK += dS^T Q              (TMEM cols 256, 384)
+//                 dV += P^T dO (after which dO_{i+1} may load), dK += dS^T Q
+//                                                         (TMEM cols 256, 384)
 //                 dQ_i = dS K into cols 0 (S^T is consumed by then)
 //   warps 2..9  two warps per TMEM lane quarter, each on half of the 128
 //               columns: P^T = exp(S^T/sqrt(d) - lse), dS^T = P^T (dP^T - D)
-//               / sqrt(d) as bf16 tiles in shared memory (the dS^T tile is also
-//               the MN-major A operand of dS K); then dQ_i is staged through
-//               the two (by then idle) tiles as fp32 in TMA's 128-byte-swizzled
-//               layout and added into the fp32 dq buffer by TMA bulk reduce-add;
+//               as bf16 tiles in shared memory (the dS^T tile is also the
+//               MN-major A operand of dS K; 1/sqrt(d) is applied to dK and dQ
+//               instead); then each warp stages its rows of dQ_i as fp32 in the
+//               parts of the two (by then idle) tiles that it writes itself and
+//               adds them into the fp32 dq buffer by TMA reduce-add (their read
+//               is awaited just before the warp's next tile stores, so it
+//               overlaps the next S^T / dP^T products and softmax);
 //               finally dK and dV of the block to global memory.
 
 constexpr int TB_SMEM = 7 * TF_BUF + 1024 + 1024 + 512;
@@ -480,15 +484,22 @@ __global__ void __launch_bounds__(320, 1)
         umma_commit(sd_full);
         if (!mbar_wait(p_full, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
+        // dV first: once it completes, dO_i is no longer read and the next
+        // block's dO can be loaded while dK and dQ run
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;   // K-major A: 16 queries per step
           const uint32_t boff = kk * 2048;                              // MN-major B: 16 query rows per step
-          const uint32_t accum = (it > 0 || kk > 0) ? 1u : 0u;
           umma_f16(tmem + 256, smem_desc_sw128(pt_addr + aoff, 16, 1024),
-                   smem_desc_sw128(do_addr + boff, TF_TILE, 1024), IDESC_KM, accum);
+                   smem_desc_sw128(do_addr + boff, TF_TILE, 1024), IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(do_empty);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          const uint32_t boff = kk * 2048;
           umma_f16(tmem + 384, smem_desc_sw128(dst_addr + aoff, 16, 1024),
-                   smem_desc_sw128(q_addr + boff, TF_TILE, 1024), IDESC_KM, accum);
+                   smem_desc_sw128(q_addr + boff, TF_TILE, 1024), IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -498,7 +509,6 @@ __global__ void __launch_bounds__(320, 1)
         }
         umma_commit(mm_done);
         umma_commit(&q_empty[s]);
-        umma_commit(do_empty);
       }
       umma_commit(drain);
       for (uint32_t x = 0; x < (1u << 22) && !mbar_try_wait(drain, 0); ++x) {}
@@ -514,34 +524,47 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float scale_log2 = scale * 1.4426950408889634f;
     bool ok = true;
-    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
-      const bool got = mbar_wait(bar, par, abort_flag, err);
+    // Named barrier 1 over the 256 softmax threads, which also tells every
+    // thread whether any of them failed its wait (so all leave the loop together)
+    auto any_fail = [&](bool got) -> bool {
       __syncwarp();
-      return __all_sync(0xffffffffu, got);
+      uint32_t f;
+      asm volatile(
+          "{\n\t.reg .pred pi, po;\n\tsetp.eq.u32 pi, %1, 0;\n\t"
+          "bar.red.or.pred po, 1, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+          : "=r"(f)
+          : "r"(got ? 1u : 0u)
+          : "memory");
+      return f != 0;
     };
-    // this thread's share of the query block's lse (log2 units; +inf past T so P = 0)
-    // or D, fetched one block ahead so the load latency hides behind a whole block
+    // this thread's share of the query block's -lse (log2 units; -inf past T so
+    // P = 0) or -D, fetched ahead so the load latency hides behind a whole block
     auto fetch = [&](int it2) -> float {
       const int q0f = (j + it2) * 128;
       if (t256 < 128) {
         const int qq = q0f + t256;
-        return qq < T ? __ldg(lse + static_cast<long long>(bh) * T + qq) * 1.4426950408889634f : INFINITY;
+        return qq < T ? __ldg(lse + static_cast<long long>(bh) * T + qq) * -1.4426950408889634f : -INFINITY;
       }
       const int qq = q0f + t256 - 128;
-      return qq < T ? __ldg(Dv + static_cast<long long>(bh) * T + qq) : 0.f;
+      return qq < T ? -__ldg(Dv + static_cast<long long>(bh) * T + qq) : 0.f;
     };
-    float staged = n_it > 0 ? fetch(0) : 0.f;
+    // lse/D of block it are written after the barrier that ends block it-1's
+    // softmax and published by the barrier at the top of block it
+    auto publish = [&](float x) {
+      if (t256 < 128) lse_s[t256] = x;
+      else dd_s[t256 - 128] = x;
+    };
+    if (n_it > 0) publish(fetch(0));
+    float staged = n_it > 1 ? fetch(1) : 0.f;
     for (int it = 0; it < n_it && ok; ++it) {
       const int i = j + it;
       const int q0 = i * 128;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (t256 < 128) lse_s[t256] = staged;
-      else dd_s[t256 - 128] = staged;
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (it + 1 < n_it) staged = fetch(it + 1);
-      if (!wait_all(sd_full, it & 1)) { ok = false; break; }
+      const bool got = mbar_wait(sd_full, it & 1, abort_flag, err);
+      if (any_fail(got)) { ok = false; break; }   // also publishes lse/D of the block
       tc_fence_after();
       const bool diag = i == j;
+      const bool masked = diag || k0 + 128 > T;   // causal diagonal block or ragged key block
+      const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
 #pragma unroll 1
       for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t sr[32], dr[32];
@@ -550,23 +573,51 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         uint32_t pk[16], dk2[16];
 #pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
-          const float4 d4 = *reinterpret_cast<const float4*>(dd_s + c * 32 + k);
-          const float la[4] = {l4.x, l4.y, l4.z, l4.w};
-          const float da[4] = {d4.x, d4.y, d4.z, d4.w};
-          float pv[4], dsv[4];
+        for (int k = 0; k < 32; k += 8) {
+          const float4 la = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
+          const float4 lb = *reinterpret_cast<const float4*>(lse_s + c * 32 + k + 4);
+          const float4 da = *reinterpret_cast<const float4*>(dd_s + c * 32 + k);
+          const float4 db = *reinterpret_cast<const float4*>(dd_s + c * 32 + k + 4);
+          const float nl[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};   // -lse * log2(e)
+          const float nd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};   // -D
+          // P = 2^(S * scale * log2(e) - lse * log2(e)): six of every eight on the
+          // MUFU unit, two by the polynomial on the FMA pipe (the two units then
+          // finish together)
+          float p[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float p = ex2_approx(fmaf(__uint_as_float(sr[k + e]), scale_log2, -la[e]));
-            if (!key_ok || (diag && key > q0 + c * 32 + k + e)) p = 0.f;
-            pv[e] = p;
-            dsv[e] = p * (__uint_as_float(dr[k + e]) - da[e]) * scale;
+          for (int e = 0; e < 8; e += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[k + e]), __uint_as_float(sr[k + e + 1])), sl2,
+                             f2_pack(nl[e], nl[e + 1])),
+                      x0, x1);
+            if (e < 6) {
+              p[e] = ex2_approx(x0);
+              p[e + 1] = ex2_approx(x1);
+            } else {
+              f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+            }
           }
-          pk[k >> 1] = pack_bf16x2(pv[0], pv[1]);
-          pk[(k >> 1) + 1] = pack_bf16x2(pv[2], pv[3]);
-          dk2[k >> 1] = pack_bf16x2(dsv[0], dsv[1]);
-          dk2[(k >> 1) + 1] = pack_bf16x2(dsv[2], dsv[3]);
+          if (masked) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (!key_ok || (diag && key > q0 + c * 32 + k + e)) p[e] = 0.f;
+          }
+          // dS' = P (dP - D); the 1/sqrt(d) of dS = dS' / sqrt(d) is applied to dK and dQ
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            float d0, d1;
+            f2_unpack(f2_mul(f2_pack(p[e], p[e + 1]),
+                             f2_add(f2_pack(__uint_as_float(dr[k + e]), __uint_as_float(dr[k + e + 1])),
+                                    f2_pack(nd[e], nd[e + 1]))),
+                      d0, d1);
+            pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+            dk2[(k + e) >> 1] = pack_bf16x2(d0, d1);
+          }
+        }
+        if (c == 2 * half) {
+          // this warp's rows of the tiles held its previous dQ boxes: TMA has read them
+          if (lane == 0) bulk_wait_read_all();
+          __syncwarp();
         }
         const int rowoff = (c >> 1) * TF_TILE + r * 128;
 #pragma unroll
@@ -582,7 +633,12 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(p_full);
       // dQ_i (TMEM lane = query row): stage it in the P^T/dS^T tiles, which the
       // finished MMAs no longer read, then add it to dq with TMA reduce-add
-      if (!wait_all(mm_done, it & 1)) { ok = false; break; }
+      const bool got_mm = mbar_wait(mm_done, it & 1, abort_flag, err);
+      // every thread is past this block's softmax (lse/D may take the next
+      // block's) and knows whether any wait failed
+      if (any_fail(got_mm)) { ok = false; break; }
+      if (it + 1 < n_it) publish(staged);
+      if (it + 2 < n_it) staged = fetch(it + 2);
       tc_fence_after();
       {
         uint32_t qa[32], qb[32];
@@ -591,38 +647,36 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(s_free);   // the S/dQ columns may take the next S^T now
-        // rows 0..63 go to the P^T tile, 64..127 to the dS^T tile; each holds four
-        // [64 rows][32 fp32] boxes of 8 KB in 128-byte-swizzled order
-        uint8_t* stage = (r < 64 ? sPt : sdSt);
-        const int rr = r & 63;
+        // dQ_i rows of this warp (query rows 32*quarter.., columns 64*half..) go to
+        // the 4 KB of the P^T tile and the 4 KB of the dS^T tile that this warp
+        // itself writes in the softmax, as two [32 rows][32 fp32] boxes in TMA's
+        // 128-byte-swizzled order; the warp alone then issues their add-reduction
+        uint8_t* box0 = sPt + half * TF_TILE + quarter * 4096;
+        uint8_t* box1 = sdSt + half * TF_TILE + quarter * 4096;
+        const uint64_t sc2 = f2_pack(scale, scale);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const uint32_t* src = cc == 0 ? qa : qb;
-          uint8_t* box = stage + (2 * half + cc) * 8192 + rr * 128;
+          uint8_t* row = (cc == 0 ? box0 : box1) + lane * 128;
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            *reinterpret_cast<uint4*>(box + ((u ^ (rr & 7)) << 4)) =
-                make_uint4(src[4 * u], src[4 * u + 1], src[4 * u + 2], src[4 * u + 3]);
+          for (int u = 0; u < 8; ++u) {
+            float a0, a1, a2, a3;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[4 * u]), __uint_as_float(src[4 * u + 1])), sc2), a0, a1);
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[4 * u + 2]), __uint_as_float(src[4 * u + 3])), sc2), a2,
+                      a3);
+            *reinterpret_cast<float4*>(row + ((u ^ (lane & 7)) << 4)) = make_float4(a0, a1, a2, a3);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tdq, box0, 64 * half, q0 + 32 * quarter, bh);
+          tma_reduce_add_3d(&tdq, box1, 64 * half + 32, q0 + 32 * quarter, bh);
+          bulk_commit();
         }
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      asm volatile("bar.sync 1, 256;" ::: "memory");
-      if (t256 == 0) {
-#pragma unroll
-        for (int rh = 0; rh < 2; ++rh)
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            asm volatile(
-                "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                    reinterpret_cast<uint64_t>(&tdq)),
-                "r"(smem_u32((rh ? sdSt : sPt) + c * 8192)), "r"(c * 32), "r"(q0 + rh * 64), "r"(bh)
-                : "memory");
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        // the tiles are rewritten by the next block's softmax: wait until TMA has read them
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-      }
     }
-    if (t256 == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (lane == 0) bulk_wait_all();
     // dK and dV of this key block (complete after the last mm_done)
     if (ok) {
       tc_fence_after();
@@ -642,10 +696,10 @@ __global__ void __launch_bounds__(320, 1)
             wv.y = pack_bf16x2(__uint_as_float(vr[g + 2]), __uint_as_float(vr[g + 3]));
             wv.z = pack_bf16x2(__uint_as_float(vr[g + 4]), __uint_as_float(vr[g + 5]));
             wv.w = pack_bf16x2(__uint_as_float(vr[g + 6]), __uint_as_float(vr[g + 7]));
-            wk.x = pack_bf16x2(__uint_as_float(kr[g]), __uint_as_float(kr[g + 1]));
-            wk.y = pack_bf16x2(__uint_as_float(kr[g + 2]), __uint_as_float(kr[g + 3]));
-            wk.z = pack_bf16x2(__uint_as_float(kr[g + 4]), __uint_as_float(kr[g + 5]));
-            wk.w = pack_bf16x2(__uint_as_float(kr[g + 6]), __uint_as_float(kr[g + 7]));
+            wk.x = pack_bf16x2(__uint_as_float(kr[g]) * scale, __uint_as_float(kr[g + 1]) * scale);
+            wk.y = pack_bf16x2(__uint_as_float(kr[g + 2]) * scale, __uint_as_float(kr[g + 3]) * scale);
+            wk.z = pack_bf16x2(__uint_as_float(kr[g + 4]) * scale, __uint_as_float(kr[g + 5]) * scale);
+            wk.w = pack_bf16x2(__uint_as_float(kr[g + 6]) * scale, __uint_as_float(kr[g + 7]) * scale);
             *reinterpret_cast<uint4*>(dvrow + c * 32 + g) = wv;
             *reinterpret_cast<uint4*>(dkrow + c * 32 + g) = wk;
           }
@@ -722,7 +776,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
-      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
+      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 32)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }

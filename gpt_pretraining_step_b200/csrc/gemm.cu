@@ -153,7 +153,18 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   // split-K partial (never both).
   CUtensorMap mc;
   p.tma_out = 0;
-  if (c.epi != EPI_QKV && !(c.batch > 1 && p.splits > 1) && (c.out_es == 2 || c.out_es == 4)) {
+  if (c.epi == EPI_QKV) {
+    // q, k, v [B, H, T, 128] bf16 as one 4-D map {dim, t, b*H + head, which};
+    // a 32-token box stays inside one sequence when T is a multiple of 32
+    const long long gap = static_cast<const char*>(p.qkv_out[1]) - static_cast<const char*>(p.qkv_out[0]);
+    const long long gap2 = static_cast<const char*>(p.qkv_out[2]) - static_cast<const char*>(p.qkv_out[1]);
+    if (p.T > 0 && p.T % 32 == 0 && c.M % p.T == 0 && gap > 0 && gap == gap2) {
+      const long long dims[4] = {128, p.T, 1ll * (c.M / p.T) * p.H, 3};
+      const long long strides[3] = {256, 256ll * p.T, gap};
+      const int box[4] = {64, 32, 1, 1};
+      if (make_map_4d(&mc, p.qkv_out[0], dims, strides, box)) p.tma_out = 1;
+    }
+  } else if (!(c.batch > 1 && p.splits > 1) && (c.out_es == 2 || c.out_es == 4)) {
     const long long n3 = p.splits > 1 ? p.splits : c.batch;
     const long long s3 = p.splits > 1 ? p.split_stride : p.out_bs;
     if (make_map(&mc, p.out, c.out_es, c.N, c.M, n3, p.ldo, s3, 128 / c.out_es, 32)) p.tma_out = 1;
@@ -168,7 +179,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
     return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, mc, p, stream);
 
   // forward
-  GPT_GEMM_CASE(bf16, 128, false, true, EPI_QKV, bf16, bf16)
+  GPT_GEMM_CASE(bf16, 256, false, true, EPI_QKV, bf16, bf16)
   GPT_GEMM_CASE(bf16, 256, false, true, EPI_ACC, float, float)
   GPT_GEMM_CASE(bf16, 256, false, true, EPI_RELU2, bf16, bf16)
   GPT_GEMM_CASE(bf16, 256, false, true, EPI_LOGITS, bf16, bf16)
@@ -193,7 +204,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, bf16, float)
   // fp8 e4m3 forward projections (operands as raw bytes)
-  GPT_GEMM_CASE(uint8_t, 128, false, true, EPI_QKV, bf16, bf16)
+  GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_QKV, bf16, bf16)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_ACC, float, float)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_RELU2, bf16, bf16)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_STORE, float, float)

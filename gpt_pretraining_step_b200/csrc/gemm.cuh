@@ -32,7 +32,7 @@ struct GemmCfg {
   static constexpr int TMEM_COLS = 2 * BN;
   // output staging: one 32-row x 128-byte box per epilogue warp
   static constexpr int STG_BYTES = 8 * 4096;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + 1024 + 256 + 1024;   // + epilogue exchange
+  static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + 1024 + 256;
 };
 
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
@@ -167,7 +167,6 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* xchg = reinterpret_cast<float*>(stg_base + C::STG_BYTES + 256);   // [2][128] row partials
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -363,17 +362,6 @@ __global__ void __launch_bounds__(320, 1)
       }
       bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
       __syncwarp();   // tcgen05.ld is warp-collective: reconverge after the spin
-      if constexpr (EPI == EPI_QKV) {
-        // the QKV epilogue synchronises its 8 warps: make the exit decision uniform
-        uint32_t any_fail;
-        asm volatile(
-            "{\n\t.reg .pred pi, po;\n\tsetp.eq.u32 pi, %1, 0;\n\t"
-            "bar.red.or.pred po, 1, 256, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
-            : "=r"(any_fail)
-            : "r"(got ? 1u : 0u)
-            : "memory");
-        got = any_fail == 0;
-      }
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + acc * BN;
@@ -384,53 +372,101 @@ __global__ void __launch_bounds__(320, 1)
       float dqs = 1.f;   // dequantisation of fp8 operands
       if constexpr (ES == 1) dqs = (p.dq_a ? p.dq_a[0] : 1.f) * (p.dq_b ? p.dq_b[0] : 1.f);
       if constexpr (EPI == EPI_QKV) {
-        // BN = 128: the tile is one head of q, k or v for 128 tokens
-        const int which = nb / p.H;
-        const int head = nb - which * p.H;
-        const int b = row / p.T;
-        const int t = row - b * p.T;
-        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.qkv_out[which]) +
-                             ((static_cast<long long>(b) * p.H + head) * p.T + t) * 128;
-        float v[32];
-        if (which == 2) {
-#pragma unroll 1
-          for (int c = c_begin; c < c_end; ++c) {
-            tmem_load32(tbase + c * 32, v);
-            if constexpr (ES == 1) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] *= dqs;
+        // BN = 256: the tile holds heads 2*nb and 2*nb+1 of the 3H heads of q|k|v
+        // for 128 tokens; the four warps of column half `half` own one head
+        // whole, so the per-head norm needs no exchange between warps
+        const int gh = 2 * nb + half;
+        if (gh < 3 * p.H) {
+          const int which = gh / p.H;
+          const int head = gh - which * p.H;
+          const int b = row / p.T;
+          const int t = row - b * p.T;
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.qkv_out[which]) +
+                               ((static_cast<long long>(b) * p.H + head) * p.T + t) * 128;
+          const uint32_t hb = tbase + half * 128;   // TMEM columns of this head
+          // the output box of 32 tokens x 64 dims at dims col0 (TMA path)
+          const int bb = box_row0 / p.T, bt = box_row0 - bb * p.T;
+          auto put_box = [&](int col0) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && box_row0 < p.M) {
+              tma_store_4d(&tmC, stg, col0, bt, bb * p.H + head, which);
+              bulk_commit();
             }
-            if (row_ok) store_row32(dst + c * 32, v, 32);
-          }
-        } else {
-          // this warp owns RoPE pairs 32*half .. 32*half+31: columns 32*half + j and 64 + 32*half + j
-          float w[32];
-          tmem_load32(tbase + half * 32, v);
-          tmem_load32(tbase + 64 + half * 32, w);
-          float ss = 0.f;
+          };
+          if (which == 2) {
+#pragma unroll 1
+            for (int c = 0; c < 4; c += 2) {
+              float v0[32], v1[32];
+              tmem_load32(hb + c * 32, v0);
+              tmem_load32(hb + (c + 1) * 32, v1);
+              if constexpr (ES == 1) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], fmaf(w[j], w[j], ss));
-          // a rotation keeps the sum of squares, so the norm is taken before RoPE;
-          // the two warps of a row exchange their partial sums
-          xchg[half * 128 + r] = ss;
-          asm volatile("bar.sync 1, 256;" ::: "memory");
-          ss += xchg[(half ^ 1) * 128 + r];
-          asm volatile("bar.sync 1, 256;" ::: "memory");
-          ss *= dqs * dqs;
-          const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
-          if (row_ok && half == 0) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
-          const float sc = rstd * dqs;
-          const float2* cs = p.rope + static_cast<long long>(t) * 64 + half * 32;
+                for (int j = 0; j < 32; ++j) { v0[j] *= dqs; v1[j] *= dqs; }
+              }
+              if (p.tma_out) {
+                box_open();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float2 e = row_ok ? cs[j] : make_float2(1.f, 0.f);
-            const float lo = v[j], hi = w[j];
-            v[j] = (lo * e.x - hi * e.y) * sc;
-            w[j] = (lo * e.y + hi * e.x) * sc;
-          }
-          if (row_ok) {
-            store_row32(dst + half * 32, v, 32);
-            store_row32(dst + 64 + half * 32, w, 32);
+                for (int u = 0; u < 4; ++u)
+                  box_put(u, make_uint4(pack_bf16x2(v0[8 * u], v0[8 * u + 1]), pack_bf16x2(v0[8 * u + 2], v0[8 * u + 3]),
+                                        pack_bf16x2(v0[8 * u + 4], v0[8 * u + 5]),
+                                        pack_bf16x2(v0[8 * u + 6], v0[8 * u + 7])));
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  box_put(4 + u, make_uint4(pack_bf16x2(v1[8 * u], v1[8 * u + 1]),
+                                            pack_bf16x2(v1[8 * u + 2], v1[8 * u + 3]),
+                                            pack_bf16x2(v1[8 * u + 4], v1[8 * u + 5]),
+                                            pack_bf16x2(v1[8 * u + 6], v1[8 * u + 7])));
+                put_box(c * 32);
+              } else if (row_ok) {
+                store_row32(dst + c * 32, v0, 32);
+                store_row32(dst + (c + 1) * 32, v1, 32);
+              }
+            }
+          } else {
+            // a rotation keeps the sum of squares, so the norm is taken before RoPE
+            float ss = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              float v[32];
+              tmem_load32(hb + c * 32, v);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) ss = fmaf(v[j], v[j], ss);
+            }
+            ss *= dqs * dqs;
+            const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
+            if (row_ok) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
+            const float sc = rstd * dqs;
+            // RoPE pairs (i, i + 64): the first 64 output dims, then the last 64
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
+              if (p.tma_out) box_open();
+#pragma unroll 1
+              for (int pc = 0; pc < 2; ++pc) {
+                float lo[32], hi[32];
+                tmem_load32(hb + pc * 32, lo);
+                tmem_load32(hb + 64 + pc * 32, hi);
+                // pair-major table: the warp's 32 consecutive tokens read one pair coalesced
+                const float2* cs = p.rope + static_cast<long long>(pc * 32) * p.T + t;
+                float o[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  const float2 e = row_ok ? cs[static_cast<long long>(j) * p.T] : make_float2(1.f, 0.f);
+                  o[j] = part == 0 ? (lo[j] * e.x - hi[j] * e.y) * sc : (lo[j] * e.y + hi[j] * e.x) * sc;
+                }
+                if (p.tma_out) {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    box_put(4 * pc + u, make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
+                                                   pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
+                                                   pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
+                                                   pack_bf16x2(o[8 * u + 6], o[8 * u + 7])));
+                } else if (row_ok) {
+                  store_row32(dst + part * 64 + pc * 32, o, 32);
+                }
+              }
+              if (p.tma_out) put_box(part * 64);
+            }
           }
         }
       } else if constexpr (EPI == EPI_LOGITS) {

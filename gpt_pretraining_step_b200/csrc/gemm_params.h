@@ -26,7 +26,7 @@ struct GemmParams {
   float* f32a;          // QKV: rstd of q [M, H];   LOGITS: (max, sumexp) pairs [M, tiles_n]
   float* f32b;          // QKV: rstd of k [M, H];   LOGITS: target logit [M]
   const int* tgt;       // LOGITS: targets of the rows
-  const float2* rope;   // QKV: (cos, sin) [T, 64]
+  const float2* rope;   // QKV: (cos, sin) pair-major [64, T]
   void* qkv_out[3];     // QKV: q, k, v [B, H, T, 128] bf16
   void* out_t;          // STORE/AXPBY: optional transposed copy of out, [N][M] with row stride ldo_t
   long long ldo_t;

@@ -32,6 +32,9 @@ __device__ __forceinline__ float4 load_bf16x4(const bf16* src) {
 
 // ------------------------------------------------------------------ RoPE
 
+// (cos, sin) of t * 10000^(-2i/128) for positions t < T and pairs i < 64, in
+// two layouts: token-major tab[t][i] and pair-major tab[T * 64 + i * T + t]
+// (the latter lets a warp of consecutive tokens read one pair coalesced)
 __global__ void rope_table_kernel(float2* tab, int T) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= T * 64) return;
@@ -39,7 +42,9 @@ __global__ void rope_table_kernel(float2* tab, int T) {
   const double inv_freq = pow(10000.0, -2.0 * i / 128.0);
   double sn, cs;
   sincos(static_cast<double>(t) * inv_freq, &sn, &cs);
-  tab[idx] = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  const float2 e = make_float2(static_cast<float>(cs), static_cast<float>(sn));
+  tab[idx] = e;
+  tab[static_cast<long long>(T) * 64 + static_cast<long long>(i) * T + t] = e;
 }
 
 // ------------------------------------------------------------- embedding
