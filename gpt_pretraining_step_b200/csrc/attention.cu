@@ -336,54 +336,79 @@ __global__ void __launch_bounds__(192, 1)
 // ------------------------------------------------ backward on tcgen05 / TMEM
 //
 // One CTA per (128-key block j, batch*head), looping over the query blocks
-// i >= j that see those keys.  320 threads:
-//   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i
-//   warp 1      TMEM owner and MMA issuer, per query block:
-//                 S^T = K Q^T and dP^T = V dO^T          (TMEM cols 0 and 128)
-//                 dV += P^T dO (after which dO_{i+1} may load), dK += dS^T Q
-//                                                         (TMEM cols 256, 384)
-//                 dQ_i = dS K into cols 0 (S^T is consumed by then)
-//   warps 2..9  two warps per TMEM lane quarter, each on half of the 128
-//               columns: P^T = exp(S^T/sqrt(d) - lse), dS^T = P^T (dP^T - D)
-//               as bf16 tiles in shared memory (the dS^T tile is also the
-//               MN-major A operand of dS K; 1/sqrt(d) is applied to dK and dQ
-//               instead); then each warp stages its rows of dQ_i as fp32 in the
-//               parts of the two (by then idle) tiles that it writes itself and
-//               adds them into the fp32 dq buffer by TMA reduce-add (their read
-//               is awaited just before the warp's next tile stores, so it
-//               overlaps the next S^T / dP^T products and softmax);
-//               finally dK and dV of the block to global memory.
+// i = j + it >= j that see those keys.  448 threads:
+//   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i.
+//   warp 1      TMEM owner and MMA issuer.  TMEM columns: [0,128) S^T_i and
+//               dQ^T_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16 in
+//               its first 64 columns; [256,384) dV; [384,512) dK.  Per query
+//               block i, once P_i is in TMEM and dS_i in shared memory:
+//                 dV += P^T dO   (A from TMEM; then dO_{i+1} may load)
+//                 dK += dS^T Q   (then Q_{i+2} may load)
+//                 dQ^T = K^T dS^T into [0,128) once S^T_{i+1} has been read
+//                 dP^T_{i+1} = V dO_{i+1}^T into [128,256)
+//                 S^T_{i+2} = K Q_{i+2}^T into [0,128) once dQ^T_i has been read
+//   warps 2..9  softmax, two warps per TMEM lane quarter, each on 64 of the
+//               128 query columns of its key rows: when dP^T_i lands,
+//               dS'_i = P_i (dP_i - D) to shared memory and P_i (computed
+//               during the previous block) over dP^T_i in TMEM; then S^T_{i+1}
+//               and P_{i+1} while the tensor cores run block i's products.
+//               1/sqrt(d) of dS = dS' / sqrt(d) is applied to dK and dQ.
+//   warps 10..13 dQ: one warp per TMEM lane quarter (lane = head dim) stages
+//               dQ^T_i as fp32 [query][dim] boxes in a 32 KB buffer, half of
+//               the queries at a time, and adds them into the fp32 dq buffer
+//               by TMA reduce-add, so the reduction runs beside the other
+//               warps' work.
+// At the end the softmax warps write dK and dV of the key block.
 
-constexpr int TB_SMEM = 7 * TF_BUF + 1024 + 1024 + 512;
+// Row r, query columns 64*half .. 64*half+63 of a [128][128] bf16 tile kept as
+// two 64-column halves of [128 rows][128 B] with the 128-byte swizzle (16-byte
+// unit u of row r at u ^ (r & 7)); w holds the 64 values as packed pairs.
+__device__ __forceinline__ void store_row_units(uint8_t* tile, const uint32_t (&w)[32], int half, int r) {
+  uint8_t* row = tile + half * TF_TILE + r * 128;
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+}
 
-__global__ void __launch_bounds__(320, 1)
+constexpr int TB_STAGE = 32768;   // dQ staging: 64 queries x 128 dims fp32
+constexpr int TB_SMEM = 6 * TF_BUF + TB_STAGE + 2048 + 256;
+
+__global__ void __launch_bounds__(448, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                       const __grid_constant__ CUtensorMap tdq,
-                       const float* __restrict__ lse, const float* __restrict__ Dv,
-                       bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int T, float scale, int* err) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+                       const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
+                       const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int T,
+                       float scale, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
+  // dynamic shared memory window provides; refuse to run otherwise
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, ERRF_SHAPE);
+    return;
+  }
+  uint8_t* sm = smem_raw;
   uint8_t* sK = sm;
   uint8_t* sV = sm + TF_BUF;
   uint8_t* sQ = sm + 2 * TF_BUF;     // two slots
   uint8_t* sdO = sm + 4 * TF_BUF;
-  uint8_t* sPt = sm + 5 * TF_BUF;
-  uint8_t* sdSt = sm + 6 * TF_BUF;
-  float* lse_s = reinterpret_cast<float*>(sm + 7 * TF_BUF);     // 128: lse * log2(e) of the query block
-  float* dd_s = lse_s + 128;                                     // 128: D of the query block
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * TF_BUF + 1024);
+  uint8_t* sdSt = sm + 5 * TF_BUF;
+  uint8_t* sStage = sm + 6 * TF_BUF;
+  float* lse_s = reinterpret_cast<float*>(sm + 6 * TF_BUF + TB_STAGE);   // [2][128]: -lse * log2(e)
+  float* dd_s = lse_s + 256;                                              // [2][128]: -D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TF_BUF + TB_STAGE + 2048);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;    // [2]
   uint64_t* q_empty = bars + 3;   // [2]
   uint64_t* do_full = bars + 5;
-  uint64_t* do_empty = bars + 6;
-  uint64_t* sd_full = bars + 7;
-  uint64_t* p_full = bars + 8;
-  uint64_t* mm_done = bars + 9;
-  uint64_t* s_free = bars + 10;
-  uint64_t* drain = bars + 11;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 12);
+  uint64_t* do_empty = bars + 6;  // dV_i complete: dO_i and P_i are no longer read
+  uint64_t* s_full = bars + 7;    // S^T_i in TMEM
+  uint64_t* s_free = bars + 8;    // S^T_i read by the softmax warps
+  uint64_t* dp_full = bars + 9;   // dP^T_i in TMEM
+  uint64_t* p_full = bars + 10;   // P_i in TMEM, dS_i in shared memory
+  uint64_t* mm_done = bars + 11;  // dV, dK, dQ^T of block i complete
+  uint64_t* dq_free = bars + 12;  // dQ^T_i read by the dQ warps
+  uint64_t* drain = bars + 13;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = warp_id(), lane = lane_id();
@@ -399,10 +424,12 @@ __global__ void __launch_bounds__(320, 1)
     for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
     mbar_init(do_full, 1);
     mbar_init(do_empty, 1);
-    mbar_init(sd_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 256);
+    mbar_init(dp_full, 1);
     mbar_init(p_full, 256);
     mbar_init(mm_done, 1);
-    mbar_init(s_free, 256);
+    mbar_init(dq_free, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -410,6 +437,7 @@ __global__ void __launch_bounds__(320, 1)
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
     tma_prefetch_desc(&tdo);
+    tma_prefetch_desc(&tdq);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -457,72 +485,154 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       // -------------------------------------------------------------- MMA
       constexpr uint32_t IDESC_KK = make_idesc(1, 128, false, false);   // S^T, dP^T
-      constexpr uint32_t IDESC_KM = make_idesc(1, 128, false, true);    // dV, dK
-      constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ
+      constexpr uint32_t IDESC_KM = make_idesc(1, 128, false, true);    // dV (A in TMEM), dK
+      constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ^T
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), do_addr = smem_u32(sdO);
-      const uint32_t pt_addr = smem_u32(sPt), dst_addr = smem_u32(sdSt);
-      bool ok = mbar_wait(kv_full, 0, abort_flag, err);
+      const uint32_t dst_addr = smem_u32(sdSt);
+      // X^T = A B^T over the 128 head dims, both operands K-major
+      auto qk_product = [&](uint32_t d_tmem, uint32_t a_addr, uint32_t b_addr) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
+          umma_f16(d_tmem, smem_desc_sw128(a_addr + off, 16, 1024), smem_desc_sw128(b_addr + off, 16, 1024),
+                   IDESC_KK, kk > 0 ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(kv_full, 0, abort_flag, err) && mbar_wait(&q_full[0], 0, abort_flag, err);
+      if (ok) {
+        tc_fence_after();
+        qk_product(tmem, k_addr, smem_u32(sQ));   // S^T_0
+        umma_commit(s_full);
+        ok = mbar_wait(do_full, 0, abort_flag, err);
+      }
+      if (ok) {
+        tc_fence_after();
+        qk_product(tmem + 128, v_addr, do_addr);   // dP^T_0
+        umma_commit(dp_full);
+        if (n_it > 1) {
+          ok = mbar_wait(s_free, 0, abort_flag, err) && mbar_wait(&q_full[1], 0, abort_flag, err);
+          if (ok) {
+            tc_fence_after();
+            qk_product(tmem, k_addr, smem_u32(sQ + TF_BUF));   // S^T_1
+            umma_commit(s_full);
+          }
+        }
+      }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it & 1;
-        const uint32_t par = (it >> 1) & 1;
-        if (!mbar_wait(&q_full[s], par, abort_flag, err) || !mbar_wait(do_full, it & 1, abort_flag, err) ||
-            !mbar_wait(s_free, (it & 1) ^ 1u, abort_flag, err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + s * TF_BUF);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          umma_f16(tmem, smem_desc_sw128(k_addr + off, 16, 1024), smem_desc_sw128(q_addr + off, 16, 1024),
-                   IDESC_KK, kk > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          umma_f16(tmem + 128, smem_desc_sw128(v_addr + off, 16, 1024), smem_desc_sw128(do_addr + off, 16, 1024),
-                   IDESC_KK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(sd_full);
         if (!mbar_wait(p_full, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
-        // dV first: once it completes, dO_i is no longer read and the next
-        // block's dO can be loaded while dK and dQ run
+        const uint32_t q_addr = smem_u32(sQ + s * TF_BUF);
+        // dV += P^T dO: A = P^T from TMEM (16 queries = 8 packed columns per step)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_tmem_a(tmem + 256, tmem + 128 + kk * 8, smem_desc_sw128(do_addr + kk * 2048, TF_TILE, 1024),
+                          IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(do_empty);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;   // K-major A: 16 queries per step
           const uint32_t boff = kk * 2048;                              // MN-major B: 16 query rows per step
-          umma_f16(tmem + 256, smem_desc_sw128(pt_addr + aoff, 16, 1024),
-                   smem_desc_sw128(do_addr + boff, TF_TILE, 1024), IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(do_empty);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          const uint32_t boff = kk * 2048;
           umma_f16(tmem + 384, smem_desc_sw128(dst_addr + aoff, 16, 1024),
                    smem_desc_sw128(q_addr + boff, TF_TILE, 1024), IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
         }
+        umma_commit(&q_empty[s]);
+        // dQ^T_i goes to [0,128), which holds S^T_{i+1} (wait until the softmax
+        // warps have read it) or, for the last block, dQ^T_{i-1} (wait until
+        // the dQ warps have read it)
+        if (it + 1 < n_it) {
+          if (!mbar_wait(s_free, (it + 1) & 1, abort_flag, err)) { ok = false; break; }
+        } else if (it > 0) {
+          if (!mbar_wait(dq_free, (it - 1) & 1, abort_flag, err)) { ok = false; break; }
+        }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = kk * 2048;   // 16 keys per step, both operands MN-major
-          umma_f16(tmem, smem_desc_sw128(dst_addr + off, TF_TILE, 1024), smem_desc_sw128(k_addr + off, TF_TILE, 1024),
+          umma_f16(tmem, smem_desc_sw128(k_addr + off, TF_TILE, 1024), smem_desc_sw128(dst_addr + off, TF_TILE, 1024),
                    IDESC_MM, kk > 0 ? 1u : 0u);
         }
         umma_commit(mm_done);
-        umma_commit(&q_empty[s]);
+        if (it + 1 < n_it) {
+          // dP^T_{i+1} overwrites P^T_i: dV_i must have completed
+          if (!mbar_wait(do_empty, it & 1, abort_flag, err) ||
+              !mbar_wait(do_full, (it + 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          qk_product(tmem + 128, v_addr, do_addr);
+          umma_commit(dp_full);
+        }
+        if (it + 2 < n_it) {
+          if (!mbar_wait(dq_free, it & 1, abort_flag, err) ||
+              !mbar_wait(&q_full[s], ((it + 2) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          qk_product(tmem, k_addr, q_addr);   // S^T_{i+2} (same Q slot as block i)
+          umma_commit(s_full);
+        }
       }
       umma_commit(drain);
       for (uint32_t x = 0; x < (1u << 22) && !mbar_try_wait(drain, 0); ++x) {}
     }
-  } else {
-    // --------------------------------------------- P^T, dS^T, dQ, dK, dV
+  } else if (warp >= 10) {
+    // ------------------------------------------------------------------ dQ
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;        // which 64 columns of the row
-    const int r = quarter * 32 + lane;       // key row for P/dS, query row for dQ
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* box = sStage + quarter * 8192;   // [64 queries][32 dims] fp32, 128-byte swizzle
+    const uint64_t sc2 = f2_pack(scale, scale);
+    bool ok = true;
+    // dims lane of this warp's quarter for 64 queries -> the box, transposed
+    auto stage = [&](const uint32_t (&va)[32], const uint32_t (&vb)[32]) {
+      if (lane == 0) bulk_wait_read_all();   // the box's previous contents have been read
+      __syncwarp();
+#pragma unroll
+      for (int qq = 0; qq < 64; qq += 2) {
+        const uint32_t (&v)[32] = qq < 32 ? va : vb;
+        const int e = qq & 31;
+        float a0, a1;
+        f2_unpack(f2_mul(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2), a0, a1);
+        *reinterpret_cast<float*>(box + qq * 128 + (((lane >> 2) ^ (qq & 7)) << 4) + (lane & 3) * 4) = a0;
+        *reinterpret_cast<float*>(box + (qq + 1) * 128 + (((lane >> 2) ^ ((qq + 1) & 7)) << 4) + (lane & 3) * 4) = a1;
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+    };
+    for (int it = 0; it < n_it && ok; ++it) {
+      const int q0 = (j + it) * 128;
+      const bool got = mbar_wait(mm_done, it & 1, abort_flag, err);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t va[32], vb[32];
+      tmem_load32_async(tmem + lane_base, va);
+      tmem_load32_async(tmem + lane_base + 32, vb);
+      tmem_wait_ld();
+      stage(va, vb);
+      if (lane == 0) {
+        tma_reduce_add_3d(&tdq, box, 32 * quarter, q0, bh);
+        bulk_commit();
+      }
+      tmem_load32_async(tmem + lane_base + 64, va);
+      tmem_load32_async(tmem + lane_base + 96, vb);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(dq_free);
+      stage(va, vb);
+      if (lane == 0) {
+        tma_reduce_add_3d(&tdq, box, 32 * quarter, q0 + 64, bh);
+        bulk_commit();
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+  } else {
+    // ------------------------------------------------------- P, dS, dK, dV
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;        // which 64 query columns of the row
+    const int r = quarter * 32 + lane;       // key row (TMEM lane)
     const int t256 = threadIdx.x - 64;       // 0..255
     const int key = k0 + r;
     const bool key_ok = key < T;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float scale_log2 = scale * 1.4426950408889634f;
+    const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
     bool ok = true;
     // Named barrier 1 over the 256 softmax threads, which also tells every
     // thread whether any of them failed its wait (so all leave the loop together)
@@ -537,8 +647,8 @@ __global__ void __launch_bounds__(320, 1)
           : "memory");
       return f != 0;
     };
-    // this thread's share of the query block's -lse (log2 units; -inf past T so
-    // P = 0) or -D, fetched ahead so the load latency hides behind a whole block
+    // this thread's share of a query block's -lse (log2 units; -inf past T so
+    // P = 0) or -D, fetched a block ahead so the load latency hides
     auto fetch = [&](int it2) -> float {
       const int q0f = (j + it2) * 128;
       if (t256 < 128) {
@@ -548,41 +658,35 @@ __global__ void __launch_bounds__(320, 1)
       const int qq = q0f + t256 - 128;
       return qq < T ? -__ldg(Dv + static_cast<long long>(bh) * T + qq) : 0.f;
     };
-    // lse/D of block it are written after the barrier that ends block it-1's
-    // softmax and published by the barrier at the top of block it
-    auto publish = [&](float x) {
-      if (t256 < 128) lse_s[t256] = x;
-      else dd_s[t256 - 128] = x;
+    // block it2's values go to buffer it2 & 1; a barrier publishes them
+    auto publish = [&](int it2, float x) {
+      float* base = (t256 < 128 ? lse_s : dd_s) + (it2 & 1) * 128;
+      base[t256 & 127] = x;
     };
-    if (n_it > 0) publish(fetch(0));
-    float staged = n_it > 1 ? fetch(1) : 0.f;
-    for (int it = 0; it < n_it && ok; ++it) {
-      const int i = j + it;
-      const int q0 = i * 128;
-      const bool got = mbar_wait(sd_full, it & 1, abort_flag, err);
-      if (any_fail(got)) { ok = false; break; }   // also publishes lse/D of the block
-      tc_fence_after();
-      const bool diag = i == j;
+    // P of block it2 for this thread's key row and 64 query columns, packed bf16
+    uint32_t pk[32];
+    auto compute_p = [&](int it2) {
+      const bool diag = it2 == 0;
       const bool masked = diag || k0 + 128 > T;   // causal diagonal block or ragged key block
-      const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
-#pragma unroll 1
-      for (int c = 2 * half; c < 2 * half + 2; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_load32_async(tmem + lane_base + c * 32, sr);
-        tmem_load32_async(tmem + lane_base + 128 + c * 32, dr);
-        tmem_wait_ld();
-        uint32_t pk[16], dk2[16];
+      const int q0 = (j + it2) * 128;
+      const float* nls = lse_s + (it2 & 1) * 128;
+      uint32_t sa[32], sb[32];
+      tmem_load32_async(tmem + lane_base + (2 * half) * 32, sa);
+      tmem_load32_async(tmem + lane_base + (2 * half + 1) * 32, sb);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(s_free);   // S^T of this block has been read
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        const int c = 2 * half + cc;
+        const uint32_t (&sr)[32] = cc == 0 ? sa : sb;
 #pragma unroll
         for (int k = 0; k < 32; k += 8) {
-          const float4 la = *reinterpret_cast<const float4*>(lse_s + c * 32 + k);
-          const float4 lb = *reinterpret_cast<const float4*>(lse_s + c * 32 + k + 4);
-          const float4 da = *reinterpret_cast<const float4*>(dd_s + c * 32 + k);
-          const float4 db = *reinterpret_cast<const float4*>(dd_s + c * 32 + k + 4);
+          const float4 la = *reinterpret_cast<const float4*>(nls + c * 32 + k);
+          const float4 lb = *reinterpret_cast<const float4*>(nls + c * 32 + k + 4);
           const float nl[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};   // -lse * log2(e)
-          const float nd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};   // -D
           // P = 2^(S * scale * log2(e) - lse * log2(e)): six of every eight on the
-          // MUFU unit, two by the polynomial on the FMA pipe (the two units then
-          // finish together)
+          // MUFU unit, two by the polynomial on the FMA pipe
           float p[8];
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
@@ -602,82 +706,75 @@ __global__ void __launch_bounds__(320, 1)
             for (int e = 0; e < 8; ++e)
               if (!key_ok || (diag && key > q0 + c * 32 + k + e)) p[e] = 0.f;
           }
-          // dS' = P (dP - D); the 1/sqrt(d) of dS = dS' / sqrt(d) is applied to dK and dQ
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            float d0, d1;
-            f2_unpack(f2_mul(f2_pack(p[e], p[e + 1]),
-                             f2_add(f2_pack(__uint_as_float(dr[k + e]), __uint_as_float(dr[k + e + 1])),
-                                    f2_pack(nd[e], nd[e + 1]))),
-                      d0, d1);
-            pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
-            dk2[(k + e) >> 1] = pack_bf16x2(d0, d1);
-          }
-        }
-        if (c == 2 * half) {
-          // this warp's rows of the tiles held its previous dQ boxes: TMA has read them
-          if (lane == 0) bulk_wait_read_all();
-          __syncwarp();
-        }
-        const int rowoff = (c >> 1) * TF_TILE + r * 128;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int unit = ((c & 1) * 4 + t) ^ (r & 7);
-          *reinterpret_cast<uint4*>(sPt + rowoff + unit * 16) = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
-          *reinterpret_cast<uint4*>(sdSt + rowoff + unit * 16) =
-              make_uint4(dk2[4 * t], dk2[4 * t + 1], dk2[4 * t + 2], dk2[4 * t + 3]);
+          for (int e = 0; e < 8; e += 2) pk[16 * cc + ((k + e) >> 1)] = pack_bf16x2(p[e], p[e + 1]);
         }
       }
-      tc_fence_before();
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(p_full);
-      // dQ_i (TMEM lane = query row): stage it in the P^T/dS^T tiles, which the
-      // finished MMAs no longer read, then add it to dq with TMA reduce-add
-      const bool got_mm = mbar_wait(mm_done, it & 1, abort_flag, err);
-      // every thread is past this block's softmax (lse/D may take the next
-      // block's) and knows whether any wait failed
-      if (any_fail(got_mm)) { ok = false; break; }
-      if (it + 1 < n_it) publish(staged);
-      if (it + 2 < n_it) staged = fetch(it + 2);
-      tc_fence_after();
-      {
-        uint32_t qa[32], qb[32];
-        tmem_load32_async(tmem + lane_base + (2 * half) * 32, qa);
-        tmem_load32_async(tmem + lane_base + (2 * half + 1) * 32, qb);
+    };
+
+    if (n_it > 0) publish(0, fetch(0));
+    float staged = n_it > 1 ? fetch(1) : 0.f;
+    // it = -1 only computes P of the first block
+    for (int it = -1; it < n_it && ok; ++it) {
+      if (it >= 0) {
+        // dS'_i = P_i (dP_i - D) once dP^T_i is in TMEM
+        const bool got = mbar_wait(dp_full, it & 1, abort_flag, err);
+        if (any_fail(got)) { ok = false; break; }
+        // every thread is past block i-1's use of buffer (i+1) & 1
+        if (it + 1 < n_it) publish(it + 1, staged);
+        if (it + 2 < n_it) staged = fetch(it + 2);
+        tc_fence_after();
+        uint32_t da[32], db[32];
+        tmem_load32_async(tmem + lane_base + 128 + (2 * half) * 32, da);
+        tmem_load32_async(tmem + lane_base + 128 + (2 * half + 1) * 32, db);
         tmem_wait_ld();
+        // P^T_i goes over the first 64 columns of dP^T_i: every warp has read its part
         tc_fence_before();
-        mbar_arrive(s_free);   // the S/dQ columns may take the next S^T now
-        // dQ_i rows of this warp (query rows 32*quarter.., columns 64*half..) go to
-        // the 4 KB of the P^T tile and the 4 KB of the dS^T tile that this warp
-        // itself writes in the softmax, as two [32 rows][32 fp32] boxes in TMA's
-        // 128-byte-swizzled order; the warp alone then issues their add-reduction
-        uint8_t* box0 = sPt + half * TF_TILE + quarter * 4096;
-        uint8_t* box1 = sdSt + half * TF_TILE + quarter * 4096;
-        const uint64_t sc2 = f2_pack(scale, scale);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        tc_fence_after();
+        tmem_store32(tmem + lane_base + 128 + 32 * half, pk);
+        const float* nds = dd_s + (it & 1) * 128;
+        uint32_t dk2[32];
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
-          const uint32_t* src = cc == 0 ? qa : qb;
-          uint8_t* row = (cc == 0 ? box0 : box1) + lane * 128;
+          const int c = 2 * half + cc;
+          const uint32_t (&dr)[32] = cc == 0 ? da : db;
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
+          for (int k = 0; k < 32; k += 4) {
+            const float4 d4 = *reinterpret_cast<const float4*>(nds + c * 32 + k);
+            const uint32_t w0 = pk[16 * cc + (k >> 1)], w1 = pk[16 * cc + (k >> 1) + 1];
             float a0, a1, a2, a3;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[4 * u]), __uint_as_float(src[4 * u + 1])), sc2), a0, a1);
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(src[4 * u + 2]), __uint_as_float(src[4 * u + 3])), sc2), a2,
-                      a3);
-            *reinterpret_cast<float4*>(row + ((u ^ (lane & 7)) << 4)) = make_float4(a0, a1, a2, a3);
+            f2_unpack(f2_mul(f2_pack(bf16_lo(w0), bf16_hi(w0)),
+                             f2_add(f2_pack(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])), f2_pack(d4.x, d4.y))),
+                      a0, a1);
+            f2_unpack(f2_mul(f2_pack(bf16_lo(w1), bf16_hi(w1)),
+                             f2_add(f2_pack(__uint_as_float(dr[k + 2]), __uint_as_float(dr[k + 3])),
+                                    f2_pack(d4.z, d4.w))),
+                      a2, a3);
+            dk2[16 * cc + (k >> 1)] = pack_bf16x2(a0, a1);
+            dk2[16 * cc + (k >> 1) + 1] = pack_bf16x2(a2, a3);
           }
         }
+        store_row_units(sdSt, dk2, half, r);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
         fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_reduce_add_3d(&tdq, box0, 64 * half, q0 + 32 * quarter, bh);
-          tma_reduce_add_3d(&tdq, box1, 64 * half + 32, q0 + 32 * quarter, bh);
-          bulk_commit();
-        }
+        mbar_arrive(p_full);
+      }
+      // P_{i+1} while the tensor cores run this block's dV, dK, dQ^T
+      if (it + 1 < n_it) {
+        const bool got1 = mbar_wait(s_full, (it + 1) & 1, abort_flag, err);
+        if (any_fail(got1)) { ok = false; break; }   // also publishes lse/D of block i+1
+        tc_fence_after();
+        compute_p(it + 1);
       }
     }
-    if (lane == 0) bulk_wait_all();
-    // dK and dV of this key block (complete after the last mm_done)
+    // dK and dV of this key block, complete with the last block's products
+    if (ok && n_it > 0) {
+      const bool got = mbar_wait(mm_done, (n_it - 1) & 1, abort_flag, err);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, got);
+    }
     if (ok) {
       tc_fence_after();
       bf16* dkrow = dk + (static_cast<long long>(bh) * T + key) * 128;
@@ -776,12 +873,12 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
-      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 32)) {
+      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }
   dim3 grid((T + 127) / 128, B * H);
-  attn_bwd_tc_kernel<<<grid, 320, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, T,
+  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, T,
                                                 1.f / sqrtf(static_cast<float>(HD)), err);
 }
 

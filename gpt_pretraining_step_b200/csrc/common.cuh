@@ -175,6 +175,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// Same with the A operand in TMEM (M rows in lanes, K along the columns, two
+// bf16 values per 32-bit column, the lower half first).
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Same with fp32 operands read as tf32.
 __device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
@@ -285,7 +297,8 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
   return d;
 }
 
-// 2^x for a pair, x in [-126, 64), on the FMA pipe instead of the MUFU unit.
+// 2^x for a pair, x in [-126, 127), on the FMA pipe instead of the MUFU unit
+// (below -125 the result loses its implicit bit but stays under 2^-125).
 // Cody-Waite split x = j + f with j = rint(x), read off the low mantissa bits
 // of x + 1.5 * 2^23, and |f| <= 1/2; 2^f from a cubic fitted by Remez
 // exchange for minimax relative error on [-1/2, 1/2] (max relative error
