@@ -820,14 +820,15 @@ int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
     for (int i = 0; i < bt.nm; ++i) {
       ProfScope ps(c, GPT_PROF_MUON_ELEM);
       const Member& mm = bt.m[i];
+      // X (d x cc) and, for tf32 steps, its transpose, from one read of the
+      // momentum, which is stored d x cc, or cc x d for the MLP down matrix
       void* dst = static_cast<uint8_t*>(X0) + static_cast<size_t>(i) * L * per * es0;
-      launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, es0, L, d, bt.cc, mm.transpose, s);
+      void* dstT = D.n_tf32 > 0 ? static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * L * per * es0 : nullptr;
+      if (!mm.transpose)
+        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, dstT, es0, L, d, bt.cc, s);
+      else
+        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, dst, es0, L, bt.cc, d, s);
       c->launches += 1;
-      if (D.n_tf32 > 0) {
-        void* dstT = static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * L * per * es0;
-        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, es0, L, bt.cc, d, !mm.transpose, s);
-        c->launches += 1;
-      }
     }
     void* res = nullptr;
     int res_es = es0;
@@ -1143,8 +1144,12 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
   GPT_CK(cudaMemsetAsync(err, 0, 16, s));
   launch_muon_momentum(X, G, static_cast<long long>(rows) * cols, batch, 0.f, 1e-7f, inv, normws, s);
   const int es0 = tf32_steps > 0 ? 4 : 2;
-  launch_muon_make_x(X, inv, X0, es0, batch, r, cc, tr, s);
-  if (tf32_steps > 0) launch_muon_make_x(X, inv, XT0, es0, batch, cc, r, !tr, s);
+  // X (r x cc) and, for tf32 steps, its transpose; the input is stored r x cc,
+  // or cc x r when it was transposed to put the smaller side first
+  if (!tr)
+    launch_muon_make_x(X, inv, X0, tf32_steps > 0 ? XT0 : nullptr, es0, batch, r, cc, s);
+  else
+    launch_muon_make_x(X, inv, tf32_steps > 0 ? XT0 : nullptr, X0, es0, batch, cc, r, s);
   GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
   void* res = nullptr;
   int res_es = es0;

@@ -383,88 +383,129 @@ __global__ void muon_norm_kernel(const float* __restrict__ part, int nmat, float
   if (lane_id() == 0) inv_norm[z] = 1.f / (sqrtf(s) + eps);
 }
 
-// X[z] (r x c) from mom[z]; when transposing, mom[z] is (c x r).
-template <typename OutT>
-__global__ void muon_make_x_kernel(const float* __restrict__ mom, const float* __restrict__ inv_norm,
-                                   OutT* __restrict__ X, int r, int c, int transpose) {
-  __shared__ float tile[32][33];
-  const int z = blockIdx.z;
-  const float s = inv_norm[z];
-  const long long n = static_cast<long long>(r) * c;
-  const float* mz = mom + z * n;
-  OutT* xz = X + z * n;
-  const int tx = threadIdx.x, ty = threadIdx.y;   // 32 x 8
-  if (!transpose) {
-    const int row0 = blockIdx.y * 32, col0 = blockIdx.x * 32;
-    for (int i = ty; i < 32; i += 8) {
-      const int rr = row0 + i, cc = col0 + tx;
-      if (rr < r && cc < c) {
-        const float v = mz[static_cast<long long>(rr) * c + cc] * s;
-        if constexpr (sizeof(OutT) == 2) xz[static_cast<long long>(rr) * c + cc] = __float2bfloat16_rn(v);
-        else xz[static_cast<long long>(rr) * c + cc] = v;
-      }
-    }
+// Both Muon elementwise passes work on 64 x 64 tiles with 256 threads: thread
+// (tx, ty) = (threadIdx.x % 16, threadIdx.x / 16) covers columns 4 tx .. 4 tx + 3
+// of rows ty, ty + 16, ty + 32, ty + 48, and a transposed write goes through a
+// padded shared-memory tile.  Matrix extents are multiples of 4.
+
+template <typename T>
+__device__ __forceinline__ void store4(T* p, float a, float b, float c, float d) {
+  if constexpr (sizeof(T) == 2) {
+    uint2 w;
+    w.x = pack_bf16x2(a, b);
+    w.y = pack_bf16x2(c, d);
+    *reinterpret_cast<uint2*>(p) = w;
   } else {
-    // source rows are X columns: read a 32x32 block of mom (c x r), write it transposed
-    const int srow0 = blockIdx.x * 32, scol0 = blockIdx.y * 32;   // mom row (< c), mom col (< r)
-    for (int i = ty; i < 32; i += 8) {
-      const int sr = srow0 + i, sc = scol0 + tx;
-      tile[i][tx] = (sr < c && sc < r) ? mz[static_cast<long long>(sr) * r + sc] * s : 0.f;
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-      const int xr = scol0 + i, xc = srow0 + tx;
-      if (xr < r && xc < c) {
-        const float v = tile[tx][i];
-        if constexpr (sizeof(OutT) == 2) xz[static_cast<long long>(xr) * c + xc] = __float2bfloat16_rn(v);
-        else xz[static_cast<long long>(xr) * c + xc] = v;
-      }
-    }
+    *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
   }
 }
 
+template <typename T>
+__device__ __forceinline__ float4 load4(const T* p) {
+  if constexpr (sizeof(T) == 2) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    return make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+  } else {
+    return *reinterpret_cast<const float4*>(p);
+  }
+}
+
+// From the momentum mom[z] (rows x cols): `same` = s_z mom[z] in the same
+// layout and `trans` = (s_z mom[z])^T (cols x rows), s_z = inv_norm[z]; either
+// output may be null.  One read of the momentum serves both.
+template <typename OutT>
+__global__ void __launch_bounds__(256) muon_make_x_kernel(const float* __restrict__ mom,
+                                                          const float* __restrict__ inv_norm, OutT* __restrict__ same,
+                                                          OutT* __restrict__ trans, int rows, int cols) {
+  __shared__ float tile[64][65];
+  const int z = blockIdx.z;
+  const float s = inv_norm[z];
+  const long long n = static_cast<long long>(rows) * cols;
+  const float* mz = mom + z * n;
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const int cc = c0 + 4 * tx;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int rr = r0 + ty + 16 * k;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rr < rows && cc < cols) {
+      v = *reinterpret_cast<const float4*>(mz + static_cast<long long>(rr) * cols + cc);
+      v.x *= s; v.y *= s; v.z *= s; v.w *= s;
+      if (same) store4(same + z * n + static_cast<long long>(rr) * cols + cc, v.x, v.y, v.z, v.w);
+    }
+    if (trans) {
+      tile[ty + 16 * k][4 * tx] = v.x;
+      tile[ty + 16 * k][4 * tx + 1] = v.y;
+      tile[ty + 16 * k][4 * tx + 2] = v.z;
+      tile[ty + 16 * k][4 * tx + 3] = v.w;
+    }
+  }
+  if (!trans) return;
+  __syncthreads();
+  // rows of the transpose are columns of the tile
+  const int oc = r0 + 4 * tx;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int orow = c0 + ty + 16 * k, tc = ty + 16 * k;
+    if (orow < cols && oc < rows)
+      store4(trans + z * n + static_cast<long long>(orow) * rows + oc, tile[4 * tx][tc], tile[4 * tx + 1][tc],
+             tile[4 * tx + 2][tc], tile[4 * tx + 3][tc]);
+  }
+}
+
+// W[z] <- decay W[z] - step U with U = X[z] (r x c, W in the same layout) or
+// U = X[z]^T (W is c x r); also refreshes the bf16 working copy.
 template <typename XT>
-__global__ void muon_apply_kernel(float* __restrict__ W, bf16* __restrict__ Wb, const XT* __restrict__ X, int r,
-                                  int c, int transpose, float decay, float step) {
-  __shared__ float tile[32][33];
+__global__ void __launch_bounds__(256) muon_apply_kernel(float* __restrict__ W, bf16* __restrict__ Wb,
+                                                         const XT* __restrict__ X, int r, int c, int transpose,
+                                                         float decay, float step) {
+  __shared__ float tile[64][65];
   const int z = blockIdx.z;
   const long long n = static_cast<long long>(r) * c;
   float* wz = W + z * n;
   bf16* wbz = Wb + z * n;
   const XT* xz = X + z * n;
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  auto ld = [](const XT* p) -> float {
-    if constexpr (sizeof(XT) == 2) return __bfloat162float(*p);
-    else return *p;
+  const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;   // a tile of X
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  auto update = [&](long long o, float4 u) {
+    float4 w = *reinterpret_cast<const float4*>(wz + o);
+    w.x = w.x * decay - step * u.x; w.y = w.y * decay - step * u.y;
+    w.z = w.z * decay - step * u.z; w.w = w.w * decay - step * u.w;
+    *reinterpret_cast<float4*>(wz + o) = w;
+    store4(wbz + o, w.x, w.y, w.z, w.w);
   };
+  const int cc = c0 + 4 * tx;
   if (!transpose) {
-    const int row0 = blockIdx.y * 32, col0 = blockIdx.x * 32;
-    for (int i = ty; i < 32; i += 8) {
-      const int rr = row0 + i, cc = col0 + tx;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rr = r0 + ty + 16 * k;
       if (rr < r && cc < c) {
         const long long o = static_cast<long long>(rr) * c + cc;
-        const float w = wz[o] * decay - step * ld(xz + o);
-        wz[o] = w;
-        wbz[o] = __float2bfloat16_rn(w);
+        update(o, load4(xz + o));
       }
     }
-  } else {
-    // W is (c x r): W[i][j] takes X[j][i]
-    const int xrow0 = blockIdx.y * 32, xcol0 = blockIdx.x * 32;
-    for (int i = ty; i < 32; i += 8) {
-      const int xr = xrow0 + i, xc = xcol0 + tx;
-      tile[i][tx] = (xr < r && xc < c) ? ld(xz + static_cast<long long>(xr) * c + xc) : 0.f;
-    }
-    __syncthreads();
-    for (int i = ty; i < 32; i += 8) {
-      const int wr = xcol0 + i, wc = xrow0 + tx;   // W row < c, W col < r
-      if (wr < c && wc < r) {
-        const long long o = static_cast<long long>(wr) * r + wc;
-        const float w = wz[o] * decay - step * tile[tx][i];
-        wz[o] = w;
-        wbz[o] = __float2bfloat16_rn(w);
-      }
-    }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int rr = r0 + ty + 16 * k;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rr < r && cc < c) u = load4(xz + static_cast<long long>(rr) * c + cc);
+    tile[ty + 16 * k][4 * tx] = u.x;
+    tile[ty + 16 * k][4 * tx + 1] = u.y;
+    tile[ty + 16 * k][4 * tx + 2] = u.z;
+    tile[ty + 16 * k][4 * tx + 3] = u.w;
+  }
+  __syncthreads();
+  // W row = X column (c0 + ...), W columns = X rows (r0 + 4 tx ..)
+  const int wc = r0 + 4 * tx;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int wr = c0 + ty + 16 * k, tc = ty + 16 * k;
+    if (wr < c && wc < r)
+      update(static_cast<long long>(wr) * r + wc,
+             make_float4(tile[4 * tx][tc], tile[4 * tx + 1][tc], tile[4 * tx + 2][tc], tile[4 * tx + 3][tc]));
   }
 }
 
@@ -631,23 +672,25 @@ void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, flo
   muon_norm_kernel<<<nmat, 32, 0, s>>>(part, nmat, eps, inv_norm);
 }
 
-void launch_muon_make_x(const float* mom, const float* inv_norm, void* X, int out_es, int nmat, int r, int c,
-                        bool transpose, cudaStream_t s) {
-  dim3 grid = transpose ? dim3(cdiv(c, 32), cdiv(r, 32), nmat) : dim3(cdiv(c, 32), cdiv(r, 32), nmat);
+void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, void* trans, int out_es, int nmat,
+                        int rows, int cols, cudaStream_t s) {
+  const dim3 grid(cdiv(cols, 64), cdiv(rows, 64), nmat);
   if (out_es == 2)
-    muon_make_x_kernel<bf16><<<grid, dim3(32, 8), 0, s>>>(mom, inv_norm, static_cast<bf16*>(X), r, c, transpose);
+    muon_make_x_kernel<bf16><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<bf16*>(same), static_cast<bf16*>(trans),
+                                                  rows, cols);
   else
-    muon_make_x_kernel<float><<<grid, dim3(32, 8), 0, s>>>(mom, inv_norm, static_cast<float*>(X), r, c, transpose);
+    muon_make_x_kernel<float><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<float*>(same),
+                                                   static_cast<float*>(trans), rows, cols);
 }
 
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
                        float lr, float wd, float scale, cudaStream_t s) {
-  dim3 grid(cdiv(c, 32), cdiv(r, 32), nmat);
+  const dim3 grid(cdiv(c, 64), cdiv(r, 64), nmat);
   const float decay = 1.f - lr * wd, step = lr * scale;
   if (x_es == 2)
-    muon_apply_kernel<bf16><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const bf16*>(X), r, c, transpose, decay, step);
+    muon_apply_kernel<bf16><<<grid, 256, 0, s>>>(W, Wb, static_cast<const bf16*>(X), r, c, transpose, decay, step);
   else
-    muon_apply_kernel<float><<<grid, dim3(32, 8), 0, s>>>(W, Wb, static_cast<const float*>(X), r, c, transpose, decay, step);
+    muon_apply_kernel<float><<<grid, 256, 0, s>>>(W, Wb, static_cast<const float*>(X), r, c, transpose, decay, step);
 }
 
 void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* amax_bits, uint8_t* q, float* inv,

@@ -57,8 +57,8 @@ void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, flo
                           float* inv_norm, void* ws, cudaStream_t s);
 
 // X[z] = mom[z] * inv_norm[z], stored [r][c] (transpose: mom is [c][r]); bf16 or fp32 out.
-void launch_muon_make_x(const float* mom, const float* inv_norm, void* X, int out_es, int nmat, int r,
-                        int c, bool transpose, cudaStream_t s);
+void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, void* trans, int out_es, int nmat,
+                        int rows, int cols, cudaStream_t s);
 
 // W[z] = W[z] (1 - lr wd) - lr * scale * X[z] (X is [r][c]; W is [c][r] when transpose).
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
