@@ -22,23 +22,28 @@ constexpr int HD = 128;
 
 // ------------------------------------------------- forward on tcgen05 / TMEM
 //
-// One CTA per (128-query tile, batch*head), 192 threads:
-//   warp 0      TMA: Q once, K_j and V_j through two-slot rings
-//   warp 1      TMEM owner and MMA issuer: S_j = Q K_j^T into one of two TMEM
-//               S buffers and O += P_j V_j into the TMEM output accumulator;
-//               S_{j+1} is issued before P_j is ready so the tensor cores
-//               keep working while the softmax runs
-//   warps 2..5  softmax, one query row (TMEM lane) per thread: the block max
-//               from a first pass over the S row, exp2 into bf16 P written to
-//               shared memory (128-byte swizzle, the A operand of P V).
+// One CTA per pair of 128-query tiles (A = 2p, B = 2p + 1) of one
+// batch*head; the pair shares every K and V block it loads.  320 threads:
+//   warp 0      TMA: Q_A and Q_B once, K_j and V_j through two-slot rings
+//   warp 1      TMEM owner and MMA issuer.  TMEM columns: S_A [0,128),
+//               S_B [128,256), O_A [256,384), O_B [384,512).  Per key block
+//               j: O_A += P_A V_j and O_B += P_B V_j, with P read from TMEM
+//               (the softmax warps write it as packed bf16 over the first 64
+//               columns of S), then S_A = Q_A K_{j+1}^T once O_A's product
+//               has read P_A, and likewise for B; the tensor cores thus work
+//               on one tile while the other tile's softmax runs.
+//   warps 2..5  softmax of tile A, warps 6..9 of tile B, one query row (TMEM
+//               lane) per thread: the block max from a first pass over the S
+//               row, exp2 into bf16 P (a quarter of the exponentials by a
+//               polynomial on the FMA pipe), the row sum.
 // The reference max of a row only moves when the block max exceeds it by
 // more than 8 (log2 units), so P stays below 2^8; when it moves, the warp
-// rescales its rows of O in TMEM after the previous P V has completed.
-// TMEM: S0 @ col 0, S1 @ 128, O @ 256 (fp32, lane = query row).
+// rescales its rows of O in TMEM (the previous P V has completed by then:
+// S of this block was issued after it).
 
 constexpr int TF_TILE = 16384;                // one [128 rows][128 B] swizzled tile
 constexpr int TF_BUF = 2 * TF_TILE;           // 128 x 128 bf16 as two 64-column tiles
-constexpr int TF_SMEM = 7 * TF_BUF + 1024 + 512;
+constexpr int TF_SMEM = 6 * TF_BUF + 256;
 constexpr float TF_RESCALE = 8.f;
 
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -59,43 +64,50 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
                        int H, int T, float scale_log2, int* err) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = sm;
-  uint8_t* sK = sm + TF_BUF;         // two slots
-  uint8_t* sV = sm + 3 * TF_BUF;     // two slots
-  uint8_t* sP = sm + 5 * TF_BUF;     // two slots
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * TF_BUF);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
+  // dynamic shared memory window provides; refuse to run otherwise
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0 && err) atomicOr(err, ERRF_SHAPE);
+    return;
+  }
+  uint8_t* sm = smem_raw;
+  uint8_t* sQ = sm;                  // two tiles: A, B
+  uint8_t* sK = sm + 2 * TF_BUF;     // two slots
+  uint8_t* sV = sm + 4 * TF_BUF;     // two slots
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TF_BUF);
   uint64_t* q_full = bars + 0;
   uint64_t* k_full = bars + 1;    // [2]
   uint64_t* k_empty = bars + 3;   // [2]
   uint64_t* v_full = bars + 5;    // [2]
   uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2]
-  uint64_t* s_free = bars + 11;   // [2]
-  uint64_t* p_full = bars + 13;   // [2]
-  uint64_t* pv_done = bars + 15;  // [2]: P slot may be rewritten; O may be rescaled or read
-  uint64_t* drain = bars + 17;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* s_full = bars + 9;    // [2] per tile: S of block j in TMEM
+  uint64_t* p_full = bars + 11;   // [2] per tile: P of block j in TMEM
+  uint64_t* pv_done = bars + 13;  // [2] per tile: P V of block j complete
+  uint64_t* drain = bars + 15;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = warp_id(), lane = lane_id();
-  const int qt = (gridDim.x - 1) - blockIdx.x;    // longest rows first
+  const int nq = (T + 127) / 128;
+  const int pair = (gridDim.x - 1) - blockIdx.x;   // longest pairs first
   const int bh = blockIdx.y;
-  const int q0 = qt * 128;
-  const int nkv = qt + 1;                          // causal: key blocks 0..qt
+  const int qtA = 2 * pair;
+  const bool hasB = qtA + 1 < nq;
+  const int nkvA = qtA + 1;                         // causal: key blocks 0..qt
+  const int nkvB = hasB ? qtA + 2 : 0;
+  const int nkv = hasB ? nkvB : nkvA;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
-      mbar_init(&s_full[i], 1); mbar_init(&s_free[i], 128);
-      mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1);
+      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 128); mbar_init(&pv_done[i], 1);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -118,9 +130,13 @@ __global__ void __launch_bounds__(192, 1)
       // -------------------------------------------------------------- TMA
       bool ok = true;
       int issued_k = 0, issued_v = 0;
-      mbar_arrive_expect_tx(q_full, TF_BUF);
-      tma_load_3d(sQ, &tq, q_full, 0, q0, bh);
-      tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, q0, bh);
+      mbar_arrive_expect_tx(q_full, hasB ? 2 * TF_BUF : TF_BUF);
+      tma_load_3d(sQ, &tq, q_full, 0, qtA * 128, bh);
+      tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, qtA * 128, bh);
+      if (hasB) {
+        tma_load_3d(sQ + TF_BUF, &tq, q_full, 0, qtA * 128 + 128, bh);
+        tma_load_3d(sQ + TF_BUF + TF_TILE, &tq, q_full, 64, qtA * 128 + 128, bh);
+      }
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
@@ -149,58 +165,84 @@ __global__ void __launch_bounds__(192, 1)
       // -------------------------------------------------------------- MMA
       constexpr uint32_t IDESC_S = make_idesc(1, 128, false, false);
       constexpr uint32_t IDESC_O = make_idesc(1, 128, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, abort_flag, err);
-      auto issue_s = [&](int j) -> bool {
-        const int s = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(&k_full[s], par, abort_flag, err)) return false;
-        if (!mbar_wait(&s_free[s], par ^ 1u, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + s * TF_BUF);
+      // S_t = Q_t K_j^T into TMEM columns 128 t
+      auto issue_s = [&](int t, int j) {
+        const uint32_t q_addr = smem_u32(sQ + t * TF_BUF);
+        const uint32_t k_addr = smem_u32(sK + (j & 1) * TF_BUF);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          umma_f16(tmem + s * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+          umma_f16(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
                    smem_desc_sw128(k_addr + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[s]);
-        umma_commit(&k_empty[s]);
-        return true;
+        umma_commit(&s_full[t]);
       };
-      auto issue_pv = [&](int j) -> bool {
+      // O_t += P_t V_j, P_t from TMEM (16 keys = 8 packed columns per step)
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t v_addr = smem_u32(sV + (j & 1) * TF_BUF);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_f16_tmem_a(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                          smem_desc_sw128(v_addr + kk * 2048, TF_TILE, 1024), IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&pv_done[t]);
+      };
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (hasB) issue_s(1, 0);
+        umma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(&p_full[s], par, abort_flag, err)) return false;
-        if (!mbar_wait(&v_full[s], par, abort_flag, err)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + s * TF_BUF);
-        const uint32_t p_addr = smem_u32(sP + s * TF_BUF);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          umma_f16(tmem + 256, smem_desc_sw128(p_addr + aoff, 16, 1024),
-                   smem_desc_sw128(v_addr + kk * 2048, TF_TILE, 1024), IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+        const bool a_on = j < nkvA, b_on = j < nkvB;
+        if (!mbar_wait(&v_full[s], par, abort_flag, err)) { ok = false; break; }
+        if (a_on) {
+          if (!mbar_wait(&p_full[0], j & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(0, j);
+        }
+        if (b_on) {
+          if (!mbar_wait(&p_full[1], j & 1, abort_flag, err)) { ok = false; break; }
+          tc_fence_after();
+          issue_pv(1, j);
         }
         umma_commit(&v_empty[s]);
-        umma_commit(&pv_done[s]);
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv) ok = issue_s(j + 1);
-        if (ok) ok = issue_pv(j);
+        if (j + 1 < nkv) {
+          const int s1 = (j + 1) & 1;
+          if (!mbar_wait(&k_full[s1], ((j + 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          // S_t of the next block goes over P_t: its P V must have read it
+          if (j + 1 < nkvA) {
+            if (!mbar_wait(&pv_done[0], j & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+          if (j + 1 < nkvB) {
+            if (!mbar_wait(&pv_done[1], j & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(1, j + 1);
+          }
+          umma_commit(&k_empty[s1]);
+        }
       }
       umma_commit(drain);
       for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
     }
   } else {
     // ---------------------------------------------------------- softmax
+    const int tile = (warp - 2) >> 2;           // 0: A, 1: B
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
+    const int qt = qtA + tile;
+    const int q0 = qt * 128;
     const int q = q0 + r;
+    const int nkv_t = tile ? nkvB : nkvA;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t t_o = tmem + lane_base + 256;
+    const uint32_t t_s = tmem + lane_base + tile * 128;
+    const uint32_t t_o = tmem + lane_base + 256 + tile * 128;
+    const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
     float m_ref = -INFINITY, l = 0.f;   // reference max (log2 units) and row sum relative to it
     bool ok = true;
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
@@ -208,26 +250,22 @@ __global__ void __launch_bounds__(192, 1)
       __syncwarp();
       return __all_sync(0xffffffffu, got);
     };
-    for (int j = 0; j < nkv && ok; ++j) {
-      const int s = j & 1;
-      if (!wait_all(&s_full[s], (j >> 1) & 1)) { ok = false; break; }
+    for (int j = 0; j < nkv_t && ok; ++j) {
+      if (!wait_all(&s_full[tile], j & 1)) { ok = false; break; }
       tc_fence_after();
-      // the whole S row at once; the S buffer is free again as soon as it is read
+      // the whole S row at once
       uint32_t sr[128];
       {
-        const uint32_t ts = tmem + lane_base + s * 128;
         uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
         uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
         uint32_t (&r2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
         uint32_t (&r3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-        tmem_load32_async(ts, r0);
-        tmem_load32_async(ts + 32, r1);
-        tmem_load32_async(ts + 64, r2);
-        tmem_load32_async(ts + 96, r3);
+        tmem_load32_async(t_s, r0);
+        tmem_load32_async(t_s + 32, r1);
+        tmem_load32_async(t_s + 64, r2);
+        tmem_load32_async(t_s + 96, r3);
         tmem_wait_ld();
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[s]);
       const int kbase = j * 128;
       if ((j == qt) || (kbase + 128 > T)) {
         // causal diagonal / ragged tail: masked scores become -inf
@@ -249,10 +287,9 @@ __global__ void __launch_bounds__(192, 1)
       const bool move = mblk > m_ref + TF_RESCALE;   // always true on the first block
       const float m_new = move ? mblk : m_ref;
       const float factor = ex2_approx(m_ref - m_new);  // 1 when the reference stays, 0 on the first block
-      // O may only be rescaled once the previous P V has accumulated into it
+      // O holds the products of blocks < j (S of this block was issued after
+      // the last of them completed), so it may be rescaled now
       if (j >= 1 && __any_sync(0xffffffffu, move)) {
-        if (!wait_all(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1)) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t ra[32];
@@ -262,43 +299,65 @@ __global__ void __launch_bounds__(192, 1)
           for (int k = 0; k < 32; ++k) ra[k] = __float_as_uint(__uint_as_float(ra[k]) * factor);
           tmem_store32(t_o + c * 32, ra);
         }
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
       }
-      // the P slot is free once the P V two blocks back has read it
-      if (j >= 2 && !wait_all(&pv_done[s], ((j >> 1) & 1) ^ 1u)) { ok = false; break; }
-      // probabilities relative to the reference, row sum, bf16 P tile (masked scores give 0)
-      const float bias = -m_new;
-      float rs8[8];
+      // probabilities relative to the reference (masked scores give 0), row sum,
+      // bf16 P over the first 64 columns of S
+      const uint64_t nb2 = f2_pack(-m_new, -m_new);
+      uint64_t rs2 = f2_pack(0.f, 0.f);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) rs8[t] = 0.f;
-      uint8_t* pslot = sP + s * TF_BUF;
+      for (int c = 0; c < 2; ++c) {
+        // the second half of the row is read again from TMEM (its first 64
+        // columns now hold P of the first half) rather than kept in registers
+        uint32_t sh[64];
+        if (c == 0) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+          for (int k = 0; k < 64; ++k) sh[k] = sr[k];
+        } else {
+          tmem_load32_async(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sh[0]));
+          tmem_load32_async(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sh[32]));
+          tmem_wait_ld();
+          if ((j == qt) || (kbase + 128 > T)) {
 #pragma unroll
-        for (int k = 0; k < 32; k += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + k]), scale_log2, bias));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c * 32 + k + 1]), scale_log2, bias));
-          rs8[(k >> 1) & 7] += p0 + p1;
-          pk[k >> 1] = pack_bf16x2(p0, p1);
+            for (int k = 0; k < 64; ++k) {
+              const int key = kbase + 64 + k;
+              if (key > q || key >= T) sh[k] = __float_as_uint(-INFINITY);
+            }
+          }
         }
-        uint8_t* prow = pslot + (c >> 1) * TF_TILE + r * 128;
+        uint32_t pk[32];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int unit = ((c & 1) * 4 + t) ^ (r & 7);
-          *reinterpret_cast<uint4*>(prow + unit * 16) =
-              make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        for (int k = 0; k < 64; k += 8) {
+          float p[8];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sh[k + e]), __uint_as_float(sh[k + e + 1])), sl2, nb2),
+                      x0, x1);
+            if (e < 6) {
+              p[e] = ex2_approx(x0);
+              p[e + 1] = ex2_approx(x1);
+            } else {
+              f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            rs2 = f2_add(rs2, f2_pack(p[e], p[e + 1]));
+            pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+          }
         }
+        tmem_store32(t_s + c * 32, pk);
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(&p_full[s]);
-      const float rs = ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3])) + ((rs8[4] + rs8[5]) + (rs8[6] + rs8[7]));
-      l = l * factor + rs;
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(&p_full[tile]);
+      float rs0, rs1;
+      f2_unpack(rs2, rs0, rs1);
+      l = l * factor + (rs0 + rs1);
       m_ref = m_new;
     }
     // epilogue: O / l once the last P V has landed
-    if (ok) ok = wait_all(&pv_done[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1);
+    if (ok && nkv_t > 0) ok = wait_all(&pv_done[tile], (nkv_t - 1) & 1);
     if (ok) {
       tc_fence_after();
       const int b = bh / H, h = bh - (bh / H) * H;
@@ -339,18 +398,21 @@ __global__ void __launch_bounds__(192, 1)
 // i = j + it >= j that see those keys.  448 threads:
 //   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i.
 //   warp 1      TMEM owner and MMA issuer.  TMEM columns: [0,128) S^T_i and
-//               dQ^T_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16 in
-//               its first 64 columns; [256,384) dV; [384,512) dK.  Per query
-//               block i, once P_i is in TMEM and dS_i in shared memory:
-//                 dV += P^T dO   (A from TMEM; then dO_{i+1} may load)
-//                 dK += dS^T Q   (then Q_{i+2} may load)
+//               dQ^T_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16
+//               (queries 0..63 at 128.., 64..127 at 192..); [256,384) dV;
+//               [384,512) dK.  Per query block i:
+//                 dV += P^T dO   once P_i is in TMEM (A from TMEM; then
+//                                dO_{i+1} may load)
+//                 dK += dS^T Q   once dS_i is in shared memory (then Q_{i+2}
+//                                may load)
 //                 dQ^T = K^T dS^T into [0,128) once S^T_{i+1} has been read
 //                 dP^T_{i+1} = V dO_{i+1}^T into [128,256)
 //                 S^T_{i+2} = K Q_{i+2}^T into [0,128) once dQ^T_i has been read
 //   warps 2..9  softmax, two warps per TMEM lane quarter, each on 64 of the
-//               128 query columns of its key rows: when dP^T_i lands,
-//               dS'_i = P_i (dP_i - D) to shared memory and P_i (computed
-//               during the previous block) over dP^T_i in TMEM; then S^T_{i+1}
+//               128 query columns of its key rows: when dP^T_i lands, P_i
+//               (computed during the previous block) over the dP^T columns the
+//               warp has read, then dS'_i = P_i (dP_i - D) to shared memory
+//               while dV runs; then S^T_{i+1}
 //               and P_{i+1} while the tensor cores run block i's products.
 //               1/sqrt(d) of dS = dS' / sqrt(d) is applied to dK and dQ.
 //   warps 10..13 dQ: one warp per TMEM lane quarter (lane = head dim) stages
@@ -404,11 +466,12 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* s_full = bars + 7;    // S^T_i in TMEM
   uint64_t* s_free = bars + 8;    // S^T_i read by the softmax warps
   uint64_t* dp_full = bars + 9;   // dP^T_i in TMEM
-  uint64_t* p_full = bars + 10;   // P_i in TMEM, dS_i in shared memory
+  uint64_t* p_ready = bars + 10;  // P_i in TMEM
   uint64_t* mm_done = bars + 11;  // dV, dK, dQ^T of block i complete
   uint64_t* dq_free = bars + 12;  // dQ^T_i read by the dQ warps
   uint64_t* drain = bars + 13;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* ds_ready = bars + 14; // dS_i in shared memory
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 15);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = warp_id(), lane = lane_id();
@@ -427,7 +490,8 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
     mbar_init(dp_full, 1);
-    mbar_init(p_full, 256);
+    mbar_init(p_ready, 256);
+    mbar_init(ds_ready, 256);
     mbar_init(mm_done, 1);
     mbar_init(dq_free, 128);
     mbar_init(drain, 1);
@@ -520,15 +584,20 @@ __global__ void __launch_bounds__(448, 1)
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const int s = it & 1;
-        if (!mbar_wait(p_full, it & 1, abort_flag, err)) { ok = false; break; }
+        if (!mbar_wait(p_ready, it & 1, abort_flag, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sQ + s * TF_BUF);
-        // dV += P^T dO: A = P^T from TMEM (16 queries = 8 packed columns per step)
+        // dV += P^T dO: A = P^T from TMEM, 16 queries = 8 packed columns per
+        // step; queries 0..63 at columns 128.., 64..127 at columns 192..
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16_tmem_a(tmem + 256, tmem + 128 + kk * 8, smem_desc_sw128(do_addr + kk * 2048, TF_TILE, 1024),
-                          IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_tmem_a(tmem + 256, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8,
+                          smem_desc_sw128(do_addr + kk * 2048, TF_TILE, 1024), IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
         umma_commit(do_empty);
+        // dK and dQ^T once dS_i is in shared memory (the softmax warps compute it
+        // while dV runs)
+        if (!mbar_wait(ds_ready, it & 1, abort_flag, err)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t aoff = (kk >> 2) * TF_TILE + (kk & 3) * 32;   // K-major A: 16 queries per step
@@ -728,11 +797,11 @@ __global__ void __launch_bounds__(448, 1)
         tmem_load32_async(tmem + lane_base + 128 + (2 * half) * 32, da);
         tmem_load32_async(tmem + lane_base + 128 + (2 * half + 1) * 32, db);
         tmem_wait_ld();
-        // P^T_i goes over the first 64 columns of dP^T_i: every warp has read its part
+        // P^T_i over the first 32 of the 64 dP^T columns this warp has just read
+        tmem_store32(tmem + lane_base + 128 + 64 * half, pk);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        tc_fence_after();
-        tmem_store32(tmem + lane_base + 128 + 32 * half, pk);
+        mbar_arrive(p_ready);
         const float* nds = dd_s + (it & 1) * 128;
         uint32_t dk2[32];
 #pragma unroll
@@ -756,10 +825,8 @@ __global__ void __launch_bounds__(448, 1)
           }
         }
         store_row_units(sdSt, dk2, half, r);
-        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
         fence_proxy_async_smem();
-        mbar_arrive(p_full);
+        mbar_arrive(ds_ready);
       }
       // P_{i+1} while the tensor cores run this block's dV, dK, dQ^T
       if (it + 1 < n_it) {
@@ -849,9 +916,9 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
     return;
   }
-  dim3 grid((T + 127) / 128, B * H);
+  dim3 grid(((T + 127) / 128 + 1) / 2, B * H);   // pairs of query tiles
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_tc_kernel<<<grid, 192, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
+  attn_fwd_tc_kernel<<<grid, 320, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
