@@ -23,18 +23,22 @@ constexpr int HD = 128;
 // ------------------------------------------------- forward on tcgen05 / TMEM
 //
 // One CTA per pair of 128-query tiles (A = 2p, B = 2p + 1) of one
-// batch*head; the pair shares every K and V block it loads.  320 threads:
+// batch*head; the pair shares every K and V block it loads.  384 threads
+// in three warp groups; the first (TMA, MMA and two idle warps) gives
+// registers to the two softmax groups (setmaxnreg 40 / 232 / 232, which adds
+// up to the 168 per thread the block is launched with), so each softmax
+// thread keeps its whole S row in registers.
 //   warp 0      TMA: Q_A and Q_B once, K_j and V_j through two-slot rings
 //   warp 1      TMEM owner and MMA issuer.  TMEM columns: S_A [0,128),
 //               S_B [128,256), O_A [256,384), O_B [384,512).  Per key block
 //               j: O_A += P_A V_j and O_B += P_B V_j, with P read from TMEM
 //               (the softmax warps write it as packed bf16 over the first 64
 //               columns of S), then S_A = Q_A K_{j+1}^T once O_A's product
-//               has read P_A, and likewise for B; the tensor cores thus work
-//               on one tile while the other tile's softmax runs.
-//   warps 2..5  softmax of tile A, warps 6..9 of tile B, one query row (TMEM
+//               has read P_A, and then the same for B; the tensor cores thus
+//               work on one tile while the other tile's softmax runs.
+//   warps 4..7  softmax of tile A, warps 8..11 of tile B, one query row (TMEM
 //               lane) per thread: the block max from a first pass over the S
-//               row, exp2 into bf16 P (a quarter of the exponentials by a
+//               row, exp2 into bf16 P (three of every eight exponentials by a
 //               polynomial on the FMA pipe), the row sum.
 // The reference max of a row only moves when the block max exceeds it by
 // more than 8 (log2 units), so P stays below 2^8; when it moves, the warp
@@ -64,7 +68,7 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
                        int H, int T, float scale_log2, int* err) {
@@ -125,6 +129,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------------- TMA
@@ -197,42 +202,33 @@ __global__ void __launch_bounds__(320, 1)
       for (int j = 0; j < nkv && ok; ++j) {
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
-        const bool a_on = j < nkvA, b_on = j < nkvB;
+        const int s1 = (j + 1) & 1;
         if (!mbar_wait(&v_full[s], par, abort_flag, err)) { ok = false; break; }
-        if (a_on) {
-          if (!mbar_wait(&p_full[0], j & 1, abort_flag, err)) { ok = false; break; }
+        if (j + 1 < nkv && !mbar_wait(&k_full[s1], ((j + 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        // per tile: O += P V_j, then S of the next block over P once that product
+        // has read it (tile B's softmax trails tile A's, so A goes first)
+        for (int t = 0; t < 2; ++t) {
+          if (j >= (t ? nkvB : nkvA)) continue;
+          if (!mbar_wait(&p_full[t], j & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(0, j);
+          issue_pv(t, j);
+          if (j + 1 < (t ? nkvB : nkvA)) {
+            if (!mbar_wait(&pv_done[t], j & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(t, j + 1);
+          }
         }
-        if (b_on) {
-          if (!mbar_wait(&p_full[1], j & 1, abort_flag, err)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(1, j);
-        }
+        if (!ok) break;
         umma_commit(&v_empty[s]);
-        if (j + 1 < nkv) {
-          const int s1 = (j + 1) & 1;
-          if (!mbar_wait(&k_full[s1], ((j + 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-          // S_t of the next block goes over P_t: its P V must have read it
-          if (j + 1 < nkvA) {
-            if (!mbar_wait(&pv_done[0], j & 1, abort_flag, err)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(0, j + 1);
-          }
-          if (j + 1 < nkvB) {
-            if (!mbar_wait(&pv_done[1], j & 1, abort_flag, err)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(1, j + 1);
-          }
-          umma_commit(&k_empty[s1]);
-        }
+        if (j + 1 < nkv) umma_commit(&k_empty[s1]);
       }
       umma_commit(drain);
       for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
     }
-  } else {
+  } else if (warp >= 4) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;\n" ::: "memory");
     // ---------------------------------------------------------- softmax
-    const int tile = (warp - 2) >> 2;           // 0: A, 1: B
+    const int tile = (warp - 4) >> 2;           // 0: A, 1: B
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const int qt = qtA + tile;
@@ -306,24 +302,6 @@ __global__ void __launch_bounds__(320, 1)
       uint64_t rs2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        // the second half of the row is read again from TMEM (its first 64
-        // columns now hold P of the first half) rather than kept in registers
-        uint32_t sh[64];
-        if (c == 0) {
-#pragma unroll
-          for (int k = 0; k < 64; ++k) sh[k] = sr[k];
-        } else {
-          tmem_load32_async(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&sh[0]));
-          tmem_load32_async(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&sh[32]));
-          tmem_wait_ld();
-          if ((j == qt) || (kbase + 128 > T)) {
-#pragma unroll
-            for (int k = 0; k < 64; ++k) {
-              const int key = kbase + 64 + k;
-              if (key > q || key >= T) sh[k] = __float_as_uint(-INFINITY);
-            }
-          }
-        }
         uint32_t pk[32];
 #pragma unroll
         for (int k = 0; k < 64; k += 8) {
@@ -331,9 +309,10 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
           for (int e = 0; e < 8; e += 2) {
             float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sh[k + e]), __uint_as_float(sh[k + e + 1])), sl2, nb2),
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c * 64 + k + e]), __uint_as_float(sr[c * 64 + k + e + 1])),
+                             sl2, nb2),
                       x0, x1);
-            if (e < 6) {
+            if (e < 4 || (e == 4 && (k & 8))) {
               p[e] = ex2_approx(x0);
               p[e + 1] = ex2_approx(x1);
             } else {
@@ -918,7 +897,7 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
   }
   dim3 grid(((T + 127) / 128 + 1) / 2, B * H);   // pairs of query tiles
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_tc_kernel<<<grid, 320, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
+  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
