@@ -43,7 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", default="d20", choices=["d12", "d20", "d24", "d26"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--ns-tf32-steps", type=int, default=3)
+    ap.add_argument("--ns-tf32-steps", type=int, default=-1,
+                    help="Newton-Schulz operand precision: -1 = fp16 (default), 0..5 = leading tf32 steps, then bf16")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
                     help="fp8: forward block projections on e4m3 operands")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -364,7 +365,7 @@ def run_ours(a):
             "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
             "config": {"workload": f"{a.config} GPT step (fwd+bwd+Muon+AdamW)", "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
-                       "parallelism": f"dp{world}", "ns_tf32_steps": a.ns_tf32_steps,
+                       "parallelism": f"dp{world}", "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
                        "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2"},
             "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
             "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",

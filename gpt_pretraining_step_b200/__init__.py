@@ -106,7 +106,7 @@ def _check(rc):
     return rc
 
 
-def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=3, lm_chunk_rows=0, seed=0,
+def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0, seed=0,
                 precision=0):
     return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
                   mlp_mult=4, precision=precision, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows,
@@ -136,7 +136,7 @@ class GPTStep:
     object; every computation runs in libgpt's kernels on ``stream``.
     """
 
-    def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=3, lm_chunk_rows=0,
+    def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0,
                  seed=0, stream=None, precision=0):
         import torch
         self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision)
@@ -303,7 +303,7 @@ def rmsnorm_fwd(x, stream=None):
     return y, r
 
 
-def newton_schulz(G, tf32_steps=3, stream=None):
+def newton_schulz(G, tf32_steps=-1, stream=None):
     import torch
     batch, rows, cols = G.shape
     X = torch.empty_like(G)
@@ -314,7 +314,7 @@ def newton_schulz(G, tf32_steps=3, stream=None):
     return X
 
 
-def newton_schulz_noalloc(G, tf32_steps=3, X=None, stream=None):
+def newton_schulz_noalloc(G, tf32_steps=-1, X=None, stream=None):
     """Newton-Schulz through the entry point that allocates no device memory.
 
     The library keeps the scratch in its own fixed device array (at most

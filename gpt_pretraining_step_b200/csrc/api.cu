@@ -93,7 +93,7 @@ int dims_from(const gpt_config* c, Dims& D) {
   if (c->head_dim != 128) return fail(GPT_EINVAL, "head_dim must be 128");
   if (c->mlp_mult != 4) return fail(GPT_EINVAL, "mlp_mult must be 4");
   if (c->precision != 0 && c->precision != 1) return fail(GPT_EINVAL, "precision must be 0 (bf16) or 1 (fp8)");
-  if (c->ns_tf32_steps < 0 || c->ns_tf32_steps > 5) return fail(GPT_EINVAL, "ns_tf32_steps must be in 0..5");
+  if (c->ns_tf32_steps < -1 || c->ns_tf32_steps > 5) return fail(GPT_EINVAL, "ns_tf32_steps must be in -1..5");
   D.L = c->depth;
   D.d = c->d_model ? c->d_model : 64 * c->depth;
   if (D.d % 128 || D.d > 2048) return fail(GPT_EINVAL, "d_model must be a multiple of 128, at most 2048");
@@ -181,9 +181,12 @@ void make_plan(const Dims& D, Plan& P) {
   const size_t xelems = std::max({L * d * 3 * d, L * d * d, 2 * L * d * F});
   P.X0 = ab.take(xelems * 4);
   P.X1 = ab.take(xelems * 4);
-  // transposed copies, read K-major by the tf32 steps of Newton-Schulz
-  P.XT0 = ab.take(D.n_tf32 > 0 ? xelems * 4 : 16);
-  P.XT1 = ab.take(D.n_tf32 > 1 ? xelems * 4 : 16);
+  // fp16 operand copies of the Newton-Schulz iterates (fp16 mode), or the
+  // transposed fp32 copies read K-major by its tf32 steps
+  const size_t xt_bytes0 = D.n_tf32 < 0 ? xelems * 2 : (D.n_tf32 > 0 ? xelems * 4 : 16);
+  const size_t xt_bytes1 = D.n_tf32 < 0 ? xelems * 2 : (D.n_tf32 > 1 ? xelems * 4 : 16);
+  P.XT0 = ab.take(xt_bytes0);
+  P.XT1 = ab.take(xt_bytes1);
   P.Abuf = ab.take(2 * L * d * d * 4);
   P.Bbuf = ab.take(2 * L * d * d * 4);
   P.inv_norm = ab.take(4 * L * 4);
@@ -655,11 +658,65 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
 int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* XT0, void* XT1, void* Ab,
                   void* Bb, int n_tf32, cudaStream_t s, int* err, void** out, int* out_es, int64_t* launches) {
   ProfScope ps(pc, GPT_PROF_NS_GEMM);
+  const double (*kPolarCoef)[3] = polar_coefficients();
+  if (n_tf32 < 0) {
+    // fp16 operands at the full tensor rate with fp32 iterates: X (fp32) in
+    // X0/X1 and its fp16 copy, written by the same epilogue, in XT0/XT1; the
+    // Gram A and B = b A + c A^2 in fp16.  The normalised X keeps every
+    // operand far inside fp16's range.
+    void* cur = X0;
+    void* nxt = X1;
+    void* curH = XT0;
+    void* nxtH = XT1;
+    for (int t = 0; t < kPolarSteps; ++t) {
+      const bool last = t + 1 == kPolarSteps;
+      const double a = kPolarCoef[t][0], b = kPolarCoef[t][1], cf = kPolarCoef[t][2];
+      {
+        GemmCall g = base_call(r, r, cc);   // A = X X^T
+        g.batch = nz; g.es = 2; g.f16 = true;
+        g.A = curH; g.lda = cc; g.a_bs = 1ll * r * cc;
+        g.B = curH; g.ldb = cc; g.b_bs = 1ll * r * cc;
+        g.bn = 128; g.sym = true; g.epi = EPI_STORE;
+        g.out_es = 2; g.out_f16 = true; g.aux_es = 2; g.aux_f16 = true;
+        g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
+        GPT_CK(gemm_run(g, s));
+      }
+      {
+        GemmCall g = base_call(r, r, r);    // B = b A + c A A
+        g.batch = nz; g.es = 2; g.f16 = true;
+        g.A = Ab; g.lda = r; g.a_bs = 1ll * r * r;
+        g.B = Ab; g.ldb = r; g.b_bs = 1ll * r * r;
+        g.bn = 128; g.sym = true; g.epi = EPI_AXPBY;
+        g.out_es = 2; g.out_f16 = true; g.aux_es = 2; g.aux_f16 = true;
+        g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
+        g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
+        g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;
+        GPT_CK(gemm_run(g, s));
+      }
+      {
+        GemmCall g = base_call(r, cc, r);   // X' = a X + B X
+        g.batch = nz; g.es = 2; g.f16 = true;
+        g.A = Bb; g.lda = r; g.a_bs = 1ll * r * r;
+        g.B = curH; g.b_mn = true; g.ldb = cc; g.b_bs = 1ll * r * cc;
+        g.bn = 256; g.epi = EPI_AXPBY; g.out_es = 4; g.aux_es = 4;
+        g.p.out = nxt; g.p.ldo = cc; g.p.out_bs = 1ll * r * cc;
+        if (!last) g.p.out2 = nxtH;
+        g.p.aux = cur; g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
+        g.p.alpha = static_cast<float>(a); g.p.beta = 1.f; g.p.err = err;
+        GPT_CK(gemm_run(g, s));
+      }
+      *launches += 3;
+      std::swap(cur, nxt);
+      std::swap(curH, nxtH);
+    }
+    *out = cur;
+    *out_es = 4;
+    return GPT_OK;
+  }
   void* cur = X0;
   void* nxt = X1;
   void* curT = XT0;
   void* nxtT = XT1;
-  const double (*kPolarCoef)[3] = polar_coefficients();
   for (int t = 0; t < kPolarSteps; ++t) {
     const int es = t < n_tf32 ? 4 : 2;
     const bool last = t + 1 == kPolarSteps;
@@ -802,7 +859,8 @@ int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
                            s);
   }
   c->launches += 8;
-  const int es0 = D.n_tf32 > 0 ? 4 : 2;
+  // first Newton-Schulz iterate: fp32 for the fp16 and tf32 modes, bf16 otherwise
+  const int es0 = D.n_tf32 != 0 ? 4 : 2;
   void* X0 = c->A<void>(P.X0);
   void* X1 = c->A<void>(P.X1);
   void* XT0 = c->A<void>(P.XT0);
@@ -824,10 +882,12 @@ int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
       // momentum, which is stored d x cc, or cc x d for the MLP down matrix
       void* dst = static_cast<uint8_t*>(X0) + static_cast<size_t>(i) * L * per * es0;
       void* dstT = D.n_tf32 > 0 ? static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * L * per * es0 : nullptr;
+      // fp16 mode: the fp16 operand copy of X, same layout as X
+      __half* dstH = D.n_tf32 < 0 ? reinterpret_cast<__half*>(XT0) + static_cast<size_t>(i) * L * per : nullptr;
       if (!mm.transpose)
-        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, dstT, es0, L, d, bt.cc, s);
+        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, dstT, es0, L, d, bt.cc, s, dstH, nullptr);
       else
-        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, dst, es0, L, bt.cc, d, s);
+        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, dst, es0, L, bt.cc, d, s, nullptr, dstH);
       c->launches += 1;
     }
     void* res = nullptr;
@@ -1122,7 +1182,7 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
                          void* stream) {
   if (!G || !X || !scratch) return fail(GPT_EINVAL, "null pointer");
   if (batch < 1 || rows < 8 || cols < 8 || rows % 8 || cols % 8) return fail(GPT_EINVAL, "bad matrix shape");
-  if (tf32_steps < 0 || tf32_steps > 5) return fail(GPT_EINVAL, "tf32_steps must be in 0..5");
+  if (tf32_steps < -1 || tf32_steps > 5) return fail(GPT_EINVAL, "tf32_steps must be in -1..5");
   if (reinterpret_cast<uintptr_t>(scratch) & (kAlign - 1)) return fail(GPT_EINVAL, "scratch must be 256-byte aligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tr = rows > cols;
@@ -1143,13 +1203,16 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
   GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
   GPT_CK(cudaMemsetAsync(err, 0, 16, s));
   launch_muon_momentum(X, G, static_cast<long long>(rows) * cols, batch, 0.f, 1e-7f, inv, normws, s);
-  const int es0 = tf32_steps > 0 ? 4 : 2;
-  // X (r x cc) and, for tf32 steps, its transpose; the input is stored r x cc,
-  // or cc x r when it was transposed to put the smaller side first
+  const int es0 = tf32_steps != 0 ? 4 : 2;
+  // X (r x cc) and, for tf32 steps, its transpose or, for fp16 steps, its fp16
+  // copy; the input is stored r x cc, or cc x r when it was transposed to put
+  // the smaller side first
+  void* xT = tf32_steps > 0 ? XT0 : nullptr;
+  __half* xH = tf32_steps < 0 ? static_cast<__half*>(XT0) : nullptr;
   if (!tr)
-    launch_muon_make_x(X, inv, X0, tf32_steps > 0 ? XT0 : nullptr, es0, batch, r, cc, s);
+    launch_muon_make_x(X, inv, X0, xT, es0, batch, r, cc, s, xH, nullptr);
   else
-    launch_muon_make_x(X, inv, tf32_steps > 0 ? XT0 : nullptr, X0, es0, batch, cc, r, s);
+    launch_muon_make_x(X, inv, xT, X0, es0, batch, cc, r, s, nullptr, xH);
   GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
   void* res = nullptr;
   int res_es = es0;

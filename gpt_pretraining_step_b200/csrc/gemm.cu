@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "gemm.cuh"
 #include "gemm.h"
@@ -28,7 +29,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3-D map over [batch][outer][inner] with 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
-              long long ld, long long bs, int box_inner, int box_outer) {
+              long long ld, long long bs, int box_inner, int box_outer, bool f16) {
   auto fn = encode_fn();
   if (!fn) return false;
   if (bs == 0 || batch == 1) bs = ld * outer;
@@ -38,8 +39,9 @@ bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long lon
   cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   if ((reinterpret_cast<uintptr_t>(ptr) & 15) || (strides[0] & 15) || (strides[1] & 15)) return false;
-  const CUtensorMapDataType dt = es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                : (es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
+  const CUtensorMapDataType dt =
+      es == 2 ? (f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+              : (es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
   CUresult r = fn(m, dt, 3,
                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -73,8 +75,8 @@ bool make_map_4d(CUtensorMap* m, const void* ptr, const long long (&dims)[4], co
 namespace {
 
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
-cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const GemmParams& p,
-                   cudaStream_t s) {
+cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& md,
+                   const GemmParams& p, cudaStream_t s) {
   using C = GemmCfg<sizeof(T), BN>;
   auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT>;
   static bool configured = false;
@@ -84,11 +86,12 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorM
     configured = true;
   }
   const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
-  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, p);
+  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, md, p);
   return cudaGetLastError();
 }
 
 using bf16 = __nv_bfloat16;
+using f16 = __half;
 
 }  // namespace
 
@@ -137,14 +140,14 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   const int mn_box = bk;   // 128 bytes of the MN dimension
   bool ok;
   if (!c.a_mn)
-    ok = make_map(&ma, c.A, c.es, c.K, c.M, c.batch, c.lda, c.a_bs, bk, 128);
+    ok = make_map(&ma, c.A, c.es, c.K, c.M, c.batch, c.lda, c.a_bs, bk, 128, c.f16);
   else
-    ok = make_map(&ma, c.A, c.es, c.M, c.K, c.batch, c.lda, c.a_bs, mn_box, bk);
+    ok = make_map(&ma, c.A, c.es, c.M, c.K, c.batch, c.lda, c.a_bs, mn_box, bk, c.f16);
   if (!ok) return cudaErrorInvalidValue;
   if (!c.b_mn)
-    ok = make_map(&mb, c.B, c.es, c.K, c.N, c.batch, c.ldb, c.b_bs, bk, c.bn);
+    ok = make_map(&mb, c.B, c.es, c.K, c.N, c.batch, c.ldb, c.b_bs, bk, c.bn, c.f16);
   else
-    ok = make_map(&mb, c.B, c.es, c.N, c.K, c.batch, c.ldb, c.b_bs, mn_box, bk);
+    ok = make_map(&mb, c.B, c.es, c.N, c.K, c.batch, c.ldb, c.b_bs, mn_box, bk, c.f16);
   if (!ok) return cudaErrorInvalidValue;
 
   // Output written by TMA stores of 32-row x 128-byte boxes when the output's
@@ -167,16 +170,27 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   } else if (!(c.batch > 1 && p.splits > 1) && (c.out_es == 2 || c.out_es == 4)) {
     const long long n3 = p.splits > 1 ? p.splits : c.batch;
     const long long s3 = p.splits > 1 ? p.split_stride : p.out_bs;
-    if (make_map(&mc, p.out, c.out_es, c.N, c.M, n3, p.ldo, s3, 128 / c.out_es, 32)) p.tma_out = 1;
+    if (make_map(&mc, p.out, c.out_es, c.N, c.M, n3, p.ldo, s3, 128 / c.out_es, 32, c.out_f16)) p.tma_out = 1;
+  }
+  // optional fp16 copy of the output (plain batched layouts only)
+  CUtensorMap md;
+  p.tma_out2 = 0;
+  if (p.out2) {
+    if (c.epi == EPI_QKV || c.epi == EPI_LOGITS || p.splits > 1 || !p.tma_out) return cudaErrorInvalidValue;
+    if (!make_map(&md, p.out2, 2, c.N, c.M, c.batch, p.ldo, p.out_bs, 64, 32, true)) return cudaErrorInvalidValue;
+    p.tma_out2 = 1;
+  } else {
+    md = ma;   // unused by the kernel
   }
   // fp32 accumulation (out += acc) is done by TMA add-reduction only
   if (c.epi == EPI_ACC && !p.tma_out) return cudaErrorInvalidValue;
   if (!p.tma_out) mc = ma;   // unused by the kernel
 
-#define GPT_GEMM_CASE(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                       \
-  if (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ && \
-      c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_))                               \
-    return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, mc, p, stream);
+#define GPT_GEMM_CASE(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                        \
+  if (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ &&  \
+      c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_) && c.f16 == std::is_same<T_, f16>::value && \
+      c.out_f16 == std::is_same<OUT_, f16>::value && c.aux_f16 == std::is_same<AUX_, f16>::value)          \
+    return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, mc, md, p, stream);
 
   // forward
   GPT_GEMM_CASE(bf16, 256, false, true, EPI_QKV, bf16, bf16)
@@ -203,6 +217,10 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(float, 128, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, bf16, float)
+  // Newton-Schulz, fp16 steps (fp32 iterates with an fp16 operand copy)
+  GPT_GEMM_CASE(f16, 128, false, false, EPI_STORE, f16, f16)
+  GPT_GEMM_CASE(f16, 128, false, false, EPI_AXPBY, f16, f16)
+  GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, float, float)
   // fp8 e4m3 forward projections (operands as raw bytes)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_QKV, bf16, bf16)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_ACC, float, float)

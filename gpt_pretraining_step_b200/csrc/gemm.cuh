@@ -13,12 +13,35 @@
 // and returns with ERRF_TIMEOUT set in the error word.
 #pragma once
 
+#include <cuda_fp16.h>
+
 #include <type_traits>
 
 #include "common.cuh"
 #include "gemm_params.h"
 
 namespace gpt {
+
+// 16-bit epilogue storage: bf16 or fp16 (pairs packed low element first)
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (std::is_same<T, __half>::value) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    return pack_bf16x2(lo, hi);
+  }
+}
+template <typename T>
+__device__ __forceinline__ float lo16(uint32_t u) {
+  if constexpr (std::is_same<T, __half>::value) return __half2float(__ushort_as_half(static_cast<unsigned short>(u & 0xFFFFu)));
+  else return bf16_lo(u);
+}
+template <typename T>
+__device__ __forceinline__ float hi16(uint32_t u) {
+  if constexpr (std::is_same<T, __half>::value) return __half2float(__ushort_as_half(static_cast<unsigned short>(u >> 16)));
+  else return bf16_hi(u);
+}
 
 template <int ES, int BN>
 struct GemmCfg {
@@ -74,11 +97,11 @@ __device__ __forceinline__ void store_row32(OutT* dst, const float (&v)[32], int
     for (int g = 0; g < 4; ++g) {
       if (8 * g < nvalid) {
         uint4 w;
-        w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
-        w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
-        w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
-        w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
-        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + 8 * g) = w;
+        w.x = pack2<OutT>(v[8 * g + 0], v[8 * g + 1]);
+        w.y = pack2<OutT>(v[8 * g + 2], v[8 * g + 3]);
+        w.z = pack2<OutT>(v[8 * g + 4], v[8 * g + 5]);
+        w.w = pack2<OutT>(v[8 * g + 6], v[8 * g + 7]);
+        *reinterpret_cast<uint4*>(dst + 8 * g) = w;
       }
     }
   } else {
@@ -98,11 +121,11 @@ __device__ __forceinline__ void load_row32(const AuxT* src, float (&v)[32], int 
     for (int g = 0; g < 4; ++g) {
       uint4 w = make_uint4(0, 0, 0, 0);
       if (8 * g < nvalid)
-        w = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(src) + 8 * g);
-      v[8 * g + 0] = bf16_lo(w.x); v[8 * g + 1] = bf16_hi(w.x);
-      v[8 * g + 2] = bf16_lo(w.y); v[8 * g + 3] = bf16_hi(w.y);
-      v[8 * g + 4] = bf16_lo(w.z); v[8 * g + 5] = bf16_hi(w.z);
-      v[8 * g + 6] = bf16_lo(w.w); v[8 * g + 7] = bf16_hi(w.w);
+        w = *reinterpret_cast<const uint4*>(src + 8 * g);
+      v[8 * g + 0] = lo16<AuxT>(w.x); v[8 * g + 1] = hi16<AuxT>(w.x);
+      v[8 * g + 2] = lo16<AuxT>(w.y); v[8 * g + 3] = hi16<AuxT>(w.y);
+      v[8 * g + 4] = lo16<AuxT>(w.z); v[8 * g + 5] = hi16<AuxT>(w.z);
+      v[8 * g + 6] = lo16<AuxT>(w.w); v[8 * g + 7] = hi16<AuxT>(w.w);
     }
   } else {
 #pragma unroll
@@ -116,7 +139,9 @@ __device__ __forceinline__ void load_row32(const AuxT* src, float (&v)[32], int 
 
 template <typename OutT>
 __device__ __forceinline__ void store_scalar(OutT* dst, float x) {
-  if constexpr (sizeof(OutT) == 2)
+  if constexpr (std::is_same<OutT, __half>::value)
+    *reinterpret_cast<__half*>(dst) = __float2half_rn(x);
+  else if constexpr (sizeof(OutT) == 2)
     *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(x);
   else
     *reinterpret_cast<float*>(dst) = x;
@@ -152,10 +177,12 @@ __device__ __forceinline__ void logits_chunk(const float (&v)[32], int col0, int
 template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ GemmParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
+                   const __grid_constant__ GemmParams p) {
   constexpr int ES = sizeof(T);
   using C = GemmCfg<ES, BN>;
-  constexpr uint32_t IDESC = make_idesc(ES == 2 ? 1 : (ES == 4 ? 2 : 0), BN, A_MN, B_MN);
+  constexpr uint32_t IDESC =
+      make_idesc(ES == 2 ? (std::is_same<T, __half>::value ? 0 : 1) : (ES == 4 ? 2 : 0), BN, A_MN, B_MN);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -186,6 +213,7 @@ __global__ void __launch_bounds__(320, 1)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
     if (p.tma_out) tma_prefetch_desc(&tmC);
+    if (p.tma_out2) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -303,45 +331,51 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
     };
     auto box_put = [&](int u, uint4 w) { *reinterpret_cast<uint4*>(stg_row + ((u ^ stg_sw) << 4)) = w; };
-    auto box_close = [&](int col0, int row0, int z3) {
+    auto box_close = [&](const CUtensorMap* map, bool reduce, int col0, int row0, int z3) {
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0 && row0 < p.M && col0 < p.N) {
-        if constexpr (EPI == EPI_ACC)
-          tma_reduce_add_3d(&tmC, stg, col0, row0, z3);
+        if (reduce)
+          tma_reduce_add_3d(map, stg, col0, row0, z3);
         else
-          tma_store_3d(&tmC, stg, col0, row0, z3);
+          tma_store_3d(map, stg, col0, row0, z3);
         bulk_commit();
       }
     };
-    // 64 accumulator columns (two 32-column halves) to boxes: one bf16 box or two fp32 boxes
-    auto emit64 = [&](const float (&v0)[32], const float (&v1)[32], int col0, int row0, int z3) {
-      if constexpr (sizeof(OutT) == 2) {
+    // 64 accumulator columns (two 32-column halves) to boxes of type OT
+    // through `map`: one 16-bit box or two fp32 boxes
+    auto emit64_to = [&](auto tag, const CUtensorMap* map, bool reduce, const float (&v0)[32],
+                         const float (&v1)[32], int col0, int row0, int z3) {
+      using OT = decltype(tag);
+      if constexpr (sizeof(OT) == 2) {
         box_open();
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          box_put(u, make_uint4(pack_bf16x2(v0[8 * u], v0[8 * u + 1]), pack_bf16x2(v0[8 * u + 2], v0[8 * u + 3]),
-                                pack_bf16x2(v0[8 * u + 4], v0[8 * u + 5]), pack_bf16x2(v0[8 * u + 6], v0[8 * u + 7])));
+          box_put(u, make_uint4(pack2<OT>(v0[8 * u], v0[8 * u + 1]), pack2<OT>(v0[8 * u + 2], v0[8 * u + 3]),
+                                pack2<OT>(v0[8 * u + 4], v0[8 * u + 5]), pack2<OT>(v0[8 * u + 6], v0[8 * u + 7])));
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          box_put(4 + u, make_uint4(pack_bf16x2(v1[8 * u], v1[8 * u + 1]), pack_bf16x2(v1[8 * u + 2], v1[8 * u + 3]),
-                                    pack_bf16x2(v1[8 * u + 4], v1[8 * u + 5]),
-                                    pack_bf16x2(v1[8 * u + 6], v1[8 * u + 7])));
-        box_close(col0, row0, z3);
+          box_put(4 + u, make_uint4(pack2<OT>(v1[8 * u], v1[8 * u + 1]), pack2<OT>(v1[8 * u + 2], v1[8 * u + 3]),
+                                    pack2<OT>(v1[8 * u + 4], v1[8 * u + 5]), pack2<OT>(v1[8 * u + 6], v1[8 * u + 7])));
+        box_close(map, reduce, col0, row0, z3);
       } else {
         box_open();
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           box_put(u, make_uint4(__float_as_uint(v0[4 * u]), __float_as_uint(v0[4 * u + 1]),
                                 __float_as_uint(v0[4 * u + 2]), __float_as_uint(v0[4 * u + 3])));
-        box_close(col0, row0, z3);
+        box_close(map, reduce, col0, row0, z3);
         box_open();
 #pragma unroll
         for (int u = 0; u < 8; ++u)
           box_put(u, make_uint4(__float_as_uint(v1[4 * u]), __float_as_uint(v1[4 * u + 1]),
                                 __float_as_uint(v1[4 * u + 2]), __float_as_uint(v1[4 * u + 3])));
-        box_close(col0 + 32, row0, z3);
+        box_close(map, reduce, col0 + 32, row0, z3);
       }
+    };
+    // the main output (EPI_ACC adds into it)
+    auto emit64 = [&](const float (&v0)[32], const float (&v1)[32], int col0, int row0, int z3) {
+      emit64_to(OutT{}, &tmC, EPI == EPI_ACC, v0, v1, col0, row0, z3);
     };
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
@@ -408,15 +442,15 @@ __global__ void __launch_bounds__(320, 1)
                 box_open();
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                  box_put(u, make_uint4(pack_bf16x2(v0[8 * u], v0[8 * u + 1]), pack_bf16x2(v0[8 * u + 2], v0[8 * u + 3]),
-                                        pack_bf16x2(v0[8 * u + 4], v0[8 * u + 5]),
-                                        pack_bf16x2(v0[8 * u + 6], v0[8 * u + 7])));
+                  box_put(u, make_uint4(pack2<OutT>(v0[8 * u], v0[8 * u + 1]), pack2<OutT>(v0[8 * u + 2], v0[8 * u + 3]),
+                                        pack2<OutT>(v0[8 * u + 4], v0[8 * u + 5]),
+                                        pack2<OutT>(v0[8 * u + 6], v0[8 * u + 7])));
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                  box_put(4 + u, make_uint4(pack_bf16x2(v1[8 * u], v1[8 * u + 1]),
-                                            pack_bf16x2(v1[8 * u + 2], v1[8 * u + 3]),
-                                            pack_bf16x2(v1[8 * u + 4], v1[8 * u + 5]),
-                                            pack_bf16x2(v1[8 * u + 6], v1[8 * u + 7])));
+                  box_put(4 + u, make_uint4(pack2<OutT>(v1[8 * u], v1[8 * u + 1]),
+                                            pack2<OutT>(v1[8 * u + 2], v1[8 * u + 3]),
+                                            pack2<OutT>(v1[8 * u + 4], v1[8 * u + 5]),
+                                            pack2<OutT>(v1[8 * u + 6], v1[8 * u + 7])));
                 put_box(c * 32);
               } else if (row_ok) {
                 store_row32(dst + c * 32, v0, 32);
@@ -457,10 +491,10 @@ __global__ void __launch_bounds__(320, 1)
                 if (p.tma_out) {
 #pragma unroll
                   for (int u = 0; u < 4; ++u)
-                    box_put(4 * pc + u, make_uint4(pack_bf16x2(o[8 * u], o[8 * u + 1]),
-                                                   pack_bf16x2(o[8 * u + 2], o[8 * u + 3]),
-                                                   pack_bf16x2(o[8 * u + 4], o[8 * u + 5]),
-                                                   pack_bf16x2(o[8 * u + 6], o[8 * u + 7])));
+                    box_put(4 * pc + u, make_uint4(pack2<OutT>(o[8 * u], o[8 * u + 1]),
+                                                   pack2<OutT>(o[8 * u + 2], o[8 * u + 3]),
+                                                   pack2<OutT>(o[8 * u + 4], o[8 * u + 5]),
+                                                   pack2<OutT>(o[8 * u + 6], o[8 * u + 7])));
                 } else if (row_ok) {
                   store_row32(dst + part * 64 + pc * 32, o, 32);
                 }
@@ -548,8 +582,8 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                   if constexpr (sizeof(AT) == 2) {
-                    a[8 * g + 2 * e] = bf16_lo(w[e]);
-                    a[8 * g + 2 * e + 1] = bf16_hi(w[e]);
+                    a[8 * g + 2 * e] = lo16<AT>(w[e]);
+                    a[8 * g + 2 * e + 1] = hi16<AT>(w[e]);
                   } else {
                     a[4 * g + e] = __uint_as_float(w[e]);
                   }
@@ -575,6 +609,8 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           if (p.tma_out) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          // optional fp16 copy of the output in the same layout
+          if (p.tma_out2) emit64_to(__half{}, &tmD, false, v[0], v[1], nb * BN + c * 32, box_row0, z3);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int col0 = nb * BN + (c + hh) * 32;

@@ -11,7 +11,7 @@ namespace gpt {
 // D[z](m, n) = sum_k A[z](m, k) B[z](n, k), z < batch.
 //   A storage: a_mn ? [K][lda] (m contiguous) : [M][lda] (k contiguous); z stride a_bs
 //   B storage: b_mn ? [K][ldb] (n contiguous) : [N][ldb] (k contiguous); z stride b_bs
-//   es: operand element size, 2 = bf16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32),
+//   es: operand element size, 2 = bf16 or (f16) fp16 (kind::f16), 4 = fp32 read as tf32 (kind::tf32),
 //       1 = fp8 e4m3 (kind::f8f6f4; p.dq_a / p.dq_b dequantise the accumulator)
 //   out_es / aux_es: element sizes of the epilogue output and auxiliary input
 //   bn: 128 or 256 output columns per tile; splits: K split count (> 1 writes
@@ -28,6 +28,7 @@ struct GemmCall {
   int bn = 256, splits = 1;
   bool sym = false;
   int epi = 0, out_es = 4, aux_es = 4;
+  bool f16 = false, out_f16 = false, aux_f16 = false;   // 16-bit operands / output / aux are fp16, not bf16
   GemmParams p{};   // epilogue fields (out, ldo, aux, ...) filled by the caller
 };
 
@@ -40,12 +41,12 @@ int gemm_tiles(const GemmCall& c);
 
 int device_sm_count();
 
-// TMA descriptor of a bf16 (es = 2) or fp32 (es = 4) tensor [batch][outer][inner]
+// TMA descriptor of a bf16 (es = 2; fp16 with f16) or fp32 (es = 4) tensor [batch][outer][inner]
 // with row stride ld and batch stride bs (elements), 128-byte swizzle, box
 // box_inner x box_outer.  False if the driver entry point is missing or the
 // base/strides are not 16-byte aligned.
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
-              long long ld, long long bs, int box_inner, int box_outer);
+              long long ld, long long bs, int box_inner, int box_outer, bool f16 = false);
 
 // 4-D bf16 map, dims {d0 (innermost), d1, d2, d3}, byte strides of dims 1..3,
 // box {b0, b1, b2, b3}, 128-byte swizzle.

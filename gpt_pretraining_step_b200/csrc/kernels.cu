@@ -10,6 +10,9 @@
 #include "common.cuh"
 #include "kernels.cuh"
 
+#include <cuda_fp16.h>
+#include <type_traits>
+
 namespace gpt {
 
 namespace {
@@ -390,7 +393,13 @@ __global__ void muon_norm_kernel(const float* __restrict__ part, int nmat, float
 
 template <typename T>
 __device__ __forceinline__ void store4(T* p, float a, float b, float c, float d) {
-  if constexpr (sizeof(T) == 2) {
+  if constexpr (std::is_same<T, __half>::value) {
+    __half2 h0 = __floats2half2_rn(a, b), h1 = __floats2half2_rn(c, d);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&h0);
+    w.y = *reinterpret_cast<uint32_t*>(&h1);
+    *reinterpret_cast<uint2*>(p) = w;
+  } else if constexpr (sizeof(T) == 2) {
     uint2 w;
     w.x = pack_bf16x2(a, b);
     w.y = pack_bf16x2(c, d);
@@ -411,12 +420,14 @@ __device__ __forceinline__ float4 load4(const T* p) {
 }
 
 // From the momentum mom[z] (rows x cols): `same` = s_z mom[z] in the same
-// layout and `trans` = (s_z mom[z])^T (cols x rows), s_z = inv_norm[z]; either
-// output may be null.  One read of the momentum serves both.
-template <typename OutT>
+// layout and `trans` = (s_z mom[z])^T (cols x rows), s_z = inv_norm[z], in
+// storage type T1, and the same pair in T2; any output may be null.  One read
+// of the momentum serves all of them.
+template <typename T1, typename T2>
 __global__ void __launch_bounds__(256) muon_make_x_kernel(const float* __restrict__ mom,
-                                                          const float* __restrict__ inv_norm, OutT* __restrict__ same,
-                                                          OutT* __restrict__ trans, int rows, int cols) {
+                                                          const float* __restrict__ inv_norm, T1* __restrict__ same1,
+                                                          T1* __restrict__ trans1, T2* __restrict__ same2,
+                                                          T2* __restrict__ trans2, int rows, int cols) {
   __shared__ float tile[64][65];
   const int z = blockIdx.z;
   const float s = inv_norm[z];
@@ -425,6 +436,7 @@ __global__ void __launch_bounds__(256) muon_make_x_kernel(const float* __restric
   const int r0 = blockIdx.y * 64, c0 = blockIdx.x * 64;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   const int cc = c0 + 4 * tx;
+  const bool want_t = trans1 || trans2;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int rr = r0 + ty + 16 * k;
@@ -432,25 +444,30 @@ __global__ void __launch_bounds__(256) muon_make_x_kernel(const float* __restric
     if (rr < rows && cc < cols) {
       v = *reinterpret_cast<const float4*>(mz + static_cast<long long>(rr) * cols + cc);
       v.x *= s; v.y *= s; v.z *= s; v.w *= s;
-      if (same) store4(same + z * n + static_cast<long long>(rr) * cols + cc, v.x, v.y, v.z, v.w);
+      const long long o = z * n + static_cast<long long>(rr) * cols + cc;
+      if (same1) store4(same1 + o, v.x, v.y, v.z, v.w);
+      if (same2) store4(same2 + o, v.x, v.y, v.z, v.w);
     }
-    if (trans) {
+    if (want_t) {
       tile[ty + 16 * k][4 * tx] = v.x;
       tile[ty + 16 * k][4 * tx + 1] = v.y;
       tile[ty + 16 * k][4 * tx + 2] = v.z;
       tile[ty + 16 * k][4 * tx + 3] = v.w;
     }
   }
-  if (!trans) return;
+  if (!want_t) return;
   __syncthreads();
   // rows of the transpose are columns of the tile
   const int oc = r0 + 4 * tx;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int orow = c0 + ty + 16 * k, tc = ty + 16 * k;
-    if (orow < cols && oc < rows)
-      store4(trans + z * n + static_cast<long long>(orow) * rows + oc, tile[4 * tx][tc], tile[4 * tx + 1][tc],
-             tile[4 * tx + 2][tc], tile[4 * tx + 3][tc]);
+    if (orow < cols && oc < rows) {
+      const long long o = z * n + static_cast<long long>(orow) * rows + oc;
+      const float a = tile[4 * tx][tc], b = tile[4 * tx + 1][tc], c = tile[4 * tx + 2][tc], d = tile[4 * tx + 3][tc];
+      if (trans1) store4(trans1 + o, a, b, c, d);
+      if (trans2) store4(trans2 + o, a, b, c, d);
+    }
   }
 }
 
@@ -673,14 +690,14 @@ void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, flo
 }
 
 void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, void* trans, int out_es, int nmat,
-                        int rows, int cols, cudaStream_t s) {
+                        int rows, int cols, cudaStream_t s, __half* same16, __half* trans16) {
   const dim3 grid(cdiv(cols, 64), cdiv(rows, 64), nmat);
   if (out_es == 2)
-    muon_make_x_kernel<bf16><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<bf16*>(same), static_cast<bf16*>(trans),
-                                                  rows, cols);
+    muon_make_x_kernel<bf16, __half><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<bf16*>(same),
+                                                          static_cast<bf16*>(trans), same16, trans16, rows, cols);
   else
-    muon_make_x_kernel<float><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<float*>(same),
-                                                   static_cast<float*>(trans), rows, cols);
+    muon_make_x_kernel<float, __half><<<grid, 256, 0, s>>>(mom, inv_norm, static_cast<float*>(same),
+                                                           static_cast<float*>(trans), same16, trans16, rows, cols);
 }
 
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -57,8 +58,11 @@ void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, flo
                           float* inv_norm, void* ws, cudaStream_t s);
 
 // X[z] = mom[z] * inv_norm[z], stored [r][c] (transpose: mom is [c][r]); bf16 or fp32 out.
+// X = mom / ||mom|| per matrix (rows x cols as stored) into `same` (same
+// layout) and/or `trans` (transposed), both of element size out_es (2: bf16,
+// 4: fp32), and optionally fp16 copies same16 / trans16; null outputs are skipped.
 void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, void* trans, int out_es, int nmat,
-                        int rows, int cols, cudaStream_t s);
+                        int rows, int cols, cudaStream_t s, __half* same16 = nullptr, __half* trans16 = nullptr);
 
 // W[z] = W[z] (1 - lr wd) - lr * scale * X[z] (X is [r][c]; W is [c][r] when transpose).
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,

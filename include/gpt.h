@@ -71,11 +71,13 @@ enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
  *             pass (q|k|v, attention output, MLP up, MLP down) on fp8 e4m3
  *             operands with dynamic per-tensor scales (448 / amax of the
  *             tensor); attention, lm_head and the backward stay bf16
- *   ns_tf32_steps  how many of the five Newton-Schulz steps run with fp32
- *             operands on the tensor cores (kind::tf32) before switching
- *             to bf16; 0..5.  Three keep the update within 1% of fp64 on
- *             the decaying spectra real gradients have; bf16-only steps
- *             amplify rounding on small singular values (up to ~8%).
+ *   ns_tf32_steps  operand precision of the five Newton-Schulz steps:
+ *             -1 = fp16 operands at the full tensor rate with fp32 iterates
+ *             (the recommended setting); 0..5 = that many leading steps with
+ *             fp32 operands read as tf32 (half rate), the rest bf16.  fp16
+ *             operands keep the update within ~1% of fp64 on the decaying
+ *             spectra real gradients have, as three tf32 steps do; bf16-only
+ *             steps amplify rounding on small singular values (up to ~8%).
  *   seed      seed of the N(0, 0.02) initial weights drawn by gpt_init
  */
 typedef struct gpt_config {
@@ -251,8 +253,9 @@ int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void*
 
 /* Newton-Schulz (Polar Express, five steps) of a batch of fp32 matrices
  * G [batch, rows, cols] -> fp32 X of the same shape, via the same kernels
- * as muon_step; scratch is a device buffer of gpt_op_newton_schulz_scratch()
- * bytes. */
+ * as muon_step; tf32_steps selects the operand precision as ns_tf32_steps
+ * does (-1 = fp16 operands, 0..5 = leading tf32 steps then bf16); scratch
+ * is a device buffer of gpt_op_newton_schulz_scratch() bytes. */
 size_t gpt_op_newton_schulz_scratch(int batch, int rows, int cols);
 int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols, int tf32_steps, void* scratch,
                          void* stream);

@@ -44,7 +44,7 @@ def relfro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def build(torch, shape, params=None, ns_tf32_steps=3, lm_chunk_rows=0):
+def build(torch, shape, params=None, ns_tf32_steps=-1, lm_chunk_rows=0):
     import gpt_pretraining_step_b200 as g
     st = g.GPTStep(depth=shape.depth, batch=shape.batch, seq_len=shape.seq_len, vocab=shape.vocab,
                    d_model=shape.d_model, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows)
@@ -207,7 +207,7 @@ def test_adamw_step_matches_oracle(torch):
             assert np.abs(got - p[tid]).max() < 1e-6, (step, tid)
 
 
-@pytest.mark.parametrize("ns_tf32_steps", [3, 5])
+@pytest.mark.parametrize("ns_tf32_steps", [-1, 3, 5])
 def test_whole_step_matches_oracle(torch, ns_tf32_steps):
     import gpt_pretraining_step_b200 as g
     s = SMALL["tiny"]
