@@ -67,6 +67,13 @@ def peaks():
 
 # ------------------------------------------------------------------ FLOPs
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# categories that can dominate the d20 step, from one ncu capture of a whole
+# d20 step of the current kernels (profiles/dram_traffic_d20.md).  Used for the
+# roofline's `traffic` only on that workload; null elsewhere.
+NCU_TRAFFIC_D20 = {"dx_gemm": 503.2e6, "attn_bwd": 960.9e6, "dw_gemm": 10.01e9}
+
+
 def model_flops_per_token(s, causal=False):
     """PaLM-style model FLOPs per token: 6 N_matmul + 12 L d T (embeddings
     excluded); with causal=True the attention term counts only the half of the
@@ -316,9 +323,12 @@ def run_ours(a):
         if kind == "tensor":
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e12
             peak = pk["bf16_tflops_sustained"]
+            traffic = (NCU_TRAFFIC_D20.get(dominant)
+                       if a.config == "d20" and a.precision == "bf16" and a.ns_tf32_steps < 0 else None)
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
-                    "peak_source": f"{pk_src} bf16_tflops_sustained"}
+                    "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
+                    "peak_source": f"{pk_src} bf16_tflops_sustained",
+                    "traffic_source": "ncu dram bytes per launch, profiles/dram_traffic_d20.md" if traffic else None}
         else:
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e9
             peak = pk["hbm_gbs"]
