@@ -98,3 +98,73 @@ def test_adamw_constant_gradient_every_step():
         p_prev = p
         p, m, v = oo.adamw_step(p, g, m, v, t, lr=1e-2, eps=0.0)
         assert np.allclose(p - p_prev, -1e-2 * np.sign(g), atol=1e-13)
+
+
+# ---------------------------------------------------------------- NorMuon
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+@pytest.mark.parametrize("shape", [(16, 48), (48, 16), (24, 24)])
+def test_normuon_keeps_frobenius_norm(shape):
+    O = _rand(shape, 1)
+    V = np.abs(_rand((min(shape),) if shape[0] != shape[1] else (shape[0],), 2))
+    Op, _ = oo.normuon(O, V, 0.95)
+    assert abs(np.linalg.norm(Op) / np.linalg.norm(O) - 1) < 1e-12
+
+
+@pytest.mark.parametrize("shape", [(16, 48), (48, 16), (24, 24)])
+def test_normuon_without_memory_equalises_neurons(shape):
+    # beta2 = 0: V is this step's mean square, so every neuron of O' ends with
+    # the same mean square over the reduction axis
+    O = _rand(shape, 3) * np.linspace(0.1, 3.0, shape[1])[None, :] * np.linspace(0.5, 2.0, shape[0])[:, None]
+    Op, V = oo.normuon(O, np.zeros(min(shape) if shape[0] != shape[1] else shape[0]), 0.0)
+    ax = oo.normuon_axis(*shape)
+    ms = np.mean(Op * Op, axis=ax)
+    assert np.allclose(ms, ms.mean(), rtol=1e-12)
+    assert np.allclose(V, np.mean(O * O, axis=ax), rtol=1e-14)
+
+
+def test_normuon_is_identity_on_a_semi_orthogonal_update():
+    # rows of a semi-orthogonal O (r <= c) have equal norms: nothing to equalise
+    Q, _ = np.linalg.qr(_rand((40, 12), 4))
+    O = Q.T                               # 12 x 40, O O^T = I
+    Op, _ = oo.normuon(O, np.zeros(12), 0.95)
+    assert np.allclose(Op, O, atol=1e-12)
+
+
+def test_normuon_axis_follows_the_longer_side():
+    O = _rand((12, 40), 5)
+    V = np.abs(_rand((12,), 6))
+    a, Va = oo.normuon(O, V, 0.9)
+    b, Vb = oo.normuon(O.T, V, 0.9)
+    assert np.allclose(a, b.T, atol=1e-14) and np.allclose(Va, Vb, atol=1e-14)
+
+
+def test_normuon_second_moment_is_an_ema():
+    O1, O2 = _rand((8, 20), 7), _rand((8, 20), 8)
+    _, V1 = oo.normuon(O1, np.zeros(8), 0.9)
+    _, V2 = oo.normuon(O2, V1, 0.9)
+    m1, m2 = np.mean(O1 * O1, axis=1), np.mean(O2 * O2, axis=1)
+    assert np.allclose(V2, 0.9 * 0.1 * m1 + 0.1 * m2, rtol=1e-14)
+
+
+def test_normuon_scales_by_the_clamped_inverse_root():
+    # two neurons with V = 4 and V = 1: the second is doubled relative to the first
+    O = np.ones((2, 6))
+    Op, _ = oo.normuon(O, np.array([4.0, 1.0]), 1.0)   # beta2 = 1 keeps V
+    assert abs(Op[1, 0] / Op[0, 0] - 2.0) < 1e-12
+    # a vanishing second moment is clamped at 1e-10, not divided by zero
+    Oz, _ = oo.normuon(np.zeros((2, 6)), np.zeros(2), 0.5)
+    assert np.all(np.isfinite(Oz)) and np.all(Oz == 0)
+
+
+def test_muon_step_with_normuon_applies_it_after_newton_schulz():
+    G = _rand((16, 48), 9)
+    W = _rand((16, 48), 10) * 0.02
+    W1, mom, V = oo.muon_step(W, G, np.zeros_like(G), lr=0.02, normuon_V=np.zeros(16), normuon_beta2=0.95)
+    O = oo.newton_schulz(G)
+    Op, Vref = oo.normuon(O, np.zeros(16), 0.95)
+    assert np.allclose(W1, W - 0.02 * oo.muon_scale(16, 48) * Op, atol=1e-14)
+    assert np.allclose(V, Vref, atol=1e-16)
