@@ -47,6 +47,8 @@ def parse():
                     help="Newton-Schulz operand precision: -1 = fp16 (default), 0..5 = leading tf32 steps, then bf16")
     ap.add_argument("--precision", default="bf16", choices=["bf16", "fp8"],
                     help="fp8: forward block projections on e4m3 operands")
+    ap.add_argument("--normuon", type=float, default=None, metavar="BETA2",
+                    help="NorMuon variance reduction on the Muon updates with this second-moment decay")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="per-category device times in the JSON line")
@@ -268,7 +270,10 @@ def run_ours(a):
         st.fwd_bwd(tok, tgt)
         if grads is not None:
             dp.average_gradients(grads)
-        st.muon_step(*hp["muon"])
+        if a.normuon is None:
+            st.muon_step(*hp["muon"])
+        else:
+            st.muon_step_normuon(*hp["muon"], a.normuon)
         st.adamw_step(*hp["adam"])
 
     # warm-up; the last warm-up step records every launch category
@@ -373,7 +378,7 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
-            "config": {"workload": f"{a.config} GPT step (fwd+bwd+Muon+AdamW)", "global_batch": s.batch * world,
+            "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)", "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
                        "parallelism": f"dp{world}", "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
                        "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2"},
@@ -412,13 +417,16 @@ def run_e2e(a, st, s, rank, world, grads, stream):
     loss_host = torch.empty(1, dtype=torch.float32).pin_memory()
 
     def one():
-        if world == 1:
+        if world == 1 and a.normuon is None:
             return st.train_step_host(tok, tgt, hp)
         dtok.copy_(tok, non_blocking=True)
         dtgt.copy_(tgt, non_blocking=True)
         loss = st.fwd_bwd(dtok, dtgt)
         dp.average_gradients(grads)
-        st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)
+        if a.normuon is None:
+            st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)
+        else:
+            st.muon_step_normuon(hp.muon_lr, hp.muon_momentum, hp.muon_wd, a.normuon)
         st.adamw_step(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd)
         loss_host.copy_(loss.reshape(1), non_blocking=True)
         stream.synchronize()
@@ -432,6 +440,10 @@ def run_e2e(a, st, s, rank, world, grads, stream):
     dt = (time.perf_counter() - t0) / a.steps
     return {"value": s.tokens / dt, "unit": "tokens/s", "ms_per_step": dt * 1e3,
             "h2d_bytes_per_step": int(tok.numel() * 4 + tgt.numel() * 4), "d2h_bytes_per_step": 4}
+
+
+def optim_name(a):
+    return "Muon" if a.normuon is None else f"NorMuon(beta2={a.normuon})"
 
 
 def main():

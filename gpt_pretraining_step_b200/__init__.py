@@ -14,14 +14,14 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgpt.so")
 
 GPT_OK, GPT_EINVAL, GPT_ERANGE, GPT_ETIMEOUT, GPT_ECUDA = 0, -1, -2, -3, -4
-KIND_PARAM, KIND_GRAD, KIND_MOM, KIND_ADAM_M, KIND_ADAM_V = 0, 1, 2, 3, 4
+KIND_PARAM, KIND_GRAD, KIND_MOM, KIND_ADAM_M, KIND_ADAM_V, KIND_NORMUON_V = 0, 1, 2, 3, 4, 5
 GROUP_ADAMW, GROUP_MUON = 0, 1
 PROF_CATEGORIES = ["qkv_gemm", "proj_gemm", "fc_gemm", "down_gemm", "attn_fwd", "attn_bwd", "logits_gemm",
                    "ce_finish", "lm_dx_gemm", "lm_dw_gemm", "dx_gemm", "dw_gemm", "norm", "qk_bwd", "embed",
                    "ns_gemm", "muon_elem", "adamw", "fp8_quant"]
 
 ABI_FUNCTIONS = [
-    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "adamw_step", "gpt_train_step_host",
+    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "muon_step_normuon", "adamw_step", "gpt_train_step_host",
     "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
     "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3",
     "gpt_op_matmul_fp8", "gpt_op_attention_fwd",
@@ -66,6 +66,7 @@ def lib():
             "gpt_init": (i32, [ctypes.POINTER(Config), vp, vp, vp, vp, ctypes.POINTER(vp)]),
             "gpt_fwd_bwd": (i32, [vp, vp, vp, vp, i32]),
             "muon_step": (i32, [vp, f32, f32, f32]),
+            "muon_step_normuon": (i32, [vp, f32, f32, f32, f32]),
             "adamw_step": (i32, [vp, f32, f32, f32, f32, f32]),
             "gpt_train_step_host": (i32, [vp, vp, vp, ctypes.POINTER(HParams), vp]),
             "gpt_num_tensors": (i32, [vp]),
@@ -166,6 +167,9 @@ class GPTStep:
     def muon_step(self, lr=0.02, momentum=0.95, weight_decay=0.0):
         _check(lib().muon_step(self.h, lr, momentum, weight_decay))
 
+    def muon_step_normuon(self, lr=0.02, momentum=0.95, weight_decay=0.0, beta2=0.95):
+        _check(lib().muon_step_normuon(self.h, lr, momentum, weight_decay, beta2))
+
     def adamw_step(self, lr=3e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.0):
         _check(lib().adamw_step(self.h, lr, beta1, beta2, eps, weight_decay))
 
@@ -187,19 +191,22 @@ class GPTStep:
         _check(lib().gpt_tensor_info(self.h, tid, ctypes.byref(r), ctypes.byref(c), ctypes.byref(g)))
         return r.value, c.value, g.value
 
+    def _shape(self, tid, kind):
+        r, c, _ = self.tensor_info(tid)
+        return (self.d_model,) if kind == KIND_NORMUON_V else (r, c)
+
     def get(self, tid, kind=KIND_PARAM):
         import torch
-        r, c, _ = self.tensor_info(tid)
-        out = torch.empty((r, c), dtype=torch.float32, device=self.bufs[0].device)
+        out = torch.empty(self._shape(tid, kind), dtype=torch.float32, device=self.bufs[0].device)
         _check(lib().gpt_get_tensor(self.h, tid, kind, _ptr(out)))
         return out
 
     def set(self, tid, value, kind=KIND_PARAM):
         import torch
-        r, c, _ = self.tensor_info(tid)
+        shape = self._shape(tid, kind)
         v = torch.as_tensor(value, dtype=torch.float32).to(self.bufs[0].device).contiguous()
-        if tuple(v.shape) != (r, c):
-            raise ValueError(f"tensor {tid} has shape {(r, c)}, got {tuple(v.shape)}")
+        if tuple(v.shape) != shape:
+            raise ValueError(f"tensor {tid} has shape {shape}, got {tuple(v.shape)}")
         _check(lib().gpt_set_tensor(self.h, tid, kind, _ptr(v)))
         self.stream.synchronize()
 

@@ -48,12 +48,13 @@ struct Plan {
   size_t param_bytes;
   // state
   size_t g[6], mom[6], am[2], av[2];
+  size_t nv;            // NorMuon second moments: 4 groups x L matrices x d floats
   size_t state_bytes;
   // activations
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
   size_t xf, rf, z, stats, zt, row_loss, loss;
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
-  size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, rope, err, tok, tgt;
+  size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, rope, err, tok, tgt;
   size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
@@ -130,6 +131,7 @@ void make_plan(const Dims& D, Plan& P) {
     P.am[i] = sb.take(numel[i] * 4);
     P.av[i] = sb.take(numel[i] * 4);
   }
+  P.nv = sb.take(4 * L * d * 4);
   P.state_bytes = sb.off;
 
   // split-K plan of the lm_head input gradient (contraction over the vocabulary)
@@ -191,6 +193,7 @@ void make_plan(const Dims& D, Plan& P) {
   P.Bbuf = ab.take(2 * L * d * d * 4);
   P.inv_norm = ab.take(4 * L * 4);
   P.normws = ab.take(muon_norm_workspace(4 * D.L));
+  P.nfac = ab.take(2 * L * d * 4);
   P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
   P.tok = ab.take(M * 4);
@@ -284,6 +287,8 @@ struct gpt_ctx {
   bf16* Wb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wb[i]); }
   float* G(int i) const { return reinterpret_cast<float*>(sbuf + P.g[i]); }
   float* Mom(int i) const { return reinterpret_cast<float*>(sbuf + P.mom[i]); }
+  // NorMuon second moments of block group i (2..5): L vectors of d floats
+  float* NV(int i) const { return reinterpret_cast<float*>(sbuf + P.nv) + static_cast<size_t>(i - 2) * D.L * D.d; }
   template <typename T>
   T* A(size_t off) const { return reinterpret_cast<T*>(abuf + off); }
   int* err() const { return A<int>(P.err); }
@@ -842,7 +847,9 @@ int gpt_fwd_bwd(gpt_ctx* c, const int32_t* tokens, const int32_t* targets, float
   return forward_backward(c, tokens, targets, loss_out, accumulate != 0);
 }
 
-int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
+// Muon over every block matrix; with normuon the orthogonalised updates get
+// the NorMuon per-neuron scaling (second-moment EMA with factor beta2) first.
+static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay, bool normuon, float beta2) {
   int rc = check_ctx(c);
   if (rc) return rc;
   const Dims& D = c->D;
@@ -895,6 +902,15 @@ int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
     rc = newton_schulz(c, bt.nz, d, bt.cc, X0, X1, XT0, XT1, Ab, Bb, D.n_tf32, s, c->err(), &res, &res_es,
                        &c->launches);
     if (rc) return rc;
+    // NorMuon: one factor per row of res (the shorter axis of every matrix);
+    // the members of a batch have contiguous second-moment vectors
+    float* rowf = nullptr;
+    if (normuon) {
+      ProfScope ps(c, GPT_PROF_MUON_ELEM);
+      rowf = c->A<float>(P.nfac);
+      launch_normuon_factor(res, res_es, bt.nz, d, bt.cc, c->NV(bt.m[0].grp), beta2, rowf, s);
+      c->launches += 2;
+    }
     for (int i = 0; i < bt.nm; ++i) {
       ProfScope ps(c, GPT_PROF_MUON_ELEM);
       const Member& mm = bt.m[i];
@@ -903,12 +919,21 @@ int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
       const float scale = sqrtf(std::max(1.f, static_cast<float>(rows) / static_cast<float>(cols)));
       const void* src = static_cast<const uint8_t*>(res) + static_cast<size_t>(i) * L * per * res_es;
       launch_muon_apply(c->W(mm.grp), c->Wb(mm.grp), src, res_es, L, d, bt.cc, mm.transpose, lr, weight_decay,
-                        scale, s);
+                        scale, s, rowf ? rowf + static_cast<size_t>(i) * L * d : nullptr);
       c->launches += 1;
     }
   }
   GPT_CK(cudaGetLastError());
   return GPT_OK;
+}
+
+int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
+  return muon_update(c, lr, momentum, weight_decay, false, 0.f);
+}
+
+int muon_step_normuon(gpt_ctx* c, float lr, float momentum, float weight_decay, float beta2) {
+  if (!(beta2 >= 0.f && beta2 < 1.f)) return fail(GPT_EINVAL, "NorMuon beta2 must be in [0, 1)");
+  return muon_update(c, lr, momentum, weight_decay, true, beta2);
 }
 
 int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay) {
@@ -983,6 +1008,16 @@ static int tensor_ptr(gpt_ctx* c, int id, int kind, float** p, size_t* n, int* g
       if (grp >= 2) return fail(GPT_EINVAL, "AdamW moments exist only for the embedding and lm_head");
       base = reinterpret_cast<float*>(c->sbuf + (kind == GPT_KIND_ADAM_M ? c->P.am[grp] : c->P.av[grp]));
       break;
+    case GPT_KIND_NORMUON_V: {
+      // one d-vector per matrix (its shorter axis): layer l's is the l-th
+      if (grp < 2) return fail(GPT_EINVAL, "NorMuon state exists only for block matrices");
+      const size_t l = off / (static_cast<size_t>(r) * cc);
+      *p = c->NV(grp) + l * c->D.d;
+      *n = static_cast<size_t>(c->D.d);
+      *grp_out = grp;
+      *off_out = off;
+      return GPT_OK;
+    }
     default:
       return fail(GPT_EINVAL, "unknown tensor kind");
   }

@@ -471,12 +471,81 @@ __global__ void __launch_bounds__(256) muon_make_x_kernel(const float* __restric
   }
 }
 
+// NorMuon ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "2. Optimizador
+// Muon", NorMuon variance reduction).  The orthogonalised update X[z] is held
+// with its shorter axis as rows (r <= c), so the per-neuron second moment is a
+// mean over each row.  First pass: the sum of squares of every row, one warp
+// per row (c is a multiple of 4).
+template <typename XT>
+__global__ void __launch_bounds__(256) row_sumsq_kernel(const XT* __restrict__ X, int r, int c,
+                                                        float* __restrict__ out) {
+  const int z = blockIdx.y;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= r) return;
+  const XT* xr = X + (static_cast<long long>(z) * r + row) * c;
+  float acc = 0.f;
+  for (int j = 4 * lane; j < c; j += 128) {
+    const float4 u = load4(xr + j);
+    acc = fmaf(u.x, u.x, acc);
+    acc = fmaf(u.y, u.y, acc);
+    acc = fmaf(u.z, u.z, acc);
+    acc = fmaf(u.w, u.w, acc);
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) out[static_cast<long long>(z) * r + row] = acc;
+}
+
+// Second pass, one block per matrix: v_mean = sumsq / c;
+// V <- beta2 V + (1 - beta2) v_mean; s = max(V, 1e-10)^(-1/2); the factor
+// f = s * ||v_mean||^(1/2) / max(||v_mean s^2||^(1/2), 1e-10) (sums over the
+// rows) keeps the Frobenius norm of the update.  f overwrites the sums.
+__global__ void __launch_bounds__(1024) normuon_factor_kernel(float* __restrict__ ss_f, float* __restrict__ V, int r,
+                                                              int c, float beta2) {
+  __shared__ float red[2][32];
+  const int z = blockIdx.x;
+  float* sf = ss_f + static_cast<long long>(z) * r;
+  float* v = V + static_cast<long long>(z) * r;
+  const float inv_c = 1.f / static_cast<float>(c);
+  float sum_m = 0.f, sum_ms = 0.f;
+  for (int i = threadIdx.x; i < r; i += blockDim.x) {
+    const float m = sf[i] * inv_c;
+    const float vn = fmaf(beta2, v[i], (1.f - beta2) * m);
+    v[i] = vn;
+    const float vc = fmaxf(vn, 1e-10f);
+    sum_m += m;
+    sum_ms += m / vc;
+  }
+  sum_m = warp_sum(sum_m);
+  sum_ms = warp_sum(sum_ms);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    red[0][w] = sum_m;
+    red[1][w] = sum_ms;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    float a = lane < nw ? red[0][lane] : 0.f, b = lane < nw ? red[1][lane] : 0.f;
+    a = warp_sum(a);
+    b = warp_sum(b);
+    if (lane == 0) {
+      red[0][0] = a;
+      red[1][0] = b;
+    }
+  }
+  __syncthreads();
+  const float ratio = sqrtf(red[0][0]) / fmaxf(sqrtf(red[1][0]), 1e-10f);
+  for (int i = threadIdx.x; i < r; i += blockDim.x) sf[i] = ratio / sqrtf(fmaxf(v[i], 1e-10f));
+}
+
 // W[z] <- decay W[z] - step U with U = X[z] (r x c, W in the same layout) or
-// U = X[z]^T (W is c x r); also refreshes the bf16 working copy.
+// U = X[z]^T (W is c x r); also refreshes the bf16 working copy.  With rowf,
+// row i of X[z] is first scaled by rowf[z r + i] (the NorMuon factor).
 template <typename XT>
 __global__ void __launch_bounds__(256) muon_apply_kernel(float* __restrict__ W, bf16* __restrict__ Wb,
-                                                         const XT* __restrict__ X, int r, int c, int transpose,
-                                                         float decay, float step) {
+                                                         const XT* __restrict__ X, const float* __restrict__ rowf,
+                                                         int r, int c, int transpose, float decay, float step) {
   __shared__ float tile[64][65];
   const int z = blockIdx.z;
   const long long n = static_cast<long long>(r) * c;
@@ -499,7 +568,12 @@ __global__ void __launch_bounds__(256) muon_apply_kernel(float* __restrict__ W, 
       const int rr = r0 + ty + 16 * k;
       if (rr < r && cc < c) {
         const long long o = static_cast<long long>(rr) * c + cc;
-        update(o, load4(xz + o));
+        float4 u = load4(xz + o);
+        if (rowf) {
+          const float f = rowf[static_cast<long long>(z) * r + rr];
+          u.x *= f; u.y *= f; u.z *= f; u.w *= f;
+        }
+        update(o, u);
       }
     }
     return;
@@ -508,7 +582,13 @@ __global__ void __launch_bounds__(256) muon_apply_kernel(float* __restrict__ W, 
   for (int k = 0; k < 4; ++k) {
     const int rr = r0 + ty + 16 * k;
     float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (rr < r && cc < c) u = load4(xz + static_cast<long long>(rr) * c + cc);
+    if (rr < r && cc < c) {
+      u = load4(xz + static_cast<long long>(rr) * c + cc);
+      if (rowf) {
+        const float f = rowf[static_cast<long long>(z) * r + rr];
+        u.x *= f; u.y *= f; u.z *= f; u.w *= f;
+      }
+    }
     tile[ty + 16 * k][4 * tx] = u.x;
     tile[ty + 16 * k][4 * tx + 1] = u.y;
     tile[ty + 16 * k][4 * tx + 2] = u.z;
@@ -701,13 +781,26 @@ void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, voi
 }
 
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
-                       float lr, float wd, float scale, cudaStream_t s) {
+                       float lr, float wd, float scale, cudaStream_t s, const float* rowf) {
   const dim3 grid(cdiv(c, 64), cdiv(r, 64), nmat);
   const float decay = 1.f - lr * wd, step = lr * scale;
   if (x_es == 2)
-    muon_apply_kernel<bf16><<<grid, 256, 0, s>>>(W, Wb, static_cast<const bf16*>(X), r, c, transpose, decay, step);
+    muon_apply_kernel<bf16><<<grid, 256, 0, s>>>(W, Wb, static_cast<const bf16*>(X), rowf, r, c, transpose, decay,
+                                                 step);
   else
-    muon_apply_kernel<float><<<grid, 256, 0, s>>>(W, Wb, static_cast<const float*>(X), r, c, transpose, decay, step);
+    muon_apply_kernel<float><<<grid, 256, 0, s>>>(W, Wb, static_cast<const float*>(X), rowf, r, c, transpose, decay,
+                                                  step);
+}
+
+void launch_normuon_factor(const void* X, int x_es, int nmat, int r, int c, float* V, float beta2, float* ws,
+                           cudaStream_t s) {
+  if (nmat <= 0 || r <= 0) return;
+  const dim3 grid(cdiv(r, 8), nmat);
+  if (x_es == 2)
+    row_sumsq_kernel<bf16><<<grid, 256, 0, s>>>(static_cast<const bf16*>(X), r, c, ws);
+  else
+    row_sumsq_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(X), r, c, ws);
+  normuon_factor_kernel<<<nmat, 1024, 0, s>>>(ws, V, r, c, beta2);
 }
 
 void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* amax_bits, uint8_t* q, float* inv,

@@ -64,9 +64,16 @@ void launch_muon_momentum(float* mom, const float* g, long long n, int nmat, flo
 void launch_muon_make_x(const float* mom, const float* inv_norm, void* same, void* trans, int out_es, int nmat,
                         int rows, int cols, cudaStream_t s, __half* same16 = nullptr, __half* trans16 = nullptr);
 
-// W[z] = W[z] (1 - lr wd) - lr * scale * X[z] (X is [r][c]; W is [c][r] when transpose).
+// W[z] = W[z] (1 - lr wd) - lr * scale * diag(rowf[z]) X[z] (X is [r][c]; W is
+// [c][r] when transpose; rowf null = no row factor).
 void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, int r, int c, bool transpose,
-                       float lr, float wd, float scale, cudaStream_t s);
+                       float lr, float wd, float scale, cudaStream_t s, const float* rowf = nullptr);
+
+// NorMuon row factors of nmat orthogonalised updates X[z] ([r][c], r <= c,
+// element size x_es): updates the second-moment EMA V[z] (r floats each) and
+// leaves the factor of row i of X[z] in ws[z r + i] (ws: nmat * r floats).
+void launch_normuon_factor(const void* X, int x_es, int nmat, int r, int c, float* V, float beta2, float* ws,
+                           cudaStream_t s);
 
 // Per-tensor e4m3 quantisation of nmat matrices of n bf16 values each (z-th at
 // x + z n): q = e4m3(x * 448 / amax) with round-to-nearest-even and saturation,

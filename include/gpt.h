@@ -54,7 +54,9 @@ enum {
   GPT_KIND_GRAD = 1,   /* fp32 gradient of the mean loss */
   GPT_KIND_MOM = 2,    /* Muon momentum (block matrices only) */
   GPT_KIND_ADAM_M = 3, /* AdamW first moment (embedding, lm_head only) */
-  GPT_KIND_ADAM_V = 4  /* AdamW second moment (embedding, lm_head only) */
+  GPT_KIND_ADAM_V = 4, /* AdamW second moment (embedding, lm_head only) */
+  GPT_KIND_NORMUON_V = 5 /* NorMuon second moment (block matrices only): d
+                          * floats, one per index of the shorter axis */
 };
 
 /* Optimizer group reported by gpt_tensor_info. */
@@ -124,6 +126,20 @@ int gpt_fwd_bwd(gpt_ctx* ctx, const int32_t* tokens, const int32_t* targets, flo
  * - lr * sqrt(max(1, rows / cols)) * X.  Refreshes the bf16 copies. */
 int muon_step(gpt_ctx* ctx, float lr, float momentum, float weight_decay);
 
+/* muon_step with the NorMuon variance reduction ("¿Cómo Entrenar Tu Propio
+ * ChatGPT por $50?", section "2. Optimizador Muon", NorMuon snippet) applied
+ * to each orthogonalised update X [rows, cols] before the weight update:
+ *   v_mean = mean of X^2 over the longer axis (the columns when square), one
+ *            value per index of the shorter axis (d values per matrix)
+ *   V      = beta2 V + (1 - beta2) v_mean   (GPT_KIND_NORMUON_V; zero at init)
+ *   s      = max(V, 1e-10)^(-1/2)
+ *   X     <- X * s (along the shorter axis) * sqrt(sum v_mean)
+ *            / max(sqrt(sum v_mean s^2), 1e-10)
+ * so the update keeps its Frobenius norm.  beta2 outside [0, 1) is
+ * GPT_EINVAL.  The page's snippet leaves the reduction axis and the second
+ * norm undefined; the reading above is the one this library implements. */
+int muon_step_normuon(gpt_ctx* ctx, float lr, float momentum, float weight_decay, float beta2);
+
 /* AdamW update of the token embedding and lm_head with bias correction
  * (the step count is kept in the context) and decoupled weight decay. */
 int adamw_step(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay);
@@ -145,7 +161,8 @@ int gpt_train_step_host(gpt_ctx* ctx, const int32_t* tokens_host, const int32_t*
 int gpt_num_tensors(const gpt_ctx* ctx);
 int gpt_tensor_info(const gpt_ctx* ctx, int id, int32_t* rows, int32_t* cols, int32_t* group);
 
-/* Device-to-device copies of rows*cols fp32 values (asynchronous). */
+/* Device-to-device copies of rows*cols fp32 values (asynchronous); d values
+ * for GPT_KIND_NORMUON_V. */
 int gpt_get_tensor(gpt_ctx* ctx, int id, int kind, float* dst);
 int gpt_set_tensor(gpt_ctx* ctx, int id, int kind, const float* src);
 

@@ -85,6 +85,7 @@ def test_null_arguments_are_einval(L):
     import gpt_pretraining_step_b200 as g
     assert L.gpt_fwd_bwd(None, None, None, None, 0) == g.GPT_EINVAL
     assert L.muon_step(None, 0.02, 0.95, 0.0) == g.GPT_EINVAL
+    assert L.muon_step_normuon(None, 0.02, 0.95, 0.0, 0.95) == g.GPT_EINVAL
     assert L.adamw_step(None, 1e-3, 0.8, 0.95, 1e-10, 0.0) == g.GPT_EINVAL
     assert L.gpt_check(None) == g.GPT_EINVAL
     assert L.gpt_num_tensors(None) == 0

@@ -186,6 +186,92 @@ def test_muon_step_matches_oracle(torch, name):
         assert np.allclose(f64(st.get(tid, g.KIND_MOM)), mom_ref, rtol=1e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("ns_tf32_steps", [-1, 5])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_normuon_two_steps_match_oracle(torch, name, ns_tf32_steps):
+    """Two NorMuon steps (the second exercises the second-moment EMA) against
+    the oracle chain: each step's update, the momentum and the state V."""
+    import gpt_pretraining_step_b200 as g
+    s = SMALL[name]
+    params = syn.init_params(s, seed=7)
+    st = build(torch, s, params, ns_tf32_steps=ns_tf32_steps)
+    specs = syn.param_specs(s)
+    lr, mom, wd, beta2 = 0.02, 0.95, 0.01, 0.9
+    W = {p: params[p].astype(np.float64) for p, *_r in specs}
+    M = {p: np.zeros((r, c)) for p, r, c, _g in specs}
+    V = {p: np.zeros(min(r, c)) for p, r, c, _g in specs}
+    for step in range(2):
+        W_before = {tid: f64(st.get(tid, g.KIND_PARAM)) for tid in range(len(specs))}
+        G = {}
+        for tid, (pname, r, c, grp) in enumerate(specs):
+            if grp == "muon":
+                G[pname] = syn.gaussian((r, c), seed=300 + 10 * step + tid)
+                st.set(tid, G[pname], kind=g.KIND_GRAD)
+        st.muon_step_normuon(lr, mom, wd, beta2)
+        st.check()
+        for tid, (pname, r, c, grp) in enumerate(specs):
+            if grp != "muon":
+                continue
+            W_prev = W[pname]
+            W[pname], M[pname], V[pname] = oo.muon_step(W_prev, G[pname], M[pname], lr, mom, wd,
+                                                        normuon_V=V[pname], normuon_beta2=beta2)
+            got = f64(st.get(tid, g.KIND_PARAM))
+            err = relfro(got - W_before[tid], W[pname] - W_prev)
+            assert err <= MUON_RELFRO, (step, pname, err)
+            assert np.allclose(f64(st.get(tid, g.KIND_MOM)), M[pname], rtol=1e-6, atol=1e-7)
+            v_got = f64(st.get(tid, g.KIND_NORMUON_V))
+            assert v_got.shape == V[pname].shape
+            assert relfro(v_got, V[pname]) <= 2 * MUON_RELFRO, (step, pname)
+
+
+def test_normuon_state_roundtrip_and_preset(torch):
+    """A preset nonzero V enters the EMA; plain Muon leaves V untouched."""
+    import gpt_pretraining_step_b200 as g
+    s = SMALL["ragged"]
+    params = syn.init_params(s, seed=8)
+    st = build(torch, s, params)
+    specs = syn.param_specs(s)
+    rng = np.random.default_rng(9)
+    V0, G = {}, {}
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if grp != "muon":
+            continue
+        V0[pname] = rng.uniform(1e-5, 1e-3, size=min(r, c))
+        st.set(tid, V0[pname], kind=g.KIND_NORMUON_V)
+        assert np.array_equal(f64(st.get(tid, g.KIND_NORMUON_V)), V0[pname].astype(np.float32))
+        G[pname] = syn.gaussian((r, c), seed=400 + tid)
+        st.set(tid, G[pname], kind=g.KIND_GRAD)
+    st.muon_step(0.02, 0.95, 0.0)
+    st.check()
+    for tid, (pname, *_r) in enumerate(specs):
+        if pname in V0:
+            assert np.array_equal(f64(st.get(tid, g.KIND_NORMUON_V)), V0[pname].astype(np.float32))
+    # reset the momentum and weights, then one NorMuon step from the preset V
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if pname in V0:
+            st.set(tid, params[pname])
+            st.set(tid, np.zeros((r, c)), kind=g.KIND_MOM)
+    st.muon_step_normuon(0.02, 0.95, 0.0, 0.5)
+    st.check()
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if pname not in V0:
+            continue
+        W0 = params[pname].astype(np.float64)
+        V0f = V0[pname].astype(np.float32).astype(np.float64)
+        W_ref, _, V_ref = oo.muon_step(W0, G[pname], np.zeros((r, c)), 0.02, 0.95, 0.0, normuon_V=V0f,
+                                       normuon_beta2=0.5)
+        assert relfro(f64(st.get(tid, g.KIND_PARAM)) - W0, W_ref - W0) <= MUON_RELFRO, pname
+        assert relfro(f64(st.get(tid, g.KIND_NORMUON_V)), V_ref) <= 2 * MUON_RELFRO, pname
+
+
+def test_normuon_rejects_bad_beta2(torch):
+    import gpt_pretraining_step_b200 as g
+    st = build(torch, SMALL["tiny"])
+    for b in (1.0, -0.1, float("nan")):
+        with pytest.raises(g.GptError):
+            st.muon_step_normuon(0.02, 0.95, 0.0, b)
+
+
 def test_adamw_step_matches_oracle(torch):
     import gpt_pretraining_step_b200 as g
     s = SMALL["ragged"]
