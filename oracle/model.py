@@ -18,7 +18,11 @@ Readings where the pages are silent (shared with the CUDA path):
     within the row.
   * QK norm: per-head gain-free RMSNorm applied after RoPE (the order does
     not matter mathematically: a rotation keeps the RMS).
-  * attention scale 1/sqrt(hd); n_kv_head = n_head; full causal window.
+  * attention scale 1/sqrt(hd); n_kv_head = n_head.
+  * attention window per layer: full causal by default; with a layer pattern
+    such as "SSSL" (section "1. Modelo GPT", sliding-window attention) the
+    pattern is repeated over the layers, S = a sliding window of
+    `short_window` earlier tokens, L = full causal.
   * weights are [in, out]; the fused projection's columns are q | k | v and
     head h owns columns h*hd .. h*hd+hd-1 of each.
 
@@ -90,6 +94,53 @@ def causal_attention_bwd(dy, q, k, v, p):
     return dq, dk, dv
 
 
+def attention_hidden(T, window=None):
+    """[T, T] boolean mask, True where key j is hidden from query t: j > t
+    (causal) or, with a sliding window of `window` earlier tokens, j < t - window
+    (so query t sees keys t - window .. t)."""
+    t = np.arange(T)[:, None]
+    j = np.arange(T)[None, :]
+    hidden = j > t
+    if window is not None:
+        hidden = hidden | (j < t - window)
+    return hidden
+
+
+def kv_for_queries(a, n_head):
+    """[B, Hkv, T, hd] -> [B, n_head, T, hd]: query head h reads kv head
+    h // (n_head / Hkv) (grouped-query attention; Hkv = n_head is plain
+    multi-head attention)."""
+    hkv = a.shape[1]
+    if n_head % hkv:
+        raise ValueError(f"{n_head} query heads do not split into {hkv} kv groups")
+    return np.repeat(a, n_head // hkv, axis=1)
+
+
+def attention(q, k, v, window=None):
+    """Causal attention with optional sliding window and grouped kv heads
+    ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "1. Modelo GPT":
+    GQA and sliding-window attention, e.g. the "SSSL" layer pattern).
+    q [B, H, T, hd]; k, v [B, Hkv, T, hd]; returns (y [B, H, T, hd], P)."""
+    hd, T, H = q.shape[-1], q.shape[-2], q.shape[1]
+    kq, vq = kv_for_queries(k, H), kv_for_queries(v, H)
+    s = np.matmul(q, np.swapaxes(kq, -1, -2)) / np.sqrt(hd)
+    s = np.where(attention_hidden(T, window), -np.inf, s)
+    s = s - np.max(s, axis=-1, keepdims=True)
+    p = np.exp(s)
+    p = p / np.sum(p, axis=-1, keepdims=True)
+    return np.matmul(p, vq), p
+
+
+def attention_bwd(dy, q, k, v, p):
+    """(dq, dk, dv) of attention(); dk and dv add up the query heads that
+    share each kv head."""
+    B, H, T, hd = q.shape
+    hkv = k.shape[1]
+    dq, dkq, dvq = causal_attention_bwd(dy, q, kv_for_queries(k, H), kv_for_queries(v, H), p)
+    g = H // hkv
+    return dq, dkq.reshape(B, hkv, g, T, hd).sum(axis=2), dvq.reshape(B, hkv, g, T, hd).sum(axis=2)
+
+
 def logsumexp(z):
     m = np.max(z, axis=-1, keepdims=True)
     return (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))[..., 0]
@@ -106,11 +157,23 @@ def _merge_heads(a):
     return a.transpose(0, 2, 1, 3).reshape(B * T, H * hd)
 
 
-def forward(params, tok, tgt, n_layer, head_dim=128, keep=True):
+def layer_windows(pattern, short_window, n_layer):
+    """Window of every layer: pattern[l % len(pattern)] is "S" (sliding window
+    of short_window earlier tokens) or "L" (full causal, None); an empty
+    pattern leaves every layer full causal."""
+    if not pattern:
+        return [None] * n_layer
+    if set(pattern) - {"S", "L"}:
+        raise ValueError(f"window pattern {pattern!r} may hold only S and L")
+    return [short_window if pattern[l % len(pattern)] == "S" else None for l in range(n_layer)]
+
+
+def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
     """Loss (and the saved activations) of one batch.
 
     params: dict of fp64-castable [in, out] matrices (wte is [V, d]).
     tok, tgt: int arrays [B, T].
+    windows: per-layer attention window (None = full causal), see layer_windows.
     """
     B, T = tok.shape
     wte = np.asarray(params["wte"], dtype=np.float64)
@@ -130,7 +193,7 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True):
         v = _split_heads(qkv[:, 2 * d:], B, T, H, head_dim)
         qn, rq = rms_norm(rope(q, cos, sin))
         kn, rk = rms_norm(rope(k, cos, sin))
-        y, P = causal_attention(qn, kn, v)
+        y, P = attention(qn, kn, v, None if windows is None else windows[l])
         ym = _merge_heads(y)
         x = x + ym @ W["c_proj"]
         xn2, r2 = rms_norm(x)
@@ -179,7 +242,7 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
         # attention: x_mid = x_in + attn(rms(x_in)) Wo
         grads[f"h{l}.c_proj"] = a["ym"].T @ dx
         dy = _split_heads(dx @ W["c_proj"].T, B, T, H, head_dim)
-        dqn, dkn, dv = causal_attention_bwd(dy, a["qn"], a["kn"], a["v"], a["P"])
+        dqn, dkn, dv = attention_bwd(dy, a["qn"], a["kn"], a["v"], a["P"])
         dq = rope_bwd(rms_norm_bwd(dqn, a["qn"], a["rq"]), cos, sin)
         dk = rope_bwd(rms_norm_bwd(dkn, a["kn"], a["rk"]), cos, sin)
         dqkv = np.concatenate([_merge_heads(dq), _merge_heads(dk), _merge_heads(dv)], axis=1)
@@ -192,6 +255,6 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
     return grads
 
 
-def fwd_bwd(params, tok, tgt, n_layer, head_dim=128):
-    loss, cache = forward(params, tok, tgt, n_layer, head_dim)
+def fwd_bwd(params, tok, tgt, n_layer, head_dim=128, windows=None):
+    loss, cache = forward(params, tok, tgt, n_layer, head_dim, windows=windows)
     return loss, backward(params, tok, tgt, cache, n_layer, head_dim), cache

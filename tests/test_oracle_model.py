@@ -171,8 +171,8 @@ def test_rmsnorm_invariants():
 
 # --- finite differences --------------------------------------------------------
 
-def _fd_check(p, tok, tgt, depth, names, n_coords=6, h=1e-5, seed=0):
-    loss, g, _ = om.fwd_bwd(p, tok, tgt, depth)
+def _fd_check(p, tok, tgt, depth, names, n_coords=6, h=1e-5, seed=0, windows=None):
+    loss, g, _ = om.fwd_bwd(p, tok, tgt, depth, windows=windows)
     rng = np.random.default_rng(seed)
     worst = 0.0
     for name in names:
@@ -191,9 +191,9 @@ def _fd_check(p, tok, tgt, depth, names, n_coords=6, h=1e-5, seed=0):
                        for _ in range(n_coords - len(coords))]
         for (i, j) in coords:
             pp = dict(p); Wp = W.copy(); Wp[i, j] += h; pp[name] = Wp
-            lp, _ = om.forward(pp, tok, tgt, depth, keep=False)
+            lp, _ = om.forward(pp, tok, tgt, depth, keep=False, windows=windows)
             Wm = W.copy(); Wm[i, j] -= h; pp[name] = Wm
-            lm, _ = om.forward(pp, tok, tgt, depth, keep=False)
+            lm, _ = om.forward(pp, tok, tgt, depth, keep=False, windows=windows)
             fd = (lp - lm) / (2 * h)
             err = abs(fd - G[i, j]) / scale
             worst = max(worst, err)
@@ -230,3 +230,105 @@ def test_embedding_forward_is_row_copy():
     x0 = p["wte"][tok.reshape(-1)].astype(np.float64)
     xf, _ = om.rms_norm(x0)
     assert np.array_equal(c["xf"], xf)
+
+
+# --- sliding window and grouped kv heads -------------------------------------
+#
+# Section "1. Modelo GPT" lists GQA (fewer kv heads than query heads) and
+# sliding-window attention with a layer pattern such as "SSSL".  Reading: a
+# window w lets query t see keys t - w .. t; query head h reads kv head
+# h // (H / Hkv).
+
+def _qkv(B, H, Hkv, T, hd, seed):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, H, T, hd)), rng.standard_normal((B, Hkv, T, hd)),
+            rng.standard_normal((B, Hkv, T, hd)))
+
+
+def test_window_covering_the_row_is_causal():
+    q, k, v = _qkv(2, 3, 3, 11, 16, 0)
+    y0, p0 = om.causal_attention(q, k, v)
+    for w in (10, 11, 50):
+        y, p = om.attention(q, k, v, window=w)
+        assert np.array_equal(y, y0) and np.array_equal(p, p0)
+
+
+def test_window_zero_returns_own_value():
+    q, k, v = _qkv(1, 4, 2, 7, 8, 1)
+    y, p = om.attention(q, k, v, window=0)
+    for h in range(4):
+        assert np.array_equal(y[0, h], v[0, h // 2])
+    assert np.array_equal(p[0, 0], np.eye(7))
+
+
+def test_window_and_groups_brute_force():
+    import math
+    B, H, Hkv, T, hd, w = 2, 4, 2, 9, 8, 3
+    q, k, v = _qkv(B, H, Hkv, T, hd, 2)
+    y, _ = om.attention(q, k, v, window=w)
+    for b in range(B):
+        for h in range(H):
+            g = h // (H // Hkv)
+            for t in range(T):
+                keys = list(range(max(0, t - w), t + 1))
+                sc = [sum(q[b, h, t, i] * k[b, g, j, i] for i in range(hd)) / math.sqrt(hd) for j in keys]
+                m = max(sc)
+                e = [math.exp(x - m) for x in sc]
+                z = sum(e)
+                ref = [sum(e[n] / z * v[b, g, j, i] for n, j in enumerate(keys)) for i in range(hd)]
+                assert np.allclose(y[b, h, t], ref, rtol=1e-12, atol=1e-12), (b, h, t)
+
+
+def test_window_hides_keys_before_it():
+    B, H, Hkv, T, hd, w = 1, 2, 1, 12, 8, 4
+    q, k, v = _qkv(B, H, Hkv, T, hd, 3)
+    y0, _ = om.attention(q, k, v, window=w)
+    t = 9
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, : t - w] += 5.0
+    v2[:, :, : t - w] -= 3.0
+    y1, _ = om.attention(q, k2, v2, window=w)
+    assert np.array_equal(y0[:, :, t:], y1[:, :, t:])
+    assert not np.allclose(y0[:, :, t - 1], y1[:, :, t - 1])
+
+
+def test_window_gqa_gradients_finite_difference():
+    B, H, Hkv, T, hd, w = 1, 4, 2, 10, 8, 3
+    q, k, v = _qkv(B, H, Hkv, T, hd, 4)
+    R = np.random.default_rng(5).standard_normal((B, H, T, hd))
+    y, p = om.attention(q, k, v, window=w)
+    dq, dk, dv = om.attention_bwd(R, q, k, v, p)
+    assert dk.shape == k.shape and dv.shape == v.shape
+    rng = np.random.default_rng(6)
+    h = 1e-6
+    for name, arr, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for _ in range(12):
+            idx = tuple(rng.integers(n) for n in arr.shape)
+            a = arr.copy()
+            a[idx] += h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = a
+            lp = np.sum(om.attention(args["q"], args["k"], args["v"], window=w)[0] * R)
+            a[idx] -= 2 * h
+            lm = np.sum(om.attention(args["q"], args["k"], args["v"], window=w)[0] * R)
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, np.abs(grad).max()), (name, idx, fd, grad[idx])
+
+
+def test_layer_windows_pattern():
+    assert om.layer_windows("SSSL", 64, 6) == [64, 64, 64, None, 64, 64]
+    assert om.layer_windows("", 64, 3) == [None, None, None]
+    assert om.layer_windows("L", 64, 2) == [None, None]
+    with pytest.raises(ValueError):
+        om.layer_windows("SXL", 64, 3)
+
+
+def test_finite_difference_with_sliding_windows():
+    s, p, tok, tgt = small_case(depth=2, d=128, vocab=48, batch=1, seq=14, std=0.05, seed=11)
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    windows = om.layer_windows("SL", 3, s.depth)
+    _fd_check(p, tok, tgt, s.depth, ["h0.c_qkv", "h1.c_qkv", "h0.c_proj"], n_coords=6, windows=windows)
+    # the window changes the loss (layer 0 sees fewer keys)
+    l0, _ = om.forward(p, tok, tgt, s.depth, keep=False)
+    l1, _ = om.forward(p, tok, tgt, s.depth, keep=False, windows=windows)
+    assert l0 != l1
