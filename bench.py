@@ -49,6 +49,8 @@ def parse():
                     help="fp8: forward block projections on e4m3 operands")
     ap.add_argument("--normuon", type=float, default=None, metavar="BETA2",
                     help="NorMuon variance reduction on the Muon updates with this second-moment decay")
+    ap.add_argument("--window-pattern", default="", help='per-layer attention windows, e.g. "SSSL" (S = sliding)')
+    ap.add_argument("--short-window", type=int, default=1024, help="left context of an S layer, tokens")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="per-category device times in the JSON line")
@@ -260,7 +262,8 @@ def run_ours(a):
     torch.cuda.set_stream(stream)
     st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
                    ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream,
-                   precision=1 if a.precision == "fp8" else 0)
+                   precision=1 if a.precision == "fp8" else 0, window_pattern=a.window_pattern,
+                   short_window=a.short_window)
     tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(1, rank))).cuda()
     tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(2, rank))).cuda()
     grads = st.grad_view() if world > 1 else None
@@ -381,7 +384,9 @@ def run_ours(a):
             "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)", "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
                        "parallelism": f"dp{world}", "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
-                       "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2"},
+                       "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
+                       "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
+                                     else "full causal")},
             "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
             "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",
             "model_tflop_per_step": fpt * s.tokens / 1e12,

@@ -25,7 +25,7 @@ ABI_FUNCTIONS = [
     "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
     "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3",
     "gpt_op_matmul_fp8", "gpt_op_attention_fwd",
-    "gpt_op_attention_bwd", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
+    "gpt_op_attention_bwd", "gpt_op_attention_fwd_ex", "gpt_op_attention_bwd_ex", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
     "gpt_op_newton_schulz_noalloc",
 ]
 
@@ -40,7 +40,8 @@ class Config(ctypes.Structure):
     _fields_ = [("depth", ctypes.c_int32), ("d_model", ctypes.c_int32), ("vocab", ctypes.c_int32),
                 ("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("mlp_mult", ctypes.c_int32), ("precision", ctypes.c_int32), ("ns_tf32_steps", ctypes.c_int32),
-                ("lm_chunk_rows", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+                ("lm_chunk_rows", ctypes.c_int32), ("seed", ctypes.c_uint64), ("short_window", ctypes.c_int32),
+                ("window_pattern", ctypes.c_char * 12)]
 
 
 class HParams(ctypes.Structure):
@@ -88,6 +89,8 @@ def lib():
             "gpt_op_matmul_fp8": (i32, [vp, vp, vp, i32, i32, i32, vp, vp, i32, vp]),
             "gpt_op_attention_fwd": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, vp]),
             "gpt_op_attention_bwd": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, vp]),
+            "gpt_op_attention_fwd_ex": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
+            "gpt_op_attention_bwd_ex": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "gpt_op_rmsnorm_fwd": (i32, [vp, vp, vp, i32, i32, vp]),
             "gpt_op_newton_schulz_scratch": (sz, [i32, i32, i32]),
             "gpt_op_newton_schulz": (i32, [vp, vp, i32, i32, i32, i32, vp, vp]),
@@ -108,10 +111,10 @@ def _check(rc):
 
 
 def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0, seed=0,
-                precision=0):
+                precision=0, window_pattern="", short_window=0):
     return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
                   mlp_mult=4, precision=precision, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows,
-                  seed=seed)
+                  seed=seed, short_window=short_window, window_pattern=window_pattern.encode("ascii"))
 
 
 def workspace_size(cfg: Config):
@@ -138,9 +141,10 @@ class GPTStep:
     """
 
     def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0,
-                 seed=0, stream=None, precision=0):
+                 seed=0, stream=None, precision=0, window_pattern="", short_window=0):
         import torch
-        self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision)
+        self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision,
+                               window_pattern, short_window)
         self.sizes = workspace_size(self.cfg)
         dev = torch.device("cuda", torch.cuda.current_device())
         self.stream = stream if stream is not None else torch.cuda.current_stream()
@@ -280,24 +284,29 @@ def matmul_fp8(A, B, M, N, K, inv_a, inv_b, b_trans=False, stream=None):
     return C
 
 
-def attention_fwd(q, k, v, stream=None):
+def attention_fwd(q, k, v, window=-1, stream=None):
+    """Causal attention; k, v may have fewer heads than q (grouped kv heads);
+    window >= 0 limits query t to keys t - window .. t."""
     import torch
     B, H, T, hd = q.shape
+    Hkv = k.shape[1]
     o = torch.empty((B, T, H, hd), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
-    _check(lib().gpt_op_attention_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, T, _stream(stream)))
+    _check(lib().gpt_op_attention_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, T, int(window),
+                                         _stream(stream)))
     return o, lse
 
 
-def attention_bwd(q, k, v, o, lse, dout, stream=None):
+def attention_bwd(q, k, v, o, lse, dout, window=-1, stream=None):
     import torch
     B, H, T, hd = q.shape
+    Hkv = k.shape[1]
     dq = torch.empty((B, H, T, hd), dtype=torch.float32, device=q.device)
     dk = torch.empty_like(k)
     dv = torch.empty_like(v)
     D = torch.empty((B, H, T), dtype=torch.float32, device=q.device)
-    _check(lib().gpt_op_attention_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(D),
-                                      _ptr(dq), _ptr(dk), _ptr(dv), B, H, T, _stream(stream)))
+    _check(lib().gpt_op_attention_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(D),
+                                         _ptr(dq), _ptr(dk), _ptr(dv), B, H, Hkv, T, int(window), _stream(stream)))
     return dq, dk, dv
 
 

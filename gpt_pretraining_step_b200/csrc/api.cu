@@ -39,6 +39,10 @@ constexpr size_t kAlign = 256;
 
 struct Dims {
   int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32, fp8;
+  int short_window, n_pat;
+  char pat[12];
+  // attention window of layer l: short_window for an 'S' layer, -1 = full causal
+  int window(int l) const { return n_pat > 0 && pat[l % n_pat] == 'S' ? short_window : -1; }
 };
 
 // Offsets (bytes) into the three caller buffers.
@@ -113,6 +117,18 @@ int dims_from(const gpt_config* c, Dims& D) {
   D.tiles_lm = (D.V + 255) / 256;
   D.n_tf32 = c->ns_tf32_steps;
   D.fp8 = c->precision == 1;
+  D.n_pat = 0;
+  bool any_s = false;
+  for (int i = 0; i < 12 && c->window_pattern[i]; ++i) {
+    const char ch = c->window_pattern[i];
+    if (ch != 'S' && ch != 'L') return fail(GPT_EINVAL, "window_pattern may hold only 'S' and 'L'");
+    any_s = any_s || ch == 'S';
+    D.pat[D.n_pat++] = ch;
+  }
+  if (D.n_pat == 12) return fail(GPT_EINVAL, "window_pattern must be NUL-terminated within 12 bytes");
+  if (any_s && (c->short_window < 0 || c->short_window >= (1 << 30)))
+    return fail(GPT_EINVAL, "short_window must be in [0, 2^30) when the pattern has an 'S' layer");
+  D.short_window = c->short_window;
   return GPT_OK;
 }
 
@@ -460,7 +476,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
-      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err);
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, H, D.window(l));
     }
     {
       GemmCall g = base_call(M, d, d);
@@ -602,7 +618,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err);
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, H, D.window(l));
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
@@ -1177,12 +1193,34 @@ int gpt_op_matmul_fp8(const void* A, const void* B, float* C, int M, int N, int 
   return GPT_OK;
 }
 
-int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
-                         void* stream) {
+int gpt_op_attention_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                            int T, int window, void* stream) {
   if (!q || !k || !v || !o || !lse) return fail(GPT_EINVAL, "null pointer");
   if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
+  if (Hkv < 1 || H % Hkv) return fail(GPT_EINVAL, "kv heads must divide the query heads");
+  if (static_cast<long long>(B) * H * T > (1ll << 31) - 1) return fail(GPT_EINVAL, "attention too large");
   launch_attn_fwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
-                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream), nullptr);
+                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream), nullptr, Hkv, window);
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int T,
+                         void* stream) {
+  return gpt_op_attention_fwd_ex(q, k, v, o, lse, B, H, H, T, -1, stream);
+}
+
+int gpt_op_attention_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int Hkv,
+                            int T, int window, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !Dscratch || !dq || !dk || !dv) return fail(GPT_EINVAL, "null pointer");
+  if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
+  if (Hkv < 1 || H % Hkv) return fail(GPT_EINVAL, "kv heads must divide the query heads");
+  if (static_cast<long long>(B) * H * T > (1ll << 31) - 1) return fail(GPT_EINVAL, "attention too large");
+  launch_attn_bwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
+                  static_cast<const bf16*>(o), static_cast<const bf16*>(dout), lse, Dscratch, dq,
+                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream), nullptr,
+                  Hkv, window);
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -1190,13 +1228,7 @@ int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, f
 int gpt_op_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                          const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int T,
                          void* stream) {
-  if (!q || !k || !v || !o || !dout || !lse || !Dscratch || !dq || !dk || !dv) return fail(GPT_EINVAL, "null pointer");
-  if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
-  launch_attn_bwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
-                  static_cast<const bf16*>(o), static_cast<const bf16*>(dout), lse, Dscratch, dq,
-                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream), nullptr);
-  GPT_CK(cudaGetLastError());
-  return GPT_OK;
+  return gpt_op_attention_bwd_ex(q, k, v, o, dout, lse, Dscratch, dq, dk, dv, B, H, H, T, -1, stream);
 }
 
 int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream) {

@@ -1,8 +1,11 @@
 // Causal flash attention, forward and backward, head_dim 128, bf16 operands
 // with fp32 softmax and accumulation (online softmax; the forward saves the
-// row log-sum-exp, the backward recomputes P from it).
+// row log-sum-exp, the backward recomputes P from it).  Optional sliding
+// window (query t sees keys t - window .. t) and grouped kv heads (query head
+// h reads kv head h / (H / Hkv)), the two attention variants of "¿Cómo
+// Entrenar Tu Propio ChatGPT por $50?", section "1. Modelo GPT".
 //
-// Layouts: q, k, v, dk, dv are [B, H, T, 128]; the forward output O and the
+// Layouts: q is [B, H, T, 128], k, v, dk, dv are [B, Hkv, T, 128]; the forward output O and the
 // incoming gradient dO are token-major [B, T, H, 128] (the rows of the
 // projection GEMMs); dq is accumulated in fp32 [B, H, T, 128]; lse and
 // D = rowsum(dO * O) are [B, H, T].
@@ -71,7 +74,7 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
-                       int H, int T, float scale_log2, int* err) {
+                       int H, int Hkv, int T, int wl, float scale_log2, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -100,10 +103,15 @@ __global__ void __launch_bounds__(384, 1)
   const int nq = (T + 127) / 128;
   const int pair = (gridDim.x - 1) - blockIdx.x;   // longest pairs first
   const int bh = blockIdx.y;
+  const int bkv = (bh / H) * Hkv + (bh - (bh / H) * H) / (H / Hkv);   // kv head of this query head
   const int qtA = 2 * pair;
   const bool hasB = qtA + 1 < nq;
-  const int nkvA = qtA + 1;                         // causal: key blocks 0..qt
-  const int nkvB = hasB ? qtA + 2 : 0;
+  // key blocks j0 .. qt (causal, and not before the first row's window); both
+  // tiles start at j0, rows for which a block lies wholly outside their window
+  // see only masked scores there
+  const int j0 = max(0, qtA * 128 - wl) / 128;
+  const int nkvA = qtA + 1 - j0;
+  const int nkvB = hasB ? qtA + 2 - j0 : 0;
   const int nkv = hasB ? nkvB : nkvA;
 
   if (threadIdx.x == 0) {
@@ -146,14 +154,15 @@ __global__ void __launch_bounds__(384, 1)
         const int s = j & 1;
         const uint32_t par = (j >> 1) & 1;
         if (!mbar_wait(&k_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
+        const int kc = (j0 + j) * 128;
         mbar_arrive_expect_tx(&k_full[s], TF_BUF);
-        tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, j * 128, bh);
-        tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, j * 128, bh);
+        tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, kc, bkv);
+        tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, kc, bkv);
         ++issued_k;
         if (!mbar_wait(&v_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[s], TF_BUF);
-        tma_load_3d(sV + s * TF_BUF, &tv, &v_full[s], 0, j * 128, bh);
-        tma_load_3d(sV + s * TF_BUF + TF_TILE, &tv, &v_full[s], 64, j * 128, bh);
+        tma_load_3d(sV + s * TF_BUF, &tv, &v_full[s], 0, kc, bkv);
+        tma_load_3d(sV + s * TF_BUF + TF_TILE, &tv, &v_full[s], 64, kc, bkv);
         ++issued_v;
       }
       if (!ok) {
@@ -262,13 +271,13 @@ __global__ void __launch_bounds__(384, 1)
         tmem_load32_async(t_s + 96, r3);
         tmem_wait_ld();
       }
-      const int kbase = j * 128;
-      if ((j == qt) || (kbase + 128 > T)) {
-        // causal diagonal / ragged tail: masked scores become -inf
+      const int kbase = (j0 + j) * 128;
+      if ((j0 + j == qt) || (kbase + 128 > T) || (kbase < q0 + 127 - wl)) {
+        // causal diagonal, ragged tail or window edge: masked scores become -inf
 #pragma unroll
         for (int k = 0; k < 128; ++k) {
           const int key = kbase + k;
-          if (key > q || key >= T) sr[k] = __float_as_uint(-INFINITY);
+          if (key > q || key >= T || key < q - wl) sr[k] = __float_as_uint(-INFINITY);
         }
       }
       // block max of the raw scores (the scale is positive), eight independent chains
@@ -280,9 +289,12 @@ __global__ void __launch_bounds__(384, 1)
       const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                                fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float mblk = mraw * scale_log2;
-      const bool move = mblk > m_ref + TF_RESCALE;   // always true on the first block
+      const bool move = mblk > m_ref + TF_RESCALE;   // true on the first block with a visible key
       const float m_new = move ? mblk : m_ref;
-      const float factor = ex2_approx(m_ref - m_new);  // 1 when the reference stays, 0 on the first block
+      // 1 when the reference stays, 0 when it leaves -inf; a row that has seen
+      // only masked scores (window edge) keeps -inf and offsets by 0 below
+      const bool none = m_new == -INFINITY;
+      const float factor = none ? 1.f : ex2_approx(m_ref - m_new);
       // O holds the products of blocks < j (S of this block was issued after
       // the last of them completed), so it may be rescaled now
       if (j >= 1 && __any_sync(0xffffffffu, move)) {
@@ -298,7 +310,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       // probabilities relative to the reference (masked scores give 0), row sum,
       // bf16 P over the first 64 columns of S
-      const uint64_t nb2 = f2_pack(-m_new, -m_new);
+      const float m_off = none ? 0.f : m_new;
+      const uint64_t nb2 = f2_pack(-m_off, -m_off);
       uint64_t rs2 = f2_pack(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -373,8 +386,10 @@ __global__ void __launch_bounds__(384, 1)
 
 // ------------------------------------------------ backward on tcgen05 / TMEM
 //
-// One CTA per (128-key block j, batch*head), looping over the query blocks
-// i = j + it >= j that see those keys.  448 threads:
+// One CTA per (128-key block j, batch*kv head), looping over the query heads
+// of the kv group and, for each, the query blocks i >= j that see those keys
+// (up to the last one inside the window); dK and dV add up over the whole
+// loop.  448 threads:
 //   warp 0      TMA: K_j and V_j once; Q_i through a two-slot ring; dO_i.
 //   warp 1      TMEM owner and MMA issuer.  TMEM columns: [0,128) S^T_i and
 //               dQ^T_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16
@@ -418,8 +433,8 @@ __global__ void __launch_bounds__(448, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                        const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
-                       const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int T,
-                       float scale, int* err) {
+                       const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int Hkv,
+                       int T, int wl, float scale, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -455,11 +470,17 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int j = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh - (bh / H) * H;
+  const int bkv = blockIdx.y;
+  const int b = bkv / Hkv, hk = bkv - (bkv / Hkv) * Hkv;
+  const int G = H / Hkv;
   const int k0 = j * 128;
   const int nq = (T + 127) / 128;
-  const int n_it = nq - j;
+  // query blocks j .. i_hi see this key block (the window ends at i_hi); the
+  // loop runs them for each of the G query heads of the group in turn
+  const int nb = min(nq - 1, (k0 + 127 + wl) / 128) - j + 1;
+  const int n_it = G * nb;
+  auto q_block = [&](int it) { return j + it % nb; };
+  auto q_head = [&](int it) { return hk * G + it / nb; };   // within the batch row
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -497,12 +518,12 @@ __global__ void __launch_bounds__(448, 1)
       bool ok = true;
       int issued_q = 0, issued_do = 0;
       mbar_arrive_expect_tx(kv_full, 2 * TF_BUF);
-      tma_load_3d(sK, &tk, kv_full, 0, k0, bh);
-      tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, k0, bh);
-      tma_load_3d(sV, &tv, kv_full, 0, k0, bh);
-      tma_load_3d(sV + TF_TILE, &tv, kv_full, 64, k0, bh);
+      tma_load_3d(sK, &tk, kv_full, 0, k0, bkv);
+      tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, k0, bkv);
+      tma_load_3d(sV, &tv, kv_full, 0, k0, bkv);
+      tma_load_3d(sV + TF_TILE, &tv, kv_full, 64, k0, bkv);
       for (int it = 0; it < n_it && ok; ++it) {
-        const int i = j + it;
+        const int i = q_block(it), h = q_head(it), bh = b * H + h;
         const int s = it & 1;
         const uint32_t par = (it >> 1) & 1;
         if (!mbar_wait(&q_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
@@ -644,7 +665,7 @@ __global__ void __launch_bounds__(448, 1)
       __syncwarp();
     };
     for (int it = 0; it < n_it && ok; ++it) {
-      const int q0 = (j + it) * 128;
+      const int q0 = q_block(it) * 128, bh = b * H + q_head(it);
       const bool got = mbar_wait(mm_done, it & 1, abort_flag, err);
       __syncwarp();
       if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -698,7 +719,8 @@ __global__ void __launch_bounds__(448, 1)
     // this thread's share of a query block's -lse (log2 units; -inf past T so
     // P = 0) or -D, fetched a block ahead so the load latency hides
     auto fetch = [&](int it2) -> float {
-      const int q0f = (j + it2) * 128;
+      const int q0f = q_block(it2) * 128;
+      const long long bh = static_cast<long long>(b) * H + q_head(it2);
       if (t256 < 128) {
         const int qq = q0f + t256;
         return qq < T ? __ldg(lse + static_cast<long long>(bh) * T + qq) * -1.4426950408889634f : -INFINITY;
@@ -714,9 +736,11 @@ __global__ void __launch_bounds__(448, 1)
     // P of block it2 for this thread's key row and 64 query columns, packed bf16
     uint32_t pk[32];
     auto compute_p = [&](int it2) {
-      const bool diag = it2 == 0;
-      const bool masked = diag || k0 + 128 > T;   // causal diagonal block or ragged key block
-      const int q0 = (j + it2) * 128;
+      const bool diag = it2 % nb == 0;
+      const int q0 = q_block(it2) * 128;
+      // causal diagonal block, ragged key block, or a query block whose last
+      // rows' windows start past this block's first key
+      const bool masked = diag || k0 + 128 > T || q0 + 127 - wl > k0;
       const float* nls = lse_s + (it2 & 1) * 128;
       uint32_t sa[32], sb[32];
       tmem_load32_async(tmem + lane_base + (2 * half) * 32, sa);
@@ -752,7 +776,7 @@ __global__ void __launch_bounds__(448, 1)
           if (masked) {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              if (!key_ok || (diag && key > q0 + c * 32 + k + e)) p[e] = 0.f;
+              if (!key_ok || (diag && key > q0 + c * 32 + k + e) || key < q0 + c * 32 + k + e - wl) p[e] = 0.f;
           }
 #pragma unroll
           for (int e = 0; e < 8; e += 2) pk[16 * cc + ((k + e) >> 1)] = pack_bf16x2(p[e], p[e + 1]);
@@ -823,8 +847,8 @@ __global__ void __launch_bounds__(448, 1)
     }
     if (ok) {
       tc_fence_after();
-      bf16* dkrow = dk + (static_cast<long long>(bh) * T + key) * 128;
-      bf16* dvrow = dv + (static_cast<long long>(bh) * T + key) * 128;
+      bf16* dkrow = dk + (static_cast<long long>(bkv) * T + key) * 128;
+      bf16* dvrow = dv + (static_cast<long long>(bkv) * T + key) * 128;
 #pragma unroll 1
       for (int c = 2 * half; c < 2 * half + 2; ++c) {
         uint32_t vr[32], kr[32];
@@ -880,52 +904,59 @@ __global__ void attn_bwd_dot_kernel(const bf16* __restrict__ o, const bf16* __re
 
 }  // namespace
 
+// Window in tokens as the kernels take it: keys t - wl .. t; "no window" is a
+// bound no row reaches (kept small enough that k0 + 127 + wl fits in an int).
+static int window_bound(int window, int T) { return window < 0 || window >= T ? (1 << 30) : window; }
+
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s, int* err) {
+                     cudaStream_t s, int* err, int Hkv, int window) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
     configured = true;
   }
+  if (Hkv <= 0) Hkv = H;
   CUtensorMap mq, mk, mv;
-  const long long bh = 1ll * B * H;
-  if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128)) {
+  const long long bh = 1ll * B * H, bhkv = 1ll * B * Hkv;
+  if (H % Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
     return;
   }
   dim3 grid(((T + 127) / 128 + 1) / 2, B * H);   // pairs of query tiles
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, T, scale_log2, err);
+  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, T, window_bound(window, T), scale_log2,
+                                                err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s, int* err) {
+                     cudaStream_t s, int* err, int Hkv, int window) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
     configured = true;
   }
+  if (Hkv <= 0) Hkv = H;
   const long long rows = 1ll * B * H * T;
   attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
   CUtensorMap mq, mk, mv, mdo, mdq;
-  const long long bh = 1ll * B * H;
+  const long long bh = 1ll * B * H, bhkv = 1ll * B * Hkv;
   const long long dims[4] = {HD, H, T, B};
   const long long strides[3] = {HD * 2ll, 1ll * H * HD * 2, 1ll * T * H * HD * 2};
   const int box[4] = {64, 1, 128, 1};
-  if (!make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mk, k, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mv, v, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
+  if (H % Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
+      !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
       !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }
-  dim3 grid((T + 127) / 128, B * H);
-  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, T,
-                                                1.f / sqrtf(static_cast<float>(HD)), err);
+  dim3 grid((T + 127) / 128, B * Hkv);
+  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, T,
+                                                window_bound(window, T), 1.f / sqrtf(static_cast<float>(HD)), err);
 }
 
 }  // namespace gpt

@@ -8,15 +8,18 @@ namespace gpt {
 
 using bf16 = __nv_bfloat16;
 
-// q, k, v [B, H, T, 128] -> o [B, T, H, 128], lse [B, H, T] (natural log).
+// q [B, H, T, 128], k, v [B, Hkv, T, 128] -> o [B, T, H, 128], lse [B, H, T]
+// (natural log).  Hkv <= 0 means Hkv = H (it must divide H); window < 0 (or
+// >= T) is full causal attention, else query t sees keys t - window .. t.
 // err: device error word for expired waits (may be null).
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s, int* err);
+                     cudaStream_t s, int* err, int Hkv = 0, int window = -1);
 
-// Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32, zeroed
-// here, then accumulated), dk, dv [B, H, T, 128]; Dv [B, H, T] is scratch.
+// Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32
+// [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, Hkv, T, 128]
+// (summed over the query heads of each kv head); Dv [B, H, T] is scratch.
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s, int* err);
+                     cudaStream_t s, int* err, int Hkv = 0, int window = -1);
 
 }  // namespace gpt

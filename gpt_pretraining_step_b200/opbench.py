@@ -45,6 +45,8 @@ def main(argv=None):
     a.add_argument("--B", type=int, default=4)
     a.add_argument("--H", type=int, default=10)
     a.add_argument("--T", type=int, default=2048)
+    a.add_argument("--kv-heads", type=int, default=0, help="grouped kv heads (0 = H)")
+    a.add_argument("--window", type=int, default=-1, help="sliding window, tokens of left context (-1 = full)")
     n = sub.add_parser("newton-schulz", help="five Polar Express steps on a batch of matrices")
     n.add_argument("--batch", type=int, default=20)
     n.add_argument("--rows", type=int, default=1280)
@@ -66,17 +68,21 @@ def main(argv=None):
         print(json.dumps({"op": "gemm", "M": args.M, "N": args.N, "K": args.K, "ms": ms,
                           "tflops": flops / (ms / 1e3) / 1e12}))
     elif args.op == "attention":
-        shape = (args.B, args.H, args.T, 128)
-        q, k, v = (torch.randn(shape, device=dev).bfloat16() for _ in range(3))
+        hkv = args.kv_heads or args.H
+        q = torch.randn((args.B, args.H, args.T, 128), device=dev).bfloat16()
+        k, v = (torch.randn((args.B, hkv, args.T, 128), device=dev).bfloat16() for _ in range(2))
         do = torch.randn((args.B, args.T, args.H, 128), device=dev).bfloat16()
-        o, lse = attention_fwd(q, k, v)
-        causal = 4.0 * args.B * args.H * 128 * args.T * (args.T + 1) / 2
-        ms_f = _time(lambda: attention_fwd(q, k, v), args.reps, args.warmup)
-        ms_b = _time(lambda: attention_bwd(q, k, v, o, lse, do), args.reps, args.warmup)
-        print(json.dumps({"op": "attention_fwd", "B": args.B, "H": args.H, "T": args.T, "ms": ms_f,
-                          "tflops": causal / (ms_f / 1e3) / 1e12}))
-        print(json.dumps({"op": "attention_bwd", "B": args.B, "H": args.H, "T": args.T, "ms": ms_b,
-                          "tflops": 2.5 * causal / (ms_b / 1e3) / 1e12}))
+        w = args.window
+        o, lse = attention_fwd(q, k, v, window=w)
+        # visible (query, key) pairs: t + 1 keys for query t, at most w + 1 with a window
+        pairs = sum(min(t, w) + 1 if w >= 0 else t + 1 for t in range(args.T))
+        flops = 4.0 * args.B * args.H * 128 * pairs
+        ms_f = _time(lambda: attention_fwd(q, k, v, window=w), args.reps, args.warmup)
+        ms_b = _time(lambda: attention_bwd(q, k, v, o, lse, do, window=w), args.reps, args.warmup)
+        common = {"B": args.B, "H": args.H, "kv_heads": hkv, "T": args.T, "window": w}
+        print(json.dumps({"op": "attention_fwd", **common, "ms": ms_f, "tflops": flops / (ms_f / 1e3) / 1e12}))
+        print(json.dumps({"op": "attention_bwd", **common, "ms": ms_b,
+                          "tflops": 2.5 * flops / (ms_b / 1e3) / 1e12}))
     else:
         G = torch.randn((args.batch, args.rows, args.cols), device=dev)
         ms = _time(lambda: newton_schulz(G, tf32_steps=args.tf32_steps), args.reps, args.warmup)

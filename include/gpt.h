@@ -94,6 +94,14 @@ typedef struct gpt_config {
   int32_t ns_tf32_steps;
   int32_t lm_chunk_rows; /* rows of logits held at once by the fused lm_head/CE; 0 = 8192 */
   uint64_t seed;
+  int32_t short_window;   /* tokens of left context of an "S" layer (0 ..) */
+  char window_pattern[12];/* per-layer attention window, repeated over the
+                           * layers: 'S' = sliding window of short_window
+                           * earlier tokens (query t sees keys t - short_window
+                           * .. t), 'L' = full causal; e.g. "SSSL"; empty (all
+                           * zero) = every layer full causal.  "¿Cómo Entrenar
+                           * Tu Propio ChatGPT por $50?", section "1. Modelo
+                           * GPT", sliding-window attention. */
 } gpt_config;
 
 typedef struct gpt_ctx gpt_ctx;
@@ -264,6 +272,20 @@ int gpt_op_attention_fwd(const void* q, const void* k, const void* v, void* o, f
 int gpt_op_attention_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
                          const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int T,
                          void* stream);
+
+/* The two attention variants of "¿Cómo Entrenar Tu Propio ChatGPT por $50?",
+ * section "1. Modelo GPT": grouped kv heads (GQA) and sliding-window
+ * attention.  q bf16 [B, H, T, 128]; k, v bf16 [B, Hkv, T, 128] with Hkv
+ * dividing H, query head h reading kv head h / (H / Hkv); window < 0 (or
+ * >= T) is full causal attention, else query t sees keys t - window .. t.
+ * Forward outputs as gpt_op_attention_fwd; the backward writes dq fp32
+ * [B, H, T, 128] and dk, dv bf16 [B, Hkv, T, 128], each the sum over the
+ * query heads of its group.  A bad head split is GPT_EINVAL. */
+int gpt_op_attention_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                            int T, int window, void* stream);
+int gpt_op_attention_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                            const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int Hkv,
+                            int T, int window, void* stream);
 
 /* Gain-free RMSNorm of fp32 rows [M, d] -> bf16 y and fp32 rstd [M]. */
 int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream);

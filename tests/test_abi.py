@@ -62,12 +62,21 @@ def test_workspace_size_valid_configs(L):
 
 
 @pytest.mark.parametrize("bad", [dict(depth=0), dict(d_model=100), dict(vocab=1001), dict(batch=0),
-                                 dict(seq_len=0), dict(vocab=4)])
+                                 dict(seq_len=0), dict(vocab=4), dict(window_pattern="SXL", short_window=8),
+                                 dict(window_pattern="SSSL", short_window=-1),
+                                 dict(window_pattern="SSSLSSSLSSSL", short_window=8)])
 def test_workspace_size_rejects_bad_config(L, bad):
     import gpt_pretraining_step_b200 as g
     with pytest.raises(g.GptError) as e:
         g.workspace_size(_cfg(**bad))
     assert e.value.code == g.GPT_EINVAL
+
+
+def test_window_pattern_configs_accepted(L):
+    import gpt_pretraining_step_b200 as g
+    base = g.workspace_size(_cfg())
+    for pat, sw in [("SSSL", 32), ("L", 0), ("S", 0), ("", -5), ("LLS", 1 << 20)]:
+        assert g.workspace_size(_cfg(window_pattern=pat, short_window=sw)) == base
 
 
 def test_bad_fields_rejected(L):

@@ -143,6 +143,62 @@ def test_attention_bwd(torch, B, H, T):
         assert relfro(got, ref) < 2e-2
 
 
+# grouped kv heads and sliding windows: windows below, at and across tile
+# edges, a window of 0 (each query sees itself), one wider than the row
+VARIANTS = [(2, 4, 2, 333, 100), (1, 3, 1, 520, 0), (1, 2, 2, 700, 128), (1, 4, 4, 1000, 255),
+            (2, 2, 1, 200, 1000), (1, 6, 3, 1024, 127), (1, 2, 1, 900, 129)]
+
+
+def _kv_inputs(B, H, Hkv, T, seed):
+    q, k, v = _attn_inputs(B, H, T, seed)
+    return q, k[:, :Hkv].copy(), v[:, :Hkv].copy()
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,window", VARIANTS)
+def test_attention_fwd_window_gqa(torch, B, H, Hkv, T, window):
+    import gpt_pretraining_step_b200 as g
+    q, k, v = _kv_inputs(B, H, Hkv, T, seed=T + window)
+    o, lse = g.attention_fwd(bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v), window=window)
+    torch.cuda.synchronize()
+    ref, _ = om.attention(q.astype(np.float64), k.astype(np.float64), v.astype(np.float64), window=window)
+    got = f64(o).transpose(0, 2, 1, 3)
+    assert relfro(got, ref) < 1e-2
+    assert np.abs(got - ref).max() < 3e-2
+    kq = om.kv_for_queries(k.astype(np.float64), H)
+    s = np.matmul(q.astype(np.float64), np.swapaxes(kq, -1, -2)) / np.sqrt(128)
+    s = np.where(om.attention_hidden(T, window), -np.inf, s)
+    assert np.abs(f64(lse) - om.logsumexp(s)).max() < 2e-3
+
+
+@pytest.mark.parametrize("B,H,Hkv,T,window", VARIANTS)
+def test_attention_bwd_window_gqa(torch, B, H, Hkv, T, window):
+    import gpt_pretraining_step_b200 as g
+    q, k, v = _kv_inputs(B, H, Hkv, T, seed=3 * T + window)
+    dout = syn.round_to_bf16(syn.gaussian((B, T, H, 128), seed=T + window + 5))
+    qt, kt, vt = bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v)
+    o, lse = g.attention_fwd(qt, kt, vt, window=window)
+    dq, dk, dv = g.attention_bwd(qt, kt, vt, o, lse, bf16_t(torch, dout), window=window)
+    torch.cuda.synchronize()
+    q64, k64, v64 = q.astype(np.float64), k.astype(np.float64), v.astype(np.float64)
+    _, P = om.attention(q64, k64, v64, window=window)
+    refs = om.attention_bwd(dout.astype(np.float64).transpose(0, 2, 1, 3), q64, k64, v64, P)
+    assert f64(dk).shape == k.shape and f64(dv).shape == v.shape
+    for name, got, ref in zip("q k v".split(), (f64(dq), f64(dk), f64(dv)), refs):
+        if window == 0 and name in "qk":
+            # one visible key per query: the softmax is constant, dq = dk = 0
+            assert np.abs(got).max() < 1e-4, name
+            continue
+        assert cosine(got, ref) > 0.9999, name
+        assert relfro(got, ref) < 2e-2, name
+
+
+def test_attention_rejects_bad_head_split(torch):
+    import gpt_pretraining_step_b200 as g
+    q, k, v = _kv_inputs(1, 3, 2, 64, seed=1)
+    with pytest.raises(g.GptError):
+        g.attention_fwd(bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v))
+
+
 @pytest.mark.parametrize("batch,rows,cols", [(2, 256, 768), (1, 640, 128), (3, 128, 128), (1, 136, 264)])
 @pytest.mark.parametrize("tf32_steps", [-1, 0, 3, 5])
 def test_newton_schulz(torch, batch, rows, cols, tf32_steps):

@@ -81,6 +81,29 @@ def test_fwd_bwd_matches_oracle(torch, name):
         assert c >= GRAD_COS, (pname, c)
 
 
+@pytest.mark.parametrize("pattern,short_window", [("SSSL", 150), ("SL", 0), ("S", 128)])
+def test_sliding_window_layers_match_oracle(torch, pattern, short_window):
+    """Per-layer attention windows ("SSSL"-style pattern repeated over the
+    layers) through the whole forward and backward."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=4, d_model=256, vocab=1000, batch=2, seq_len=520)
+    params = syn.init_params(s, seed=21)
+    tok, tgt = syn.tokens(s, seed=22), syn.targets(s, seed=23)
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   window_pattern=pattern, short_window=short_window)
+    for tid, (name, *_rest) in enumerate(syn.param_specs(s)):
+        st.set(tid, params[name])
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    windows = om.layer_windows(pattern, short_window, s.depth)
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth, windows=windows)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL
+    assert np.abs(f64(st.row_loss()).ravel() - cache["row_loss"]).max() < 2e-2
+    for tid, (pname, *_r) in enumerate(syn.param_specs(s)):
+        c = cosine(f64(st.get(tid, g.KIND_GRAD)), grads[pname])
+        assert c >= GRAD_COS, (pname, c)
+
+
 def test_embedding_and_target_indexing_exact(torch):
     # with a zero lm_head the logits vanish: loss = ln V exactly, and dW_lm has
     # one shared column for every vocabulary id that is not a target, so the set
