@@ -58,7 +58,7 @@ struct Plan {
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
   size_t xf, rf, z, stats, zt, row_loss, loss;
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
-  size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, rope, err, tok, tgt;
+  size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
   size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
@@ -210,6 +210,7 @@ void make_plan(const Dims& D, Plan& P) {
   P.inv_norm = ab.take(4 * L * 4);
   P.normws = ab.take(muon_norm_workspace(4 * D.L));
   P.nfac = ab.take(2 * L * d * 4);
+  P.sched = ab.take(64);   // work counters of the persistent attention kernels
   P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
   P.tok = ab.take(M * 4);
@@ -476,7 +477,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
-      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, H, D.window(l));
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, H, D.window(l), c->A<int>(P.sched));
     }
     {
       GemmCall g = base_call(M, d, d);

@@ -13,6 +13,8 @@
 // Both directions run on the 5th-generation tensor cores (tcgen05.mma with
 // TMEM accumulators), fed by TMA; softmax work runs in dedicated warps that
 // exchange tiles with the MMA issuer through mbarriers.
+#include <algorithm>
+
 #include "attention.cuh"
 #include "common.cuh"
 #include "gemm.h"
@@ -25,13 +27,23 @@ constexpr int HD = 128;
 
 // ------------------------------------------------- forward on tcgen05 / TMEM
 //
-// One CTA per pair of 128-query tiles (A = 2p, B = 2p + 1) of one
-// batch*head; the pair shares every K and V block it loads.  384 threads
-// in three warp groups; the first (TMA, MMA and two idle warps) gives
-// registers to the two softmax groups (setmaxnreg 40 / 232 / 232, which adds
-// up to the 168 per thread the block is launched with), so each softmax
+// Persistent: one CTA per SM takes work items, a pair of 128-query tiles
+// (A = 2p, B = 2p + 1) of one batch*head, until none are left; the pair
+// shares every K and V block it loads.  Items are numbered head-major, the
+// longest pair of a head first, so the CTAs running at one time share the
+// K/V of a few heads in L2; a scheduler word in device memory hands them out
+// in that order (an atomic counter, zeroed before the launch), and with no
+// word each CTA takes every gridDim.x-th item.  The next item's Q loads and
+// first S = Q K^T run while the softmax warps finish the previous item, so
+// the per-item load and pipeline-fill latency is hidden.
+// 384 threads in three warp groups; the first (TMA, MMA and two idle warps)
+// gives registers to the two softmax groups (setmaxnreg 56 / 224 / 224, which
+// adds up to the 168 per thread the block is launched with), so each softmax
 // thread keeps its whole S row in registers.
-//   warp 0      TMA: Q_A and Q_B once, K_j and V_j through two-slot rings
+//   warp 0      TMA: takes the items and publishes their numbers in a shared
+//               ring, loads Q_A and Q_B of each (once every warp has read the
+//               item number and the previous Q is no longer read), K_j and
+//               V_j through two-slot rings that run on across items
 //   warp 1      TMEM owner and MMA issuer.  TMEM columns: S_A [0,128),
 //               S_B [128,256), O_A [256,384), O_B [384,512).  Per key block
 //               j: O_A += P_A V_j and O_B += P_B V_j, with P read from TMEM
@@ -42,7 +54,8 @@ constexpr int HD = 128;
 //   warps 4..7  softmax of tile A, warps 8..11 of tile B, one query row (TMEM
 //               lane) per thread: the block max from a first pass over the S
 //               row, exp2 into bf16 P (three of every eight exponentials by a
-//               polynomial on the FMA pipe), the row sum.
+//               polynomial on the FMA pipe), the row sum; after the last
+//               block, O / l and the log-sum-exp.
 // The reference max of a row only moves when the block max exceeds it by
 // more than 8 (log2 units), so P stays below 2^8; when it moves, the warp
 // rescales its rows of O in TMEM (the previous P V has completed by then:
@@ -71,10 +84,34 @@ __device__ __forceinline__ void tmem_store32(uint32_t taddr, const uint32_t (&r)
       : "memory");
 }
 
+// Item n: batch*head bh and the pair's first query tile, key blocks j0 ..
+// (causal end), per tile counts nkvA, nkvB (0: tile B past the sequence).
+struct FwdItem {
+  int bh, bkv, qtA, j0, nkvA, nkvB, nkv;
+  bool hasB;
+};
+
+__device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int wl) {
+  FwdItem it;
+  const int npairs = (nq + 1) / 2;
+  it.bh = n / npairs;
+  const int pair = npairs - 1 - (n - it.bh * npairs);
+  it.bkv = (it.bh / H) * Hkv + (it.bh - (it.bh / H) * H) / (H / Hkv);
+  it.qtA = 2 * pair;
+  it.hasB = it.qtA + 1 < nq;
+  // both tiles start at the first key block any row of tile A sees; rows for
+  // which a block lies wholly outside their window see only masked scores
+  it.j0 = max(0, it.qtA * 128 - wl) / 128;
+  it.nkvA = it.qtA + 1 - it.j0;
+  it.nkvB = it.hasB ? it.qtA + 2 - it.j0 : 0;
+  it.nkv = it.hasB ? it.nkvB : it.nkvA;
+  return it;
+}
+
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
-                       int H, int Hkv, int T, int wl, float scale_log2, int* err) {
+                       int H, int Hkv, int T, int wl, float scale_log2, int n_items, int* sched, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -87,35 +124,26 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* sK = sm + 2 * TF_BUF;     // two slots
   uint8_t* sV = sm + 4 * TF_BUF;     // two slots
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TF_BUF);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* k_empty = bars + 3;   // [2]
-  uint64_t* v_full = bars + 5;    // [2]
-  uint64_t* v_empty = bars + 7;   // [2]
-  uint64_t* s_full = bars + 9;    // [2] per tile: S of block j in TMEM
-  uint64_t* p_full = bars + 11;   // [2] per tile: P of block j in TMEM
-  uint64_t* pv_done = bars + 13;  // [2] per tile: P V of block j complete
-  uint64_t* drain = bars + 15;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* q_full = bars + 0;    // Q of item n landed (or the end marker)
+  uint64_t* q_empty = bars + 1;   // item n's S products done and every warp has its number
+  uint64_t* k_full = bars + 2;    // [2]
+  uint64_t* k_empty = bars + 4;   // [2]
+  uint64_t* v_full = bars + 6;    // [2]
+  uint64_t* v_empty = bars + 8;   // [2]
+  uint64_t* s_full = bars + 10;   // [2] per tile: S of a block in TMEM
+  uint64_t* p_full = bars + 12;   // [2] per tile: P of a block in TMEM
+  uint64_t* pv_done = bars + 14;  // [2] per tile: P V of a block complete
+  uint64_t* drain = bars + 16;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 17);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_holder + 2);   // [4]
 
   const int warp = warp_id(), lane = lane_id();
   const int nq = (T + 127) / 128;
-  const int pair = (gridDim.x - 1) - blockIdx.x;   // longest pairs first
-  const int bh = blockIdx.y;
-  const int bkv = (bh / H) * Hkv + (bh - (bh / H) * H) / (H / Hkv);   // kv head of this query head
-  const int qtA = 2 * pair;
-  const bool hasB = qtA + 1 < nq;
-  // key blocks j0 .. qt (causal, and not before the first row's window); both
-  // tiles start at j0, rows for which a block lies wholly outside their window
-  // see only masked scores there
-  const int j0 = max(0, qtA * 128 - wl) / 128;
-  const int nkvA = qtA + 1 - j0;
-  const int nkvB = hasB ? qtA + 2 - j0 : 0;
-  const int nkv = hasB ? nkvB : nkvA;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1 + 8);   // the MMA commit and one arrival per softmax warp
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
@@ -137,41 +165,60 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 40;\n" ::: "memory");
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------------- TMA
       bool ok = true;
-      int issued_k = 0, issued_v = 0;
-      mbar_arrive_expect_tx(q_full, hasB ? 2 * TF_BUF : TF_BUF);
-      tma_load_3d(sQ, &tq, q_full, 0, qtA * 128, bh);
-      tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, qtA * 128, bh);
-      if (hasB) {
-        tma_load_3d(sQ + TF_BUF, &tq, q_full, 0, qtA * 128 + 128, bh);
-        tma_load_3d(sQ + TF_BUF + TF_TILE, &tq, q_full, 64, qtA * 128 + 128, bh);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        if (!mbar_wait(&k_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
-        const int kc = (j0 + j) * 128;
-        mbar_arrive_expect_tx(&k_full[s], TF_BUF);
-        tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, kc, bkv);
-        tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, kc, bkv);
-        ++issued_k;
-        if (!mbar_wait(&v_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
-        mbar_arrive_expect_tx(&v_full[s], TF_BUF);
-        tma_load_3d(sV + s * TF_BUF, &tv, &v_full[s], 0, kc, bkv);
-        tma_load_3d(sV + s * TF_BUF + TF_TILE, &tv, &v_full[s], 64, kc, bkv);
-        ++issued_v;
+      int g = 0, last_q = -1;   // ring position of the next K/V block; last item whose Q was loaded
+      for (int n = 0;; ++n) {
+        // the previous item's Q is no longer read and every warp has its number
+        if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1, abort_flag, err)) { ok = false; break; }
+        int idx = sched ? atomicAdd(sched, 1) : n * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
+        if (idx >= n_items) idx = -1;
+        item_ring[n & 3] = idx;
+        if (idx < 0) {
+          mbar_arrive(q_full);   // end marker: releases the ring entry
+          break;
+        }
+        const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+        mbar_arrive_expect_tx(q_full, it.hasB ? 2 * TF_BUF : TF_BUF);
+        tma_load_3d(sQ, &tq, q_full, 0, it.qtA * 128, it.bh);
+        tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, it.qtA * 128, it.bh);
+        if (it.hasB) {
+          tma_load_3d(sQ + TF_BUF, &tq, q_full, 0, it.qtA * 128 + 128, it.bh);
+          tma_load_3d(sQ + TF_BUF + TF_TILE, &tq, q_full, 64, it.qtA * 128 + 128, it.bh);
+        }
+        last_q = n;
+        for (int j = 0; j < it.nkv; ++j) {
+          const int s = g & 1;
+          const uint32_t par = (g >> 1) & 1;
+          const int kc = (it.j0 + j) * 128;
+          if (!mbar_wait(&k_empty[s], par ^ 1u, abort_flag, err)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[s], TF_BUF);
+          tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, kc, it.bkv);
+          tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, kc, it.bkv);
+          if (!mbar_wait(&v_empty[s], par ^ 1u, abort_flag, err)) {
+            // K of this block is in flight: count it, V is not
+            for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&k_full[s], par); ++i) {}
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[s], TF_BUF);
+          tma_load_3d(sV + s * TF_BUF, &tv, &v_full[s], 0, kc, it.bkv);
+          tma_load_3d(sV + s * TF_BUF + TF_TILE, &tv, &v_full[s], 64, kc, it.bkv);
+          ++g;
+        }
+        if (!ok) break;
       }
       if (!ok) {
         // let the copies already started land before the CTA exits
-        for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(q_full, 0); ++i) {}
-        for (int j = (issued_k > 2 ? issued_k - 2 : 0); j < issued_k; ++j)
-          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&k_full[j & 1], (j >> 1) & 1); ++i) {}
-        for (int j = (issued_v > 2 ? issued_v - 2 : 0); j < issued_v; ++j)
-          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&v_full[j & 1], (j >> 1) & 1); ++i) {}
+        if (last_q >= 0)
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(q_full, last_q & 1); ++i) {}
+        for (int x = (g > 2 ? g - 2 : 0); x < g; ++x) {
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&k_full[x & 1], (x >> 1) & 1); ++i) {}
+          for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&v_full[x & 1], (x >> 1) & 1); ++i) {}
+        }
       }
     }
   } else if (warp == 1) {
@@ -179,200 +226,234 @@ __global__ void __launch_bounds__(384, 1)
       // -------------------------------------------------------------- MMA
       constexpr uint32_t IDESC_S = make_idesc(1, 128, false, false);
       constexpr uint32_t IDESC_O = make_idesc(1, 128, false, true);
-      bool ok = mbar_wait(q_full, 0, abort_flag, err);
-      // S_t = Q_t K_j^T into TMEM columns 128 t
-      auto issue_s = [&](int t, int j) {
-        const uint32_t q_addr = smem_u32(sQ + t * TF_BUF);
-        const uint32_t k_addr = smem_u32(sK + (j & 1) * TF_BUF);
+      // The descriptors of a product are its first one plus the byte offset / 16
+      // (the start address field); the empty asm keeps the compiler from
+      // hoisting every descriptor of the kernel into registers.
+      // S_t = Q_t K^T (K in ring slot ks) into TMEM columns 128 t
+      auto issue_s = [&](int t, int ks) {
+        uint64_t dq = smem_desc_sw128(smem_u32(sQ + t * TF_BUF), 16, 1024);
+        uint64_t dk = smem_desc_sw128(smem_u32(sK + ks * TF_BUF), 16, 1024);
+        asm volatile("" : "+l"(dq), "+l"(dk));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * TF_TILE + (kk & 3) * 32;
-          umma_f16(tmem + t * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                   smem_desc_sw128(k_addr + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+          const uint32_t off16 = ((kk >> 2) * TF_TILE + (kk & 3) * 32) >> 4;
+          umma_f16(tmem + t * 128, dq + off16, dk + off16, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[t]);
       };
-      // O_t += P_t V_j, P_t from TMEM (16 keys = 8 packed columns per step)
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t v_addr = smem_u32(sV + (j & 1) * TF_BUF);
+      // O_t (+)= P_t V (V in ring slot vs), P_t from TMEM (16 keys = 8 packed columns per step)
+      auto issue_pv = [&](int t, int vs, bool acc) {
+        uint64_t dv = smem_desc_sw128(smem_u32(sV + vs * TF_BUF), TF_TILE, 1024);
+        asm volatile("" : "+l"(dv));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_f16_tmem_a(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                          smem_desc_sw128(v_addr + kk * 2048, TF_TILE, 1024), IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_f16_tmem_a(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, dv + ((kk * 2048) >> 4), IDESC_O,
+                          (acc || kk > 0) ? 1u : 0u);
         umma_commit(&pv_done[t]);
       };
-      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, err);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        if (hasB) issue_s(1, 0);
-        umma_commit(&k_empty[0]);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int s = j & 1;
-        const uint32_t par = (j >> 1) & 1;
-        const int s1 = (j + 1) & 1;
-        if (!mbar_wait(&v_full[s], par, abort_flag, err)) { ok = false; break; }
-        if (j + 1 < nkv && !mbar_wait(&k_full[s1], ((j + 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
-        // per tile: O += P V_j, then S of the next block over P once that product
-        // has read it (tile B's softmax trails tile A's, so A goes first)
-        for (int t = 0; t < 2; ++t) {
-          if (j >= (t ? nkvB : nkvA)) continue;
-          if (!mbar_wait(&p_full[t], j & 1, abort_flag, err)) { ok = false; break; }
+      bool ok = true;
+      int g0 = 0;                  // ring position of the item's first key block
+      uint32_t npv[2] = {0u, 0u};  // P V products issued per tile so far
+      for (int n = 0; ok; ++n) {
+        if (!mbar_wait(q_full, n & 1, abort_flag, err)) { ok = false; break; }
+        const int idx = item_ring[n & 3];
+        if (idx < 0) break;
+        const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+        // S of the first block on both tiles, each once its previous P V (which
+        // reads P from the same columns) has completed
+        if (!mbar_wait(&k_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err)) { ok = false; break; }
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (t == 1 && !it.hasB) break;
+          if (npv[t] > 0 && !mbar_wait(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err)) { ok = false; break; }
           tc_fence_after();
-          issue_pv(t, j);
-          if (j + 1 < (t ? nkvB : nkvA)) {
-            if (!mbar_wait(&pv_done[t], j & 1, abort_flag, err)) { ok = false; break; }
-            tc_fence_after();
-            issue_s(t, j + 1);
-          }
+          issue_s(t, g0 & 1);
         }
         if (!ok) break;
-        umma_commit(&v_empty[s]);
-        if (j + 1 < nkv) umma_commit(&k_empty[s1]);
+        if (it.nkv == 1) umma_commit(q_empty);   // the item's last S
+        umma_commit(&k_empty[g0 & 1]);
+        for (int j = 0; j < it.nkv && ok; ++j) {
+          const int gj = g0 + j;
+          const int s = gj & 1;
+          const int s1 = (gj + 1) & 1;
+          if (!mbar_wait(&v_full[s], (gj >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          if (j + 1 < it.nkv && !mbar_wait(&k_full[s1], ((gj + 1) >> 1) & 1, abort_flag, err)) { ok = false; break; }
+          // per tile: O += P V_j, then S of the next block over P once that product
+          // has read it (tile B's softmax trails tile A's, so A goes first)
+          for (int t = 0; t < 2; ++t) {
+            const int nkv_t = t ? it.nkvB : it.nkvA;
+            if (j >= nkv_t) continue;
+            if (!mbar_wait(&p_full[t], npv[t] & 1, abort_flag, err)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(t, s, j > 0);
+            ++npv[t];
+            if (j + 1 < nkv_t) {
+              if (!mbar_wait(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err)) { ok = false; break; }
+              tc_fence_after();
+              issue_s(t, s1);
+              if (j + 1 == it.nkv - 1) umma_commit(q_empty);   // the item's last S
+            }
+          }
+          if (!ok) break;
+          umma_commit(&v_empty[s]);
+          if (j + 1 < it.nkv) umma_commit(&k_empty[s1]);
+        }
+        g0 += it.nkv;
       }
       umma_commit(drain);
       for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
     }
   } else if (warp >= 4) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;\n" ::: "memory");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
     // ---------------------------------------------------------- softmax
     const int tile = (warp - 4) >> 2;           // 0: A, 1: B
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int qt = qtA + tile;
-    const int q0 = qt * 128;
-    const int q = q0 + r;
-    const int nkv_t = tile ? nkvB : nkvA;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t t_s = tmem + lane_base + tile * 128;
     const uint32_t t_o = tmem + lane_base + 256 + tile * 128;
     const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
-    float m_ref = -INFINITY, l = 0.f;   // reference max (log2 units) and row sum relative to it
     bool ok = true;
+    uint32_t nblk = 0;   // S blocks consumed on this tile so far
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
       const bool got = mbar_wait(bar, par, abort_flag, err);
       __syncwarp();
       return __all_sync(0xffffffffu, got);
     };
-    for (int j = 0; j < nkv_t && ok; ++j) {
-      if (!wait_all(&s_full[tile], j & 1)) { ok = false; break; }
-      tc_fence_after();
-      // the whole S row at once
-      uint32_t sr[128];
-      {
-        uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t (&r2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-        uint32_t (&r3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-        tmem_load32_async(t_s, r0);
-        tmem_load32_async(t_s + 32, r1);
-        tmem_load32_async(t_s + 64, r2);
-        tmem_load32_async(t_s + 96, r3);
-        tmem_wait_ld();
-      }
-      const int kbase = (j0 + j) * 128;
-      if ((j0 + j == qt) || (kbase + 128 > T) || (kbase < q0 + 127 - wl)) {
-        // causal diagonal, ragged tail or window edge: masked scores become -inf
-#pragma unroll
-        for (int k = 0; k < 128; ++k) {
-          const int key = kbase + k;
-          if (key > q || key >= T || key < q - wl) sr[k] = __float_as_uint(-INFINITY);
+    for (int n = 0; ok; ++n) {
+      if (!wait_all(q_full, n & 1)) { ok = false; break; }
+      const int idx = item_ring[n & 3];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_empty);   // this warp has the item number
+      if (idx < 0) break;
+      const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+      if (tile == 1 && !it.hasB) continue;
+      const int qt = it.qtA + tile;
+      const int q0 = qt * 128;
+      const int q = q0 + r;
+      const int nkv_t = tile ? it.nkvB : it.nkvA;
+      float m_ref = -INFINITY, l = 0.f;   // reference max (log2 units) and row sum relative to it
+      for (int j = 0; j < nkv_t && ok; ++j) {
+        if (!wait_all(&s_full[tile], nblk & 1)) { ok = false; break; }
+        ++nblk;
+        tc_fence_after();
+        // the whole S row at once
+        uint32_t sr[128];
+        {
+          uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+          uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+          uint32_t (&r2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+          uint32_t (&r3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+          tmem_load32_async(t_s, r0);
+          tmem_load32_async(t_s + 32, r1);
+          tmem_load32_async(t_s + 64, r2);
+          tmem_load32_async(t_s + 96, r3);
+          tmem_wait_ld();
         }
+        const int kbase = (it.j0 + j) * 128;
+        if ((it.j0 + j == qt) || (kbase + 128 > T) || (kbase < q0 + 127 - wl)) {
+          // causal diagonal, ragged tail or window edge: masked scores become -inf
+#pragma unroll
+          for (int k = 0; k < 128; ++k) {
+            const int key = kbase + k;
+            if (key > q || key >= T || key < q - wl) sr[k] = __float_as_uint(-INFINITY);
+          }
+        }
+        // block max of the raw scores (the scale is positive), eight independent chains
+        float mx8[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
+#pragma unroll
+        for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(sr[k]));
+        const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mblk = mraw * scale_log2;
+        const bool move = mblk > m_ref + TF_RESCALE;   // true on the first block with a visible key
+        const float m_new = move ? mblk : m_ref;
+        // 1 when the reference stays, 0 when it leaves -inf; a row that has seen
+        // only masked scores (window edge) keeps -inf and offsets by 0 below
+        const bool none = m_new == -INFINITY;
+        const float factor = none ? 1.f : ex2_approx(m_ref - m_new);
+        // O holds the products of blocks < j (S of this block was issued after
+        // the last of them completed), so it may be rescaled now
+        if (j >= 1 && __any_sync(0xffffffffu, move)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ra[32];
+            tmem_load32_async(t_o + c * 32, ra);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ra[k] = __float_as_uint(__uint_as_float(ra[k]) * factor);
+            tmem_store32(t_o + c * 32, ra);
+          }
+        }
+        // probabilities relative to the reference (masked scores give 0), row sum,
+        // bf16 P over the first 64 columns of S
+        const float m_off = none ? 0.f : m_new;
+        const uint64_t nb2 = f2_pack(-m_off, -m_off);
+        uint64_t rs2 = f2_pack(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int k = 0; k < 64; k += 8) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c * 64 + k + e]), __uint_as_float(sr[c * 64 + k + e + 1])),
+                               sl2, nb2),
+                        x0, x1);
+              if (e < 4 || (e == 4 && (k & 8))) {
+                p[e] = ex2_approx(x0);
+                p[e + 1] = ex2_approx(x1);
+              } else {
+                f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+              }
+            }
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              rs2 = f2_add(rs2, f2_pack(p[e], p[e + 1]));
+              pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
+            }
+          }
+          tmem_store32(t_s + c * 32, pk);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(&p_full[tile]);
+        float rs0, rs1;
+        f2_unpack(rs2, rs0, rs1);
+        l = l * factor + (rs0 + rs1);
+        m_ref = m_new;
       }
-      // block max of the raw scores (the scale is positive), eight independent chains
-      float mx8[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
-#pragma unroll
-      for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(sr[k]));
-      const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      const float mblk = mraw * scale_log2;
-      const bool move = mblk > m_ref + TF_RESCALE;   // true on the first block with a visible key
-      const float m_new = move ? mblk : m_ref;
-      // 1 when the reference stays, 0 when it leaves -inf; a row that has seen
-      // only masked scores (window edge) keeps -inf and offsets by 0 below
-      const bool none = m_new == -INFINITY;
-      const float factor = none ? 1.f : ex2_approx(m_ref - m_new);
-      // O holds the products of blocks < j (S of this block was issued after
-      // the last of them completed), so it may be rescaled now
-      if (j >= 1 && __any_sync(0xffffffffu, move)) {
+      // epilogue: O / l once the last P V has landed
+      if (ok) ok = wait_all(&pv_done[tile], (nblk - 1) & 1);
+      if (ok) {
+        tc_fence_after();
+        const int b = it.bh / H, h = it.bh - (it.bh / H) * H;
+        const float inv = 1.f / l;
+        bf16* orow = o + (static_cast<long long>(b) * T + q) * (static_cast<long long>(H) * 128) + h * 128;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t ra[32];
           tmem_load32_async(t_o + c * 32, ra);
           tmem_wait_ld();
+          if (q < T) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) ra[k] = __float_as_uint(__uint_as_float(ra[k]) * factor);
-          tmem_store32(t_o + c * 32, ra);
-        }
-      }
-      // probabilities relative to the reference (masked scores give 0), row sum,
-      // bf16 P over the first 64 columns of S
-      const float m_off = none ? 0.f : m_new;
-      const uint64_t nb2 = f2_pack(-m_off, -m_off);
-      uint64_t rs2 = f2_pack(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 64; k += 8) {
-          float p[8];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c * 64 + k + e]), __uint_as_float(sr[c * 64 + k + e + 1])),
-                             sl2, nb2),
-                      x0, x1);
-            if (e < 4 || (e == 4 && (k & 8))) {
-              p[e] = ex2_approx(x0);
-              p[e + 1] = ex2_approx(x1);
-            } else {
-              f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+            for (int k = 0; k < 32; k += 8) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(ra[k]) * inv, __uint_as_float(ra[k + 1]) * inv);
+              w.y = pack_bf16x2(__uint_as_float(ra[k + 2]) * inv, __uint_as_float(ra[k + 3]) * inv);
+              w.z = pack_bf16x2(__uint_as_float(ra[k + 4]) * inv, __uint_as_float(ra[k + 5]) * inv);
+              w.w = pack_bf16x2(__uint_as_float(ra[k + 6]) * inv, __uint_as_float(ra[k + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + c * 32 + k) = w;
             }
           }
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            rs2 = f2_add(rs2, f2_pack(p[e], p[e + 1]));
-            pk[(k + e) >> 1] = pack_bf16x2(p[e], p[e + 1]);
-          }
         }
-        tmem_store32(t_s + c * 32, pk);
+        if (q < T) lse[static_cast<long long>(it.bh) * T + q] = (m_ref + log2f(l)) * 0.69314718055994531f;
+        // O of this tile has been read: the next item's first P V may overwrite it
+        tc_fence_before();
       }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(&p_full[tile]);
-      float rs0, rs1;
-      f2_unpack(rs2, rs0, rs1);
-      l = l * factor + (rs0 + rs1);
-      m_ref = m_new;
-    }
-    // epilogue: O / l once the last P V has landed
-    if (ok && nkv_t > 0) ok = wait_all(&pv_done[tile], (nkv_t - 1) & 1);
-    if (ok) {
-      tc_fence_after();
-      const int b = bh / H, h = bh - (bh / H) * H;
-      const float inv = 1.f / l;
-      bf16* orow = o + (static_cast<long long>(b) * T + q) * (static_cast<long long>(H) * 128) + h * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t ra[32];
-        tmem_load32_async(t_o + c * 32, ra);
-        tmem_wait_ld();
-        if (q < T) {
-#pragma unroll
-          for (int k = 0; k < 32; k += 8) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(ra[k]) * inv, __uint_as_float(ra[k + 1]) * inv);
-            w.y = pack_bf16x2(__uint_as_float(ra[k + 2]) * inv, __uint_as_float(ra[k + 3]) * inv);
-            w.z = pack_bf16x2(__uint_as_float(ra[k + 4]) * inv, __uint_as_float(ra[k + 5]) * inv);
-            w.w = pack_bf16x2(__uint_as_float(ra[k + 6]) * inv, __uint_as_float(ra[k + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + k) = w;
-          }
-        }
-      }
-      if (q < T) lse[static_cast<long long>(bh) * T + q] = (m_ref + log2f(l)) * 0.69314718055994531f;
     }
   }
 
@@ -908,8 +989,35 @@ __global__ void attn_bwd_dot_kernel(const bf16* __restrict__ o, const bf16* __re
 // bound no row reaches (kept small enough that k0 + 127 + wl fits in an int).
 static int window_bound(int window, int T) { return window < 0 || window >= T ? (1 << 30) : window; }
 
+static int sm_count() {
+  static int n = 0;
+  if (n <= 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// Scheduler words for callers that bring none: a ring of 64 library-owned
+// counters, one per launch in turn, each zeroed on the launch's stream
+// before use (so up to 64 such launches may be in flight at once).
+__device__ int g_sched_ring[64];
+
+static int* sched_word(int* sched, cudaStream_t s) {
+  if (!sched) {
+    static unsigned next = 0;
+    int* base = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&base), g_sched_ring) != cudaSuccess) return nullptr;
+    sched = base + (next++ & 63u);
+  }
+  cudaMemsetAsync(sched, 0, sizeof(int), s);
+  return sched;
+}
+
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s, int* err, int Hkv, int window) {
+                     cudaStream_t s, int* err, int Hkv, int window, int* sched) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
@@ -924,10 +1032,12 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
     return;
   }
-  dim3 grid(((T + 127) / 128 + 1) / 2, B * H);   // pairs of query tiles
+  // persistent: one CTA per SM over the pairs of query tiles of every head
+  const long long n_items = ((T + 127) / 128 + 1) / 2 * bh;
+  const int grid = static_cast<int>(std::min<long long>(n_items, sm_count()));
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
   attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, T, window_bound(window, T), scale_log2,
-                                                err);
+                                                static_cast<int>(n_items), sched_word(sched, s), err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,

@@ -11,9 +11,11 @@ using bf16 = __nv_bfloat16;
 // q [B, H, T, 128], k, v [B, Hkv, T, 128] -> o [B, T, H, 128], lse [B, H, T]
 // (natural log).  Hkv <= 0 means Hkv = H (it must divide H); window < 0 (or
 // >= T) is full causal attention, else query t sees keys t - window .. t.
-// err: device error word for expired waits (may be null).
+// err: device error word for expired waits (may be null).  sched: a device
+// int the persistent kernel hands out its work with (zeroed here, on s); null
+// takes one of the library's own.
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s, int* err, int Hkv = 0, int window = -1);
+                     cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr);
 
 // Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32
 // [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, Hkv, T, 128]
