@@ -619,7 +619,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, H, D.window(l));
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, H, D.window(l), c->A<int>(P.sched));
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);

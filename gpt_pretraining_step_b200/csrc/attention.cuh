@@ -19,9 +19,10 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 
 // Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32
 // [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, Hkv, T, 128]
-// (summed over the query heads of each kv head); Dv [B, H, T] is scratch.
+// (summed over the query heads of each kv head); Dv [B, H, T] is scratch;
+// sched as for the forward.
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s, int* err, int Hkv = 0, int window = -1);
+                     cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr);
 
 }  // namespace gpt
