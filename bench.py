@@ -51,6 +51,8 @@ def parse():
                     help="NorMuon variance reduction on the Muon updates with this second-moment decay")
     ap.add_argument("--window-pattern", default="", help='per-layer attention windows, e.g. "SSSL" (S = sliding)')
     ap.add_argument("--short-window", type=int, default=1024, help="left context of an S layer, tokens")
+    ap.add_argument("--shard-optimizer", action="store_true",
+                    help="N > 1: each rank runs Muon on its own layer range (three-phase ZeRO-2 style exchange)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--breakdown", action="store_true", help="per-category device times in the JSON line")
@@ -271,6 +273,10 @@ def run_ours(a):
 
     def step():
         st.fwd_bwd(tok, tgt)
+        if a.shard_optimizer and world > 1:
+            dp.sharded_optimizer_step(st, s.depth, muon=hp["muon"], adam=hp["adam"],
+                                      normuon_beta2=-1.0 if a.normuon is None else a.normuon)
+            return
         if grads is not None:
             dp.average_gradients(grads)
         if a.normuon is None:
@@ -383,7 +389,7 @@ def run_ours(a):
             "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
             "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)", "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
-                       "parallelism": f"dp{world}", "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
+                       "parallelism": f"dp{world}" + ("+sharded-optimizer" if a.shard_optimizer and world > 1 else ""), "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
                        "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
                        "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
                                      else "full causal")},
@@ -427,6 +433,13 @@ def run_e2e(a, st, s, rank, world, grads, stream):
         dtok.copy_(tok, non_blocking=True)
         dtgt.copy_(tgt, non_blocking=True)
         loss = st.fwd_bwd(dtok, dtgt)
+        if a.shard_optimizer and world > 1:
+            dp.sharded_optimizer_step(st, s.depth, muon=(hp.muon_lr, hp.muon_momentum, hp.muon_wd),
+                                      adam=(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd),
+                                      normuon_beta2=-1.0 if a.normuon is None else a.normuon)
+            loss_host.copy_(loss.reshape(1), non_blocking=True)
+            stream.synchronize()
+            return float(loss_host[0])
         dp.average_gradients(grads)
         if a.normuon is None:
             st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)

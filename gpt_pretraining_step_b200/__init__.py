@@ -15,13 +15,14 @@ LIB_PATH = os.path.join(HERE, "libgpt.so")
 
 GPT_OK, GPT_EINVAL, GPT_ERANGE, GPT_ETIMEOUT, GPT_ECUDA = 0, -1, -2, -3, -4
 KIND_PARAM, KIND_GRAD, KIND_MOM, KIND_ADAM_M, KIND_ADAM_V, KIND_NORMUON_V = 0, 1, 2, 3, 4, 5
+REGION_MASTER, REGION_BF16, REGION_GRAD = 0, 1, 2
 GROUP_ADAMW, GROUP_MUON = 0, 1
 PROF_CATEGORIES = ["qkv_gemm", "proj_gemm", "fc_gemm", "down_gemm", "attn_fwd", "attn_bwd", "logits_gemm",
                    "ce_finish", "lm_dx_gemm", "lm_dw_gemm", "dx_gemm", "dw_gemm", "norm", "qk_bwd", "embed",
                    "ns_gemm", "muon_elem", "adamw", "fp8_quant"]
 
 ABI_FUNCTIONS = [
-    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "muon_step_normuon", "adamw_step", "gpt_train_step_host",
+    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "muon_step_normuon", "muon_step_layers", "gpt_block_region", "adamw_step", "gpt_train_step_host",
     "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
     "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3",
     "gpt_op_matmul_fp8", "gpt_op_attention_fwd",
@@ -68,6 +69,8 @@ def lib():
             "gpt_fwd_bwd": (i32, [vp, vp, vp, vp, i32]),
             "muon_step": (i32, [vp, f32, f32, f32]),
             "muon_step_normuon": (i32, [vp, f32, f32, f32, f32]),
+            "muon_step_layers": (i32, [vp, f32, f32, f32, f32, i32, i32]),
+            "gpt_block_region": (i32, [vp, i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
             "adamw_step": (i32, [vp, f32, f32, f32, f32, f32]),
             "gpt_train_step_host": (i32, [vp, vp, vp, ctypes.POINTER(HParams), vp]),
             "gpt_num_tensors": (i32, [vp]),
@@ -173,6 +176,31 @@ class GPTStep:
 
     def muon_step_normuon(self, lr=0.02, momentum=0.95, weight_decay=0.0, beta2=0.95):
         _check(lib().muon_step_normuon(self.h, lr, momentum, weight_decay, beta2))
+
+    def muon_step_layers(self, l0, l1, lr=0.02, momentum=0.95, weight_decay=0.0, normuon_beta2=-1.0):
+        """Muon (or NorMuon with normuon_beta2 >= 0) of layers l0 .. l1-1 only."""
+        _check(lib().muon_step_layers(self.h, lr, momentum, weight_decay, normuon_beta2, int(l0), int(l1)))
+
+    def block_region(self, what, kind, l0, l1):
+        """Tensor view of block matrix kind (0 q|k|v, 1 attention output, 2 MLP
+        up, 3 MLP down) for layers l0 .. l1-1: REGION_MASTER (fp32), REGION_BF16
+        (bf16 working copies) or REGION_GRAD (fp32 gradients)."""
+        import torch
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_block_region(self.h, int(what), int(kind), int(l0), int(l1), ctypes.byref(off),
+                                      ctypes.byref(n)))
+        buf = self.bufs[1] if what == REGION_GRAD else self.bufs[0]
+        return buf[off.value:off.value + n.value].view(torch.bfloat16 if what == REGION_BF16 else torch.float32)
+
+    def adamw_grad_view(self):
+        """fp32 gradients of the token embedding and lm_head (the part of the
+        gradient span before the block matrices)."""
+        import torch
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_grad_region(self.h, ctypes.byref(off), ctypes.byref(n)))
+        first, size = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_block_region(self.h, REGION_GRAD, 0, 0, 0, ctypes.byref(first), ctypes.byref(size)))
+        return self.bufs[1][off.value:first.value].view(torch.float32)
 
     def adamw_step(self, lr=3e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.0):
         _check(lib().adamw_step(self.h, lr, beta1, beta2, eps, weight_decay))

@@ -864,23 +864,29 @@ int gpt_fwd_bwd(gpt_ctx* c, const int32_t* tokens, const int32_t* targets, float
   return forward_backward(c, tokens, targets, loss_out, accumulate != 0);
 }
 
-// Muon over every block matrix; with normuon the orthogonalised updates get
-// the NorMuon per-neuron scaling (second-moment EMA with factor beta2) first.
-static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay, bool normuon, float beta2) {
+// Muon over the block matrices of layers [l0, l1); with normuon the
+// orthogonalised updates get the NorMuon per-neuron scaling (second-moment
+// EMA with factor beta2) first.  Every matrix is updated on its own, so a
+// range gives bit-for-bit the result the whole set gives for those layers.
+static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay, bool normuon, float beta2, int l0,
+                       int l1) {
   int rc = check_ctx(c);
   if (rc) return rc;
   const Dims& D = c->D;
   const Plan& P = c->P;
+  if (l0 < 0 || l1 > D.L || l0 > l1) return fail(GPT_EINVAL, "layer range out of bounds");
+  if (l0 == l1) return GPT_OK;
   cudaStream_t s = c->stream;
   const int L = D.L, d = D.d, F = D.F;
+  const int nl = l1 - l0;
   float* inv = c->A<float>(P.inv_norm);
-  // momentum and Frobenius norms of every block matrix
+  // momentum and Frobenius norms of every block matrix in the range
   const long long ne[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
   {
     ProfScope ps(c, GPT_PROF_MUON_ELEM);
     for (int j = 0; j < 4; ++j)
-      launch_muon_momentum(c->Mom(2 + j), c->G(2 + j), ne[j], L, momentum, 1e-7f, inv + j * L, c->A<void>(P.normws),
-                           s);
+      launch_muon_momentum(c->Mom(2 + j) + l0 * ne[j], c->G(2 + j) + l0 * ne[j], ne[j], nl, momentum, 1e-7f,
+                           inv + j * L + l0, c->A<void>(P.normws), s);
   }
   c->launches += 8;
   // first Newton-Schulz iterate: fp32 for the fp16 and tf32 modes, bf16 otherwise
@@ -895,8 +901,8 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
   // output (c = d), and MLP up plus transposed MLP down (c = 4d)
   struct Member { int grp; bool transpose; };
   struct Batch { int nz; int cc; Member m[2]; int nm; };
-  const Batch batches[3] = {{L, 3 * d, {{2, false}}, 1}, {L, d, {{3, false}}, 1},
-                            {2 * L, F, {{4, false}, {5, true}}, 2}};
+  const Batch batches[3] = {{nl, 3 * d, {{2, false}}, 1}, {nl, d, {{3, false}}, 1},
+                            {2 * nl, F, {{4, false}, {5, true}}, 2}};
   for (const Batch& bt : batches) {
     const size_t per = static_cast<size_t>(d) * bt.cc;
     for (int i = 0; i < bt.nm; ++i) {
@@ -904,14 +910,16 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
       const Member& mm = bt.m[i];
       // X (d x cc) and, for tf32 steps, its transpose, from one read of the
       // momentum, which is stored d x cc, or cc x d for the MLP down matrix
-      void* dst = static_cast<uint8_t*>(X0) + static_cast<size_t>(i) * L * per * es0;
-      void* dstT = D.n_tf32 > 0 ? static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * L * per * es0 : nullptr;
+      void* dst = static_cast<uint8_t*>(X0) + static_cast<size_t>(i) * nl * per * es0;
+      void* dstT = D.n_tf32 > 0 ? static_cast<uint8_t*>(XT0) + static_cast<size_t>(i) * nl * per * es0 : nullptr;
       // fp16 mode: the fp16 operand copy of X, same layout as X
-      __half* dstH = D.n_tf32 < 0 ? reinterpret_cast<__half*>(XT0) + static_cast<size_t>(i) * L * per : nullptr;
+      __half* dstH = D.n_tf32 < 0 ? reinterpret_cast<__half*>(XT0) + static_cast<size_t>(i) * nl * per : nullptr;
+      const float* mom = c->Mom(mm.grp) + l0 * per;
+      const float* invg = inv + (mm.grp - 2) * L + l0;
       if (!mm.transpose)
-        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dst, dstT, es0, L, d, bt.cc, s, dstH, nullptr);
+        launch_muon_make_x(mom, invg, dst, dstT, es0, nl, d, bt.cc, s, dstH, nullptr);
       else
-        launch_muon_make_x(c->Mom(mm.grp), inv + (mm.grp - 2) * L, dstT, dst, es0, L, bt.cc, d, s, nullptr, dstH);
+        launch_muon_make_x(mom, invg, dstT, dst, es0, nl, bt.cc, d, s, nullptr, dstH);
       c->launches += 1;
     }
     void* res = nullptr;
@@ -919,24 +927,22 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
     rc = newton_schulz(c, bt.nz, d, bt.cc, X0, X1, XT0, XT1, Ab, Bb, D.n_tf32, s, c->err(), &res, &res_es,
                        &c->launches);
     if (rc) return rc;
-    // NorMuon: one factor per row of res (the shorter axis of every matrix);
-    // the members of a batch have contiguous second-moment vectors
-    float* rowf = nullptr;
-    if (normuon) {
-      ProfScope ps(c, GPT_PROF_MUON_ELEM);
-      rowf = c->A<float>(P.nfac);
-      launch_normuon_factor(res, res_es, bt.nz, d, bt.cc, c->NV(bt.m[0].grp), beta2, rowf, s);
-      c->launches += 2;
-    }
     for (int i = 0; i < bt.nm; ++i) {
       ProfScope ps(c, GPT_PROF_MUON_ELEM);
       const Member& mm = bt.m[i];
       const int rows = mm.grp == 5 ? F : d;
       const int cols = mm.grp == 2 ? 3 * d : (mm.grp == 3 ? d : (mm.grp == 4 ? F : d));
       const float scale = sqrtf(std::max(1.f, static_cast<float>(rows) / static_cast<float>(cols)));
-      const void* src = static_cast<const uint8_t*>(res) + static_cast<size_t>(i) * L * per * res_es;
-      launch_muon_apply(c->W(mm.grp), c->Wb(mm.grp), src, res_es, L, d, bt.cc, mm.transpose, lr, weight_decay,
-                        scale, s, rowf ? rowf + static_cast<size_t>(i) * L * d : nullptr);
+      const void* src = static_cast<const uint8_t*>(res) + static_cast<size_t>(i) * nl * per * res_es;
+      // NorMuon: one factor per row of res (the shorter axis of every matrix)
+      float* rowf = nullptr;
+      if (normuon) {
+        rowf = c->A<float>(P.nfac) + static_cast<size_t>(i) * nl * d;
+        launch_normuon_factor(src, res_es, nl, d, bt.cc, c->NV(mm.grp) + static_cast<size_t>(l0) * d, beta2, rowf, s);
+        c->launches += 2;
+      }
+      launch_muon_apply(c->W(mm.grp) + l0 * per, c->Wb(mm.grp) + l0 * per, src, res_es, nl, d, bt.cc, mm.transpose,
+                        lr, weight_decay, scale, s, rowf);
       c->launches += 1;
     }
   }
@@ -945,12 +951,41 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
 }
 
 int muon_step(gpt_ctx* c, float lr, float momentum, float weight_decay) {
-  return muon_update(c, lr, momentum, weight_decay, false, 0.f);
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  return muon_update(c, lr, momentum, weight_decay, false, 0.f, 0, c->D.L);
 }
 
 int muon_step_normuon(gpt_ctx* c, float lr, float momentum, float weight_decay, float beta2) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
   if (!(beta2 >= 0.f && beta2 < 1.f)) return fail(GPT_EINVAL, "NorMuon beta2 must be in [0, 1)");
-  return muon_update(c, lr, momentum, weight_decay, true, beta2);
+  return muon_update(c, lr, momentum, weight_decay, true, beta2, 0, c->D.L);
+}
+
+int muon_step_layers(gpt_ctx* c, float lr, float momentum, float weight_decay, float normuon_beta2, int l0,
+                     int l1) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!(normuon_beta2 < 1.f)) return fail(GPT_EINVAL, "NorMuon beta2 must be below 1 (negative: plain Muon)");
+  return muon_update(c, lr, momentum, weight_decay, normuon_beta2 >= 0.f, normuon_beta2, l0, l1);
+}
+
+int gpt_block_region(const gpt_ctx* c, int what, int kind, int l0, int l1, size_t* offset_bytes,
+                     size_t* size_bytes) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (kind < 0 || kind > 3) return fail(GPT_EINVAL, "block matrix kind must be 0..3");
+  if (what < GPT_REGION_MASTER || what > GPT_REGION_GRAD) return fail(GPT_EINVAL, "unknown region");
+  if (l0 < 0 || l1 > c->D.L || l0 > l1) return fail(GPT_EINVAL, "layer range out of bounds");
+  const int grp = 2 + kind;
+  const size_t d = c->D.d, F = c->D.F;
+  const size_t per[4] = {d * 3 * d, d * d, d * F, F * d};
+  const size_t es = what == GPT_REGION_BF16 ? 2 : 4;
+  const size_t base = what == GPT_REGION_MASTER ? c->P.w[grp] : (what == GPT_REGION_BF16 ? c->P.wb[grp] : c->P.g[grp]);
+  if (offset_bytes) *offset_bytes = base + static_cast<size_t>(l0) * per[kind] * es;
+  if (size_bytes) *size_bytes = static_cast<size_t>(l1 - l0) * per[kind] * es;
+  return GPT_OK;
 }
 
 int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay) {

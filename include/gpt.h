@@ -148,6 +148,27 @@ int muon_step(gpt_ctx* ctx, float lr, float momentum, float weight_decay);
  * norm undefined; the reading above is the one this library implements. */
 int muon_step_normuon(gpt_ctx* ctx, float lr, float momentum, float weight_decay, float beta2);
 
+/* Muon (normuon_beta2 < 0) or NorMuon (0 <= normuon_beta2 < 1, as
+ * muon_step_normuon) of the block matrices of layers l0 .. l1-1 only, for
+ * data-parallel ranks that split the optimizer work by layer: every matrix
+ * is updated on its own, so the ranges of all ranks together give exactly
+ * what one whole-model call gives.  The bf16 working copies of the updated
+ * layers then have to reach the other ranks (gpt_block_region gives their
+ * bytes).  0 <= l0 <= l1 <= depth, else GPT_EINVAL; l0 == l1 does nothing. */
+int muon_step_layers(gpt_ctx* ctx, float lr, float momentum, float weight_decay, float normuon_beta2, int l0,
+                     int l1);
+
+/* Byte range of block matrix kind (0 fused q|k|v, 1 attention output, 2 MLP
+ * up, 3 MLP down) for layers l0 .. l1-1: inside param_buf for
+ * GPT_REGION_MASTER (fp32 masters) and GPT_REGION_BF16 (bf16 working
+ * copies), inside state_buf for GPT_REGION_GRAD (fp32 gradients).  The
+ * layers of one kind are contiguous, so the range is one span; the block
+ * gradients follow those of the embedding and lm_head inside the
+ * gpt_grad_region span. */
+enum { GPT_REGION_MASTER = 0, GPT_REGION_BF16 = 1, GPT_REGION_GRAD = 2 };
+int gpt_block_region(const gpt_ctx* ctx, int what, int kind, int l0, int l1, size_t* offset_bytes,
+                     size_t* size_bytes);
+
 /* AdamW update of the token embedding and lm_head with bias correction
  * (the step count is kept in the context) and decoupled weight decay. */
 int adamw_step(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay);

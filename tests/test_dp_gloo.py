@@ -84,3 +84,139 @@ def test_single_process_helpers_are_identity():
     t = torch.arange(5, dtype=torch.float32)
     assert torch.equal(dp.average_gradients(t.clone()), t)
     assert dp.max_over_ranks(3.5) == 3.5
+
+
+# --- sharded optimizer (three-phase, layer ranges per rank) ---------------------
+
+D_FAKE, L_FAKE, V_FAKE = 8, 4, 16
+
+
+def _fake_shapes():
+    d = D_FAKE
+    return [(d, 3 * d), (d, d), (d, 4 * d), (4 * d, d)]
+
+
+class _FakeStep:
+    """Host stand-in for GPTStep with the same optimizer-side interface; the
+    update of each matrix is the fp64 oracle's."""
+
+    def __init__(self, seed):
+        from oracle import optim as oo
+        self.oo = oo
+        rng = np.random.default_rng(seed)
+        d = D_FAKE
+        self.shapes = _fake_shapes()
+        self.master = [torch.tensor(rng.standard_normal((L_FAKE, r, c)) * 0.02, dtype=torch.float32)
+                       for r, c in self.shapes]
+        self.bf16 = [m.to(torch.bfloat16) for m in self.master]
+        self.mom = [torch.zeros_like(m) for m in self.master]
+        self.emb = torch.tensor(rng.standard_normal((V_FAKE + d, d)) * 0.02, dtype=torch.float32)
+        self.m = torch.zeros_like(self.emb)
+        self.v = torch.zeros_like(self.emb)
+        self.t = 0
+        n_emb = self.emb.numel()
+        self.grad = torch.zeros(n_emb + sum(L_FAKE * r * c for r, c in self.shapes), dtype=torch.float32)
+        self.offs = []
+        o = n_emb
+        for r, c in self.shapes:
+            self.offs.append(o)
+            o += L_FAKE * r * c
+        self.n_emb = n_emb
+
+    def set_grads(self, seed):
+        self.grad.copy_(torch.tensor(np.random.default_rng(seed).standard_normal(self.grad.numel()),
+                                     dtype=torch.float32))
+
+    def block_region(self, what, kind, l0, l1):
+        r, c = self.shapes[kind]
+        if what == 2:
+            return self.grad[self.offs[kind] + l0 * r * c:self.offs[kind] + l1 * r * c]
+        t = self.master[kind] if what == 0 else self.bf16[kind]
+        return t.view(-1)[l0 * r * c:l1 * r * c]
+
+    def adamw_grad_view(self):
+        return self.grad[:self.n_emb]
+
+    def muon_step_layers(self, l0, l1, lr, momentum, wd, normuon_beta2):
+        for kind, (r, c) in enumerate(self.shapes):
+            g = self.block_region(2, kind, 0, L_FAKE).view(L_FAKE, r, c)
+            for l in range(l0, l1):
+                W, M = self.oo.muon_step(self.master[kind][l].double().numpy(), g[l].double().numpy(),
+                                         self.mom[kind][l].double().numpy(), lr, momentum, wd)
+                self.master[kind][l] = torch.tensor(W, dtype=torch.float32)
+                self.mom[kind][l] = torch.tensor(M, dtype=torch.float32)
+                self.bf16[kind][l] = self.master[kind][l].to(torch.bfloat16)
+
+    def adamw_step(self, lr, beta1, beta2, eps, wd):
+        self.t += 1
+        p, m, v = self.oo.adamw_step(self.emb.double().numpy(), self.adamw_grad_view().view_as(self.emb).double().numpy(),
+                                     self.m.double().numpy(), self.v.double().numpy(), self.t, lr, beta1, beta2, eps, wd)
+        self.emb = torch.tensor(p, dtype=torch.float32)
+        self.m = torch.tensor(m, dtype=torch.float32)
+        self.v = torch.tensor(v, dtype=torch.float32)
+
+
+def _shard_worker(rank, world, port, outdir):
+    import sys
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    from gpt_pretraining_step_b200 import dp
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    st = _FakeStep(seed=5)                      # identical parameters on every rank
+    for step in range(2):
+        st.set_grads(seed=100 * step + rank)    # each rank: its own batch's gradients
+        dp.sharded_optimizer_step(st, L_FAKE, muon=(0.02, 0.95, 0.01), adam=(3e-3, 0.8, 0.95, 1e-10, 0.0),
+                                  sync_masters=(step == 1))
+    out = {f"bf16_{k}": st.bf16[k].float().numpy() for k in range(4)}
+    out.update({f"master_{k}": st.master[k].numpy() for k in range(4)})
+    out["emb"] = st.emb.numpy()
+    np.savez(os.path.join(outdir, f"shard{rank}.npz"), **out)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(300)
+def test_sharded_optimizer_equals_replicated(tmp_path):
+    """Three ranks over four layers (uneven shards): after two sharded steps
+    every rank holds the parameters one replicated step sequence on the mean
+    gradients gives (bf16 copies identical on every rank)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    world = 3
+    mp.start_processes(_shard_worker, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    ref = _FakeStep(seed=5)
+    for step in range(2):
+        gs = []
+        for r in range(world):
+            ref.set_grads(seed=100 * step + r)
+            gs.append(ref.grad.clone())
+        ref.grad.copy_(sum(gs) / world)
+        ref.muon_step_layers(0, L_FAKE, 0.02, 0.95, 0.01, -1.0)
+        ref.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.0)
+    res = [np.load(tmp_path / f"shard{r}.npz") for r in range(world)]
+    for k in range(4):
+        for r in range(world):
+            assert np.array_equal(res[r][f"bf16_{k}"], res[0][f"bf16_{k}"]), (k, r)
+            # masters were broadcast by their owners on the last step
+            assert np.allclose(res[r][f"master_{k}"], ref.master[k].numpy(), rtol=1e-5, atol=1e-7), (k, r)
+        assert np.allclose(res[0][f"bf16_{k}"], ref.bf16[k].float().numpy(), rtol=1e-2, atol=1e-6), k
+    for r in range(world):
+        assert np.allclose(res[r]["emb"], ref.emb.numpy(), rtol=1e-6, atol=1e-9)
+
+
+def test_layer_shards_cover_and_balance():
+    import sys
+    sys.path.insert(0, ROOT)
+    from gpt_pretraining_step_b200 import dp
+    for n_layer in (1, 4, 20, 26):
+        for world in (1, 2, 3, 8):
+            sh = dp.layer_shards(n_layer, world)
+            assert len(sh) == world and sh[0][0] == 0 and sh[-1][1] == n_layer
+            assert all(a <= b for a, b in sh) and all(sh[i][1] == sh[i + 1][0] for i in range(world - 1))
+            sizes = [b - a for a, b in sh]
+            assert max(sizes) - min(sizes) <= 1 and sizes == sorted(sizes, reverse=True)

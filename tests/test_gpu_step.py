@@ -295,6 +295,47 @@ def test_normuon_rejects_bad_beta2(torch):
             st.muon_step_normuon(0.02, 0.95, 0.0, b)
 
 
+@pytest.mark.parametrize("normuon_beta2", [-1.0, 0.9])
+def test_muon_by_layer_ranges_equals_whole_model(torch, normuon_beta2):
+    """The ranges of a sharded optimizer step (layers 0-1, 2, 3) give bit for
+    bit the whole-model Muon / NorMuon update, and the block regions address
+    the tensors gpt_get_tensor returns."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=4, d_model=256, vocab=1000, batch=2, seq_len=64)
+    params = syn.init_params(s, seed=31)
+    specs = syn.param_specs(s)
+    a, b = build(torch, s, params), build(torch, s, params)
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if grp == "muon":
+            G = syn.gaussian((r, c), seed=500 + tid)
+            a.set(tid, G, kind=g.KIND_GRAD)
+            b.set(tid, G, kind=g.KIND_GRAD)
+    for _ in range(2):
+        if normuon_beta2 < 0:
+            a.muon_step(0.02, 0.95, 0.01)
+        else:
+            a.muon_step_normuon(0.02, 0.95, 0.01, normuon_beta2)
+        for l0, l1 in ((0, 2), (2, 3), (3, 3), (3, 4)):
+            b.muon_step_layers(l0, l1, 0.02, 0.95, 0.01, normuon_beta2)
+    a.check()
+    b.check()
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if grp != "muon":
+            continue
+        for kind in (g.KIND_PARAM, g.KIND_MOM) + ((g.KIND_NORMUON_V,) if normuon_beta2 >= 0 else ()):
+            assert torch.equal(a.get(tid, kind), b.get(tid, kind)), (pname, kind)
+    for kind in range(4):
+        assert torch.equal(a.block_region(g.REGION_BF16, kind, 0, 4), b.block_region(g.REGION_BF16, kind, 0, 4))
+        l, (pname, r, c, _) = 2, specs[2 + 4 * 2 + kind]
+        master = b.block_region(g.REGION_MASTER, kind, l, l + 1).view(r, c)
+        assert torch.equal(master, b.get(2 + 4 * l + kind, g.KIND_PARAM))
+        assert torch.equal(b.block_region(g.REGION_BF16, kind, l, l + 1).view(r, c), master.to(torch.bfloat16))
+        assert torch.equal(b.block_region(g.REGION_GRAD, kind, l, l + 1).view(r, c),
+                           b.get(2 + 4 * l + kind, g.KIND_GRAD))
+    with pytest.raises(g.GptError):
+        b.muon_step_layers(3, 5)
+
+
 def test_adamw_step_matches_oracle(torch):
     import gpt_pretraining_step_b200 as g
     s = SMALL["ragged"]
