@@ -19,6 +19,14 @@ Readings where the pages are silent (shared with the CUDA path):
   * QK norm: per-head gain-free RMSNorm applied after RoPE (the order does
     not matter mathematically: a rotation keeps the RMS).
   * attention scale 1/sqrt(hd); n_kv_head = n_head.
+  * residual extras ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section
+    "1. Modelo GPT", efficiency tricks 1 and 3), present when params holds a
+    "scalars" vector [2L + 1] = (resid lambdas, x0 lambdas, backout lambda):
+    before block i, x <- resid[i] x + x0l[i] x0 with x0 the embedding output;
+    after the last block, x <- x - backout * x_mid with x_mid the residual
+    stream entering block L // 2 (before its scaling).  Initial values 1, 0
+    and 0 make the network the plain one.  Smear and value embeddings are
+    not part of this oracle.
   * attention window per layer: full causal by default; with a layer pattern
     such as "SSSL" (section "1. Modelo GPT", sliding-window attention) the
     pattern is repeated over the layers, S = a sliding window of
@@ -181,8 +189,20 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
     H = d // head_dim
     cos, sin = rope_angles(T, head_dim)
     x = wte[tok.reshape(-1)]                         # [M, d] exact row copy
+    sc = params.get("scalars")
+    if sc is not None:
+        sc = np.asarray(sc, dtype=np.float64).reshape(-1)
+        if sc.size != 2 * n_layer + 1:
+            raise ValueError("scalars must hold 2 * n_layer + 1 values")
+    x0 = x
+    x_in, x_mid = [], None
     acts = []
     for l in range(n_layer):
+        if sc is not None:
+            x_in.append(x)
+            if l == n_layer // 2:
+                x_mid = x
+            x = sc[l] * x + sc[n_layer + l] * x0
         W = {n: np.asarray(params[f"h{l}.{n}"], dtype=np.float64)
              for n in ("c_qkv", "c_proj", "c_fc", "mlp_proj")}
         a = {}
@@ -204,6 +224,8 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
             a.update(xn1=xn1, r1=r1, qn=qn, rq=rq, kn=kn, rk=rk, v=v, P=P, ym=ym,
                      xn2=xn2, r2=r2, u=u, h=h)
         acts.append(a)
+    if sc is not None:
+        x = x - sc[2 * n_layer] * x_mid
     xf, rf = rms_norm(x)
     z = xf @ np.asarray(params["lm_head"], dtype=np.float64)
     lse = logsumexp(z)
@@ -211,7 +233,7 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
     row_loss = lse - z[np.arange(z.shape[0]), t]
     loss = float(np.mean(row_loss))
     cache = dict(acts=acts, xf=xf, rf=rf, z=z, lse=lse, row_loss=row_loss,
-                 B=B, T=T, H=H, d=d, cos=cos, sin=sin) if keep else None
+                 B=B, T=T, H=H, d=d, cos=cos, sin=sin, scalars=sc, x0=x0, x_in=x_in, x_mid=x_mid) if keep else None
     return loss, cache
 
 
@@ -229,6 +251,12 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
     Wlm = np.asarray(params["lm_head"], dtype=np.float64)
     grads["lm_head"] = cache["xf"].T @ dz
     dx = rms_norm_bwd(dz @ Wlm.T, cache["xf"], cache["rf"])
+    sc = cache["scalars"]
+    if sc is not None:
+        dsc = np.zeros(2 * n_layer + 1)
+        dx_final = dx                                # gradient at the backout output
+        dsc[2 * n_layer] = -np.sum(cache["x_mid"] * dx_final)
+        dx0 = np.zeros_like(dx)
     for l in reversed(range(n_layer)):
         a = cache["acts"][l]
         W = {n: np.asarray(params[f"h{l}.{n}"], dtype=np.float64)
@@ -248,6 +276,17 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
         dqkv = np.concatenate([_merge_heads(dq), _merge_heads(dk), _merge_heads(dv)], axis=1)
         grads[f"h{l}.c_qkv"] = a["xn1"].T @ dqkv
         dx = dx + rms_norm_bwd(dqkv @ W["c_qkv"].T, a["xn1"], a["r1"])
+        if sc is not None:
+            # x' = resid[l] x_in + x0l[l] x0 (and x_in of block L // 2 feeds the backout)
+            dsc[l] = np.sum(cache["x_in"][l] * dx)
+            dsc[n_layer + l] = np.sum(cache["x0"] * dx)
+            dx0 = dx0 + sc[n_layer + l] * dx
+            dx = sc[l] * dx
+            if l == n_layer // 2:
+                dx = dx - sc[2 * n_layer] * dx_final
+    if sc is not None:
+        dx = dx + dx0
+        grads["scalars"] = dsc.reshape(1, -1)
     V = params["wte"].shape[0]
     dwte = np.zeros((V, d))
     np.add.at(dwte, tok.reshape(-1), dx)

@@ -64,7 +64,7 @@ def config_shape(name: str) -> Shape:
     return make_shape(**CONFIGS[name])
 
 
-def param_specs(s: Shape):
+def param_specs(s: Shape, extras: bool = False):
     """(name, rows, cols, group) for every parameter; matrices are [in, out].
 
     Order: token embedding, lm_head, then per layer the fused q|k|v projection,
@@ -78,6 +78,9 @@ def param_specs(s: Shape):
                 (f"h{layer}.c_proj", d, d, "muon"),
                 (f"h{layer}.c_fc", d, f, "muon"),
                 (f"h{layer}.mlp_proj", f, d, "muon")]
+    if extras:
+        # per-layer residual and x0 scales, then the backout scale
+        out.append(("scalars", 1, 2 * s.depth + 1, "adamw"))
     return out
 
 
@@ -95,14 +98,28 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
     return (a.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def init_params(s: Shape, seed: int = 0, std: float = 0.02):
-    """N(0, std) weights rounded to bf16, as float32 arrays keyed by name."""
+def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False):
+    """N(0, std) weights rounded to bf16, as float32 arrays keyed by name;
+    with extras also the scalar vector at its neutral values (residual
+    scales 1, x0 and backout scales 0)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     params = {}
     for name, r, c, _ in param_specs(s):
         w = rng.standard_normal((r, c), dtype=np.float32) * np.float32(std)
         params[name] = round_to_bf16(w)
+    if extras:
+        sc = np.zeros((1, 2 * s.depth + 1), dtype=np.float32)
+        sc[0, :s.depth] = 1.0
+        params["scalars"] = sc
     return params
+
+
+def random_scalars(s: Shape, seed: int) -> np.ndarray:
+    """Residual scales in [0.5, 1.5], x0 and backout scales in [-0.5, 0.5]."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    sc = rng.uniform(-0.5, 0.5, size=(1, 2 * s.depth + 1)).astype(np.float32)
+    sc[0, :s.depth] += 1.0
+    return sc
 
 
 def tokens(s: Shape, seed: int = 1) -> np.ndarray:

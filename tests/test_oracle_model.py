@@ -332,3 +332,63 @@ def test_finite_difference_with_sliding_windows():
     l0, _ = om.forward(p, tok, tgt, s.depth, keep=False)
     l1, _ = om.forward(p, tok, tgt, s.depth, keep=False, windows=windows)
     assert l0 != l1
+
+
+# --- residual extras: per-layer residual / x0 scales and backout ---------------
+#
+# Section "1. Modelo GPT", efficiency tricks 1 and 3: x <- resid[i] x + x0l[i]
+# x0 before block i, and x <- x - backout * x_mid after the last block, x_mid
+# being the residual stream entering block L // 2.
+
+def _extras_case(depth=2, seed=0, **kw):
+    s, p, tok, tgt = small_case(depth=depth, seed=seed, **kw)
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    return s, p, tok, tgt
+
+
+def test_neutral_scalars_give_the_plain_model():
+    s, p, tok, tgt = _extras_case(std=0.05)
+    sc = np.zeros((1, 2 * s.depth + 1))
+    sc[0, :s.depth] = 1.0
+    l0, g0, _ = om.fwd_bwd(p, tok, tgt, s.depth)
+    l1, g1, _ = om.fwd_bwd(dict(p, scalars=sc), tok, tgt, s.depth)
+    assert l0 == l1
+    for k in g0:
+        assert np.array_equal(g0[k], g1[k]), k
+    assert g1["scalars"].shape == (1, 2 * s.depth + 1)
+
+
+def test_x0_only_inputs_reduce_to_the_last_block():
+    # resid = 0, x0 scale = 1: every block reads the embedding, so only the
+    # last block's contribution survives: a one-block model with its weights
+    depth = 3
+    s, p, tok, tgt = _extras_case(depth=depth, std=0.05, seed=4)
+    sc = np.zeros((1, 2 * depth + 1))
+    sc[0, depth:2 * depth] = 1.0
+    loss, _ = om.forward(dict(p, scalars=sc), tok, tgt, depth, keep=False)
+    one = {"wte": p["wte"], "lm_head": p["lm_head"]}
+    for n in ("c_qkv", "c_proj", "c_fc", "mlp_proj"):
+        one[f"h0.{n}"] = p[f"h{depth - 1}.{n}"]
+    ref, _ = om.forward(one, tok, tgt, 1, keep=False)
+    assert abs(loss - ref) < 1e-12
+
+
+def test_backout_of_the_whole_stream_before_the_middle():
+    # depth 2 with backout 1: the final stream is x_mid + f1(x_mid) - x_mid,
+    # i.e. the last block's contribution alone on top of nothing
+    s, p, tok, tgt = _extras_case(depth=2, std=0.05, seed=6)
+    sc = np.array([[1.0, 1.0, 0.0, 0.0, 1.0]])
+    _, c = om.forward(dict(p, scalars=sc), tok, tgt, 2)
+    _, cp = om.forward(p, tok, tgt, 2)
+    # the stream entering block 1 is the final stream of block 0 alone
+    _, c1 = om.forward({k: v for k, v in p.items() if not k.startswith("h1.")}, tok, tgt, 1)
+    x_mid = c1["xf"] / c1["rf"]
+    xf_ref, _ = om.rms_norm(cp["xf"] / cp["rf"] - x_mid)
+    assert np.allclose(c["xf"], xf_ref, rtol=1e-9, atol=1e-12)
+
+
+def test_finite_difference_with_residual_extras():
+    s, p, tok, tgt = _extras_case(depth=2, std=0.05, seed=8, vocab=48, seq=12)
+    p["scalars"] = syn.random_scalars(s, seed=9).astype(np.float64)
+    names = [n for n, *_ in syn.param_specs(s, extras=True)]
+    _fd_check(p, tok, tgt, s.depth, names, n_coords=4)
