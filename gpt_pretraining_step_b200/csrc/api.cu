@@ -41,6 +41,8 @@ struct Dims {
   int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32, fp8;
   int short_window, n_pat;
   char pat[12];
+  int extras;   // residual / x0 scales and backout (2L+1 scalars)
+  int nsc;      // scalar count rounded up to a multiple of 4
   // attention window of layer l: short_window for an 'S' layer, -1 = full causal
   int window(int l) const { return n_pat > 0 && pat[l % n_pat] == 'S' ? short_window : -1; }
 };
@@ -53,12 +55,14 @@ struct Plan {
   // state
   size_t g[6], mom[6], am[2], av[2];
   size_t nv;            // NorMuon second moments: 4 groups x L matrices x d floats
+  size_t ws, wsb, gs, ams, avs;   // residual-extras scalars: master, bf16 scratch, grad, AdamW m, v
   size_t state_bytes;
   // activations
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
   size_t xf, rf, z, stats, zt, row_loss, loss;
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
+  size_t x0, xin, dx0, dxfin, scws;   // residual extras (allocated only when on)
   size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
@@ -129,6 +133,9 @@ int dims_from(const gpt_config* c, Dims& D) {
   if (any_s && (c->short_window < 0 || c->short_window >= (1 << 30)))
     return fail(GPT_EINVAL, "short_window must be in [0, 2^30) when the pattern has an 'S' layer");
   D.short_window = c->short_window;
+  if (c->residual_extras != 0 && c->residual_extras != 1) return fail(GPT_EINVAL, "residual_extras must be 0 or 1");
+  D.extras = c->residual_extras;
+  D.nsc = (2 * D.L + 1 + 3) / 4 * 4;
   return GPT_OK;
 }
 
@@ -138,9 +145,16 @@ void make_plan(const Dims& D, Plan& P) {
   Bump pb;
   for (int i = 0; i < 6; ++i) P.w[i] = pb.take(numel[i] * 4);
   for (int i = 0; i < 6; ++i) P.wb[i] = pb.take(numel[i] * 2);
+  const size_t nsc = D.extras ? static_cast<size_t>(D.nsc) : 0;
+  P.ws = pb.take(std::max<size_t>(nsc, 4) * 4);
+  P.wsb = pb.take(std::max<size_t>(nsc, 4) * 2);
   P.param_bytes = pb.off;
   Bump sb;
-  for (int i = 0; i < 6; ++i) P.g[i] = sb.take(numel[i] * 4);
+  // gradients: embedding, lm_head, the scalars, then the block matrices (one
+  // span; everything before the first block gradient goes to AdamW)
+  for (int i = 0; i < 2; ++i) P.g[i] = sb.take(numel[i] * 4);
+  P.gs = sb.take(std::max<size_t>(nsc, 4) * 4);
+  for (int i = 2; i < 6; ++i) P.g[i] = sb.take(numel[i] * 4);
   P.mom[0] = P.mom[1] = 0;
   for (int i = 2; i < 6; ++i) P.mom[i] = sb.take(numel[i] * 4);
   for (int i = 0; i < 2; ++i) {
@@ -148,6 +162,8 @@ void make_plan(const Dims& D, Plan& P) {
     P.av[i] = sb.take(numel[i] * 4);
   }
   P.nv = sb.take(4 * L * d * 4);
+  P.ams = sb.take(std::max<size_t>(nsc, 4) * 4);
+  P.avs = sb.take(std::max<size_t>(nsc, 4) * 4);
   P.state_bytes = sb.off;
 
   // split-K plan of the lm_head input gradient (contraction over the vocabulary)
@@ -211,6 +227,15 @@ void make_plan(const Dims& D, Plan& P) {
   P.normws = ab.take(muon_norm_workspace(4 * D.L));
   P.nfac = ab.take(2 * L * d * 4);
   P.sched = ab.take(64);   // work counters of the persistent attention kernels
+  if (D.extras) {
+    P.x0 = ab.take(M * d * 4);
+    P.xin = ab.take(L * M * d * 4);
+    P.dx0 = ab.take(M * d * 4);
+    P.dxfin = ab.take(M * d * 4);
+    P.scws = ab.take(static_cast<size_t>(2 * L + 1) * resid_partial_blocks() * 4);
+  } else {
+    P.x0 = P.xin = P.dx0 = P.dxfin = P.scws = 0;
+  }
   P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
   P.tok = ab.take(M * 4);
@@ -304,6 +329,8 @@ struct gpt_ctx {
   bf16* Wb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wb[i]); }
   float* G(int i) const { return reinterpret_cast<float*>(sbuf + P.g[i]); }
   float* Mom(int i) const { return reinterpret_cast<float*>(sbuf + P.mom[i]); }
+  // residual-extras scalars (fp32, in the parameter buffer)
+  float* Scal() const { return reinterpret_cast<float*>(pbuf + P.ws); }
   // NorMuon second moments of block group i (2..5): L vectors of d floats
   float* NV(int i) const { return reinterpret_cast<float*>(sbuf + P.nv) + static_cast<size_t>(i - 2) * D.L * D.d; }
   template <typename T>
@@ -338,6 +365,10 @@ bool locate(const gpt_ctx* c, int id, int& grp, size_t& off, int& rows, int& col
   if (id == 0) { grp = 0; off = 0; rows = D.V; cols = D.d; return true; }
   if (id == 1) { grp = 1; off = 0; rows = D.d; cols = D.V; return true; }
   const int k = id - 2;
+  if (D.extras && k == 4 * D.L) {   // the residual-extras scalars
+    grp = 6; off = 0; rows = 1; cols = 2 * D.L + 1;
+    return true;
+  }
   if (k < 0 || k >= 4 * D.L) return false;
   const int l = k / 4, j = k % 4;
   const int shp[4][2] = {{D.d, 3 * D.d}, {D.d, D.d}, {D.d, D.F}, {D.F, D.d}};
@@ -459,6 +490,12 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     bf16* ol = o + l * Md;
     bf16* hl = h + static_cast<size_t>(l) * M * F;
     float* lsel = lse + static_cast<size_t>(l) * M * H;
+    if (D.extras) {
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_resid_fwd(x, c->A<float>(P.xin) + l * Md, c->A<float>(P.x0), c->Scal(), l, L,
+                       static_cast<long long>(Md), l == 0, s);
+      c->launches += 1;
+    }
     {
       ProfScope ps(c, GPT_PROF_NORM);
       launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
@@ -511,6 +548,12 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       GPT_CK(gemm_run(g, s));
     }
     c->launches += 7;
+  }
+  if (D.extras) {
+    ProfScope ps(c, GPT_PROF_NORM);
+    launch_backout_fwd(x, c->A<float>(P.xin) + static_cast<size_t>(L / 2) * Md, c->Scal(), L,
+                       static_cast<long long>(Md), s);
+    c->launches += 1;
   }
   {
     ProfScope ps(c, GPT_PROF_NORM);
@@ -576,6 +619,14 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     launch_rmsnorm_bwd(dxn, xf, rf, dx, gmlp(L - 1), M, d, false, s);
   }
   c->launches += 1;
+  if (D.extras) {
+    // the backout output's gradient, kept for the block whose input it read
+    ProfScope ps(c, GPT_PROF_NORM);
+    GPT_CK(cudaMemcpyAsync(c->A<float>(P.dxfin), dx, Md * 4, cudaMemcpyDeviceToDevice, s));
+    launch_backout_grad_partial(c->A<float>(P.xin) + static_cast<size_t>(L / 2) * Md, dx, L,
+                                static_cast<long long>(Md), c->A<float>(P.scws), s);
+    c->launches += 1;
+  }
   for (int l = L - 1; l >= 0; --l) {
     bf16* xn2l = xn2 + l * Md;
     bf16* hl = h + static_cast<size_t>(l) * M * F;
@@ -641,6 +692,16 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
                          l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), M, d, true, s);
     }
     c->launches += 1;
+    if (D.extras) {
+      // through x' = resid[l] x_in + x0s[l] x0: dx becomes the gradient at
+      // block l's unscaled input, and its bf16 copy replaces the one above
+      ProfScope ps(c, GPT_PROF_NORM);
+      launch_resid_bwd(dx, c->A<float>(P.xin) + l * Md, c->A<float>(P.x0), c->A<float>(P.dx0),
+                       l == L / 2 ? c->A<float>(P.dxfin) : nullptr, c->Scal(), l, L,
+                       static_cast<long long>(Md), l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), c->A<float>(P.scws),
+                       l == L - 1, l == 0, s);
+      c->launches += 1;
+    }
   }
   // weight gradients of every block matrix, each kind as one GEMM batched over the layers:
   // dW[l] = act[l]^T grad[l], contraction over the M tokens
@@ -663,6 +724,11 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       GPT_CK(gemm_run(g, s));
     }
     c->launches += 4;
+  }
+  if (D.extras) {
+    ProfScope ps(c, GPT_PROF_NORM);
+    launch_scalar_grad_finish(c->A<float>(P.scws), L, reinterpret_cast<float*>(c->sbuf + P.gs), acc, s);
+    c->launches += 1;
   }
   {
     ProfScope ps(c, GPT_PROF_EMBED);
@@ -848,6 +914,14 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
     init_normal_kernel<<<1024, 256, 0, s>>>(c->W(i), c->Wb(i), static_cast<long long>(numel[i]), cfg->seed, i, 0.02f);
   }
   launch_rope_table(c->A<float2>(c->P.rope), D.T, s);
+  std::vector<float> sc0;
+  if (D.extras) {
+    // residual scales 1, x0 and backout scales 0 (and zero padding): the plain network
+    sc0.assign(D.nsc, 0.f);
+    for (int l = 0; l < D.L; ++l) sc0[l] = 1.f;
+    if ((e = cudaMemcpyAsync(c->pbuf + c->P.ws, sc0.data(), sc0.size() * 4, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+      return bad(e, "init scalars");
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return bad(e, "init kernels");
   if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return bad(e, "init sync");
   c->launches = 7;
@@ -1003,6 +1077,14 @@ int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float 
                  bc1, bc2, c->stream);
   }
   c->launches += 2;
+  if (c->D.extras) {
+    // the scalars (zero padding stays zero: zero gradient, zero value)
+    launch_adamw(reinterpret_cast<float*>(c->pbuf + c->P.ws), reinterpret_cast<float*>(c->sbuf + c->P.gs),
+                 reinterpret_cast<float*>(c->sbuf + c->P.ams), reinterpret_cast<float*>(c->sbuf + c->P.avs),
+                 reinterpret_cast<bf16*>(c->pbuf + c->P.wsb), c->D.nsc, lr, beta1, beta2, eps, weight_decay, bc1, bc2,
+                 c->stream);
+    c->launches += 1;
+  }
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -1029,7 +1111,7 @@ int gpt_train_step_host(gpt_ctx* c, const int32_t* tokens_host, const int32_t* t
   return gpt_check(c);
 }
 
-int gpt_num_tensors(const gpt_ctx* c) { return c ? 2 + 4 * c->D.L : 0; }
+int gpt_num_tensors(const gpt_ctx* c) { return c ? 2 + 4 * c->D.L + c->D.extras : 0; }
 
 int gpt_tensor_info(const gpt_ctx* c, int id, int32_t* rows, int32_t* cols, int32_t* group) {
   int rc = check_ctx(c);
@@ -1039,7 +1121,7 @@ int gpt_tensor_info(const gpt_ctx* c, int id, int32_t* rows, int32_t* cols, int3
   if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
   if (rows) *rows = r;
   if (cols) *cols = cc;
-  if (group) *group = grp < 2 ? GPT_GROUP_ADAMW : GPT_GROUP_MUON;
+  if (group) *group = (grp < 2 || grp == 6) ? GPT_GROUP_ADAMW : GPT_GROUP_MUON;
   return GPT_OK;
 }
 
@@ -1048,6 +1130,20 @@ static int tensor_ptr(gpt_ctx* c, int id, int kind, float** p, size_t* n, int* g
   size_t off;
   if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
   float* base = nullptr;
+  if (grp == 6) {
+    size_t o;
+    switch (kind) {
+      case GPT_KIND_PARAM: *p = reinterpret_cast<float*>(c->pbuf + c->P.ws); break;
+      case GPT_KIND_GRAD: o = c->P.gs; *p = reinterpret_cast<float*>(c->sbuf + o); break;
+      case GPT_KIND_ADAM_M: o = c->P.ams; *p = reinterpret_cast<float*>(c->sbuf + o); break;
+      case GPT_KIND_ADAM_V: o = c->P.avs; *p = reinterpret_cast<float*>(c->sbuf + o); break;
+      default: return fail(GPT_EINVAL, "the scalars have a value, a gradient and AdamW moments only");
+    }
+    *n = static_cast<size_t>(r) * cc;
+    *grp_out = grp;
+    *off_out = 0;
+    return GPT_OK;
+  }
   switch (kind) {
     case GPT_KIND_PARAM: base = c->W(grp); break;
     case GPT_KIND_GRAD: base = c->G(grp); break;
@@ -1103,7 +1199,7 @@ int gpt_set_tensor(gpt_ctx* c, int id, int kind, const float* src) {
   rc = tensor_ptr(c, id, kind, &p, &n, &grp, &off);
   if (rc) return rc;
   GPT_CK(cudaMemcpyAsync(p, src, n * 4, cudaMemcpyDeviceToDevice, c->stream));
-  if (kind == GPT_KIND_PARAM) {
+  if (kind == GPT_KIND_PARAM && grp != 6) {   // the scalars are read in fp32 and have no bf16 copy
     launch_cast_bf16(p, c->Wb(grp) + off, static_cast<long long>(n), c->stream);
     c->launches += 1;
   }

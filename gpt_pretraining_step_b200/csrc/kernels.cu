@@ -187,6 +187,138 @@ __global__ void __launch_bounds__(128) rmsnorm_bwd_kernel(const float* __restric
   }
 }
 
+// ------------------------------------------- residual scales and backout
+//
+// Per-layer residual scaling and backout ("¿Cómo Entrenar Tu Propio ChatGPT
+// por $50?", section "1. Modelo GPT", efficiency tricks 1 and 3).  lam holds
+// (resid[0..L), x0[0..L), backout).
+
+// Before block l: x_in[l] = x; x = resid[l] x + x0[l] x0 (block 0 also
+// stores x0 = x, the embedding output).
+__global__ void resid_fwd_kernel(float* __restrict__ x, float* __restrict__ x_in, float* __restrict__ x0,
+                                 const float* __restrict__ lam, int l, int L, long long n4, int first) {
+  const float a = lam[l], b = lam[L + l];
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(x)[i];
+    reinterpret_cast<float4*>(x_in)[i] = v;
+    float4 z;
+    if (first) {
+      z = v;
+      reinterpret_cast<float4*>(x0)[i] = v;
+    } else {
+      z = reinterpret_cast<const float4*>(x0)[i];
+    }
+    reinterpret_cast<float4*>(x)[i] =
+        make_float4(a * v.x + b * z.x, a * v.y + b * z.y, a * v.z + b * z.z, a * v.w + b * z.w);
+  }
+}
+
+// After the last block: x -= backout * x_mid.
+__global__ void backout_fwd_kernel(float* __restrict__ x, const float* __restrict__ x_mid,
+                                   const float* __restrict__ lam, int L, long long n4) {
+  const float c = lam[2 * L];
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 v = reinterpret_cast<float4*>(x)[i];
+    const float4 m = reinterpret_cast<const float4*>(x_mid)[i];
+    v.x -= c * m.x; v.y -= c * m.y; v.z -= c * m.z; v.w -= c * m.w;
+    reinterpret_cast<float4*>(x)[i] = v;
+  }
+}
+
+// Block sum of two per-thread values into part_a[blockIdx.x], part_b[blockIdx.x]
+// (a fixed grid and a fixed reduction tree, so the result does not depend on
+// scheduling).
+__device__ __forceinline__ void block_sum2(float sa, float sb, float* part_a, float* part_b) {
+  __shared__ float ra[32], rb[32];
+  sa = warp_sum(sa);
+  sb = warp_sum(sb);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    ra[w] = sa;
+    rb[w] = sb;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const int nw = blockDim.x >> 5;
+    float a = lane < nw ? ra[lane] : 0.f, b = lane < nw ? rb[lane] : 0.f;
+    a = warp_sum(a);
+    b = warp_sum(b);
+    if (lane == 0) {
+      if (part_a) part_a[blockIdx.x] = a;
+      if (part_b) part_b[blockIdx.x] = b;
+    }
+  }
+}
+
+// Backward through x' = resid[l] x_in + x0[l] x0 given g = dL/dx' in dx:
+// partial sums of x_in . g and x0 . g, dx0 (+)= x0[l] g, dx = resid[l] g
+// (minus backout * dx_final for the block whose input the backout read), and
+// the bf16 copy of dx for the block below; for block 0 dx also takes dx0 (the
+// embedding output fed every block through x0).
+__global__ void __launch_bounds__(256) resid_bwd_kernel(float* __restrict__ dx, const float* __restrict__ x_in,
+                                                        const float* __restrict__ x0, float* __restrict__ dx0,
+                                                        const float* __restrict__ dx_final,
+                                                        const float* __restrict__ lam, int l, int L, long long n4,
+                                                        bf16* __restrict__ gout, float* __restrict__ part_r,
+                                                        float* __restrict__ part_0, int first, int last) {
+  const float a = lam[l], b = lam[L + l], c = dx_final ? lam[2 * L] : 0.f;
+  float sr = 0.f, s0 = 0.f;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 g = reinterpret_cast<const float4*>(dx)[i];
+    const float4 xi = reinterpret_cast<const float4*>(x_in)[i];
+    const float4 z = reinterpret_cast<const float4*>(x0)[i];
+    sr += xi.x * g.x + xi.y * g.y + xi.z * g.z + xi.w * g.w;
+    s0 += z.x * g.x + z.y * g.y + z.z * g.z + z.w * g.w;
+    float4 d0 = first ? make_float4(0.f, 0.f, 0.f, 0.f) : reinterpret_cast<const float4*>(dx0)[i];
+    d0.x += b * g.x; d0.y += b * g.y; d0.z += b * g.z; d0.w += b * g.w;
+    float4 o = make_float4(a * g.x, a * g.y, a * g.z, a * g.w);
+    if (dx_final) {
+      const float4 f = reinterpret_cast<const float4*>(dx_final)[i];
+      o.x -= c * f.x; o.y -= c * f.y; o.z -= c * f.z; o.w -= c * f.w;
+    }
+    if (last) {
+      o.x += d0.x; o.y += d0.y; o.z += d0.z; o.w += d0.w;
+    } else {
+      reinterpret_cast<float4*>(dx0)[i] = d0;
+    }
+    reinterpret_cast<float4*>(dx)[i] = o;
+    store_bf16x4(gout + 4 * i, o);
+  }
+  block_sum2(sr, s0, part_r, part_0);
+}
+
+// Partial sums of a . b (the backout scale's gradient is -sum x_mid . dx_final).
+__global__ void __launch_bounds__(256) dot_partial_kernel(const float* __restrict__ a, const float* __restrict__ b,
+                                                          long long n4, float* __restrict__ part) {
+  float s = 0.f;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(a)[i];
+    const float4 y = reinterpret_cast<const float4*>(b)[i];
+    s += x.x * y.x + x.y * y.y + x.z * y.z + x.w * y.w;
+  }
+  block_sum2(s, 0.f, part, nullptr);
+}
+
+// Scalar gradients from their partial sums (nb per scalar, summed in a fixed
+// order by one warp each): grad[j] (+)= sign[j] * sum_k part[j][k].
+__global__ void scalar_grad_finish_kernel(const float* __restrict__ part, int nb, int count, float last_sign,
+                                          float* __restrict__ grad, int accumulate) {
+  const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= count) return;
+  float s = 0.f;
+  for (int k = lane; k < nb; k += 32) s += part[static_cast<long long>(j) * nb + k];
+  s = warp_sum(s);
+  if (lane == 0) {
+    if (j == count - 1) s *= last_sign;
+    grad[j] = accumulate ? grad[j] + s : s;
+  }
+}
+
 // -------------------------------------------------- QK-norm / RoPE backward
 
 __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restrict__ dk,
@@ -752,6 +884,41 @@ void launch_splitk_reduce(const float* part, int splits, long long stride, long 
                           cudaStream_t s) {
   const long long n4 = n / 4;
   splitk_reduce_kernel<<<stream_grid(n4, 256), 256, 0, s>>>(part, splits, stride, n4, out, accumulate ? 1 : 0);
+}
+
+constexpr int kResidBlocks = 4 * 148;
+
+int resid_partial_blocks() { return kResidBlocks; }
+
+void launch_resid_fwd(float* x, float* x_in, float* x0, const float* lam, int l, int L, long long n, bool first,
+                      cudaStream_t s) {
+  resid_fwd_kernel<<<stream_grid(n / 4, 256), 256, 0, s>>>(x, x_in, x0, lam, l, L, n / 4, first ? 1 : 0);
+}
+
+void launch_backout_fwd(float* x, const float* x_mid, const float* lam, int L, long long n, cudaStream_t s) {
+  backout_fwd_kernel<<<stream_grid(n / 4, 256), 256, 0, s>>>(x, x_mid, lam, L, n / 4);
+}
+
+void launch_resid_bwd(float* dx, const float* x_in, const float* x0, float* dx0, const float* dx_final,
+                      const float* lam, int l, int L, long long n, bf16* gout, float* part, bool first, bool last,
+                      cudaStream_t s) {
+  // partial sums of scalar j go to part[j * kResidBlocks ...]
+  resid_bwd_kernel<<<kResidBlocks, 256, 0, s>>>(dx, x_in, x0, dx0, dx_final, lam, l, L, n / 4, gout,
+                                                part + static_cast<long long>(l) * kResidBlocks,
+                                                part + static_cast<long long>(L + l) * kResidBlocks, first ? 1 : 0,
+                                                last ? 1 : 0);
+}
+
+void launch_backout_grad_partial(const float* x_mid, const float* dx_final, int L, long long n, float* part,
+                                 cudaStream_t s) {
+  dot_partial_kernel<<<kResidBlocks, 256, 0, s>>>(x_mid, dx_final, n / 4,
+                                                  part + static_cast<long long>(2 * L) * kResidBlocks);
+}
+
+void launch_scalar_grad_finish(const float* part, int L, float* grad, bool accumulate, cudaStream_t s) {
+  const int count = 2 * L + 1;
+  scalar_grad_finish_kernel<<<cdiv(count, 8), 256, 0, s>>>(part, kResidBlocks, count, -1.f, grad,
+                                                           accumulate ? 1 : 0);
 }
 
 void launch_adamw(float* p, const float* g, float* m, float* v, bf16* pb, long long n, float lr, float b1, float b2,

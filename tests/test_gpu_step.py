@@ -104,6 +104,65 @@ def test_sliding_window_layers_match_oracle(torch, pattern, short_window):
         assert c >= GRAD_COS, (pname, c)
 
 
+def _build_extras(torch, s, params):
+    import gpt_pretraining_step_b200 as g
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   residual_extras=True)
+    for tid, (name, *_rest) in enumerate(syn.param_specs(s, extras=True)):
+        st.set(tid, params[name])
+    return st
+
+
+def test_neutral_residual_extras_are_bit_identical_to_plain(torch):
+    """Scales 1 / 0 / 0 (the initial values) change nothing, bit for bit."""
+    import gpt_pretraining_step_b200 as g
+    s = SMALL["ragged"]
+    params = syn.init_params(s, seed=41, extras=True)
+    tok, tgt = torch.tensor(syn.tokens(s, seed=42)).cuda(), torch.tensor(syn.targets(s, seed=43)).cuda()
+    plain = build(torch, s, params)
+    ext = _build_extras(torch, s, params)
+    assert ext.num_tensors() == plain.num_tensors() + 1
+    assert torch.equal(ext.get(ext.num_tensors() - 1), torch.tensor(params["scalars"]).cuda())
+    la = float(plain.fwd_bwd(tok, tgt).item())
+    lb = float(ext.fwd_bwd(tok, tgt).item())
+    plain.check()
+    ext.check()
+    assert la == lb
+    for tid in range(plain.num_tensors()):
+        assert torch.equal(plain.get(tid, g.KIND_GRAD), ext.get(tid, g.KIND_GRAD)), tid
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_residual_extras_match_oracle(torch, name):
+    """Random residual / x0 / backout scales through the forward, the backward
+    (the scalars' gradients included) and the AdamW step of the scalars."""
+    import gpt_pretraining_step_b200 as g
+    s = SMALL[name]
+    params = syn.init_params(s, seed=44, extras=True)
+    params["scalars"] = syn.random_scalars(s, seed=45)
+    tok, tgt = syn.tokens(s, seed=46), syn.targets(s, seed=47)
+    st = _build_extras(torch, s, params)
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL
+    assert np.abs(f64(st.row_loss()).ravel() - cache["row_loss"]).max() < 2e-2
+    specs = syn.param_specs(s, extras=True)
+    for tid, (pname, *_r) in enumerate(specs):
+        got = f64(st.get(tid, g.KIND_GRAD))
+        c = cosine(got, grads[pname])
+        assert c >= GRAD_COS, (pname, c)
+    sid = len(specs) - 1
+    gs = f64(st.get(sid, g.KIND_GRAD))
+    assert relfro(gs, grads["scalars"]) <= 3e-2
+    # AdamW moves the scalars like the oracle does given the same gradient
+    st.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.0)
+    st.check()
+    p_ref, _, _ = oo.adamw_step(params["scalars"].astype(np.float64), gs, np.zeros_like(gs), np.zeros_like(gs), 1,
+                                3e-3, 0.8, 0.95, 1e-10, 0.0)
+    assert np.abs(f64(st.get(sid, g.KIND_PARAM)) - p_ref).max() < 1e-6
+
+
 def test_embedding_and_target_indexing_exact(torch):
     # with a zero lm_head the logits vanish: loss = ln V exactly, and dW_lm has
     # one shared column for every vocabulary id that is not a target, so the set
