@@ -41,7 +41,7 @@ struct Dims {
   int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32, fp8;
   int short_window, n_pat;
   char pat[12];
-  int extras;   // residual / x0 scales and backout (2L+1 scalars)
+  int extras;   // residual / x0 scales, backout and smear (2L+26 scalars)
   int nsc;      // scalar count rounded up to a multiple of 4
   // attention window of layer l: short_window for an 'S' layer, -1 = full causal
   int window(int l) const { return n_pat > 0 && pat[l % n_pat] == 'S' ? short_window : -1; }
@@ -62,7 +62,7 @@ struct Plan {
   size_t xf, rf, z, stats, zt, row_loss, loss;
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
-  size_t x0, xin, dx0, dxfin, scws;   // residual extras (allocated only when on)
+  size_t x0, xin, dx0, dxfin, scws, xe, sig;   // residual extras (allocated only when on)
   size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
@@ -135,7 +135,7 @@ int dims_from(const gpt_config* c, Dims& D) {
   D.short_window = c->short_window;
   if (c->residual_extras != 0 && c->residual_extras != 1) return fail(GPT_EINVAL, "residual_extras must be 0 or 1");
   D.extras = c->residual_extras;
-  D.nsc = (2 * D.L + 1 + 3) / 4 * 4;
+  D.nsc = (2 * D.L + 26 + 3) / 4 * 4;
   return GPT_OK;
 }
 
@@ -232,9 +232,11 @@ void make_plan(const Dims& D, Plan& P) {
     P.xin = ab.take(L * M * d * 4);
     P.dx0 = ab.take(M * d * 4);
     P.dxfin = ab.take(M * d * 4);
-    P.scws = ab.take(static_cast<size_t>(2 * L + 1) * resid_partial_blocks() * 4);
+    P.scws = ab.take(static_cast<size_t>(2 * L + 26) * resid_partial_blocks() * 4);
+    P.xe = ab.take(M * d * 4);
+    P.sig = ab.take(M * 4);
   } else {
-    P.x0 = P.xin = P.dx0 = P.dxfin = P.scws = 0;
+    P.x0 = P.xin = P.dx0 = P.dxfin = P.scws = P.xe = P.sig = 0;
   }
   P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
@@ -366,7 +368,7 @@ bool locate(const gpt_ctx* c, int id, int& grp, size_t& off, int& rows, int& col
   if (id == 1) { grp = 1; off = 0; rows = D.d; cols = D.V; return true; }
   const int k = id - 2;
   if (D.extras && k == 4 * D.L) {   // the residual-extras scalars
-    grp = 6; off = 0; rows = 1; cols = 2 * D.L + 1;
+    grp = 6; off = 0; rows = 1; cols = 2 * D.L + 26;
     return true;
   }
   if (k < 0 || k >= 4 * D.L) return false;
@@ -446,6 +448,13 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     if (tgt_in != tgt) clamp_targets_kernel<<<64, 256, 0, s>>>(tgt_in, tgt, M, V);
     else clamp_targets_kernel<<<64, 256, 0, s>>>(tgt, tgt, M, V);
     launch_embed_fwd(tok, c->Wb(0), x, M, d, V, err, s);
+  }
+  if (D.extras) {
+    // smear: the embedding is kept for the backward, x takes the smeared one
+    ProfScope ps(c, GPT_PROF_EMBED);
+    GPT_CK(cudaMemcpyAsync(c->A<float>(P.xe), x, static_cast<size_t>(M) * d * 4, cudaMemcpyDeviceToDevice, s));
+    launch_smear_fwd(c->A<float>(P.xe), x, c->A<float>(P.sig), c->Scal(), L, D.T, M, d, s);
+    c->launches += 1;
   }
   // fp8: e4m3 copies of every block matrix, one scale per matrix
   uint8_t* act8 = c->A<uint8_t>(P.act8);
@@ -725,14 +734,19 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     c->launches += 4;
   }
+  // the embedding's gradient: through the smear when the extras are on
+  float* demb = dx;
   if (D.extras) {
-    ProfScope ps(c, GPT_PROF_NORM);
+    ProfScope ps(c, GPT_PROF_EMBED);
+    demb = c->A<float>(P.dx0);   // free once block 0 has added it into dx
+    launch_smear_bwd(dx, c->A<float>(P.xe), c->A<float>(P.sig), c->Scal(), demb, c->A<float>(P.scws), L, D.T, M, d,
+                     s);
     launch_scalar_grad_finish(c->A<float>(P.scws), L, reinterpret_cast<float*>(c->sbuf + P.gs), acc, s);
-    c->launches += 1;
+    c->launches += 2;
   }
   {
     ProfScope ps(c, GPT_PROF_EMBED);
-    launch_embed_bwd(tok, dx, c->G(0), M, d, V, c->A<void>(P.embws), acc, s);
+    launch_embed_bwd(tok, demb, c->G(0), M, d, V, c->A<void>(P.embws), acc, s);
   }
   c->launches += 2 * ((M + 32767) / 32768);
   GPT_CK(cudaGetLastError());

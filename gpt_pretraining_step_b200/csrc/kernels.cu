@@ -303,9 +303,95 @@ __global__ void __launch_bounds__(256) dot_partial_kernel(const float* __restric
   block_sum2(s, 0.f, part, nullptr);
 }
 
+// Smear (efficiency trick 2): x[t] = e[t] + gate[t] e[t-1] for t > 0 within
+// a sequence, gate[t] = lam_s * sigmoid(w . e[t, :24]) with lam_s = lam[2L+1]
+// and w = lam[2L+2 .. 2L+26).  One warp per token; sig[t] is kept for the
+// backward.
+constexpr int kSmearChannels = 24;
+
+__global__ void __launch_bounds__(256) smear_fwd_kernel(const float* __restrict__ e, float* __restrict__ x,
+                                                        float* __restrict__ sig, const float* __restrict__ lam,
+                                                        int L, int T, int M, int d) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  const float* er = e + static_cast<long long>(t) * d;
+  float z = lane < kSmearChannels ? lam[2 * L + 2 + lane] * er[lane] : 0.f;
+  z = warp_sum(z);
+  const float sg = 1.f / (1.f + expf(-z));
+  const float gate = (t % T) > 0 ? lam[2 * L + 1] * sg : 0.f;
+  if (lane == 0) sig[t] = sg;
+  float* xr = x + static_cast<long long>(t) * d;
+  for (int c = 4 * lane; c < d; c += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(er + c);
+    float4 o = v;
+    if (gate != 0.f) {
+      const float4 p = *reinterpret_cast<const float4*>(er - d + c);
+      o.x += gate * p.x; o.y += gate * p.y; o.z += gate * p.z; o.w += gate * p.w;
+    }
+    *reinterpret_cast<float4*>(xr + c) = o;
+  }
+}
+
+// Backward of the smear: g = dL/dx, output de = dL/de; partial sums of the
+// smear scale's and gate weights' gradients per block (part[j * nb + block]
+// for scalar j = 2L+1 .. 2L+25).  A fixed grid of warps strides over the
+// tokens, so the sums do not depend on scheduling.
+__global__ void __launch_bounds__(256) smear_bwd_kernel(const float* __restrict__ g, const float* __restrict__ e,
+                                                        const float* __restrict__ sig, const float* __restrict__ lam,
+                                                        float* __restrict__ de, float* __restrict__ part, int L,
+                                                        int T, int M, int d) {
+  __shared__ float acc[8][kSmearChannels + 1];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float lam_s = lam[2 * L + 1];
+  const float wc = lane < kSmearChannels ? lam[2 * L + 2 + lane] : 0.f;
+  float a_lam = 0.f, a_w = 0.f;   // this lane's share: the scale (lane 0) and gate weight `lane`
+  for (int t = blockIdx.x * 8 + w; t < M; t += gridDim.x * 8) {
+    const long long off = static_cast<long long>(t) * d;
+    const int pos = t % T;
+    // s = dL/dgate[t] = g[t] . e[t-1]
+    float sdot = 0.f;
+    if (pos > 0) {
+      for (int c = 4 * lane; c < d; c += 128) {
+        const float4 a = *reinterpret_cast<const float4*>(g + off + c);
+        const float4 b = *reinterpret_cast<const float4*>(e + off - d + c);
+        sdot += a.x * b.x + a.y * b.y + a.z * b.z + a.w * b.w;
+      }
+    }
+    sdot = warp_sum(sdot);
+    const float sg = sig[t];
+    const float dz = sdot * lam_s * sg * (1.f - sg);
+    const float gnext = (pos + 1 < T && t + 1 < M) ? lam_s * sig[t + 1] : 0.f;   // e[t] feeds position t + 1
+    for (int c = 4 * lane; c < d; c += 128) {
+      float4 o = *reinterpret_cast<const float4*>(g + off + c);
+      if (gnext != 0.f) {
+        const float4 n = *reinterpret_cast<const float4*>(g + off + d + c);
+        o.x += gnext * n.x; o.y += gnext * n.y; o.z += gnext * n.z; o.w += gnext * n.w;
+      }
+      *reinterpret_cast<float4*>(de + off + c) = o;
+    }
+    __syncwarp();
+    if (lane < kSmearChannels) {
+      // the gate reads channels 0..23: d(de[t, c]) = dz w[c]; dw[c] += dz e[t, c]
+      de[off + lane] += dz * wc;
+      a_w += dz * e[off + lane];
+    }
+    a_lam += sdot * sg;
+  }
+  if (lane < kSmearChannels) acc[w][1 + lane] = a_w;
+  if (lane == 0) acc[w][0] = a_lam;
+  __syncthreads();
+  if (threadIdx.x < kSmearChannels + 1) {
+    float sum = 0.f;
+    for (int k = 0; k < 8; ++k) sum += acc[k][threadIdx.x];
+    part[static_cast<long long>(2 * L + 1 + threadIdx.x) * gridDim.x + blockIdx.x] = sum;
+  }
+}
+
 // Scalar gradients from their partial sums (nb per scalar, summed in a fixed
-// order by one warp each): grad[j] (+)= sign[j] * sum_k part[j][k].
-__global__ void scalar_grad_finish_kernel(const float* __restrict__ part, int nb, int count, float last_sign,
+// order by one warp each): grad[j] (+)= sum_k part[j][k], negated for j =
+// neg_index (the backout scale, whose partials are sums of x_mid . dx).
+__global__ void scalar_grad_finish_kernel(const float* __restrict__ part, int nb, int count, int neg_index,
                                           float* __restrict__ grad, int accumulate) {
   const int j = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -314,7 +400,7 @@ __global__ void scalar_grad_finish_kernel(const float* __restrict__ part, int nb
   for (int k = lane; k < nb; k += 32) s += part[static_cast<long long>(j) * nb + k];
   s = warp_sum(s);
   if (lane == 0) {
-    if (j == count - 1) s *= last_sign;
+    if (j == neg_index) s = -s;
     grad[j] = accumulate ? grad[j] + s : s;
   }
 }
@@ -916,9 +1002,19 @@ void launch_backout_grad_partial(const float* x_mid, const float* dx_final, int 
 }
 
 void launch_scalar_grad_finish(const float* part, int L, float* grad, bool accumulate, cudaStream_t s) {
-  const int count = 2 * L + 1;
-  scalar_grad_finish_kernel<<<cdiv(count, 8), 256, 0, s>>>(part, kResidBlocks, count, -1.f, grad,
+  const int count = 2 * L + 26;
+  scalar_grad_finish_kernel<<<cdiv(count, 8), 256, 0, s>>>(part, kResidBlocks, count, 2 * L, grad,
                                                            accumulate ? 1 : 0);
+}
+
+void launch_smear_fwd(const float* e, float* x, float* sig, const float* lam, int L, int T, int M, int d,
+                      cudaStream_t s) {
+  smear_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(e, x, sig, lam, L, T, M, d);
+}
+
+void launch_smear_bwd(const float* g, const float* e, const float* sig, const float* lam, float* de, float* part,
+                      int L, int T, int M, int d, cudaStream_t s) {
+  smear_bwd_kernel<<<kResidBlocks, 256, 0, s>>>(g, e, sig, lam, de, part, L, T, M, d);
 }
 
 void launch_adamw(float* p, const float* g, float* m, float* v, bf16* pb, long long n, float lr, float b1, float b2,

@@ -75,19 +75,27 @@ void launch_muon_apply(float* W, bf16* Wb, const void* X, int x_es, int nmat, in
 void launch_normuon_factor(const void* X, int x_es, int nmat, int r, int c, float* V, float beta2, float* ws,
                            cudaStream_t s);
 
-// Residual extras (per-layer residual / x0 scales and backout); lam holds
-// (resid[0..L), x0[0..L), backout), n is the element count (multiple of 4).
+// Residual extras (per-layer residual / x0 scales, backout, smear); lam holds
+// (resid[0..L), x0[0..L), backout, smear scale, smear gate weights[24]), n is
+// the element count (multiple of 4).
 void launch_resid_fwd(float* x, float* x_in, float* x0, const float* lam, int l, int L, long long n, bool first,
                       cudaStream_t s);
 void launch_backout_fwd(float* x, const float* x_mid, const float* lam, int L, long long n, cudaStream_t s);
 // dx holds dL/dx' on entry and dL/dx_in on return (for block 0 plus dx0);
-// part: (2L+1) x resid_partial_blocks() floats of partial sums.
+// part: (2L+26) x resid_partial_blocks() floats of partial sums.
 void launch_resid_bwd(float* dx, const float* x_in, const float* x0, float* dx0, const float* dx_final,
                       const float* lam, int l, int L, long long n, bf16* gout, float* part, bool first, bool last,
                       cudaStream_t s);
 void launch_backout_grad_partial(const float* x_mid, const float* dx_final, int L, long long n, float* part,
                                  cudaStream_t s);
 void launch_scalar_grad_finish(const float* part, int L, float* grad, bool accumulate, cudaStream_t s);
+// Smear: x = e + lam_s sigmoid(w . e[:, :24]) e(previous position); sig [M]
+// kept for the backward, which writes de = dL/de and the partial sums of the
+// smear scalars' gradients.
+void launch_smear_fwd(const float* e, float* x, float* sig, const float* lam, int L, int T, int M, int d,
+                      cudaStream_t s);
+void launch_smear_bwd(const float* g, const float* e, const float* sig, const float* lam, float* de, float* part,
+                      int L, int T, int M, int d, cudaStream_t s);
 int resid_partial_blocks();
 
 // Per-tensor e4m3 quantisation of nmat matrices of n bf16 values each (z-th at

@@ -102,15 +102,18 @@ typedef struct gpt_config {
                            * zero) = every layer full causal.  "¿Cómo Entrenar
                            * Tu Propio ChatGPT por $50?", section "1. Modelo
                            * GPT", sliding-window attention. */
-  int32_t residual_extras;/* 1: per-layer residual and x0 scales and the
-                           * backout scale of section "1. Modelo GPT"
-                           * (efficiency tricks 1 and 3): before block i,
-                           * x <- resid[i] x + x0s[i] x0 (x0 = embedding
-                           * output); after the last block,
+  int32_t residual_extras;/* 1: the smear, per-layer residual and x0 scales
+                           * and the backout of section "1. Modelo GPT"
+                           * (efficiency tricks 1-3): the embedding e of
+                           * position t becomes e[t] + smear sigmoid(w .
+                           * e[t, :24]) e[t-1] (t > 0); before block i,
+                           * x <- resid[i] x + x0s[i] x0 (x0 = the smeared
+                           * embedding); after the last block,
                            * x <- x - backout * (stream entering block
-                           * depth/2).  2*depth+1 scalars, tensor id
+                           * depth/2).  2*depth+26 scalars, tensor id
                            * 2 + 4*depth, trained by adamw_step, initialised
-                           * to resid = 1, x0s = 0, backout = 0.  0: off. */
+                           * to resid = 1 and everything else 0 (the plain
+                           * network).  0: off. */
 } gpt_config;
 
 typedef struct gpt_ctx gpt_ctx;
@@ -196,8 +199,8 @@ int gpt_train_step_host(gpt_ctx* ctx, const int32_t* tokens_host, const int32_t*
 /* Parameter tensors: id 0 = token embedding [vocab, d], 1 = lm_head [d, vocab],
  * 2 + 4 l + j for block l with j = 0 fused q|k|v [d, 3d], 1 attention output
  * [d, d], 2 MLP up [d, 4d], 3 MLP down [4d, d]; with residual_extras, id
- * 2 + 4 depth = the scalars [1, 2 depth + 1] (resid[0..depth),
- * x0s[0..depth), backout). */
+ * 2 + 4 depth = the scalars [1, 2 depth + 26] (resid[0..depth),
+ * x0s[0..depth), backout, smear, smear gate weights[24]). */
 int gpt_num_tensors(const gpt_ctx* ctx);
 int gpt_tensor_info(const gpt_ctx* ctx, int id, int32_t* rows, int32_t* cols, int32_t* group);
 

@@ -20,13 +20,17 @@ Readings where the pages are silent (shared with the CUDA path):
     not matter mathematically: a rotation keeps the RMS).
   * attention scale 1/sqrt(hd); n_kv_head = n_head.
   * residual extras ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section
-    "1. Modelo GPT", efficiency tricks 1 and 3), present when params holds a
-    "scalars" vector [2L + 1] = (resid lambdas, x0 lambdas, backout lambda):
-    before block i, x <- resid[i] x + x0l[i] x0 with x0 the embedding output;
-    after the last block, x <- x - backout * x_mid with x_mid the residual
-    stream entering block L // 2 (before its scaling).  Initial values 1, 0
-    and 0 make the network the plain one.  Smear and value embeddings are
-    not part of this oracle.
+    "1. Modelo GPT", efficiency tricks 1, 2 and 3), present when params holds
+    a "scalars" vector [2L + 26] = (resid lambdas [L], x0 lambdas [L],
+    backout lambda, smear lambda, smear gate weights [24]):
+      smear: the embedding e of position t takes gate[t] = smear_lambda *
+      sigmoid(w . e[t, :24]) times the previous position's embedding,
+      x[t] = e[t] + gate[t] e[t-1] (t > 0 within the sequence);
+      before block i, x <- resid[i] x + x0l[i] x0 with x0 the smeared
+      embedding; after the last block, x <- x - backout * x_mid with x_mid
+      the residual stream entering block L // 2 (before its scaling).
+    Initial values resid 1 and everything else 0 make the network the plain
+    one.  Value embeddings are not part of this oracle.
   * attention window per layer: full causal by default; with a layer pattern
     such as "SSSL" (section "1. Modelo GPT", sliding-window attention) the
     pattern is repeated over the layers, S = a sliding window of
@@ -42,6 +46,7 @@ import numpy as np
 
 EPS = 1e-6
 ROPE_BASE = 10000.0
+SMEAR_CHANNELS = 24   # embedding channels the smear gate reads
 
 
 # --- building blocks -------------------------------------------------------
@@ -190,10 +195,19 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
     cos, sin = rope_angles(T, head_dim)
     x = wte[tok.reshape(-1)]                         # [M, d] exact row copy
     sc = params.get("scalars")
+    e = x
     if sc is not None:
         sc = np.asarray(sc, dtype=np.float64).reshape(-1)
-        if sc.size != 2 * n_layer + 1:
-            raise ValueError("scalars must hold 2 * n_layer + 1 values")
+        if sc.size != 2 * n_layer + 26:
+            raise ValueError("scalars must hold 2 * n_layer + 26 values")
+        lam_s, w_s = sc[2 * n_layer + 1], sc[2 * n_layer + 2:]
+        e3 = e.reshape(B, T, -1)
+        zg = e3[:, :, :SMEAR_CHANNELS] @ w_s                 # [B, T]
+        sig = 1.0 / (1.0 + np.exp(-zg))
+        gate = lam_s * sig
+        prev = np.concatenate([np.zeros_like(e3[:, :1]), e3[:, :-1]], axis=1)
+        gate = gate * (np.arange(T) > 0)[None, :]
+        x = (e3 + gate[:, :, None] * prev).reshape(B * T, -1)
     x0 = x
     x_in, x_mid = [], None
     acts = []
@@ -233,7 +247,8 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
     row_loss = lse - z[np.arange(z.shape[0]), t]
     loss = float(np.mean(row_loss))
     cache = dict(acts=acts, xf=xf, rf=rf, z=z, lse=lse, row_loss=row_loss,
-                 B=B, T=T, H=H, d=d, cos=cos, sin=sin, scalars=sc, x0=x0, x_in=x_in, x_mid=x_mid) if keep else None
+                 B=B, T=T, H=H, d=d, cos=cos, sin=sin, scalars=sc, x0=x0, x_in=x_in, x_mid=x_mid,
+                 emb=e, smear_sig=sig if sc is not None else None) if keep else None
     return loss, cache
 
 
@@ -253,7 +268,7 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
     dx = rms_norm_bwd(dz @ Wlm.T, cache["xf"], cache["rf"])
     sc = cache["scalars"]
     if sc is not None:
-        dsc = np.zeros(2 * n_layer + 1)
+        dsc = np.zeros(2 * n_layer + 26)
         dx_final = dx                                # gradient at the backout output
         dsc[2 * n_layer] = -np.sum(cache["x_mid"] * dx_final)
         dx0 = np.zeros_like(dx)
@@ -286,6 +301,22 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
                 dx = dx - sc[2 * n_layer] * dx_final
     if sc is not None:
         dx = dx + dx0
+        # smear: x[t] = e[t] + lam sig(w . e[t, :24]) e[t-1]
+        lam_s, w_s = sc[2 * n_layer + 1], sc[2 * n_layer + 2:]
+        e3 = cache["emb"].reshape(B, T, -1)
+        g3 = dx.reshape(B, T, -1)
+        sig = cache["smear_sig"]
+        live = (np.arange(T) > 0)[None, :]
+        prev = np.concatenate([np.zeros_like(e3[:, :1]), e3[:, :-1]], axis=1)
+        sdot = np.sum(g3 * prev, axis=-1) * live               # dL/dgate[t]
+        de = g3.copy()
+        gate = lam_s * sig * live
+        de[:, :-1] += gate[:, 1:, None] * g3[:, 1:]            # e[t] is the previous token of t + 1
+        dz = sdot * lam_s * sig * (1.0 - sig)
+        de[:, :, :SMEAR_CHANNELS] += dz[:, :, None] * w_s[None, None, :]
+        dsc[2 * n_layer + 1] = np.sum(sdot * sig)
+        dsc[2 * n_layer + 2:] = np.einsum("bt,btc->c", dz, e3[:, :, :SMEAR_CHANNELS])
+        dx = de.reshape(B * T, -1)
         grads["scalars"] = dsc.reshape(1, -1)
     V = params["wte"].shape[0]
     dwte = np.zeros((V, d))

@@ -79,8 +79,9 @@ def param_specs(s: Shape, extras: bool = False):
                 (f"h{layer}.c_fc", d, f, "muon"),
                 (f"h{layer}.mlp_proj", f, d, "muon")]
     if extras:
-        # per-layer residual and x0 scales, then the backout scale
-        out.append(("scalars", 1, 2 * s.depth + 1, "adamw"))
+        # per-layer residual and x0 scales, the backout scale, the smear scale
+        # and the smear gate's 24 weights
+        out.append(("scalars", 1, 2 * s.depth + 26, "adamw"))
     return out
 
 
@@ -101,24 +102,27 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
 def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False):
     """N(0, std) weights rounded to bf16, as float32 arrays keyed by name;
     with extras also the scalar vector at its neutral values (residual
-    scales 1, x0 and backout scales 0)."""
+    scales 1, everything else 0)."""
     rng = np.random.Generator(np.random.PCG64(seed))
     params = {}
     for name, r, c, _ in param_specs(s):
         w = rng.standard_normal((r, c), dtype=np.float32) * np.float32(std)
         params[name] = round_to_bf16(w)
     if extras:
-        sc = np.zeros((1, 2 * s.depth + 1), dtype=np.float32)
+        sc = np.zeros((1, 2 * s.depth + 26), dtype=np.float32)
         sc[0, :s.depth] = 1.0
         params["scalars"] = sc
     return params
 
 
 def random_scalars(s: Shape, seed: int) -> np.ndarray:
-    """Residual scales in [0.5, 1.5], x0 and backout scales in [-0.5, 0.5]."""
+    """Residual scales in [0.5, 1.5]; x0, backout and smear scales in
+    [-0.5, 0.5]; smear gate weights N(0, 1) (the gate reads embedding
+    channels of size ~0.02, so this keeps it away from saturation)."""
     rng = np.random.Generator(np.random.PCG64(seed))
-    sc = rng.uniform(-0.5, 0.5, size=(1, 2 * s.depth + 1)).astype(np.float32)
+    sc = rng.uniform(-0.5, 0.5, size=(1, 2 * s.depth + 26)).astype(np.float32)
     sc[0, :s.depth] += 1.0
+    sc[0, 2 * s.depth + 2:] = rng.standard_normal(24).astype(np.float32) * 10.0
     return sc
 
 

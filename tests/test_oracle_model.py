@@ -348,14 +348,14 @@ def _extras_case(depth=2, seed=0, **kw):
 
 def test_neutral_scalars_give_the_plain_model():
     s, p, tok, tgt = _extras_case(std=0.05)
-    sc = np.zeros((1, 2 * s.depth + 1))
+    sc = np.zeros((1, 2 * s.depth + 26))
     sc[0, :s.depth] = 1.0
     l0, g0, _ = om.fwd_bwd(p, tok, tgt, s.depth)
     l1, g1, _ = om.fwd_bwd(dict(p, scalars=sc), tok, tgt, s.depth)
     assert l0 == l1
     for k in g0:
         assert np.array_equal(g0[k], g1[k]), k
-    assert g1["scalars"].shape == (1, 2 * s.depth + 1)
+    assert g1["scalars"].shape == (1, 2 * s.depth + 26)
 
 
 def test_x0_only_inputs_reduce_to_the_last_block():
@@ -363,7 +363,7 @@ def test_x0_only_inputs_reduce_to_the_last_block():
     # last block's contribution survives: a one-block model with its weights
     depth = 3
     s, p, tok, tgt = _extras_case(depth=depth, std=0.05, seed=4)
-    sc = np.zeros((1, 2 * depth + 1))
+    sc = np.zeros((1, 2 * depth + 26))
     sc[0, depth:2 * depth] = 1.0
     loss, _ = om.forward(dict(p, scalars=sc), tok, tgt, depth, keep=False)
     one = {"wte": p["wte"], "lm_head": p["lm_head"]}
@@ -377,7 +377,9 @@ def test_backout_of_the_whole_stream_before_the_middle():
     # depth 2 with backout 1: the final stream is x_mid + f1(x_mid) - x_mid,
     # i.e. the last block's contribution alone on top of nothing
     s, p, tok, tgt = _extras_case(depth=2, std=0.05, seed=6)
-    sc = np.array([[1.0, 1.0, 0.0, 0.0, 1.0]])
+    sc = np.zeros((1, 2 * 2 + 26))
+    sc[0, :2] = 1.0
+    sc[0, 4] = 1.0
     _, c = om.forward(dict(p, scalars=sc), tok, tgt, 2)
     _, cp = om.forward(p, tok, tgt, 2)
     # the stream entering block 1 is the final stream of block 0 alone
@@ -392,3 +394,19 @@ def test_finite_difference_with_residual_extras():
     p["scalars"] = syn.random_scalars(s, seed=9).astype(np.float64)
     names = [n for n, *_ in syn.param_specs(s, extras=True)]
     _fd_check(p, tok, tgt, s.depth, names, n_coords=4)
+
+
+def test_smear_mixes_the_previous_embedding():
+    # smear scale c with a zero gate weight vector: gate = c / 2, so the stream
+    # entering block 0 is e[t] + (c / 2) e[t-1] (e[t] alone at t = 0)
+    s, p, tok, tgt = _extras_case(depth=1, std=0.05, seed=12)
+    sc = np.zeros((1, 2 + 26))
+    sc[0, 0] = 1.0
+    sc[0, 3] = 0.8
+    _, c = om.forward(dict(p, scalars=sc), tok, tgt, 1)
+    e = p["wte"][tok]                                    # [B, T, d]
+    ref = e.copy()
+    ref[:, 1:] += 0.4 * e[:, :-1]
+    assert np.allclose(c["x0"].reshape(e.shape), ref, rtol=1e-12, atol=1e-15)
+    # a token's smear never reaches across the sequence boundary
+    assert np.array_equal(c["x0"].reshape(e.shape)[:, 0], e[:, 0])
