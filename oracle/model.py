@@ -30,7 +30,12 @@ Readings where the pages are silent (shared with the CUDA path):
       embedding; after the last block, x <- x - backout * x_mid with x_mid
       the residual stream entering block L // 2 (before its scaling).
     Initial values resid 1 and everything else 0 make the network the plain
-    one.  Value embeddings are not part of this oracle.
+    one.
+  * value embeddings (section "1. Modelo GPT", value residual), present when
+    params holds "ve{l}" tables [V, d] for the layers l with l % 2 == 0 and
+    "ve_gate" [C, H] (one block of C rows per such layer, stacked
+    [n_ve * C, H]): v[t, h] += 3 sigmoid(xn1[t, :C] . ve_gate_l[:, h])
+    ve_l[tok[t], h*hd:(h+1)*hd], xn1 being the block's attention input.
   * attention window per layer: full causal by default; with a layer pattern
     such as "SSSL" (section "1. Modelo GPT", sliding-window attention) the
     pattern is repeated over the layers, S = a sliding window of
@@ -170,6 +175,11 @@ def _merge_heads(a):
     return a.transpose(0, 2, 1, 3).reshape(B * T, H * hd)
 
 
+def ve_layer_count(n_layer):
+    """Layers with a value embedding: l % 2 == 0."""
+    return (n_layer + 1) // 2
+
+
 def layer_windows(pattern, short_window, n_layer):
     """Window of every layer: pattern[l % len(pattern)] is "S" (sliding window
     of short_window earlier tokens) or "L" (full causal, None); an empty
@@ -225,6 +235,15 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
         q = _split_heads(qkv[:, :d], B, T, H, head_dim)
         k = _split_heads(qkv[:, d:2 * d], B, T, H, head_dim)
         v = _split_heads(qkv[:, 2 * d:], B, T, H, head_dim)
+        if f"ve{l}" in params:
+            # value residual: v + 3 sigmoid(gate) * ve, per head
+            C = params["ve_gate"].shape[0] // ve_layer_count(n_layer)
+            Wg = np.asarray(params["ve_gate"], dtype=np.float64)[(l // 2) * C:(l // 2 + 1) * C]
+            ve = np.asarray(params[f"ve{l}"], dtype=np.float64)[tok.reshape(-1)]      # [M, d]
+            sg = 1.0 / (1.0 + np.exp(-(xn1[:, :C] @ Wg)))                           # [M, H]
+            v = v + _split_heads(np.repeat(3.0 * sg, head_dim, axis=1) * ve, B, T, H, head_dim)
+            if keep:
+                a.update(ve=ve, ve_sig=sg, ve_C=C)
         qn, rq = rms_norm(rope(q, cos, sin))
         kn, rk = rms_norm(rope(k, cos, sin))
         y, P = attention(qn, kn, v, None if windows is None else windows[l])
@@ -290,7 +309,22 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
         dk = rope_bwd(rms_norm_bwd(dkn, a["kn"], a["rk"]), cos, sin)
         dqkv = np.concatenate([_merge_heads(dq), _merge_heads(dk), _merge_heads(dv)], axis=1)
         grads[f"h{l}.c_qkv"] = a["xn1"].T @ dqkv
-        dx = dx + rms_norm_bwd(dqkv @ W["c_qkv"].T, a["xn1"], a["r1"])
+        dxn1 = dqkv @ W["c_qkv"].T
+        if "ve" in a:
+            C, sg, ve = a["ve_C"], a["ve_sig"], a["ve"]
+            dvm = _merge_heads(dv)                                                   # [M, d]
+            dve = np.repeat(3.0 * sg, head_dim, axis=1) * dvm
+            gve = np.zeros_like(np.asarray(params[f"ve{l}"], dtype=np.float64))
+            np.add.at(gve, tok.reshape(-1), dve)
+            grads[f"ve{l}"] = gve
+            dgate = (ve * dvm).reshape(-1, H, head_dim).sum(axis=-1)                # [M, H]
+            dz = dgate * 3.0 * sg * (1.0 - sg)
+            Wg = np.asarray(params["ve_gate"], dtype=np.float64)[(l // 2) * C:(l // 2 + 1) * C]
+            if "ve_gate" not in grads:
+                grads["ve_gate"] = np.zeros_like(np.asarray(params["ve_gate"], dtype=np.float64))
+            grads["ve_gate"][(l // 2) * C:(l // 2 + 1) * C] = a["xn1"][:, :C].T @ dz
+            dxn1[:, :C] += dz @ Wg.T
+        dx = dx + rms_norm_bwd(dxn1, a["xn1"], a["r1"])
         if sc is not None:
             # x' = resid[l] x_in + x0l[l] x0 (and x_in of block L // 2 feeds the backout)
             dsc[l] = np.sum(cache["x_in"][l] * dx)

@@ -64,7 +64,12 @@ def config_shape(name: str) -> Shape:
     return make_shape(**CONFIGS[name])
 
 
-def param_specs(s: Shape, extras: bool = False):
+def ve_layers(depth: int):
+    """Layers with a value embedding (every other layer, from the first)."""
+    return [l for l in range(depth) if l % 2 == 0]
+
+
+def param_specs(s: Shape, extras: bool = False, ve_channels: int = 0):
     """(name, rows, cols, group) for every parameter; matrices are [in, out].
 
     Order: token embedding, lm_head, then per layer the fused q|k|v projection,
@@ -82,6 +87,10 @@ def param_specs(s: Shape, extras: bool = False):
         # per-layer residual and x0 scales, the backout scale, the smear scale
         # and the smear gate's 24 weights
         out.append(("scalars", 1, 2 * s.depth + 26, "adamw"))
+    if ve_channels:
+        # value embedding tables, then the gates of all of them stacked
+        out += [(f"ve{l}", s.vocab, d, "adamw") for l in ve_layers(s.depth)]
+        out.append(("ve_gate", ve_channels * len(ve_layers(s.depth)), s.n_head, "adamw"))
     return out
 
 
@@ -99,7 +108,7 @@ def bf16_bits(a: np.ndarray) -> np.ndarray:
     return (a.view(np.uint32) >> 16).astype(np.uint16)
 
 
-def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False):
+def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False, ve_channels: int = 0):
     """N(0, std) weights rounded to bf16, as float32 arrays keyed by name;
     with extras also the scalar vector at its neutral values (residual
     scales 1, everything else 0)."""
@@ -112,6 +121,13 @@ def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False
         sc = np.zeros((1, 2 * s.depth + 26), dtype=np.float32)
         sc[0, :s.depth] = 1.0
         params["scalars"] = sc
+    if ve_channels:
+        # value embedding tables N(0, std) like the token embedding; gates zero
+        # (every gate then starts at 3 sigmoid(0) = 1.5)
+        for l in ve_layers(s.depth):
+            params[f"ve{l}"] = round_to_bf16(rng.standard_normal((s.vocab, s.d_model), dtype=np.float32)
+                                             * np.float32(std))
+        params["ve_gate"] = np.zeros((ve_channels * len(ve_layers(s.depth)), s.n_head), dtype=np.float32)
     return params
 
 

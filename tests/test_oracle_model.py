@@ -410,3 +410,51 @@ def test_smear_mixes_the_previous_embedding():
     assert np.allclose(c["x0"].reshape(e.shape), ref, rtol=1e-12, atol=1e-15)
     # a token's smear never reaches across the sequence boundary
     assert np.array_equal(c["x0"].reshape(e.shape)[:, 0], e[:, 0])
+
+
+# --- value embeddings ------------------------------------------------------------
+#
+# Section "1. Modelo GPT", value residual: on every other layer (from the
+# first) v[t, h] += 3 sigmoid(xn1[t, :C] . W_g[:, h]) ve[tok[t], head h].
+
+def _ve_case(depth=2, C=8, seed=0, **kw):
+    s = syn.make_shape(depth=depth, batch=kw.pop("batch", 2), seq_len=kw.pop("seq", 10),
+                       vocab=kw.pop("vocab", 40), d_model=kw.pop("d", 256))
+    p = syn.init_params(s, seed=seed, std=0.05, ve_channels=C)
+    rng = np.random.default_rng(seed + 1)
+    p["ve_gate"] = rng.standard_normal(p["ve_gate"].shape).astype(np.float32) * 2.0
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    return s, p, syn.tokens(s, seed=seed + 2), syn.targets(s, seed=seed + 3)
+
+
+def test_zero_value_embeddings_give_the_plain_model():
+    s, p, tok, tgt = _ve_case()
+    for l in syn.ve_layers(s.depth):
+        p[f"ve{l}"] = np.zeros_like(p[f"ve{l}"])
+    plain = {k: v for k, v in p.items() if not k.startswith("ve")}
+    l0, g0, _ = om.fwd_bwd(plain, tok, tgt, s.depth)
+    l1, g1, _ = om.fwd_bwd(p, tok, tgt, s.depth)
+    assert l0 == l1
+    for k in g0:
+        assert np.array_equal(g0[k], g1[k]), k
+
+
+def test_value_embedding_brute_force():
+    import math
+    s, p, tok, tgt = _ve_case(depth=1, C=4, batch=1, seq=5, d=256)
+    _, c = om.forward(p, tok, tgt, 1)
+    _, c0 = om.forward({k: v for k, v in p.items() if not k.startswith("ve")}, tok, tgt, 1)
+    a, a0 = c["acts"][0], c0["acts"][0]
+    H, hd = s.n_head, 128
+    for t in range(5):
+        for h in range(H):
+            z = sum(a["xn1"][t, cc] * p["ve_gate"][cc, h] for cc in range(4))
+            g = 3.0 / (1.0 + math.exp(-z))
+            ref = a0["v"][0, h, t] + g * p["ve0"][tok[0, t], h * hd:(h + 1) * hd]
+            assert np.allclose(a["v"][0, h, t], ref, rtol=1e-12, atol=1e-14), (t, h)
+
+
+def test_finite_difference_with_value_embeddings():
+    s, p, tok, tgt = _ve_case(depth=2, C=8, seed=5, d=256, vocab=32, seq=8)
+    names = ["ve0", "ve_gate", "h0.c_qkv", "h1.c_qkv", "wte"]
+    _fd_check(p, tok, tgt, s.depth, names, n_coords=6)
