@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--short-window", type=int, default=1024, help="left context of an S layer, tokens")
     ap.add_argument("--residual-extras", action="store_true",
                     help="per-layer residual / x0 scales and backout (scalar parameters trained by AdamW)")
+    ap.add_argument("--value-embeds", type=int, default=0, metavar="C",
+                    help="value embeddings on layers 0, 2, ... with C gate channels (0 = off)")
     ap.add_argument("--shard-optimizer", action="store_true",
                     help="N > 1: each rank runs Muon on its own layer range (three-phase ZeRO-2 style exchange)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -267,7 +269,7 @@ def run_ours(a):
     st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
                    ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream,
                    precision=1 if a.precision == "fp8" else 0, window_pattern=a.window_pattern,
-                   short_window=a.short_window, residual_extras=a.residual_extras)
+                   short_window=a.short_window, residual_extras=a.residual_extras, ve_gate_channels=a.value_embeds)
     tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(1, rank))).cuda()
     tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(2, rank))).cuda()
     grads = st.grad_view() if world > 1 else None
@@ -395,7 +397,7 @@ def run_ours(a):
                        "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
                        "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
                                      else "full causal"),
-                       "residual_extras": bool(a.residual_extras)},
+                       "residual_extras": bool(a.residual_extras), "value_embed_channels": a.value_embeds},
             "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
             "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",
             "model_tflop_per_step": fpt * s.tokens / 1e12,

@@ -42,7 +42,8 @@ class Config(ctypes.Structure):
                 ("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("mlp_mult", ctypes.c_int32), ("precision", ctypes.c_int32), ("ns_tf32_steps", ctypes.c_int32),
                 ("lm_chunk_rows", ctypes.c_int32), ("seed", ctypes.c_uint64), ("short_window", ctypes.c_int32),
-                ("window_pattern", ctypes.c_char * 12), ("residual_extras", ctypes.c_int32)]
+                ("window_pattern", ctypes.c_char * 12), ("residual_extras", ctypes.c_int32),
+                ("ve_gate_channels", ctypes.c_int32)]
 
 
 class HParams(ctypes.Structure):
@@ -114,11 +115,11 @@ def _check(rc):
 
 
 def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0, seed=0,
-                precision=0, window_pattern="", short_window=0, residual_extras=False):
+                precision=0, window_pattern="", short_window=0, residual_extras=False, ve_gate_channels=0):
     return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
                   mlp_mult=4, precision=precision, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows,
                   seed=seed, short_window=short_window, window_pattern=window_pattern.encode("ascii"),
-                  residual_extras=int(bool(residual_extras)))
+                  residual_extras=int(bool(residual_extras)), ve_gate_channels=int(ve_gate_channels))
 
 
 def workspace_size(cfg: Config):
@@ -145,10 +146,11 @@ class GPTStep:
     """
 
     def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0,
-                 seed=0, stream=None, precision=0, window_pattern="", short_window=0, residual_extras=False):
+                 seed=0, stream=None, precision=0, window_pattern="", short_window=0, residual_extras=False,
+                 ve_gate_channels=0):
         import torch
         self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision,
-                               window_pattern, short_window, residual_extras)
+                               window_pattern, short_window, residual_extras, ve_gate_channels)
         self.sizes = workspace_size(self.cfg)
         dev = torch.device("cuda", torch.cuda.current_device())
         self.stream = stream if stream is not None else torch.cuda.current_stream()

@@ -43,6 +43,9 @@ struct Dims {
   char pat[12];
   int extras;   // residual / x0 scales, backout and smear (2L+26 scalars)
   int nsc;      // scalar count rounded up to a multiple of 4
+  int veC, nve, ngp;   // value embeddings: gate width, layers with a table, gate values (padded to 4)
+  // value-embedding slot of layer l, or -1
+  int ve_slot(int l) const { return veC > 0 && l % 2 == 0 ? l / 2 : -1; }
   // attention window of layer l: short_window for an 'S' layer, -1 = full causal
   int window(int l) const { return n_pat > 0 && pat[l % n_pat] == 'S' ? short_window : -1; }
 };
@@ -56,6 +59,8 @@ struct Plan {
   size_t g[6], mom[6], am[2], av[2];
   size_t nv;            // NorMuon second moments: 4 groups x L matrices x d floats
   size_t ws, wsb, gs, ams, avs;   // residual-extras scalars: master, bf16 scratch, grad, AdamW m, v
+  size_t wve, wveb, gve, amve, avve;   // value-embedding tables [nve][V][d]
+  size_t wg, wgb, gg, amg, avg;        // their gates [nve * C][H]
   size_t state_bytes;
   // activations
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
@@ -63,6 +68,7 @@ struct Plan {
   size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
   size_t x0, xin, dx0, dxfin, scws, xe, sig;   // residual extras (allocated only when on)
+  size_t vesig, vedz, vepart;                  // value embeddings (allocated only when on)
   size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
   size_t act_bytes;
   size_t splitk_elems;
@@ -136,6 +142,11 @@ int dims_from(const gpt_config* c, Dims& D) {
   if (c->residual_extras != 0 && c->residual_extras != 1) return fail(GPT_EINVAL, "residual_extras must be 0 or 1");
   D.extras = c->residual_extras;
   D.nsc = (2 * D.L + 26 + 3) / 4 * 4;
+  if (c->ve_gate_channels < 0 || c->ve_gate_channels > std::min(D.d, 128) || c->ve_gate_channels * D.H > 1024)
+    return fail(GPT_EINVAL, "ve_gate_channels must be in [0, min(d_model, 128)] with channels * heads <= 1024");
+  D.veC = c->ve_gate_channels;
+  D.nve = D.veC ? (D.L + 1) / 2 : 0;
+  D.ngp = (D.nve * D.veC * D.H + 3) / 4 * 4;
   return GPT_OK;
 }
 
@@ -148,12 +159,20 @@ void make_plan(const Dims& D, Plan& P) {
   const size_t nsc = D.extras ? static_cast<size_t>(D.nsc) : 0;
   P.ws = pb.take(std::max<size_t>(nsc, 4) * 4);
   P.wsb = pb.take(std::max<size_t>(nsc, 4) * 2);
+  const size_t nvel = static_cast<size_t>(D.nve) * V * d;
+  const size_t ngp = std::max<size_t>(D.ngp, 4);
+  P.wve = pb.take(std::max<size_t>(nvel, 4) * 4);
+  P.wveb = pb.take(std::max<size_t>(nvel, 4) * 2);
+  P.wg = pb.take(ngp * 4);
+  P.wgb = pb.take(ngp * 2);
   P.param_bytes = pb.off;
   Bump sb;
   // gradients: embedding, lm_head, the scalars, then the block matrices (one
   // span; everything before the first block gradient goes to AdamW)
   for (int i = 0; i < 2; ++i) P.g[i] = sb.take(numel[i] * 4);
   P.gs = sb.take(std::max<size_t>(nsc, 4) * 4);
+  P.gve = sb.take(std::max<size_t>(nvel, 4) * 4);
+  P.gg = sb.take(ngp * 4);
   for (int i = 2; i < 6; ++i) P.g[i] = sb.take(numel[i] * 4);
   P.mom[0] = P.mom[1] = 0;
   for (int i = 2; i < 6; ++i) P.mom[i] = sb.take(numel[i] * 4);
@@ -164,6 +183,10 @@ void make_plan(const Dims& D, Plan& P) {
   P.nv = sb.take(4 * L * d * 4);
   P.ams = sb.take(std::max<size_t>(nsc, 4) * 4);
   P.avs = sb.take(std::max<size_t>(nsc, 4) * 4);
+  P.amve = sb.take(std::max<size_t>(nvel, 4) * 4);
+  P.avve = sb.take(std::max<size_t>(nvel, 4) * 4);
+  P.amg = sb.take(ngp * 4);
+  P.avg = sb.take(ngp * 4);
   P.state_bytes = sb.off;
 
   // split-K plan of the lm_head input gradient (contraction over the vocabulary)
@@ -237,6 +260,13 @@ void make_plan(const Dims& D, Plan& P) {
     P.sig = ab.take(M * 4);
   } else {
     P.x0 = P.xin = P.dx0 = P.dxfin = P.scws = P.xe = P.sig = 0;
+  }
+  if (D.nve) {
+    P.vesig = ab.take(static_cast<size_t>(D.nve) * M * H * 4);
+    P.vedz = ab.take(M * H * 4);
+    P.vepart = ab.take(static_cast<size_t>(D.veC) * H * resid_partial_blocks() * 4);
+  } else {
+    P.vesig = P.vedz = P.vepart = 0;
   }
   P.rope = ab.take(static_cast<size_t>(D.T) * 64 * 8 * 2);   // token-major and pair-major
   P.err = ab.take(16);
@@ -333,6 +363,12 @@ struct gpt_ctx {
   float* Mom(int i) const { return reinterpret_cast<float*>(sbuf + P.mom[i]); }
   // residual-extras scalars (fp32, in the parameter buffer)
   float* Scal() const { return reinterpret_cast<float*>(pbuf + P.ws); }
+  // value-embedding table i (fp32 master, bf16 copy, gradient) and gate block i
+  float* VeW(int i) const { return reinterpret_cast<float*>(pbuf + P.wve) + static_cast<size_t>(i) * D.V * D.d; }
+  bf16* VeWb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wveb) + static_cast<size_t>(i) * D.V * D.d; }
+  float* VeG(int i) const { return reinterpret_cast<float*>(sbuf + P.gve) + static_cast<size_t>(i) * D.V * D.d; }
+  float* GateW(int i) const { return reinterpret_cast<float*>(pbuf + P.wg) + static_cast<size_t>(i) * D.veC * D.H; }
+  float* GateG(int i) const { return reinterpret_cast<float*>(sbuf + P.gg) + static_cast<size_t>(i) * D.veC * D.H; }
   // NorMuon second moments of block group i (2..5): L vectors of d floats
   float* NV(int i) const { return reinterpret_cast<float*>(sbuf + P.nv) + static_cast<size_t>(i - 2) * D.L * D.d; }
   template <typename T>
@@ -367,11 +403,26 @@ bool locate(const gpt_ctx* c, int id, int& grp, size_t& off, int& rows, int& col
   if (id == 0) { grp = 0; off = 0; rows = D.V; cols = D.d; return true; }
   if (id == 1) { grp = 1; off = 0; rows = D.d; cols = D.V; return true; }
   const int k = id - 2;
-  if (D.extras && k == 4 * D.L) {   // the residual-extras scalars
-    grp = 6; off = 0; rows = 1; cols = 2 * D.L + 26;
-    return true;
+  if (k >= 4 * D.L) {
+    int x = k - 4 * D.L;
+    if (D.extras) {
+      if (x == 0) {   // the residual-extras scalars
+        grp = 6; off = 0; rows = 1; cols = 2 * D.L + 26;
+        return true;
+      }
+      --x;
+    }
+    if (x < D.nve) {   // value-embedding table x
+      grp = 7; off = static_cast<size_t>(x) * D.V * D.d; rows = D.V; cols = D.d;
+      return true;
+    }
+    if (D.nve && x == D.nve) {   // all gates, stacked
+      grp = 8; off = 0; rows = D.nve * D.veC; cols = D.H;
+      return true;
+    }
+    return false;
   }
-  if (k < 0 || k >= 4 * D.L) return false;
+  if (k < 0) return false;
   const int l = k / 4, j = k % 4;
   const int shp[4][2] = {{D.d, 3 * D.d}, {D.d, D.d}, {D.d, D.F}, {D.F, D.d}};
   grp = 2 + j;
@@ -520,6 +571,14 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.p.f32b = rk + static_cast<size_t>(l) * M * H;
       g.p.rope = rope + static_cast<size_t>(D.T) * 64; g.p.T = D.T; g.p.H = H; g.p.err = err;
       GPT_CK(gemm_run(g, s));
+    }
+    if (D.ve_slot(l) >= 0) {
+      // value embedding: v += 3 sigmoid(gate) ve[tok] per head
+      const int i = D.ve_slot(l);
+      ProfScope ps(c, GPT_PROF_EMBED);
+      launch_ve_fwd(xn1l, tok, c->VeWb(i), c->GateW(i), c->A<float>(P.vesig) + static_cast<size_t>(i) * M * H, vl, M,
+                    D.T, H, D.veC, V, s);
+      c->launches += 1;
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
@@ -687,12 +746,30 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
                     rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s);
     }
     c->launches += 3;
+    const int vs = D.ve_slot(l);
+    if (vs >= 0) {
+      // value embedding: the table's gradient (3 sigmoid dv, scattered by token
+      // through the fp32 buffer the attention backward no longer needs) and
+      // the gate's
+      ProfScope ps(c, GPT_PROF_EMBED);
+      launch_ve_bwd(dv, tok, c->VeWb(vs), c->A<float>(P.vesig) + static_cast<size_t>(vs) * M * H, dqf,
+                    c->A<float>(P.vedz), M, D.T, H, V, s);
+      launch_embed_bwd(tok, dqf, c->VeG(vs), M, d, V, c->A<void>(P.embws), acc, s);
+      launch_ve_gate_grad(xn1 + l * Md, c->A<float>(P.vedz), c->A<float>(P.vepart), c->GateG(vs), M, d, H, D.veC,
+                          acc, s);
+      c->launches += 3 + 2 * ((M + 32767) / 32768);
+    }
     {
       GemmCall g = base_call(M, d, 3 * d);   // dxn1 = dqkv W_qkv^T
       g.A = dqkv; g.lda = 3 * d;
       g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.ldb = 3 * d;
       int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
       if (rc) return rc;
+    }
+    if (vs >= 0) {
+      ProfScope ps(c, GPT_PROF_EMBED);
+      launch_ve_dxn(dxn, c->A<float>(P.vedz), c->GateW(vs), M, d, H, D.veC, s);   // the gate read xn1[:, :C]
+      c->launches += 1;
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
@@ -928,6 +1005,13 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
     init_normal_kernel<<<1024, 256, 0, s>>>(c->W(i), c->Wb(i), static_cast<long long>(numel[i]), cfg->seed, i, 0.02f);
   }
   launch_rope_table(c->A<float2>(c->P.rope), D.T, s);
+  if (D.nve) {
+    // value-embedding tables N(0, 0.02) like the token embedding; gates zero
+    init_normal_kernel<<<1024, 256, 0, s>>>(c->VeW(0), c->VeWb(0), static_cast<long long>(D.nve) * D.V * D.d,
+                                            cfg->seed, 7, 0.02f);
+    if ((e = cudaMemsetAsync(c->pbuf + c->P.wg, 0, static_cast<size_t>(D.ngp) * 4, s)) != cudaSuccess)
+      return bad(e, "zero gates");
+  }
   std::vector<float> sc0;
   if (D.extras) {
     // residual scales 1, x0 and backout scales 0 (and zero padding): the plain network
@@ -1091,6 +1175,17 @@ int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float 
                  bc1, bc2, c->stream);
   }
   c->launches += 2;
+  if (c->D.nve) {
+    // value-embedding tables and their gates
+    launch_adamw(c->VeW(0), c->VeG(0), reinterpret_cast<float*>(c->sbuf + c->P.amve),
+                 reinterpret_cast<float*>(c->sbuf + c->P.avve), c->VeWb(0),
+                 static_cast<long long>(c->D.nve) * c->D.V * c->D.d, lr, beta1, beta2, eps, weight_decay, bc1, bc2,
+                 c->stream);
+    launch_adamw(c->GateW(0), c->GateG(0), reinterpret_cast<float*>(c->sbuf + c->P.amg),
+                 reinterpret_cast<float*>(c->sbuf + c->P.avg), reinterpret_cast<bf16*>(c->pbuf + c->P.wgb), c->D.ngp,
+                 lr, beta1, beta2, eps, weight_decay, bc1, bc2, c->stream);
+    c->launches += 2;
+  }
   if (c->D.extras) {
     // the scalars (zero padding stays zero: zero gradient, zero value)
     launch_adamw(reinterpret_cast<float*>(c->pbuf + c->P.ws), reinterpret_cast<float*>(c->sbuf + c->P.gs),
@@ -1125,7 +1220,9 @@ int gpt_train_step_host(gpt_ctx* c, const int32_t* tokens_host, const int32_t* t
   return gpt_check(c);
 }
 
-int gpt_num_tensors(const gpt_ctx* c) { return c ? 2 + 4 * c->D.L + c->D.extras : 0; }
+int gpt_num_tensors(const gpt_ctx* c) {
+  return c ? 2 + 4 * c->D.L + c->D.extras + (c->D.nve ? c->D.nve + 1 : 0) : 0;
+}
 
 int gpt_tensor_info(const gpt_ctx* c, int id, int32_t* rows, int32_t* cols, int32_t* group) {
   int rc = check_ctx(c);
@@ -1135,7 +1232,7 @@ int gpt_tensor_info(const gpt_ctx* c, int id, int32_t* rows, int32_t* cols, int3
   if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
   if (rows) *rows = r;
   if (cols) *cols = cc;
-  if (group) *group = (grp < 2 || grp == 6) ? GPT_GROUP_ADAMW : GPT_GROUP_MUON;
+  if (group) *group = (grp < 2 || grp >= 6) ? GPT_GROUP_ADAMW : GPT_GROUP_MUON;
   return GPT_OK;
 }
 
@@ -1144,6 +1241,21 @@ static int tensor_ptr(gpt_ctx* c, int id, int kind, float** p, size_t* n, int* g
   size_t off;
   if (!locate(c, id, grp, off, r, cc)) return fail(GPT_EINVAL, "tensor id out of range");
   float* base = nullptr;
+  if (grp == 7 || grp == 8) {
+    const size_t pw = grp == 7 ? c->P.wve : c->P.wg, gw = grp == 7 ? c->P.gve : c->P.gg;
+    const size_t am = grp == 7 ? c->P.amve : c->P.amg, av = grp == 7 ? c->P.avve : c->P.avg;
+    switch (kind) {
+      case GPT_KIND_PARAM: *p = reinterpret_cast<float*>(c->pbuf + pw) + off; break;
+      case GPT_KIND_GRAD: *p = reinterpret_cast<float*>(c->sbuf + gw) + off; break;
+      case GPT_KIND_ADAM_M: *p = reinterpret_cast<float*>(c->sbuf + am) + off; break;
+      case GPT_KIND_ADAM_V: *p = reinterpret_cast<float*>(c->sbuf + av) + off; break;
+      default: return fail(GPT_EINVAL, "value embeddings have a value, a gradient and AdamW moments only");
+    }
+    *n = static_cast<size_t>(r) * cc;
+    *grp_out = grp;
+    *off_out = off;
+    return GPT_OK;
+  }
   if (grp == 6) {
     size_t o;
     switch (kind) {
@@ -1213,8 +1325,9 @@ int gpt_set_tensor(gpt_ctx* c, int id, int kind, const float* src) {
   rc = tensor_ptr(c, id, kind, &p, &n, &grp, &off);
   if (rc) return rc;
   GPT_CK(cudaMemcpyAsync(p, src, n * 4, cudaMemcpyDeviceToDevice, c->stream));
-  if (kind == GPT_KIND_PARAM && grp != 6) {   // the scalars are read in fp32 and have no bf16 copy
-    launch_cast_bf16(p, c->Wb(grp) + off, static_cast<long long>(n), c->stream);
+  if (kind == GPT_KIND_PARAM && (grp < 6 || grp == 7)) {   // scalars and gates are read in fp32
+    launch_cast_bf16(p, grp == 7 ? reinterpret_cast<bf16*>(c->pbuf + c->P.wveb) + off : c->Wb(grp) + off,
+                     static_cast<long long>(n), c->stream);
     c->launches += 1;
   }
   GPT_CK(cudaGetLastError());

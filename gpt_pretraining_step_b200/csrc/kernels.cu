@@ -388,6 +388,102 @@ __global__ void __launch_bounds__(256) smear_bwd_kernel(const float* __restrict_
   }
 }
 
+// Value embeddings (section "1. Modelo GPT", value residual): on a value-
+// embedding layer, v[t, h] += 3 sigmoid(xn1[t, :C] . Wg[:, h]) ve[tok[t], h].
+// v is [B, H, T, 128] bf16 (the attention input), ve the bf16 copy of the
+// layer's [V, d] table, Wg [C, H] fp32.  One warp per token; sig [M, H] is
+// kept for the backward.  Ids outside [0, V) read row 0 (they are latched as
+// errors by the range check).
+__global__ void __launch_bounds__(256) ve_fwd_kernel(const bf16* __restrict__ xn1, const int* __restrict__ tok,
+                                                     const bf16* __restrict__ ve, const float* __restrict__ wg,
+                                                     float* __restrict__ sig, bf16* __restrict__ v, int M, int T,
+                                                     int H, int C, int V) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  const int d = H * 128;
+  const int b = t / T, pos = t - b * T;
+  int id = tok[t];
+  id = static_cast<unsigned>(id) < static_cast<unsigned>(V) ? id : 0;
+  const bf16* xr = xn1 + static_cast<long long>(t) * d;
+  const bf16* er = ve + static_cast<long long>(id) * d;
+  for (int h = 0; h < H; ++h) {
+    float z = 0.f;
+    for (int c = lane; c < C; c += 32) z += __bfloat162float(xr[c]) * wg[c * H + h];
+    z = warp_sum(z);
+    const float sg = 1.f / (1.f + expf(-z));
+    if (lane == 0) sig[static_cast<long long>(t) * H + h] = sg;
+    const float gate = 3.f * sg;
+    bf16* vr = v + ((static_cast<long long>(b) * H + h) * T + pos) * 128 + 4 * lane;
+    const uint2 a = *reinterpret_cast<const uint2*>(vr);
+    const uint2 e = *reinterpret_cast<const uint2*>(er + h * 128 + 4 * lane);
+    uint2 o;
+    o.x = pack_bf16x2(bf16_lo(a.x) + gate * bf16_lo(e.x), bf16_hi(a.x) + gate * bf16_hi(e.x));
+    o.y = pack_bf16x2(bf16_lo(a.y) + gate * bf16_lo(e.y), bf16_hi(a.y) + gate * bf16_hi(e.y));
+    *reinterpret_cast<uint2*>(vr) = o;
+  }
+}
+
+// Backward, given dv [B, H, T, 128] (the gradient at the attention input):
+// dve[t, h] = 3 sig dv[t, h] (fp32 [M, d], scattered into the table's
+// gradient afterwards) and dz[t, h] = (ve[t, h] . dv[t, h]) 3 sig (1 - sig).
+__global__ void __launch_bounds__(256) ve_bwd_kernel(const bf16* __restrict__ dv, const int* __restrict__ tok,
+                                                     const bf16* __restrict__ ve, const float* __restrict__ sig,
+                                                     float* __restrict__ dve, float* __restrict__ dz, int M, int T,
+                                                     int H, int V) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  const int d = H * 128;
+  const int b = t / T, pos = t - b * T;
+  int id = tok[t];
+  id = static_cast<unsigned>(id) < static_cast<unsigned>(V) ? id : 0;
+  const bf16* er = ve + static_cast<long long>(id) * d;
+  for (int h = 0; h < H; ++h) {
+    const uint2 g = *reinterpret_cast<const uint2*>(dv + ((static_cast<long long>(b) * H + h) * T + pos) * 128 +
+                                                    4 * lane);
+    const uint2 e = *reinterpret_cast<const uint2*>(er + h * 128 + 4 * lane);
+    const float g0 = bf16_lo(g.x), g1 = bf16_hi(g.x), g2 = bf16_lo(g.y), g3 = bf16_hi(g.y);
+    float dot = g0 * bf16_lo(e.x) + g1 * bf16_hi(e.x) + g2 * bf16_lo(e.y) + g3 * bf16_hi(e.y);
+    dot = warp_sum(dot);
+    const float sg = sig[static_cast<long long>(t) * H + h];
+    const float gate = 3.f * sg;
+    *reinterpret_cast<float4*>(dve + static_cast<long long>(t) * d + h * 128 + 4 * lane) =
+        make_float4(gate * g0, gate * g1, gate * g2, gate * g3);
+    if (lane == 0) dz[static_cast<long long>(t) * H + h] = dot * 3.f * sg * (1.f - sg);
+  }
+}
+
+// Partial sums of dWg[c, h] = sum_t xn1[t, c] dz[t, h]: block k takes a fixed
+// range of tokens, thread (c, h) its own pair (C * H <= blockDim.x);
+// part[(c * H + h) * gridDim.x + k].
+__global__ void __launch_bounds__(1024) ve_gate_grad_kernel(const bf16* __restrict__ xn1,
+                                                            const float* __restrict__ dz, float* __restrict__ part,
+                                                            int M, int d, int H, int C) {
+  const int pair = threadIdx.x;
+  const int per = (M + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * per, t1 = min(M, t0 + per);
+  if (pair >= C * H) return;
+  const int c = pair / H, h = pair - (pair / H) * H;
+  float s = 0.f;
+  for (int t = t0; t < t1; ++t)
+    s += __bfloat162float(xn1[static_cast<long long>(t) * d + c]) * dz[static_cast<long long>(t) * H + h];
+  part[static_cast<long long>(pair) * gridDim.x + blockIdx.x] = s;
+}
+
+// dxn1[t, c] += sum_h dz[t, h] Wg[c, h] for c < C (the gate reads xn1[:, :C]).
+__global__ void __launch_bounds__(256) ve_dxn_kernel(float* __restrict__ dxn, const float* __restrict__ dz,
+                                                     const float* __restrict__ wg, int M, int d, int H, int C) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= M) return;
+  for (int c = lane; c < C; c += 32) {
+    float s = 0.f;
+    for (int h = 0; h < H; ++h) s += dz[static_cast<long long>(t) * H + h] * wg[c * H + h];
+    dxn[static_cast<long long>(t) * d + c] += s;
+  }
+}
+
 // Scalar gradients from their partial sums (nb per scalar, summed in a fixed
 // order by one warp each): grad[j] (+)= sum_k part[j][k], negated for j =
 // neg_index (the backout scale, whose partials are sums of x_mid . dx).
@@ -1005,6 +1101,26 @@ void launch_scalar_grad_finish(const float* part, int L, float* grad, bool accum
   const int count = 2 * L + 26;
   scalar_grad_finish_kernel<<<cdiv(count, 8), 256, 0, s>>>(part, kResidBlocks, count, 2 * L, grad,
                                                            accumulate ? 1 : 0);
+}
+
+void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float* wg, float* sig, bf16* v, int M,
+                   int T, int H, int C, int V, cudaStream_t s) {
+  ve_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(xn1, tok, ve, wg, sig, v, M, T, H, C, V);
+}
+
+void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
+                   int T, int H, int V, cudaStream_t s) {
+  ve_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dv, tok, ve, sig, dve, dz, M, T, H, V);
+}
+
+void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,
+                         bool accumulate, cudaStream_t s) {
+  ve_gate_grad_kernel<<<kResidBlocks, 1024, 0, s>>>(xn1, dz, part, M, d, H, C);
+  scalar_grad_finish_kernel<<<cdiv(C * H, 8), 256, 0, s>>>(part, kResidBlocks, C * H, -1, grad, accumulate ? 1 : 0);
+}
+
+void launch_ve_dxn(float* dxn, const float* dz, const float* wg, int M, int d, int H, int C, cudaStream_t s) {
+  ve_dxn_kernel<<<cdiv(M, 8), 256, 0, s>>>(dxn, dz, wg, M, d, H, C);
 }
 
 void launch_smear_fwd(const float* e, float* x, float* sig, const float* lam, int L, int T, int M, int d,

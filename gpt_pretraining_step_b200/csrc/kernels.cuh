@@ -98,6 +98,18 @@ void launch_smear_bwd(const float* g, const float* e, const float* sig, const fl
                       int L, int T, int M, int d, cudaStream_t s);
 int resid_partial_blocks();
 
+// Value embeddings: v[t, h] += 3 sigmoid(xn1[t, :C] . wg[:, h]) ve[tok[t], h]
+// (v [B, H, T, 128] bf16, ve the bf16 [V, d] table, wg [C, H]); the backward
+// writes dve (fp32 [M, d], to be scattered into the table's gradient) and dz
+// [M, H]; the gate gradient (C * H <= 1024) and the xn1 gradient correction.
+void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float* wg, float* sig, bf16* v, int M,
+                   int T, int H, int C, int V, cudaStream_t s);
+void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
+                   int T, int H, int V, cudaStream_t s);
+void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,
+                         bool accumulate, cudaStream_t s);
+void launch_ve_dxn(float* dxn, const float* dz, const float* wg, int M, int d, int H, int C, cudaStream_t s);
+
 // Per-tensor e4m3 quantisation of nmat matrices of n bf16 values each (z-th at
 // x + z n): q = e4m3(x * 448 / amax) with round-to-nearest-even and saturation,
 // inv[z] = amax / 448 (1 for an all-zero matrix).  amax_bits: nmat words of scratch.

@@ -114,6 +114,14 @@ typedef struct gpt_config {
                            * 2 + 4*depth, trained by adamw_step, initialised
                            * to resid = 1 and everything else 0 (the plain
                            * network).  0: off. */
+  int32_t ve_gate_channels; /* > 0: value embeddings of section "1. Modelo
+                           * GPT" (value residual) on layers 0, 2, 4, ...:
+                           * v[t, h] += 3 sigmoid(xn1[t, :C] . g[:, h])
+                           * ve[tok[t], head h] with C = ve_gate_channels
+                           * (at most min(d_model, 128), C * heads <= 1024),
+                           * a [vocab, d] table and a [C, heads] gate per such
+                           * layer, trained by adamw_step (tables N(0, 0.02),
+                           * gates 0 at init).  0: off. */
 } gpt_config;
 
 typedef struct gpt_ctx gpt_ctx;
@@ -200,7 +208,10 @@ int gpt_train_step_host(gpt_ctx* ctx, const int32_t* tokens_host, const int32_t*
  * 2 + 4 l + j for block l with j = 0 fused q|k|v [d, 3d], 1 attention output
  * [d, d], 2 MLP up [d, 4d], 3 MLP down [4d, d]; with residual_extras, id
  * 2 + 4 depth = the scalars [1, 2 depth + 26] (resid[0..depth),
- * x0s[0..depth), backout, smear, smear gate weights[24]). */
+ * x0s[0..depth), backout, smear, smear gate weights[24]); with value
+ * embeddings, the next ceil(depth / 2) ids are their tables [vocab, d] (layers
+ * 0, 2, ...) and the one after them all gates [n * C, heads] (layer 2i's
+ * gate in rows i*C .. i*C+C-1). */
 int gpt_num_tensors(const gpt_ctx* ctx);
 int gpt_tensor_info(const gpt_ctx* ctx, int id, int32_t* rows, int32_t* cols, int32_t* group);
 

@@ -64,7 +64,8 @@ def test_workspace_size_valid_configs(L):
 @pytest.mark.parametrize("bad", [dict(depth=0), dict(d_model=100), dict(vocab=1001), dict(batch=0),
                                  dict(seq_len=0), dict(vocab=4), dict(window_pattern="SXL", short_window=8),
                                  dict(window_pattern="SSSL", short_window=-1),
-                                 dict(window_pattern="SSSLSSSLSSSL", short_window=8)])
+                                 dict(window_pattern="SSSLSSSLSSSL", short_window=8), dict(ve_gate_channels=-1),
+                                 dict(ve_gate_channels=129)])
 def test_workspace_size_rejects_bad_config(L, bad):
     import gpt_pretraining_step_b200 as g
     with pytest.raises(g.GptError) as e:

@@ -163,6 +163,68 @@ def test_residual_extras_match_oracle(torch, name):
     assert np.abs(f64(st.get(sid, g.KIND_PARAM)) - p_ref).max() < 1e-6
 
 
+VE_C = 16
+
+
+def _build_ve(torch, s, params, extras=False):
+    import gpt_pretraining_step_b200 as g
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   residual_extras=extras, ve_gate_channels=VE_C)
+    for tid, (name, *_rest) in enumerate(syn.param_specs(s, extras=extras, ve_channels=VE_C)):
+        st.set(tid, params[name])
+    return st
+
+
+def test_zero_value_embeddings_are_bit_identical_to_plain(torch):
+    import gpt_pretraining_step_b200 as g
+    s = SMALL["ragged"]
+    params = syn.init_params(s, seed=51, ve_channels=VE_C)
+    for l in syn.ve_layers(s.depth):
+        params[f"ve{l}"] = np.zeros_like(params[f"ve{l}"])
+    params["ve_gate"] = syn.gaussian(params["ve_gate"].shape, seed=52)
+    tok, tgt = torch.tensor(syn.tokens(s, seed=53)).cuda(), torch.tensor(syn.targets(s, seed=54)).cuda()
+    plain = build(torch, s, params)
+    ve = _build_ve(torch, s, params)
+    assert ve.num_tensors() == plain.num_tensors() + len(syn.ve_layers(s.depth)) + 1
+    la = float(plain.fwd_bwd(tok, tgt).item())
+    lb = float(ve.fwd_bwd(tok, tgt).item())
+    plain.check()
+    ve.check()
+    assert la == lb
+    for tid in range(plain.num_tensors()):
+        assert torch.equal(plain.get(tid, g.KIND_GRAD), ve.get(tid, g.KIND_GRAD)), tid
+
+
+@pytest.mark.parametrize("name,extras", [("tiny", False), ("ragged", False), ("ragged", True)])
+def test_value_embeddings_match_oracle(torch, name, extras):
+    """Random tables and gates (with and without the residual extras): loss,
+    every gradient (tables and gates included), and the gates' AdamW step."""
+    import gpt_pretraining_step_b200 as g
+    s = SMALL[name]
+    params = syn.init_params(s, seed=55, extras=extras, ve_channels=VE_C)
+    params["ve_gate"] = syn.gaussian(params["ve_gate"].shape, seed=56, std=2.0)
+    if extras:
+        params["scalars"] = syn.random_scalars(s, seed=57)
+    tok, tgt = syn.tokens(s, seed=58), syn.targets(s, seed=59)
+    st = _build_ve(torch, s, params, extras)
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL
+    assert np.abs(f64(st.row_loss()).ravel() - cache["row_loss"]).max() < 2e-2
+    specs = syn.param_specs(s, extras=extras, ve_channels=VE_C)
+    for tid, (pname, *_r) in enumerate(specs):
+        c = cosine(f64(st.get(tid, g.KIND_GRAD)), grads[pname])
+        assert c >= GRAD_COS, (pname, c)
+    gid = len(specs) - 1
+    gg = f64(st.get(gid, g.KIND_GRAD))
+    st.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.0)
+    st.check()
+    p_ref, _, _ = oo.adamw_step(params["ve_gate"].astype(np.float64), gg, np.zeros_like(gg), np.zeros_like(gg), 1,
+                                3e-3, 0.8, 0.95, 1e-10, 0.0)
+    assert np.abs(f64(st.get(gid, g.KIND_PARAM)) - p_ref).max() < 1e-6
+
+
 def test_embedding_and_target_indexing_exact(torch):
     # with a zero lm_head the logits vanish: loss = ln V exactly, and dW_lm has
     # one shared column for every vocabulary id that is not a target, so the set
