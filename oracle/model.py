@@ -18,7 +18,9 @@ Readings where the pages are silent (shared with the CUDA path):
     within the row.
   * QK norm: per-head gain-free RMSNorm applied after RoPE (the order does
     not matter mathematically: a rotation keeps the RMS).
-  * attention scale 1/sqrt(hd); n_kv_head = n_head.
+  * attention scale 1/sqrt(hd); grouped kv heads when the fused projection
+    is narrower than 3d: its columns are q (d) | k | v (Hkv * hd each), and
+    query head h reads kv head h // (H / Hkv).
   * residual extras ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section
     "1. Modelo GPT", efficiency tricks 1, 2 and 3), present when params holds
     a "scalars" vector [2L + 26] = (resid lambdas [L], x0 lambdas [L],
@@ -32,10 +34,11 @@ Readings where the pages are silent (shared with the CUDA path):
     Initial values resid 1 and everything else 0 make the network the plain
     one.
   * value embeddings (section "1. Modelo GPT", value residual), present when
-    params holds "ve{l}" tables [V, d] for the layers l with l % 2 == 0 and
-    "ve_gate" [C, H] (one block of C rows per such layer, stacked
-    [n_ve * C, H]): v[t, h] += 3 sigmoid(xn1[t, :C] . ve_gate_l[:, h])
-    ve_l[tok[t], h*hd:(h+1)*hd], xn1 being the block's attention input.
+    params holds "ve{l}" tables [V, Hkv hd] for the layers l with l % 2 == 0
+    and "ve_gate" [C, Hkv] (one block of C rows per such layer, stacked
+    [n_ve * C, Hkv]): v[t, h] += 3 sigmoid(xn1[t, :C] . ve_gate_l[:, h])
+    ve_l[tok[t], h*hd:(h+1)*hd] for every kv head h, xn1 being the block's
+    attention input.
   * attention window per layer: full causal by default; with a layer pattern
     such as "SSSL" (section "1. Modelo GPT", sliding-window attention) the
     pattern is repeated over the layers, S = a sliding window of
@@ -232,16 +235,19 @@ def forward(params, tok, tgt, n_layer, head_dim=128, keep=True, windows=None):
         a = {}
         xn1, r1 = rms_norm(x)
         qkv = xn1 @ W["c_qkv"]
+        # q | k | v columns; k and v have Hkv = (cols - d) / (2 hd) heads
+        kvd = (qkv.shape[1] - d) // 2
+        Hkv = kvd // head_dim
         q = _split_heads(qkv[:, :d], B, T, H, head_dim)
-        k = _split_heads(qkv[:, d:2 * d], B, T, H, head_dim)
-        v = _split_heads(qkv[:, 2 * d:], B, T, H, head_dim)
+        k = _split_heads(qkv[:, d:d + kvd], B, T, Hkv, head_dim)
+        v = _split_heads(qkv[:, d + kvd:], B, T, Hkv, head_dim)
         if f"ve{l}" in params:
             # value residual: v + 3 sigmoid(gate) * ve, per head
             C = params["ve_gate"].shape[0] // ve_layer_count(n_layer)
             Wg = np.asarray(params["ve_gate"], dtype=np.float64)[(l // 2) * C:(l // 2 + 1) * C]
             ve = np.asarray(params[f"ve{l}"], dtype=np.float64)[tok.reshape(-1)]      # [M, d]
             sg = 1.0 / (1.0 + np.exp(-(xn1[:, :C] @ Wg)))                           # [M, H]
-            v = v + _split_heads(np.repeat(3.0 * sg, head_dim, axis=1) * ve, B, T, H, head_dim)
+            v = v + _split_heads(np.repeat(3.0 * sg, head_dim, axis=1) * ve, B, T, Hkv, head_dim)
             if keep:
                 a.update(ve=ve, ve_sig=sg, ve_C=C)
         qn, rq = rms_norm(rope(q, cos, sin))
@@ -317,7 +323,7 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
             gve = np.zeros_like(np.asarray(params[f"ve{l}"], dtype=np.float64))
             np.add.at(gve, tok.reshape(-1), dve)
             grads[f"ve{l}"] = gve
-            dgate = (ve * dvm).reshape(-1, H, head_dim).sum(axis=-1)                # [M, H]
+            dgate = (ve * dvm).reshape(-1, dvm.shape[1] // head_dim, head_dim).sum(axis=-1)   # [M, Hkv]
             dz = dgate * 3.0 * sg * (1.0 - sg)
             Wg = np.asarray(params["ve_gate"], dtype=np.float64)[(l // 2) * C:(l // 2 + 1) * C]
             if "ve_gate" not in grads:

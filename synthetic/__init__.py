@@ -33,21 +33,33 @@ class Shape:
     vocab: int
     batch: int
     seq_len: int
+    n_kv_head: int = 0   # 0: as many kv heads as query heads
 
     @property
     def tokens(self) -> int:
         return self.batch * self.seq_len
 
+    @property
+    def kv_heads(self) -> int:
+        return self.n_kv_head or self.n_head
+
+    @property
+    def qkv_cols(self) -> int:
+        """Width of the fused projection: q (d) | k | v (kv_heads * head_dim each)."""
+        return self.d_model + 2 * self.kv_heads * self.head_dim
+
 
 def make_shape(depth: int, batch: int, seq_len: int, vocab: int = VOCAB,
                d_model: int = 0, head_dim: int = HEAD_DIM,
-               mlp_mult: int = MLP_MULT) -> Shape:
+               mlp_mult: int = MLP_MULT, n_kv_head: int = 0) -> Shape:
     """Derive every width from ``depth`` (``d_model`` may override 64*depth)."""
     d = d_model if d_model else 64 * depth
     if d % head_dim:
         raise ValueError(f"d_model {d} is not a multiple of head_dim {head_dim}")
+    if n_kv_head and (d // head_dim) % n_kv_head:
+        raise ValueError(f"{n_kv_head} kv heads do not divide {d // head_dim} query heads")
     return Shape(depth=depth, d_model=d, n_head=d // head_dim, head_dim=head_dim,
-                 mlp_hidden=mlp_mult * d, vocab=vocab, batch=batch, seq_len=seq_len)
+                 mlp_hidden=mlp_mult * d, vocab=vocab, batch=batch, seq_len=seq_len, n_kv_head=n_kv_head)
 
 
 # The workloads, named by what they are.
@@ -79,7 +91,7 @@ def param_specs(s: Shape, extras: bool = False, ve_channels: int = 0):
     d, f = s.d_model, s.mlp_hidden
     out = [("wte", s.vocab, d, "adamw"), ("lm_head", d, s.vocab, "adamw")]
     for layer in range(s.depth):
-        out += [(f"h{layer}.c_qkv", d, 3 * d, "muon"),
+        out += [(f"h{layer}.c_qkv", d, s.qkv_cols, "muon"),
                 (f"h{layer}.c_proj", d, d, "muon"),
                 (f"h{layer}.c_fc", d, f, "muon"),
                 (f"h{layer}.mlp_proj", f, d, "muon")]
@@ -89,8 +101,9 @@ def param_specs(s: Shape, extras: bool = False, ve_channels: int = 0):
         out.append(("scalars", 1, 2 * s.depth + 26, "adamw"))
     if ve_channels:
         # value embedding tables, then the gates of all of them stacked
-        out += [(f"ve{l}", s.vocab, d, "adamw") for l in ve_layers(s.depth)]
-        out.append(("ve_gate", ve_channels * len(ve_layers(s.depth)), s.n_head, "adamw"))
+        kvd = s.kv_heads * s.head_dim
+        out += [(f"ve{l}", s.vocab, kvd, "adamw") for l in ve_layers(s.depth)]
+        out.append(("ve_gate", ve_channels * len(ve_layers(s.depth)), s.kv_heads, "adamw"))
     return out
 
 
@@ -125,9 +138,9 @@ def init_params(s: Shape, seed: int = 0, std: float = 0.02, extras: bool = False
         # value embedding tables N(0, std) like the token embedding; gates zero
         # (every gate then starts at 3 sigmoid(0) = 1.5)
         for l in ve_layers(s.depth):
-            params[f"ve{l}"] = round_to_bf16(rng.standard_normal((s.vocab, s.d_model), dtype=np.float32)
-                                             * np.float32(std))
-        params["ve_gate"] = np.zeros((ve_channels * len(ve_layers(s.depth)), s.n_head), dtype=np.float32)
+            params[f"ve{l}"] = round_to_bf16(rng.standard_normal((s.vocab, s.kv_heads * s.head_dim),
+                                                                 dtype=np.float32) * np.float32(std))
+        params["ve_gate"] = np.zeros((ve_channels * len(ve_layers(s.depth)), s.kv_heads), dtype=np.float32)
     return params
 
 

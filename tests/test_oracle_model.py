@@ -458,3 +458,31 @@ def test_finite_difference_with_value_embeddings():
     s, p, tok, tgt = _ve_case(depth=2, C=8, seed=5, d=256, vocab=32, seq=8)
     names = ["ve0", "ve_gate", "h0.c_qkv", "h1.c_qkv", "wte"]
     _fd_check(p, tok, tgt, s.depth, names, n_coords=6)
+
+
+# --- grouped kv heads in the model -------------------------------------------
+
+def test_gqa_model_equals_mha_with_repeated_kv_columns():
+    # a q|k|v projection with Hkv kv heads gives the same loss as the full one
+    # whose k and v columns repeat each kv head for its group of query heads
+    s = syn.make_shape(depth=2, d_model=512, vocab=40, batch=2, seq_len=9, n_kv_head=2)
+    p = syn.init_params(s, seed=3, std=0.05)
+    p = {k: v.astype(np.float64) for k, v in p.items()}
+    tok, tgt = syn.tokens(s, seed=4), syn.targets(s, seed=5)
+    d, kvd, hd = 512, 256, 128
+    full = dict(p)
+    for l in range(2):
+        W = p[f"h{l}.c_qkv"]
+        assert W.shape == (d, d + 2 * kvd)
+        rep = lambda blk: np.concatenate([blk[:, (h // 2) * hd:(h // 2 + 1) * hd] for h in range(4)], axis=1)
+        full[f"h{l}.c_qkv"] = np.concatenate([W[:, :d], rep(W[:, d:d + kvd]), rep(W[:, d + kvd:])], axis=1)
+    l_gqa, _ = om.forward(p, tok, tgt, 2, keep=False)
+    l_mha, _ = om.forward(full, tok, tgt, 2, keep=False)
+    assert abs(l_gqa - l_mha) < 1e-12
+
+
+def test_finite_difference_gqa_model():
+    s = syn.make_shape(depth=1, d_model=512, vocab=32, batch=1, seq_len=8, n_kv_head=2)
+    p = {k: v.astype(np.float64) for k, v in syn.init_params(s, seed=6, std=0.05).items()}
+    tok, tgt = syn.tokens(s, seed=7), syn.targets(s, seed=8)
+    _fd_check(p, tok, tgt, 1, ["h0.c_qkv", "h0.c_proj", "wte"], n_coords=6)
