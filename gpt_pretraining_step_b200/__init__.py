@@ -43,7 +43,7 @@ class Config(ctypes.Structure):
                 ("mlp_mult", ctypes.c_int32), ("precision", ctypes.c_int32), ("ns_tf32_steps", ctypes.c_int32),
                 ("lm_chunk_rows", ctypes.c_int32), ("seed", ctypes.c_uint64), ("short_window", ctypes.c_int32),
                 ("window_pattern", ctypes.c_char * 12), ("residual_extras", ctypes.c_int32),
-                ("ve_gate_channels", ctypes.c_int32)]
+                ("ve_gate_channels", ctypes.c_int32), ("n_kv_head", ctypes.c_int32)]
 
 
 class HParams(ctypes.Structure):
@@ -115,11 +115,13 @@ def _check(rc):
 
 
 def make_config(depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0, seed=0,
-                precision=0, window_pattern="", short_window=0, residual_extras=False, ve_gate_channels=0):
+                precision=0, window_pattern="", short_window=0, residual_extras=False, ve_gate_channels=0,
+                n_kv_head=0):
     return Config(depth=depth, d_model=d_model, vocab=vocab, batch=batch, seq_len=seq_len, head_dim=128,
                   mlp_mult=4, precision=precision, ns_tf32_steps=ns_tf32_steps, lm_chunk_rows=lm_chunk_rows,
                   seed=seed, short_window=short_window, window_pattern=window_pattern.encode("ascii"),
-                  residual_extras=int(bool(residual_extras)), ve_gate_channels=int(ve_gate_channels))
+                  residual_extras=int(bool(residual_extras)), ve_gate_channels=int(ve_gate_channels),
+                  n_kv_head=int(n_kv_head))
 
 
 def workspace_size(cfg: Config):
@@ -147,10 +149,10 @@ class GPTStep:
 
     def __init__(self, depth, batch, seq_len, vocab=32768, d_model=0, ns_tf32_steps=-1, lm_chunk_rows=0,
                  seed=0, stream=None, precision=0, window_pattern="", short_window=0, residual_extras=False,
-                 ve_gate_channels=0):
+                 ve_gate_channels=0, n_kv_head=0):
         import torch
         self.cfg = make_config(depth, batch, seq_len, vocab, d_model, ns_tf32_steps, lm_chunk_rows, seed, precision,
-                               window_pattern, short_window, residual_extras, ve_gate_channels)
+                               window_pattern, short_window, residual_extras, ve_gate_channels, n_kv_head)
         self.sizes = workspace_size(self.cfg)
         dev = torch.device("cuda", torch.cuda.current_device())
         self.stream = stream if stream is not None else torch.cuda.current_stream()

@@ -39,6 +39,7 @@ constexpr size_t kAlign = 256;
 
 struct Dims {
   int L, d, H, F, V, B, T, M, Mc, tiles_lm, n_tf32, fp8;
+  int Hkv, qc;   // kv heads; columns of the fused projection: d + 2 * 128 * Hkv
   int short_window, n_pat;
   char pat[12];
   int extras;   // residual / x0 scales, backout and smear (2L+26 scalars)
@@ -144,22 +145,28 @@ int dims_from(const gpt_config* c, Dims& D) {
   D.nsc = (2 * D.L + 26 + 3) / 4 * 4;
   if (c->ve_gate_channels < 0 || c->ve_gate_channels > std::min(D.d, 128) || c->ve_gate_channels * D.H > 1024)
     return fail(GPT_EINVAL, "ve_gate_channels must be in [0, min(d_model, 128)] with channels * heads <= 1024");
+  if (c->n_kv_head < 0 || (c->n_kv_head > 0 && D.H % c->n_kv_head))
+    return fail(GPT_EINVAL, "n_kv_head must divide the number of heads (0: as many as the heads)");
+  D.Hkv = c->n_kv_head ? c->n_kv_head : D.H;
+  D.qc = D.d + 2 * 128 * D.Hkv;
+  if (c->ve_gate_channels * D.Hkv > 1024) return fail(GPT_EINVAL, "ve_gate_channels * kv heads must be <= 1024");
   D.veC = c->ve_gate_channels;
   D.nve = D.veC ? (D.L + 1) / 2 : 0;
-  D.ngp = (D.nve * D.veC * D.H + 3) / 4 * 4;
+  D.ngp = (D.nve * D.veC * D.Hkv + 3) / 4 * 4;
   return GPT_OK;
 }
 
 void make_plan(const Dims& D, Plan& P) {
   const size_t L = D.L, d = D.d, F = D.F, V = D.V, M = D.M, H = D.H;
-  const size_t numel[6] = {V * d, d * V, L * d * 3 * d, L * d * d, L * d * F, L * F * d};
+  const size_t qc = D.qc, kvd = 128 * static_cast<size_t>(D.Hkv);
+  const size_t numel[6] = {V * d, d * V, L * d * qc, L * d * d, L * d * F, L * F * d};
   Bump pb;
   for (int i = 0; i < 6; ++i) P.w[i] = pb.take(numel[i] * 4);
   for (int i = 0; i < 6; ++i) P.wb[i] = pb.take(numel[i] * 2);
   const size_t nsc = D.extras ? static_cast<size_t>(D.nsc) : 0;
   P.ws = pb.take(std::max<size_t>(nsc, 4) * 4);
   P.wsb = pb.take(std::max<size_t>(nsc, 4) * 2);
-  const size_t nvel = static_cast<size_t>(D.nve) * V * d;
+  const size_t nvel = static_cast<size_t>(D.nve) * V * kvd;
   const size_t ngp = std::max<size_t>(D.ngp, 4);
   P.wve = pb.take(std::max<size_t>(nvel, 4) * 4);
   P.wveb = pb.take(std::max<size_t>(nvel, 4) * 2);
@@ -232,10 +239,10 @@ void make_plan(const Dims& D, Plan& P) {
   P.dk = ab.take(M * d * 2);
   P.dv = ab.take(M * d * 2);
   P.Dv = ab.take(M * H * 4);
-  P.dqkv = ab.take(L * M * 3 * d * 2);
+  P.dqkv = ab.take(L * M * qc * 2);
   P.splitk = ab.take(std::max<size_t>(sk, 4) * 4);
   P.embws = ab.take(embed_bwd_workspace(D.M));
-  const size_t xelems = std::max({L * d * 3 * d, L * d * d, 2 * L * d * F});
+  const size_t xelems = std::max({L * d * qc, L * d * d, 2 * L * d * F});
   P.X0 = ab.take(xelems * 4);
   P.X1 = ab.take(xelems * 4);
   // fp16 operand copies of the Newton-Schulz iterates (fp16 mode), or the
@@ -262,9 +269,9 @@ void make_plan(const Dims& D, Plan& P) {
     P.x0 = P.xin = P.dx0 = P.dxfin = P.scws = P.xe = P.sig = 0;
   }
   if (D.nve) {
-    P.vesig = ab.take(static_cast<size_t>(D.nve) * M * H * 4);
-    P.vedz = ab.take(M * H * 4);
-    P.vepart = ab.take(static_cast<size_t>(D.veC) * H * resid_partial_blocks() * 4);
+    P.vesig = ab.take(static_cast<size_t>(D.nve) * M * D.Hkv * 4);
+    P.vedz = ab.take(M * D.Hkv * 4);
+    P.vepart = ab.take(static_cast<size_t>(D.veC) * D.Hkv * resid_partial_blocks() * 4);
   } else {
     P.vesig = P.vedz = P.vepart = 0;
   }
@@ -275,7 +282,7 @@ void make_plan(const Dims& D, Plan& P) {
   {
     // fp8 e4m3 copies of the block weights and one activation operand, with their scales
     const bool f8 = D.fp8 != 0;
-    const size_t wn[4] = {L * d * 3 * d, L * d * d, L * d * F, L * F * d};
+    const size_t wn[4] = {L * d * qc, L * d * d, L * d * F, L * F * d};
     for (int i = 0; i < 4; ++i) P.wq8[i] = ab.take(f8 ? wn[i] : 16);
     P.winv = ab.take(4 * L * 4);
     P.wamax = ab.take(4 * L * 4);
@@ -364,11 +371,12 @@ struct gpt_ctx {
   // residual-extras scalars (fp32, in the parameter buffer)
   float* Scal() const { return reinterpret_cast<float*>(pbuf + P.ws); }
   // value-embedding table i (fp32 master, bf16 copy, gradient) and gate block i
-  float* VeW(int i) const { return reinterpret_cast<float*>(pbuf + P.wve) + static_cast<size_t>(i) * D.V * D.d; }
-  bf16* VeWb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wveb) + static_cast<size_t>(i) * D.V * D.d; }
-  float* VeG(int i) const { return reinterpret_cast<float*>(sbuf + P.gve) + static_cast<size_t>(i) * D.V * D.d; }
-  float* GateW(int i) const { return reinterpret_cast<float*>(pbuf + P.wg) + static_cast<size_t>(i) * D.veC * D.H; }
-  float* GateG(int i) const { return reinterpret_cast<float*>(sbuf + P.gg) + static_cast<size_t>(i) * D.veC * D.H; }
+  size_t ve_elems() const { return static_cast<size_t>(D.V) * 128 * D.Hkv; }   // one table [V, 128 Hkv]
+  float* VeW(int i) const { return reinterpret_cast<float*>(pbuf + P.wve) + i * ve_elems(); }
+  bf16* VeWb(int i) const { return reinterpret_cast<bf16*>(pbuf + P.wveb) + i * ve_elems(); }
+  float* VeG(int i) const { return reinterpret_cast<float*>(sbuf + P.gve) + i * ve_elems(); }
+  float* GateW(int i) const { return reinterpret_cast<float*>(pbuf + P.wg) + static_cast<size_t>(i) * D.veC * D.Hkv; }
+  float* GateG(int i) const { return reinterpret_cast<float*>(sbuf + P.gg) + static_cast<size_t>(i) * D.veC * D.Hkv; }
   // NorMuon second moments of block group i (2..5): L vectors of d floats
   float* NV(int i) const { return reinterpret_cast<float*>(sbuf + P.nv) + static_cast<size_t>(i - 2) * D.L * D.d; }
   template <typename T>
@@ -413,18 +421,18 @@ bool locate(const gpt_ctx* c, int id, int& grp, size_t& off, int& rows, int& col
       --x;
     }
     if (x < D.nve) {   // value-embedding table x
-      grp = 7; off = static_cast<size_t>(x) * D.V * D.d; rows = D.V; cols = D.d;
+      grp = 7; off = static_cast<size_t>(x) * D.V * 128 * D.Hkv; rows = D.V; cols = 128 * D.Hkv;
       return true;
     }
     if (D.nve && x == D.nve) {   // all gates, stacked
-      grp = 8; off = 0; rows = D.nve * D.veC; cols = D.H;
+      grp = 8; off = 0; rows = D.nve * D.veC; cols = D.Hkv;
       return true;
     }
     return false;
   }
   if (k < 0) return false;
   const int l = k / 4, j = k % 4;
-  const int shp[4][2] = {{D.d, 3 * D.d}, {D.d, D.d}, {D.d, D.F}, {D.F, D.d}};
+  const int shp[4][2] = {{D.d, D.qc}, {D.d, D.d}, {D.d, D.F}, {D.F, D.d}};
   grp = 2 + j;
   rows = shp[j][0];
   cols = shp[j][1];
@@ -514,7 +522,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   float* winv = c->A<float>(P.winv);
   if (D.fp8) {
     ProfScope ps(c, GPT_PROF_FP8_QUANT);
-    const long long wn[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+    const long long wn[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
     for (int gi = 0; gi < 4; ++gi)
       launch_quantize_e4m3(c->Wb(2 + gi), wn[gi], L, c->A<unsigned int>(P.wamax) + gi * L,
                            c->A<uint8_t>(P.wq8[gi]), winv + gi * L, s);
@@ -533,7 +541,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     g.es = 1;
     g.A = act8;
-    const long long wn[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+    const long long wn[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
     g.B = c->A<uint8_t>(P.wq8[grp - 2]) + static_cast<size_t>(l) * wn[grp - 2];
     g.p.dq_a = act_inv;
     g.p.dq_b = winv + (grp - 2) * L + l;
@@ -561,28 +569,28 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
     }
     {
-      GemmCall g = base_call(M, 3 * d, d);
-      g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.b_mn = true; g.ldb = 3 * d;
+      GemmCall g = base_call(M, D.qc, d);
+      g.B = c->Wb(2) + static_cast<size_t>(l) * d * D.qc; g.b_mn = true; g.ldb = D.qc;
       fwd_a(g, xn1l, M, d, 2, l); g.lda = d;
       ProfScope ps(c, GPT_PROF_QKV_GEMM);
       g.bn = 256; g.epi = EPI_QKV; g.out_es = 2; g.aux_es = 2;
       g.p.qkv_out[0] = ql; g.p.qkv_out[1] = kl; g.p.qkv_out[2] = vl;
       g.p.f32a = rq + static_cast<size_t>(l) * M * H;
       g.p.f32b = rk + static_cast<size_t>(l) * M * H;
-      g.p.rope = rope + static_cast<size_t>(D.T) * 64; g.p.T = D.T; g.p.H = H; g.p.err = err;
+      g.p.rope = rope + static_cast<size_t>(D.T) * 64; g.p.T = D.T; g.p.H = H; g.p.Hkv = D.Hkv; g.p.err = err;
       GPT_CK(gemm_run(g, s));
     }
     if (D.ve_slot(l) >= 0) {
       // value embedding: v += 3 sigmoid(gate) ve[tok] per head
       const int i = D.ve_slot(l);
       ProfScope ps(c, GPT_PROF_EMBED);
-      launch_ve_fwd(xn1l, tok, c->VeWb(i), c->GateW(i), c->A<float>(P.vesig) + static_cast<size_t>(i) * M * H, vl, M,
-                    D.T, H, D.veC, V, s);
+      launch_ve_fwd(xn1l, tok, c->VeWb(i), c->GateW(i), c->A<float>(P.vesig) + static_cast<size_t>(i) * M * D.Hkv, vl,
+                    M, D.T, H, D.Hkv, D.veC, V, s);
       c->launches += 1;
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
-      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, H, D.window(l), c->A<int>(P.sched));
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H);
     }
     {
       GemmCall g = base_call(M, d, d);
@@ -700,7 +708,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     bf16* hl = h + static_cast<size_t>(l) * M * F;
     bf16* ol = o + l * Md;
     bf16* du = du_all + static_cast<size_t>(l) * M * F;
-    bf16* dqkv = dqkv_all + static_cast<size_t>(l) * M * 3 * d;
+    bf16* dqkv = dqkv_all + static_cast<size_t>(l) * M * D.qc;
     // MLP down: dh = dx W_d^T, du = dh * 2 relu(u) with relu(u) = sqrt(h)
     {
       ProfScope ps(c, GPT_PROF_DX_GEMM);
@@ -738,12 +746,12 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, H, D.window(l), c->A<int>(P.sched));
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H);
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
       launch_qk_bwd(dqf, dk, dv, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
-                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s);
+                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv);
     }
     c->launches += 3;
     const int vs = D.ve_slot(l);
@@ -752,23 +760,23 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       // through the fp32 buffer the attention backward no longer needs) and
       // the gate's
       ProfScope ps(c, GPT_PROF_EMBED);
-      launch_ve_bwd(dv, tok, c->VeWb(vs), c->A<float>(P.vesig) + static_cast<size_t>(vs) * M * H, dqf,
-                    c->A<float>(P.vedz), M, D.T, H, V, s);
-      launch_embed_bwd(tok, dqf, c->VeG(vs), M, d, V, c->A<void>(P.embws), acc, s);
-      launch_ve_gate_grad(xn1 + l * Md, c->A<float>(P.vedz), c->A<float>(P.vepart), c->GateG(vs), M, d, H, D.veC,
-                          acc, s);
+      launch_ve_bwd(dv, tok, c->VeWb(vs), c->A<float>(P.vesig) + static_cast<size_t>(vs) * M * D.Hkv, dqf,
+                    c->A<float>(P.vedz), M, D.T, H, D.Hkv, V, s);
+      launch_embed_bwd(tok, dqf, c->VeG(vs), M, 128 * D.Hkv, V, c->A<void>(P.embws), acc, s);
+      launch_ve_gate_grad(xn1 + l * Md, c->A<float>(P.vedz), c->A<float>(P.vepart), c->GateG(vs), M, d, D.Hkv,
+                          D.veC, acc, s);
       c->launches += 3 + 2 * ((M + 32767) / 32768);
     }
     {
-      GemmCall g = base_call(M, d, 3 * d);   // dxn1 = dqkv W_qkv^T
-      g.A = dqkv; g.lda = 3 * d;
-      g.B = c->Wb(2) + static_cast<size_t>(l) * d * 3 * d; g.ldb = 3 * d;
+      GemmCall g = base_call(M, d, D.qc);   // dxn1 = dqkv W_qkv^T
+      g.A = dqkv; g.lda = D.qc;
+      g.B = c->Wb(2) + static_cast<size_t>(l) * d * D.qc; g.ldb = D.qc;
       int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
       if (rc) return rc;
     }
     if (vs >= 0) {
       ProfScope ps(c, GPT_PROF_EMBED);
-      launch_ve_dxn(dxn, c->A<float>(P.vedz), c->GateW(vs), M, d, H, D.veC, s);   // the gate read xn1[:, :C]
+      launch_ve_dxn(dxn, c->A<float>(P.vedz), c->GateW(vs), M, d, D.Hkv, D.veC, s);   // the gate read xn1[:, :C]
       c->launches += 1;
     }
     {
@@ -795,7 +803,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     ProfScope ps(c, GPT_PROF_DW_GEMM);
     struct DW { const bf16* a; long long lda, a_bs; const bf16* b; long long ldb, b_bs; int rows, cols; float* out; };
     const DW dws[4] = {
-        {xn1, d, static_cast<long long>(Md), dqkv_all, 3ll * d, 3ll * Md, d, 3 * d, c->G(2)},
+        {xn1, d, static_cast<long long>(Md), dqkv_all, D.qc, 1ll * M * D.qc, d, D.qc, c->G(2)},
         {o, d, static_cast<long long>(Md), gx, d, 2ll * Md, d, d, c->G(3)},
         {xn2, d, static_cast<long long>(Md), du_all, F, 1ll * M * F, d, F, c->G(4)},
         {h, F, 1ll * M * F, gx + Md, d, 2ll * Md, F, d, c->G(5)},
@@ -999,7 +1007,7 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
   if ((e = cudaMemsetAsync(c->sbuf, 0, c->P.state_bytes, s)) != cudaSuccess) return bad(e, "zero state");
   if ((e = cudaMemsetAsync(c->A<int>(c->P.err), 0, 16, s)) != cudaSuccess) return bad(e, "zero error word");
   const size_t numel[6] = {static_cast<size_t>(D.V) * D.d, static_cast<size_t>(D.d) * D.V,
-                           static_cast<size_t>(D.L) * D.d * 3 * D.d, static_cast<size_t>(D.L) * D.d * D.d,
+                           static_cast<size_t>(D.L) * D.d * D.qc, static_cast<size_t>(D.L) * D.d * D.d,
                            static_cast<size_t>(D.L) * D.d * D.F, static_cast<size_t>(D.L) * D.F * D.d};
   for (int i = 0; i < 6; ++i) {
     init_normal_kernel<<<1024, 256, 0, s>>>(c->W(i), c->Wb(i), static_cast<long long>(numel[i]), cfg->seed, i, 0.02f);
@@ -1007,7 +1015,7 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
   launch_rope_table(c->A<float2>(c->P.rope), D.T, s);
   if (D.nve) {
     // value-embedding tables N(0, 0.02) like the token embedding; gates zero
-    init_normal_kernel<<<1024, 256, 0, s>>>(c->VeW(0), c->VeWb(0), static_cast<long long>(D.nve) * D.V * D.d,
+    init_normal_kernel<<<1024, 256, 0, s>>>(c->VeW(0), c->VeWb(0), static_cast<long long>(D.nve * c->ve_elems()),
                                             cfg->seed, 7, 0.02f);
     if ((e = cudaMemsetAsync(c->pbuf + c->P.wg, 0, static_cast<size_t>(D.ngp) * 4, s)) != cudaSuccess)
       return bad(e, "zero gates");
@@ -1053,7 +1061,7 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
   const int nl = l1 - l0;
   float* inv = c->A<float>(P.inv_norm);
   // momentum and Frobenius norms of every block matrix in the range
-  const long long ne[4] = {1ll * d * 3 * d, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+  const long long ne[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
   {
     ProfScope ps(c, GPT_PROF_MUON_ELEM);
     for (int j = 0; j < 4; ++j)
@@ -1073,7 +1081,7 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
   // output (c = d), and MLP up plus transposed MLP down (c = 4d)
   struct Member { int grp; bool transpose; };
   struct Batch { int nz; int cc; Member m[2]; int nm; };
-  const Batch batches[3] = {{nl, 3 * d, {{2, false}}, 1}, {nl, d, {{3, false}}, 1},
+  const Batch batches[3] = {{nl, D.qc, {{2, false}}, 1}, {nl, d, {{3, false}}, 1},
                             {2 * nl, F, {{4, false}, {5, true}}, 2}};
   for (const Batch& bt : batches) {
     const size_t per = static_cast<size_t>(d) * bt.cc;
@@ -1103,7 +1111,7 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
       ProfScope ps(c, GPT_PROF_MUON_ELEM);
       const Member& mm = bt.m[i];
       const int rows = mm.grp == 5 ? F : d;
-      const int cols = mm.grp == 2 ? 3 * d : (mm.grp == 3 ? d : (mm.grp == 4 ? F : d));
+      const int cols = mm.grp == 2 ? D.qc : (mm.grp == 3 ? d : (mm.grp == 4 ? F : d));
       const float scale = sqrtf(std::max(1.f, static_cast<float>(rows) / static_cast<float>(cols)));
       const void* src = static_cast<const uint8_t*>(res) + static_cast<size_t>(i) * nl * per * res_es;
       // NorMuon: one factor per row of res (the shorter axis of every matrix)
@@ -1152,7 +1160,7 @@ int gpt_block_region(const gpt_ctx* c, int what, int kind, int l0, int l1, size_
   if (l0 < 0 || l1 > c->D.L || l0 > l1) return fail(GPT_EINVAL, "layer range out of bounds");
   const int grp = 2 + kind;
   const size_t d = c->D.d, F = c->D.F;
-  const size_t per[4] = {d * 3 * d, d * d, d * F, F * d};
+  const size_t per[4] = {d * static_cast<size_t>(c->D.qc), d * d, d * F, F * d};
   const size_t es = what == GPT_REGION_BF16 ? 2 : 4;
   const size_t base = what == GPT_REGION_MASTER ? c->P.w[grp] : (what == GPT_REGION_BF16 ? c->P.wb[grp] : c->P.g[grp]);
   if (offset_bytes) *offset_bytes = base + static_cast<size_t>(l0) * per[kind] * es;
@@ -1179,7 +1187,7 @@ int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float 
     // value-embedding tables and their gates
     launch_adamw(c->VeW(0), c->VeG(0), reinterpret_cast<float*>(c->sbuf + c->P.amve),
                  reinterpret_cast<float*>(c->sbuf + c->P.avve), c->VeWb(0),
-                 static_cast<long long>(c->D.nve) * c->D.V * c->D.d, lr, beta1, beta2, eps, weight_decay, bc1, bc2,
+                 static_cast<long long>(c->D.nve * c->ve_elems()), lr, beta1, beta2, eps, weight_decay, bc1, bc2,
                  c->stream);
     launch_adamw(c->GateW(0), c->GateG(0), reinterpret_cast<float*>(c->sbuf + c->P.amg),
                  reinterpret_cast<float*>(c->sbuf + c->P.avg), reinterpret_cast<bf16*>(c->pbuf + c->P.wgb), c->D.ngp,

@@ -91,12 +91,13 @@ struct FwdItem {
   bool hasB;
 };
 
-__device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int wl) {
+__device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int kvs, int wl) {
   FwdItem it;
   const int npairs = (nq + 1) / 2;
   it.bh = n / npairs;
   const int pair = npairs - 1 - (n - it.bh * npairs);
-  it.bkv = (it.bh / H) * Hkv + (it.bh - (it.bh / H) * H) / (H / Hkv);
+  // k/v row of this query head's kv head: batch rows of kvs heads each
+  it.bkv = (it.bh / H) * kvs + (it.bh - (it.bh / H) * H) / (H / Hkv);
   it.qtA = 2 * pair;
   it.hasB = it.qtA + 1 < nq;
   // both tiles start at the first key block any row of tile A sees; rows for
@@ -111,7 +112,8 @@ __device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int w
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
-                       int H, int Hkv, int T, int wl, float scale_log2, int n_items, int* sched, int* err) {
+                       int H, int Hkv, int kvs, int T, int wl, float scale_log2, int n_items, int* sched,
+                       int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive(q_full);   // end marker: releases the ring entry
           break;
         }
-        const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+        const FwdItem it = fwd_item(idx, nq, H, Hkv, kvs, wl);
         mbar_arrive_expect_tx(q_full, it.hasB ? 2 * TF_BUF : TF_BUF);
         tma_load_3d(sQ, &tq, q_full, 0, it.qtA * 128, it.bh);
         tma_load_3d(sQ + TF_TILE, &tq, q_full, 64, it.qtA * 128, it.bh);
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(q_full, n & 1, abort_flag, err)) { ok = false; break; }
         const int idx = item_ring[n & 3];
         if (idx < 0) break;
-        const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+        const FwdItem it = fwd_item(idx, nq, H, Hkv, kvs, wl);
         // S of the first block on both tiles, each once its previous P V (which
         // reads P from the same columns) has completed
         if (!mbar_wait(&k_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err)) { ok = false; break; }
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(q_empty);   // this warp has the item number
       if (idx < 0) break;
-      const FwdItem it = fwd_item(idx, nq, H, Hkv, wl);
+      const FwdItem it = fwd_item(idx, nq, H, Hkv, kvs, wl);
       if (tile == 1 && !it.hasB) continue;
       const int qt = it.qtA + tile;
       const int q0 = qt * 128;
@@ -525,13 +527,13 @@ constexpr int TB_SMEM = 6 * TF_BUF + TB_STAGE + 2048 + 256;
 // Query-block loop of key block j: nb query blocks j .. (window end) for each
 // of the G query heads of the group.
 struct BwdBlock {
-  int bkv, j, k0, nb, n_it, b, hk, G;
+  int bkv, kvrow, j, k0, nb, n_it, b, hk, G;   // kvrow: the k/v row (batch rows of kvs heads)
   __device__ __forceinline__ int q_block(int it) const { return j + it % nb; }
   __device__ __forceinline__ int q_head(int it) const { return hk * G + it / nb; }   // within the batch row
 };
 
 // Item idx: kv head idx / nq, key block idx mod nq.
-__device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int nq, int wl) {
+__device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int kvs, int nq, int wl) {
   BwdBlock k;
   k.bkv = idx / nq;
   const int j = idx - k.bkv * nq;
@@ -540,6 +542,7 @@ __device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int nq, i
   k.k0 = j * 128;
   k.b = bkv / Hkv;
   k.hk = bkv - k.b * Hkv;
+  k.kvrow = k.b * kvs + k.hk;
   k.G = H / Hkv;
   k.nb = min(nq - 1, (k.k0 + 127 + wl) / 128) - j + 1;
   k.n_it = k.G * k.nb;
@@ -551,7 +554,7 @@ __global__ void __launch_bounds__(448, 1)
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                        const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
                        const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int Hkv,
-                       int T, int wl, float scale, int n_units, int* sched, int* err) {
+                       int kvs, int T, int wl, float scale, int n_units, int* sched, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -667,17 +670,17 @@ __global__ void __launch_bounds__(448, 1)
           mbar_arrive(kv_full);
           break;
         }
-        const BwdBlock kb = bwd_block(idx, H, Hkv, nq, wl);
+        const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         // the first query block's Q and dO may load while the previous item
         // finishes; K and V (which publish the item number) once its last
         // products are done
         if (!load_q_do(kb, 0)) { ok = false; break; }
         if (n > 0 && !mbar_wait(kv_empty, (n - 1) & 1, abort_flag, err)) { ok = false; break; }
         mbar_arrive_expect_tx(kv_full, 2 * TF_BUF);
-        tma_load_3d(sK, &tk, kv_full, 0, kb.k0, kb.bkv);
-        tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, kb.k0, kb.bkv);
-        tma_load_3d(sV, &tv, kv_full, 0, kb.k0, kb.bkv);
-        tma_load_3d(sV + TF_TILE, &tv, kv_full, 64, kb.k0, kb.bkv);
+        tma_load_3d(sK, &tk, kv_full, 0, kb.k0, kb.kvrow);
+        tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, kb.k0, kb.kvrow);
+        tma_load_3d(sV, &tv, kv_full, 0, kb.k0, kb.kvrow);
+        tma_load_3d(sV + TF_TILE, &tv, kv_full, 64, kb.k0, kb.kvrow);
         ++nblk;
         for (int it = 1; it < kb.n_it; ++it)
           if (!load_q_do(kb, it)) { ok = false; break; }
@@ -718,7 +721,7 @@ __global__ void __launch_bounds__(448, 1)
         const int idx = item_ring[n & 3];
         if (idx < 0) break;
         {
-          const BwdBlock kb = bwd_block(idx, H, Hkv, nq, wl);
+          const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
           const int n_it = kb.n_it;
           // S^T of the first query block goes where the previous key block's
           // last dQ^T was (wait until the dQ warps have read it), dP^T where
@@ -852,7 +855,7 @@ __global__ void __launch_bounds__(448, 1)
       if (lane == 0) mbar_arrive(kv_empty);   // this warp has the item number
       if (idx < 0) break;
       {
-        const BwdBlock kb = bwd_block(idx, H, Hkv, nq, wl);
+        const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         for (int it = 0; it < kb.n_it && ok; ++it, ++g) {
           const int q0 = kb.q_block(it) * 128, bh = kb.b * H + kb.q_head(it);
           const bool got = mbar_wait(mm_done, g & 1, abort_flag, err);
@@ -917,8 +920,8 @@ __global__ void __launch_bounds__(448, 1)
       if (lane == 0) mbar_arrive(kv_empty);   // this warp has the item number
       if (idx < 0) break;
       {
-        const BwdBlock kb = bwd_block(idx, H, Hkv, nq, wl);
-        const int n_it = kb.n_it, k0 = kb.k0, bkv = kb.bkv;
+        const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
+        const int n_it = kb.n_it, k0 = kb.k0, bkv = kb.kvrow;
         const int key = k0 + r;
         const bool key_ok = key < T;
         // this thread's share of a query block's -lse (log2 units; -inf past T so
@@ -1149,16 +1152,17 @@ static int* sched_word(int* sched, cudaStream_t s) {
 }
 
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
-                     cudaStream_t s, int* err, int Hkv, int window, int* sched) {
+                     cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
     configured = true;
   }
   if (Hkv <= 0) Hkv = H;
+  if (kv_stride <= 0) kv_stride = Hkv;
   CUtensorMap mq, mk, mv;
-  const long long bh = 1ll * B * H, bhkv = 1ll * B * Hkv;
-  if (H % Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+  const long long bh = 1ll * B * H, bhkv = 1ll * B * kv_stride;
+  if (H % Hkv || kv_stride < Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
@@ -1168,13 +1172,14 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
   const long long n_items = ((T + 127) / 128 + 1) / 2 * bh;
   const int grid = static_cast<int>(std::min<long long>(n_items, sm_count()));
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, T, window_bound(window, T), scale_log2,
+  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, kv_stride, T, window_bound(window, T),
+                                                scale_log2,
                                                 static_cast<int>(n_items), sched_word(sched, s), err);
 }
 
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
-                     cudaStream_t s, int* err, int Hkv, int window, int* sched) {
+                     cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride) {
   static bool configured = false;
   if (!configured) {
     cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
@@ -1185,11 +1190,12 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
   CUtensorMap mq, mk, mv, mdo, mdq;
-  const long long bh = 1ll * B * H, bhkv = 1ll * B * Hkv;
+  if (kv_stride <= 0) kv_stride = Hkv;
+  const long long bh = 1ll * B * H, bhkv = 1ll * B * kv_stride;
   const long long dims[4] = {HD, H, T, B};
   const long long strides[3] = {HD * 2ll, 1ll * H * HD * 2, 1ll * T * H * HD * 2};
   const int box[4] = {64, 1, 128, 1};
-  if (H % Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
+  if (H % Hkv || kv_stride < Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
       !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
@@ -1205,7 +1211,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const int grid = static_cast<int>(std::min<long long>(n_units, sm_count()));
   const int wl = window_bound(window, T);
   int* word = wl >= T ? nullptr : sched_word(sched, s);
-  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, T, wl,
+  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
                                                 1.f / sqrtf(static_cast<float>(HD)), static_cast<int>(n_units),
                                                 word, err);
 }

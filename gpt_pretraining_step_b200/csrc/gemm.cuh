@@ -406,13 +406,14 @@ __global__ void __launch_bounds__(320, 1)
       float dqs = 1.f;   // dequantisation of fp8 operands
       if constexpr (ES == 1) dqs = (p.dq_a ? p.dq_a[0] : 1.f) * (p.dq_b ? p.dq_b[0] : 1.f);
       if constexpr (EPI == EPI_QKV) {
-        // BN = 256: the tile holds heads 2*nb and 2*nb+1 of the 3H heads of q|k|v
-        // for 128 tokens; the four warps of column half `half` own one head
-        // whole, so the per-head norm needs no exchange between warps
+        // BN = 256: the tile holds heads 2*nb and 2*nb+1 of the H + 2 Hkv heads
+        // of q|k|v for 128 tokens; the four warps of column half `half` own one
+        // head whole, so the per-head norm needs no exchange between warps
         const int gh = 2 * nb + half;
-        if (gh < 3 * p.H) {
-          const int which = gh / p.H;
-          const int head = gh - which * p.H;
+        const int hkv = p.Hkv > 0 ? p.Hkv : p.H;
+        if (gh < p.H + 2 * hkv) {
+          const int which = gh < p.H ? 0 : (gh < p.H + hkv ? 1 : 2);
+          const int head = gh - (which == 0 ? 0 : (which == 1 ? p.H : p.H + hkv));
           const int b = row / p.T;
           const int t = row - b * p.T;
           __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.qkv_out[which]) +

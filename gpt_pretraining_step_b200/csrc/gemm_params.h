@@ -33,6 +33,8 @@ struct GemmParams {
   const float* dq_a;    // fp8 operands: device inverse scales of A and B; the accumulator is
   const float* dq_b;    //   multiplied by dq_a[0] * dq_b[0] before the epilogue (null: 1)
   int T, H;
+  int Hkv;              // QKV: kv heads (0: H); columns are q (H heads) | k | v (Hkv heads each),
+                        //   k and v stored at head rows b*H + j of their [B, H, T, 128] buffers
   int tma_out;          // 1: the main output is written by TMA stores through the output tensor map
   int tma_out2;         // 1: also an fp16 copy of the output, same layout, through the second map
   void* out2;           //   (its base; row stride ldo, batch stride out_bs)

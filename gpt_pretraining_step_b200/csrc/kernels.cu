@@ -397,22 +397,22 @@ __global__ void __launch_bounds__(256) smear_bwd_kernel(const float* __restrict_
 __global__ void __launch_bounds__(256) ve_fwd_kernel(const bf16* __restrict__ xn1, const int* __restrict__ tok,
                                                      const bf16* __restrict__ ve, const float* __restrict__ wg,
                                                      float* __restrict__ sig, bf16* __restrict__ v, int M, int T,
-                                                     int H, int C, int V) {
+                                                     int H, int Hkv, int C, int V) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
-  const int d = H * 128;
+  const int d = H * 128, kvd = Hkv * 128;
   const int b = t / T, pos = t - b * T;
   int id = tok[t];
   id = static_cast<unsigned>(id) < static_cast<unsigned>(V) ? id : 0;
   const bf16* xr = xn1 + static_cast<long long>(t) * d;
-  const bf16* er = ve + static_cast<long long>(id) * d;
-  for (int h = 0; h < H; ++h) {
+  const bf16* er = ve + static_cast<long long>(id) * kvd;
+  for (int h = 0; h < Hkv; ++h) {   // kv head h sits at head row b*H + h of v
     float z = 0.f;
-    for (int c = lane; c < C; c += 32) z += __bfloat162float(xr[c]) * wg[c * H + h];
+    for (int c = lane; c < C; c += 32) z += __bfloat162float(xr[c]) * wg[c * Hkv + h];
     z = warp_sum(z);
     const float sg = 1.f / (1.f + expf(-z));
-    if (lane == 0) sig[static_cast<long long>(t) * H + h] = sg;
+    if (lane == 0) sig[static_cast<long long>(t) * Hkv + h] = sg;
     const float gate = 3.f * sg;
     bf16* vr = v + ((static_cast<long long>(b) * H + h) * T + pos) * 128 + 4 * lane;
     const uint2 a = *reinterpret_cast<const uint2*>(vr);
@@ -430,27 +430,27 @@ __global__ void __launch_bounds__(256) ve_fwd_kernel(const bf16* __restrict__ xn
 __global__ void __launch_bounds__(256) ve_bwd_kernel(const bf16* __restrict__ dv, const int* __restrict__ tok,
                                                      const bf16* __restrict__ ve, const float* __restrict__ sig,
                                                      float* __restrict__ dve, float* __restrict__ dz, int M, int T,
-                                                     int H, int V) {
+                                                     int H, int Hkv, int V) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
-  const int d = H * 128;
+  const int kvd = Hkv * 128;
   const int b = t / T, pos = t - b * T;
   int id = tok[t];
   id = static_cast<unsigned>(id) < static_cast<unsigned>(V) ? id : 0;
-  const bf16* er = ve + static_cast<long long>(id) * d;
-  for (int h = 0; h < H; ++h) {
+  const bf16* er = ve + static_cast<long long>(id) * kvd;
+  for (int h = 0; h < Hkv; ++h) {
     const uint2 g = *reinterpret_cast<const uint2*>(dv + ((static_cast<long long>(b) * H + h) * T + pos) * 128 +
                                                     4 * lane);
     const uint2 e = *reinterpret_cast<const uint2*>(er + h * 128 + 4 * lane);
     const float g0 = bf16_lo(g.x), g1 = bf16_hi(g.x), g2 = bf16_lo(g.y), g3 = bf16_hi(g.y);
     float dot = g0 * bf16_lo(e.x) + g1 * bf16_hi(e.x) + g2 * bf16_lo(e.y) + g3 * bf16_hi(e.y);
     dot = warp_sum(dot);
-    const float sg = sig[static_cast<long long>(t) * H + h];
+    const float sg = sig[static_cast<long long>(t) * Hkv + h];
     const float gate = 3.f * sg;
-    *reinterpret_cast<float4*>(dve + static_cast<long long>(t) * d + h * 128 + 4 * lane) =
+    *reinterpret_cast<float4*>(dve + static_cast<long long>(t) * kvd + h * 128 + 4 * lane) =
         make_float4(gate * g0, gate * g1, gate * g2, gate * g3);
-    if (lane == 0) dz[static_cast<long long>(t) * H + h] = dot * 3.f * sg * (1.f - sg);
+    if (lane == 0) dz[static_cast<long long>(t) * Hkv + h] = dot * 3.f * sg * (1.f - sg);
   }
 }
 
@@ -507,7 +507,7 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
                               const bf16* __restrict__ dv, const bf16* __restrict__ qn,
                               const bf16* __restrict__ kn, const float* __restrict__ rq,
                               const float* __restrict__ rk, const float2* __restrict__ rope,
-                              bf16* __restrict__ dqkv, int B, int T, int H) {
+                              bf16* __restrict__ dqkv, int B, int T, int H, int Hkv) {
   const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + warp_id();
   const long long total = static_cast<long long>(B) * H * T;
   if (w >= total) return;
@@ -516,13 +516,16 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
   const int h = static_cast<int>((w / T) % H);
   const int b = static_cast<int>(w / (static_cast<long long>(T) * H));
   const long long m = static_cast<long long>(b) * T + t;
-  const int d = H * 128;
-  const long long src = w * 128;
+  const int d = H * 128, kvd = Hkv * 128;
+  const long long src = w * 128;   // k/v heads j < Hkv sit at the same head rows as q's
   const int i0 = 2 * lane_id();
   const float2 e0 = rope[t * 64 + i0], e1 = rope[t * 64 + i0 + 1];
-  bf16* out = dqkv + m * 3 * d + h * 128;
+  // row of dqkv: q (d) | k (kvd) | v (kvd); head h of k and v only for h < Hkv
+  bf16* out = dqkv + m * (d + 2 * kvd) + h * 128;
+  const bool has_kv = h < Hkv;
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
+    if (which == 1 && !has_kv) break;
     const bf16* yv = which == 0 ? qn : kn;
     const float r = (which == 0 ? rq : rk)[m * H + h];
     float gl0, gl1, gh0, gh1;
@@ -548,8 +551,10 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
     *reinterpret_cast<uint32_t*>(out + which * d + i0) = pack_bf16x2(ol0, ol1);
     *reinterpret_cast<uint32_t*>(out + which * d + 64 + i0) = pack_bf16x2(oh0, oh1);
   }
-  const uint2 vv = *reinterpret_cast<const uint2*>(dv + src + 4 * lane_id());
-  *reinterpret_cast<uint2*>(out + 2 * d + 4 * lane_id()) = vv;
+  if (has_kv) {
+    const uint2 vv = *reinterpret_cast<const uint2*>(dv + src + 4 * lane_id());
+    *reinterpret_cast<uint2*>(out + d + kvd + 4 * lane_id()) = vv;
+  }
 }
 
 // ------------------------------------------------------- cross-entropy finish
@@ -1027,9 +1032,9 @@ void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float
 }
 
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn, const float* rq,
-                   const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s) {
+                   const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s, int Hkv) {
   const long long rows = 1ll * B * H * T;
-  qk_bwd_kernel<<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H);
+  qk_bwd_kernel<<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, Hkv > 0 ? Hkv : H);
 }
 
 void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* tgt, float* row_loss, int rows,
@@ -1104,13 +1109,13 @@ void launch_scalar_grad_finish(const float* part, int L, float* grad, bool accum
 }
 
 void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float* wg, float* sig, bf16* v, int M,
-                   int T, int H, int C, int V, cudaStream_t s) {
-  ve_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(xn1, tok, ve, wg, sig, v, M, T, H, C, V);
+                   int T, int H, int Hkv, int C, int V, cudaStream_t s) {
+  ve_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(xn1, tok, ve, wg, sig, v, M, T, H, Hkv, C, V);
 }
 
 void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
-                   int T, int H, int V, cudaStream_t s) {
-  ve_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dv, tok, ve, sig, dve, dz, M, T, H, V);
+                   int T, int H, int Hkv, int V, cudaStream_t s) {
+  ve_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dv, tok, ve, sig, dve, dz, M, T, H, Hkv, V);
 }
 
 void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,

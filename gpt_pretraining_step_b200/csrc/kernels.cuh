@@ -24,11 +24,12 @@ void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cuda
 void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dx_bf16,
                         int M, int d, bool accumulate, cudaStream_t s);
 
-// Per-head QK-norm and RoPE backward plus the v copy, into dqkv [M, 3d]
-// (dq is the fp32 attention-backward accumulator, dk and dv bf16).
+// Per-head QK-norm and RoPE backward plus the v copy, into dqkv [M, d + 2
+// Hkv 128] (dq is the fp32 attention-backward accumulator, dk and dv bf16,
+// kv head j of batch b at head row b*H + j; Hkv 0 = H).
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn,
                    const float* rq, const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H,
-                   cudaStream_t s);
+                   cudaStream_t s, int Hkv = 0);
 
 // Per row: lse from the (max, sumexp) tile partials, row loss = lse - z[target],
 // and z <- (softmax(z) - onehot(target)) * inv_count in place.
@@ -99,13 +100,16 @@ void launch_smear_bwd(const float* g, const float* e, const float* sig, const fl
 int resid_partial_blocks();
 
 // Value embeddings: v[t, h] += 3 sigmoid(xn1[t, :C] . wg[:, h]) ve[tok[t], h]
-// (v [B, H, T, 128] bf16, ve the bf16 [V, d] table, wg [C, H]); the backward
-// writes dve (fp32 [M, d], to be scattered into the table's gradient) and dz
-// [M, H]; the gate gradient (C * H <= 1024) and the xn1 gradient correction.
+// for the Hkv kv heads (v [B, H, T, 128] bf16 with kv head h at head row
+// b*H + h, xn1 [M, 128 H], ve the bf16 [V, 128 Hkv] table, wg [C, Hkv]); the
+// backward writes dve (fp32 [M, 128 Hkv], to be scattered into the table's
+// gradient) and dz [M, Hkv]; the gate gradient (C * Hkv <= 1024, the H
+// argument of launch_ve_gate_grad / launch_ve_dxn is Hkv) and the xn1
+// gradient correction.
 void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float* wg, float* sig, bf16* v, int M,
-                   int T, int H, int C, int V, cudaStream_t s);
+                   int T, int H, int Hkv, int C, int V, cudaStream_t s);
 void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
-                   int T, int H, int V, cudaStream_t s);
+                   int T, int H, int Hkv, int V, cudaStream_t s);
 void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,
                          bool accumulate, cudaStream_t s);
 void launch_ve_dxn(float* dxn, const float* dz, const float* wg, int M, int d, int H, int C, cudaStream_t s);

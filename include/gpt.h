@@ -122,6 +122,13 @@ typedef struct gpt_config {
                            * a [vocab, d] table and a [C, heads] gate per such
                            * layer, trained by adamw_step (tables N(0, 0.02),
                            * gates 0 at init).  0: off. */
+  int32_t n_kv_head;      /* grouped kv heads (section "1. Modelo GPT", GQA):
+                           * 0 = one per query head; else a divisor of the
+                           * heads; the fused projection is then
+                           * [d, d + 2 * 128 * n_kv_head] with columns
+                           * q | k | v, query head h reading kv head
+                           * h / (heads / n_kv_head); value-embedding tables
+                           * and gates are per kv head. */
 } gpt_config;
 
 typedef struct gpt_ctx gpt_ctx;
@@ -149,7 +156,7 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
 int gpt_fwd_bwd(gpt_ctx* ctx, const int32_t* tokens, const int32_t* targets, float* loss_out, int accumulate);
 
 /* Muon update of every 2-D block matrix (fused q|k|v, attention output, MLP
- * up, MLP down): mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
+ * up, MLP down; q|k|v is [d, 3d], narrower with grouped kv heads): mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
  * with the Polar Express coefficients; W = W (1 - lr * weight_decay)
  * - lr * sqrt(max(1, rows / cols)) * X.  Refreshes the bf16 copies. */
 int muon_step(gpt_ctx* ctx, float lr, float momentum, float weight_decay);
@@ -205,7 +212,8 @@ int gpt_train_step_host(gpt_ctx* ctx, const int32_t* tokens_host, const int32_t*
                         const gpt_hparams* hp, float* loss_host);
 
 /* Parameter tensors: id 0 = token embedding [vocab, d], 1 = lm_head [d, vocab],
- * 2 + 4 l + j for block l with j = 0 fused q|k|v [d, 3d], 1 attention output
+ * 2 + 4 l + j for block l with j = 0 fused q|k|v [d, 3d] (d + 256 n_kv_head
+ * columns with grouped kv heads), 1 attention output
  * [d, d], 2 MLP up [d, 4d], 3 MLP down [4d, d]; with residual_extras, id
  * 2 + 4 depth = the scalars [1, 2 depth + 26] (resid[0..depth),
  * x0s[0..depth), backout, smear, smear gate weights[24]); with value

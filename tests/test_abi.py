@@ -65,7 +65,7 @@ def test_workspace_size_valid_configs(L):
                                  dict(seq_len=0), dict(vocab=4), dict(window_pattern="SXL", short_window=8),
                                  dict(window_pattern="SSSL", short_window=-1),
                                  dict(window_pattern="SSSLSSSLSSSL", short_window=8), dict(ve_gate_channels=-1),
-                                 dict(ve_gate_channels=129)])
+                                 dict(ve_gate_channels=129), dict(n_kv_head=3), dict(n_kv_head=-1)])
 def test_workspace_size_rejects_bad_config(L, bad):
     import gpt_pretraining_step_b200 as g
     with pytest.raises(g.GptError) as e:

@@ -225,6 +225,54 @@ def test_value_embeddings_match_oracle(torch, name, extras):
     assert np.abs(f64(st.get(gid, g.KIND_PARAM)) - p_ref).max() < 1e-6
 
 
+GQA_SHAPES = {
+    "ragged_kv1": syn.make_shape(depth=2, d_model=256, vocab=1000, batch=2, seq_len=200, n_kv_head=1),
+    "four_heads_kv2": syn.make_shape(depth=3, d_model=512, vocab=512, batch=1, seq_len=320, n_kv_head=2),
+}
+
+
+@pytest.mark.parametrize("name,extras,ve", [("ragged_kv1", False, 0), ("four_heads_kv2", False, 0),
+                                            ("four_heads_kv2", True, 16)])
+def test_grouped_kv_model_matches_oracle(torch, name, extras, ve):
+    """Grouped kv heads through the narrower q|k|v projection, its epilogue,
+    the attention kernels (kv heads at their query-head rows), the dq|dk|dv
+    assembly and, with it, value embeddings and the residual extras; then one
+    Muon step on the narrower matrices."""
+    import gpt_pretraining_step_b200 as g
+    s = GQA_SHAPES[name]
+    params = syn.init_params(s, seed=61, extras=extras, ve_channels=ve)
+    if ve:
+        params["ve_gate"] = syn.gaussian(params["ve_gate"].shape, seed=62, std=2.0)
+    if extras:
+        params["scalars"] = syn.random_scalars(s, seed=63)
+    tok, tgt = syn.tokens(s, seed=64), syn.targets(s, seed=65)
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   residual_extras=extras, ve_gate_channels=ve, n_kv_head=s.n_kv_head)
+    specs = syn.param_specs(s, extras=extras, ve_channels=ve)
+    assert st.num_tensors() == len(specs)
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        assert st.tensor_info(tid)[:2] == (r, c), pname
+        st.set(tid, params[pname])
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL
+    assert np.abs(f64(st.row_loss()).ravel() - cache["row_loss"]).max() < 2e-2
+    G = {}
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        G[pname] = f64(st.get(tid, g.KIND_GRAD))
+        cs = cosine(G[pname], grads[pname])
+        assert cs >= GRAD_COS, (pname, cs)
+    st.muon_step(0.02, 0.95, 0.0)
+    st.check()
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if grp != "muon":
+            continue
+        W0 = params[pname].astype(np.float64)
+        W_ref, _ = oo.muon_step(W0, G[pname], np.zeros((r, c)), 0.02, 0.95, 0.0)
+        assert relfro(f64(st.get(tid, g.KIND_PARAM)) - W0, W_ref - W0) <= MUON_RELFRO, pname
+
+
 def test_embedding_and_target_indexing_exact(torch):
     # with a zero lm_head the logits vanish: loss = ln V exactly, and dW_lm has
     # one shared column for every vocabulary id that is not a target, so the set
