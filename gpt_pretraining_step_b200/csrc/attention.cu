@@ -1124,16 +1124,6 @@ __global__ void attn_bwd_dot_kernel(const bf16* __restrict__ o, const bf16* __re
 // bound no row reaches (kept small enough that k0 + 127 + wl fits in an int).
 static int window_bound(int window, int T) { return window < 0 || window >= T ? (1 << 30) : window; }
 
-static int sm_count() {
-  static int n = 0;
-  if (n <= 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 // Scheduler words for callers that bring none: a ring of 64 library-owned
 // counters, one per launch in turn, each zeroed on the launch's stream
@@ -1142,7 +1132,7 @@ __device__ int g_sched_ring[64];
 
 static int* sched_word(int* sched, cudaStream_t s) {
   if (!sched) {
-    static unsigned next = 0;
+    static std::atomic<unsigned> next{0};
     int* base = nullptr;
     if (cudaGetSymbolAddress(reinterpret_cast<void**>(&base), g_sched_ring) != cudaSuccess) return nullptr;
     sched = base + (next++ & 63u);
@@ -1153,10 +1143,10 @@ static int* sched_word(int* sched, cudaStream_t s) {
 
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride) {
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
-    configured = true;
+  static std::atomic<unsigned long long> configured{0};
+  if (set_smem_limit_once(attn_fwd_tc_kernel, TF_SMEM, configured) != cudaSuccess) {
+    if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
+    return;
   }
   if (Hkv <= 0) Hkv = H;
   if (kv_stride <= 0) kv_stride = Hkv;
@@ -1170,7 +1160,7 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
   }
   // persistent: one CTA per SM over the pairs of query tiles of every head
   const long long n_items = ((T + 127) / 128 + 1) / 2 * bh;
-  const int grid = static_cast<int>(std::min<long long>(n_items, sm_count()));
+  const int grid = static_cast<int>(std::min<long long>(n_items, device_sm_count()));
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
   attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, kv_stride, T, window_bound(window, T),
                                                 scale_log2,
@@ -1180,10 +1170,10 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride) {
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
-    configured = true;
+  static std::atomic<unsigned long long> configured{0};
+  if (set_smem_limit_once(attn_bwd_tc_kernel, TB_SMEM, configured) != cudaSuccess) {
+    if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
+    return;
   }
   if (Hkv <= 0) Hkv = H;
   const long long rows = 1ll * B * H * T;
@@ -1208,7 +1198,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   // CTA's next unit ahead of time); with one, unit costs differ and the
   // counter balances them.
   const long long n_units = 1ll * B * Hkv * (((T + 127) / 128 + 1) / 2);
-  const int grid = static_cast<int>(std::min<long long>(n_units, sm_count()));
+  const int grid = static_cast<int>(std::min<long long>(n_units, device_sm_count()));
   const int wl = window_bound(window, T);
   int* word = wl >= T ? nullptr : sched_word(sched, s);
   attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,

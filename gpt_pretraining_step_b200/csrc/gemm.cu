@@ -79,12 +79,9 @@ cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorM
                    const GemmParams& p, cudaStream_t s) {
   using C = GemmCfg<sizeof(T), BN>;
   auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> configured{0};
+  cudaError_t e = set_smem_limit_once(kern, C::SMEM, configured);
+  if (e != cudaSuccess) return e;
   const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
   kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, md, p);
   return cudaGetLastError();
@@ -96,14 +93,18 @@ using f16 = __half;
 }  // namespace
 
 int device_sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  // per device (a process may drive GPUs of different sizes)
+  static std::atomic<int> n[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::atomic<int>& slot = n[dev & 63];
+  int v = slot.load(std::memory_order_relaxed);
+  if (v <= 0) {
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    if (v <= 0) v = 148;
+    slot.store(v, std::memory_order_relaxed);
   }
-  return n;
+  return v;
 }
 
 int gemm_tiles(const GemmCall& c) {

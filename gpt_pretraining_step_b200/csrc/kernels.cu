@@ -1051,11 +1051,8 @@ size_t embed_bwd_workspace(int M) { return static_cast<size_t>(kEmbChunk) * size
 
 void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws, bool accumulate,
                       cudaStream_t s) {
-  static bool configured = false;
-  if (!configured) {
-    cudaFuncSetAttribute(embed_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kEmbChunk * 4);
-    configured = true;
-  }
+  static std::atomic<unsigned long long> configured{0};
+  set_smem_limit_once(embed_sort_kernel, kEmbChunk * 4, configured);   // a failure shows at the launch
   if (!accumulate) cudaMemsetAsync(dwte, 0, static_cast<size_t>(V) * d * sizeof(float), s);
   uint32_t* keys = static_cast<uint32_t*>(ws);
   for (int base = 0; base < M; base += kEmbChunk) {
