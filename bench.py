@@ -81,7 +81,7 @@ def peaks():
 # categories that can dominate the d20 step, from one ncu capture of a whole
 # d20 step of the current kernels (profiles/dram_traffic_d20.md).  Used for the
 # roofline's `traffic` only on that workload; null elsewhere.
-NCU_TRAFFIC_D20 = {"dx_gemm": 504.3e6, "attn_bwd": 961.5e6, "dw_gemm": 12.16e9, "attn_fwd": 312.2e6}
+NCU_TRAFFIC_D20 = {"dx_gemm": 511.9e6, "attn_bwd": 958.9e6, "dw_gemm": 9.59e9, "attn_fwd": 312.1e6}
 
 
 def model_flops_per_token(s, causal=False):

@@ -503,6 +503,9 @@ __global__ void scalar_grad_finish_kernel(const float* __restrict__ part, int nb
 
 // -------------------------------------------------- QK-norm / RoPE backward
 
+// kGrouped: fewer kv heads than query heads (the plain case keeps the
+// unconditional k/v path).
+template <bool kGrouped>
 __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restrict__ dk,
                               const bf16* __restrict__ dv, const bf16* __restrict__ qn,
                               const bf16* __restrict__ kn, const float* __restrict__ rq,
@@ -522,7 +525,7 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
   const float2 e0 = rope[t * 64 + i0], e1 = rope[t * 64 + i0 + 1];
   // row of dqkv: q (d) | k (kvd) | v (kvd); head h of k and v only for h < Hkv
   bf16* out = dqkv + m * (d + 2 * kvd) + h * 128;
-  const bool has_kv = h < Hkv;
+  const bool has_kv = !kGrouped || h < Hkv;
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
     if (which == 1 && !has_kv) break;
@@ -1034,7 +1037,10 @@ void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn, const float* rq,
                    const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s, int Hkv) {
   const long long rows = 1ll * B * H * T;
-  qk_bwd_kernel<<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, Hkv > 0 ? Hkv : H);
+  if (Hkv <= 0 || Hkv == H)
+    qk_bwd_kernel<false><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, H);
+  else
+    qk_bwd_kernel<true><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, Hkv);
 }
 
 void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* tgt, float* row_loss, int rows,
