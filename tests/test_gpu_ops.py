@@ -192,6 +192,35 @@ def test_attention_bwd_window_gqa(torch, B, H, Hkv, T, window):
         assert relfro(got, ref) < 2e-2, name
 
 
+@pytest.mark.parametrize("Hkv,window", [(10, 1024), (2, -1), (5, 512)])
+def test_attention_variants_at_d20_shape_sampled(torch, Hkv, window):
+    """The d20 attention shape (B 16, H 10, T 2048) with grouped kv heads and
+    windows, checked on sampled heads: o, lse and dq of two query heads, dk
+    and dv of one kv head (the sum over its whole group)."""
+    import gpt_pretraining_step_b200 as g
+    B, H, T = 16, 10, 2048
+    G = H // Hkv
+    q, k, v = _kv_inputs(B, H, Hkv, T, seed=Hkv + 7)
+    dout = syn.round_to_bf16(syn.gaussian((B, T, H, 128), seed=Hkv + 9))
+    qt, kt, vt = bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v)
+    o, lse = g.attention_fwd(qt, kt, vt, window=window)
+    dq, dk, dv = g.attention_bwd(qt, kt, vt, o, lse, bf16_t(torch, dout), window=window)
+    torch.cuda.synchronize()
+    w = None if window < 0 else window
+    for b, hk in ((3, 0), (12, Hkv - 1)):
+        heads = list(range(hk * G, hk * G + G))
+        q64 = q[b:b + 1, heads].astype(np.float64)
+        k64, v64 = k[b:b + 1, hk:hk + 1].astype(np.float64), v[b:b + 1, hk:hk + 1].astype(np.float64)
+        ref, P = om.attention(q64, k64, v64, window=w)
+        got_o = f64(o[b, :, heads]).transpose(1, 0, 2)[None]
+        assert relfro(got_o, ref) < 1e-2, (b, hk)
+        dy = dout[b:b + 1, :, heads].astype(np.float64).transpose(0, 2, 1, 3)
+        dq_r, dk_r, dv_r = om.attention_bwd(dy, q64, k64, v64, P)
+        for got, r in ((f64(dq[b, heads])[None], dq_r), (f64(dk[b, hk])[None, None], dk_r),
+                       (f64(dv[b, hk])[None, None], dv_r)):
+            assert cosine(got, r) > 0.9999 and relfro(got, r) < 2e-2, (b, hk)
+
+
 def test_attention_rejects_bad_head_split(torch):
     import gpt_pretraining_step_b200 as g
     q, k, v = _kv_inputs(1, 3, 2, 64, seed=1)
