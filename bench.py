@@ -391,9 +391,11 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
-            "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)", "global_batch": s.batch * world,
+            "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)",
+                       "global_batch": s.batch * world,
                        "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
-                       "parallelism": f"dp{world}" + ("+sharded-optimizer" if a.shard_optimizer and world > 1 else ""), "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
+                       "parallelism": f"dp{world}" + ("+sharded-optimizer" if a.shard_optimizer and world > 1 else ""),
+                       "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
                        "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
                        "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
                                      else "full causal"),

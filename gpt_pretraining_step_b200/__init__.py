@@ -22,11 +22,13 @@ PROF_CATEGORIES = ["qkv_gemm", "proj_gemm", "fc_gemm", "down_gemm", "attn_fwd", 
                    "ns_gemm", "muon_elem", "adamw", "fp8_quant"]
 
 ABI_FUNCTIONS = [
-    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "muon_step_normuon", "muon_step_layers", "gpt_block_region", "adamw_step", "gpt_train_step_host",
-    "gpt_num_tensors", "gpt_tensor_info", "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
-    "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error", "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3",
-    "gpt_op_matmul_fp8", "gpt_op_attention_fwd",
-    "gpt_op_attention_bwd", "gpt_op_attention_fwd_ex", "gpt_op_attention_bwd_ex", "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
+    "gpt_workspace_size", "gpt_init", "gpt_fwd_bwd", "muon_step", "muon_step_normuon", "muon_step_layers",
+    "gpt_block_region", "adamw_step", "gpt_train_step_host", "gpt_num_tensors", "gpt_tensor_info",
+    "gpt_get_tensor", "gpt_set_tensor", "gpt_get_row_loss", "gpt_grad_region", "gpt_check",
+    "gpt_launch_count", "gpt_profile_enable", "gpt_profile_read", "gpt_destroy", "gpt_last_error",
+    "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3", "gpt_op_matmul_fp8",
+    "gpt_op_attention_fwd", "gpt_op_attention_bwd", "gpt_op_attention_fwd_ex", "gpt_op_attention_bwd_ex",
+    "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
     "gpt_op_newton_schulz_noalloc",
 ]
 

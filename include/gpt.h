@@ -156,7 +156,8 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
 int gpt_fwd_bwd(gpt_ctx* ctx, const int32_t* tokens, const int32_t* targets, float* loss_out, int accumulate);
 
 /* Muon update of every 2-D block matrix (fused q|k|v, attention output, MLP
- * up, MLP down; q|k|v is [d, 3d], narrower with grouped kv heads): mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
+ * up, MLP down; q|k|v is [d, 3d], narrower with grouped kv heads):
+ * mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
  * with the Polar Express coefficients; W = W (1 - lr * weight_decay)
  * - lr * sqrt(max(1, rows / cols)) * X.  Refreshes the bf16 copies. */
 int muon_step(gpt_ctx* ctx, float lr, float momentum, float weight_decay);
