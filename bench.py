@@ -10,7 +10,9 @@ resident in HBM when the timed region starts; the activations (tens of GB)
 exceed the 126 MB L2 many times over, so no L2 flush is needed between steps.
 For N > 1 (launched by torch.distributed.run) every rank trains on its own
 batch and the gradients are averaged with one NCCL all-reduce per step before
-the (replicated) optimizer step; the reported time is the max over ranks.
+the (replicated) optimizer step, or, with --shard-optimizer, exchanged in three
+phases around a Muon step split by layer; the reported time is the max over
+ranks.
 
 Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle
 on a bounded sample of the same workload instead (rank 0 only).
