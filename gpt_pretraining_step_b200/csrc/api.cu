@@ -804,9 +804,9 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     struct DW { const bf16* a; long long lda, a_bs; const bf16* b; long long ldb, b_bs; int rows, cols; float* out; };
     const DW dws[4] = {
         {xn1, d, static_cast<long long>(Md), dqkv_all, D.qc, 1ll * M * D.qc, d, D.qc, c->G(2)},
-        {o, d, static_cast<long long>(Md), gx, d, 2ll * Md, d, d, c->G(3)},
+        {o, d, static_cast<long long>(Md), gx, d, 2 * static_cast<long long>(Md), d, d, c->G(3)},
         {xn2, d, static_cast<long long>(Md), du_all, F, 1ll * M * F, d, F, c->G(4)},
-        {h, F, 1ll * M * F, gx + Md, d, 2ll * Md, F, d, c->G(5)},
+        {h, F, 1ll * M * F, gx + Md, d, 2 * static_cast<long long>(Md), F, d, c->G(5)},
     };
     for (const DW& w : dws) {
       GemmCall g = base_call(w.rows, w.cols, M);

@@ -17,8 +17,6 @@ namespace gpt {
 
 namespace {
 
-constexpr int kMaxVec = 16;   // float4 per lane per row: d <= 2048
-
 inline int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
 __device__ __forceinline__ void store_bf16x4(bf16* dst, float4 v) {
@@ -1053,7 +1051,8 @@ void launch_sum_scale(const float* v, int n, float scale, float* out, cudaStream
   sum_scale_kernel<<<1, 1024, 0, s>>>(v, n, scale, out);
 }
 
-size_t embed_bwd_workspace(int M) { return static_cast<size_t>(kEmbChunk) * sizeof(uint32_t) + 256; }
+// the sort runs in chunks of kEmbChunk tokens, so the workspace does not grow with M
+size_t embed_bwd_workspace(int /*M*/) { return static_cast<size_t>(kEmbChunk) * sizeof(uint32_t) + 256; }
 
 void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws, bool accumulate,
                       cudaStream_t s) {
