@@ -29,7 +29,7 @@ ABI_FUNCTIONS = [
     "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3", "gpt_op_matmul_fp8",
     "gpt_op_attention_fwd", "gpt_op_attention_bwd", "gpt_op_attention_fwd_ex", "gpt_op_attention_bwd_ex",
     "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
-    "gpt_op_newton_schulz_noalloc",
+    "gpt_op_newton_schulz_noalloc", "gpt_get_adam_step", "gpt_set_adam_step",
 ]
 
 
@@ -83,6 +83,8 @@ def lib():
             "gpt_set_tensor": (i32, [vp, i32, i32, vp]),
             "gpt_get_row_loss": (i32, [vp, vp]),
             "gpt_grad_region": (i32, [vp, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+            "gpt_get_adam_step": (i32, [vp, ctypes.POINTER(ctypes.c_int64)]),
+            "gpt_set_adam_step": (i32, [vp, ctypes.c_int64]),
             "gpt_check": (i32, [vp]),
             "gpt_launch_count": (ctypes.c_int64, [vp]),
             "gpt_profile_enable": (i32, [vp, ctypes.c_uint32]),
@@ -264,6 +266,30 @@ class GPTStep:
 
     def check(self):
         return _check(lib().gpt_check(self.h))
+
+    # -- checkpoint
+    def _state_kinds(self, tid):
+        _, _, group = self.tensor_info(tid)
+        if group == GROUP_MUON:
+            return (KIND_PARAM, KIND_MOM, KIND_NORMUON_V)
+        return (KIND_PARAM, KIND_ADAM_M, KIND_ADAM_V)
+
+    def state_dict(self):
+        """Every tensor's value and optimizer state (host float32 arrays, keyed
+        (tensor id, kind)) and the AdamW step count: what a checkpoint needs."""
+        step = ctypes.c_int64()
+        _check(lib().gpt_get_adam_step(self.h, ctypes.byref(step)))
+        tensors = {}
+        for tid in range(self.num_tensors()):
+            for kind in self._state_kinds(tid):
+                tensors[(tid, kind)] = self.get(tid, kind).cpu().numpy()
+        return {"tensors": tensors, "adam_step": int(step.value)}
+
+    def load_state_dict(self, state):
+        """Restore what state_dict returned (same configuration)."""
+        for (tid, kind), value in state["tensors"].items():
+            self.set(tid, value, kind)
+        _check(lib().gpt_set_adam_step(self.h, int(state["adam_step"])))
 
     def launch_count(self):
         return lib().gpt_launch_count(self.h)

@@ -1228,6 +1228,22 @@ int gpt_train_step_host(gpt_ctx* c, const int32_t* tokens_host, const int32_t* t
   return gpt_check(c);
 }
 
+int gpt_get_adam_step(const gpt_ctx* c, int64_t* step) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (!step) return fail(GPT_EINVAL, "null destination");
+  *step = c->adam_step;
+  return GPT_OK;
+}
+
+int gpt_set_adam_step(gpt_ctx* c, int64_t step) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (step < 0) return fail(GPT_EINVAL, "the AdamW step count cannot be negative");
+  c->adam_step = step;
+  return GPT_OK;
+}
+
 int gpt_num_tensors(const gpt_ctx* c) {
   return c ? 2 + 4 * c->D.L + c->D.extras + (c->D.nve ? c->D.nve + 1 : 0) : 0;
 }

@@ -53,8 +53,8 @@ enum {
   GPT_KIND_PARAM = 0,  /* fp32 master weight (setting it also refreshes the bf16 copy) */
   GPT_KIND_GRAD = 1,   /* fp32 gradient of the mean loss */
   GPT_KIND_MOM = 2,    /* Muon momentum (block matrices only) */
-  GPT_KIND_ADAM_M = 3, /* AdamW first moment (embedding, lm_head only) */
-  GPT_KIND_ADAM_V = 4, /* AdamW second moment (embedding, lm_head only) */
+  GPT_KIND_ADAM_M = 3, /* AdamW first moment (tensors of the AdamW group only) */
+  GPT_KIND_ADAM_V = 4, /* AdamW second moment (tensors of the AdamW group only) */
   GPT_KIND_NORMUON_V = 5 /* NorMuon second moment (block matrices only): d
                           * floats, one per index of the shorter axis */
 };
@@ -197,9 +197,17 @@ enum { GPT_REGION_MASTER = 0, GPT_REGION_BF16 = 1, GPT_REGION_GRAD = 2 };
 int gpt_block_region(const gpt_ctx* ctx, int what, int kind, int l0, int l1, size_t* offset_bytes,
                      size_t* size_bytes);
 
-/* AdamW update of the token embedding and lm_head with bias correction
- * (the step count is kept in the context) and decoupled weight decay. */
+/* AdamW update of the token embedding and lm_head (and of the residual-extras
+ * scalars and value-embedding tables and gates when those are on) with bias
+ * correction (the step count is kept in the context) and decoupled weight
+ * decay. */
 int adamw_step(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay);
+
+/* The number of adamw_step calls so far (its bias correction uses it), for a
+ * checkpoint: with every tensor's value and optimizer state (gpt_get_tensor)
+ * it restores a context exactly.  A negative count is GPT_EINVAL. */
+int gpt_get_adam_step(const gpt_ctx* ctx, int64_t* step);
+int gpt_set_adam_step(gpt_ctx* ctx, int64_t step);
 
 /* Whole step from HOST buffers: copies tokens and targets (int32
  * [batch, seq_len], pinned memory recommended) to the device, runs

@@ -98,6 +98,8 @@ def test_null_arguments_are_einval(L):
     assert L.muon_step_normuon(None, 0.02, 0.95, 0.0, 0.95) == g.GPT_EINVAL
     assert L.muon_step_layers(None, 0.02, 0.95, 0.0, -1.0, 0, 1) == g.GPT_EINVAL
     assert L.gpt_block_region(None, 0, 0, 0, 1, None, None) == g.GPT_EINVAL
+    assert L.gpt_set_adam_step(None, 3) == g.GPT_EINVAL
+    assert L.gpt_get_adam_step(None, None) == g.GPT_EINVAL
     assert L.adamw_step(None, 1e-3, 0.8, 0.95, 1e-10, 0.0) == g.GPT_EINVAL
     assert L.gpt_check(None) == g.GPT_EINVAL
     assert L.gpt_num_tensors(None) == 0

@@ -75,3 +75,42 @@ def test_every_option_together_matches_oracle(torch):
             W_ref, _, _ = oo.adamw_step(W0, G[pname], np.zeros((r, c)), np.zeros((r, c)), 1, 3e-3, 0.8, 0.95,
                                         1e-10, 0.0)
             assert np.abs(f64(st.get(tid, g.KIND_PARAM)) - W_ref).max() < 1e-6, pname
+
+
+def test_checkpoint_restores_the_step_exactly(torch):
+    """state_dict / load_state_dict (every value, momentum, NorMuon and AdamW
+    state and the AdamW step count) give a fresh context the same next step."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=2, d_model=256, vocab=1000, batch=2, seq_len=200)
+    params = syn.init_params(s, seed=81, extras=True, ve_channels=8)
+    cfg = dict(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+               residual_extras=True, ve_gate_channels=8)
+    specs = syn.param_specs(s, extras=True, ve_channels=8)
+    a = g.GPTStep(**cfg)
+    for tid, (pname, *_r) in enumerate(specs):
+        a.set(tid, params[pname])
+    batches = [(torch.tensor(syn.tokens(s, seed=82 + 2 * i)).cuda(), torch.tensor(syn.targets(s, seed=83 + 2 * i)).cuda())
+               for i in range(2)]
+
+    def step(st, tok, tgt):
+        loss = float(st.fwd_bwd(tok, tgt).item())
+        st.muon_step_normuon(0.02, 0.95, 0.01, 0.9)
+        st.adamw_step(3e-3, 0.8, 0.95, 1e-10, 0.01)
+        st.check()
+        return loss
+
+    step(a, *batches[0])
+    state = a.state_dict()
+    assert state["adam_step"] == 1
+    b = g.GPTStep(**cfg)
+    b.load_state_dict(state)
+    again = b.state_dict()
+    assert again["adam_step"] == 1 and again["tensors"].keys() == state["tensors"].keys()
+    for key, value in state["tensors"].items():
+        assert np.array_equal(again["tensors"][key], value), key
+    la, lb = step(a, *batches[1]), step(b, *batches[1])
+    assert la == lb                                   # identical weights: the same forward, bit for bit
+    for tid, (pname, *_r) in enumerate(specs):
+        # the attention backward adds dq partial sums in no fixed order, so the
+        # updates agree to rounding
+        assert np.allclose(f64(a.get(tid)), f64(b.get(tid)), rtol=1e-5, atol=1e-7), pname
