@@ -486,3 +486,21 @@ def test_finite_difference_gqa_model():
     p = {k: v.astype(np.float64) for k, v in syn.init_params(s, seed=6, std=0.05).items()}
     tok, tgt = syn.tokens(s, seed=7), syn.targets(s, seed=8)
     _fd_check(p, tok, tgt, 1, ["h0.c_qkv", "h0.c_proj", "wte"], n_coords=6)
+
+
+def test_finite_difference_every_scalar():
+    # every residual, x0, backout and smear value (3 layers: the x0 and
+    # residual scales of layers past the first see streams that differ)
+    s, p, tok, tgt = _extras_case(depth=3, std=0.05, seed=14, vocab=40, seq=10)
+    p["scalars"] = syn.random_scalars(s, seed=15).astype(np.float64)
+    _, g, _ = om.fwd_bwd(p, tok, tgt, s.depth)
+    h = 1e-6
+    G = g["scalars"][0]
+    for j in range(p["scalars"].shape[1]):
+        pp = dict(p)
+        sp = p["scalars"].copy(); sp[0, j] += h; pp["scalars"] = sp
+        lp, _ = om.forward(pp, tok, tgt, s.depth, keep=False)
+        sm = p["scalars"].copy(); sm[0, j] -= h; pp["scalars"] = sm
+        lm, _ = om.forward(pp, tok, tgt, s.depth, keep=False)
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - G[j]) <= 1e-6 * max(1.0, np.abs(G).max()), (j, fd, G[j])
