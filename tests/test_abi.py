@@ -116,3 +116,23 @@ def test_null_arguments_are_einval(L):
 def test_split_plan_matches_header_contract(L):
     # the scratch query is pure host arithmetic
     assert L.gpt_op_newton_schulz_scratch(2, 128, 384) > 2 * 128 * 384 * 4 * 2
+
+
+def test_workspace_sizes_follow_the_options(L):
+    """Grouped kv heads shrink the q|k|v parameters; value embeddings add
+    their tables; the residual extras add their saved streams."""
+    import gpt_pretraining_step_b200 as g
+    base = dict(depth=4, batch=2, seq_len=64, vocab=512, d_model=512)
+    p0, s0, a0 = g.workspace_size(g.make_config(**base))
+    p1, s1, a1 = g.workspace_size(g.make_config(**base, n_kv_head=1))
+    d, L = 512, 4
+    # q|k|v goes from [d, 3d] to [d, d + 256] per layer: fp32 master + bf16 copy
+    assert p0 - p1 >= 6 * L * d * (3 * d - (d + 256)) - 256 * 16
+    assert s1 < s0 and a1 < a0
+    p2, s2, a2 = g.workspace_size(g.make_config(**base, ve_gate_channels=8))
+    n_ve = (L + 1) // 2
+    slack = 4096                                # small placeholder allocations when an option is off
+    assert p2 - p0 >= 6 * n_ve * 512 * d - slack        # tables: fp32 master + bf16 copy
+    assert s2 - s0 >= 12 * n_ve * 512 * d - slack       # gradient + AdamW m, v
+    p3, s3, a3 = g.workspace_size(g.make_config(**base, residual_extras=True))
+    assert a3 - a0 >= 4 * L * 2 * 64 * d        # the saved block inputs, fp32
