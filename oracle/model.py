@@ -358,11 +358,18 @@ def backward(params, tok, tgt, cache, n_layer, head_dim=128):
         dsc[2 * n_layer + 2:] = np.einsum("bt,btc->c", dz, e3[:, :, :SMEAR_CHANNELS])
         dx = de.reshape(B * T, -1)
         grads["scalars"] = dsc.reshape(1, -1)
-    V = params["wte"].shape[0]
-    dwte = np.zeros((V, d))
-    np.add.at(dwte, tok.reshape(-1), dx)
-    grads["wte"] = dwte
+    grads["wte"] = embedding_bwd(tok, dx, params["wte"].shape[0])
     return grads
+
+
+def embedding_bwd(tok, dx, vocab):
+    """Gradient of the row copy x0[m] = wte[tok[m]]: row v of the result is
+    the sum of dx[m] over the positions m that hold token v (zero for tokens
+    that do not occur)."""
+    dx = np.asarray(dx, dtype=np.float64).reshape(np.size(tok), -1)
+    dwte = np.zeros((vocab, dx.shape[1]))
+    np.add.at(dwte, np.asarray(tok).reshape(-1), dx)
+    return dwte
 
 
 def fwd_bwd(params, tok, tgt, n_layer, head_dim=128, windows=None):

@@ -223,6 +223,23 @@ def test_embedding_grad_rows():
     assert np.all(g["wte"][absent] == 0.0)
 
 
+def test_embedding_bwd_brute_force_with_repeated_tokens():
+    # the gradient of a row copy, summed position by position in a plain loop;
+    # a skewed id stream puts many positions on the same row
+    rng = np.random.default_rng(7)
+    tok = np.array([3, 3, 0, 5, 3, 5, 3, 9, 3, 0], dtype=np.int32)
+    dx = rng.standard_normal((tok.size, 4))
+    ref = np.zeros((10, 4))
+    for m in range(tok.size):
+        for c in range(4):
+            ref[tok[m], c] += dx[m, c]
+    got = om.embedding_bwd(tok, dx, 10)
+    assert np.allclose(got, ref, rtol=0, atol=1e-14)
+    assert np.all(got[[1, 2, 4, 6, 7, 8]] == 0.0)
+    # a token on every position: the column sums
+    assert np.allclose(om.embedding_bwd(np.full(10, 2), dx, 4)[2], dx.sum(axis=0), atol=1e-14)
+
+
 def test_embedding_forward_is_row_copy():
     s, p, tok, tgt = small_case()
     # depth 0 and zero lm_head: xf = rms(wte[tok]); check via the cache
