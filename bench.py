@@ -35,6 +35,7 @@ sys.path.insert(0, ROOT)
 import synthetic as syn  # noqa: E402
 
 METRIC = "training tokens/sec and MFU (fwd+bwd+Muon step) on 1 B200, d20 seq 2048 bf16"
+N_BATCHES = 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -78,13 +79,6 @@ def peaks():
 
 
 # ------------------------------------------------------------------ FLOPs
-
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# categories that can dominate the d20 step, from one ncu capture of a whole
-# d20 step of the current kernels (profiles/dram_traffic_d20.md).  Used for the
-# roofline's `traffic` only on that workload; null elsewhere.
-NCU_TRAFFIC_D20 = {"dx_gemm": 511.9e6, "attn_bwd": 958.9e6, "dw_gemm": 9.59e9, "attn_fwd": 312.1e6}
-
 
 def model_flops_per_token(s, causal=False):
     """PaLM-style model FLOPs per token: 6 N_matmul + 12 L d T (embeddings
@@ -177,73 +171,138 @@ class ClockSampler:
 
 # --------------------------------------------------------------- CPU oracle
 
-def oracle_sample(s, tokens_per_sample=128, seed=0, ns_kinds=(0, 1, 2, 3), adam_frac=1 / 32):
-    """Times the fp64 oracle on a bounded slice of one step and scales it to the step.
-
-    Returns (scaled step seconds, description, threads): forward+backward of the
-    whole model on one sequence prefix of ``tokens_per_sample`` tokens (scaled by
-    tokens), Newton-Schulz on one matrix per block kind (scaled by the number of
-    matrices of that kind) and AdamW on a fraction of the embedding and lm_head.
-    """
-    import numpy as np
-    from oracle import model as om
-    from oracle import optim as oo
+def _oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count()
-    params = syn.init_params(s, seed=seed)
-    tok = syn.tokens(s)[:1, :tokens_per_sample]
-    tgt = syn.targets(s)[:1, :tokens_per_sample]
-    t0 = time.perf_counter()
-    _, grads, _ = om.fwd_bwd(params, tok, tgt, s.depth)
-    t_fb = time.perf_counter() - t0
-    kinds = ["c_qkv", "c_proj", "c_fc", "mlp_proj"]
-    t_ns = {}
-    for k in ns_kinds:
-        G = grads[f"h0.{kinds[k]}"]
-        W = params[f"h0.{kinds[k]}"]
+        return os.cpu_count()
+
+
+def _layer_params(params, layers):
+    """The embedding, lm_head and the first `layers` blocks of a parameter set."""
+    keep = {"wte", "lm_head"} | {f"h{l}.{n}" for l in range(layers) for n in ("c_qkv", "c_proj", "c_fc", "mlp_proj")}
+    return {k: v for k, v in params.items() if k in keep}
+
+
+class OracleSampler:
+    """Times the fp64 oracle on bounded samples of one step, at the step's real
+    sequence length, and scales them to the whole step.
+
+    Samples: the forward+backward of the head alone (embedding, final norm,
+    lm_head, cross-entropy) on one sequence of T tokens, and of the head plus
+    one decoder block on the same sequence (their difference is one block's
+    time, attention's T^2 term included); Newton-Schulz + Muon on one matrix
+    of a block-matrix kind; AdamW on a fraction of the embedding.  The step
+    estimate is B (L t_block + t_head) + sum over kinds of (matrices of the
+    kind) t_muon + t_adamw scaled to the embedding and lm_head.
+    """
+
+    KINDS = ("c_qkv", "c_proj", "c_fc", "mlp_proj")
+
+    def __init__(self, s, seed=0, adam_frac=1 / 32):
+        from oracle import model as om
+        from oracle import optim as oo
+        self.om, self.oo = om, oo
+        self.s = s
+        self.params = _layer_params(syn.init_params(syn.make_shape(depth=1, batch=1, seq_len=s.seq_len,
+                                                                   vocab=s.vocab, d_model=s.d_model), seed=seed), 1)
+        self.tok = syn.tokens(s)[:1]
+        self.tgt = syn.targets(s)[:1]
+        self.adam_frac = adam_frac
+        self.times = {}
+
+    def run(self, what):
+        """Run one sample ("head", "block", "muon:<kind>" or "adamw"); returns its seconds."""
+        import numpy as np
+        om, oo, p = self.om, self.oo, self.params
         t0 = time.perf_counter()
-        oo.muon_step(W, G, np.zeros_like(G), 0.02)
-        t_ns[k] = time.perf_counter() - t0
-    n = int(s.vocab * s.d_model * adam_frac)
-    p = params["wte"].ravel()[:n].astype(np.float64)
-    g = grads["wte"].ravel()[:n]
-    t0 = time.perf_counter()
-    oo.adamw_step(p, g, np.zeros(n), np.zeros(n), 1, 3e-3)
-    t_ad = time.perf_counter() - t0
-    mean_ns = sum(t_ns.values()) / len(t_ns)
-    step = t_fb * s.tokens / tokens_per_sample + sum(s.depth * t_ns.get(k, mean_ns) for k in range(4)) \
-        + t_ad * 2 / adam_frac
-    desc = (f"fp64 oracle: fwd+bwd of all {s.depth} layers on 1x{tokens_per_sample} tokens scaled x"
-            f"{s.tokens // tokens_per_sample}; Newton-Schulz on {len(t_ns)} matrices scaled to {4 * s.depth}; "
-            f"AdamW on {adam_frac:.3f} of the embedding scaled to wte+lm_head")
-    return step, desc, threads, t_fb + sum(t_ns.values()) + t_ad
+        if what == "head":
+            om.fwd_bwd(_layer_params(p, 0), self.tok, self.tgt, 0)
+        elif what == "block":
+            om.fwd_bwd(p, self.tok, self.tgt, 1)
+        elif what.startswith("muon:"):
+            W = p[f"h0.{what[5:]}"].astype(np.float64)
+            G = syn.gaussian(W.shape, seed=5)
+            oo.muon_step(W, G, np.zeros_like(W), 0.02)
+        elif what == "adamw":
+            n = int(self.s.vocab * self.s.d_model * self.adam_frac)
+            pp = p["wte"].ravel()[:n].astype(np.float64)
+            oo.adamw_step(pp, syn.gaussian((n,), seed=6).astype(np.float64), np.zeros(n), np.zeros(n), 1, 3e-3)
+        else:
+            raise ValueError(what)
+        dt = time.perf_counter() - t0
+        self.times.setdefault(what, []).append(dt)
+        return dt
+
+    def schedule(self):
+        return ["head", "block"] + [f"muon:{k}" for k in self.KINDS] + ["adamw"]
+
+    def step_seconds(self):
+        s, t = self.s, {k: statistics.mean(v) for k, v in self.times.items()}
+        block = max(t["block"] - t["head"], 0.0)
+        nmat = {"c_qkv": s.depth, "c_proj": s.depth, "c_fc": s.depth, "mlp_proj": s.depth}
+        muon = sum(nmat[k] * t[f"muon:{k}"] for k in self.KINDS)
+        return s.batch * (s.depth * block + t["head"]) + muon + t["adamw"] * 2 / self.adam_frac
+
+    def describe(self):
+        s = self.s
+        return (f"fp64 oracle at T={s.seq_len}: fwd+bwd of the head alone and of the head plus one block on one "
+                f"sequence (block time = difference, scaled x{s.depth} blocks x{s.batch} sequences), Muon on one "
+                f"matrix per kind (x{s.depth} each), AdamW on {self.adam_frac:.4f} of the embedding (scaled to wte "
+                f"and lm_head)")
+
+
+def oracle_sample(s):
+    """(step seconds, description, threads, seconds of CPU work) for the cpu_baseline."""
+    o = OracleSampler(s)
+    spent = sum(o.run(w) for w in o.schedule())
+    return o.step_seconds(), o.describe(), _oracle_threads(), spent
+
+
+def bench_config(a, s, world):
+    """The `config` object of both arms' JSON lines (the same workload)."""
+    return {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)", "global_batch": s.batch * world,
+            "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
+            "precision": a.precision,
+            "parallelism": f"dp{world}" + ("+sharded-optimizer" if a.shard_optimizer and world > 1 else ""),
+            "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
+            "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
+            "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
+                          else "full causal"),
+            "residual_extras": bool(a.residual_extras), "value_embed_channels": a.value_embeds,
+            "batches": f"{N_BATCHES} resident seeded batches, used in turn"}
 
 
 def run_reference(a):
+    """The oracle as the reference arm: each step is one bounded sample of the
+    workload (the samples of OracleSampler in turn), timed for real; `value`
+    is the workload's tokens/s estimated from the mean time of each sample."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     s = syn.config_shape(a.config)
-    times, wall, threads, desc = [], 0.0, 1, ""
-    for i in range(a.warmup + a.steps):
-        step, desc, threads, spent = oracle_sample(s, tokens_per_sample=64, ns_kinds=(i % 4,), adam_frac=1 / 64)
-        if i >= a.warmup:
-            times.append(step)
-            wall += spent
-    st = statistics.mean(times)
-    value = s.tokens / st
-    sample = desc + f"; {a.steps} timed steps, {wall:.1f} s of CPU work"
+    o = OracleSampler(s, adam_frac=1 / 256)
+    sched = o.schedule()
+    # each step runs every sample once; warm-up steps are discarded
+    for _ in range(a.warmup):
+        for w in sched:
+            o.run(w)
+    o.times = {}
+    timed = [sum(o.run(w) for w in sched) for _ in range(a.steps)]
+    ms = statistics.mean(timed) * 1e3
+    value = s.tokens / o.step_seconds()
+    sample = o.describe() + (f"; each timed step runs every sample once ({a.steps} steps, {sum(timed):.1f} s of "
+                             f"CPU work); value = tokens of the workload's step / its estimated time")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": a.gpus,
-        "steps": a.steps, "warmup": a.warmup, "ms_per_step": st * 1e3, "higher_is_better": True,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{a.config} GPT step", "global_batch": s.batch, "seq_len": s.seq_len,
-                   "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": sample},
+        "config": bench_config(a, s, 1),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": _oracle_threads(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "estimated_step_seconds": o.step_seconds(),
     }), flush=True)
 
 
@@ -272,12 +331,17 @@ def run_ours(a):
                    ns_tf32_steps=a.ns_tf32_steps, seed=1234, stream=stream,
                    precision=1 if a.precision == "fp8" else 0, window_pattern=a.window_pattern,
                    short_window=a.short_window, residual_extras=a.residual_extras, ve_gate_channels=a.value_embeds)
-    tok = torch.tensor(syn.tokens(s, seed=dp.rank_seed(1, rank))).cuda()
-    tgt = torch.tensor(syn.targets(s, seed=dp.rank_seed(2, rank))).cuda()
+    # a few resident seeded batches used in turn, so the printed loss is not
+    # the loss of one memorised batch
+    batches = [(torch.tensor(syn.tokens(s, seed=dp.rank_seed(1 + 100 * i, rank))).cuda(),
+                torch.tensor(syn.targets(s, seed=dp.rank_seed(2 + 100 * i, rank))).cuda()) for i in range(N_BATCHES)]
     grads = st.grad_view() if world > 1 else None
     hp = dict(muon=(0.02, 0.95, 0.0), adam=(3e-3, 0.8, 0.95, 1e-10, 0.0))
+    counter = [0]
 
     def step():
+        tok, tgt = batches[counter[0] % N_BATCHES]
+        counter[0] += 1
         st.fwd_bwd(tok, tgt)
         if a.shard_optimizer and world > 1:
             dp.sharded_optimizer_step(st, s.depth, muon=hp["muon"], adam=hp["adam"],
@@ -291,16 +355,19 @@ def run_ours(a):
             st.muon_step_normuon(*hp["muon"], a.normuon)
         st.adamw_step(*hp["adam"])
 
-    # warm-up; the last warm-up step records every launch category
+    # warm-up; the first step's loss is kept (the initial weights give a known
+    # value) and the last warm-up step records every launch category
+    first_loss = None
     for i in range(a.warmup):
         if i == a.warmup - 1:
             st.profile_enable(g.PROF_CATEGORIES)
         step()
+        if i == 0:
+            first_loss = float(st.loss[0].item())
     torch.cuda.synchronize()
     st.check()
     prof = st.profile_read()
     work = category_work(s)
-    tensor_cats = [c for c in prof if work.get(c, ("", 0))[0] == "tensor"]
     dominant = max(prof, key=lambda c: prof[c][0]) if prof else None
     st.profile_enable([dominant] if dominant else [])
 
@@ -343,12 +410,11 @@ def run_ours(a):
         if kind == "tensor":
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e12
             peak = pk["bf16_tflops_sustained"]
-            traffic = (NCU_TRAFFIC_D20.get(dominant)
-                       if a.config == "d20" and a.precision == "bf16" and a.ns_tf32_steps < 0 else None)
+            # DRAM traffic needs hardware counters (an ncu capture), which a timed
+            # run does not take: reported as null here
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": traffic, "kernel": dominant,
-                    "peak_source": f"{pk_src} bf16_tflops_sustained",
-                    "traffic_source": "ncu dram bytes per launch, profiles/dram_traffic_d20.md" if traffic else None}
+                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
+                    "peak_source": f"{pk_src} bf16_tflops_sustained"}
         else:
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e9
             peak = pk["hbm_gbs"]
@@ -382,6 +448,28 @@ def run_ours(a):
             e2e["ms_per_step"] = dp.max_over_ranks(e2e["ms_per_step"], device="cuda")
             e2e["value"] = tokens_per_step / (e2e["ms_per_step"] / 1e3)
 
+    # Newton-Schulz over every block matrix on its own (the Muon step without
+    # the forward and backward), timed with events on the library's stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.profile_enable(["ns_gemm"])
+    e0.record(stream)
+    st.muon_step(*hp["muon"])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ns_prof = st.profile_read()
+    st.profile_enable([])
+    ns_ms = ns_prof.get("ns_gemm", (0.0, 0))[0]
+    ns_alone = {"muon_step_ms": e0.elapsed_time(e1), "newton_schulz_ms": ns_ms,
+                "newton_schulz_tflops": work["ns_gemm"][1] / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None,
+                "matrices": 4 * s.depth,
+                "shapes": [[s.d_model, s.qkv_cols], [s.d_model, s.d_model], [s.d_model, s.mlp_hidden],
+                           [s.mlp_hidden, s.d_model]]}
+    sig2 = 0.02 ** 2 * s.d_model
+    first_loss_expect = math.log(s.vocab) + sig2 / 2 - (math.exp(sig2) - 1) / (2 * s.vocab)
+    clock_peak = None
+    if clocks.get("sm_mhz") and clocks.get("sm_max_mhz"):
+        clock_peak = 2.25e15 * clocks["sm_mhz"] / clocks["sm_max_mhz"]
+
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         step_s, desc, threads, spent = oracle_sample(s)
@@ -393,16 +481,13 @@ def run_ours(a):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": a.steps,
             "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if a.precision == "bf16" else "bf16+e4m3", "data": "synthetic",
-            "config": {"workload": f"{a.config} GPT step (fwd+bwd+{optim_name(a)}+AdamW)",
-                       "global_batch": s.batch * world,
-                       "seq_len": s.seq_len, "depth": s.depth, "d_model": s.d_model, "vocab": s.vocab,
-                       "parallelism": f"dp{world}" + ("+sharded-optimizer" if a.shard_optimizer and world > 1 else ""),
-                       "ns_operands": "fp16" if a.ns_tf32_steps < 0 else f"tf32 x{a.ns_tf32_steps} + bf16",
-                       "l2": "no flush: step working set (activations ~20 GB) far exceeds the 126 MB L2",
-                       "attention": (f"windows {a.window_pattern} (S = {a.short_window} tokens)" if a.window_pattern
-                                     else "full causal"),
-                       "residual_extras": bool(a.residual_extras), "value_embed_channels": a.value_embeds},
+            "config": bench_config(a, s, world),
             "mfu": mfu_sust, "mfu_vs_nominal_2250": mfu_nominal,
+            "mfu_vs_dense_at_sampled_clock": (fpt * s.tokens / (ms / 1e3) / clock_peak) if clock_peak else None,
+            "first_step_loss": first_loss, "first_step_loss_closed_form": first_loss_expect,
+            "first_step_loss_ok": (first_loss is not None and
+                                   abs(first_loss - first_loss_expect) / first_loss_expect <= 1e-2),
+            "newton_schulz_alone": ns_alone,
             "mfu_peak": f"{pk_src} bf16_tflops_sustained {pk['bf16_tflops_sustained']}",
             "model_tflop_per_step": fpt * s.tokens / 1e12,
             "mfu_attention_causal_half": mfu_causal,

@@ -29,7 +29,8 @@ ABI_FUNCTIONS = [
     "gpt_op_matmul_bf16", "gpt_op_matmul_tf32", "gpt_op_quantize_e4m3", "gpt_op_matmul_fp8",
     "gpt_op_attention_fwd", "gpt_op_attention_bwd", "gpt_op_attention_fwd_ex", "gpt_op_attention_bwd_ex",
     "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
-    "gpt_op_newton_schulz_noalloc", "gpt_get_adam_step", "gpt_set_adam_step",
+    "gpt_op_newton_schulz_noalloc", "gpt_get_adam_step", "gpt_set_adam_step", "gpt_set_wait_limit",
+    "gpt_op_check", "gpt_op_set_wait_limit", "gpt_op_embedding_bwd_scratch", "gpt_op_embedding_bwd",
 ]
 
 
@@ -86,6 +87,9 @@ def lib():
             "gpt_get_adam_step": (i32, [vp, ctypes.POINTER(ctypes.c_int64)]),
             "gpt_set_adam_step": (i32, [vp, ctypes.c_int64]),
             "gpt_check": (i32, [vp]),
+            "gpt_set_wait_limit": (i32, [vp, ctypes.c_longlong]),
+            "gpt_op_check": (i32, [vp]),
+            "gpt_op_set_wait_limit": (i32, [ctypes.c_longlong]),
             "gpt_launch_count": (ctypes.c_int64, [vp]),
             "gpt_profile_enable": (i32, [vp, ctypes.c_uint32]),
             "gpt_profile_read": (i32, [vp, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64)]),
@@ -100,6 +104,8 @@ def lib():
             "gpt_op_attention_fwd_ex": (i32, [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "gpt_op_attention_bwd_ex": (i32, [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]),
             "gpt_op_rmsnorm_fwd": (i32, [vp, vp, vp, i32, i32, vp]),
+            "gpt_op_embedding_bwd_scratch": (sz, [i32, i32]),
+            "gpt_op_embedding_bwd": (i32, [vp, vp, vp, i32, i32, i32, i32, vp, vp]),
             "gpt_op_newton_schulz_scratch": (sz, [i32, i32, i32]),
             "gpt_op_newton_schulz": (i32, [vp, vp, i32, i32, i32, i32, vp, vp]),
             "gpt_op_newton_schulz_noalloc": (i32, [vp, vp, i32, i32, i32, i32, vp]),
@@ -178,6 +184,7 @@ class GPTStep:
     def fwd_bwd(self, tokens, targets, accumulate=False, loss_out=None):
         out = self.loss if loss_out is None else loss_out
         _check(lib().gpt_fwd_bwd(self.h, _ptr(tokens), _ptr(targets), _ptr(out), int(bool(accumulate))))
+        self._join_current_stream()
         return out[0] if loss_out is None else out
 
     def muon_step(self, lr=0.02, momentum=0.95, weight_decay=0.0):
@@ -237,10 +244,21 @@ class GPTStep:
         return (self.d_model,) if kind == KIND_NORMUON_V else (r, c)
 
     def get(self, tid, kind=KIND_PARAM):
+        """A copy of the tensor, ordered before later work on torch's current
+        stream (the copy runs on the context's stream)."""
         import torch
         out = torch.empty(self._shape(tid, kind), dtype=torch.float32, device=self.bufs[0].device)
         _check(lib().gpt_get_tensor(self.h, tid, kind, _ptr(out)))
+        self._join_current_stream()
         return out
+
+    def _join_current_stream(self):
+        # work queued on the context's stream (a copy into a torch tensor)
+        # completes before anything torch's current stream runs next
+        import torch
+        cur = torch.cuda.current_stream(self.bufs[0].device)
+        if cur.cuda_stream != self.stream.cuda_stream:
+            cur.wait_stream(self.stream)
 
     def set(self, tid, value, kind=KIND_PARAM):
         import torch
@@ -262,10 +280,15 @@ class GPTStep:
         import torch
         out = torch.empty((self.cfg.batch, self.cfg.seq_len), dtype=torch.float32, device=self.bufs[0].device)
         _check(lib().gpt_get_row_loss(self.h, _ptr(out)))
+        self._join_current_stream()
         return out
 
     def check(self):
         return _check(lib().gpt_check(self.h))
+
+    def set_wait_limit(self, cycles):
+        """Bound of the kernels' device-side waits in SM cycles (<= 0: the default)."""
+        _check(lib().gpt_set_wait_limit(self.h, int(cycles)))
 
     # -- checkpoint
     def _state_kinds(self, tid):
@@ -311,6 +334,17 @@ class GPTStep:
 
 
 # ---------------------------------------------------------------- op level
+
+def op_check(stream=None):
+    """Synchronise the stream and raise GptError (GPT_ETIMEOUT) if a bounded
+    device wait of an op-level call expired since the last check."""
+    return _check(lib().gpt_op_check(_stream(stream)))
+
+
+def op_set_wait_limit(cycles):
+    """Bound of the device-side waits of later op-level calls (<= 0: default)."""
+    _check(lib().gpt_op_set_wait_limit(int(cycles)))
+
 
 def matmul_bf16(A, B, M, N, K, batch=1, a_trans=False, b_trans=False, out=None, stream=None):
     import torch
@@ -378,6 +412,17 @@ def rmsnorm_fwd(x, stream=None):
     r = torch.empty((M,), dtype=torch.float32, device=x.device)
     _check(lib().gpt_op_rmsnorm_fwd(_ptr(x), _ptr(y), _ptr(r), M, d, _stream(stream)))
     return y, r
+
+
+def embedding_bwd(tokens, dx, vocab, dwte=None, accumulate=False, stream=None):
+    """dwte [vocab, d] (+)= rows of dx [M, d] scattered by token (int32 [M])."""
+    import torch
+    M, d = dx.shape
+    out = torch.zeros((vocab, d), dtype=torch.float32, device=dx.device) if dwte is None else dwte
+    scratch = torch.empty(max(lib().gpt_op_embedding_bwd_scratch(M, d), 256), dtype=torch.uint8, device=dx.device)
+    _check(lib().gpt_op_embedding_bwd(_ptr(tokens), _ptr(dx), _ptr(out), M, d, vocab, int(bool(accumulate)),
+                                      _ptr(scratch), _stream(stream)))
+    return out
 
 
 def newton_schulz(G, tf32_steps=-1, stream=None):

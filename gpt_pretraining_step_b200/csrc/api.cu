@@ -241,7 +241,7 @@ void make_plan(const Dims& D, Plan& P) {
   P.Dv = ab.take(M * H * 4);
   P.dqkv = ab.take(L * M * qc * 2);
   P.splitk = ab.take(std::max<size_t>(sk, 4) * 4);
-  P.embws = ab.take(embed_bwd_workspace(D.M));
+  P.embws = ab.take(embed_bwd_workspace(D.M, std::max(d, kvd)));
   const size_t xelems = std::max({L * d * qc, L * d * d, 2 * L * d * F});
   P.X0 = ab.take(xelems * 4);
   P.X1 = ab.take(xelems * 4);
@@ -339,6 +339,7 @@ struct gpt_ctx {
   uint8_t* sbuf;
   uint8_t* abuf;
   cudaStream_t stream;
+  long long wait_cycles = 0;   // bound of the kernels' device-side waits (<= 0: the default)
   long long adam_step = 0;
   int64_t launches = 0;
   // event profiler
@@ -446,6 +447,12 @@ GemmCall base_call(int M, int N, int K) {
   return c;
 }
 
+// gemm_run with the caller's bound on the kernel's waits
+cudaError_t run_gemm(GemmCall& g, cudaStream_t s, long long wait_cycles) {
+  g.p.wait_cycles = wait_cycles;
+  return gemm_run(g, s);
+}
+
 // fp32 output [M][N] (contiguous), optionally split over K with a deterministic reduce.
 int run_f32(gpt_ctx* c, GemmCall g, float* out, bool accumulate, int splits, int cat) {
   ProfScope ps(c, cat);
@@ -457,7 +464,7 @@ int run_f32(gpt_ctx* c, GemmCall g, float* out, bool accumulate, int splits, int
     g.splits = 1;
     g.p.out = out;
     g.p.ldo = g.N;
-    GPT_CK(gemm_run(g, c->stream));
+    GPT_CK(run_gemm(g, c->stream, c->wait_cycles));
     c->launches += 1;
     return GPT_OK;
   }
@@ -469,7 +476,7 @@ int run_f32(gpt_ctx* c, GemmCall g, float* out, bool accumulate, int splits, int
   g.p.out = part;
   g.p.ldo = g.N;
   g.p.split_stride = n;
-  GPT_CK(gemm_run(g, c->stream));
+  GPT_CK(run_gemm(g, c->stream, c->wait_cycles));
   launch_splitk_reduce(part, g.p.splits, n, n, out, accumulate, c->stream);
   c->launches += 2;
   return GPT_OK;
@@ -578,7 +585,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.p.f32a = rq + static_cast<size_t>(l) * M * H;
       g.p.f32b = rk + static_cast<size_t>(l) * M * H;
       g.p.rope = rope + static_cast<size_t>(D.T) * 64; g.p.T = D.T; g.p.H = H; g.p.Hkv = D.Hkv; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     if (D.ve_slot(l) >= 0) {
       // value embedding: v += 3 sigmoid(gate) ve[tok] per head
@@ -590,7 +597,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_FWD);
-      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H);
+      launch_attn_fwd(ql, kl, vl, ol, lsel, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H,
+                      c->wait_cycles);
     }
     {
       GemmCall g = base_call(M, d, d);
@@ -599,7 +607,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       ProfScope ps(c, GPT_PROF_PROJ_GEMM);
       g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
       g.p.out = x; g.p.ldo = d; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
@@ -612,7 +620,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       ProfScope ps(c, GPT_PROF_FC_GEMM);
       g.epi = EPI_RELU2; g.out_es = 2; g.aux_es = 2;
       g.p.out = hl; g.p.ldo = F; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     {
       GemmCall g = base_call(M, d, F);
@@ -621,7 +629,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       ProfScope ps(c, GPT_PROF_DOWN_GEMM);
       g.epi = EPI_ACC; g.out_es = 4; g.aux_es = 4;
       g.p.out = x; g.p.ldo = d; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     c->launches += 7;
   }
@@ -651,7 +659,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.epi = EPI_LOGITS; g.out_es = 2; g.aux_es = 2;
       g.p.out = z; g.p.ldo = V;
       g.p.f32a = c->A<float>(P.stats); g.p.f32b = c->A<float>(P.zt); g.p.tgt = tgt + r0; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     {
       ProfScope ps(c, GPT_PROF_CE_FINISH);
@@ -717,7 +725,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.ldb = d;   // B(n = F index, k = d index)
       g.epi = EPI_DRELU2; g.out_es = 2; g.aux_es = 2;
       g.p.out = du; g.p.ldo = F; g.p.aux = hl; g.p.ld_aux = F; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
       c->launches += 1;
     }
     {
@@ -740,13 +748,14 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.ldb = d;
       g.epi = EPI_STORE; g.out_es = 2; g.aux_es = 2;
       g.p.out = dy; g.p.ldo = d; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
       c->launches += 1;
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H);
+                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H,
+                      c->wait_cycles);
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
@@ -765,7 +774,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       launch_embed_bwd(tok, dqf, c->VeG(vs), M, 128 * D.Hkv, V, c->A<void>(P.embws), acc, s);
       launch_ve_gate_grad(xn1 + l * Md, c->A<float>(P.vedz), c->A<float>(P.vepart), c->GateG(vs), M, d, D.Hkv,
                           D.veC, acc, s);
-      c->launches += 3 + 2 * ((M + 32767) / 32768);
+      c->launches += 3 + 3 * ((M + 32767) / 32768);
     }
     {
       GemmCall g = base_call(M, d, D.qc);   // dxn1 = dqkv W_qkv^T
@@ -815,7 +824,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.B = w.b; g.b_mn = true; g.ldb = w.ldb; g.b_bs = w.b_bs;
       g.epi = acc ? EPI_ACC : EPI_STORE; g.out_es = 4; g.aux_es = 4;
       g.p.out = w.out; g.p.ldo = w.cols; g.p.out_bs = 1ll * w.rows * w.cols; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     c->launches += 4;
   }
@@ -833,7 +842,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     ProfScope ps(c, GPT_PROF_EMBED);
     launch_embed_bwd(tok, demb, c->G(0), M, d, V, c->A<void>(P.embws), acc, s);
   }
-  c->launches += 2 * ((M + 32767) / 32768);
+  c->launches += 3 * ((M + 32767) / 32768);
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -843,7 +852,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
 // t < n_tf32, then on bf16.  A tf32 step reads X^T (XT0, [z][c][r]) as its
 // K-major B operand and, when the next step is tf32 too, writes X'^T beside X'.
 int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* XT0, void* XT1, void* Ab,
-                  void* Bb, int n_tf32, cudaStream_t s, int* err, void** out, int* out_es, int64_t* launches) {
+                  void* Bb, int n_tf32, cudaStream_t s, int* err, void** out, int* out_es, int64_t* launches,
+                  long long wait_cycles) {
   ProfScope ps(pc, GPT_PROF_NS_GEMM);
   const double (*kPolarCoef)[3] = polar_coefficients();
   if (n_tf32 < 0) {
@@ -866,7 +876,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         g.bn = 128; g.sym = true; g.epi = EPI_STORE;
         g.out_es = 2; g.out_f16 = true; g.aux_es = 2; g.aux_f16 = true;
         g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
-        GPT_CK(gemm_run(g, s));
+        GPT_CK(run_gemm(g, s, wait_cycles));
       }
       {
         GemmCall g = base_call(r, r, r);    // B = b A + c A A
@@ -878,7 +888,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
         g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
         g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;
-        GPT_CK(gemm_run(g, s));
+        GPT_CK(run_gemm(g, s, wait_cycles));
       }
       {
         GemmCall g = base_call(r, cc, r);   // X' = a X + B X
@@ -890,7 +900,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         if (!last) g.p.out2 = nxtH;
         g.p.aux = cur; g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
         g.p.alpha = static_cast<float>(a); g.p.beta = 1.f; g.p.err = err;
-        GPT_CK(gemm_run(g, s));
+        GPT_CK(run_gemm(g, s, wait_cycles));
       }
       *launches += 3;
       std::swap(cur, nxt);
@@ -917,7 +927,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
       g.B = cur; g.ldb = cc; g.b_bs = 1ll * r * cc;
       g.bn = 128; g.sym = true; g.epi = EPI_STORE; g.out_es = es; g.aux_es = es;
       g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, wait_cycles));
     }
     {
       GemmCall g = base_call(r, r, r);    // B = b A + c A A
@@ -928,7 +938,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
       g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
       g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
       g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, wait_cycles));
     }
     {
       GemmCall g = base_call(r, cc, r);   // X' = a X + B X
@@ -947,7 +957,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
       }
       g.p.aux = cur; g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
       g.p.alpha = static_cast<float>(a); g.p.beta = 1.f; g.p.err = err;
-      GPT_CK(gemm_run(g, s));
+      GPT_CK(run_gemm(g, s, wait_cycles));
     }
     *launches += 3;
     std::swap(cur, nxt);
@@ -1105,7 +1115,7 @@ static int muon_update(gpt_ctx* c, float lr, float momentum, float weight_decay,
     void* res = nullptr;
     int res_es = es0;
     rc = newton_schulz(c, bt.nz, d, bt.cc, X0, X1, XT0, XT1, Ab, Bb, D.n_tf32, s, c->err(), &res, &res_es,
-                       &c->launches);
+                       &c->launches, c->wait_cycles);
     if (rc) return rc;
     for (int i = 0; i < bt.nm; ++i) {
       ProfScope ps(c, GPT_PROF_MUON_ELEM);
@@ -1421,6 +1431,61 @@ int gpt_profile_read(gpt_ctx* c, double* ms, int64_t* launches) {
 void gpt_destroy(gpt_ctx* c) { delete c; }
 
 // ------------------------------------------------------------ op-level calls
+//
+// The op-level entry points have no context, so the library keeps their
+// device error word itself: one word per device (a __device__ variable
+// exists once on every GPU that loads the library), ORed into by every
+// op-level kernel and read and cleared by gpt_op_check.  Their wait bound is
+// one process-wide value.
+
+}  // extern "C"
+
+namespace {
+
+__device__ int g_op_err_word[4];
+std::atomic<long long> g_op_wait_cycles{0};
+
+// Device address of the op-level error word on the current device, looked
+// up on every call (cheap once the library's device code is loaded), so a
+// context created after a device reset gets its own address.
+int op_err(int** out) {
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_op_err_word);
+  if (e != cudaSuccess || !p)
+    return fail(GPT_ECUDA, std::string("cudaGetSymbolAddress of the op-level error word: ") + cudaGetErrorString(e));
+  *out = static_cast<int*>(p);
+  return GPT_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gpt_op_set_wait_limit(long long cycles) {
+  g_op_wait_cycles.store(cycles > 0 ? cycles : 0);
+  return GPT_OK;
+}
+
+int gpt_op_check(void* stream) {
+  GPT_CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int* word = nullptr;
+  int rc = op_err(&word);
+  if (rc) return rc;
+  int flag = 0;
+  GPT_CK(cudaMemcpy(&flag, word, sizeof(int), cudaMemcpyDeviceToHost));
+  if (flag) GPT_CK(cudaMemset(word, 0, sizeof(int)));
+  if (flag & ERRF_TIMEOUT) return fail(GPT_ETIMEOUT, "a bounded device wait of an op-level call expired");
+  if (flag & ERRF_TOKEN_RANGE) return fail(GPT_ERANGE, "token or target id outside [0, vocab)");
+  if (flag) return fail(GPT_ECUDA, "op-level device error flag set");
+  return GPT_OK;
+}
+
+int gpt_set_wait_limit(gpt_ctx* c, long long cycles) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  c->wait_cycles = cycles > 0 ? cycles : 0;
+  return GPT_OK;
+}
 
 int gpt_op_matmul_bf16(const void* A, const void* B, float* C, int M, int N, int K, int batch, int a_trans,
                        int b_trans, void* stream) {
@@ -1433,7 +1498,9 @@ int gpt_op_matmul_bf16(const void* A, const void* B, float* C, int M, int N, int
   g.B = B; g.b_mn = b_trans == 0; g.ldb = b_trans ? K : N; g.b_bs = 1ll * K * N;
   g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
   g.p.out = C; g.p.ldo = N; g.p.out_bs = 1ll * M * N;
-  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  int rc = op_err(&g.p.err);
+  if (rc) return rc;
+  GPT_CK(run_gemm(g, static_cast<cudaStream_t>(stream), g_op_wait_cycles.load()));
   return GPT_OK;
 }
 
@@ -1447,7 +1514,9 @@ int gpt_op_matmul_tf32(const float* A, const float* B, float* C, int M, int N, i
   g.B = B; g.ldb = K;
   g.bn = 128; g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
   g.p.out = C; g.p.ldo = N;
-  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  int rc = op_err(&g.p.err);
+  if (rc) return rc;
+  GPT_CK(run_gemm(g, static_cast<cudaStream_t>(stream), g_op_wait_cycles.load()));
   return GPT_OK;
 }
 
@@ -1472,7 +1541,9 @@ int gpt_op_matmul_fp8(const void* A, const void* B, float* C, int M, int N, int 
   g.B = B; g.b_mn = b_trans == 0; g.ldb = b_trans ? K : N;
   g.epi = EPI_STORE; g.out_es = 4; g.aux_es = 4;
   g.p.out = C; g.p.ldo = N; g.p.dq_a = inv_a; g.p.dq_b = inv_b;
-  GPT_CK(gemm_run(g, static_cast<cudaStream_t>(stream)));
+  int rc = op_err(&g.p.err);
+  if (rc) return rc;
+  GPT_CK(run_gemm(g, static_cast<cudaStream_t>(stream), g_op_wait_cycles.load()));
   return GPT_OK;
 }
 
@@ -1482,8 +1553,12 @@ int gpt_op_attention_fwd_ex(const void* q, const void* k, const void* v, void* o
   if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
   if (Hkv < 1 || H % Hkv) return fail(GPT_EINVAL, "kv heads must divide the query heads");
   if (static_cast<long long>(B) * H * T > (1ll << 31) - 1) return fail(GPT_EINVAL, "attention too large");
+  int* err = nullptr;
+  int rc = op_err(&err);
+  if (rc) return rc;
   launch_attn_fwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
-                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream), nullptr, Hkv, window);
+                  static_cast<bf16*>(o), lse, B, H, T, static_cast<cudaStream_t>(stream), err, Hkv, window, nullptr,
+                  0, g_op_wait_cycles.load());
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -1500,10 +1575,13 @@ int gpt_op_attention_bwd_ex(const void* q, const void* k, const void* v, const v
   if (B < 1 || H < 1 || T < 1) return fail(GPT_EINVAL, "bad attention shape");
   if (Hkv < 1 || H % Hkv) return fail(GPT_EINVAL, "kv heads must divide the query heads");
   if (static_cast<long long>(B) * H * T > (1ll << 31) - 1) return fail(GPT_EINVAL, "attention too large");
+  int* err = nullptr;
+  int rc = op_err(&err);
+  if (rc) return rc;
   launch_attn_bwd(static_cast<const bf16*>(q), static_cast<const bf16*>(k), static_cast<const bf16*>(v),
                   static_cast<const bf16*>(o), static_cast<const bf16*>(dout), lse, Dscratch, dq,
-                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream), nullptr,
-                  Hkv, window);
+                  static_cast<bf16*>(dk), static_cast<bf16*>(dv), B, H, T, static_cast<cudaStream_t>(stream), err,
+                  Hkv, window, nullptr, 0, g_op_wait_cycles.load());
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -1522,10 +1600,27 @@ int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void*
   return GPT_OK;
 }
 
+size_t gpt_op_embedding_bwd_scratch(int M, int d) {
+  return M < 0 || d < 128 || d % 128 ? 0 : embed_bwd_workspace(M, d);
+}
+
+int gpt_op_embedding_bwd(const int32_t* tokens, const float* dx, float* dwte, int M, int d, int vocab, int accumulate,
+                         void* scratch, void* stream) {
+  if (!tokens || !dx || !dwte || !scratch) return fail(GPT_EINVAL, "null pointer");
+  if (M < 0 || d < 128 || d % 128 || vocab < 1 || vocab > 131072)
+    return fail(GPT_EINVAL, "bad embedding shape (d: a multiple of 128; vocab in [1, 131072])");
+  if ((reinterpret_cast<uintptr_t>(dx) | reinterpret_cast<uintptr_t>(dwte)) & 15)
+    return fail(GPT_EINVAL, "dx and dwte must be 16-byte aligned");
+  if (reinterpret_cast<uintptr_t>(scratch) & (kAlign - 1)) return fail(GPT_EINVAL, "scratch must be 256-byte aligned");
+  launch_embed_bwd(tokens, dx, dwte, M, d, vocab, scratch, accumulate != 0, static_cast<cudaStream_t>(stream));
+  GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
 size_t gpt_op_newton_schulz_scratch(int batch, int rows, int cols) {
   const size_t r = std::min(rows, cols), cc = std::max(rows, cols), n = static_cast<size_t>(batch) * r * cc;
   return 4 * al(n * 4) + 2 * al(static_cast<size_t>(batch) * r * r * 4) + al(batch * 4) +
-         al(muon_norm_workspace(batch)) + al(n * 2) + al(16);
+         al(muon_norm_workspace(batch)) + al(n * 2);
 }
 
 int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols, int tf32_steps, void* scratch,
@@ -1549,9 +1644,10 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
   float* inv = reinterpret_cast<float*>(base + b.take(batch * 4));
   void* normws = base + b.take(muon_norm_workspace(batch));
   bf16* Xb = reinterpret_cast<bf16*>(base + b.take(n * 2));
-  int* err = reinterpret_cast<int*>(base + b.take(16));
+  int* err = nullptr;
+  int rc = op_err(&err);
+  if (rc) return rc;
   GPT_CK(cudaMemsetAsync(X, 0, n * 4, s));
-  GPT_CK(cudaMemsetAsync(err, 0, 16, s));
   launch_muon_momentum(X, G, static_cast<long long>(rows) * cols, batch, 0.f, 1e-7f, inv, normws, s);
   const int es0 = tf32_steps != 0 ? 4 : 2;
   // X (r x cc) and, for tf32 steps, its transpose or, for fp16 steps, its fp16
@@ -1567,8 +1663,8 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
   void* res = nullptr;
   int res_es = es0;
   int64_t launches = 0;
-  int rc = newton_schulz(nullptr, batch, r, cc, X0, X1, XT0, XT1, Ab, Bb, tf32_steps, s, err, &res, &res_es,
-                         &launches);
+  rc = newton_schulz(nullptr, batch, r, cc, X0, X1, XT0, XT1, Ab, Bb, tf32_steps, s, err, &res, &res_es,
+                     &launches, g_op_wait_cycles.load());
   if (rc) return rc;
   // X = 0 * (1 - 0) + 1 * NS(G): the apply kernel with lr = -1 writes the (un-transposed) result
   launch_muon_apply(X, Xb, res, res_es, batch, r, cc, tr, -1.f, 0.f, 1.f, s);
@@ -1593,29 +1689,23 @@ constexpr size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 // layout of gpt_op_newton_schulz's scratch at the largest accepted size
 // (its r x r products never exceed the r x c inputs)
 constexpr size_t kNsStaticBytes = 6 * align256(kNsStaticMaxElems * 4) + align256(kNsStaticMaxBatch * 4) +
-                                  align256(kNsStaticMaxBatch * 64 * 4) + align256(kNsStaticMaxElems * 2) +
-                                  align256(16);
+                                  align256(kNsStaticMaxBatch * 64 * 4) + align256(kNsStaticMaxElems * 2);
 
 // Every GPU that loads the library holds this array until the process exits.
 static __device__ __align__(256) unsigned char g_ns_static_scratch[kNsStaticBytes];
 
-std::mutex g_ns_static_mu;
-void* g_ns_static_ptr[256] = {};
-
-// Device address of the array on the current device, looked up once per device.
+// Device address of the array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// the device current, on every call: the lookup is cheap once the library's
+// device code is loaded on that device (the first lookup loads it), and a
+// context created after a device reset gets its own address instead of a
+// stale one.
 int ns_static_scratch(void** out) {
-  int dev = 0;
-  GPT_CK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 256) return fail(GPT_EINVAL, "device ordinal out of range");
-  std::lock_guard<std::mutex> lock(g_ns_static_mu);
-  if (!g_ns_static_ptr[dev]) {
-    void* p = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(GPT_ECUDA, std::string("cudaGetSymbolAddress of the static scratch: ") + cudaGetErrorString(e));
-    g_ns_static_ptr[dev] = p;
-  }
-  *out = g_ns_static_ptr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_ns_static_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(GPT_ECUDA, std::string("cudaGetSymbolAddress of the static scratch: ") + cudaGetErrorString(e));
+  *out = p;
   return GPT_OK;
 }
 
@@ -1634,9 +1724,10 @@ int gpt_op_newton_schulz_noalloc(const float* G, float* X, int batch, int rows, 
   int rc = ns_static_scratch(&scratch);
   if (rc) return rc;
   // The same computation as gpt_op_newton_schulz on the static array.  It
-  // clears the error word and the output before use; every other scratch
-  // region is written before it is read, so leftovers of an earlier call
-  // cannot leak into this one.
+  // clears the output before use; every scratch region is written before it
+  // is read, so leftovers of an earlier call cannot leak into this one.
+  // Expired device waits are latched in the op-level error word
+  // (gpt_op_check).
   return gpt_op_newton_schulz(G, X, batch, rows, cols, tf32_steps, scratch, stream);
 }
 

@@ -15,10 +15,11 @@ using bf16 = __nv_bfloat16;
 // int the persistent kernel hands out its work with (zeroed here, on s); null
 // takes one of the library's own.  kv_stride: heads per batch row in the
 // k/v (and dk/dv) buffers, kv head j of batch b at row b*kv_stride + j (0:
-// Hkv, dense).
+// Hkv, dense).  wait_cycles: bound of every device-side wait in SM cycles
+// (<= 0: the library default).
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr,
-                     int kv_stride = 0);
+                     int kv_stride = 0, long long wait_cycles = 0);
 
 // Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32
 // [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, Hkv, T, 128]
@@ -27,6 +28,6 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr,
-                     int kv_stride = 0);
+                     int kv_stride = 0, long long wait_cycles = 0);
 
 }  // namespace gpt

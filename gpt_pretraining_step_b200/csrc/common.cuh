@@ -19,10 +19,17 @@ enum : int {
   ERRF_SHAPE = 4,         // a launch saw a shape it cannot handle
 };
 
-// A wait gives up after this many SM clock cycles (about 2 s at 2 GHz, longer
-// at lower clocks).  The SM-local cycle counter is cheap to read, unlike the
-// global nanosecond timer.
+// By default a wait gives up after this many SM clock cycles (about 2 s at
+// 2 GHz, longer at lower clocks).  The SM-local cycle counter is cheap to
+// read, unlike the global nanosecond timer.  Kernels take the limit as a
+// launch argument, so a caller may shorten it (a failure-detection test
+// makes waits expire on purpose that way).
 constexpr long long kWaitLimitCycles = 4000000000ll;
+
+// The limit a launch uses: the caller's value, or the default for <= 0.
+__host__ __device__ __forceinline__ long long wait_limit_or_default(long long cycles) {
+  return cycles > 0 ? cycles : kWaitLimitCycles;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -68,18 +75,48 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same phase completion.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Limits below this many cycles are polled with the non-blocking test and a
+// clock check on every probe: a blocking try_wait may suspend the thread for
+// longer than such a limit, and the limit would not be kept.
+constexpr long long kShortWaitCycles = 1000000ll;
+
 // Wait for the phase with the given parity to complete.  Returns false if
-// another thread raised *abort or the wait ran past kWaitLimitCycles; in the
+// another thread raised *abort or the wait ran past `limit` SM cycles; in the
 // latter case this thread raises *abort itself and sets the error flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
+                                          int* err, long long limit) {
+  if (limit < kShortWaitCycles) {
+    const long long t0 = clock64();
+    for (;;) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        *abort = 1;
+        if (err) atomicOr(err, ERRF_TIMEOUT);
+        return false;
+      }
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         *abort = 1;
         if (err) atomicOr(err, ERRF_TIMEOUT);
         return false;

@@ -197,6 +197,7 @@ __global__ void __launch_bounds__(320, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
+  const long long wlim = wait_limit_or_default(p.wait_cycles);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(320, 1)
         int z, mb, nb, kb0, kb1, split;
         decode_unit(p, u, z, mb, nb, kb0, kb1, split);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
           mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
@@ -281,11 +282,11 @@ __global__ void __launch_bounds__(320, 1)
         decode_unit(p, u, z, mb, nb, kb0, kb1, split);
         const int acc = local & 1;
         const uint32_t acc_par = (local >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err)) { ok = false; break; }
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.err)) { ok = false; break; }
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, wlim)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t b0 = a0 + C::A_BYTES;
@@ -394,7 +395,7 @@ __global__ void __launch_bounds__(320, 1)
           asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
         }
       }
-      bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err);
+      bool got = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err, wlim);
       __syncwarp();   // tcgen05.ld is warp-collective: reconverge after the spin
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();

@@ -39,6 +39,7 @@ struct GemmParams {
   int tma_out2;         // 1: also an fp16 copy of the output, same layout, through the second map
   void* out2;           //   (its base; row stride ldo, batch stride out_bs)
   int* err;
+  long long wait_cycles;   // bound of every mbarrier wait (SM cycles; <= 0: the library default)
 };
 
 }  // namespace gpt

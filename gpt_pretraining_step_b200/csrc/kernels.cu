@@ -101,25 +101,98 @@ __global__ void __launch_bounds__(1024) embed_sort_kernel(const int* __restrict_
   for (int i = threadIdx.x; i < n; i += blockDim.x) keys_out[i] = keys[i];
 }
 
-// One warp per run of equal tokens in the sorted keys: sums dx rows in position order.
-__global__ void embed_segsum_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ dx,
-                                    int base, float* __restrict__ dwte, int d) {
-  const int w = blockIdx.x * (blockDim.x / 32) + warp_id();
+// Segmented sum of dx rows by token over the sorted keys, robust to skewed
+// token histograms (natural text puts thousands of rows on a few tokens).
+// The sorted positions are cut into aligned chunks of kEmbPiece rows; a run
+// of equal tokens is split at the chunk boundaries into pieces, each summed
+// by one warp per 128 columns in position order.  A run inside one chunk is
+// added to its row of dwte directly; the pieces of a run that crosses
+// chunks leave partial sums in the workspace (slot 2c for the piece at the
+// start of chunk c, 2c + 1 for a piece that starts inside chunk c and runs
+// on into the next one), which embed_join_kernel adds in position order.
+// Every sum has a fixed order, so the result is deterministic.
+constexpr int kEmbPiece = 64;
+
+__device__ __forceinline__ uint32_t emb_tok(const uint32_t* keys, int i) { return keys[i] / kEmbChunk; }
+
+__global__ void embed_piece_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ dx, int base,
+                                   float* __restrict__ dwte, float* __restrict__ part, int d) {
+  const int nchunk = d / 128;
+  const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + warp_id();
+  const int w = static_cast<int>(gw / nchunk);
+  const int c0 = static_cast<int>(gw - static_cast<long long>(w) * nchunk) * 128;
   if (w >= n) return;
-  const uint32_t tokw = keys[w] / kEmbChunk;
-  if (w > 0 && keys[w - 1] / kEmbChunk == tokw) return;
-  int end = w + 1;
-  while (end < n && keys[end] / kEmbChunk == tokw) ++end;
-  float* dst = dwte + static_cast<long long>(tokw) * d;
-  for (int c = lane_id() * 4; c < d; c += 128) {
-    float4 acc = *reinterpret_cast<const float4*>(dst + c);
-    for (int j = w; j < end; ++j) {
-      const int m = base + static_cast<int>(keys[j] % kEmbChunk);
-      const float4 v = *reinterpret_cast<const float4*>(dx + static_cast<long long>(m) * d + c);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    *reinterpret_cast<float4*>(dst + c) = acc;
+  const uint32_t tw = emb_tok(keys, w);
+  const bool at_chunk = w % kEmbPiece == 0;
+  const bool run_start = w == 0 || emb_tok(keys, w - 1) != tw;
+  if (!at_chunk && !run_start) return;
+  // the piece ends at the run's end or the chunk's end, whichever is first
+  const int cend = min(n, (w / kEmbPiece + 1) * kEmbPiece);
+  int e = cend;
+  for (int j0 = w + 1; j0 < cend; j0 += 32) {
+    const int j = j0 + lane_id();
+    const bool other = j < cend && emb_tok(keys, j) != tw;
+    const unsigned m = __ballot_sync(0xffffffffu, other);
+    if (m) { e = j0 + __ffs(m) - 1; break; }
   }
+  const bool continues_before = at_chunk && !run_start;
+  const bool continues_after = e == cend && cend < n && emb_tok(keys, cend) == tw;
+  const int c = lane_id() * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = w; j < e; j += 8) {
+    float4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j + u < e) {
+        const int m = base + static_cast<int>(keys[j + u] % kEmbChunk);
+        v[u] = *reinterpret_cast<const float4*>(dx + static_cast<long long>(m) * d + c0 + c);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+    }
+  }
+  if (!continues_before && !continues_after) {
+    float* dst = dwte + static_cast<long long>(tw) * d + c0 + c;
+    const float4 o = *reinterpret_cast<const float4*>(dst);
+    *reinterpret_cast<float4*>(dst) = make_float4(o.x + acc.x, o.y + acc.y, o.z + acc.z, o.w + acc.w);
+    return;
+  }
+  const int slot = 2 * (w / kEmbPiece) + (at_chunk ? 0 : 1);
+  *reinterpret_cast<float4*>(part + static_cast<long long>(slot) * d + c0 + c) = acc;
+}
+
+// One warp per (run that crosses a chunk boundary, 128 columns): the sum of
+// its pieces' partials in position order, added to the token's row.
+__global__ void embed_join_kernel(const uint32_t* __restrict__ keys, int n, const float* __restrict__ part,
+                                  float* __restrict__ dwte, int d) {
+  const int nchunk = d / 128;
+  const long long gw = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + warp_id();
+  const int w = static_cast<int>(gw / nchunk);
+  const int c0 = static_cast<int>(gw - static_cast<long long>(w) * nchunk) * 128;
+  if (w >= n) return;
+  const uint32_t tw = emb_tok(keys, w);
+  if (w > 0 && emb_tok(keys, w - 1) == tw) return;           // not a run start
+  const int b = (w / kEmbPiece + 1) * kEmbPiece;               // the next chunk boundary
+  if (b >= n || emb_tok(keys, b) != tw) return;              // the run stays inside its chunk
+  // the run's last position: the last key of token tw
+  int lo = b, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (emb_tok(keys, mid) == tw) lo = mid; else hi = mid - 1;
+  }
+  const int c = lane_id() * 4;
+  const float* p0 = part + static_cast<long long>(2 * (w / kEmbPiece) + (w % kEmbPiece == 0 ? 0 : 1)) * d + c0 + c;
+  float4 acc = *reinterpret_cast<const float4*>(p0);
+  for (int ch = b / kEmbPiece; ch <= lo / kEmbPiece; ++ch) {
+    const float4 v = *reinterpret_cast<const float4*>(part + static_cast<long long>(2 * ch) * d + c0 + c);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  float* dst = dwte + static_cast<long long>(tw) * d + c0 + c;
+  const float4 o = *reinterpret_cast<const float4*>(dst);
+  *reinterpret_cast<float4*>(dst) = make_float4(o.x + acc.x, o.y + acc.y, o.z + acc.z, o.w + acc.w);
 }
 
 // --------------------------------------------------------------- RMSNorm
@@ -1051,8 +1124,12 @@ void launch_sum_scale(const float* v, int n, float scale, float* out, cudaStream
   sum_scale_kernel<<<1, 1024, 0, s>>>(v, n, scale, out);
 }
 
-// the sort runs in chunks of kEmbChunk tokens, so the workspace does not grow with M
-size_t embed_bwd_workspace(int /*M*/) { return static_cast<size_t>(kEmbChunk) * sizeof(uint32_t) + 256; }
+// the sort runs in chunks of kEmbChunk tokens, so the workspace does not grow
+// with M: the sorted keys, then two partial rows of d floats per piece chunk
+size_t embed_bwd_workspace(int /*M*/, int d) {
+  return static_cast<size_t>(kEmbChunk) * sizeof(uint32_t) +
+         static_cast<size_t>(2 * (kEmbChunk / kEmbPiece)) * d * sizeof(float) + 256;
+}
 
 void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws, bool accumulate,
                       cudaStream_t s) {
@@ -1060,12 +1137,16 @@ void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d
   set_smem_limit_once(embed_sort_kernel, kEmbChunk * 4, configured);   // a failure shows at the launch
   if (!accumulate) cudaMemsetAsync(dwte, 0, static_cast<size_t>(V) * d * sizeof(float), s);
   uint32_t* keys = static_cast<uint32_t*>(ws);
+  float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + static_cast<size_t>(kEmbChunk) * sizeof(uint32_t));
+  const int nchunk = d / 128;
   for (int base = 0; base < M; base += kEmbChunk) {
     const int n = M - base < kEmbChunk ? M - base : kEmbChunk;
     int npow2 = 1;
     while (npow2 < n) npow2 <<= 1;
     embed_sort_kernel<<<1, 1024, npow2 * 4, s>>>(tok + base, n, npow2, keys, V);
-    embed_segsum_kernel<<<cdiv(n, 8), 256, 0, s>>>(keys, n, dx, base, dwte, d);
+    const long long warps = static_cast<long long>(n) * nchunk;
+    embed_piece_kernel<<<static_cast<int>((warps + 7) / 8), 256, 0, s>>>(keys, n, dx, base, dwte, part, d);
+    embed_join_kernel<<<static_cast<int>((warps + 7) / 8), 256, 0, s>>>(keys, n, part, dwte, d);
   }
 }
 

@@ -39,8 +39,10 @@ void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* 
 // loss = sum(row_loss) * scale, deterministic single-block reduction.
 void launch_sum_scale(const float* v, int n, float scale, float* out, cudaStream_t s);
 
-// Deterministic embedding gradient: dwte (+)= scatter of dx rows by token.
-size_t embed_bwd_workspace(int M);
+// Deterministic embedding gradient: dwte (+)= scatter of dx rows by token
+// (d a multiple of 128; the workspace holds the sorted ids and the partial
+// sums of tokens with many rows).  Three launches per 32768 tokens.
+size_t embed_bwd_workspace(int M, int d);
 void launch_embed_bwd(const int* tok, const float* dx, float* dwte, int M, int d, int V, void* ws,
                       bool accumulate, cudaStream_t s);
 

@@ -142,12 +142,20 @@ int gpt_workspace_size(const gpt_config* cfg, size_t* param_bytes, size_t* state
 
 /* Binds the buffers and the CUDA stream (a cudaStream_t; NULL = legacy
  * default stream) to a new context.  Draws the initial weights on the
- * device (N(0, 0.02) rounded to bf16, masters equal to their bf16 copies),
- * zeroes gradients and optimizer state.  Synchronous. */
+ * device (N(0, 0.02) rounded to bf16, masters equal to their bf16 copies:
+ * the fp32 master weights of "Como Treinar Seu Próprio ChatGPT por 50
+ * Dólares?", section "3. Gerenciamento de Precisão"), zeroes gradients and
+ * optimizer state.  Synchronous. */
 int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_buf, void* stream,
              gpt_ctx** out);
 
-/* Forward and backward pass over one batch.
+/* Forward and backward pass over one batch of the decoder of "¿Cómo Entrenar
+ * Tu Propio ChatGPT por $50?", section "1. Modelo GPT" (token embedding;
+ * per block a gain-free RMSNorm, the fused q|k|v projection with rotary
+ * embeddings and QK normalisation, causal attention, the output projection,
+ * a second norm and the ReLU^2 MLP; a final norm, the untied lm_head and the
+ * mean next-token cross-entropy), bf16 operands with fp32 accumulation
+ * (section "3. Gestión de Precisión").
  *   tokens, targets  device int32 [batch, seq_len]; position t of a row
  *                    predicts targets[row, t] from tokens[row, 0..t]
  *   loss_out         device fp32 scalar, receives the mean cross-entropy
@@ -155,8 +163,10 @@ int gpt_init(const gpt_config* cfg, void* param_buf, void* state_buf, void* act_
  * Ids outside [0, vocab) are treated as 0 and latched as GPT_ERANGE. */
 int gpt_fwd_bwd(gpt_ctx* ctx, const int32_t* tokens, const int32_t* targets, float* loss_out, int accumulate);
 
-/* Muon update of every 2-D block matrix (fused q|k|v, attention output, MLP
- * up, MLP down; q|k|v is [d, 3d], narrower with grouped kv heads):
+/* Muon update ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "2.
+ * Optimizador Muon": momentum orthogonalised by five quintic Newton-Schulz
+ * "Polar Express" steps) of every 2-D block matrix (fused q|k|v, attention
+ * output, MLP up, MLP down; q|k|v is [d, 3d], narrower with grouped kv heads):
  * mom = momentum * mom + grad; X = NS5(mom / (||mom||_F + 1e-7))
  * with the Polar Express coefficients; W = W (1 - lr * weight_decay)
  * - lr * sqrt(max(1, rows / cols)) * X.  Refreshes the bf16 copies. */
@@ -197,7 +207,9 @@ enum { GPT_REGION_MASTER = 0, GPT_REGION_BF16 = 1, GPT_REGION_GRAD = 2 };
 int gpt_block_region(const gpt_ctx* ctx, int what, int kind, int l0, int l1, size_t* offset_bytes,
                      size_t* size_bytes);
 
-/* AdamW update of the token embedding and lm_head (and of the residual-extras
+/* AdamW update ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "2.
+ * Optimizador Muon", parameter table: embeddings and lm_head go to AdamW)
+ * of the token embedding and lm_head (and of the residual-extras
  * scalars and value-embedding tables and gates when those are on) with bias
  * correction (the step count is kept in the context) and decoupled weight
  * decay. */
@@ -283,6 +295,16 @@ int gpt_profile_read(gpt_ctx* ctx, double* ms, int64_t* launches);
 /* Synchronises the stream and reports (then clears) latched device errors. */
 int gpt_check(gpt_ctx* ctx);
 
+/* Bound of every device-side wait of this context's kernels, in SM clock
+ * cycles (the waits of the TMA / tensor-core / softmax pipelines inside the
+ * GEMM and attention kernels); cycles <= 0 restores the default of 4e9
+ * (about 2 s at 2 GHz).  When a wait runs past its bound the kernel stops,
+ * lets its in-flight copies land, frees its tensor memory and returns;
+ * gpt_check then reports GPT_ETIMEOUT and the step's results are invalid,
+ * but the context stays usable.  A short bound is for failure-detection
+ * tests only: it makes ordinary waits expire. */
+int gpt_set_wait_limit(gpt_ctx* ctx, long long cycles);
+
 /* Number of kernels the library has launched through this context. */
 int64_t gpt_launch_count(const gpt_ctx* ctx);
 
@@ -292,8 +314,23 @@ const char* gpt_last_error(void);
 /* --------------------------------------------------------------------
  * Op-level entry points: single kernels of the step on caller buffers,
  * for testing and for composing other models.  All pointers are device
- * pointers; the stream is a cudaStream_t; asynchronous.
+ * pointers; the stream is a cudaStream_t; asynchronous.  The return code
+ * covers argument checks and the launch; failures inside the kernels (an
+ * expired bounded wait) are latched in a device error word that the
+ * library keeps for each GPU and reported by gpt_op_check.
  * ------------------------------------------------------------------ */
+
+/* Synchronises the stream, then reports and clears the op-level error word
+ * of the current device: GPT_ETIMEOUT if a bounded device wait of an
+ * op-level call expired since the last check (that call's outputs are
+ * invalid), GPT_OK otherwise.  The word is shared by every op-level call on
+ * the device, whatever its stream or thread. */
+int gpt_op_check(void* stream);
+
+/* Bound of the device-side waits of every later op-level call in this
+ * process, in SM clock cycles; cycles <= 0 restores the default (4e9).  As
+ * for gpt_set_wait_limit, a short bound is for failure-detection tests. */
+int gpt_op_set_wait_limit(long long cycles);
 
 /* C[z] = A[z] * B[z] with fp32 accumulation on the tensor cores.
  *   A [M, K] row-major bf16 (z stride M*K), B [K, N] row-major bf16 (z stride K*N),
@@ -350,10 +387,25 @@ int gpt_op_attention_bwd_ex(const void* q, const void* k, const void* v, const v
                             const float* lse, float* Dscratch, float* dq, void* dk, void* dv, int B, int H, int Hkv,
                             int T, int window, void* stream);
 
+/* Embedding gradient ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section
+ * "1. Modelo GPT": the token embedding x0 = wte[tok]; its gradient scatters
+ * the rows of dx by token): dwte[v] (+)= sum of dx[m] over the positions m
+ * with tokens[m] = v, summed in position order (deterministic, whatever the
+ * token histogram).
+ *   tokens  device int32 [M]; ids outside [0, vocab) count as 0
+ *   dx      fp32 [M, d]; dwte fp32 [vocab, d] (zeroed first unless
+ *           accumulate); d a multiple of 128, both 16-byte aligned
+ *   scratch device buffer of gpt_op_embedding_bwd_scratch(M, d) bytes,
+ *           256-byte aligned (0 for a bad shape) */
+size_t gpt_op_embedding_bwd_scratch(int M, int d);
+int gpt_op_embedding_bwd(const int32_t* tokens, const float* dx, float* dwte, int M, int d, int vocab, int accumulate,
+                         void* scratch, void* stream);
+
 /* Gain-free RMSNorm of fp32 rows [M, d] -> bf16 y and fp32 rstd [M]. */
 int gpt_op_rmsnorm_fwd(const float* x, void* y, float* rstd, int M, int d, void* stream);
 
-/* Newton-Schulz (Polar Express, five steps) of a batch of fp32 matrices
+/* Newton-Schulz ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "2.
+ * Optimizador Muon": Polar Express, five steps) of a batch of fp32 matrices
  * G [batch, rows, cols] -> fp32 X of the same shape, via the same kernels
  * as muon_step; tf32_steps selects the operand precision as ns_tf32_steps
  * does (-1 = fp16 operands, 0..5 = leading tf32 steps then bf16); scratch
@@ -370,11 +422,13 @@ int gpt_op_newton_schulz(const float* G, float* X, int batch, int rows, int cols
  * another allocator, runtimes that forbid cudaMalloc after start-up, and
  * interfaces with no place for a scratch pointer.
  *   Limits: batch * rows * cols <= 262144 fp32 elements and batch <= 64;
- *   larger inputs return GPT_EINVAL.  The array (6,832,640 bytes) stays
+ *   larger inputs return GPT_EINVAL.  The array (6,832,384 bytes) stays
  *   resident on every GPU that loads the library until the process exits.
- *   The first call on a device looks up the array's device address (once
- *   per device, with that device current); make that first call before
- *   any stream capture.
+ *   Every call looks up the array's device address with the current device
+ *   (so after a device reset the new context's address is used); the first
+ *   lookup on a device loads the library's device code there, so make the
+ *   first call on each device before any stream capture.  Expired device
+ *   waits are reported by gpt_op_check.
  *   All calls share the one array: calls that overlap on the GPU (other
  *   streams, other threads) race on it and must be serialised by the caller.
  * This call performs no cudaMalloc/cudaFree and calls no allocating

@@ -86,7 +86,11 @@ def test_checkpoint_restores_the_step_exactly(torch):
     cfg = dict(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
                residual_extras=True, ve_gate_channels=8)
     specs = syn.param_specs(s, extras=True, ve_channels=8)
-    a = g.GPTStep(**cfg)
+    # the first context runs on a stream of its own: a checkpoint read from it
+    # must still see every copy completed (the binding orders them before
+    # torch's current stream)
+    side = torch.cuda.Stream()
+    a = g.GPTStep(**cfg, stream=side)
     for tid, (pname, *_r) in enumerate(specs):
         a.set(tid, params[pname])
     batches = [(torch.tensor(syn.tokens(s, seed=82 + 2 * i)).cuda(), torch.tensor(syn.targets(s, seed=83 + 2 * i)).cuda())

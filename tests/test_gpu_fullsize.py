@@ -1,0 +1,185 @@
+"""Whole-step parity at the headline widths (B200 only).
+
+The d20 model of "¿Cómo Entrenar Tu Propio ChatGPT por $50?" (section "1.
+Modelo GPT"; d_model 1280, 10 heads of 128, vocabulary 32,768, sequences of
+2048 tokens) against the fp64 oracle: the loss, the per-position losses,
+every parameter's gradient, the embedding's row set, the Muon update of
+every block matrix and the AdamW update of the embedding and lm_head.  The
+oracle runs whole steps, so the batch is small (1-2 sequences) and, except
+for the full-depth case, so is the depth; the widths, the vocabulary, the
+sequence length and therefore every kernel's tile grid along those axes are
+the benchmark's.  The batch-16 launch shape of the benchmark is covered with
+one block (M = 32768 tokens, the length of every weight-gradient
+contraction there) by running the oracle on each sequence and averaging:
+the mean loss over B sequences is the mean of the per-sequence mean losses,
+so its gradient is the mean of theirs.
+
+Tolerances as the rest of the suite (stated for the step): loss relative
+error <= 1e-2 (3e-2 with fp8 projections), gradient cosine >= 0.999 (0.99
+fp8), Muon update relative Frobenius error <= 2e-2, indexing exact.  The
+optimizer updates are compared on identical inputs: the oracle's Muon and
+AdamW take the gradients the GPU computed.
+"""
+import numpy as np
+import pytest
+
+import synthetic as syn
+from oracle import model as om
+from oracle import optim as oo
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-2
+GRAD_COS = 0.999
+MUON_RELFRO = 2e-2
+FP8_LOSS_RTOL = 3e-2
+FP8_GRAD_COS = 0.99
+
+HP_MUON = (0.02, 0.95, 0.0)
+HP_ADAM = (3e-3, 0.8, 0.95, 1e-10, 0.0)
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as t
+    import gpt_pretraining_step_b200 as g
+    g.lib()
+    return t
+
+
+def f64(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def cosine(a, b):
+    a, b = np.ravel(a), np.ravel(b)
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b) + 1e-300))
+
+
+def relfro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def _gpu_step(torch, s, params, tok, tgt, precision=0, lm_chunk_rows=0):
+    import gpt_pretraining_step_b200 as g
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   precision=precision, lm_chunk_rows=lm_chunk_rows)
+    for tid, (name, *_r) in enumerate(syn.param_specs(s)):
+        st.set(tid, params[name])
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    return st, loss
+
+
+def _check_grads(g, st, s, grads, cos_min):
+    worst = (None, 1.0)
+    for tid, (pname, *_r) in enumerate(syn.param_specs(s)):
+        c = cosine(f64(st.get(tid, g.KIND_GRAD)), grads[pname])
+        if c < worst[1]:
+            worst = (pname, c)
+        assert c >= cos_min, (pname, c)
+    return worst
+
+
+def _check_optimizer(g, st, s, params, kinds=None):
+    """Muon and AdamW updates against the oracle on the GPU's own gradients."""
+    specs = syn.param_specs(s)
+    G = {tid: f64(st.get(tid, g.KIND_GRAD)) for tid in range(len(specs))}
+    st.muon_step(*HP_MUON)
+    st.adamw_step(*HP_ADAM)
+    st.check()
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        if kinds is not None and grp == "muon" and tid not in kinds:
+            continue
+        W0 = params[pname].astype(np.float64)
+        got = f64(st.get(tid, g.KIND_PARAM))
+        if grp == "muon":
+            W_ref, _ = oo.muon_step(W0, G[tid], np.zeros((r, c)), *HP_MUON)
+            err = relfro(got - W0, W_ref - W0)
+            assert err <= MUON_RELFRO, (pname, err)
+        else:
+            W_ref, _, _ = oo.adamw_step(W0, G[tid], np.zeros((r, c)), np.zeros((r, c)), 1, *HP_ADAM)
+            assert np.abs(got - W_ref).max() < 1e-6, pname
+
+
+HEADLINE = {
+    # depth, batch, token stream, rows of logits per lm_head chunk (0 = default 8192)
+    "d1280_L2_B1": (2, 1, "uniform", 0),
+    "d1280_L2_B1_zipf": (2, 1, "zipf", 0),
+    "d1280_L4_B2_two_chunks": (4, 2, "uniform", 2048),
+}
+
+
+@pytest.mark.parametrize("name", list(HEADLINE))
+def test_headline_width_step_matches_oracle(torch, name):
+    import gpt_pretraining_step_b200 as g
+    depth, batch, stream, chunk = HEADLINE[name]
+    s = syn.make_shape(depth=depth, d_model=1280, vocab=32768, batch=batch, seq_len=2048)
+    params = syn.init_params(s, seed=0)
+    tok = syn.zipf_tokens(s, seed=3) if stream == "zipf" else syn.tokens(s, seed=1)
+    tgt = syn.targets(s, seed=2)
+    st, loss = _gpu_step(torch, s, params, tok, tgt, lm_chunk_rows=chunk)
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL, (loss, loss_ref)
+    row = f64(st.row_loss()).ravel()
+    assert np.abs(row - cache["row_loss"]).max() < 5e-2
+    # exact embedding row set: the rows of the tokens present, and only those
+    E = st.get(0, g.KIND_GRAD)
+    nz = torch.nonzero(E.abs().sum(dim=1) > 0).flatten().cpu().numpy()
+    assert set(nz.tolist()) == set(np.unique(tok).tolist())
+    _check_grads(g, st, s, grads, GRAD_COS)
+    _check_optimizer(g, st, s, params)
+
+
+def test_d20_full_depth_step_matches_oracle(torch):
+    """The d20 model itself (20 blocks, d 1280, V 32768, T 2048) on one
+    sequence: every gradient, then Muon on one matrix of each kind spread
+    over the depth, and AdamW."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=20, batch=1, seq_len=2048)
+    params = syn.init_params(s, seed=0)
+    tok, tgt = syn.tokens(s, seed=1), syn.targets(s, seed=2)
+    st, loss = _gpu_step(torch, s, params, tok, tgt)
+    loss_ref, grads, cache = om.fwd_bwd(params, tok, tgt, s.depth)
+    del cache
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL, (loss, loss_ref)
+    _check_grads(g, st, s, grads, GRAD_COS)
+    del grads
+    _check_optimizer(g, st, s, params, kinds={2, 2 + 4 * 7 + 1, 2 + 4 * 13 + 2, 2 + 4 * 19 + 3})
+
+
+def test_benchmark_launch_shape_one_block_matches_oracle(torch):
+    """Batch 16 x 2048 tokens (the benchmark's M = 32768: lm_head in four
+    8192-row chunks, weight-gradient contractions over 32768 tokens) with one
+    block; the oracle runs the sequences one at a time and averages."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=1, batch=16, seq_len=2048, d_model=1280)
+    params = syn.init_params(s, seed=0)
+    tok, tgt = syn.tokens(s, seed=1), syn.targets(s, seed=2)
+    st, loss = _gpu_step(torch, s, params, tok, tgt)
+    one = syn.make_shape(depth=1, batch=1, seq_len=2048, d_model=1280)
+    loss_ref, grads, rows = 0.0, None, []
+    for b in range(s.batch):
+        lb, gb, cb = om.fwd_bwd(params, tok[b:b + 1], tgt[b:b + 1], one.depth)
+        loss_ref += lb / s.batch
+        rows.append(cb["row_loss"])
+        grads = {k: v / s.batch for k, v in gb.items()} if grads is None else \
+            {k: grads[k] + gb[k] / s.batch for k in grads}
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL, (loss, loss_ref)
+    assert np.abs(f64(st.row_loss()).ravel() - np.concatenate(rows)).max() < 5e-2
+    _check_grads(g, st, s, grads, GRAD_COS)
+    _check_optimizer(g, st, s, params)
+
+
+def test_d26_width_fp8_step_matches_oracle(torch):
+    """d26 widths (d_model 1664, 13 heads) with the fp8 e4m3 projections
+    against the bf16-math oracle at the fp8 tolerances."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=2, d_model=1664, vocab=32768, batch=1, seq_len=2048)
+    params = syn.init_params(s, seed=0)
+    tok, tgt = syn.tokens(s, seed=1), syn.targets(s, seed=2)
+    st, loss = _gpu_step(torch, s, params, tok, tgt, precision=1)
+    loss_ref, grads, _ = om.fwd_bwd(params, tok, tgt, s.depth)
+    assert abs(loss - loss_ref) / loss_ref <= FP8_LOSS_RTOL, (loss, loss_ref)
+    _check_grads(g, st, s, grads, FP8_GRAD_COS)
+    _check_optimizer(g, st, s, params)

@@ -276,3 +276,36 @@ def test_matmul_fp8(torch, b_trans, M, N, K):
     torch.cuda.synchronize()
     ref = (qa @ qb) * 0.5 * 0.125
     assert relfro(f64(C), ref) < 1e-6
+
+
+@pytest.mark.parametrize("stream", ["zipf", "uniform"])
+def test_embedding_bwd_at_benchmark_size(torch, stream):
+    """The embedding gradient at the benchmark's 32768 positions and width
+    1280: a Zipf(1.1) id stream (the skew of natural text: thousands of
+    positions on the first ids) and a uniform one, against the oracle's
+    scatter.  A row that occurs once is an exact copy; rows are summed in
+    fp32, so a row of n positions agrees to a few ulps of its magnitude
+    sum; the result is deterministic and accumulate adds onto the output."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=20, batch=16, seq_len=2048)
+    tok = (syn.zipf_tokens(s, seed=3) if stream == "zipf" else syn.tokens(s, seed=1)).reshape(-1)
+    dx = syn.gaussian((s.tokens, s.d_model), seed=31)
+    ref = om.embedding_bwd(tok, dx.astype(np.float64), s.vocab)
+    mag = om.embedding_bwd(tok, np.abs(dx).astype(np.float64), s.vocab)
+    t_tok = torch.tensor(tok).cuda()
+    t_dx = torch.tensor(dx).cuda()
+    got = g.embedding_bwd(t_tok, t_dx, s.vocab)
+    again = g.embedding_bwd(t_tok, t_dx, s.vocab)
+    torch.cuda.synchronize()
+    assert torch.equal(got, again)
+    counts = np.bincount(tok, minlength=s.vocab)
+    if stream == "zipf":
+        assert counts.max() > 2000
+    G = f64(got)
+    assert np.all(G[counts == 0] == 0.0)
+    once = counts == 1
+    assert np.array_equal(G[once], ref[once])
+    assert np.all(np.abs(G - ref) <= 1e-6 * mag + 1e-30)
+    twice = g.embedding_bwd(t_tok, t_dx, s.vocab, dwte=got.clone(), accumulate=True)
+    torch.cuda.synchronize()
+    assert np.all(np.abs(f64(twice) - 2 * ref) <= 2e-6 * mag + 1e-30)

@@ -1,15 +1,21 @@
 """The Newton-Schulz entry point that allocates no device memory.
 
-Callers whose device memory is owned by another allocator, or who cannot
-pass device scratch, use gpt_op_newton_schulz_noalloc: its scratch is a
-fixed array inside the loaded library.  This file is collected last so a
-stop-at-first-failure run has exercised everything else first; it also runs
+Some callers cannot give this library device scratch: their device memory
+belongs to another allocator (a framework's caching pool that has already
+reserved the GPU), their runtime forbids cudaMalloc after start-up, or their
+interface has no place for a scratch pointer.  gpt_op_newton_schulz_noalloc
+keeps its scratch in a fixed array inside the loaded library instead.  These
+tests compare it with the fp64 oracle's Newton-Schulz (and with the
+allocating entry point) on two calls in a row that share the array, and
+check its size limit.  This file is collected last, so a run that stops at
+the first failure has exercised everything else first; it also passes run
 alone in a fresh process.
 """
 import numpy as np
 import pytest
 
 import synthetic as syn
+from oracle import optim as oo
 
 pytestmark = pytest.mark.gpu
 
@@ -20,20 +26,27 @@ def _relfro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def test_noalloc_matches_allocating_entry_point_on_consecutive_calls():
+@pytest.mark.parametrize("tf32_steps", [-1, 3])
+def test_noalloc_matches_oracle_on_consecutive_calls(tf32_steps):
     import torch
 
     import gpt_pretraining_step_b200 as g
     g.lib()
-    # two different inputs, one call each, back to back on the shared array
+    # two different inputs, one call each, back to back on the shared array;
+    # the second is wider than tall (the transposed path)
     shapes = [(3, 256, 320), (2, 384, 128)]
     for i, shape in enumerate(shapes):
-        G = torch.tensor(syn.gaussian(shape, seed=500 + i)).cuda()
-        ref = g.newton_schulz(G, tf32_steps=3)
-        got = g.newton_schulz_noalloc(G, tf32_steps=3)
-        torch.cuda.synchronize()
-        err = _relfro(got.double().cpu().numpy(), ref.double().cpu().numpy())
-        assert err <= MUON_RELFRO, (shape, err)
+        G = syn.gaussian(shape, seed=500 + i)
+        tG = torch.tensor(G).cuda()
+        got = g.newton_schulz_noalloc(tG, tf32_steps=tf32_steps)
+        ref_gpu = g.newton_schulz(tG, tf32_steps=tf32_steps)
+        g.op_check()
+        got64 = got.double().cpu().numpy()
+        for z in range(shape[0]):
+            ref = oo.newton_schulz(G[z].astype(np.float64))
+            err = _relfro(got64[z], ref)
+            assert err <= MUON_RELFRO, (shape, z, err)
+        assert _relfro(got64, ref_gpu.double().cpu().numpy()) <= MUON_RELFRO, shape
 
 
 def test_noalloc_rejects_inputs_beyond_its_limit():
