@@ -338,15 +338,17 @@ def run_ours(a):
     grads = st.grad_view() if world > 1 else None
     hp = dict(muon=(0.02, 0.95, 0.0), adam=(3e-3, 0.8, 0.95, 1e-10, 0.0))
     counter = [0]
+    # the pages' ZeRO-2 exchange: bucket reduces overlapped with the backward,
+    # Muon by layer ranges, AdamW by rows
+    ex = dp.ShardedExchange(st, s.depth, s.vocab, s.d_model) if a.shard_optimizer and world > 1 else None
 
     def step():
         tok, tgt = batches[counter[0] % N_BATCHES]
         counter[0] += 1
-        st.fwd_bwd(tok, tgt)
-        if a.shard_optimizer and world > 1:
-            dp.sharded_optimizer_step(st, s.depth, muon=hp["muon"], adam=hp["adam"],
-                                      normuon_beta2=-1.0 if a.normuon is None else a.normuon)
+        if ex is not None:
+            ex.step(tok, tgt, muon=hp["muon"], adam=hp["adam"], normuon_beta2=-1.0 if a.normuon is None else a.normuon)
             return
+        st.fwd_bwd(tok, tgt)
         if grads is not None:
             dp.average_gradients(grads)
         if a.normuon is None:
@@ -443,7 +445,7 @@ def run_ours(a):
 
     e2e = None
     if not a.no_e2e:
-        e2e = run_e2e(a, st, s, rank, world, grads, stream)
+        e2e = run_e2e(a, st, s, rank, world, grads, stream, ex)
         if world > 1:
             e2e["ms_per_step"] = dp.max_over_ranks(e2e["ms_per_step"], device="cuda")
             e2e["value"] = tokens_per_step / (e2e["ms_per_step"] / 1e3)
@@ -503,7 +505,7 @@ def run_ours(a):
         dist.destroy_process_group()
 
 
-def run_e2e(a, st, s, rank, world, grads, stream):
+def run_e2e(a, st, s, rank, world, grads, stream, ex=None):
     """Whole steps through the public API from host buffers: H2D of tokens and
     targets from pinned memory, the step, D2H of the loss, all timed.  One GPU
     uses the single host-buffer entry point; data-parallel ranks compose the
@@ -526,14 +528,14 @@ def run_e2e(a, st, s, rank, world, grads, stream):
             return st.train_step_host(tok, tgt, hp)
         dtok.copy_(tok, non_blocking=True)
         dtgt.copy_(tgt, non_blocking=True)
-        loss = st.fwd_bwd(dtok, dtgt)
-        if a.shard_optimizer and world > 1:
-            dp.sharded_optimizer_step(st, s.depth, muon=(hp.muon_lr, hp.muon_momentum, hp.muon_wd),
-                                      adam=(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd),
-                                      normuon_beta2=-1.0 if a.normuon is None else a.normuon)
+        if ex is not None:
+            loss = ex.step(dtok, dtgt, muon=(hp.muon_lr, hp.muon_momentum, hp.muon_wd),
+                           adam=(hp.adam_lr, hp.adam_beta1, hp.adam_beta2, hp.adam_eps, hp.adam_wd),
+                           normuon_beta2=-1.0 if a.normuon is None else a.normuon)
             loss_host.copy_(loss.reshape(1), non_blocking=True)
             stream.synchronize()
             return float(loss_host[0])
+        loss = st.fwd_bwd(dtok, dtgt)
         dp.average_gradients(grads)
         if a.normuon is None:
             st.muon_step(hp.muon_lr, hp.muon_momentum, hp.muon_wd)

@@ -31,7 +31,9 @@ ABI_FUNCTIONS = [
     "gpt_op_rmsnorm_fwd", "gpt_op_newton_schulz_scratch", "gpt_op_newton_schulz",
     "gpt_op_newton_schulz_noalloc", "gpt_get_adam_step", "gpt_set_adam_step", "gpt_set_wait_limit",
     "gpt_op_check", "gpt_op_set_wait_limit", "gpt_op_embedding_bwd_scratch", "gpt_op_embedding_bwd",
+    "adamw_step_shard", "gpt_tensor_region", "gpt_grad_bucket", "gpt_set_grad_events",
 ]
+GRAD_BUCKETS = 6
 
 
 class GptError(RuntimeError):
@@ -76,6 +78,10 @@ def lib():
             "muon_step_layers": (i32, [vp, f32, f32, f32, f32, i32, i32]),
             "gpt_block_region": (i32, [vp, i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
             "adamw_step": (i32, [vp, f32, f32, f32, f32, f32]),
+            "adamw_step_shard": (i32, [vp, f32, f32, f32, f32, f32, i32, i32]),
+            "gpt_tensor_region": (i32, [vp, i32, i32, i32, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+            "gpt_grad_bucket": (i32, [vp, i32, ctypes.POINTER(sz), ctypes.POINTER(sz)]),
+            "gpt_set_grad_events": (i32, [vp, ctypes.POINTER(ctypes.c_void_p), i32]),
             "gpt_train_step_host": (i32, [vp, vp, vp, ctypes.POINTER(HParams), vp]),
             "gpt_num_tensors": (i32, [vp]),
             "gpt_tensor_info": (i32, [vp, i32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32),
@@ -220,6 +226,39 @@ class GPTStep:
 
     def adamw_step(self, lr=3e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.0):
         _check(lib().adamw_step(self.h, lr, beta1, beta2, eps, weight_decay))
+
+    def adamw_step_shard(self, part, nparts, lr=3e-3, beta1=0.8, beta2=0.95, eps=1e-10, weight_decay=0.0):
+        """AdamW on share `part` of `nparts` of the embedding and lm_head rows
+        (the other AdamW tensors whole)."""
+        _check(lib().adamw_step_shard(self.h, lr, beta1, beta2, eps, weight_decay, int(part), int(nparts)))
+
+    def tensor_region(self, what, tid, row0, row1):
+        """Tensor view of rows row0 .. row1-1 of tensor tid (embedding, lm_head or
+        a block matrix): REGION_MASTER, REGION_BF16 or REGION_GRAD."""
+        import torch
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_tensor_region(self.h, int(what), int(tid), int(row0), int(row1), ctypes.byref(off),
+                                       ctypes.byref(n)))
+        buf = self.bufs[1] if what == REGION_GRAD else self.bufs[0]
+        return buf[off.value:off.value + n.value].view(torch.bfloat16 if what == REGION_BF16 else torch.float32)
+
+    def grad_bucket(self, i):
+        """fp32 view of gradient bucket i (see gpt_grad_bucket)."""
+        import torch
+        off, n = ctypes.c_size_t(), ctypes.c_size_t()
+        _check(lib().gpt_grad_bucket(self.h, int(i), ctypes.byref(off), ctypes.byref(n)))
+        return self.bufs[1][off.value:off.value + n.value].view(torch.float32)
+
+    def set_grad_events(self, events):
+        """Register torch.cuda.Event objects: events[i] is recorded on the
+        context's stream when gradient bucket i is complete (empty: stop)."""
+        self._grad_events = list(events)   # kept alive while registered
+        handles = []
+        for e in self._grad_events:
+            e.record(self.stream)           # creates the event on this device
+            handles.append(ctypes.c_void_p(e.cuda_event))
+        arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
+        _check(lib().gpt_set_grad_events(self.h, arr, len(handles)))
 
     def train_step_host(self, tokens_host, targets_host, hp: HParams):
         """Whole step from host int32 arrays (numpy or pinned torch); returns the loss."""

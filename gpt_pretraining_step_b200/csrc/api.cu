@@ -70,7 +70,12 @@ struct Plan {
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
   size_t x0, xin, dx0, dxfin, scws, xe, sig;   // residual extras (allocated only when on)
   size_t vesig, vedz, vepart;                  // value embeddings (allocated only when on)
-  size_t wq8[4], winv, wamax, act8, act_inv, act_amax;   // fp8 copies (precision 1)
+  size_t wq8[4], winv, wamax;   // fp8 copies of the block weights with their scales (precision 1)
+  // fp8 per-layer copies of the four GEMM activations (xn1, o, xn2, h) and the
+  // four gradients they meet (dqkv, the gradient at the attention output and
+  // at the block output, du), kept for the batched weight-gradient GEMMs
+  size_t act8[4], grad8[4];
+  size_t f8slots, f8inv;   // [8][L][kAmaxSlots] scale words, [8][L] inverse scales: acts 0..3, grads 4..7
   size_t act_bytes;
   size_t splitk_elems;
   int splits_lm;      // lm_head dx split-K factor
@@ -174,9 +179,13 @@ void make_plan(const Dims& D, Plan& P) {
   P.wgb = pb.take(ngp * 2);
   P.param_bytes = pb.off;
   Bump sb;
-  // gradients: embedding, lm_head, the scalars, then the block matrices (one
-  // span; everything before the first block gradient goes to AdamW)
-  for (int i = 0; i < 2; ++i) P.g[i] = sb.take(numel[i] * 4);
+  // gradients: lm_head, embedding, the scalars and value-embedding tables and
+  // gates, then the block matrices (one span; everything before the first
+  // block gradient goes to AdamW).  The order is that of the buckets in which
+  // the backward completes them: lm_head first, the block kinds after the
+  // backward sweep, the embedding and the extras last (gpt_grad_bucket).
+  P.g[1] = sb.take(numel[1] * 4);
+  P.g[0] = sb.take(numel[0] * 4);
   P.gs = sb.take(std::max<size_t>(nsc, 4) * 4);
   P.gve = sb.take(std::max<size_t>(nvel, 4) * 4);
   P.gg = sb.take(ngp * 4);
@@ -280,15 +289,20 @@ void make_plan(const Dims& D, Plan& P) {
   P.tok = ab.take(M * 4);
   P.tgt = ab.take(M * 4);
   {
-    // fp8 e4m3 copies of the block weights and one activation operand, with their scales
+    // fp8 e4m3 copies of the block weights, of every layer's GEMM activations
+    // and of the gradients they meet, with their scales
     const bool f8 = D.fp8 != 0;
     const size_t wn[4] = {L * d * qc, L * d * d, L * d * F, L * F * d};
     for (int i = 0; i < 4; ++i) P.wq8[i] = ab.take(f8 ? wn[i] : 16);
     P.winv = ab.take(4 * L * 4);
     P.wamax = ab.take(4 * L * 4);
-    P.act8 = ab.take(f8 ? M * F : 16);
-    P.act_inv = ab.take(16);
-    P.act_amax = ab.take(16);
+    const size_t acols[4] = {d, d, d, F}, gcols[4] = {qc, d, F, d};
+    for (int i = 0; i < 4; ++i) {
+      P.act8[i] = ab.take(f8 ? L * M * acols[i] : 16);
+      P.grad8[i] = ab.take(f8 ? L * M * gcols[i] : 16);
+    }
+    P.f8slots = ab.take(8 * L * kAmaxSlots * 4);
+    P.f8inv = ab.take(8 * L * 4);
   }
   P.act_bytes = ab.off;
 }
@@ -340,6 +354,11 @@ struct gpt_ctx {
   uint8_t* abuf;
   cudaStream_t stream;
   long long wait_cycles = 0;   // bound of the kernels' device-side waits (<= 0: the default)
+  cudaEvent_t grad_ev[GPT_GRAD_BUCKETS] = {};   // caller's events, recorded as gradient buckets complete
+  int n_grad_ev = 0;
+  void grad_ready(int bucket) {
+    if (bucket < n_grad_ev && grad_ev[bucket]) cudaEventRecord(grad_ev[bucket], stream);
+  }
   long long adam_step = 0;
   int64_t launches = 0;
   // event profiler
@@ -522,36 +541,70 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     launch_smear_fwd(c->A<float>(P.xe), x, c->A<float>(P.sig), c->Scal(), L, D.T, M, d, s);
     c->launches += 1;
   }
-  // fp8: e4m3 copies of every block matrix, one scale per matrix
-  uint8_t* act8 = c->A<uint8_t>(P.act8);
-  float* act_inv = c->A<float>(P.act_inv);
-  unsigned int* act_amax = c->A<unsigned int>(P.act_amax);
+  // fp8 ("3. Gestión de Precisión": FP8 with per-tensor scaling): e4m3 copies
+  // of every block matrix, one scale per matrix; every GEMM operand that is an
+  // activation or an activation gradient is quantised per tensor with the
+  // amax its producer kept (scale words zeroed here, once per step)
   float* winv = c->A<float>(P.winv);
+  unsigned int* f8slots = c->A<unsigned int>(P.f8slots);
+  float* f8inv = c->A<float>(P.f8inv);
+  const long long wn[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+  const long long acols[4] = {d, d, d, F}, gcols[4] = {D.qc, d, F, d};
+  // tensor t of layer l: activations t = 0..3 (xn1, o, xn2, h), gradients 4..7
+  // (dqkv, the gradients at the attention output and at the block output, du)
+  // in the order of the weight kinds they meet
+  auto slots8 = [&](int t, int l) { return D.fp8 ? f8slots + (static_cast<size_t>(t) * L + l) * kAmaxSlots : nullptr; };
+  auto inv8 = [&](int t, int l) { return f8inv + t * L + l; };
+  auto act8 = [&](int k, int l) { return c->A<uint8_t>(P.act8[k]) + static_cast<size_t>(l) * M * acols[k]; };
+  auto grad8 = [&](int k, int l) { return c->A<uint8_t>(P.grad8[k]) + static_cast<size_t>(l) * M * gcols[k]; };
   if (D.fp8) {
     ProfScope ps(c, GPT_PROF_FP8_QUANT);
-    const long long wn[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
+    GPT_CK(cudaMemsetAsync(f8slots, 0, static_cast<size_t>(8) * L * kAmaxSlots * 4, s));
     for (int gi = 0; gi < 4; ++gi)
       launch_quantize_e4m3(c->Wb(2 + gi), wn[gi], L, c->A<unsigned int>(P.wamax) + gi * L,
                            c->A<uint8_t>(P.wq8[gi]), winv + gi * L, s);
     c->launches += 8;
   }
-  // operand A of a forward projection: bf16 as it is, or quantised to e4m3 into act8
+  // operand A of a forward projection of weight kind k: bf16 as it is, or its
+  // e4m3 copy (kept for the weight gradient) with the weight's e4m3 copy as B
   auto fwd_a = [&](GemmCall& g, const bf16* a, long long rows, long long cols, int grp, int l) {
+    if (!D.fp8) {
+      g.A = a;
+      return;
+    }
+    const int k = grp - 2;
+    {
+      ProfScope ps(c, GPT_PROF_FP8_QUANT);
+      if (k == 1) {   // the attention output keeps no amax of its own
+        launch_amax_slots(a, rows * cols, slots8(k, l), s);
+        c->launches += 1;
+      }
+      launch_quantize_e4m3_slots(a, rows * cols, slots8(k, l), act8(k, l), inv8(k, l), s);
+      c->launches += 1;
+    }
+    g.es = 1;
+    g.A = act8(k, l);
+    g.B = c->A<uint8_t>(P.wq8[k]) + static_cast<size_t>(l) * wn[k];
+    g.p.dq_a = inv8(k, l);
+    g.p.dq_b = winv + k * L + l;
+  };
+  // operand A of an activation-gradient GEMM against weight kind k: the bf16
+  // gradient, or its e4m3 copy with the weight's e4m3 copy as B (K-major)
+  auto bwd_a = [&](GemmCall& g, const bf16* a, long long cols, int k, int l) {
     if (!D.fp8) {
       g.A = a;
       return;
     }
     {
       ProfScope ps(c, GPT_PROF_FP8_QUANT);
-      launch_quantize_e4m3(a, rows * cols, 1, act_amax, act8, act_inv, s);
-      c->launches += 2;
+      launch_quantize_e4m3_slots(a, 1ll * M * cols, slots8(4 + k, l), grad8(k, l), inv8(4 + k, l), s);
+      c->launches += 1;
     }
     g.es = 1;
-    g.A = act8;
-    const long long wn[4] = {1ll * d * D.qc, 1ll * d * d, 1ll * d * F, 1ll * F * d};
-    g.B = c->A<uint8_t>(P.wq8[grp - 2]) + static_cast<size_t>(l) * wn[grp - 2];
-    g.p.dq_a = act_inv;
-    g.p.dq_b = winv + (grp - 2) * L + l;
+    g.A = grad8(k, l);
+    g.B = c->A<uint8_t>(P.wq8[k]) + static_cast<size_t>(l) * wn[k];
+    g.p.dq_a = inv8(4 + k, l);
+    g.p.dq_b = winv + k * L + l;
   };
   c->launches += 3;
 
@@ -573,7 +626,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
+      launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s, slots8(0, l));
     }
     {
       GemmCall g = base_call(M, D.qc, d);
@@ -611,7 +664,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_fwd(x, xn2l, r2 + static_cast<size_t>(l) * M, M, d, s);
+      launch_rmsnorm_fwd(x, xn2l, r2 + static_cast<size_t>(l) * M, M, d, s, slots8(2, l));
     }
     {
       GemmCall g = base_call(M, F, d);
@@ -619,7 +672,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       fwd_a(g, xn2l, M, d, 4, l); g.lda = d;
       ProfScope ps(c, GPT_PROF_FC_GEMM);
       g.epi = EPI_RELU2; g.out_es = 2; g.aux_es = 2;
-      g.p.out = hl; g.p.ldo = F; g.p.err = err;
+      g.p.out = hl; g.p.ldo = F; g.p.err = err; g.p.amax_out = slots8(3, l);
       GPT_CK(run_gemm(g, s, c->wait_cycles));
     }
     {
@@ -686,6 +739,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   }
   launch_sum_scale(row_loss, M, 1.f / static_cast<float>(M), loss_out, s);
   c->launches += 1;
+  c->grad_ready(0);   // the lm_head gradient is complete
 
   // --------------------------------------------------------------- backward
   float* dx = c->A<float>(P.dx);
@@ -700,7 +754,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   auto gmlp = [&](int l) { return gx + (2 * static_cast<size_t>(l) + 1) * Md; };   // grad at block output
   {
     ProfScope ps(c, GPT_PROF_NORM);
-    launch_rmsnorm_bwd(dxn, xf, rf, dx, gmlp(L - 1), M, d, false, s);
+    launch_rmsnorm_bwd(dxn, xf, rf, dx, gmlp(L - 1), M, d, false, s, slots8(7, L - 1));
   }
   c->launches += 1;
   if (D.extras) {
@@ -719,33 +773,33 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     bf16* dqkv = dqkv_all + static_cast<size_t>(l) * M * D.qc;
     // MLP down: dh = dx W_d^T, du = dh * 2 relu(u) with relu(u) = sqrt(h)
     {
-      ProfScope ps(c, GPT_PROF_DX_GEMM);
       GemmCall g = base_call(M, F, d);
-      g.A = gmlp(l); g.lda = d;
       g.B = c->Wb(5) + static_cast<size_t>(l) * F * d; g.ldb = d;   // B(n = F index, k = d index)
+      bwd_a(g, gmlp(l), d, 3, l); g.lda = d;
+      ProfScope ps(c, GPT_PROF_DX_GEMM);
       g.epi = EPI_DRELU2; g.out_es = 2; g.aux_es = 2;
-      g.p.out = du; g.p.ldo = F; g.p.aux = hl; g.p.ld_aux = F; g.p.err = err;
+      g.p.out = du; g.p.ldo = F; g.p.aux = hl; g.p.ld_aux = F; g.p.err = err; g.p.amax_out = slots8(6, l);
       GPT_CK(run_gemm(g, s, c->wait_cycles));
       c->launches += 1;
     }
     {
       GemmCall g = base_call(M, d, F);   // dxn2 = du W_fc^T
-      g.A = du; g.lda = F;
       g.B = c->Wb(4) + static_cast<size_t>(l) * d * F; g.ldb = F;
+      bwd_a(g, du, F, 2, l); g.lda = F;
       int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
       if (rc) return rc;
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_bwd(dxn, xn2l, r2 + static_cast<size_t>(l) * M, dx, gatt(l), M, d, true, s);
+      launch_rmsnorm_bwd(dxn, xn2l, r2 + static_cast<size_t>(l) * M, dx, gatt(l), M, d, true, s, slots8(5, l));
     }
     c->launches += 1;
     // attention output projection
     {
-      ProfScope ps(c, GPT_PROF_DX_GEMM);
       GemmCall g = base_call(M, d, d);   // dy = dx W_o^T
-      g.A = gatt(l); g.lda = d;
       g.B = c->Wb(3) + static_cast<size_t>(l) * d * d; g.ldb = d;
+      bwd_a(g, gatt(l), d, 1, l); g.lda = d;
+      ProfScope ps(c, GPT_PROF_DX_GEMM);
       g.epi = EPI_STORE; g.out_es = 2; g.aux_es = 2;
       g.p.out = dy; g.p.ldo = d; g.p.err = err;
       GPT_CK(run_gemm(g, s, c->wait_cycles));
@@ -760,7 +814,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
       launch_qk_bwd(dqf, dk, dv, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
-                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv);
+                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv, slots8(4, l));
     }
     c->launches += 3;
     const int vs = D.ve_slot(l);
@@ -778,8 +832,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       GemmCall g = base_call(M, d, D.qc);   // dxn1 = dqkv W_qkv^T
-      g.A = dqkv; g.lda = D.qc;
       g.B = c->Wb(2) + static_cast<size_t>(l) * d * D.qc; g.ldb = D.qc;
+      bwd_a(g, dqkv, D.qc, 0, l); g.lda = D.qc;
       int rc = run_f32(c, g, dxn, false, 1, GPT_PROF_DX_GEMM);
       if (rc) return rc;
     }
@@ -792,7 +846,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       ProfScope ps(c, GPT_PROF_NORM);
       // the bf16 copy feeds the next (lower) block; below block 0 only the fp32 gradient is used
       launch_rmsnorm_bwd(dxn, xn1 + l * Md, r1 + static_cast<size_t>(l) * M, dx,
-                         l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), M, d, true, s);
+                         l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), M, d, true, s,
+                         l > 0 && !D.extras ? slots8(7, l - 1) : nullptr);
     }
     c->launches += 1;
     if (D.extras) {
@@ -804,6 +859,10 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
                        static_cast<long long>(Md), l > 0 ? gmlp(l - 1) : c->A<bf16>(P.dxb), c->A<float>(P.scws),
                        l == L - 1, l == 0, s);
       c->launches += 1;
+      if (D.fp8 && l > 0) {   // the bf16 copy was rewritten: its amax anew
+        launch_amax_slots(gmlp(l - 1), static_cast<long long>(Md), slots8(7, l - 1), s);
+        c->launches += 1;
+      }
     }
   }
   // weight gradients of every block matrix, each kind as one GEMM batched over the layers:
@@ -817,14 +876,25 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
         {xn2, d, static_cast<long long>(Md), du_all, F, 1ll * M * F, d, F, c->G(4)},
         {h, F, 1ll * M * F, gx + Md, d, 2 * static_cast<long long>(Md), F, d, c->G(5)},
     };
-    for (const DW& w : dws) {
+    for (int kind = 0; kind < 4; ++kind) {
+      const DW& w = dws[kind];
       GemmCall g = base_call(w.rows, w.cols, M);
       g.batch = L;
       g.A = w.a; g.a_mn = true; g.lda = w.lda; g.a_bs = w.a_bs;
       g.B = w.b; g.b_mn = true; g.ldb = w.ldb; g.b_bs = w.b_bs;
+      if (D.fp8) {
+        // e4m3 copies of the activations and gradients, one scale pair per layer
+        g.es = 1;
+        g.A = act8(kind, 0); g.lda = acols[kind]; g.a_bs = 1ll * M * acols[kind];
+        g.B = grad8(kind, 0); g.ldb = gcols[kind]; g.b_bs = 1ll * M * gcols[kind];
+        g.p.dq_a = inv8(kind, 0);
+        g.p.dq_b = inv8(4 + kind, 0);
+        g.p.dq_zs = 1;
+      }
       g.epi = acc ? EPI_ACC : EPI_STORE; g.out_es = 4; g.aux_es = 4;
       g.p.out = w.out; g.p.ldo = w.cols; g.p.out_bs = 1ll * w.rows * w.cols; g.p.err = err;
       GPT_CK(run_gemm(g, s, c->wait_cycles));
+      c->grad_ready(1 + kind);   // this block matrix kind's gradients, every layer
     }
     c->launches += 4;
   }
@@ -843,6 +913,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     launch_embed_bwd(tok, demb, c->G(0), M, d, V, c->A<void>(P.embws), acc, s);
   }
   c->launches += 3 * ((M + 32767) / 32768);
+  c->grad_ready(5);   // the embedding and the extras
   GPT_CK(cudaGetLastError());
   return GPT_OK;
 }
@@ -1178,21 +1249,26 @@ int gpt_block_region(const gpt_ctx* c, int what, int kind, int l0, int l1, size_
   return GPT_OK;
 }
 
-int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay) {
-  int rc = check_ctx(c);
-  if (rc) return rc;
+// AdamW of the embedding and lm_head rows of share `part` of `nparts` (rows
+// [part R / nparts, (part + 1) R / nparts) of each), and of every other
+// AdamW tensor whole.
+static int adamw_update(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay, int part,
+                        int nparts) {
   c->adam_step += 1;
   const double t = static_cast<double>(c->adam_step);
   const float bc1 = static_cast<float>(1.0 - pow(static_cast<double>(beta1), t));
   const float bc2 = static_cast<float>(1.0 - pow(static_cast<double>(beta2), t));
-  const long long n = 1ll * c->D.V * c->D.d;
   ProfScope ps(c, GPT_PROF_ADAMW);
   for (int i = 0; i < 2; ++i) {
-    launch_adamw(c->W(i), c->G(i), reinterpret_cast<float*>(c->sbuf + c->P.am[i]),
-                 reinterpret_cast<float*>(c->sbuf + c->P.av[i]), c->Wb(i), n, lr, beta1, beta2, eps, weight_decay,
-                 bc1, bc2, c->stream);
+    const long long rows = i == 0 ? c->D.V : c->D.d, cols = i == 0 ? c->D.d : c->D.V;
+    const long long r0 = rows * part / nparts, r1 = rows * (part + 1) / nparts;
+    if (r1 <= r0) continue;
+    const size_t off = static_cast<size_t>(r0 * cols);
+    launch_adamw(c->W(i) + off, c->G(i) + off, reinterpret_cast<float*>(c->sbuf + c->P.am[i]) + off,
+                 reinterpret_cast<float*>(c->sbuf + c->P.av[i]) + off, c->Wb(i) + off, (r1 - r0) * cols, lr, beta1,
+                 beta2, eps, weight_decay, bc1, bc2, c->stream);
+    c->launches += 1;
   }
-  c->launches += 2;
   if (c->D.nve) {
     // value-embedding tables and their gates
     launch_adamw(c->VeW(0), c->VeG(0), reinterpret_cast<float*>(c->sbuf + c->P.amve),
@@ -1213,6 +1289,71 @@ int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float 
     c->launches += 1;
   }
   GPT_CK(cudaGetLastError());
+  return GPT_OK;
+}
+
+int gpt_tensor_region(const gpt_ctx* c, int what, int id, int row0, int row1, size_t* offset_bytes,
+                      size_t* size_bytes) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (what < GPT_REGION_MASTER || what > GPT_REGION_GRAD) return fail(GPT_EINVAL, "unknown region");
+  int grp, rows, cols;
+  size_t off;
+  if (!locate(c, id, grp, off, rows, cols) || grp >= 6)
+    return fail(GPT_EINVAL, "tensor id must name the embedding, the lm_head or a block matrix");
+  if (row0 < 0 || row1 > rows || row0 > row1) return fail(GPT_EINVAL, "row range out of bounds");
+  const size_t es = what == GPT_REGION_BF16 ? 2 : 4;
+  const size_t base = what == GPT_REGION_MASTER ? c->P.w[grp] : (what == GPT_REGION_BF16 ? c->P.wb[grp] : c->P.g[grp]);
+  if (offset_bytes) *offset_bytes = base + (off + static_cast<size_t>(row0) * cols) * es;
+  if (size_bytes) *size_bytes = static_cast<size_t>(row1 - row0) * cols * es;
+  return GPT_OK;
+}
+
+int adamw_step(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  return adamw_update(c, lr, beta1, beta2, eps, weight_decay, 0, 1);
+}
+
+int adamw_step_shard(gpt_ctx* c, float lr, float beta1, float beta2, float eps, float weight_decay, int part,
+                     int nparts) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (nparts < 1 || part < 0 || part >= nparts) return fail(GPT_EINVAL, "need 0 <= part < nparts");
+  return adamw_update(c, lr, beta1, beta2, eps, weight_decay, part, nparts);
+}
+
+int gpt_set_grad_events(gpt_ctx* c, void* const* events, int n) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  if (n < 0 || n > GPT_GRAD_BUCKETS || (n > 0 && !events)) return fail(GPT_EINVAL, "0..GPT_GRAD_BUCKETS events");
+  for (int i = 0; i < GPT_GRAD_BUCKETS; ++i) c->grad_ev[i] = i < n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  c->n_grad_ev = n;
+  return GPT_OK;
+}
+
+int gpt_grad_bucket(const gpt_ctx* c, int bucket, size_t* offset_bytes, size_t* size_bytes) {
+  int rc = check_ctx(c);
+  if (rc) return rc;
+  const Plan& P = c->P;
+  const Dims& D = c->D;
+  size_t b = 0, e = 0;
+  if (bucket == 0) {
+    b = P.g[1];
+    e = P.g[1] + static_cast<size_t>(D.d) * D.V * 4;
+  } else if (bucket >= 1 && bucket <= 4) {
+    const size_t d = D.d, F = D.F;
+    const size_t per[4] = {d * static_cast<size_t>(D.qc), d * d, d * F, F * d};
+    b = P.g[1 + bucket];
+    e = b + static_cast<size_t>(D.L) * per[bucket - 1] * 4;
+  } else if (bucket == 5) {
+    b = P.g[0];
+    e = P.g[2];   // the embedding, then the extras' gradients, up to the first block gradient
+  } else {
+    return fail(GPT_EINVAL, "bucket must be 0..GPT_GRAD_BUCKETS-1");
+  }
+  if (offset_bytes) *offset_bytes = b;
+  if (size_bytes) *size_bytes = e - b;
   return GPT_OK;
 }
 
@@ -1372,8 +1513,8 @@ int gpt_grad_region(const gpt_ctx* c, size_t* offset_bytes, size_t* size_bytes) 
   int rc = check_ctx(c);
   if (rc) return rc;
   const size_t last = c->P.g[5] + static_cast<size_t>(c->D.L) * c->D.F * c->D.d * 4;
-  if (offset_bytes) *offset_bytes = c->P.g[0];
-  if (size_bytes) *size_bytes = al(last) - c->P.g[0];
+  if (offset_bytes) *offset_bytes = c->P.g[1];
+  if (size_bytes) *size_bytes = al(last) - c->P.g[1];
   return GPT_OK;
 }
 

@@ -228,6 +228,12 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_RELU2, bf16, bf16)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_STORE, float, float)
   GPT_GEMM_CASE(uint8_t, 256, false, false, EPI_STORE, float, float)
+  // fp8 e4m3 backward: activation gradients against K-major weights, and the
+  // weight gradients with both operands token-major
+  GPT_GEMM_CASE(uint8_t, 256, false, false, EPI_DRELU2, bf16, bf16)
+  GPT_GEMM_CASE(uint8_t, 256, false, false, EPI_STORE, bf16, bf16)
+  GPT_GEMM_CASE(uint8_t, 256, true, true, EPI_STORE, float, float)
+  GPT_GEMM_CASE(uint8_t, 256, true, true, EPI_ACC, float, float)
 #undef GPT_GEMM_CASE
   return cudaErrorInvalidValue;
 }

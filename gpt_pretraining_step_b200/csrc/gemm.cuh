@@ -224,6 +224,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  float amax = 0.f;   // DRELU2 epilogue: this thread's max |out| (of the bf16-rounded values) over its tiles
 
   if (warp == 0) {
     if (lane == 0) {
@@ -405,7 +406,8 @@ __global__ void __launch_bounds__(320, 1)
       const int box_row0 = mb * 128 + quarter * 32;
       const int z3 = p.splits > 1 ? split : z;   // third coordinate of the output map
       float dqs = 1.f;   // dequantisation of fp8 operands
-      if constexpr (ES == 1) dqs = (p.dq_a ? p.dq_a[0] : 1.f) * (p.dq_b ? p.dq_b[0] : 1.f);
+      if constexpr (ES == 1)
+        dqs = (p.dq_a ? p.dq_a[z * p.dq_zs] : 1.f) * (p.dq_b ? p.dq_b[z * p.dq_zs] : 1.f);
       if constexpr (EPI == EPI_QKV) {
         // BN = 256: the tile holds heads 2*nb and 2*nb+1 of the H + 2 Hkv heads
         // of q|k|v for 128 tokens; the four warps of column half `half` own one
@@ -596,6 +598,12 @@ __global__ void __launch_bounds__(320, 1)
             if constexpr (EPI == EPI_RELU2) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) { const float t = fmaxf(v[hh][j], 0.f); v[hh][j] = t * t; }
+              if (p.amax_out && row_ok) {
+                const int nv = min(32, p.N - (nb * BN + cc * 32));
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) amax = fmaxf(amax, fabsf(__bfloat162float(__float2bfloat16_rn(v[hh][j]))));
+              }
             } else if constexpr (EPI == EPI_DRELU2) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -604,6 +612,12 @@ __global__ void __launch_bounds__(320, 1)
                 float rt;
                 asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(rt) : "f"(a[j]));
                 v[hh][j] *= 2.f * rt;
+              }
+              if (p.amax_out && row_ok) {
+                const int nv = min(32, p.N - (nb * BN + cc * 32));
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nv) amax = fmaxf(amax, fabsf(__bfloat162float(__float2bfloat16_rn(v[hh][j]))));
               }
             } else if constexpr (EPI == EPI_AXPBY) {
 #pragma unroll
@@ -639,6 +653,12 @@ __global__ void __launch_bounds__(320, 1)
     }
   }
 
+  if constexpr (EPI == EPI_DRELU2 || EPI == EPI_RELU2) {
+    if (warp >= 2 && p.amax_out) {
+      const float m = warp_max(amax);
+      if (lane == 0) atomicMax(p.amax_out + ((blockIdx.x * 8 + warp) & 31), __float_as_uint(m));
+    }
+  }
   if (warp >= 2 && lane == 0) bulk_wait_all();   // output boxes written before the CTA exits
   tc_fence_before();
   __syncthreads();

@@ -31,7 +31,10 @@ struct GemmParams {
   void* out_t;          // STORE/AXPBY: optional transposed copy of out, [N][M] with row stride ldo_t
   long long ldo_t;
   const float* dq_a;    // fp8 operands: device inverse scales of A and B; the accumulator is
-  const float* dq_b;    //   multiplied by dq_a[0] * dq_b[0] before the epilogue (null: 1)
+  const float* dq_b;    //   multiplied by dq_a[z * dq_zs] * dq_b[z * dq_zs] before the epilogue
+  int dq_zs;            //   (null: 1; dq_zs 1 = one scale per batch entry z, 0 = one for all)
+  unsigned int* amax_out;   // RELU2 / DRELU2: optional 32 fp8 scale words, atomically raised to the
+                            //   bits of max |bf16(out)| (each warp in one of them)
   int T, H;
   int Hkv;              // QKV: kv heads (0: H); columns are q (H heads) | k | v (Hkv heads each),
                         //   k and v stored at head rows b*H + j of their [B, H, T, 128] buffers

@@ -200,9 +200,20 @@ __global__ void embed_join_kernel(const uint32_t* __restrict__ keys, int n, cons
 // One warp per row of d = 128 * NV fp32 values; every load of the row is
 // issued before the warp reduction so one memory latency covers the row.
 
+// Largest |value| of a warp's bf16-rounded outputs into one of 32 slots of an
+// fp8 scale word set (32 slots spread the atomics; the quantiser takes the
+// max over them).  m: this lane's max.
+__device__ __forceinline__ void amax_slot_update(unsigned int* slots, float m, long long key) {
+  m = warp_max(m);
+  if (lane_id() == 0) atomicMax(slots + (key & 31), __float_as_uint(m));
+}
+
+__device__ __forceinline__ float abs_bf16(float v) { return fabsf(__bfloat162float(__float2bfloat16_rn(v))); }
+
 template <int NV>
 __global__ void __launch_bounds__(128) rmsnorm_fwd_kernel(const float* __restrict__ x, bf16* __restrict__ y,
-                                                          float* __restrict__ rstd, int M) {
+                                                          float* __restrict__ rstd, int M,
+                                                          unsigned int* __restrict__ amax) {
   constexpr int d = 128 * NV;
   const int row = blockIdx.x * 4 + warp_id();
   if (row >= M) return;
@@ -220,12 +231,21 @@ __global__ void __launch_bounds__(128) rmsnorm_fwd_kernel(const float* __restric
   for (int i = 0; i < NV; ++i)
     store_bf16x4(yr + (i * 32 + lane_id()) * 4, make_float4(buf[i].x * r, buf[i].y * r, buf[i].z * r, buf[i].w * r));
   if (lane_id() == 0) rstd[row] = r;
+  if (amax) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i)
+      m = fmaxf(m, fmaxf(fmaxf(abs_bf16(buf[i].x * r), abs_bf16(buf[i].y * r)),
+                         fmaxf(abs_bf16(buf[i].z * r), abs_bf16(buf[i].w * r))));
+    amax_slot_update(amax, m, row);
+  }
 }
 
 template <int NV>
 __global__ void __launch_bounds__(128) rmsnorm_bwd_kernel(const float* __restrict__ dy, const bf16* __restrict__ y,
                                                           const float* __restrict__ rstd, float* __restrict__ dx,
-                                                          bf16* __restrict__ dxb, int M, int accumulate) {
+                                                          bf16* __restrict__ dxb, int M, int accumulate,
+                                                          unsigned int* __restrict__ amax) {
   constexpr int d = 128 * NV;
   const int row = blockIdx.x * 4 + warp_id();
   if (row >= M) return;
@@ -245,6 +265,7 @@ __global__ void __launch_bounds__(128) rmsnorm_bwd_kernel(const float* __restric
   for (int i = 0; i < NV; ++i)
     dot += g[i].x * bf16_lo(yy[i].x) + g[i].y * bf16_hi(yy[i].x) + g[i].z * bf16_lo(yy[i].y) + g[i].w * bf16_hi(yy[i].y);
   dot = warp_sum(dot) * (1.f / d);
+  float m = 0.f;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const int c = (i * 32 + lane_id()) * 4;
@@ -255,7 +276,9 @@ __global__ void __launch_bounds__(128) rmsnorm_bwd_kernel(const float* __restric
     o.w = p[i].w + r * (g[i].w - bf16_hi(yy[i].y) * dot);
     *reinterpret_cast<float4*>(dx + off + c) = o;
     store_bf16x4(dxb + off + c, o);
+    if (amax) m = fmaxf(m, fmaxf(fmaxf(abs_bf16(o.x), abs_bf16(o.y)), fmaxf(abs_bf16(o.z), abs_bf16(o.w))));
   }
+  if (amax) amax_slot_update(amax, m, row);
 }
 
 // ------------------------------------------- residual scales and backout
@@ -581,7 +604,8 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
                               const bf16* __restrict__ dv, const bf16* __restrict__ qn,
                               const bf16* __restrict__ kn, const float* __restrict__ rq,
                               const float* __restrict__ rk, const float2* __restrict__ rope,
-                              bf16* __restrict__ dqkv, int B, int T, int H, int Hkv) {
+                              bf16* __restrict__ dqkv, int B, int T, int H, int Hkv,
+                              unsigned int* __restrict__ amax) {
   const long long w = static_cast<long long>(blockIdx.x) * (blockDim.x / 32) + warp_id();
   const long long total = static_cast<long long>(B) * H * T;
   if (w >= total) return;
@@ -597,6 +621,7 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
   // row of dqkv: q (d) | k (kvd) | v (kvd); head h of k and v only for h < Hkv
   bf16* out = dqkv + m * (d + 2 * kvd) + h * 128;
   const bool has_kv = !kGrouped || h < Hkv;
+  float am = 0.f;   // max |written value| (for fp8 scales)
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
     if (which == 1 && !has_kv) break;
@@ -624,11 +649,16 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
     const float ol1 = rl1 * e1.x + rh1 * e1.y, oh1 = -rl1 * e1.y + rh1 * e1.x;
     *reinterpret_cast<uint32_t*>(out + which * d + i0) = pack_bf16x2(ol0, ol1);
     *reinterpret_cast<uint32_t*>(out + which * d + 64 + i0) = pack_bf16x2(oh0, oh1);
+    if (amax) am = fmaxf(am, fmaxf(fmaxf(abs_bf16(ol0), abs_bf16(ol1)), fmaxf(abs_bf16(oh0), abs_bf16(oh1))));
   }
   if (has_kv) {
     const uint2 vv = *reinterpret_cast<const uint2*>(dv + src + 4 * lane_id());
     *reinterpret_cast<uint2*>(out + d + kvd + 4 * lane_id()) = vv;
+    if (amax)
+      am = fmaxf(am, fmaxf(fmaxf(fabsf(bf16_lo(vv.x)), fabsf(bf16_hi(vv.x))),
+                           fmaxf(fabsf(bf16_lo(vv.y)), fabsf(bf16_hi(vv.y)))));
   }
+  if (amax) amax_slot_update(amax, am, w);
 }
 
 // ------------------------------------------------------- cross-entropy finish
@@ -1032,11 +1062,15 @@ __global__ void __launch_bounds__(256) amax_bf16_kernel(const bf16* __restrict__
   }
 }
 
+// amax of matrix z: the max over its nslots words (1: one word per matrix)
 __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const bf16* __restrict__ x, long long n,
                                                             const unsigned int* __restrict__ amax_bits,
-                                                            uint8_t* __restrict__ q, float* __restrict__ inv) {
+                                                            uint8_t* __restrict__ q, float* __restrict__ inv,
+                                                            int nslots) {
   const int z = blockIdx.y;
-  const float amax = __uint_as_float(amax_bits[z]);
+  unsigned int ab = 0;
+  for (int i = 0; i < nslots; ++i) ab = max(ab, amax_bits[z * nslots + i]);
+  const float amax = __uint_as_float(ab);
   const float sc = amax > 0.f ? 448.f / amax : 1.f;
   if (blockIdx.x == 0 && threadIdx.x == 0) inv[z] = amax > 0.f ? amax / 448.f : 1.f;
   const bf16* xz = x + z * n;
@@ -1083,10 +1117,10 @@ void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, i
 
 #define GPT_NV_CASES(X) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16)
 
-void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s) {
+void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s, unsigned int* amax) {
   if (M <= 0) return;
   switch (d / 128) {
-#define GPT_FWD_CASE(n) case n: rmsnorm_fwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(x, y, rstd, M); break;
+#define GPT_FWD_CASE(n) case n: rmsnorm_fwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(x, y, rstd, M, amax); break;
     GPT_NV_CASES(GPT_FWD_CASE)
 #undef GPT_FWD_CASE
     default: break;
@@ -1094,11 +1128,11 @@ void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cuda
 }
 
 void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dxb, int M, int d,
-                        bool accumulate, cudaStream_t s) {
+                        bool accumulate, cudaStream_t s, unsigned int* amax) {
   if (M <= 0) return;
   switch (d / 128) {
 #define GPT_BWD_CASE(n) \
-  case n: rmsnorm_bwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(dy, y, rstd, dx, dxb, M, accumulate ? 1 : 0); break;
+  case n: rmsnorm_bwd_kernel<n><<<cdiv(M, 4), 128, 0, s>>>(dy, y, rstd, dx, dxb, M, accumulate ? 1 : 0, amax); break;
     GPT_NV_CASES(GPT_BWD_CASE)
 #undef GPT_BWD_CASE
     default: break;
@@ -1106,12 +1140,13 @@ void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float
 }
 
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn, const float* rq,
-                   const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s, int Hkv) {
+                   const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s, int Hkv,
+                   unsigned int* amax) {
   const long long rows = 1ll * B * H * T;
   if (Hkv <= 0 || Hkv == H)
-    qk_bwd_kernel<false><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, H);
+    qk_bwd_kernel<false><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, H, amax);
   else
-    qk_bwd_kernel<true><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, Hkv);
+    qk_bwd_kernel<true><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, Hkv, amax);
 }
 
 void launch_ce_finish(bf16* z, const float2* stats, const float* zt, const int* tgt, float* row_loss, int rows,
@@ -1276,7 +1311,20 @@ void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* am
   cudaMemsetAsync(amax_bits, 0, static_cast<size_t>(nmat) * sizeof(unsigned int), s);
   const int blocks = static_cast<int>(std::min<long long>((n / 8 + 255) / 256 + 1, 4 * 148));
   amax_bf16_kernel<<<dim3(blocks, nmat), 256, 0, s>>>(x, n, amax_bits);
-  quantize_e4m3_kernel<<<dim3(blocks, nmat), 256, 0, s>>>(x, n, amax_bits, q, inv);
+  quantize_e4m3_kernel<<<dim3(blocks, nmat), 256, 0, s>>>(x, n, amax_bits, q, inv, 1);
+}
+
+void launch_amax_slots(const bf16* x, long long n, unsigned int* slots, cudaStream_t s) {
+  if (n <= 0) return;
+  const int blocks = static_cast<int>(std::min<long long>((n / 8 + 255) / 256 + 1, 4 * 148));
+  amax_bf16_kernel<<<dim3(blocks, 1), 256, 0, s>>>(x, n, slots);
+}
+
+void launch_quantize_e4m3_slots(const bf16* x, long long n, const unsigned int* slots, uint8_t* q, float* inv,
+                                cudaStream_t s) {
+  if (n <= 0) return;
+  const int blocks = static_cast<int>(std::min<long long>((n / 8 + 255) / 256 + 1, 4 * 148));
+  quantize_e4m3_kernel<<<dim3(blocks, 1), 256, 0, s>>>(x, n, slots, q, inv, kAmaxSlots);
 }
 
 void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s) {

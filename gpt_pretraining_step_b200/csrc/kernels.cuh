@@ -17,19 +17,27 @@ void launch_rope_table(float2* tab, int T, cudaStream_t s);
 void launch_embed_fwd(const int* tok, const bf16* wte, float* x, int M, int d, int V, int* err,
                       cudaStream_t s);
 
-// y = x / sqrt(mean(x^2) + 1e-6) per row (bf16 out), rstd saved; d a multiple of 128, <= 2048.
-void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s);
+// fp8 scale words: a tensor's amax is kept in kAmaxSlots words (zeroed before
+// its producer runs) that the producer raises with atomicMax on the bits of
+// max |bf16 output|; the quantiser takes the max over them.
+constexpr int kAmaxSlots = 32;
 
-// dx (+)= rstd * (dy - y * mean(dy * y)); also writes dx in bf16.
+// y = x / sqrt(mean(x^2) + 1e-6) per row (bf16 out), rstd saved; d a multiple
+// of 128, <= 2048; amax: optional scale words of y.
+void launch_rmsnorm_fwd(const float* x, bf16* y, float* rstd, int M, int d, cudaStream_t s,
+                        unsigned int* amax = nullptr);
+
+// dx (+)= rstd * (dy - y * mean(dy * y)); also writes dx in bf16 (amax:
+// optional scale words of that copy).
 void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float* dx, bf16* dx_bf16,
-                        int M, int d, bool accumulate, cudaStream_t s);
+                        int M, int d, bool accumulate, cudaStream_t s, unsigned int* amax = nullptr);
 
 // Per-head QK-norm and RoPE backward plus the v copy, into dqkv [M, d + 2
 // Hkv 128] (dq is the fp32 attention-backward accumulator, dk and dv bf16,
 // kv head j of batch b at head row b*H + j; Hkv 0 = H).
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn,
                    const float* rq, const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H,
-                   cudaStream_t s, int Hkv = 0);
+                   cudaStream_t s, int Hkv = 0, unsigned int* amax = nullptr);
 
 // Per row: lse from the (max, sumexp) tile partials, row loss = lse - z[target],
 // and z <- (softmax(z) - onehot(target)) * inv_count in place.
@@ -121,6 +129,13 @@ void launch_ve_dxn(float* dxn, const float* dz, const float* wg, int M, int d, i
 // inv[z] = amax / 448 (1 for an all-zero matrix).  amax_bits: nmat words of scratch.
 void launch_quantize_e4m3(const bf16* x, long long n, int nmat, unsigned int* amax_bits, uint8_t* q, float* inv,
                           cudaStream_t s);
+
+// fp8 with precomputed scale words: the amax of x (n bf16 values) into slot 0
+// of `slots` (for a tensor whose producer does not keep it), and the e4m3
+// quantisation of x with the max over the kAmaxSlots words.
+void launch_amax_slots(const bf16* x, long long n, unsigned int* slots, cudaStream_t s);
+void launch_quantize_e4m3_slots(const bf16* x, long long n, const unsigned int* slots, uint8_t* q, float* inv,
+                                cudaStream_t s);
 
 // dst = bf16(src), n elements.
 void launch_cast_bf16(const float* src, bf16* dst, long long n, cudaStream_t s);

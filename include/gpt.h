@@ -69,10 +69,14 @@ enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
  *   vocab     vocabulary size, a multiple of 8 (32768 in the pages' runs)
  *   batch     sequences per step; seq_len tokens each
  *   head_dim  must be 128; mlp_mult must be 4
- *   precision 0 = bf16 GEMMs; 1 = the four block projections of the forward
- *             pass (q|k|v, attention output, MLP up, MLP down) on fp8 e4m3
+ *   precision 0 = bf16 GEMMs; 1 = every GEMM of the four block projections
+ *             (q|k|v, attention output, MLP up, MLP down) on fp8 e4m3
  *             operands with dynamic per-tensor scales (448 / amax of the
- *             tensor); attention, lm_head and the backward stay bf16
+ *             tensor, the amax kept by the kernel that produced it): the
+ *             forward products X W, the activation gradients dY W^T and the
+ *             weight gradients X^T dY, with X, W and dY quantised ("3.
+ *             Gestión de Precisión": FP8 with per-tensor scaling on most
+ *             layers); attention and the lm_head stay bf16
  *   ns_tf32_steps  operand precision of the five Newton-Schulz steps:
  *             -1 = fp16 operands at the full tensor rate with fp32 iterates
  *             (the recommended setting); 0..5 = that many leading steps with
@@ -215,6 +219,19 @@ int gpt_block_region(const gpt_ctx* ctx, int what, int kind, int l0, int l1, siz
  * decay. */
 int adamw_step(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay);
 
+/* adamw_step for data-parallel ranks that shard the AdamW state by rows
+ * ("¿Cómo Entrenar Tu Propio ChatGPT por $50?", section "2. Optimizador
+ * Muon", distributed training: ZeRO-2 sharding): only rows
+ * [part R / nparts, (part + 1) R / nparts) of the token embedding (R = vocab)
+ * and of the lm_head (R = d_model) are updated, with their moments and bf16
+ * working copies; the residual-extras scalars and value-embedding tables and
+ * gates, when on, are updated whole.  The step count advances by one, as for
+ * adamw_step.  The parts of all ranks together give exactly what one
+ * adamw_step gives; each rank then shares its rows' bf16 copies
+ * (gpt_tensor_region).  0 <= part < nparts, else GPT_EINVAL. */
+int adamw_step_shard(gpt_ctx* ctx, float lr, float beta1, float beta2, float eps, float weight_decay, int part,
+                     int nparts);
+
 /* The number of adamw_step calls so far (its bias correction uses it), for a
  * checkpoint: with every tensor's value and optimizer state (gpt_get_tensor)
  * it restores a context exactly.  A negative count is GPT_EINVAL. */
@@ -248,6 +265,34 @@ int gpt_tensor_info(const gpt_ctx* ctx, int id, int32_t* rows, int32_t* cols, in
  * for GPT_KIND_NORMUON_V. */
 int gpt_get_tensor(gpt_ctx* ctx, int id, int kind, float* dst);
 int gpt_set_tensor(gpt_ctx* ctx, int id, int kind, const float* src);
+
+/* Byte range of rows row0 .. row1-1 of tensor id (the embedding, the lm_head
+ * or a block matrix; ids as for gpt_tensor_info) inside param_buf for
+ * GPT_REGION_MASTER (fp32) and GPT_REGION_BF16 (the bf16 working copy), or
+ * inside state_buf for GPT_REGION_GRAD (fp32 gradient).  Rows are contiguous
+ * (row-major), so the range is one span.  Other ids, or a row range outside
+ * [0, rows], are GPT_EINVAL. */
+int gpt_tensor_region(const gpt_ctx* ctx, int what, int id, int row0, int row1, size_t* offset_bytes,
+                      size_t* size_bytes);
+
+/* Gradient buckets, in the order in which gpt_fwd_bwd completes them: 0 the
+ * lm_head (done once the last lm_head chunk is through, early in the
+ * backward), 1..4 one block matrix kind over every layer (fused q|k|v,
+ * attention output, MLP up, MLP down; each done by one batched
+ * weight-gradient launch after the backward sweep), 5 the token embedding
+ * with the residual-extras and value-embedding gradients (done at the end).
+ * Each bucket is one span of state_buf (gpt_grad_bucket); together they tile
+ * the gpt_grad_region span, which is laid out in this order. */
+enum { GPT_GRAD_BUCKETS = 6 };
+int gpt_grad_bucket(const gpt_ctx* ctx, int bucket, size_t* offset_bytes, size_t* size_bytes);
+
+/* Registers n <= GPT_GRAD_BUCKETS caller-owned CUDA events (cudaEvent_t,
+ * created by the caller on the context's device): every later gpt_fwd_bwd
+ * records events[i] on the context's stream as soon as bucket i is complete,
+ * so a data-parallel caller can start reducing a bucket on another stream
+ * (cudaStreamWaitEvent) while the backward still runs.  n = 0 stops the
+ * recording.  The events must outlive their registration. */
+int gpt_set_grad_events(gpt_ctx* ctx, void* const* events, int n);
 
 /* Byte range of the fp32 gradients of every parameter inside state_buf
  * (one contiguous span; alignment padding inside it stays zero).  Data
