@@ -293,13 +293,13 @@ void make_plan(const Dims& D, Plan& P) {
     // and of the gradients they meet, with their scales
     const bool f8 = D.fp8 != 0;
     const size_t wn[4] = {L * d * qc, L * d * d, L * d * F, L * F * d};
-    for (int i = 0; i < 4; ++i) P.wq8[i] = ab.take(f8 ? wn[i] : 16);
+    for (int i = 0; i < 4; ++i) P.wq8[i] = ab.take(f8 && i > 0 ? wn[i] : 16);   // q|k|v stays bf16
     P.winv = ab.take(4 * L * 4);
     P.wamax = ab.take(4 * L * 4);
     const size_t acols[4] = {d, d, d, F}, gcols[4] = {qc, d, F, d};
     for (int i = 0; i < 4; ++i) {
-      P.act8[i] = ab.take(f8 ? L * M * acols[i] : 16);
-      P.grad8[i] = ab.take(f8 ? L * M * gcols[i] : 16);
+      P.act8[i] = ab.take(f8 && i > 0 ? L * M * acols[i] : 16);
+      P.grad8[i] = ab.take(f8 && i > 0 ? L * M * gcols[i] : 16);
     }
     P.f8slots = ab.take(8 * L * kAmaxSlots * 4);
     P.f8inv = ab.take(8 * L * 4);
@@ -555,24 +555,27 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   // in the order of the weight kinds they meet
   auto slots8 = [&](int t, int l) { return D.fp8 ? f8slots + (static_cast<size_t>(t) * L + l) * kAmaxSlots : nullptr; };
   auto inv8 = [&](int t, int l) { return f8inv + t * L + l; };
+  // the q|k|v projection (weight kind 0) stays bf16: its rounding error enters
+  // the QK-normalised attention logits, which the softmax amplifies
+  auto f8 = [&](int k) { return D.fp8 && k != 0; };
   auto act8 = [&](int k, int l) { return c->A<uint8_t>(P.act8[k]) + static_cast<size_t>(l) * M * acols[k]; };
   auto grad8 = [&](int k, int l) { return c->A<uint8_t>(P.grad8[k]) + static_cast<size_t>(l) * M * gcols[k]; };
   if (D.fp8) {
     ProfScope ps(c, GPT_PROF_FP8_QUANT);
     GPT_CK(cudaMemsetAsync(f8slots, 0, static_cast<size_t>(8) * L * kAmaxSlots * 4, s));
-    for (int gi = 0; gi < 4; ++gi)
+    for (int gi = 1; gi < 4; ++gi)
       launch_quantize_e4m3(c->Wb(2 + gi), wn[gi], L, c->A<unsigned int>(P.wamax) + gi * L,
                            c->A<uint8_t>(P.wq8[gi]), winv + gi * L, s);
-    c->launches += 8;
+    c->launches += 6;
   }
   // operand A of a forward projection of weight kind k: bf16 as it is, or its
   // e4m3 copy (kept for the weight gradient) with the weight's e4m3 copy as B
   auto fwd_a = [&](GemmCall& g, const bf16* a, long long rows, long long cols, int grp, int l) {
-    if (!D.fp8) {
+    const int k = grp - 2;
+    if (!f8(k)) {
       g.A = a;
       return;
     }
-    const int k = grp - 2;
     {
       ProfScope ps(c, GPT_PROF_FP8_QUANT);
       if (k == 1) {   // the attention output keeps no amax of its own
@@ -591,7 +594,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   // operand A of an activation-gradient GEMM against weight kind k: the bf16
   // gradient, or its e4m3 copy with the weight's e4m3 copy as B (K-major)
   auto bwd_a = [&](GemmCall& g, const bf16* a, long long cols, int k, int l) {
-    if (!D.fp8) {
+    if (!f8(k)) {
       g.A = a;
       return;
     }
@@ -626,7 +629,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_NORM);
-      launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s, slots8(0, l));
+      launch_rmsnorm_fwd(x, xn1l, r1 + static_cast<size_t>(l) * M, M, d, s);
     }
     {
       GemmCall g = base_call(M, D.qc, d);
@@ -814,7 +817,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
       launch_qk_bwd(dqf, dk, dv, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
-                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv, slots8(4, l));
+                    rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv);
     }
     c->launches += 3;
     const int vs = D.ve_slot(l);
@@ -882,7 +885,7 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       g.batch = L;
       g.A = w.a; g.a_mn = true; g.lda = w.lda; g.a_bs = w.a_bs;
       g.B = w.b; g.b_mn = true; g.ldb = w.ldb; g.b_bs = w.b_bs;
-      if (D.fp8) {
+      if (f8(kind)) {
         // e4m3 copies of the activations and gradients, one scale pair per layer
         g.es = 1;
         g.A = act8(kind, 0); g.lda = acols[kind]; g.a_bs = 1ll * M * acols[kind];

@@ -61,6 +61,19 @@ constexpr int HD = 128;
 // rescales its rows of O in TMEM (the previous P V has completed by then:
 // S of this block was issued after it).
 
+// Exponentials per group of 8 scores evaluated on the MUFU unit (the rest by
+// the polynomial on the FMA pipe): forward, alternating between two values
+// over consecutive groups; backward, one value.  Even numbers (pairs).
+#ifndef GPT_FWD_MUFU_EVEN
+#define GPT_FWD_MUFU_EVEN 6
+#endif
+#ifndef GPT_FWD_MUFU_ODD
+#define GPT_FWD_MUFU_ODD 6
+#endif
+#ifndef GPT_BWD_MUFU
+#define GPT_BWD_MUFU 8
+#endif
+
 constexpr int TF_TILE = 16384;                // one [128 rows][128 B] swizzled tile
 constexpr int TF_BUF = 2 * TF_TILE;           // 128 x 128 bf16 as two 64-column tiles
 constexpr int TF_SMEM = 6 * TF_BUF + 256;
@@ -406,7 +419,7 @@ __global__ void __launch_bounds__(384, 1)
               f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c * 64 + k + e]), __uint_as_float(sr[c * 64 + k + e + 1])),
                                sl2, nb2),
                         x0, x1);
-              if (e < 4 || (e == 4 && (k & 8))) {
+              if (e < ((k & 8) ? GPT_FWD_MUFU_ODD : GPT_FWD_MUFU_EVEN)) {
                 p[e] = ex2_approx(x0);
                 p[e + 1] = ex2_approx(x1);
               } else {
@@ -522,9 +535,8 @@ __device__ __forceinline__ void store_row_units(uint8_t* tile, const uint32_t (&
     *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
 }
 
-// K, V, two Q slots, two dO slots, dS^T; then -lse / -D of two query blocks
-// and the barriers
-constexpr int TB_SMEM = 7 * TF_BUF + 2048 + 256;
+constexpr int TB_STAGE = 32768;   // dQ staging: 64 queries x 128 dims fp32
+constexpr int TB_SMEM = 6 * TF_BUF + TB_STAGE + 2048 + 256;
 
 // Query-block loop of key block j: nb query blocks j .. (window end) for each
 // of the G query heads of the group.
@@ -554,7 +566,7 @@ __device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int kvs, 
 __global__ void __launch_bounds__(448, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
-                       float* __restrict__ dq, const float* __restrict__ lse,
+                       const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
                        const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int Hkv,
                        int kvs, int T, int wl, float scale, int n_units, int* sched, int* err,
                        long long wait_cycles) {
@@ -569,26 +581,27 @@ __global__ void __launch_bounds__(448, 1)
   uint8_t* sK = sm;
   uint8_t* sV = sm + TF_BUF;
   uint8_t* sQ = sm + 2 * TF_BUF;     // two slots
-  uint8_t* sdO = sm + 4 * TF_BUF;     // two slots
-  uint8_t* sdSt = sm + 6 * TF_BUF;
-  float* lse_s = reinterpret_cast<float*>(sm + 7 * TF_BUF);   // [2][128]: -lse * log2(e)
-  float* dd_s = lse_s + 256;                                   // [2][128]: -D
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 7 * TF_BUF + 2048);
+  uint8_t* sdO = sm + 4 * TF_BUF;
+  uint8_t* sdSt = sm + 5 * TF_BUF;
+  uint8_t* sStage = sm + 6 * TF_BUF;
+  float* lse_s = reinterpret_cast<float*>(sm + 6 * TF_BUF + TB_STAGE);   // [2][128]: -lse * log2(e)
+  float* dd_s = lse_s + 256;                                              // [2][128]: -D
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 6 * TF_BUF + TB_STAGE + 2048);
   uint64_t* kv_full = bars + 0;
   uint64_t* q_full = bars + 1;    // [2]
   uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* do_full = bars + 5;   // [2]
-  uint64_t* do_empty = bars + 7;  // [2] dV_i complete: dO_i and P_i are no longer read
-  uint64_t* s_full = bars + 9;    // S^T_i in TMEM
-  uint64_t* s_free = bars + 10;   // S^T_i read by the softmax warps
-  uint64_t* dp_full = bars + 11;  // dP^T_i in TMEM
-  uint64_t* p_ready = bars + 12;  // P_i in TMEM
-  uint64_t* mm_done = bars + 13;  // dV, dK, dQ^T of block i complete
-  uint64_t* dq_free = bars + 14;  // dQ^T_i read by the dQ warps
-  uint64_t* drain = bars + 15;
-  uint64_t* ds_ready = bars + 16; // dS_i in shared memory
-  uint64_t* kv_empty = bars + 17; // an item's last products complete (K and V free) and every warp has its number
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 18);
+  uint64_t* do_full = bars + 5;
+  uint64_t* do_empty = bars + 6;  // dV_i complete: dO_i and P_i are no longer read
+  uint64_t* s_full = bars + 7;    // S^T_i in TMEM
+  uint64_t* s_free = bars + 8;    // S^T_i read by the softmax warps
+  uint64_t* dp_full = bars + 9;   // dP^T_i in TMEM
+  uint64_t* p_ready = bars + 10;  // P_i in TMEM
+  uint64_t* mm_done = bars + 11;  // dV, dK, dQ^T of block i complete
+  uint64_t* dq_free = bars + 12;  // dQ^T_i read by the dQ warps
+  uint64_t* drain = bars + 13;
+  uint64_t* ds_ready = bars + 14; // dS_i in shared memory
+  uint64_t* kv_empty = bars + 15; // an item's last products complete (K and V free) and every warp has its number
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 16);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* item_ring = reinterpret_cast<volatile int*>(tmem_holder + 2);   // [4]
 
@@ -599,10 +612,9 @@ __global__ void __launch_bounds__(448, 1)
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1 + 12);   // the MMA commit and one arrival per softmax and dQ warp
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
-      mbar_init(&do_full[i], 1); mbar_init(&do_empty[i], 1);
-    }
+    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+    mbar_init(do_full, 1);
+    mbar_init(do_empty, 1);
     mbar_init(s_full, 1);
     mbar_init(s_free, 256);
     mbar_init(dp_full, 1);
@@ -617,6 +629,7 @@ __global__ void __launch_bounds__(448, 1)
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
     tma_prefetch_desc(&tdo);
+    tma_prefetch_desc(&tdq);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, 512);
@@ -641,11 +654,10 @@ __global__ void __launch_bounds__(448, 1)
         tma_load_3d(sQ + s * TF_BUF, &tq, &q_full[s], 0, i * 128, bh);
         tma_load_3d(sQ + s * TF_BUF + TF_TILE, &tq, &q_full[s], 64, i * 128, bh);
         ++issued_q;
-        // dO_i goes to slot i & 1 once dV_{i-2} has read that slot
-        if (!mbar_wait(&do_empty[s], ((g >> 1) & 1) ^ 1u, abort_flag, err, wlim)) return false;
-        mbar_arrive_expect_tx(&do_full[s], TF_BUF);
-        tma_load_4d(sdO + s * TF_BUF, &tdo, &do_full[s], 0, h, i * 128, kb.b);
-        tma_load_4d(sdO + s * TF_BUF + TF_TILE, &tdo, &do_full[s], 64, h, i * 128, kb.b);
+        if (!mbar_wait(do_empty, (g & 1) ^ 1u, abort_flag, err, wlim)) return false;
+        mbar_arrive_expect_tx(do_full, TF_BUF);
+        tma_load_4d(sdO, &tdo, do_full, 0, h, i * 128, kb.b);
+        tma_load_4d(sdO + TF_TILE, &tdo, do_full, 64, h, i * 128, kb.b);
         ++issued_do;
         ++g;
         return true;
@@ -695,8 +707,8 @@ __global__ void __launch_bounds__(448, 1)
           for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(kv_full, (nblk - 1) & 1); ++x) {}
         for (int it = (issued_q > 2 ? issued_q - 2 : 0); it < issued_q; ++it)
           for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(&q_full[it & 1], (it >> 1) & 1); ++x) {}
-        for (int it = (issued_do > 2 ? issued_do - 2 : 0); it < issued_do; ++it)
-          for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(&do_full[it & 1], (it >> 1) & 1); ++x) {}
+        if (issued_do > 0)
+          for (uint32_t x = 0; x < (1u << 20) && !mbar_try_wait(do_full, (issued_do - 1) & 1); ++x) {}
       }
     }
   } else if (warp == 1) {
@@ -705,8 +717,7 @@ __global__ void __launch_bounds__(448, 1)
       constexpr uint32_t IDESC_KK = make_idesc(1, 128, false, false);   // S^T, dP^T
       constexpr uint32_t IDESC_KM = make_idesc(1, 128, false, true);    // dV (A in TMEM), dK
       constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ^T
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      auto do_addr = [&](int gi) { return smem_u32(sdO + (gi & 1) * TF_BUF); };
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), do_addr = smem_u32(sdO);
       const uint32_t dst_addr = smem_u32(sdSt);
       // X^T = A B^T over the 128 head dims, both operands K-major; the empty
       // asm keeps the descriptors from being hoisted into registers
@@ -737,11 +748,11 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           qk_product(tmem, k_addr, smem_u32(sQ + (g0 & 1) * TF_BUF));   // S^T of the first block
           umma_commit(s_full);
-          ok = mbar_wait(&do_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim) &&
-               (g0 == 0 || mbar_wait(&do_empty[(g0 - 1) & 1], ((g0 - 1) >> 1) & 1, abort_flag, err, wlim));
+          ok = mbar_wait(do_full, g0 & 1, abort_flag, err, wlim) &&
+               (g0 == 0 || mbar_wait(do_empty, (g0 - 1) & 1, abort_flag, err, wlim));
           if (!ok) break;
           tc_fence_after();
-          qk_product(tmem + 128, v_addr, do_addr(g0));   // dP^T of the first block
+          qk_product(tmem + 128, v_addr, do_addr);   // dP^T of the first block
           umma_commit(dp_full);
           if (n_it > 1) {
             ok = mbar_wait(s_free, g0 & 1, abort_flag, err, wlim) &&
@@ -760,14 +771,14 @@ __global__ void __launch_bounds__(448, 1)
             // dV += P^T dO: A = P^T from TMEM, 16 queries = 8 packed columns per
             // step; queries 0..63 at columns 128.., 64..127 at columns 192..
             {
-              uint64_t ddo = smem_desc_sw128(do_addr(gi), TF_TILE, 1024);
+              uint64_t ddo = smem_desc_sw128(do_addr, TF_TILE, 1024);
               asm volatile("" : "+l"(ddo));
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
                 umma_f16_tmem_a(tmem + 256, tmem + 128 + (kk >> 2) * 64 + (kk & 3) * 8, ddo + ((kk * 2048) >> 4),
                                 IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
             }
-            umma_commit(&do_empty[s]);
+            umma_commit(do_empty);
             // dK and dQ^T once dS_i is in shared memory (the softmax warps compute it
             // while dV runs)
             if (!mbar_wait(ds_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
@@ -805,13 +816,10 @@ __global__ void __launch_bounds__(448, 1)
             if (it + 1 == n_it) umma_commit(kv_empty);   // K and V of this key block are free
             if (it + 1 < n_it) {
               // dP^T_{i+1} overwrites P^T_i: dV_i must have completed
-              if (!mbar_wait(&do_empty[s], (gi >> 1) & 1, abort_flag, err, wlim) ||
-                  !mbar_wait(&do_full[(gi + 1) & 1], ((gi + 1) >> 1) & 1, abort_flag, err, wlim)) {
-                ok = false;
-                break;
-              }
+              if (!mbar_wait(do_empty, gi & 1, abort_flag, err, wlim) ||
+                  !mbar_wait(do_full, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
               tc_fence_after();
-              qk_product(tmem + 128, v_addr, do_addr(gi + 1));
+              qk_product(tmem + 128, v_addr, do_addr);
               umma_commit(dp_full);
             }
             if (it + 2 < n_it) {
@@ -830,24 +838,26 @@ __global__ void __launch_bounds__(448, 1)
     }
   } else if (warp >= 10) {
     // ------------------------------------------------------------------ dQ
-    // Lane i of warp quarter q holds head dim 32 q + i of dQ^T for the
-    // block's 128 queries; for each query the warp adds its 32 consecutive
-    // dims into the fp32 dq rows with one coalesced reduction (128 bytes).
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    uint8_t* box = sStage + quarter * 8192;   // [64 queries][32 dims] fp32, 128-byte swizzle
     const uint64_t sc2 = f2_pack(scale, scale);
     bool ok = true;
-    // queries q0 + c0 .. q0 + c0 + 63 from the two loaded 32-column chunks
-    auto add_rows = [&](const uint32_t (&va)[32], const uint32_t (&vb)[32], float* base, int nrows) {
+    // dims lane of this warp's quarter for 64 queries -> the box, transposed
+    auto stage = [&](const uint32_t (&va)[32], const uint32_t (&vb)[32]) {
+      if (lane == 0) bulk_wait_read_all();   // the box's previous contents have been read
+      __syncwarp();
 #pragma unroll
       for (int qq = 0; qq < 64; qq += 2) {
         const uint32_t (&v)[32] = qq < 32 ? va : vb;
         const int e = qq & 31;
         float a0, a1;
         f2_unpack(f2_mul(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2), a0, a1);
-        if (qq < nrows) atomicAdd(base + qq * HD, a0);
-        if (qq + 1 < nrows) atomicAdd(base + (qq + 1) * HD, a1);
+        *reinterpret_cast<float*>(box + qq * 128 + (((lane >> 2) ^ (qq & 7)) << 4) + (lane & 3) * 4) = a0;
+        *reinterpret_cast<float*>(box + (qq + 1) * 128 + (((lane >> 2) ^ ((qq + 1) & 7)) << 4) + (lane & 3) * 4) = a1;
       }
+      fence_proxy_async_smem();
+      __syncwarp();
     };
     int g = 0;
     for (int n = 0; ok; ++n) {
@@ -864,8 +874,6 @@ __global__ void __launch_bounds__(448, 1)
         const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         for (int it = 0; it < kb.n_it && ok; ++it, ++g) {
           const int q0 = kb.q_block(it) * 128, bh = kb.b * H + kb.q_head(it);
-          float* rows = dq + (static_cast<long long>(bh) * T + q0) * HD + quarter * 32 + lane;
-          const int nrows = min(128, T - q0);
           const bool got = mbar_wait(mm_done, g & 1, abort_flag, err, wlim);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
@@ -874,16 +882,25 @@ __global__ void __launch_bounds__(448, 1)
           tmem_load32_async(tmem + lane_base, va);
           tmem_load32_async(tmem + lane_base + 32, vb);
           tmem_wait_ld();
-          add_rows(va, vb, rows, nrows);
+          stage(va, vb);
+          if (lane == 0) {
+            tma_reduce_add_3d(&tdq, box, 32 * quarter, q0, bh);
+            bulk_commit();
+          }
           tmem_load32_async(tmem + lane_base + 64, va);
           tmem_load32_async(tmem + lane_base + 96, vb);
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(dq_free);
-          add_rows(va, vb, rows + 64 * HD, nrows - 64);
+          stage(va, vb);
+          if (lane == 0) {
+            tma_reduce_add_3d(&tdq, box, 32 * quarter, q0 + 64, bh);
+            bulk_commit();
+          }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();
   } else {
     // ------------------------------------------------------- P, dS, dK, dV
     const int quarter = warp & 3;
@@ -975,7 +992,7 @@ __global__ void __launch_bounds__(448, 1)
                 f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[kq + e]), __uint_as_float(sr[kq + e + 1])), sl2,
                                  f2_pack(nl[e], nl[e + 1])),
                           x0, x1);
-                if (e < 6) {
+                if (e < GPT_BWD_MUFU) {
                   p[e] = ex2_approx(x0);
                   p[e + 1] = ex2_approx(x1);
                 } else {
@@ -1181,7 +1198,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const long long rows = 1ll * B * H * T;
   attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (kv_stride <= 0) kv_stride = Hkv;
   const long long bh = 1ll * B * H, bhkv = 1ll * B * kv_stride;
   const long long dims[4] = {HD, H, T, B};
@@ -1189,7 +1206,8 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const int box[4] = {64, 1, 128, 1};
   if (H % Hkv || kv_stride < Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
-      !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box)) {
+      !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
+      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }
@@ -1202,7 +1220,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const int grid = static_cast<int>(std::min<long long>(n_units, device_sm_count()));
   const int wl = window_bound(window, T);
   int* word = wl >= T ? nullptr : sched_word(sched, s);
-  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, dq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
+  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
                                                 1.f / sqrtf(static_cast<float>(HD)), static_cast<int>(n_units),
                                                 word, err, wait_cycles);
 }

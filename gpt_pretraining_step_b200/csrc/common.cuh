@@ -95,26 +95,19 @@ constexpr long long kShortWaitCycles = 1000000ll;
 
 // Wait for the phase with the given parity to complete.  Returns false if
 // another thread raised *abort or the wait ran past `limit` SM cycles; in the
-// latter case this thread raises *abort itself and sets the error flag.
+// latter case this thread raises *abort itself and sets the error flag.  One
+// polling loop serves both kinds of limit (the kernels have dozens of wait
+// sites, so each must stay small): a short limit polls with the non-blocking
+// test and reads the clock on every probe, a long one with try_wait and
+// reads the clock every 64 probes.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err, long long limit) {
-  if (limit < kShortWaitCycles) {
-    const long long t0 = clock64();
-    for (;;) {
-      if (mbar_test_wait(bar, parity)) return true;
-      if (*abort) return false;
-      if (clock64() - t0 > limit) {
-        *abort = 1;
-        if (err) atomicOr(err, ERRF_TIMEOUT);
-        return false;
-      }
-    }
-  }
-  if (mbar_try_wait(bar, parity)) return true;
+  const bool fine = limit < kShortWaitCycles;
+  if (!fine && mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
+    if (fine ? mbar_test_wait(bar, parity) : mbar_try_wait(bar, parity)) return true;
+    if (fine || (i & 63u) == 0) {
       if (*abort) return false;
       if (clock64() - t0 > limit) {
         *abort = 1;

@@ -69,14 +69,15 @@ enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
  *   vocab     vocabulary size, a multiple of 8 (32768 in the pages' runs)
  *   batch     sequences per step; seq_len tokens each
  *   head_dim  must be 128; mlp_mult must be 4
- *   precision 0 = bf16 GEMMs; 1 = every GEMM of the four block projections
- *             (q|k|v, attention output, MLP up, MLP down) on fp8 e4m3
- *             operands with dynamic per-tensor scales (448 / amax of the
- *             tensor, the amax kept by the kernel that produced it): the
- *             forward products X W, the activation gradients dY W^T and the
- *             weight gradients X^T dY, with X, W and dY quantised ("3.
- *             Gestión de Precisión": FP8 with per-tensor scaling on most
- *             layers); attention and the lm_head stay bf16
+ *   precision 0 = bf16 GEMMs; 1 = every GEMM of the attention output, MLP
+ *             up and MLP down projections on fp8 e4m3 operands with dynamic
+ *             per-tensor scales (448 / amax of the tensor, the amax kept by
+ *             the kernel that produced it): the forward products X W, the
+ *             activation gradients dY W^T and the weight gradients X^T dY,
+ *             with X, W and dY quantised ("3. Gestión de Precisión": FP8
+ *             with per-tensor scaling on most layers); the q|k|v projection
+ *             (its rounding enters the QK-normalised attention logits),
+ *             attention and the lm_head stay bf16
  *   ns_tf32_steps  operand precision of the five Newton-Schulz steps:
  *             -1 = fp16 operands at the full tensor rate with fp32 iterates
  *             (the recommended setting); 0..5 = that many leading steps with
