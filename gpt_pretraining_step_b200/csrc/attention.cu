@@ -65,10 +65,10 @@ constexpr int HD = 128;
 // the polynomial on the FMA pipe): forward, alternating between two values
 // over consecutive groups; backward, one value.  Even numbers (pairs).
 #ifndef GPT_FWD_MUFU_EVEN
-#define GPT_FWD_MUFU_EVEN 6
+#define GPT_FWD_MUFU_EVEN 8
 #endif
 #ifndef GPT_FWD_MUFU_ODD
-#define GPT_FWD_MUFU_ODD 6
+#define GPT_FWD_MUFU_ODD 8
 #endif
 #ifndef GPT_BWD_MUFU
 #define GPT_BWD_MUFU 8
@@ -122,6 +122,7 @@ __device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int k
   return it;
 }
 
+template <bool kFine>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, bf16* __restrict__ o, float* __restrict__ lse,
@@ -189,7 +190,7 @@ __global__ void __launch_bounds__(384, 1)
       int g = 0, last_q = -1;   // ring position of the next K/V block; last item whose Q was loaded
       for (int n = 0;; ++n) {
         // the previous item's Q is no longer read and every warp has its number
-        if (n > 0 && !mbar_wait(q_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+        if (n > 0 && !mbar_wait_t<kFine>(q_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
         int idx = sched ? atomicAdd(sched, 1) : n * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
         if (idx >= n_items) idx = -1;
         item_ring[n & 3] = idx;
@@ -210,11 +211,11 @@ __global__ void __launch_bounds__(384, 1)
           const int s = g & 1;
           const uint32_t par = (g >> 1) & 1;
           const int kc = (it.j0 + j) * 128;
-          if (!mbar_wait(&k_empty[s], par ^ 1u, abort_flag, err, wlim)) { ok = false; break; }
+          if (!mbar_wait_t<kFine>(&k_empty[s], par ^ 1u, abort_flag, err, wlim)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[s], TF_BUF);
           tma_load_3d(sK + s * TF_BUF, &tk, &k_full[s], 0, kc, it.bkv);
           tma_load_3d(sK + s * TF_BUF + TF_TILE, &tk, &k_full[s], 64, kc, it.bkv);
-          if (!mbar_wait(&v_empty[s], par ^ 1u, abort_flag, err, wlim)) {
+          if (!mbar_wait_t<kFine>(&v_empty[s], par ^ 1u, abort_flag, err, wlim)) {
             // K of this block is in flight: count it, V is not
             for (uint32_t i = 0; i < (1u << 20) && !mbar_try_wait(&k_full[s], par); ++i) {}
             ok = false;
@@ -271,16 +272,16 @@ __global__ void __launch_bounds__(384, 1)
       int g0 = 0;                  // ring position of the item's first key block
       uint32_t npv[2] = {0u, 0u};  // P V products issued per tile so far
       for (int n = 0; ok; ++n) {
-        if (!mbar_wait(q_full, n & 1, abort_flag, err, wlim)) { ok = false; break; }
+        if (!mbar_wait_t<kFine>(q_full, n & 1, abort_flag, err, wlim)) { ok = false; break; }
         const int idx = item_ring[n & 3];
         if (idx < 0) break;
         const FwdItem it = fwd_item(idx, nq, H, Hkv, kvs, wl);
         // S of the first block on both tiles, each once its previous P V (which
         // reads P from the same columns) has completed
-        if (!mbar_wait(&k_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+        if (!mbar_wait_t<kFine>(&k_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
         for (int t = 0; t < 2 && ok; ++t) {
           if (t == 1 && !it.hasB) break;
-          if (npv[t] > 0 && !mbar_wait(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+          if (npv[t] > 0 && !mbar_wait_t<kFine>(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
           tc_fence_after();
           issue_s(t, g0 & 1);
         }
@@ -291,19 +292,19 @@ __global__ void __launch_bounds__(384, 1)
           const int gj = g0 + j;
           const int s = gj & 1;
           const int s1 = (gj + 1) & 1;
-          if (!mbar_wait(&v_full[s], (gj >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
-          if (j + 1 < it.nkv && !mbar_wait(&k_full[s1], ((gj + 1) >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+          if (!mbar_wait_t<kFine>(&v_full[s], (gj >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+          if (j + 1 < it.nkv && !mbar_wait_t<kFine>(&k_full[s1], ((gj + 1) >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
           // per tile: O += P V_j, then S of the next block over P once that product
           // has read it (tile B's softmax trails tile A's, so A goes first)
           for (int t = 0; t < 2; ++t) {
             const int nkv_t = t ? it.nkvB : it.nkvA;
             if (j >= nkv_t) continue;
-            if (!mbar_wait(&p_full[t], npv[t] & 1, abort_flag, err, wlim)) { ok = false; break; }
+            if (!mbar_wait_t<kFine>(&p_full[t], npv[t] & 1, abort_flag, err, wlim)) { ok = false; break; }
             tc_fence_after();
             issue_pv(t, s, j > 0);
             ++npv[t];
             if (j + 1 < nkv_t) {
-              if (!mbar_wait(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+              if (!mbar_wait_t<kFine>(&pv_done[t], (npv[t] - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
               tc_fence_after();
               issue_s(t, s1);
               if (j + 1 == it.nkv - 1) umma_commit(q_empty);   // the item's last S
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     uint32_t nblk = 0;   // S blocks consumed on this tile so far
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
-      const bool got = mbar_wait(bar, par, abort_flag, err, wlim);
+      const bool got = mbar_wait_t<kFine>(bar, par, abort_flag, err, wlim);
       __syncwarp();
       return __all_sync(0xffffffffu, got);
     };
@@ -374,14 +375,18 @@ __global__ void __launch_bounds__(384, 1)
             if (key > q || key >= T || key < q - wl) sr[k] = __float_as_uint(-INFINITY);
           }
         }
-        // block max of the raw scores (the scale is positive), eight independent chains
+        // block max of the raw scores (the scale is positive), eight independent
+        // chains of three-input maxima (two new scores per instruction)
         float mx8[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) mx8[t] = __uint_as_float(sr[t]);
+        for (int t = 0; t < 8; ++t) mx8[t] = fmaxf(__uint_as_float(sr[2 * t]), __uint_as_float(sr[2 * t + 1]));
 #pragma unroll
-        for (int k = 8; k < 128; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], __uint_as_float(sr[k]));
-        const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                 fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int k = 16; k < 128; k += 16) {
+#pragma unroll
+          for (int t = 0; t < 8; ++t)
+            mx8[t] = fmax3(mx8[t], __uint_as_float(sr[k + 2 * t]), __uint_as_float(sr[k + 2 * t + 1]));
+        }
+        const float mraw = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
         const float mblk = mraw * scale_log2;
         const bool move = mblk > m_ref + TF_RESCALE;   // true on the first block with a visible key
         const float m_new = move ? mblk : m_ref;
@@ -563,6 +568,7 @@ __device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int kvs, 
   return k;
 }
 
+template <bool kFine>
 __global__ void __launch_bounds__(448, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -649,12 +655,12 @@ __global__ void __launch_bounds__(448, 1)
       auto load_q_do = [&](const BwdBlock& kb, int it) -> bool {
         const int i = kb.q_block(it), h = kb.q_head(it), bh = kb.b * H + h;
         const int s = g & 1;
-        if (!mbar_wait(&q_empty[s], ((g >> 1) & 1) ^ 1u, abort_flag, err, wlim)) return false;
+        if (!mbar_wait_t<kFine>(&q_empty[s], ((g >> 1) & 1) ^ 1u, abort_flag, err, wlim)) return false;
         mbar_arrive_expect_tx(&q_full[s], TF_BUF);
         tma_load_3d(sQ + s * TF_BUF, &tq, &q_full[s], 0, i * 128, bh);
         tma_load_3d(sQ + s * TF_BUF + TF_TILE, &tq, &q_full[s], 64, i * 128, bh);
         ++issued_q;
-        if (!mbar_wait(do_empty, (g & 1) ^ 1u, abort_flag, err, wlim)) return false;
+        if (!mbar_wait_t<kFine>(do_empty, (g & 1) ^ 1u, abort_flag, err, wlim)) return false;
         mbar_arrive_expect_tx(do_full, TF_BUF);
         tma_load_4d(sdO, &tdo, do_full, 0, h, i * 128, kb.b);
         tma_load_4d(sdO + TF_TILE, &tdo, do_full, 64, h, i * 128, kb.b);
@@ -682,7 +688,7 @@ __global__ void __launch_bounds__(448, 1)
         item_ring[n & 3] = idx;
         if (idx < 0) {
           // end marker, once every warp has the previous item's number
-          if (n > 0 && !mbar_wait(kv_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+          if (n > 0 && !mbar_wait_t<kFine>(kv_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
           mbar_arrive(kv_full);
           break;
         }
@@ -691,7 +697,7 @@ __global__ void __launch_bounds__(448, 1)
         // finishes; K and V (which publish the item number) once its last
         // products are done
         if (!load_q_do(kb, 0)) { ok = false; break; }
-        if (n > 0 && !mbar_wait(kv_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+        if (n > 0 && !mbar_wait_t<kFine>(kv_empty, (n - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
         mbar_arrive_expect_tx(kv_full, 2 * TF_BUF);
         tma_load_3d(sK, &tk, kv_full, 0, kb.k0, kb.kvrow);
         tma_load_3d(sK + TF_TILE, &tk, kv_full, 64, kb.k0, kb.kvrow);
@@ -733,7 +739,7 @@ __global__ void __launch_bounds__(448, 1)
       bool ok = true;
       int g0 = 0;   // query blocks done so far
       for (int n = 0; ok; ++n) {
-        if (!mbar_wait(kv_full, n & 1, abort_flag, err, wlim)) { ok = false; break; }
+        if (!mbar_wait_t<kFine>(kv_full, n & 1, abort_flag, err, wlim)) { ok = false; break; }
         const int idx = item_ring[n & 3];
         if (idx < 0) break;
         {
@@ -742,21 +748,21 @@ __global__ void __launch_bounds__(448, 1)
           // S^T of the first query block goes where the previous key block's
           // last dQ^T was (wait until the dQ warps have read it), dP^T where
           // its last P was (wait until that dV is done)
-          ok = mbar_wait(&q_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim) &&
-               (g0 == 0 || mbar_wait(dq_free, (g0 - 1) & 1, abort_flag, err, wlim));
+          ok = mbar_wait_t<kFine>(&q_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim) &&
+               (g0 == 0 || mbar_wait_t<kFine>(dq_free, (g0 - 1) & 1, abort_flag, err, wlim));
           if (!ok) break;
           tc_fence_after();
           qk_product(tmem, k_addr, smem_u32(sQ + (g0 & 1) * TF_BUF));   // S^T of the first block
           umma_commit(s_full);
-          ok = mbar_wait(do_full, g0 & 1, abort_flag, err, wlim) &&
-               (g0 == 0 || mbar_wait(do_empty, (g0 - 1) & 1, abort_flag, err, wlim));
+          ok = mbar_wait_t<kFine>(do_full, g0 & 1, abort_flag, err, wlim) &&
+               (g0 == 0 || mbar_wait_t<kFine>(do_empty, (g0 - 1) & 1, abort_flag, err, wlim));
           if (!ok) break;
           tc_fence_after();
           qk_product(tmem + 128, v_addr, do_addr);   // dP^T of the first block
           umma_commit(dp_full);
           if (n_it > 1) {
-            ok = mbar_wait(s_free, g0 & 1, abort_flag, err, wlim) &&
-                 mbar_wait(&q_full[(g0 + 1) & 1], ((g0 + 1) >> 1) & 1, abort_flag, err, wlim);
+            ok = mbar_wait_t<kFine>(s_free, g0 & 1, abort_flag, err, wlim) &&
+                 mbar_wait_t<kFine>(&q_full[(g0 + 1) & 1], ((g0 + 1) >> 1) & 1, abort_flag, err, wlim);
             if (!ok) break;
             tc_fence_after();
             qk_product(tmem, k_addr, smem_u32(sQ + ((g0 + 1) & 1) * TF_BUF));   // S^T of the second block
@@ -765,7 +771,7 @@ __global__ void __launch_bounds__(448, 1)
           for (int it = 0; it < n_it && ok; ++it) {
             const int gi = g0 + it;
             const int s = gi & 1;
-            if (!mbar_wait(p_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
+            if (!mbar_wait_t<kFine>(p_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
             tc_fence_after();
             const uint32_t q_addr = smem_u32(sQ + s * TF_BUF);
             // dV += P^T dO: A = P^T from TMEM, 16 queries = 8 packed columns per
@@ -781,7 +787,7 @@ __global__ void __launch_bounds__(448, 1)
             umma_commit(do_empty);
             // dK and dQ^T once dS_i is in shared memory (the softmax warps compute it
             // while dV runs)
-            if (!mbar_wait(ds_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
+            if (!mbar_wait_t<kFine>(ds_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
             tc_fence_after();
             {
               uint64_t dsa = smem_desc_sw128(dst_addr, 16, 1024), dqb = smem_desc_sw128(q_addr, TF_TILE, 1024);
@@ -798,9 +804,9 @@ __global__ void __launch_bounds__(448, 1)
             // warps have read it) or, for the last block, dQ^T_{i-1} (wait until
             // the dQ warps have read it)
             if (it + 1 < n_it) {
-              if (!mbar_wait(s_free, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+              if (!mbar_wait_t<kFine>(s_free, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
             } else if (it > 0) {
-              if (!mbar_wait(dq_free, (gi - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+              if (!mbar_wait_t<kFine>(dq_free, (gi - 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
             }
             tc_fence_after();
             {
@@ -816,15 +822,15 @@ __global__ void __launch_bounds__(448, 1)
             if (it + 1 == n_it) umma_commit(kv_empty);   // K and V of this key block are free
             if (it + 1 < n_it) {
               // dP^T_{i+1} overwrites P^T_i: dV_i must have completed
-              if (!mbar_wait(do_empty, gi & 1, abort_flag, err, wlim) ||
-                  !mbar_wait(do_full, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+              if (!mbar_wait_t<kFine>(do_empty, gi & 1, abort_flag, err, wlim) ||
+                  !mbar_wait_t<kFine>(do_full, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
               tc_fence_after();
               qk_product(tmem + 128, v_addr, do_addr);
               umma_commit(dp_full);
             }
             if (it + 2 < n_it) {
-              if (!mbar_wait(dq_free, gi & 1, abort_flag, err, wlim) ||
-                  !mbar_wait(&q_full[s], ((gi + 2) >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
+              if (!mbar_wait_t<kFine>(dq_free, gi & 1, abort_flag, err, wlim) ||
+                  !mbar_wait_t<kFine>(&q_full[s], ((gi + 2) >> 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
               tc_fence_after();
               qk_product(tmem, k_addr, q_addr);   // S^T_{i+2} (same Q slot as block i)
               umma_commit(s_full);
@@ -862,7 +868,7 @@ __global__ void __launch_bounds__(448, 1)
     int g = 0;
     for (int n = 0; ok; ++n) {
       {
-        const bool got = mbar_wait(kv_full, n & 1, abort_flag, err, wlim);
+        const bool got = mbar_wait_t<kFine>(kv_full, n & 1, abort_flag, err, wlim);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
       }
@@ -874,7 +880,7 @@ __global__ void __launch_bounds__(448, 1)
         const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         for (int it = 0; it < kb.n_it && ok; ++it, ++g) {
           const int q0 = kb.q_block(it) * 128, bh = kb.b * H + kb.q_head(it);
-          const bool got = mbar_wait(mm_done, g & 1, abort_flag, err, wlim);
+          const bool got = mbar_wait_t<kFine>(mm_done, g & 1, abort_flag, err, wlim);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
           tc_fence_after();
@@ -930,7 +936,7 @@ __global__ void __launch_bounds__(448, 1)
     int g0 = 0;
     for (int n = 0; ok; ++n) {
       {
-        const bool got = mbar_wait(kv_full, n & 1, abort_flag, err, wlim);
+        const bool got = mbar_wait_t<kFine>(kv_full, n & 1, abort_flag, err, wlim);
         if (any_fail(got)) { ok = false; break; }
       }
       const int idx = item_ring[n & 3];
@@ -1017,7 +1023,7 @@ __global__ void __launch_bounds__(448, 1)
           const int gi = g0 + it;
           if (it >= 0) {
             // dS'_i = P_i (dP_i - D) once dP^T_i is in TMEM
-            const bool got = mbar_wait(dp_full, gi & 1, abort_flag, err, wlim);
+            const bool got = mbar_wait_t<kFine>(dp_full, gi & 1, abort_flag, err, wlim);
             if (any_fail(got)) { ok = false; break; }
             // every thread is past block i-1's use of buffer (i+1) & 1
             if (it + 1 < n_it) publish(it + 1, staged);
@@ -1061,7 +1067,7 @@ __global__ void __launch_bounds__(448, 1)
           }
           // P_{i+1} while the tensor cores run this block's dV, dK, dQ^T
           if (it + 1 < n_it) {
-            const bool got1 = mbar_wait(s_full, (gi + 1) & 1, abort_flag, err, wlim);
+            const bool got1 = mbar_wait_t<kFine>(s_full, (gi + 1) & 1, abort_flag, err, wlim);
             if (any_fail(got1)) { ok = false; break; }   // also publishes lse/D of block i+1
             tc_fence_after();
             compute_p(it + 1);
@@ -1069,7 +1075,7 @@ __global__ void __launch_bounds__(448, 1)
         }
         // dK and dV of this key block, complete with the last block's products
         if (ok) {
-          const bool got = mbar_wait(mm_done, (g0 + n_it - 1) & 1, abort_flag, err, wlim);
+          const bool got = mbar_wait_t<kFine>(mm_done, (g0 + n_it - 1) & 1, abort_flag, err, wlim);
           ok = !any_fail(got);
         }
         if (ok) {
@@ -1161,8 +1167,11 @@ static int* sched_word(int* sched, cudaStream_t s) {
 void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float* lse, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride,
                      long long wait_cycles) {
-  static std::atomic<unsigned long long> configured{0};
-  if (set_smem_limit_once(attn_fwd_tc_kernel, TF_SMEM, configured) != cudaSuccess) {
+  // a limit shorter than one blocking probe needs the finely polling build
+  const bool fine = wait_limit_or_default(wait_cycles) < kShortWaitCycles;
+  auto kern = fine ? attn_fwd_tc_kernel<true> : attn_fwd_tc_kernel<false>;
+  static std::atomic<unsigned long long> configured[2] = {};
+  if (set_smem_limit_once(kern, TF_SMEM, configured[fine ? 1 : 0]) != cudaSuccess) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
     return;
   }
@@ -1180,7 +1189,7 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
   const long long n_items = ((T + 127) / 128 + 1) / 2 * bh;
   const int grid = static_cast<int>(std::min<long long>(n_items, device_sm_count()));
   const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
-  attn_fwd_tc_kernel<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, kv_stride, T, window_bound(window, T),
+  kern<<<grid, 384, TF_SMEM, s>>>(mq, mk, mv, o, lse, H, Hkv, kv_stride, T, window_bound(window, T),
                                                 scale_log2,
                                                 static_cast<int>(n_items), sched_word(sched, s), err, wait_cycles);
 }
@@ -1189,8 +1198,10 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride,
                      long long wait_cycles) {
-  static std::atomic<unsigned long long> configured{0};
-  if (set_smem_limit_once(attn_bwd_tc_kernel, TB_SMEM, configured) != cudaSuccess) {
+  const bool fine = wait_limit_or_default(wait_cycles) < kShortWaitCycles;
+  auto kern = fine ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
+  static std::atomic<unsigned long long> configured[2] = {};
+  if (set_smem_limit_once(kern, TB_SMEM, configured[fine ? 1 : 0]) != cudaSuccess) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);   // latched as a device error
     return;
   }
@@ -1220,7 +1231,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const int grid = static_cast<int>(std::min<long long>(n_units, device_sm_count()));
   const int wl = window_bound(window, T);
   int* word = wl >= T ? nullptr : sched_word(sched, s);
-  attn_bwd_tc_kernel<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
+  kern<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
                                                 1.f / sqrtf(static_cast<float>(HD)), static_cast<int>(n_units),
                                                 word, err, wait_cycles);
 }

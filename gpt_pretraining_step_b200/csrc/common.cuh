@@ -95,11 +95,45 @@ constexpr long long kShortWaitCycles = 1000000ll;
 
 // Wait for the phase with the given parity to complete.  Returns false if
 // another thread raised *abort or the wait ran past `limit` SM cycles; in the
-// latter case this thread raises *abort itself and sets the error flag.  One
-// polling loop serves both kinds of limit (the kernels have dozens of wait
-// sites, so each must stay small): a short limit polls with the non-blocking
-// test and reads the clock on every probe, a long one with try_wait and
-// reads the clock every 64 probes.
+// latter case this thread raises *abort itself and sets the error flag.
+// kFine = false (the kernels' normal build): blocking try_wait probes, the
+// clock read every 64 probes.  kFine = true (a second build of a kernel,
+// launched only for a limit under kShortWaitCycles): non-blocking probes and
+// a clock read on each, so that the limit holds even when it is shorter than
+// one blocking probe.  Keeping the two apart keeps each wait site small in
+// the normal build (a kernel has dozens of them).
+template <bool kFine>
+__device__ __forceinline__ bool mbar_wait_t(uint64_t* bar, uint32_t parity, volatile int* abort, int* err,
+                                            long long limit) {
+  if constexpr (kFine) {
+    const long long t0 = clock64();
+    for (;;) {
+      if (mbar_test_wait(bar, parity)) return true;
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        *abort = 1;
+        if (err) atomicOr(err, ERRF_TIMEOUT);
+        return false;
+      }
+    }
+  } else {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+      if ((i & 63u) == 0) {
+        if (*abort) return false;
+        if (clock64() - t0 > limit) {
+          *abort = 1;
+          if (err) atomicOr(err, ERRF_TIMEOUT);
+          return false;
+        }
+      }
+    }
+  }
+}
+
+// The same with the kind of polling chosen at run time (one loop for both).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           int* err, long long limit) {
   const bool fine = limit < kShortWaitCycles;
@@ -348,6 +382,13 @@ __device__ __forceinline__ uint64_t f2_exp2_poly(uint64_t x) {
   f2_unpack(p, p0, p1);
   return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
                  __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
+
+// max(a, b, c) in one instruction (three-input max of sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
