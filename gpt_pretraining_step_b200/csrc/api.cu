@@ -947,7 +947,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         g.batch = nz; g.es = 2; g.f16 = true;
         g.A = curH; g.lda = cc; g.a_bs = 1ll * r * cc;
         g.B = curH; g.ldb = cc; g.b_bs = 1ll * r * cc;
-        g.bn = 128; g.sym = true; g.epi = EPI_STORE;
+        g.bn = 256; g.sym = true; g.epi = EPI_STORE;
         g.out_es = 2; g.out_f16 = true; g.aux_es = 2; g.aux_f16 = true;
         g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
         GPT_CK(run_gemm(g, s, wait_cycles));
@@ -957,7 +957,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         g.batch = nz; g.es = 2; g.f16 = true;
         g.A = Ab; g.lda = r; g.a_bs = 1ll * r * r;
         g.B = Ab; g.ldb = r; g.b_bs = 1ll * r * r;
-        g.bn = 128; g.sym = true; g.epi = EPI_AXPBY;
+        g.bn = 256; g.sym = true; g.epi = EPI_AXPBY;
         g.out_es = 2; g.out_f16 = true; g.aux_es = 2; g.aux_f16 = true;
         g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
         g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
@@ -999,7 +999,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
       g.batch = nz; g.es = es;
       g.A = cur; g.lda = cc; g.a_bs = 1ll * r * cc;
       g.B = cur; g.ldb = cc; g.b_bs = 1ll * r * cc;
-      g.bn = 128; g.sym = true; g.epi = EPI_STORE; g.out_es = es; g.aux_es = es;
+      g.bn = es == 4 ? 128 : 256; g.sym = true; g.epi = EPI_STORE; g.out_es = es; g.aux_es = es;
       g.p.out = Ab; g.p.ldo = r; g.p.out_bs = 1ll * r * r; g.p.err = err;
       GPT_CK(run_gemm(g, s, wait_cycles));
     }
@@ -1008,7 +1008,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
       g.batch = nz; g.es = es;
       g.A = Ab; g.lda = r; g.a_bs = 1ll * r * r;
       g.B = Ab; g.ldb = r; g.b_bs = 1ll * r * r;
-      g.bn = 128; g.sym = true; g.epi = EPI_AXPBY; g.out_es = es; g.aux_es = es;
+      g.bn = es == 4 ? 128 : 256; g.sym = true; g.epi = EPI_AXPBY; g.out_es = es; g.aux_es = es;
       g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
       g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
       g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;

@@ -73,11 +73,6 @@ constexpr int HD = 128;
 #ifndef GPT_BWD_MUFU
 #define GPT_BWD_MUFU 8
 #endif
-// Backward: issue dP^T of the next query block before dQ^T of this one when
-// its dO tile has already landed (1), or always after it (0).
-#ifndef GPT_BWD_DP_EARLY
-#define GPT_BWD_DP_EARLY 0
-#endif
 
 constexpr int TF_TILE = 16384;                // one [128 rows][128 B] swizzled tile
 constexpr int TF_BUF = 2 * TF_TILE;           // 128 x 128 bf16 as two 64-column tiles
@@ -805,21 +800,6 @@ __global__ void __launch_bounds__(448, 1)
               }
             }
             umma_commit(&q_empty[s]);
-            // dP^T_{i+1} ahead of dQ^T_i when dO_{i+1} has landed already: the
-            // softmax warps then get it one product earlier (it overwrites P^T_i,
-            // so dV_i must have completed)
-            bool dp_issued = false;
-#if GPT_BWD_DP_EARLY
-            if (it + 1 < n_it) {
-              if (!mbar_wait_t<kFine>(do_empty, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
-              if (mbar_try_wait(do_full, (gi + 1) & 1)) {
-                tc_fence_after();
-                qk_product(tmem + 128, v_addr, do_addr);
-                umma_commit(dp_full);
-                dp_issued = true;
-              }
-            }
-#endif
             // dQ^T_i goes to [0,128), which holds S^T_{i+1} (wait until the softmax
             // warps have read it) or, for the last block, dQ^T_{i-1} (wait until
             // the dQ warps have read it)
@@ -840,7 +820,7 @@ __global__ void __launch_bounds__(448, 1)
             }
             umma_commit(mm_done);
             if (it + 1 == n_it) umma_commit(kv_empty);   // K and V of this key block are free
-            if (it + 1 < n_it && !dp_issued) {
+            if (it + 1 < n_it) {
               // dP^T_{i+1} overwrites P^T_i: dV_i must have completed
               if (!mbar_wait_t<kFine>(do_empty, gi & 1, abort_flag, err, wlim) ||
                   !mbar_wait_t<kFine>(do_full, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }

@@ -116,7 +116,7 @@ int gemm_tiles(const GemmCall& c) {
 cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   if (c.M <= 0 || c.N <= 0 || c.batch <= 0) return cudaSuccess;
   if (c.K <= 0 || (c.bn != 128 && c.bn != 256) || (c.es != 1 && c.es != 2 && c.es != 4)) return cudaErrorInvalidValue;
-  if (c.sym && (c.M != c.N || c.bn != 128)) return cudaErrorInvalidValue;
+  if (c.sym && c.M != c.N) return cudaErrorInvalidValue;
   if (c.N % 8) return cudaErrorInvalidValue;
   // 32-bit operands are staged K-major only (the 128-byte swizzle atom used here
   // describes MN-major layouts of 16-bit types)
@@ -132,7 +132,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
   p.sym = c.sym ? 1 : 0;
-  const long long ntiles = c.sym ? 1ll * p.tiles_m * (p.tiles_m + 1) / 2 : 1ll * p.tiles_m * p.tiles_n;
+  const long long ntiles = c.sym ? sym_tile_count(p.tiles_m, p.tiles_n, c.bn / 128) : 1ll * p.tiles_m * p.tiles_n;
   const long long units = ntiles * p.splits * c.batch;
   if (units > 0x7fffffffll) return cudaErrorInvalidValue;
   p.units = static_cast<int>(units);
@@ -221,6 +221,9 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   // Newton-Schulz, fp16 steps (fp32 iterates with an fp16 operand copy)
   GPT_GEMM_CASE(f16, 128, false, false, EPI_STORE, f16, f16)
   GPT_GEMM_CASE(f16, 128, false, false, EPI_AXPBY, f16, f16)
+  GPT_GEMM_CASE(f16, 256, false, false, EPI_STORE, f16, f16)
+  GPT_GEMM_CASE(f16, 256, false, false, EPI_AXPBY, f16, f16)
+  GPT_GEMM_CASE(bf16, 256, false, false, EPI_AXPBY, bf16, bf16)
   GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, float, float)
   // fp8 e4m3 forward projections (operands as raw bytes)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_QKV, bf16, bf16)

@@ -58,9 +58,19 @@ struct GemmCfg {
   static constexpr int SMEM = STAGES * STAGE_BYTES + STG_BYTES + 1024 + 256;
 };
 
+// Tiles of a symmetric product (M == N) on or above the diagonal: row block m
+// (128 rows) needs the column blocks (BN wide) from m / (BN / 128) on.
+__host__ __device__ __forceinline__ int sym_tile_count(int tiles_m, int tiles_n, int rows_per_col_block) {
+  int n = 0;
+  for (int m = 0; m < tiles_m; ++m) n += tiles_n - m / rows_per_col_block;
+  return n;
+}
+
+template <int BN>
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
                                             int& kb0, int& kb1, int& split) {
-  const int ntiles = p.sym ? p.tiles_m * (p.tiles_m + 1) / 2 : p.tiles_m * p.tiles_n;
+  constexpr int R = BN / 128;
+  const int ntiles = p.sym ? sym_tile_count(p.tiles_m, p.tiles_n, R) : p.tiles_m * p.tiles_n;
   const int per_z = ntiles * p.splits;
   z = u / per_z;
   int r = u - z * per_z;
@@ -68,12 +78,12 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, 
   int t = r - split * ntiles;
   if (p.sym) {
     int m = 0;
-    while (t >= p.tiles_m - m) {
-      t -= p.tiles_m - m;
+    while (t >= p.tiles_n - m / R) {
+      t -= p.tiles_n - m / R;
       ++m;
     }
     mb = m;
-    nb = m + t;
+    nb = m / R + t;
   } else {
     constexpr int G = 16;
     const int gsz = G * p.tiles_n;
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
         int z, mb, nb, kb0, kb1, split;
-        decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+        decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
@@ -280,7 +290,7 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++local) {
         int z, mb, nb, kb0, kb1, split;
-        decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+        decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
         const int acc = local & 1;
         const uint32_t acc_par = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
@@ -382,7 +392,7 @@ __global__ void __launch_bounds__(320, 1)
     int local = 0;
     for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
       int z, mb, nb, kb0, kb1, split;
-      decode_unit(p, u, z, mb, nb, kb0, kb1, split);
+      decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if constexpr (EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
@@ -541,7 +551,15 @@ __global__ void __launch_bounds__(320, 1)
       } else {
         OutT* obase = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(z) * p.out_bs +
                       static_cast<long long>(split) * p.split_stride;
-        const bool mirror = p.sym && nb != mb;
+        // Symmetric products: with square tiles (BN 128) the diagonal tiles are
+        // written whole and the others mirrored whole; with 128 x 256 tiles an
+        // element is written directly on or above the diagonal and mirrored
+        // from above it, so each is written exactly once, and a tile that
+        // holds elements below the diagonal stores per thread with that mask.
+        constexpr bool kRect = BN == 256;
+        const bool sym_cross = kRect && p.sym && nb * BN < mb * 128 + 128;
+        const bool mirror = p.sym && (kRect || nb != mb);
+        const bool tma_here = p.tma_out && !sym_cross;
         // Auxiliary input of the epilogue, prefetched one 32-column chunk ahead to
         // hide its load latency.  (EPI_ACC adds into the output by TMA
         // add-reduction and reads nothing.)
@@ -624,7 +642,7 @@ __global__ void __launch_bounds__(320, 1)
               for (int j = 0; j < 32; ++j) v[hh][j] = p.alpha * a[j] + p.beta * v[hh][j];
             }
           }
-          if (p.tma_out) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          if (tma_here) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
           // optional fp16 copy of the output in the same layout
           if (p.tma_out2) emit64_to(__half{}, &tmD, false, v[0], v[1], nb * BN + c * 32, box_row0, z3);
 #pragma unroll
@@ -632,7 +650,19 @@ __global__ void __launch_bounds__(320, 1)
             const int col0 = nb * BN + (c + hh) * 32;
             const int nvalid = min(32, p.N - col0);
             if (!row_ok || nvalid <= 0) continue;
-            if (!p.tma_out) store_row32(obase + static_cast<long long>(row) * p.ldo + col0, v[hh], nvalid);
+            if (sym_cross) {
+              // the columns on or above the diagonal of this row
+              OutT* drow = obase + static_cast<long long>(row) * p.ldo;
+              if (col0 >= row) {
+                store_row32(drow + col0, v[hh], nvalid);
+              } else if (col0 + nvalid > row) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if (j < nvalid && col0 + j >= row) store_scalar(drow + col0 + j, v[hh][j]);
+              }
+            } else if (!tma_here) {
+              store_row32(obase + static_cast<long long>(row) * p.ldo + col0, v[hh], nvalid);
+            }
             if (p.out_t) {
               OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
 #pragma unroll
@@ -643,7 +673,8 @@ __global__ void __launch_bounds__(320, 1)
               // the transposed tile of a symmetric product: lanes write consecutive columns
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
+                if (j < nvalid && (!kRect || col0 + j > row))
+                  store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
             }
           }
         }
