@@ -931,19 +931,25 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
   ProfScope ps(pc, GPT_PROF_NS_GEMM);
   const double (*kPolarCoef)[3] = polar_coefficients();
   if (n_tf32 < 0) {
-    // fp16 operands at the full tensor rate with fp32 iterates: X (fp32) in
-    // X0/X1 and its fp16 copy, written by the same epilogue, in XT0/XT1; the
-    // Gram A and B = b A + c A^2 in fp16.  The normalised X keeps every
+    // fp16 operands at the full tensor rate.  The iterate is carried as an
+    // unevaluated pair X = hi + lo of fp16 matrices (hi = fp16(X), lo = the
+    // rounding residual), ~22 significant bits, so that the update's epilogue
+    // reads and writes 6 bytes per element instead of an fp32 X plus its fp16
+    // copy (10).  The step X' = a X + B X becomes X' = (a I + B) hi + a lo: the
+    // tensor cores multiply by hi only, as they did with the fp16 copy, and the
+    // diagonal a I is folded into B by the polynomial's epilogue.  The first
+    // step reads the fp32 X0 (with its fp16 copy hi in XT0) and the last writes
+    // fp32.  The two lo buffers share X1's bytes.  The normalised X keeps every
     // operand far inside fp16's range.
-    void* cur = X0;
-    void* nxt = X1;
-    void* curH = XT0;
-    void* nxtH = XT1;
+    const size_t nx = static_cast<size_t>(nz) * r * cc;
+    void* hi[2] = {XT0, XT1};
+    void* lo[2] = {X1, static_cast<uint8_t*>(X1) + nx * 2};
     for (int t = 0; t < kPolarSteps; ++t) {
-      const bool last = t + 1 == kPolarSteps;
+      const bool first = t == 0, last = t + 1 == kPolarSteps;
       const double a = kPolarCoef[t][0], b = kPolarCoef[t][1], cf = kPolarCoef[t][2];
+      void* curH = hi[t & 1];
       {
-        GemmCall g = base_call(r, r, cc);   // A = X X^T
+        GemmCall g = base_call(r, r, cc);   // A = hi hi^T
         g.batch = nz; g.es = 2; g.f16 = true;
         g.A = curH; g.lda = cc; g.a_bs = 1ll * r * cc;
         g.B = curH; g.ldb = cc; g.b_bs = 1ll * r * cc;
@@ -953,7 +959,7 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         GPT_CK(run_gemm(g, s, wait_cycles));
       }
       {
-        GemmCall g = base_call(r, r, r);    // B = b A + c A A
+        GemmCall g = base_call(r, r, r);    // B = b A + c A A (+ a I after the first step)
         g.batch = nz; g.es = 2; g.f16 = true;
         g.A = Ab; g.lda = r; g.a_bs = 1ll * r * r;
         g.B = Ab; g.ldb = r; g.b_bs = 1ll * r * r;
@@ -962,25 +968,34 @@ int newton_schulz(gpt_ctx* pc, int nz, int r, int cc, void* X0, void* X1, void* 
         g.p.out = Bb; g.p.ldo = r; g.p.out_bs = 1ll * r * r;
         g.p.aux = Ab; g.p.ld_aux = r; g.p.aux_bs = 1ll * r * r;
         g.p.alpha = static_cast<float>(b); g.p.beta = static_cast<float>(cf); g.p.err = err;
+        g.p.gamma = first ? 0.f : static_cast<float>(a);
         GPT_CK(run_gemm(g, s, wait_cycles));
       }
       {
-        GemmCall g = base_call(r, cc, r);   // X' = a X + B X
+        GemmCall g = base_call(r, cc, r);   // X' = B hi + a X  (first step),  (a I + B) hi + a lo  (later)
         g.batch = nz; g.es = 2; g.f16 = true;
         g.A = Bb; g.lda = r; g.a_bs = 1ll * r * r;
         g.B = curH; g.b_mn = true; g.ldb = cc; g.b_bs = 1ll * r * cc;
-        g.bn = 256; g.epi = EPI_AXPBY; g.out_es = 4; g.aux_es = 4;
-        g.p.out = nxt; g.p.ldo = cc; g.p.out_bs = 1ll * r * cc;
-        if (!last) g.p.out2 = nxtH;
-        g.p.aux = cur; g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
+        g.bn = 256; g.epi = EPI_AXPBY;
+        if (first) {
+          g.aux_es = 4; g.p.aux = X0;
+        } else {
+          g.aux_es = 2; g.aux_f16 = true; g.p.aux = lo[(t + 1) & 1];
+        }
+        g.p.ld_aux = cc; g.p.aux_bs = 1ll * r * cc;
+        if (last) {
+          g.out_es = 4; g.p.out = X0;
+        } else {
+          g.out_es = 2; g.out_f16 = true; g.p.out = hi[(t + 1) & 1];
+          g.p.out2 = lo[t & 1]; g.p.split_lo = 1;
+        }
+        g.p.ldo = cc; g.p.out_bs = 1ll * r * cc;
         g.p.alpha = static_cast<float>(a); g.p.beta = 1.f; g.p.err = err;
         GPT_CK(run_gemm(g, s, wait_cycles));
       }
       *launches += 3;
-      std::swap(cur, nxt);
-      std::swap(curH, nxtH);
     }
-    *out = cur;
+    *out = X0;
     *out_es = 4;
     return GPT_OK;
   }

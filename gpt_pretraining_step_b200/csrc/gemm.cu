@@ -176,6 +176,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   // optional fp16 copy of the output (plain batched layouts only)
   CUtensorMap md;
   p.tma_out2 = 0;
+  if (p.split_lo && (!p.out2 || p.out_t || c.out_es != 2 || !c.out_f16 || c.sym)) return cudaErrorInvalidValue;
   if (p.out2) {
     if (c.epi == EPI_QKV || c.epi == EPI_LOGITS || p.splits > 1 || !p.tma_out) return cudaErrorInvalidValue;
     if (!make_map(&md, p.out2, 2, c.N, c.M, c.batch, p.ldo, p.out_bs, 64, 32, true)) return cudaErrorInvalidValue;
@@ -218,13 +219,15 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(float, 128, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, float, float)
   GPT_GEMM_CASE(float, 256, false, false, EPI_AXPBY, bf16, float)
-  // Newton-Schulz, fp16 steps (fp32 iterates with an fp16 operand copy)
+  // Newton-Schulz, fp16 steps (iterates as fp16 hi / lo pairs)
   GPT_GEMM_CASE(f16, 128, false, false, EPI_STORE, f16, f16)
   GPT_GEMM_CASE(f16, 128, false, false, EPI_AXPBY, f16, f16)
   GPT_GEMM_CASE(f16, 256, false, false, EPI_STORE, f16, f16)
   GPT_GEMM_CASE(f16, 256, false, false, EPI_AXPBY, f16, f16)
   GPT_GEMM_CASE(bf16, 256, false, false, EPI_AXPBY, bf16, bf16)
-  GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, float, float)
+  GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, f16, float)   // first step: fp32 X in, hi / lo out
+  GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, f16, f16)     // middle steps: lo in, hi / lo out
+  GPT_GEMM_CASE(f16, 256, false, true, EPI_AXPBY, float, f16)   // last step: lo in, fp32 X out
   // fp8 e4m3 forward projections (operands as raw bytes)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_QKV, bf16, bf16)
   GPT_GEMM_CASE(uint8_t, 256, false, true, EPI_ACC, float, float)

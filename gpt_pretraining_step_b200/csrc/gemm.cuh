@@ -640,11 +640,28 @@ __global__ void __launch_bounds__(320, 1)
             } else if constexpr (EPI == EPI_AXPBY) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[hh][j] = p.alpha * a[j] + p.beta * v[hh][j];
+              if (p.gamma != 0.f) {
+                const int dj = row - (nb * BN + cc * 32);   // this row's diagonal column in the chunk
+                if (dj >= 0 && dj < 32) {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j)
+                    if (j == dj) v[hh][j] += p.gamma;
+                }
+              }
             }
           }
           if (tma_here) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
-          // optional fp16 copy of the output in the same layout
-          if (p.tma_out2) emit64_to(__half{}, &tmD, false, v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          // optional fp16 copy of the output in the same layout, or the rounding
+          // residual of an fp16 main output (then the TMA path alone stores v)
+          if (p.tma_out2) {
+            if (p.split_lo) {
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[hh][j] -= __half2float(__float2half_rn(v[hh][j]));
+            }
+            emit64_to(__half{}, &tmD, false, v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          }
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
             const int col0 = nb * BN + (c + hh) * 32;

@@ -23,6 +23,9 @@ struct GemmParams {
   const void* aux;
   long long ld_aux, aux_bs;
   float alpha, beta;
+  float gamma;          // AXPBY: added to the diagonal elements (row == column) of every output matrix
+  int split_lo;         // 1: the second (fp16) output holds out - fp16(out), the rounding residual of
+                        //   the fp16 main output, so that the pair carries ~22 significant bits
   float* f32a;          // QKV: rstd of q [M, H];   LOGITS: (max, sumexp) pairs [M, tiles_n]
   float* f32b;          // QKV: rstd of k [M, H];   LOGITS: target logit [M]
   const int* tgt;       // LOGITS: targets of the rows

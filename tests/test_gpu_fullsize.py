@@ -183,3 +183,45 @@ def test_d26_width_fp8_step_matches_oracle(torch):
     assert abs(loss - loss_ref) / loss_ref <= FP8_LOSS_RTOL, (loss, loss_ref)
     _check_grads(g, st, s, grads, FP8_GRAD_COS)
     _check_optimizer(g, st, s, params)
+
+
+def test_headline_width_every_option_matches_oracle(torch):
+    """Every option of the step at the headline widths (d_model 1280, V
+    32768, T 2048): grouped kv heads (10 query heads on 2 kv heads), an
+    "SSL" window pattern with 1024-token windows, the residual extras and
+    value embeddings with 32 gate channels; then a NorMuon step and AdamW on
+    the GPU's gradients."""
+    import gpt_pretraining_step_b200 as g
+    s = syn.make_shape(depth=3, d_model=1280, vocab=32768, batch=1, seq_len=2048, n_kv_head=2)
+    params = syn.init_params(s, seed=71, extras=True, ve_channels=32)
+    params["ve_gate"] = syn.gaussian(params["ve_gate"].shape, seed=72, std=2.0)
+    params["scalars"] = syn.random_scalars(s, seed=73)
+    tok, tgt = syn.tokens(s, seed=74), syn.targets(s, seed=75)
+    st = g.GPTStep(depth=s.depth, batch=s.batch, seq_len=s.seq_len, vocab=s.vocab, d_model=s.d_model,
+                   residual_extras=True, ve_gate_channels=32, n_kv_head=2, window_pattern="SSL", short_window=1024)
+    specs = syn.param_specs(s, extras=True, ve_channels=32)
+    for tid, (pname, *_r) in enumerate(specs):
+        st.set(tid, params[pname])
+    loss = float(st.fwd_bwd(torch.tensor(tok).cuda(), torch.tensor(tgt).cuda()).item())
+    st.check()
+    windows = om.layer_windows("SSL", 1024, s.depth)
+    loss_ref, grads, _ = om.fwd_bwd(params, tok, tgt, s.depth, windows=windows)
+    assert abs(loss - loss_ref) / loss_ref <= LOSS_RTOL, (loss, loss_ref)
+    G = {}
+    for tid, (pname, *_r) in enumerate(specs):
+        G[pname] = f64(st.get(tid, g.KIND_GRAD))
+        c = cosine(G[pname], grads[pname])
+        assert c >= GRAD_COS, (pname, c)
+    st.muon_step_normuon(0.02, 0.95, 0.01, 0.9)
+    st.adamw_step(*HP_ADAM)
+    st.check()
+    for tid, (pname, r, c, grp) in enumerate(specs):
+        W0 = params[pname].astype(np.float64)
+        got = f64(st.get(tid, g.KIND_PARAM))
+        if grp == "muon":
+            W_ref, _, _ = oo.muon_step(W0, G[pname], np.zeros((r, c)), 0.02, 0.95, 0.01,
+                                       normuon_V=np.zeros(min(r, c)), normuon_beta2=0.9)
+            assert relfro(got - W0, W_ref - W0) <= MUON_RELFRO, pname
+        else:
+            W_ref, _, _ = oo.adamw_step(W0, G[pname], np.zeros((r, c)), np.zeros((r, c)), 1, *HP_ADAM)
+            assert np.abs(got - W_ref).max() < 1e-6, pname
