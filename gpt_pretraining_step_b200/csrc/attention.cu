@@ -502,21 +502,25 @@ __global__ void __launch_bounds__(384, 1)
 // dK and dV add up over the whole loop.  The barrier phases run on across
 // key blocks, so the next block's Q and dO loads start while the previous
 // block's last products run, and its K and V load as soon as those are done.
-// 448 threads:
+// 512 threads in four warp groups (the first and the last give registers to
+// the softmax groups: 72 / 168 / 168 / 96 per thread):
 //   warp 0      TMA: Q_i through a two-slot ring; dO_i; K_j and V_j once per
 //               key block (after the previous block's last product).
 //   warp 1      TMEM owner and MMA issuer.  TMEM columns: [0,128) S^T_i and
-//               dQ^T_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16
+//               dQ_i in turn; [128,256) dP^T_i, then P^T_i as packed bf16
 //               (queries 0..63 at 128.., 64..127 at 192..); [256,384) dV;
 //               [384,512) dK.  Per query block i:
 //                 dV += P^T dO   once P_i is in TMEM (A from TMEM; then
 //                                dO_{i+1} may load)
 //                 dK += dS^T Q   once dS_i is in shared memory (then Q_{i+2}
 //                                may load)
-//                 dQ^T = K^T dS^T into [0,128) once S^T_{i+1} has been read
+//                 dQ = dS K into [0,128) once S^T_{i+1} has been read (A is
+//                                dS^T in shared memory read MN-major, so
+//                                the queries land in the TMEM lanes)
 //                 dP^T_{i+1} = V dO_{i+1}^T into [128,256)
-//                 S^T_{i+2} = K Q_{i+2}^T into [0,128) once dQ^T_i has been read
-//   warps 2..9  softmax, two warps per TMEM lane quarter, each on 64 of the
+//                 S^T_{i+2} = K Q_{i+2}^T into [0,128) once dQ_i has been read
+//   warps 2, 3  idle
+//   warps 4..11 softmax, two warps per TMEM lane quarter, each on 64 of the
 //               128 query columns of its key rows: when dP^T_i lands, P_i
 //               (computed during the previous block) over the dP^T columns the
 //               warp has read, then dS'_i = P_i (dP_i - D) to shared memory
@@ -524,11 +528,14 @@ __global__ void __launch_bounds__(384, 1)
 //               and P_{i+1} while the tensor cores run block i's products.
 //               1/sqrt(d) of dS = dS' / sqrt(d) is applied to dK and dQ.
 //               After a key block's last products they write its dK and dV.
-//   warps 10..13 dQ: one warp per TMEM lane quarter (lane = head dim) stages
-//               dQ^T_i as fp32 [query][dim] boxes in a 32 KB buffer, half of
-//               the queries at a time, and adds them into the fp32 dq buffer
-//               by TMA reduce-add, so the reduction runs beside the other
-//               warps' work.
+//   warps 12..15 dQ: one warp per TMEM lane quarter (lane = query), each
+//               thread staging its query's row of dQ_i, 64 dims at a time, as
+//               fp32 [32 queries][32 dims] boxes (eight 16-byte stores per
+//               row) in a 32 KB buffer, and adding them into the fp32 dq
+//               buffer by TMA reduce-add, so the reduction runs beside the
+//               other warps' work.  (Adding each row with 16-byte vector
+//               reductions from registers measured 0.925 ms against 0.68 ms
+//               at B 16, H 10, T 2048.)
 
 // Row r, query columns 64*half .. 64*half+63 of a [128][128] bf16 tile kept as
 // two 64-column halves of [128 rows][128 B] with the 128-byte swizzle (16-byte
@@ -540,7 +547,7 @@ __device__ __forceinline__ void store_row_units(uint8_t* tile, const uint32_t (&
     *reinterpret_cast<uint4*>(row + ((u ^ (r & 7)) << 4)) = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
 }
 
-constexpr int TB_STAGE = 32768;   // dQ staging: 64 queries x 128 dims fp32
+constexpr int TB_STAGE = 32768;   // dQ staging: 4 warps x two [32 queries][32 dims] fp32 boxes
 constexpr int TB_SMEM = 6 * TF_BUF + TB_STAGE + 2048 + 256;
 
 // Query-block loop of key block j: nb query blocks j .. (window end) for each
@@ -569,7 +576,7 @@ __device__ __forceinline__ BwdBlock bwd_block(int idx, int H, int Hkv, int kvs, 
 }
 
 template <bool kFine>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                        const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
@@ -602,8 +609,8 @@ __global__ void __launch_bounds__(448, 1)
   uint64_t* s_free = bars + 8;    // S^T_i read by the softmax warps
   uint64_t* dp_full = bars + 9;   // dP^T_i in TMEM
   uint64_t* p_ready = bars + 10;  // P_i in TMEM
-  uint64_t* mm_done = bars + 11;  // dV, dK, dQ^T of block i complete
-  uint64_t* dq_free = bars + 12;  // dQ^T_i read by the dQ warps
+  uint64_t* mm_done = bars + 11;  // dV, dK, dQ of block i complete
+  uint64_t* dq_free = bars + 12;  // dQ_i read by the dQ warps
   uint64_t* drain = bars + 13;
   uint64_t* ds_ready = bars + 14; // dS_i in shared memory
   uint64_t* kv_empty = bars + 15; // an item's last products complete (K and V free) and every warp has its number
@@ -646,6 +653,10 @@ __global__ void __launch_bounds__(448, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // registers: 72 for the TMA / MMA warp group, 96 for the dQ group, 168 for
+  // the two softmax groups (4*72 + 4*96 + 8*168 = 2016 per lane of a warp,
+  // within the 16 warps x 128 the block is launched with)
+  if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
   if (warp == 0) {
     if (lane == 0) {
       // -------------------------------------------------------------- TMA
@@ -722,7 +733,7 @@ __global__ void __launch_bounds__(448, 1)
       // -------------------------------------------------------------- MMA
       constexpr uint32_t IDESC_KK = make_idesc(1, 128, false, false);   // S^T, dP^T
       constexpr uint32_t IDESC_KM = make_idesc(1, 128, false, true);    // dV (A in TMEM), dK
-      constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ^T
+      constexpr uint32_t IDESC_MM = make_idesc(1, 128, true, true);     // dQ
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), do_addr = smem_u32(sdO);
       const uint32_t dst_addr = smem_u32(sdSt);
       // X^T = A B^T over the 128 head dims, both operands K-major; the empty
@@ -746,7 +757,7 @@ __global__ void __launch_bounds__(448, 1)
           const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
           const int n_it = kb.n_it;
           // S^T of the first query block goes where the previous key block's
-          // last dQ^T was (wait until the dQ warps have read it), dP^T where
+          // last dQ was (wait until the dQ warps have read it), dP^T where
           // its last P was (wait until that dV is done)
           ok = mbar_wait_t<kFine>(&q_full[g0 & 1], (g0 >> 1) & 1, abort_flag, err, wlim) &&
                (g0 == 0 || mbar_wait_t<kFine>(dq_free, (g0 - 1) & 1, abort_flag, err, wlim));
@@ -785,7 +796,7 @@ __global__ void __launch_bounds__(448, 1)
                                 IDESC_KM, (it > 0 || kk > 0) ? 1u : 0u);
             }
             umma_commit(do_empty);
-            // dK and dQ^T once dS_i is in shared memory (the softmax warps compute it
+            // dK and dQ once dS_i is in shared memory (the softmax warps compute it
             // while dV runs)
             if (!mbar_wait_t<kFine>(ds_ready, gi & 1, abort_flag, err, wlim)) { ok = false; break; }
             tc_fence_after();
@@ -800,8 +811,8 @@ __global__ void __launch_bounds__(448, 1)
               }
             }
             umma_commit(&q_empty[s]);
-            // dQ^T_i goes to [0,128), which holds S^T_{i+1} (wait until the softmax
-            // warps have read it) or, for the last block, dQ^T_{i-1} (wait until
+            // dQ_i goes to [0,128), which holds S^T_{i+1} (wait until the softmax
+            // warps have read it) or, for the last block, dQ_{i-1} (wait until
             // the dQ warps have read it)
             if (it + 1 < n_it) {
               if (!mbar_wait_t<kFine>(s_free, (gi + 1) & 1, abort_flag, err, wlim)) { ok = false; break; }
@@ -815,7 +826,7 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t off16 = (kk * 2048) >> 4;   // 16 keys per step, both operands MN-major
-                umma_f16(tmem, dka + off16, dsb + off16, IDESC_MM, kk > 0 ? 1u : 0u);
+                umma_f16(tmem, dsb + off16, dka + off16, IDESC_MM, kk > 0 ? 1u : 0u);   // dQ = dS K
               }
             }
             umma_commit(mm_done);
@@ -842,29 +853,17 @@ __global__ void __launch_bounds__(448, 1)
       umma_commit(drain);
       for (uint32_t x = 0; x < (1u << 22) && !mbar_try_wait(drain, 0); ++x) {}
     }
-  } else if (warp >= 10) {
+  } else if (warp >= 12) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;\n" ::: "memory");
     // ------------------------------------------------------------------ dQ
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    uint8_t* box = sStage + quarter * 8192;   // [64 queries][32 dims] fp32, 128-byte swizzle
     const uint64_t sc2 = f2_pack(scale, scale);
     bool ok = true;
-    // dims lane of this warp's quarter for 64 queries -> the box, transposed
-    auto stage = [&](const uint32_t (&va)[32], const uint32_t (&vb)[32]) {
-      if (lane == 0) bulk_wait_read_all();   // the box's previous contents have been read
-      __syncwarp();
-#pragma unroll
-      for (int qq = 0; qq < 64; qq += 2) {
-        const uint32_t (&v)[32] = qq < 32 ? va : vb;
-        const int e = qq & 31;
-        float a0, a1;
-        f2_unpack(f2_mul(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2), a0, a1);
-        *reinterpret_cast<float*>(box + qq * 128 + (((lane >> 2) ^ (qq & 7)) << 4) + (lane & 3) * 4) = a0;
-        *reinterpret_cast<float*>(box + (qq + 1) * 128 + (((lane >> 2) ^ ((qq + 1) & 7)) << 4) + (lane & 3) * 4) = a1;
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-    };
+    // dQ of one query block: this thread's query row (TMEM lane) of 128 dims,
+    // staged 64 dims at a time as two [32 queries][32 dims] fp32 boxes (a row
+    // is 128 bytes: eight 16-byte stores) and added into dq by TMA reduce-add
+    uint8_t* box = sStage + quarter * 8192;
     int g = 0;
     for (int n = 0; ok; ++n) {
       {
@@ -879,40 +878,52 @@ __global__ void __launch_bounds__(448, 1)
       {
         const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         for (int it = 0; it < kb.n_it && ok; ++it, ++g) {
-          const int q0 = kb.q_block(it) * 128, bh = kb.b * H + kb.q_head(it);
+          const int q0 = kb.q_block(it) * 128 + quarter * 32, bh = kb.b * H + kb.q_head(it);
           const bool got = mbar_wait_t<kFine>(mm_done, g & 1, abort_flag, err, wlim);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
           tc_fence_after();
-          uint32_t va[32], vb[32];
-          tmem_load32_async(tmem + lane_base, va);
-          tmem_load32_async(tmem + lane_base + 32, vb);
-          tmem_wait_ld();
-          stage(va, vb);
-          if (lane == 0) {
-            tma_reduce_add_3d(&tdq, box, 32 * quarter, q0, bh);
-            bulk_commit();
-          }
-          tmem_load32_async(tmem + lane_base + 64, va);
-          tmem_load32_async(tmem + lane_base + 96, vb);
-          tmem_wait_ld();
-          tc_fence_before();
-          mbar_arrive(dq_free);
-          stage(va, vb);
-          if (lane == 0) {
-            tma_reduce_add_3d(&tdq, box, 32 * quarter, q0 + 64, bh);
-            bulk_commit();
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t va[32], vb[32];
+            tmem_load32_async(tmem + lane_base + hh * 64, va);
+            tmem_load32_async(tmem + lane_base + hh * 64 + 32, vb);
+            tmem_wait_ld();
+            if (hh == 1) {
+              tc_fence_before();
+              mbar_arrive(dq_free);
+            }
+            if (lane == 0) bulk_wait_read_all();   // the boxes' previous contents have been read
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+              const uint32_t (&v)[32] = j < 32 ? va : vb;
+              const int e = j & 31;
+              float a0, a1, a2, a3;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), sc2), a0, a1);
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3])), sc2), a2, a3);
+              *reinterpret_cast<float4*>(box + (j >> 5) * 4096 + lane * 128 + ((((e >> 2) ^ lane) & 7) << 4)) =
+                  make_float4(a0, a1, a2, a3);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_3d(&tdq, box, hh * 64, q0, bh);
+              tma_reduce_add_3d(&tdq, box + 4096, hh * 64 + 32, q0, bh);
+              bulk_commit();
+            }
           }
         }
       }
     }
     if (lane == 0) bulk_wait_all();
-  } else {
+  } else if (warp >= 4) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 168;\n" ::: "memory");
     // ------------------------------------------------------- P, dS, dK, dV
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;        // which 64 query columns of the row
+    const int half = (warp - 4) >> 2;        // which 64 query columns of the row
     const int r = quarter * 32 + lane;       // key row (TMEM lane)
-    const int t256 = threadIdx.x - 64;       // 0..255
+    const int t256 = threadIdx.x - 128;      // 0..255
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     const float scale_log2 = scale * 1.4426950408889634f;
     const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
@@ -1065,7 +1076,7 @@ __global__ void __launch_bounds__(448, 1)
             fence_proxy_async_smem();
             mbar_arrive(ds_ready);
           }
-          // P_{i+1} while the tensor cores run this block's dV, dK, dQ^T
+          // P_{i+1} while the tensor cores run this block's dV, dK, dQ
           if (it + 1 < n_it) {
             const bool got1 = mbar_wait_t<kFine>(s_full, (gi + 1) & 1, abort_flag, err, wlim);
             if (any_fail(got1)) { ok = false; break; }   // also publishes lse/D of block i+1
@@ -1218,7 +1229,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   if (H % Hkv || kv_stride < Hkv || !make_map(&mq, q, 2, HD, T, bh, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mk, k, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) ||
       !make_map(&mv, v, 2, HD, T, bhkv, HD, 1ll * T * HD, 64, 128) || !make_map_4d(&mdo, dout, dims, strides, box) ||
-      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 64)) {
+      !make_map(&mdq, dq, 4, HD, T, bh, HD, 1ll * T * HD, 32, 32)) {
     if (err) cudaMemsetAsync(err, 0xff, sizeof(int), s);
     return;
   }
@@ -1231,7 +1242,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   const int grid = static_cast<int>(std::min<long long>(n_units, device_sm_count()));
   const int wl = window_bound(window, T);
   int* word = wl >= T ? nullptr : sched_word(sched, s);
-  kern<<<grid, 448, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
+  kern<<<grid, 512, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
                                                 1.f / sqrtf(static_cast<float>(HD)), static_cast<int>(n_units),
                                                 word, err, wait_cycles);
 }
