@@ -113,7 +113,9 @@ def category_work(s):
         # fp32 dx, write fp32 dx and bf16 dx backward
         "norm": ("hbm", (2 * L + 1) * M * d * 6 + (2 * L + 1) * M * d * 14),
         "ce_finish": ("hbm", M * V * 2 * 2),
-        "qk_bwd": ("hbm", L * M * d * (4 + 2 * 4 + 3 * 2)),
+        # q only (the attention backward writes the k and v columns): read fp32
+        # dq and bf16 q, write bf16
+        "qk_bwd": ("hbm", L * M * d * (4 + 2 + 2)),
         "embed": ("hbm", M * d * (2 + 4) + M * d * 4 + V * d * 4),
         "muon_elem": ("hbm", L * 12 * d * d * (12 + 4 + 4 + 10)),
         "adamw": ("hbm", 2 * V * d * 30),

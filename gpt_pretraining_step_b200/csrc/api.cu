@@ -66,7 +66,7 @@ struct Plan {
   // activations
   size_t x, xn1, r1, q, k, v, rq, rk, o, lse, xn2, r2, h;   // per-layer arrays (stride below)
   size_t xf, rf, z, stats, zt, row_loss, loss;
-  size_t dx, dxb, dxn, du, dy, dqf, dk, dv, Dv, dqkv, gx;
+  size_t dx, dxb, dxn, du, dy, dqf, Dv, dqkv, gx;
   size_t splitk, embws, X0, X1, XT0, XT1, Abuf, Bbuf, inv_norm, normws, nfac, sched, rope, err, tok, tgt;
   size_t x0, xin, dx0, dxfin, scws, xe, sig;   // residual extras (allocated only when on)
   size_t vesig, vedz, vepart;                  // value embeddings (allocated only when on)
@@ -245,8 +245,6 @@ void make_plan(const Dims& D, Plan& P) {
   P.du = ab.take(L * M * F * 2);
   P.dy = ab.take(M * d * 2);
   P.dqf = ab.take(M * d * 4);
-  P.dk = ab.take(M * d * 2);
-  P.dv = ab.take(M * d * 2);
   P.Dv = ab.take(M * H * 4);
   P.dqkv = ab.take(L * M * qc * 2);
   P.splitk = ab.take(std::max<size_t>(sk, 4) * 4);
@@ -748,8 +746,6 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
   float* dx = c->A<float>(P.dx);
   bf16* dy = c->A<bf16>(P.dy);
   float* dqf = c->A<float>(P.dqf);
-  bf16* dk = c->A<bf16>(P.dk);
-  bf16* dv = c->A<bf16>(P.dv);
   bf16* gx = c->A<bf16>(P.gx);
   bf16* du_all = c->A<bf16>(P.du);
   bf16* dqkv_all = c->A<bf16>(P.dqkv);
@@ -810,24 +806,27 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
     }
     {
       ProfScope ps(c, GPT_PROF_ATTN_BWD);
+      // dK (through the QK-norm and rotation backward) and dV go straight to
+      // their columns of the q|k|v gradient rows
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
-                      c->A<float>(P.Dv), dqf, dk, dv, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H,
-                      c->wait_cycles);
+                      c->A<float>(P.Dv), dqf, nullptr, nullptr, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H,
+                      c->wait_cycles, rk + static_cast<size_t>(l) * M * H, rope, dqkv);
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
-      launch_qk_bwd(dqf, dk, dv, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
+      launch_qk_bwd(dqf, nullptr, nullptr, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
                     rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv);
     }
     c->launches += 3;
     const int vs = D.ve_slot(l);
     if (vs >= 0) {
-      // value embedding: the table's gradient (3 sigmoid dv, scattered by token
-      // through the fp32 buffer the attention backward no longer needs) and
-      // the gate's
+      // value embedding: the table's gradient (3 sigmoid dv, from the v columns
+      // of the q|k|v gradient rows, scattered by token through the fp32
+      // buffer the attention backward no longer needs) and the gate's
       ProfScope ps(c, GPT_PROF_EMBED);
-      launch_ve_bwd(dv, tok, c->VeWb(vs), c->A<float>(P.vesig) + static_cast<size_t>(vs) * M * D.Hkv, dqf,
-                    c->A<float>(P.vedz), M, D.T, H, D.Hkv, V, s);
+      launch_ve_bwd(dqkv + d + 128 * D.Hkv, D.qc, tok, c->VeWb(vs),
+                    c->A<float>(P.vesig) + static_cast<size_t>(vs) * M * D.Hkv, dqf, c->A<float>(P.vedz), M, D.Hkv, V,
+                    s);
       launch_embed_bwd(tok, dqf, c->VeG(vs), M, 128 * D.Hkv, V, c->A<void>(P.embws), acc, s);
       launch_ve_gate_grad(xn1 + l * Md, c->A<float>(P.vedz), c->A<float>(P.vepart), c->GateG(vs), M, d, D.Hkv,
                           D.veC, acc, s);

@@ -582,7 +582,8 @@ __global__ void __launch_bounds__(512, 1)
                        const __grid_constant__ CUtensorMap tdq, const float* __restrict__ lse,
                        const float* __restrict__ Dv, bf16* __restrict__ dk, bf16* __restrict__ dv, int H, int Hkv,
                        int kvs, int T, int wl, float scale, int n_units, int* sched, int* err,
-                       long long wait_cycles) {
+                       long long wait_cycles, const float* __restrict__ rk, const float2* __restrict__ rope,
+                       bf16* __restrict__ dqkv) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // the 128-byte-swizzled tiles need a 1024-byte-aligned base, which the
   // dynamic shared memory window provides; refuse to run otherwise
@@ -952,13 +953,21 @@ __global__ void __launch_bounds__(512, 1)
       }
       const int idx = item_ring[n & 3];
       __syncwarp();
-      if (lane == 0) mbar_arrive(kv_empty);   // this warp has the item number
+      // this warp has the item number; when dK goes through the QK-norm
+      // backward, K stays until the item's epilogue has read its rows
+      if (lane == 0 && (idx < 0 || !dqkv)) mbar_arrive(kv_empty);
       if (idx < 0) break;
       {
         const BwdBlock kb = bwd_block(idx, H, Hkv, kvs, nq, wl);
         const int n_it = kb.n_it, k0 = kb.k0, bkv = kb.kvrow;
         const int key = k0 + r;
         const bool key_ok = key < T;
+        if (dqkv && key_ok) {
+          // the epilogue's rotation table row and inverse RMS, on their way to L2
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rope + static_cast<long long>(key) * 64 + 32 * half));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rope + static_cast<long long>(key) * 64 + 32 * half + 16));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(rk + (static_cast<long long>(kb.b) * T + key) * H + kb.hk));
+        }
         // this thread's share of a query block's -lse (log2 units; -inf past T so
         // P = 0) or -D, fetched a block ahead so the load latency hides
         auto fetch = [&](int it2) -> float {
@@ -1089,7 +1098,111 @@ __global__ void __launch_bounds__(512, 1)
           const bool got = mbar_wait_t<kFine>(mm_done, (g0 + n_it - 1) & 1, abort_flag, err, wlim);
           ok = !any_fail(got);
         }
-        if (ok) {
+        if (ok && dqkv) {
+          // straight into the token-major q|k|v gradient rows: dV as it is, dK
+          // through the backward of the QK RMS norm and of the rotation
+          // (head dims i and 64 + i form a rotated pair; this thread takes the
+          // pairs 32 * half .. 32 * half + 31, the other half's thread the rest
+          // of the row, and the two add up the row's <dK, k> in shared memory)
+          tc_fence_after();
+          const long long m = static_cast<long long>(kb.b) * T + key;
+          const int dqk = H * 128, kvd = Hkv * 128;
+          bf16* orow = dqkv + m * (dqk + 2 * kvd) + dqk + kb.hk * 128;
+          // the normalised rotated k of this row at the same dims, from the K
+          // tile in shared memory (two 64-column halves of [128 rows][128 B],
+          // 16-byte unit u of row r at u ^ (r & 7)); then K may be replaced
+          uint4 yl[4], yh[4];
+#pragma unroll
+          for (int x = 0; x < 4; ++x) {
+            const int u = (4 * half + x) ^ (r & 7);
+            yl[x] = *reinterpret_cast<const uint4*>(sK + r * 128 + u * 16);
+            yh[x] = *reinterpret_cast<const uint4*>(sK + TF_TILE + r * 128 + u * 16);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(kv_empty);
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t vr[32];
+            tmem_load32_async(tmem + lane_base + 256 + 64 * half + 32 * c, vr);
+            tmem_wait_ld();
+            if (key_ok) {
+#pragma unroll
+              for (int gg = 0; gg < 32; gg += 8) {
+                uint4 wv;
+                wv.x = pack_bf16x2(__uint_as_float(vr[gg]), __uint_as_float(vr[gg + 1]));
+                wv.y = pack_bf16x2(__uint_as_float(vr[gg + 2]), __uint_as_float(vr[gg + 3]));
+                wv.z = pack_bf16x2(__uint_as_float(vr[gg + 4]), __uint_as_float(vr[gg + 5]));
+                wv.w = pack_bf16x2(__uint_as_float(vr[gg + 6]), __uint_as_float(vr[gg + 7]));
+                *reinterpret_cast<uint4*>(orow + kvd + 64 * half + 32 * c + gg) = wv;
+              }
+            }
+          }
+          // <dK, k> over this thread's pairs, 16 at a time (dK read from TMEM
+          // twice, here and for the result, to keep the registers down)
+          float part = 0.f;
+#pragma unroll
+          for (int hq = 0; hq < 2; ++hq) {
+            uint32_t gl[16], gh[16];
+            tmem_load16_async(tmem + lane_base + 384 + 32 * half + 16 * hq, gl);
+            tmem_load16_async(tmem + lane_base + 448 + 32 * half + 16 * hq, gh);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              const uint4 a = yl[2 * hq + x], bq = yh[2 * hq + x];
+              const uint32_t wl4[4] = {a.x, a.y, a.z, a.w};
+              const uint32_t wh4[4] = {bq.x, bq.y, bq.z, bq.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int i = 8 * x + 2 * e;
+                part += __uint_as_float(gl[i]) * bf16_lo(wl4[e]) + __uint_as_float(gl[i + 1]) * bf16_hi(wl4[e]) +
+                        __uint_as_float(gh[i]) * bf16_lo(wh4[e]) + __uint_as_float(gh[i + 1]) * bf16_hi(wh4[e]);
+              }
+            }
+          }
+          // the two halves of the row meet in the softmax warps' lse buffer,
+          // which no thread reads again before the next item's first vote
+          lse_s[half * 128 + r] = part;
+          asm volatile("bar.sync 1, 256;" ::: "memory");
+          // dK = scale * (the TMEM sums); <dK, k> / 128 over the whole row
+          const float dot = (part + lse_s[(half ^ 1) * 128 + r]) * scale * (1.f / 128.f);
+          const float rr = key_ok ? rk[m * H + kb.hk] : 0.f;
+          const float4* e4 = reinterpret_cast<const float4*>(rope + static_cast<long long>(key_ok ? key : 0) * 64 +
+                                                             32 * half);
+#pragma unroll
+          for (int hq = 0; hq < 2; ++hq) {
+            uint32_t gl[16], gh[16];
+            tmem_load16_async(tmem + lane_base + 384 + 32 * half + 16 * hq, gl);
+            tmem_load16_async(tmem + lane_base + 448 + 32 * half + 16 * hq, gh);
+            tmem_wait_ld();
+            if (key_ok) {
+#pragma unroll
+              for (int x = 0; x < 2; ++x) {
+                const uint4 a = yl[2 * hq + x], bq = yh[2 * hq + x];
+                const uint32_t wl4[4] = {a.x, a.y, a.z, a.w};
+                const uint32_t wh4[4] = {bq.x, bq.y, bq.z, bq.w};
+                uint32_t ol[4], oh[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int i = 8 * x + 2 * e;
+                  const float4 cs = __ldg(e4 + ((16 * hq + i) >> 1));   // (cos, sin) of pairs i and i + 1
+                  // gradient w.r.t. the rotated vector, then the transposed rotation
+                  const float rl0 = rr * (__uint_as_float(gl[i]) * scale - bf16_lo(wl4[e]) * dot);
+                  const float rl1 = rr * (__uint_as_float(gl[i + 1]) * scale - bf16_hi(wl4[e]) * dot);
+                  const float rh0 = rr * (__uint_as_float(gh[i]) * scale - bf16_lo(wh4[e]) * dot);
+                  const float rh1 = rr * (__uint_as_float(gh[i + 1]) * scale - bf16_hi(wh4[e]) * dot);
+                  ol[e] = pack_bf16x2(rl0 * cs.x + rh0 * cs.y, rl1 * cs.z + rh1 * cs.w);
+                  oh[e] = pack_bf16x2(-rl0 * cs.y + rh0 * cs.x, -rl1 * cs.w + rh1 * cs.z);
+                }
+                const int col = 32 * half + 16 * hq + 8 * x;
+                *reinterpret_cast<uint4*>(orow + col) = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+                *reinterpret_cast<uint4*>(orow + 64 + col) = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+              }
+            }
+          }
+          // dK and dV have been read: the next key block's first products may
+          // overwrite them (they follow this thread's next p_ready / ds_ready)
+          tc_fence_before();
+        } else if (ok) {
           tc_fence_after();
           bf16* dkrow = dk + (static_cast<long long>(bkv) * T + key) * 128;
           bf16* dvrow = dv + (static_cast<long long>(bkv) * T + key) * 128;
@@ -1208,7 +1321,7 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride,
-                     long long wait_cycles) {
+                     long long wait_cycles, const float* rk, const float2* rope, bf16* dqkv) {
   const bool fine = wait_limit_or_default(wait_cycles) < kShortWaitCycles;
   auto kern = fine ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
   static std::atomic<unsigned long long> configured[2] = {};
@@ -1244,7 +1357,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   int* word = wl >= T ? nullptr : sched_word(sched, s);
   kern<<<grid, 512, TB_SMEM, s>>>(mq, mk, mv, mdo, mdq, lse, Dv, dk, dv, H, Hkv, kv_stride, T, wl,
                                                 1.f / sqrtf(static_cast<float>(HD)), static_cast<int>(n_units),
-                                                word, err, wait_cycles);
+                                                word, err, wait_cycles, rk, rope, dqkv);
 }
 
 }  // namespace gpt

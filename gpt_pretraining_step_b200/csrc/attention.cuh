@@ -22,12 +22,19 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
                      int kv_stride = 0, long long wait_cycles = 0);
 
 // Gradients of o w.r.t. q, k, v given dout [B, T, H, 128]: dq (fp32
-// [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, Hkv, T, 128]
-// (summed over the query heads of each kv head); Dv [B, H, T] is scratch;
-// sched as for the forward.
+// [B, H, T, 128], zeroed here, then accumulated), dk, dv [B, kv_stride, T,
+// 128] with the kv heads at rows h < Hkv (summed over the query heads of each
+// kv head); Dv [B, H, T] is scratch; sched as for the forward.
+// With dqkv, dk and dv are not written: dV goes to the v columns of the
+// token-major gradient rows dqkv [B*T, (H + 2 Hkv) * 128] and dK, taken
+// through the backward of the QK RMS norm (k holds the normalised rotated
+// keys, rk [B*T, H] their inverse RMS, kv head h at column h) and of the
+// rotation (rope [T, 64] (cos, sin) of the pairs (i, 64 + i)), to its k
+// columns; the q columns are left to the caller.
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr,
-                     int kv_stride = 0, long long wait_cycles = 0);
+                     int kv_stride = 0, long long wait_cycles = 0, const float* rk = nullptr,
+                     const float2* rope = nullptr, bf16* dqkv = nullptr);
 
 }  // namespace gpt

@@ -521,21 +521,19 @@ __global__ void __launch_bounds__(256) ve_fwd_kernel(const bf16* __restrict__ xn
 // Backward, given dv [B, H, T, 128] (the gradient at the attention input):
 // dve[t, h] = 3 sig dv[t, h] (fp32 [M, d], scattered into the table's
 // gradient afterwards) and dz[t, h] = (ve[t, h] . dv[t, h]) 3 sig (1 - sig).
-__global__ void __launch_bounds__(256) ve_bwd_kernel(const bf16* __restrict__ dv, const int* __restrict__ tok,
-                                                     const bf16* __restrict__ ve, const float* __restrict__ sig,
-                                                     float* __restrict__ dve, float* __restrict__ dz, int M, int T,
-                                                     int H, int Hkv, int V) {
+__global__ void __launch_bounds__(256) ve_bwd_kernel(const bf16* __restrict__ dv, long long ldv,
+                                                     const int* __restrict__ tok, const bf16* __restrict__ ve,
+                                                     const float* __restrict__ sig, float* __restrict__ dve,
+                                                     float* __restrict__ dz, int M, int Hkv, int V) {
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= M) return;
   const int kvd = Hkv * 128;
-  const int b = t / T, pos = t - b * T;
   int id = tok[t];
   id = static_cast<unsigned>(id) < static_cast<unsigned>(V) ? id : 0;
   const bf16* er = ve + static_cast<long long>(id) * kvd;
   for (int h = 0; h < Hkv; ++h) {
-    const uint2 g = *reinterpret_cast<const uint2*>(dv + ((static_cast<long long>(b) * H + h) * T + pos) * 128 +
-                                                    4 * lane);
+    const uint2 g = *reinterpret_cast<const uint2*>(dv + static_cast<long long>(t) * ldv + h * 128 + 4 * lane);
     const uint2 e = *reinterpret_cast<const uint2*>(er + h * 128 + 4 * lane);
     const float g0 = bf16_lo(g.x), g1 = bf16_hi(g.x), g2 = bf16_lo(g.y), g3 = bf16_hi(g.y);
     float dot = g0 * bf16_lo(e.x) + g1 * bf16_hi(e.x) + g2 * bf16_lo(e.y) + g3 * bf16_hi(e.y);
@@ -620,7 +618,7 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
   const float2 e0 = rope[t * 64 + i0], e1 = rope[t * 64 + i0 + 1];
   // row of dqkv: q (d) | k (kvd) | v (kvd); head h of k and v only for h < Hkv
   bf16* out = dqkv + m * (d + 2 * kvd) + h * 128;
-  const bool has_kv = !kGrouped || h < Hkv;
+  const bool has_kv = dk && (!kGrouped || h < Hkv);   // no dk: the k and v columns are written elsewhere
   float am = 0.f;   // max |written value| (for fp8 scales)
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
@@ -1231,9 +1229,9 @@ void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float*
   ve_fwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(xn1, tok, ve, wg, sig, v, M, T, H, Hkv, C, V);
 }
 
-void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
-                   int T, int H, int Hkv, int V, cudaStream_t s) {
-  ve_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dv, tok, ve, sig, dve, dz, M, T, H, Hkv, V);
+void launch_ve_bwd(const bf16* dv, long long ldv, const int* tok, const bf16* ve, const float* sig, float* dve,
+                   float* dz, int M, int Hkv, int V, cudaStream_t s) {
+  ve_bwd_kernel<<<cdiv(M, 8), 256, 0, s>>>(dv, ldv, tok, ve, sig, dve, dz, M, Hkv, V);
 }
 
 void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,

@@ -34,7 +34,8 @@ void launch_rmsnorm_bwd(const float* dy, const bf16* y, const float* rstd, float
 
 // Per-head QK-norm and RoPE backward plus the v copy, into dqkv [M, d + 2
 // Hkv 128] (dq is the fp32 attention-backward accumulator, dk and dv bf16,
-// kv head j of batch b at head row b*H + j; Hkv 0 = H).
+// kv head j of batch b at head row b*H + j; Hkv 0 = H).  With dk null only
+// the q columns are written (the attention backward wrote the k and v ones).
 void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* qn, const bf16* kn,
                    const float* rq, const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H,
                    cudaStream_t s, int Hkv = 0, unsigned int* amax = nullptr);
@@ -118,8 +119,9 @@ int resid_partial_blocks();
 // gradient correction.
 void launch_ve_fwd(const bf16* xn1, const int* tok, const bf16* ve, const float* wg, float* sig, bf16* v, int M,
                    int T, int H, int Hkv, int C, int V, cudaStream_t s);
-void launch_ve_bwd(const bf16* dv, const int* tok, const bf16* ve, const float* sig, float* dve, float* dz, int M,
-                   int T, int H, int Hkv, int V, cudaStream_t s);
+// (dv: the v gradient of token t, kv head h at dv[t * ldv + h * 128 ..])
+void launch_ve_bwd(const bf16* dv, long long ldv, const int* tok, const bf16* ve, const float* sig, float* dve,
+                   float* dz, int M, int Hkv, int V, cudaStream_t s);
 void launch_ve_gate_grad(const bf16* xn1, const float* dz, float* part, float* grad, int M, int d, int H, int C,
                          bool accumulate, cudaStream_t s);
 void launch_ve_dxn(float* dxn, const float* dz, const float* wg, int M, int d, int H, int C, cudaStream_t s);
