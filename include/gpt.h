@@ -79,7 +79,8 @@ enum { GPT_GROUP_ADAMW = 0, GPT_GROUP_MUON = 1 };
  *             (its rounding enters the QK-normalised attention logits),
  *             attention and the lm_head stay bf16
  *   ns_tf32_steps  operand precision of the five Newton-Schulz steps:
- *             -1 = fp16 operands at the full tensor rate with fp32 iterates
+ *             -1 = fp16 operands at the full tensor rate, iterates carried as
+ *             fp16 (high, low) pairs of about 22 significant bits
  *             (the recommended setting); 0..5 = that many leading steps with
  *             fp32 operands read as tf32 (half rate), the rest bf16.  fp16
  *             operands keep the update within ~1% of fp64 on the decaying
