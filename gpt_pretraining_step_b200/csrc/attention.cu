@@ -14,6 +14,7 @@
 // TMEM accumulators), fed by TMA; softmax work runs in dedicated warps that
 // exchange tiles with the MMA issuer through mbarriers.
 #include <algorithm>
+#include <type_traits>
 
 #include "attention.cuh"
 #include "common.cuh"
@@ -120,6 +121,18 @@ __device__ __forceinline__ FwdItem fwd_item(int n, int nq, int H, int Hkv, int k
   it.nkvB = it.hasB ? it.qtA + 2 - it.j0 : 0;
   it.nkv = it.hasB ? it.nkvB : it.nkvA;
   return it;
+}
+
+// S row of query row 32 Q + lane of a causal diagonal block: keys 32 Q + lane
+// + 1 .. 127 become -inf (the keys of chunk Q above the lane, then every
+// later chunk); Q is the warp's TMEM lane quarter, so no branch diverges.
+template <int Q>
+__device__ __forceinline__ void causal_mask_row(uint32_t (&sr)[128], int lane) {
+#pragma unroll
+  for (int k = 0; k < 32; ++k)
+    if (k > lane) sr[32 * Q + k] = __float_as_uint(-INFINITY);
+#pragma unroll
+  for (int k = 32 * (Q + 1); k < 128; ++k) sr[k] = __float_as_uint(-INFINITY);
 }
 
 template <bool kFine>
@@ -367,8 +380,18 @@ __global__ void __launch_bounds__(384, 1)
           tmem_wait_ld();
         }
         const int kbase = (it.j0 + j) * 128;
-        if ((it.j0 + j == qt) || (kbase + 128 > T) || (kbase < q0 + 127 - wl)) {
-          // causal diagonal, ragged tail or window edge: masked scores become -inf
+        const bool diag = it.j0 + j == qt, edge = (kbase + 128 > T) || (kbase < q0 + 127 - wl);
+        if (diag && !edge) {
+          // causal diagonal block: only the keys above the row are masked, so
+          // per element in one 32-key chunk, whole chunks beyond it
+          switch (quarter) {
+            case 0: causal_mask_row<0>(sr, lane); break;
+            case 1: causal_mask_row<1>(sr, lane); break;
+            case 2: causal_mask_row<2>(sr, lane); break;
+            default: causal_mask_row<3>(sr, lane); break;
+          }
+        } else if (diag || edge) {
+          // ragged tail or window edge: masked scores become -inf
 #pragma unroll
           for (int k = 0; k < 128; ++k) {
             const int key = kbase + k;
@@ -992,7 +1015,8 @@ __global__ void __launch_bounds__(512, 1)
           const int q0 = kb.q_block(it2) * 128;
           // causal diagonal block, ragged key block, or a query block whose last
           // rows' windows start past this block's first key
-          const bool masked = diag || k0 + 128 > T || q0 + 127 - wl > k0;
+          const bool edge = k0 + 128 > T || q0 + 127 - wl > k0;
+          const bool masked = diag || edge;
           const float* nls = lse_s + ((g0 + it2) & 1) * 128;
           uint32_t sa[32], sb[32];
           tmem_load32_async(tmem + lane_base + (2 * half) * 32, sa);
@@ -1000,40 +1024,76 @@ __global__ void __launch_bounds__(512, 1)
           tmem_wait_ld();
           tc_fence_before();
           mbar_arrive(s_free);   // S^T of this block has been read
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
+          // One 32-query chunk of the row in one of four forms, chosen per
+          // chunk by a warp-uniform test: no mask, the causal diagonal's lane
+          // mask (queries below the key row), all masked (P = 0), or the general
+          // mask (ragged keys, window edge).  A per-element mask inside one loop
+          // was if-converted into every block's path and cost more than the
+          // exponentials.
+          auto run_chunk = [&](auto kCC, auto kMode) {
+            constexpr int cc = decltype(kCC)::value, mode = decltype(kMode)::value;
             const int c = 2 * half + cc;
             const uint32_t (&sr)[32] = cc == 0 ? sa : sb;
+            if constexpr (mode == 3) {
 #pragma unroll
-            for (int kq = 0; kq < 32; kq += 8) {
-              const float4 la = *reinterpret_cast<const float4*>(nls + c * 32 + kq);
-              const float4 lb = *reinterpret_cast<const float4*>(nls + c * 32 + kq + 4);
-              const float nl[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};   // -lse * log2(e)
-              // P = 2^(S * scale * log2(e) - lse * log2(e)): six of every eight on the
-              // MUFU unit, two by the polynomial on the FMA pipe
-              float p[8];
+              for (int x = 0; x < 16; ++x) pk[16 * cc + x] = 0u;
+            } else {
 #pragma unroll
-              for (int e = 0; e < 8; e += 2) {
-                float x0, x1;
-                f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[kq + e]), __uint_as_float(sr[kq + e + 1])), sl2,
-                                 f2_pack(nl[e], nl[e + 1])),
-                          x0, x1);
-                if (e < GPT_BWD_MUFU) {
-                  p[e] = ex2_approx(x0);
-                  p[e + 1] = ex2_approx(x1);
-                } else {
-                  f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+              for (int kq = 0; kq < 32; kq += 8) {
+                const float4 la = *reinterpret_cast<const float4*>(nls + c * 32 + kq);
+                const float4 lb = *reinterpret_cast<const float4*>(nls + c * 32 + kq + 4);
+                const float nl[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};   // -lse * log2(e)
+                // P = 2^(S * scale * log2(e) - lse * log2(e)): GPT_BWD_MUFU of every
+                // eight on the MUFU unit, the rest by the polynomial on the FMA pipe
+                float p[8];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                  float x0, x1;
+                  f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[kq + e]), __uint_as_float(sr[kq + e + 1])), sl2,
+                                   f2_pack(nl[e], nl[e + 1])),
+                            x0, x1);
+                  if (e < GPT_BWD_MUFU) {
+                    p[e] = ex2_approx(x0);
+                    p[e + 1] = ex2_approx(x1);
+                  } else {
+                    f2_unpack(f2_exp2_poly(f2_pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f))), p[e], p[e + 1]);
+                  }
                 }
-              }
-              if (masked) {
+                if constexpr (mode == 1) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                  if (!key_ok || (diag && key > q0 + c * 32 + kq + e) || key < q0 + c * 32 + kq + e - wl) p[e] = 0.f;
-              }
+                  for (int e = 0; e < 8; ++e)
+                    if (kq + e < lane) p[e] = 0.f;
+                } else if constexpr (mode == 2) {
 #pragma unroll
-              for (int e = 0; e < 8; e += 2) pk[16 * cc + ((kq + e) >> 1)] = pack_bf16x2(p[e], p[e + 1]);
+                  for (int e = 0; e < 8; ++e)
+                    if (!key_ok || (diag && key > q0 + c * 32 + kq + e) || key < q0 + c * 32 + kq + e - wl) p[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) pk[16 * cc + ((kq + e) >> 1)] = pack_bf16x2(p[e], p[e + 1]);
+              }
             }
-          }
+          };
+          using M0 = std::integral_constant<int, 0>;
+          using M1 = std::integral_constant<int, 1>;
+          using M2 = std::integral_constant<int, 2>;
+          using M3 = std::integral_constant<int, 3>;
+          auto do_chunk = [&](auto kCC) {
+            const int c = 2 * half + decltype(kCC)::value;
+            if (diag && !edge) {
+              if (c < quarter)
+                run_chunk(kCC, M3{});
+              else if (c == quarter)
+                run_chunk(kCC, M1{});
+              else
+                run_chunk(kCC, M0{});
+            } else if (masked) {
+              run_chunk(kCC, M2{});
+            } else {
+              run_chunk(kCC, M0{});
+            }
+          };
+          do_chunk(std::integral_constant<int, 0>{});
+          do_chunk(std::integral_constant<int, 1>{});
         };
 
         publish(0, fetch(0));
