@@ -801,6 +801,8 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       ProfScope ps(c, GPT_PROF_DX_GEMM);
       g.epi = EPI_STORE; g.out_es = 2; g.aux_es = 2;
       g.p.out = dy; g.p.ldo = d; g.p.err = err;
+      // and the attention backward's D = rowsum(dO * O) per head
+      g.p.row_dot = 1; g.p.aux = ol; g.p.ld_aux = d; g.p.f32a = c->A<float>(P.Dv); g.p.T = D.T; g.p.H = H;
       GPT_CK(run_gemm(g, s, c->wait_cycles));
       c->launches += 1;
     }
@@ -810,14 +812,14 @@ int forward_backward(gpt_ctx* c, const int* tok, const int* tgt_in, float* loss_
       // their columns of the q|k|v gradient rows
       launch_attn_bwd(q + l * Md, k + l * Md, v + l * Md, ol, dy, lse + static_cast<size_t>(l) * M * H,
                       c->A<float>(P.Dv), dqf, nullptr, nullptr, D.B, H, D.T, s, err, D.Hkv, D.window(l), c->A<int>(P.sched), H,
-                      c->wait_cycles, rk + static_cast<size_t>(l) * M * H, rope, dqkv);
+                      c->wait_cycles, rk + static_cast<size_t>(l) * M * H, rope, dqkv, true);
     }
     {
       ProfScope ps(c, GPT_PROF_QK_BWD);
       launch_qk_bwd(dqf, nullptr, nullptr, q + l * Md, k + l * Md, rq + static_cast<size_t>(l) * M * H,
                     rk + static_cast<size_t>(l) * M * H, rope, dqkv, D.B, D.T, H, s, D.Hkv);
     }
-    c->launches += 3;
+    c->launches += 2;
     const int vs = D.ve_slot(l);
     if (vs >= 0) {
       // value embedding: the table's gradient (3 sigmoid dv, from the v columns

@@ -1381,7 +1381,7 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv, int window, int* sched, int kv_stride,
-                     long long wait_cycles, const float* rk, const float2* rope, bf16* dqkv) {
+                     long long wait_cycles, const float* rk, const float2* rope, bf16* dqkv, bool d_ready) {
   const bool fine = wait_limit_or_default(wait_cycles) < kShortWaitCycles;
   auto kern = fine ? attn_bwd_tc_kernel<true> : attn_bwd_tc_kernel<false>;
   static std::atomic<unsigned long long> configured[2] = {};
@@ -1391,7 +1391,7 @@ void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o,
   }
   if (Hkv <= 0) Hkv = H;
   const long long rows = 1ll * B * H * T;
-  attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
+  if (!d_ready) attn_bwd_dot_kernel<<<static_cast<int>((rows + 7) / 8), 256, 0, s>>>(o, dout, Dv, B, H, T);
   cudaMemsetAsync(dq, 0, static_cast<size_t>(rows) * HD * sizeof(float), s);
   CUtensorMap mq, mk, mv, mdo, mdq;
   if (kv_stride <= 0) kv_stride = Hkv;

@@ -30,11 +30,12 @@ void launch_attn_fwd(const bf16* q, const bf16* k, const bf16* v, bf16* o, float
 // through the backward of the QK RMS norm (k holds the normalised rotated
 // keys, rk [B*T, H] their inverse RMS, kv head h at column h) and of the
 // rotation (rope [T, 64] (cos, sin) of the pairs (i, 64 + i)), to its k
-// columns; the q columns are left to the caller.
+// columns; the q columns are left to the caller.  d_ready: Dv already holds
+// D = rowsum(dout * o) (the dout GEMM's epilogue computed it).
 void launch_attn_bwd(const bf16* q, const bf16* k, const bf16* v, const bf16* o, const bf16* dout,
                      const float* lse, float* Dv, float* dq, bf16* dk, bf16* dv, int B, int H, int T,
                      cudaStream_t s, int* err, int Hkv = 0, int window = -1, int* sched = nullptr,
                      int kv_stride = 0, long long wait_cycles = 0, const float* rk = nullptr,
-                     const float2* rope = nullptr, bf16* dqkv = nullptr);
+                     const float2* rope = nullptr, bf16* dqkv = nullptr, bool d_ready = false);
 
 }  // namespace gpt

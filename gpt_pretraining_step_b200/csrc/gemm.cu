@@ -177,6 +177,10 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   CUtensorMap md;
   p.tma_out2 = 0;
   if (p.split_lo && (!p.out2 || p.out_t || c.out_es != 2 || !c.out_f16 || c.sym)) return cudaErrorInvalidValue;
+  if (p.row_dot && (c.epi != EPI_STORE || c.out_es != 2 || c.out_f16 || c.bn != 256 || c.batch != 1 || c.sym ||
+                    p.splits > 1 || c.N % 128 || !p.aux || !p.f32a || p.T <= 0 || c.M % p.T || p.H * 128 != c.N ||
+                    (p.ld_aux & 7) || (reinterpret_cast<uintptr_t>(p.aux) & 15)))
+    return cudaErrorInvalidValue;
   if (p.out2) {
     if (c.epi == EPI_QKV || c.epi == EPI_LOGITS || p.splits > 1 || !p.tma_out) return cudaErrorInvalidValue;
     if (!make_map(&md, p.out2, 2, c.N, c.M, c.batch, p.ldo, p.out_bs, 64, 32, true)) return cudaErrorInvalidValue;

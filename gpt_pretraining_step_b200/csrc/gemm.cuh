@@ -584,6 +584,9 @@ __global__ void __launch_bounds__(320, 1)
           }
         };
         prefetch(c_begin);
+        float rdot = 0.f;   // row_dot: this row's <out, aux> over the thread's 128 columns
+        // (N is a multiple of 128, so the thread's columns are all inside or all past N)
+        const bool dot_here = p.row_dot && row_ok && nb * BN + c_begin * 32 < p.N;
 #pragma unroll 1
         for (int c = c_begin; c < c_end; c += 2) {
           uint32_t ra[32], rb[32];
@@ -651,6 +654,26 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           if (tma_here) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          if constexpr (EPI == EPI_STORE && std::is_same<OutT, __nv_bfloat16>::value) {
+            if (dot_here) {
+              // the stored (bf16-rounded) values against the same columns of aux
+              const uint4* arow = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.aux) +
+                                                                 static_cast<long long>(row) * p.ld_aux +
+                                                                 nb * BN + c * 32);
+#pragma unroll
+              for (int g = 0; g < 8; ++g) {
+                const uint4 w = __ldg(arow + g);
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                const float (&vv)[32] = v[g >> 2];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const int j = (g & 3) * 8 + 2 * e;
+                  rdot += __bfloat162float(__float2bfloat16_rn(vv[j])) * __uint_as_float(ws[e] << 16) +
+                          __bfloat162float(__float2bfloat16_rn(vv[j + 1])) * __uint_as_float(ws[e] & 0xFFFF0000u);
+                }
+              }
+            }
+          }
           // optional fp16 copy of the output in the same layout, or the rounding
           // residual of an fp16 main output (then the TMA path alone stores v)
           if (p.tma_out2) {
@@ -693,6 +716,13 @@ __global__ void __launch_bounds__(320, 1)
                 if (j < nvalid && (!kRect || col0 + j > row))
                   store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
             }
+          }
+        }
+        if constexpr (EPI == EPI_STORE && std::is_same<OutT, __nv_bfloat16>::value) {
+          // one 128-column head per thread: D[(b H + h) T + t] for row b T + t
+          if (dot_here) {
+            const int b = row / p.T, t = row - b * p.T, h = (nb * BN + c_begin * 32) >> 7;
+            p.f32a[(static_cast<long long>(b) * p.H + h) * p.T + t] = rdot;
           }
         }
       }

@@ -26,6 +26,8 @@ struct GemmParams {
   float gamma;          // AXPBY: added to the diagonal elements (row == column) of every output matrix
   int split_lo;         // 1: the second (fp16) output holds out - fp16(out), the rounding residual of
                         //   the fp16 main output, so that the pair carries ~22 significant bits
+  int row_dot;          // STORE, bf16 output, BN 256: also f32a[(b H + h) T + t] = the sum over head h's
+                        //   128 columns of row b T + t of the stored values times aux (bf16, ld_aux)
   float* f32a;          // QKV: rstd of q [M, H];   LOGITS: (max, sumexp) pairs [M, tiles_n]
   float* f32b;          // QKV: rstd of k [M, H];   LOGITS: target logit [M]
   const int* tgt;       // LOGITS: targets of the rows
