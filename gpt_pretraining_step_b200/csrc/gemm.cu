@@ -74,21 +74,77 @@ bool make_map_4d(CUtensorMap* m, const void* ptr, const long long (&dims)[4], co
 
 namespace {
 
-template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
+using bf16 = __nv_bfloat16;
+using f16 = __half;
+
+// The paired variants compiled (16-bit operands, BN 256), one line each:
+// operand type, A and B MN-major, epilogue, output and aux types.
+#define GPT_GEMM_PAIR_LIST(X)                            \
+  X(bf16, false, true, EPI_QKV, bf16, bf16)              \
+  X(bf16, false, true, EPI_ACC, float, float)            \
+  X(bf16, false, true, EPI_RELU2, bf16, bf16)            \
+  X(bf16, false, true, EPI_LOGITS, bf16, bf16)           \
+  X(bf16, false, true, EPI_STORE, bf16, bf16)            \
+  X(bf16, false, true, EPI_STORE, float, float)          \
+  X(bf16, false, false, EPI_DRELU2, bf16, bf16)          \
+  X(bf16, false, false, EPI_STORE, float, float)         \
+  X(bf16, false, false, EPI_STORE, bf16, bf16)           \
+  X(bf16, true, true, EPI_STORE, float, float)           \
+  X(bf16, true, true, EPI_ACC, float, float)             \
+  X(bf16, true, false, EPI_STORE, float, float)          \
+  X(f16, false, true, EPI_AXPBY, f16, float)             \
+  X(f16, false, true, EPI_AXPBY, f16, f16)               \
+  X(f16, false, true, EPI_AXPBY, float, f16)
+
+bool pair_variant_exists(const GemmCall& c) {
+#define GPT_GEMM_PAIR_HAS(T_, AMN_, BMN_, EPI_, OUT_, AUX_)                                                     \
+  if (c.es == (int)sizeof(T_) && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ &&                          \
+      c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_) && c.f16 == std::is_same<T_, f16>::value && \
+      c.out_f16 == std::is_same<OUT_, f16>::value && c.aux_f16 == std::is_same<AUX_, f16>::value)                \
+    return true;
+  GPT_GEMM_PAIR_LIST(GPT_GEMM_PAIR_HAS)
+#undef GPT_GEMM_PAIR_HAS
+  return false;
+}
+
+template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT, bool PAIR = false>
 cudaError_t launch(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mc, const CUtensorMap& md,
                    const GemmParams& p, cudaStream_t s) {
-  using C = GemmCfg<sizeof(T), BN>;
-  auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT>;
+  using C = GemmCfg<sizeof(T), BN, PAIR>;
+  auto kern = gemm_tc_kernel<T, BN, A_MN, B_MN, EPI, OutT, AuxT, PAIR>;
   static std::atomic<unsigned long long> configured{0};
   cudaError_t e = set_smem_limit_once(kern, C::SMEM, configured);
   if (e != cudaSuccess) return e;
-  const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
-  kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, md, p);
+  if constexpr (!PAIR) {
+    const int grid = p.units < device_sm_count() ? p.units : device_sm_count();
+    kern<<<grid, 320, C::SMEM, s>>>(ma, mb, mc, md, p);
+  } else {
+    // persistent pairs: as many clusters of two as fit at once, at most one per unit
+    static std::atomic<int> max_clusters{0};
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.blockDim = dim3(320, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int mc2 = max_clusters.load(std::memory_order_relaxed);
+    if (mc2 <= 0) {
+      cfg.gridDim = dim3(2 * (device_sm_count() / 2), 1, 1);
+      if (cudaOccupancyMaxActiveClusters(&mc2, kern, &cfg) != cudaSuccess || mc2 <= 0) return cudaErrorInvalidValue;
+      max_clusters.store(mc2, std::memory_order_relaxed);
+    }
+    const int nclusters = p.units < mc2 ? p.units : mc2;
+    cfg.gridDim = dim3(2 * nclusters, 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kern, ma, mb, mc, md, p);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
-
-using bf16 = __nv_bfloat16;
-using f16 = __half;
 
 }  // namespace
 
@@ -132,6 +188,9 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
   p.sym = c.sym ? 1 : 0;
+  c.pair = c.allow_pair && c.bn == 256 && !c.sym && p.splits == 1 && c.es == 2 && c.M > 128 &&
+           wait_limit_or_default(p.wait_cycles) >= kShortWaitCycles && pair_variant_exists(c);
+  if (c.pair) p.tiles_m = (p.tiles_m + 1) / 2;   // one unit per 256-row block: the kernel's index counts pairs
   const long long ntiles = c.sym ? sym_tile_count(p.tiles_m, p.tiles_n, c.bn / 128) : 1ll * p.tiles_m * p.tiles_n;
   const long long units = ntiles * p.splits * c.batch;
   if (units > 0x7fffffffll) return cudaErrorInvalidValue;
@@ -146,7 +205,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
     ok = make_map(&ma, c.A, c.es, c.M, c.K, c.batch, c.lda, c.a_bs, mn_box, bk, c.f16);
   if (!ok) return cudaErrorInvalidValue;
   if (!c.b_mn)
-    ok = make_map(&mb, c.B, c.es, c.K, c.N, c.batch, c.ldb, c.b_bs, bk, c.bn, c.f16);
+    ok = make_map(&mb, c.B, c.es, c.K, c.N, c.batch, c.ldb, c.b_bs, bk, c.pair ? c.bn / 2 : c.bn, c.f16);
   else
     ok = make_map(&mb, c.B, c.es, c.N, c.K, c.batch, c.ldb, c.b_bs, mn_box, bk, c.f16);
   if (!ok) return cudaErrorInvalidValue;
@@ -192,11 +251,19 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   if (c.epi == EPI_ACC && !p.tma_out) return cudaErrorInvalidValue;
   if (!p.tma_out) mc = ma;   // unused by the kernel
 
+#define GPT_GEMM_MATCH(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                        \
+  (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ &&       \
+   c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_) && c.f16 == std::is_same<T_, f16>::value && \
+   c.out_f16 == std::is_same<OUT_, f16>::value && c.aux_f16 == std::is_same<AUX_, f16>::value)
 #define GPT_GEMM_CASE(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_)                                        \
-  if (c.es == (int)sizeof(T_) && c.bn == BN_ && c.a_mn == AMN_ && c.b_mn == BMN_ && c.epi == EPI_ &&  \
-      c.out_es == (int)sizeof(OUT_) && c.aux_es == (int)sizeof(AUX_) && c.f16 == std::is_same<T_, f16>::value && \
-      c.out_f16 == std::is_same<OUT_, f16>::value && c.aux_f16 == std::is_same<AUX_, f16>::value)          \
+  if (!c.pair && GPT_GEMM_MATCH(T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_))                            \
     return launch<T_, BN_, AMN_, BMN_, EPI_, OUT_, AUX_>(ma, mb, mc, md, p, stream);
+#define GPT_GEMM_PAIR_CASE(T_, AMN_, BMN_, EPI_, OUT_, AUX_)                                       \
+  if (c.pair && GPT_GEMM_MATCH(T_, 256, AMN_, BMN_, EPI_, OUT_, AUX_))                             \
+    return launch<T_, 256, AMN_, BMN_, EPI_, OUT_, AUX_, true>(ma, mb, mc, md, p, stream);
+
+  // CTA pairs
+  GPT_GEMM_PAIR_LIST(GPT_GEMM_PAIR_CASE)
 
   // forward
   GPT_GEMM_CASE(bf16, 256, false, true, EPI_QKV, bf16, bf16)
@@ -245,6 +312,8 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   GPT_GEMM_CASE(uint8_t, 256, true, true, EPI_STORE, float, float)
   GPT_GEMM_CASE(uint8_t, 256, true, true, EPI_ACC, float, float)
 #undef GPT_GEMM_CASE
+#undef GPT_GEMM_PAIR_CASE
+#undef GPT_GEMM_MATCH
   return cudaErrorInvalidValue;
 }
 

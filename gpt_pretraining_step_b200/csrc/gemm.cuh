@@ -43,14 +43,15 @@ __device__ __forceinline__ float hi16(uint32_t u) {
   else return bf16_hi(u);
 }
 
-template <int ES, int BN>
+template <int ES, int BN, bool PAIR = false>
 struct GemmCfg {
   static constexpr int BK = 128 / ES;                 // elements of K per stage (one 128 B row)
   static constexpr int MMA_K = 32 / ES;               // K per tcgen05.mma (16 bf16, 8 tf32, 32 fp8)
   static constexpr int A_BYTES = 128 * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_ROWS = PAIR ? BN / 2 : BN;   // rows (N) of B this CTA stages
+  static constexpr int B_BYTES = B_ROWS * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = B_ROWS == 256 ? 4 : 6;
   static constexpr int CHUNK_BYTES = BK * 128;        // one MN-major box: BK rows of 128 B
   static constexpr int TMEM_COLS = 2 * BN;
   // output staging: one 32-row x 128-byte box per epilogue warp
@@ -184,15 +185,18 @@ __device__ __forceinline__ void logits_chunk(const float (&v)[32], int col0, int
 
 // ------------------------------------------------------------------ kernel
 
-template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT>
+// PAIR: a cluster of two CTAs per M = 256 tile (see common.cuh); units then
+// count tile pairs and p.tiles_m counts 256-row blocks.
+template <typename T, int BN, bool A_MN, bool B_MN, int EPI, typename OutT, typename AuxT, bool PAIR = false>
 __global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmD,
                    const __grid_constant__ GemmParams p) {
   constexpr int ES = sizeof(T);
-  using C = GemmCfg<ES, BN>;
-  constexpr uint32_t IDESC =
-      make_idesc(ES == 2 ? (std::is_same<T, __half>::value ? 0 : 1) : (ES == 4 ? 2 : 0), BN, A_MN, B_MN);
+  using C = GemmCfg<ES, BN, PAIR>;
+  static_assert(!PAIR || (ES == 2 && BN == 256), "CTA pairs: 16-bit operands, 256-wide tiles");
+  constexpr uint32_t IDESC = make_idesc(ES == 2 ? (std::is_same<T, __half>::value ? 0 : 1) : (ES == 4 ? 2 : 0), BN,
+                                        A_MN, B_MN, PAIR ? 256 : 128);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,6 +212,11 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = warp_id();
   const int lane = lane_id();
   const long long wlim = wait_limit_or_default(p.wait_cycles);
+  // work units: CTA pairs take every (gridDim.x / 2)-th unit, rank 1 the upper 128 rows
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int u_first = PAIR ? static_cast<int>(blockIdx.x) / 2 : static_cast<int>(blockIdx.x);
+  const int u_step = PAIR ? static_cast<int>(gridDim.x) / 2 : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -216,7 +225,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
+      mbar_init(&tempty[a], PAIR ? 512 : 256);   // every epilogue thread (of both CTAs of a pair)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -227,11 +236,17 @@ __global__ void __launch_bounds__(320, 1)
     if (p.tma_out2) tma_prefetch_desc(&tmD);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    if constexpr (PAIR) {
+      tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(tmem_holder, C::TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // both CTAs' barriers exist before either signals the other
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   float amax = 0.f;   // DRELU2 epilogue: this thread's max |out| (of the bf16-rounded values) over its tiles
@@ -243,15 +258,36 @@ __global__ void __launch_bounds__(320, 1)
       uint32_t phase = 0;
       long long issued = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+      for (int u = u_first; u < p.units && ok; u += u_step) {
         int z, mb, nb, kb0, kb1, split;
         decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
+        if constexpr (PAIR) mb = 2 * mb + static_cast<int>(rank);
+        const int n0 = nb * BN + (PAIR ? 128 * static_cast<int>(rank) : 0);   // first B row staged here
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           const int k0 = kb * C::BK;
+          if constexpr (PAIR) {
+            // both CTAs' bytes complete on the leader's barrier, which the leader expects
+            const uint32_t cb = cluster_addr(&full[stage], 0);
+            if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+            if constexpr (!A_MN) {
+              tma_load_3d_pair(sA, &tmA, cb, k0, mb * 128, z);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 128 / C::BK; ++j)
+                tma_load_3d_pair(sA + j * C::CHUNK_BYTES, &tmA, cb, mb * 128 + j * C::BK, k0, z);
+            }
+            if constexpr (!B_MN) {
+              tma_load_3d_pair(sB, &tmB, cb, k0, n0, z);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::B_ROWS / C::BK; ++j)
+                tma_load_3d_pair(sB + j * C::CHUNK_BYTES, &tmB, cb, n0 + j * C::BK, k0, z);
+            }
+          } else {
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
           if constexpr (!A_MN) {
             tma_load_3d(sA, &tmA, &full[stage], k0, mb * 128, z);
           } else {
@@ -260,18 +296,21 @@ __global__ void __launch_bounds__(320, 1)
               tma_load_3d(sA + j * C::CHUNK_BYTES, &tmA, &full[stage], mb * 128 + j * C::BK, k0, z);
           }
           if constexpr (!B_MN) {
-            tma_load_3d(sB, &tmB, &full[stage], k0, nb * BN, z);
+            tma_load_3d(sB, &tmB, &full[stage], k0, n0, z);
           } else {
 #pragma unroll
             for (int j = 0; j < BN / C::BK; ++j)
-              tma_load_3d(sB + j * C::CHUNK_BYTES, &tmB, &full[stage], nb * BN + j * C::BK, k0, z);
+              tma_load_3d(sB + j * C::CHUNK_BYTES, &tmB, &full[stage], n0 + j * C::BK, k0, z);
+          }
           }
           ++issued;
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
       }
-      if (!ok) {
-        // let every copy this thread started land before the CTA exits
+      if (!ok && (!PAIR || leader)) {
+        // let every copy this thread started land before the CTA exits (a pair's
+        // copies complete on the leader's barriers, so only the leader can tell;
+        // the closing cluster barrier keeps the other CTA until then)
         for (int s = 0; s < C::STAGES; ++s) {
           const bool used = s < stage || issued >= C::STAGES;
           const uint32_t par = s < stage ? phase : (phase ^ 1u);
@@ -282,13 +321,13 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       // ----------------------------------------------------------------- MMA
       int stage = 0;
       uint32_t phase = 0;
       int local = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++local) {
+      for (int u = u_first; u < p.units && ok; u += u_step, ++local) {
         int z, mb, nb, kb0, kb1, split;
         decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
         const int acc = local & 1;
@@ -308,21 +347,32 @@ __global__ void __launch_bounds__(320, 1)
             const uint64_t bd = B_MN ? smem_desc_sw128(b0 + kk * C::MMA_K * 128, C::CHUNK_BYTES, 1024)
                                      : smem_desc_sw128(b0 + kk * 32, 16, 1024);
             const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
-            if constexpr (ES == 2)
+            if constexpr (PAIR)
+              umma_f16_pair(d_tmem, ad, bd, IDESC, accum);
+            else if constexpr (ES == 2)
               umma_f16(d_tmem, ad, bd, IDESC, accum);
             else if constexpr (ES == 4)
               umma_tf32(d_tmem, ad, bd, IDESC, accum);
             else
               umma_f8(d_tmem, ad, bd, IDESC, accum);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (PAIR)
+            umma_commit_pair_both(&empty[stage]);
+          else
+            umma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (PAIR)
+          umma_commit_pair_both(&tfull[acc]);
+        else
+          umma_commit(&tfull[acc]);
       }
       // all MMAs of this thread complete before TMEM is released
-      umma_commit(drain);
+      if constexpr (PAIR)
+        umma_commit_pair_own(drain);
+      else
+        umma_commit(drain);
       for (uint32_t i = 0; i < (1u << 22) && !mbar_try_wait(drain, 0); ++i) {}
     }
   } else {
@@ -390,9 +440,10 @@ __global__ void __launch_bounds__(320, 1)
       emit64_to(OutT{}, &tmC, EPI == EPI_ACC, v0, v1, col0, row0, z3);
     };
     int local = 0;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x, ++local) {
+    for (int u = u_first; u < p.units; u += u_step, ++local) {
       int z, mb, nb, kb0, kb1, split;
       decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
+      if constexpr (PAIR) mb = 2 * mb + static_cast<int>(rank);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
       if constexpr (EPI == EPI_DRELU2 || EPI == EPI_AXPBY) {
@@ -727,7 +778,10 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if constexpr (PAIR)
+        mbar_arrive_cluster(cluster_addr(&tempty[acc], 0));   // the leader's MMAs refill this TMEM
+      else
+        mbar_arrive(&tempty[acc]);
     }
   }
 
@@ -740,9 +794,13 @@ __global__ void __launch_bounds__(320, 1)
   if (warp >= 2 && lane == 0) bulk_wait_all();   // output boxes written before the CTA exits
   tc_fence_before();
   __syncthreads();
+  if constexpr (PAIR) cluster_sync();   // neither CTA leaves while the other may still signal it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (PAIR)
+      tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else
+      tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 

@@ -27,6 +27,11 @@ struct GemmCall {
   long long ldb = 0, b_bs = 0;
   int bn = 256, splits = 1;
   bool sym = false;
+  // CTA pairs (2-CTA clusters, M = 256 per tile) where the call allows them:
+  // BN 256, 16-bit operands, no sym, no K split, a bound on waits of at least
+  // kShortWaitCycles, and a compiled paired variant; else one CTA per tile
+  bool allow_pair = true;
+  bool pair = false;   // set by gemm_run: the call runs on CTA pairs
   int epi = 0, out_es = 4, aux_es = 4;
   bool f16 = false, out_f16 = false, aux_f16 = false;   // 16-bit operands / output / aux are fp16, not bf16
   GemmParams p{};   // epilogue fields (out, ldo, aux, ...) filled by the caller
