@@ -77,7 +77,7 @@ namespace {
 using bf16 = __nv_bfloat16;
 using f16 = __half;
 
-// The paired variants compiled (16-bit operands, BN 256), one line each:
+// The paired variants compiled (16- and 8-bit operands, BN 256), one line each:
 // operand type, A and B MN-major, epilogue, output and aux types.
 #define GPT_GEMM_PAIR_LIST(X)                            \
   X(bf16, false, true, EPI_QKV, bf16, bf16)              \
@@ -94,7 +94,15 @@ using f16 = __half;
   X(bf16, true, false, EPI_STORE, float, float)          \
   X(f16, false, true, EPI_AXPBY, f16, float)             \
   X(f16, false, true, EPI_AXPBY, f16, f16)               \
-  X(f16, false, true, EPI_AXPBY, float, f16)
+  X(f16, false, true, EPI_AXPBY, float, f16)             \
+  X(uint8_t, false, true, EPI_ACC, float, float)         \
+  X(uint8_t, false, true, EPI_RELU2, bf16, bf16)         \
+  X(uint8_t, false, true, EPI_STORE, float, float)       \
+  X(uint8_t, false, false, EPI_STORE, float, float)      \
+  X(uint8_t, false, false, EPI_DRELU2, bf16, bf16)       \
+  X(uint8_t, false, false, EPI_STORE, bf16, bf16)        \
+  X(uint8_t, true, true, EPI_STORE, float, float)        \
+  X(uint8_t, true, true, EPI_ACC, float, float)
 
 bool pair_variant_exists(const GemmCall& c) {
 #define GPT_GEMM_PAIR_HAS(T_, AMN_, BMN_, EPI_, OUT_, AUX_)                                                     \
@@ -188,7 +196,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
   p.sym = c.sym ? 1 : 0;
-  c.pair = c.allow_pair && c.bn == 256 && !c.sym && p.splits == 1 && c.es == 2 && c.M > 128 &&
+  c.pair = c.allow_pair && c.bn == 256 && !c.sym && p.splits == 1 && (c.es == 2 || c.es == 1) && c.M > 128 &&
            wait_limit_or_default(p.wait_cycles) >= kShortWaitCycles && pair_variant_exists(c);
   if (c.pair) p.tiles_m = (p.tiles_m + 1) / 2;   // one unit per 256-row block: the kernel's index counts pairs
   const long long ntiles = c.sym ? sym_tile_count(p.tiles_m, p.tiles_n, c.bn / 128) : 1ll * p.tiles_m * p.tiles_n;

@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(320, 1)
                    const __grid_constant__ GemmParams p) {
   constexpr int ES = sizeof(T);
   using C = GemmCfg<ES, BN, PAIR>;
-  static_assert(!PAIR || (ES == 2 && BN == 256), "CTA pairs: 16-bit operands, 256-wide tiles");
+  static_assert(!PAIR || ((ES == 2 || ES == 1) && BN == 256), "CTA pairs: 16- or 8-bit operands, 256-wide tiles");
   constexpr uint32_t IDESC = make_idesc(ES == 2 ? (std::is_same<T, __half>::value ? 0 : 1) : (ES == 4 ? 2 : 0), BN,
                                         A_MN, B_MN, PAIR ? 256 : 128);
 
@@ -347,8 +347,10 @@ __global__ void __launch_bounds__(320, 1)
             const uint64_t bd = B_MN ? smem_desc_sw128(b0 + kk * C::MMA_K * 128, C::CHUNK_BYTES, 1024)
                                      : smem_desc_sw128(b0 + kk * 32, 16, 1024);
             const uint32_t accum = (kb > kb0 || kk > 0) ? 1u : 0u;
-            if constexpr (PAIR)
+            if constexpr (PAIR && ES == 2)
               umma_f16_pair(d_tmem, ad, bd, IDESC, accum);
+            else if constexpr (PAIR)
+              umma_f8_pair(d_tmem, ad, bd, IDESC, accum);
             else if constexpr (ES == 2)
               umma_f16(d_tmem, ad, bd, IDESC, accum);
             else if constexpr (ES == 4)
