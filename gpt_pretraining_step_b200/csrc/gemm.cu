@@ -95,6 +95,8 @@ using f16 = __half;
   X(f16, false, true, EPI_AXPBY, f16, float)             \
   X(f16, false, true, EPI_AXPBY, f16, f16)               \
   X(f16, false, true, EPI_AXPBY, float, f16)             \
+  X(f16, false, false, EPI_STORE, f16, f16)              \
+  X(f16, false, false, EPI_AXPBY, f16, f16)              \
   X(uint8_t, false, true, EPI_ACC, float, float)         \
   X(uint8_t, false, true, EPI_RELU2, bf16, bf16)         \
   X(uint8_t, false, true, EPI_STORE, float, float)       \
@@ -196,10 +198,11 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
   p.sym = c.sym ? 1 : 0;
-  c.pair = c.allow_pair && c.bn == 256 && !c.sym && p.splits == 1 && (c.es == 2 || c.es == 1) && c.M > 128 &&
+  c.pair = c.allow_pair && c.bn == 256 && p.splits == 1 && (c.es == 2 || c.es == 1) && c.M > 128 &&
            wait_limit_or_default(p.wait_cycles) >= kShortWaitCycles && pair_variant_exists(c);
   if (c.pair) p.tiles_m = (p.tiles_m + 1) / 2;   // one unit per 256-row block: the kernel's index counts pairs
-  const long long ntiles = c.sym ? sym_tile_count(p.tiles_m, p.tiles_n, c.bn / 128) : 1ll * p.tiles_m * p.tiles_n;
+  const long long ntiles =
+      c.sym ? sym_tile_count(p.tiles_m, p.tiles_n, c.pair ? 1 : c.bn / 128) : 1ll * p.tiles_m * p.tiles_n;
   const long long units = ntiles * p.splits * c.batch;
   if (units > 0x7fffffffll) return cudaErrorInvalidValue;
   p.units = static_cast<int>(units);

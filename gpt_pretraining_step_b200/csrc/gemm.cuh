@@ -67,10 +67,12 @@ __host__ __device__ __forceinline__ int sym_tile_count(int tiles_m, int tiles_n,
   return n;
 }
 
-template <int BN>
+// (PAIR: mb counts 256-row blocks, so a row block of a symmetric product needs
+// the column blocks from mb on)
+template <int BN, bool PAIR = false>
 __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, int& mb, int& nb,
                                             int& kb0, int& kb1, int& split) {
-  constexpr int R = BN / 128;
+  constexpr int R = PAIR ? 1 : BN / 128;
   const int ntiles = p.sym ? sym_tile_count(p.tiles_m, p.tiles_n, R) : p.tiles_m * p.tiles_n;
   const int per_z = ntiles * p.splits;
   z = u / per_z;
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int u = u_first; u < p.units && ok; u += u_step) {
         int z, mb, nb, kb0, kb1, split;
-        decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
+        decode_unit<BN, PAIR>(p, u, z, mb, nb, kb0, kb1, split);
         if constexpr (PAIR) mb = 2 * mb + static_cast<int>(rank);
         const int n0 = nb * BN + (PAIR ? 128 * static_cast<int>(rank) : 0);   // first B row staged here
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = true;
       for (int u = u_first; u < p.units && ok; u += u_step, ++local) {
         int z, mb, nb, kb0, kb1, split;
-        decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
+        decode_unit<BN, PAIR>(p, u, z, mb, nb, kb0, kb1, split);
         const int acc = local & 1;
         const uint32_t acc_par = (local >> 1) & 1;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, wlim)) { ok = false; break; }
@@ -444,7 +446,7 @@ __global__ void __launch_bounds__(320, 1)
     int local = 0;
     for (int u = u_first; u < p.units; u += u_step, ++local) {
       int z, mb, nb, kb0, kb1, split;
-      decode_unit<BN>(p, u, z, mb, nb, kb0, kb1, split);
+      decode_unit<BN, PAIR>(p, u, z, mb, nb, kb0, kb1, split);
       if constexpr (PAIR) mb = 2 * mb + static_cast<int>(rank);
       const int acc = local & 1;
       const uint32_t acc_par = (local >> 1) & 1;
