@@ -198,7 +198,7 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
   p.kb_per_split = (p.kblocks + splits - 1) / splits;
   p.splits = (p.kblocks + p.kb_per_split - 1) / p.kb_per_split;
   p.sym = c.sym ? 1 : 0;
-  c.pair = c.allow_pair && c.bn == 256 && p.splits == 1 && (c.es == 2 || c.es == 1) && c.M > 128 &&
+  c.pair = c.allow_pair && c.bn == 256 && (c.es == 2 || c.es == 1) && c.M > 128 &&
            wait_limit_or_default(p.wait_cycles) >= kShortWaitCycles && pair_variant_exists(c);
   if (c.pair) p.tiles_m = (p.tiles_m + 1) / 2;   // one unit per 256-row block: the kernel's index counts pairs
   const long long ntiles =

@@ -28,7 +28,7 @@ struct GemmCall {
   int bn = 256, splits = 1;
   bool sym = false;
   // CTA pairs (2-CTA clusters, M = 256 per tile) where the call allows them:
-  // BN 256, 16- or 8-bit operands, no K split, a bound on waits of at least
+  // BN 256, 16- or 8-bit operands, a bound on waits of at least
   // kShortWaitCycles, and a compiled paired variant; else one CTA per tile
   bool allow_pair = true;
   bool pair = false;   // set by gemm_run: the call runs on CTA pairs
