@@ -105,7 +105,8 @@ def _attn_inputs(B, H, T, seed):
     return q, k, v
 
 
-@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 64), (1, 1, 384), (2, 1, 129)])
+@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 64), (1, 1, 384), (2, 1, 129),
+                                   (1, 2, 640), (2, 1, 1100), (1, 1, 1537)])
 def test_attention_fwd(torch, B, H, T):
     import gpt_pretraining_step_b200 as g
     q, k, v = _attn_inputs(B, H, T, seed=T)
