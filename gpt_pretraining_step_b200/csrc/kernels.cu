@@ -659,6 +659,72 @@ __global__ void qk_bwd_kernel(const float* __restrict__ dq, const bf16* __restri
   if (amax) amax_slot_update(amax, am, w);
 }
 
+// q alone (the attention backward writes the k and v columns): half a warp
+// per (b, h, t) row, lane l of the half holding dims 4l..4l+3 and
+// 64+4l..64+4l+3, so that each rotation pair (i, i + 64) sits in one thread
+// and every access is a 16- or 8-byte vector; 32-bit indices (the launcher
+// checks the row count).
+__global__ void __launch_bounds__(256) qk_bwd_q_kernel(const float* __restrict__ dq, const bf16* __restrict__ qn,
+                                                       const float* __restrict__ rq, const float2* __restrict__ rope,
+                                                       bf16* __restrict__ dqkv, int total, int T, int H, int row_len,
+                                                       unsigned int* __restrict__ amax) {
+  const int w = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 4);
+  if ((w & ~1) >= total) return;   // both rows of the warp past the end
+  const bool valid = w < total;
+  const int l = threadIdx.x & 15;
+  const int t = w % T, bh = w / T;
+  const int h = bh % H, b = bh / H;
+  const int m = b * T + t;
+  float am = 0.f;
+  float g[8], y[8];
+  float4 e[4];   // (cos, sin) of dims 4l .. 4l+3 as float2 pairs
+  float r = 0.f;
+  if (valid) {
+    const long long src = static_cast<long long>(w) * 128 + 4 * l;
+    const float4 a = *reinterpret_cast<const float4*>(dq + src);
+    const float4 c = *reinterpret_cast<const float4*>(dq + src + 64);
+    const uint2 ylo = *reinterpret_cast<const uint2*>(qn + src);
+    const uint2 yhi = *reinterpret_cast<const uint2*>(qn + src + 64);
+    const float4* ep = reinterpret_cast<const float4*>(rope + static_cast<long long>(t) * 64 + 4 * l);
+    e[0] = ep[0]; e[1] = ep[1];
+    r = rq[static_cast<long long>(m) * H + h];
+    g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w;
+    g[4] = c.x; g[5] = c.y; g[6] = c.z; g[7] = c.w;
+    y[0] = bf16_lo(ylo.x); y[1] = bf16_hi(ylo.x); y[2] = bf16_lo(ylo.y); y[3] = bf16_hi(ylo.y);
+    y[4] = bf16_lo(yhi.x); y[5] = bf16_hi(yhi.x); y[6] = bf16_lo(yhi.y); y[7] = bf16_hi(yhi.y);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) g[i] = y[i] = 0.f;
+    e[0] = e[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dot += g[i] * y[i];
+  // sum over the half warp's 16 lanes
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  dot *= 1.f / 128.f;
+  if (valid) {
+    // gradient w.r.t. the rotated vector, then the transposed rotation
+    const float cs[4] = {e[0].x, e[0].z, e[1].x, e[1].z};
+    const float sn[4] = {e[0].y, e[0].w, e[1].y, e[1].w};
+    float ol[4], oh[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float rl = r * (g[i] - y[i] * dot), rh = r * (g[4 + i] - y[4 + i] * dot);
+      ol[i] = rl * cs[i] + rh * sn[i];
+      oh[i] = -rl * sn[i] + rh * cs[i];
+    }
+    bf16* out = dqkv + static_cast<long long>(m) * row_len + h * 128 + 4 * l;
+    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(ol[0], ol[1]), pack_bf16x2(ol[2], ol[3]));
+    *reinterpret_cast<uint2*>(out + 64) = make_uint2(pack_bf16x2(oh[0], oh[1]), pack_bf16x2(oh[2], oh[3]));
+    if (amax)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) am = fmaxf(am, fmaxf(abs_bf16(ol[i]), abs_bf16(oh[i])));
+  }
+  if (amax) amax_slot_update(amax, am, w);
+}
+
 // ------------------------------------------------------- cross-entropy finish
 
 __global__ void __launch_bounds__(256) ce_finish_kernel(bf16* __restrict__ z, const float2* __restrict__ stats,
@@ -1141,6 +1207,13 @@ void launch_qk_bwd(const float* dq, const bf16* dk, const bf16* dv, const bf16* 
                    const float* rk, const float2* rope, bf16* dqkv, int B, int T, int H, cudaStream_t s, int Hkv,
                    unsigned int* amax) {
   const long long rows = 1ll * B * H * T;
+  if (!dk && rows <= 0x3fffffffll) {
+    // q alone: two rows per warp
+    const int d = H * 128, kvd = (Hkv <= 0 ? H : Hkv) * 128;
+    qk_bwd_q_kernel<<<static_cast<int>(cdiv(rows, 16)), 256, 0, s>>>(dq, qn, rq, rope, dqkv, static_cast<int>(rows), T,
+                                                                      H, d + 2 * kvd, amax);
+    return;
+  }
   if (Hkv <= 0 || Hkv == H)
     qk_bwd_kernel<false><<<cdiv(rows, 8), 256, 0, s>>>(dq, dk, dv, qn, kn, rq, rk, rope, dqkv, B, T, H, H, amax);
   else
