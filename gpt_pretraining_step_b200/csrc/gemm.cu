@@ -29,7 +29,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // 3-D map over [batch][outer][inner] with 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
-              long long ld, long long bs, int box_inner, int box_outer, bool f16) {
+              long long ld, long long bs, int box_inner, int box_outer, bool f16, bool swizzle) {
   auto fn = encode_fn();
   if (!fn) return false;
   if (bs == 0 || batch == 1) bs = ld * outer;
@@ -44,7 +44,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long lon
               : (es == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8);
   CUresult r = fn(m, dt, 3,
                   const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -251,10 +251,16 @@ cudaError_t gemm_run(GemmCall& c, cudaStream_t stream) {
                     p.splits > 1 || c.N % 128 || !p.aux || !p.f32a || p.T <= 0 || c.M % p.T || p.H * 128 != c.N ||
                     (p.ld_aux & 7) || (reinterpret_cast<uintptr_t>(p.aux) & 15)))
     return cudaErrorInvalidValue;
+  p.tma_mirror = 0;
   if (p.out2) {
     if (c.epi == EPI_QKV || c.epi == EPI_LOGITS || p.splits > 1 || !p.tma_out) return cudaErrorInvalidValue;
     if (!make_map(&md, p.out2, 2, c.N, c.M, c.batch, p.ldo, p.out_bs, 64, 32, true)) return cudaErrorInvalidValue;
     p.tma_out2 = 1;
+  } else if (c.sym && p.tma_out && c.out_es == 2 && !p.out_t && p.splits == 1 &&
+             make_map(&md, p.out, 2, c.N, c.M, c.batch, p.ldo, p.out_bs, 32, 64, c.out_f16, false)) {
+    // the transposed copies of a symmetric product's off-diagonal tiles: a
+    // warp's 32 rows x 64 columns land as 64 rows x 32 columns
+    p.tma_mirror = 1;
   } else {
     md = ma;   // unused by the kernel
   }

@@ -606,15 +606,16 @@ __global__ void __launch_bounds__(320, 1)
       } else {
         OutT* obase = reinterpret_cast<OutT*>(p.out) + static_cast<long long>(z) * p.out_bs +
                       static_cast<long long>(split) * p.split_stride;
-        // Symmetric products: with square tiles (BN 128) the diagonal tiles are
-        // written whole and the others mirrored whole; with 128 x 256 tiles an
-        // element is written directly on or above the diagonal and mirrored
-        // from above it, so each is written exactly once, and a tile that
-        // holds elements below the diagonal stores per thread with that mask.
+        // Symmetric products: the tiles that hold diagonal elements are written
+        // whole, and the tiles wholly above the diagonal are written and
+        // mirrored whole, so each element is written exactly once (with 128 x
+        // 256 tiles the two row blocks of a diagonal 256-column block are both
+        // computed and together cover it).  The mirror goes by TMA when the
+        // host built its map, else by per-thread stores.
         constexpr bool kRect = BN == 256;
-        const bool sym_cross = kRect && p.sym && nb * BN < mb * 128 + 128;
-        const bool mirror = p.sym && (kRect || nb != mb);
-        const bool tma_here = p.tma_out && !sym_cross;
+        const bool sym_cross = kRect ? nb * BN < mb * 128 + 128 : nb == mb;
+        const bool mirror = p.sym && !sym_cross;
+        const bool tma_here = p.tma_out;
         // Auxiliary input of the epilogue, prefetched one 32-column chunk ahead to
         // hide its load latency.  (EPI_ACC adds into the output by TMA
         // add-reduction and reads nothing.)
@@ -709,6 +710,17 @@ __global__ void __launch_bounds__(320, 1)
             }
           }
           if (tma_here) emit64(v[0], v[1], nb * BN + c * 32, box_row0, z3);
+          if (mirror && p.tma_mirror) {
+            // this warp's 32 rows x 64 columns transposed: staging row j (column
+            // nb BN + 32 c + j) holds the 32 rows, 64 bytes, for a 32 x 64 box
+            box_open();
+            OutT* st = reinterpret_cast<OutT*>(stg);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) store_scalar(st + j * 32 + lane, v[0][j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) store_scalar(st + (32 + j) * 32 + lane, v[1][j]);
+            box_close(&tmD, false, box_row0, nb * BN + c * 32, z3);
+          }
           if constexpr (EPI == EPI_STORE && std::is_same<OutT, __nv_bfloat16>::value) {
             if (dot_here) {
               // the stored (bf16-rounded) values against the same columns of aux
@@ -745,31 +757,18 @@ __global__ void __launch_bounds__(320, 1)
             const int col0 = nb * BN + (c + hh) * 32;
             const int nvalid = min(32, p.N - col0);
             if (!row_ok || nvalid <= 0) continue;
-            if (sym_cross) {
-              // the columns on or above the diagonal of this row
-              OutT* drow = obase + static_cast<long long>(row) * p.ldo;
-              if (col0 >= row) {
-                store_row32(drow + col0, v[hh], nvalid);
-              } else if (col0 + nvalid > row) {
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                  if (j < nvalid && col0 + j >= row) store_scalar(drow + col0 + j, v[hh][j]);
-              }
-            } else if (!tma_here) {
-              store_row32(obase + static_cast<long long>(row) * p.ldo + col0, v[hh], nvalid);
-            }
+            if (!tma_here) store_row32(obase + static_cast<long long>(row) * p.ldo + col0, v[hh], nvalid);
             if (p.out_t) {
               OutT* tb = reinterpret_cast<OutT*>(p.out_t) + static_cast<long long>(z) * p.out_bs;
 #pragma unroll
               for (int j = 0; j < 32; ++j)
                 if (j < nvalid) store_scalar(tb + static_cast<long long>(col0 + j) * p.ldo_t + row, v[hh][j]);
             }
-            if (mirror) {
+            if (mirror && !p.tma_mirror) {
               // the transposed tile of a symmetric product: lanes write consecutive columns
 #pragma unroll
               for (int j = 0; j < 32; ++j)
-                if (j < nvalid && (!kRect || col0 + j > row))
-                  store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
+                if (j < nvalid) store_scalar(obase + static_cast<long long>(col0 + j) * p.ldo + row, v[hh][j]);
             }
           }
         }

@@ -47,11 +47,11 @@ int gemm_tiles(const GemmCall& c);
 int device_sm_count();
 
 // TMA descriptor of a bf16 (es = 2; fp16 with f16) or fp32 (es = 4) tensor [batch][outer][inner]
-// with row stride ld and batch stride bs (elements), 128-byte swizzle, box
-// box_inner x box_outer.  False if the driver entry point is missing or the
-// base/strides are not 16-byte aligned.
+// with row stride ld and batch stride bs (elements), 128-byte swizzle (or
+// none), box box_inner x box_outer.  False if the driver entry point is
+// missing or the base/strides are not 16-byte aligned.
 bool make_map(CUtensorMap* m, const void* ptr, int es, long long inner, long long outer, long long batch,
-              long long ld, long long bs, int box_inner, int box_outer, bool f16 = false);
+              long long ld, long long bs, int box_inner, int box_outer, bool f16 = false, bool swizzle = true);
 
 // 4-D bf16 map, dims {d0 (innermost), d1, d2, d3}, byte strides of dims 1..3,
 // box {b0, b1, b2, b3}, 128-byte swizzle.

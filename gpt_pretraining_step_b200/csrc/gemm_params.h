@@ -45,6 +45,8 @@ struct GemmParams {
                         //   k and v stored at head rows b*H + j of their [B, H, T, 128] buffers
   int tma_out;          // 1: the main output is written by TMA stores through the output tensor map
   int tma_out2;         // 1: also an fp16 copy of the output, same layout, through the second map
+  int tma_mirror;       // symmetric products, 16-bit output: the mirrored (transposed) tiles are
+                        //   written by TMA through the second map (box 32 x 64, no swizzle)
   void* out2;           //   (its base; row stride ldo, batch stride out_bs)
   int* err;
   long long wait_cycles;   // bound of every mbarrier wait (SM cycles; <= 0: the library default)
