@@ -229,7 +229,8 @@ def test_attention_rejects_bad_head_split(torch):
         g.attention_fwd(bf16_t(torch, q), bf16_t(torch, k), bf16_t(torch, v))
 
 
-@pytest.mark.parametrize("batch,rows,cols", [(2, 256, 768), (1, 640, 128), (3, 128, 128), (1, 136, 264)])
+@pytest.mark.parametrize("batch,rows,cols", [(2, 256, 768), (1, 640, 128), (3, 128, 128), (1, 136, 264),
+                                              (1, 600, 700), (2, 520, 1030)])
 @pytest.mark.parametrize("tf32_steps", [-1, 0, 3, 5])
 def test_newton_schulz(torch, batch, rows, cols, tf32_steps):
     import gpt_pretraining_step_b200 as g
