@@ -540,35 +540,49 @@ __global__ void __launch_bounds__(320, 1)
             const float rstd = rsqrtf(ss * (1.f / 128.f) + 1e-6f);
             if (row_ok) (which == 0 ? p.f32a : p.f32b)[static_cast<long long>(row) * p.H + head] = rstd;
             const float sc = rstd * dqs;
-            // RoPE pairs (i, i + 64): the first 64 output dims, then the last 64
+            // RoPE pairs (i, i + 64): each (cos, sin) is read once and gives output
+            // dims i (into the staging box) and 64 + i (kept packed until the
+            // first box has gone out)
+            uint32_t keep[32];
+            if (p.tma_out) box_open();
 #pragma unroll 1
-            for (int part = 0; part < 2; ++part) {
-              if (p.tma_out) box_open();
-#pragma unroll 1
-              for (int pc = 0; pc < 2; ++pc) {
-                float lo[32], hi[32];
-                tmem_load32(hb + pc * 32, lo);
-                tmem_load32(hb + 64 + pc * 32, hi);
-                // pair-major table: the warp's 32 consecutive tokens read one pair coalesced
-                const float2* cs = p.rope + static_cast<long long>(pc * 32) * p.T + t;
-                float o[32];
+            for (int pc = 0; pc < 2; ++pc) {
+              float lo[32], hi[32];
+              tmem_load32(hb + pc * 32, lo);
+              tmem_load32(hb + 64 + pc * 32, hi);
+              // pair-major table: the warp's 32 consecutive tokens read one pair coalesced
+              const float2* cs = p.rope + static_cast<long long>(pc * 32) * p.T + t;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
+              for (int u = 0; u < 4; ++u) {
+                float o0[8], o1[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                  const int j = 8 * u + jj;
                   const float2 e = row_ok ? cs[static_cast<long long>(j) * p.T] : make_float2(1.f, 0.f);
-                  o[j] = part == 0 ? (lo[j] * e.x - hi[j] * e.y) * sc : (lo[j] * e.y + hi[j] * e.x) * sc;
+                  o0[jj] = (lo[j] * e.x - hi[j] * e.y) * sc;
+                  o1[jj] = (lo[j] * e.y + hi[j] * e.x) * sc;
                 }
+                const uint4 w0 = make_uint4(pack2<OutT>(o0[0], o0[1]), pack2<OutT>(o0[2], o0[3]),
+                                            pack2<OutT>(o0[4], o0[5]), pack2<OutT>(o0[6], o0[7]));
+                const uint4 w1 = make_uint4(pack2<OutT>(o1[0], o1[1]), pack2<OutT>(o1[2], o1[3]),
+                                            pack2<OutT>(o1[4], o1[5]), pack2<OutT>(o1[6], o1[7]));
                 if (p.tma_out) {
-#pragma unroll
-                  for (int u = 0; u < 4; ++u)
-                    box_put(4 * pc + u, make_uint4(pack2<OutT>(o[8 * u], o[8 * u + 1]),
-                                                   pack2<OutT>(o[8 * u + 2], o[8 * u + 3]),
-                                                   pack2<OutT>(o[8 * u + 4], o[8 * u + 5]),
-                                                   pack2<OutT>(o[8 * u + 6], o[8 * u + 7])));
+                  box_put(4 * pc + u, w0);
+                  keep[16 * pc + 4 * u] = w1.x; keep[16 * pc + 4 * u + 1] = w1.y;
+                  keep[16 * pc + 4 * u + 2] = w1.z; keep[16 * pc + 4 * u + 3] = w1.w;
                 } else if (row_ok) {
-                  store_row32(dst + part * 64 + pc * 32, o, 32);
+                  *reinterpret_cast<uint4*>(dst + pc * 32 + 8 * u) = w0;
+                  *reinterpret_cast<uint4*>(dst + 64 + pc * 32 + 8 * u) = w1;
                 }
               }
-              if (p.tma_out) put_box(part * 64);
+            }
+            if (p.tma_out) {
+              put_box(0);
+              box_open();
+#pragma unroll
+              for (int u = 0; u < 8; ++u)
+                box_put(u, make_uint4(keep[4 * u], keep[4 * u + 1], keep[4 * u + 2], keep[4 * u + 3]));
+              put_box(64);
             }
           }
         }
