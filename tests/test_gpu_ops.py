@@ -122,7 +122,7 @@ def test_attention_fwd(torch, B, H, T):
     assert np.abs(f64(lse) - lse_ref).max() < 2e-3
 
 
-@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 256), (1, 1, 333)])
+@pytest.mark.parametrize("B,H,T", [(2, 3, 200), (1, 1, 1), (1, 2, 256), (1, 1, 333), (1, 2, 640), (2, 1, 1100)])
 def test_attention_bwd(torch, B, H, T):
     import gpt_pretraining_step_b200 as g
     q, k, v = _attn_inputs(B, H, T, seed=7 * T)
