@@ -88,14 +88,18 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, 
     mb = m;
     nb = m / R + t;
   } else {
+    // groups of 16 row blocks; inside a group the column blocks of a row come
+    // one after another, so the CTAs (clusters) that share a row block of A
+    // have adjacent indices and, in practice, sit on the same die and its
+    // half of L2 (with rows first, A was read from DRAM about twice)
     constexpr int G = 16;
     const int gsz = G * p.tiles_n;
     const int g = t / gsz;
     const int first = g * G;
     const int gm = min(G, p.tiles_m - first);
     const int tt = t - g * gsz;
-    mb = first + tt % gm;
-    nb = tt / gm;
+    mb = first + tt / p.tiles_n;
+    nb = tt % p.tiles_n;
   }
   kb0 = split * p.kb_per_split;
   kb1 = min(p.kblocks, kb0 + p.kb_per_split);
