@@ -122,6 +122,21 @@ def category_work(s):
     }
 
 
+def fp8_fraction(category, s):
+    """Share of a category's FLOPs that run on e4m3 operands with --precision fp8:
+    the attention output, MLP up and MLP down projections in all three of their
+    GEMMs (forward, activation gradient, weight gradient); q|k|v, attention,
+    the lm_head and Newton-Schulz stay 16-bit.  Per layer and token the block
+    dX (and dW) GEMMs take 2 d (d + 2 F) FLOPs on e4m3 against 2 d qkv_cols
+    for q|k|v (18 of 24 d^2 with F = 4 d and full kv heads)."""
+    if category in ("proj_gemm", "fc_gemm", "down_gemm"):
+        return 1.0
+    if category in ("dx_gemm", "dw_gemm"):
+        e4m3 = s.d_model * (s.d_model + 2 * s.mlp_hidden)
+        return e4m3 / (e4m3 + s.d_model * s.qkv_cols)
+    return 0.0
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -414,11 +429,17 @@ def run_ours(a):
         if kind == "tensor":
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e12
             peak = pk["bf16_tflops_sustained"]
+            src = f"{pk_src} bf16_tflops_sustained"
+            f8 = fp8_fraction(dominant, s) if a.precision == "fp8" else 0.0
+            if f8 > 0:
+                # the category's fp8 FLOPs against twice the bf16 figure (the nominal
+                # dense ratio), the rest against the bf16 figure
+                peak = 1.0 / ((1.0 - f8) / peak + f8 / (2.0 * peak))
+                src += f" blended with 2x for the fp8 share ({f8:.2f} of the FLOPs)"
             # DRAM traffic needs hardware counters (an ncu capture), which a timed
             # run does not take: reported as null here
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None, "kernel": dominant,
-                    "peak_source": f"{pk_src} bf16_tflops_sustained"}
+                    "frac": achieved / peak, "traffic": None, "kernel": dominant, "peak_source": src}
         else:
             achieved = per_launch_work / (per_launch_ms / 1e3) / 1e9
             peak = pk["hbm_gbs"]

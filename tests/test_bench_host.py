@@ -39,6 +39,21 @@ def test_projection_categories_add_up_to_the_matmul_flops(name):
     assert w["attn_bwd"][1] == 2.5 * w["attn_fwd"][1]
 
 
+def test_fp8_share_of_the_block_gradient_gemms():
+    # with F = 4 d and full kv heads the e4m3 projections (attention output, MLP
+    # up, MLP down) are 18 of the 24 d^2 FLOPs per token of the block dX and dW
+    # GEMMs; the forward projection categories are wholly fp8 or wholly 16-bit
+    s = syn.config_shape("d26")
+    assert abs(bench.fp8_fraction("dx_gemm", s) - 18 / 24) < 1e-12
+    assert bench.fp8_fraction("dw_gemm", s) == bench.fp8_fraction("dx_gemm", s)
+    assert bench.fp8_fraction("fc_gemm", s) == 1.0 and bench.fp8_fraction("qkv_gemm", s) == 0.0
+    assert bench.fp8_fraction("attn_bwd", s) == 0.0 and bench.fp8_fraction("ns_gemm", s) == 0.0
+    # the share matches the per-category work: proj + fc + down over all four
+    w = bench.category_work(s)
+    fp8_fwd = w["proj_gemm"][1] + w["fc_gemm"][1] + w["down_gemm"][1]
+    assert abs(fp8_fwd / (fp8_fwd + w["qkv_gemm"][1]) - bench.fp8_fraction("dx_gemm", s)) < 1e-12
+
+
 def test_clock_record_parsing_and_reasons(tmp_path):
     sampler = bench.ClockSampler(0)
 
