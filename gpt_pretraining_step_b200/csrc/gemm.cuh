@@ -88,18 +88,25 @@ __device__ __forceinline__ void decode_unit(const GemmParams& p, int u, int& z, 
     mb = m;
     nb = m / R + t;
   } else {
-    // groups of 16 row blocks; inside a group the column blocks of a row come
-    // one after another, so the CTAs (clusters) that share a row block of A
-    // have adjacent indices and, in practice, sit on the same die and its
-    // half of L2 (with rows first, A was read from DRAM about twice)
+    // Groups of 16 row blocks.  Inside a group, tiles that follow one another
+    // go to CTAs (clusters) with adjacent indices, which in practice sit on
+    // the same die and its half of L2, so they share the larger operand: the
+    // column blocks of a row one after another when A (M x K) is the larger,
+    // else the row blocks of a column (sharing the other way read the larger
+    // operand from DRAM about twice, and for M << N many times over)
     constexpr int G = 16;
     const int gsz = G * p.tiles_n;
     const int g = t / gsz;
     const int first = g * G;
     const int gm = min(G, p.tiles_m - first);
     const int tt = t - g * gsz;
-    mb = first + tt / p.tiles_n;
-    nb = tt % p.tiles_n;
+    if (p.tiles_m >= p.tiles_n) {
+      mb = first + tt / p.tiles_n;
+      nb = tt % p.tiles_n;
+    } else {
+      mb = first + tt % gm;
+      nb = tt / gm;
+    }
   }
   kb0 = split * p.kb_per_split;
   kb1 = min(p.kblocks, kb0 + p.kb_per_split);
